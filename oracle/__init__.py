@@ -1,0 +1,157 @@
+"""fp64 CPU oracle for the Key-only GLA token mixer of GTR.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  The CUDA library in
+``linear_vision_backbone_b200`` never imports, links or runs it, and the two
+share no code: the oracle is plain C (``gla_oracle.c``) compiled with gcc, in
+IEEE fp64 (no fast-math), driven through ctypes from here.
+
+Functions (each cites the page passage it follows in ``gla_oracle.c``):
+
+* :func:`gate` -- ``g = logsigmoid(x W_down W_up + b) / tau`` (GTR article,
+  方法详解 §1, low-rank forget gate with temperature).
+* :func:`gla_fwd` -- the token-by-token recurrence ``S_t = diag(exp g_t) S_{t-1}
+  + k_t^T v_t``, ``o_t = q_t S_t``, then ``RMSNorm(o_t) * SiLU(z_t)``, over the
+  grid in one of the four scan orders, written back in grid order (GTR article,
+  方法详解 §1).
+* :func:`chunk_states` -- the state after every chunk of scan positions (GTR
+  article, 方法详解 §4, the boundary states of the chunkwise operator).
+* :func:`scan_index` -- the grid index visited at a scan position.
+
+Pins: every function here is checked in ``tests/test_oracle_pins.py`` against
+results fixed independently of it (the quadratic masked form, plain causal
+linear attention at g = 0, the memoryless limit, T = 1, explicit grid flips and
+transposes, closed forms of the gate).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gla_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+DIRS = {"LR": 0, "RL": 1, "TB": 2, "BT": 3, "ROTATE": 4}
+
+
+def build(force: bool = False) -> str:
+    """Compile ``gla_oracle.c`` with gcc (fp64, -O2, OpenMP, no fast-math)."""
+    os.makedirs(_BUILD, exist_ok=True)
+    stale = (not os.path.exists(_LIB_PATH)) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)
+    if force or stale:
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-fno-fast-math",
+               "-ffp-contract=off", _SRC, "-o", tmp, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB_PATH)
+            P = ctypes.c_void_p
+            i, l, d = ctypes.c_int, ctypes.c_long, ctypes.c_double
+            lib.oracle_gate_f64.argtypes = [P, P, P, P, P, l, i, i, i, d]
+            lib.oracle_gate_f64.restype = i
+            lib.oracle_gla_fwd_f64.argtypes = [P, P, P, P, P, P, P, P, i, i, i, i, i, i, i, d]
+            lib.oracle_gla_fwd_f64.restype = i
+            lib.oracle_gla_chunk_states_f64.argtypes = [P, P, P, P, i, i, i, i, i, i, i, i]
+            lib.oracle_gla_chunk_states_f64.restype = i
+            lib.oracle_scan_index.argtypes = [i, l, l, l]
+            lib.oracle_scan_index.restype = l
+            lib.oracle_set_threads.argtypes = [i]
+            lib.oracle_set_threads.restype = i
+            _lib = lib
+    return _lib
+
+
+def _f64(a) -> np.ndarray:
+    """Exact widening to a C-contiguous fp64 array (accepts numpy or torch CPU tensors)."""
+    if hasattr(a, "detach"):
+        a = a.detach().to("cpu")
+        a = a.double().numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def set_threads(n: int) -> int:
+    """Set the OpenMP thread count of the oracle; returns the count in effect."""
+    return int(_load().oracle_set_threads(int(n)))
+
+
+def scan_index(direction: str, s: int, gh: int, gw: int) -> int:
+    return int(_load().oracle_scan_index(DIRS[direction], int(s), int(gh), int(gw)))
+
+
+def gate(x, w_down, w_up, bias=None, tau: float = 16.0) -> np.ndarray:
+    """g[n, :] = logsigmoid(x[n] @ w_down @ w_up + bias) / tau, fp64.
+
+    ``x`` may have any leading shape; the last axis is the model width.
+    """
+    x = _f64(x)
+    lead = x.shape[:-1]
+    dm = x.shape[-1]
+    x2 = x.reshape(-1, dm)
+    wd, wu = _f64(w_down), _f64(w_up)
+    rank, HD = wu.shape
+    assert wd.shape == (dm, rank)
+    b = None if bias is None else _f64(bias).reshape(HD)
+    out = np.empty((x2.shape[0], HD), dtype=np.float64)
+    rc = _load().oracle_gate_f64(_ptr(x2), _ptr(wd), _ptr(wu), None if b is None else _ptr(b),
+                                 _ptr(out), x2.shape[0], dm, rank, HD, float(tau))
+    if rc != 0:
+        raise ValueError(f"oracle_gate_f64 rejected its arguments (rc={rc})")
+    return out.reshape(*lead, HD)
+
+
+def gla_fwd(q, k, v, g, z, w=None, *, gh: int, gw: int, direction: str = "LR",
+            eps: float = 1e-5, return_o: bool = False):
+    """y = RMSNorm(o) * SiLU(z) with o from the Key-only gated recurrence, fp64.
+
+    q, k, g: [B, T, H, dk]; v, z: [B, T, H, dv]; w: [dv] or None; T = gh * gw.
+    Returns y (and o before the normalisation when ``return_o``).
+    """
+    q, k, v, g, z = (_f64(a) for a in (q, k, v, g, z))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    assert T == gh * gw and k.shape == q.shape and g.shape == q.shape
+    assert v.shape == (B, T, H, dv) and z.shape == v.shape
+    wv = None if w is None else _f64(w).reshape(dv)
+    y = np.empty((B, T, H, dv), dtype=np.float64)
+    o = np.empty_like(y) if return_o else None
+    rc = _load().oracle_gla_fwd_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(z),
+                                    None if wv is None else _ptr(wv), _ptr(y),
+                                    None if o is None else _ptr(o),
+                                    B, H, gh, gw, dk, dv, DIRS[direction], float(eps))
+    if rc != 0:
+        raise ValueError(f"oracle_gla_fwd_f64 rejected its arguments (rc={rc})")
+    return (y, o) if return_o else y
+
+
+def chunk_states(k, v, g, *, gh: int, gw: int, direction: str = "LR", chunk: int = 64) -> np.ndarray:
+    """State after each chunk of ``chunk`` scan positions: [B, H, ceil(T/chunk), dk, dv]."""
+    k, v, g = (_f64(a) for a in (k, v, g))
+    B, T, H, dk = k.shape
+    dv = v.shape[-1]
+    nc = (T + chunk - 1) // chunk
+    st = np.empty((B, H, nc, dk, dv), dtype=np.float64)
+    rc = _load().oracle_gla_chunk_states_f64(_ptr(k), _ptr(v), _ptr(g), _ptr(st), B, H, gh, gw,
+                                             dk, dv, DIRS[direction], int(chunk))
+    if rc != 0:
+        raise ValueError(f"oracle_gla_chunk_states_f64 rejected its arguments (rc={rc})")
+    return st
