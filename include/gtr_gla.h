@@ -1,0 +1,182 @@
+/*
+ * gtr_gla.h -- C ABI of the B200 (sm_100a) Key-only gated linear attention
+ * token mixer of GTR.
+ *
+ * Operator (GTR article "端侧实时感知新标杆！通用线性骨干网络GTR开源",
+ * shuwu5.cn/article/3124, 方法详解 §1 "骨干架构：Key-only 门控递归与四向交替扫描";
+ * the page's formulas were lost in extraction, the surviving prose fixes this
+ * reading): for every batch entry b and head h, scanning the grid_h x grid_w
+ * token grid in one direction,
+ *
+ *     S_s = diag(exp(g_s)) S_{s-1} + k_s^T v_s          (dk x dv state, S_-1 = 0)
+ *     o_s = q_s S_s
+ *     y_s = o_s / sqrt(mean(o_s^2) + 1e-5) * w * SiLU(z_s)
+ *
+ * with the value-side decay fixed to 1 and the key-side forget gate
+ *
+ *     g = logsigmoid(x W_down W_up + bias) / tau          (low-rank projection)
+ *
+ * computed by gtr_gate_fwd.  gtr_gla_fwd evaluates the recurrence chunk by
+ * chunk in three stages (方法详解 §4 "硬件感知分块推理算子": chunk summaries on
+ * tensor cores, a light sequential pass over chunk-boundary states, chunk
+ * outputs with the output gate fused into the epilogue).
+ *
+ * Scan orders (方法详解 §1, four alternating directions, grid order restored
+ * after the scan).  Sequence position s visits grid index t = row*grid_w + col:
+ *     GTR_LR: t = s                                   (row-major raster)
+ *     GTR_RL: t = T-1-s                               (LR reversed)
+ *     GTR_TB: t = (s mod grid_h)*grid_w + s/grid_h    (down each column, columns left to right)
+ *     GTR_BT: TB reversed
+ *     GTR_ROTATE_BATCH: batch entry b uses direction (b mod 4) of the four above.
+ * Output y is stored at the grid index its token came from, so every tensor
+ * stays in grid order.
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are caller-owned DEVICE pointers, C-contiguous, in grid order:
+ *       q, k, g      : [B, T, H, dk]     (T = grid_h * grid_w)
+ *       v, z, out    : [B, T, H, dv]
+ *       x            : [B, T, d_model]
+ *     q, k, v, z and out share one element type `dtype` (gtr_dtype_t); the gate
+ *     tensor g is always fp32.  Every tensor pointer must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls are asynchronous on it, never synchronise and launch no
+ *     work on any other stream.
+ *   - Errors are returned as a gtr_status_t; nothing is thrown and no device
+ *     trap is raised.  All argument checks run before any launch; a rejected
+ *     call launches nothing.  A launch failure maps to GTR_ERR_CUDA.
+ *   - Sizes of zero (B, H, grid_h or grid_w == 0) are an empty problem:
+ *     GTR_OK, nothing launched, pointers unused.  Negative sizes are invalid.
+ */
+#ifndef GTR_GLA_H
+#define GTR_GLA_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__) || defined(__clang__)
+#define GTR_API __attribute__((visibility("default")))
+#else
+#define GTR_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GTR_OK = 0,
+    GTR_ERR_INVALID_ARG = -1,   /* null pointer, negative size, bad enum, overflow */
+    GTR_ERR_UNSUPPORTED = -2,   /* valid but not implemented (head dim, chunk, rank) */
+    GTR_ERR_ALIGNMENT = -3,     /* a tensor pointer is not 16-byte aligned */
+    GTR_ERR_NO_MEMORY = -4,     /* workspace could not be obtained */
+    GTR_ERR_CUDA = -5,          /* a CUDA runtime call or launch failed */
+    GTR_ERR_DEVICE_CHECK = -6   /* a device-side check recorded a failure */
+} gtr_status_t;
+
+typedef enum { GTR_F32 = 0, GTR_F16 = 1, GTR_BF16 = 2 } gtr_dtype_t;
+
+typedef enum { GTR_LR = 0, GTR_RL = 1, GTR_TB = 2, GTR_BT = 3, GTR_ROTATE_BATCH = 4 } gtr_dir_t;
+
+/* Kernel families gtr_gla_fwd can run (see gtr_gla_set_path). */
+typedef enum {
+    GTR_PATH_AUTO = 0,  /* tensor-core path where supported, else SIMT */
+    GTR_PATH_SIMT = 1,  /* exact fp32 CUDA-core path, every dtype and head dim */
+    GTR_PATH_TC = 2     /* tcgen05/TMEM path: 16-bit dtypes, dk = dv = 64 */
+} gtr_path_t;
+
+#define GTR_ABI_VERSION 1
+
+/* ABI version of the loaded library (GTR_ABI_VERSION). */
+GTR_API int gtr_abi_version(void);
+
+/* Static text for a status code; never NULL. */
+GTR_API const char *gtr_status_string(int status);
+
+/*
+ * Gate projection (GTR article 方法详解 §1, low-rank forget gate with
+ * temperature):  g[n, j] = logsigmoid(sum_r (x[n,:] . w_down[:,r]) w_up[r,j]
+ *                                      + bias[j]) / tau,    j < H*dk.
+ *   x       [B*T, d_model] in x_dtype (gtr_dtype_t)
+ *   w_down  [d_model, rank] fp32, w_up [rank, H*dk] fp32, bias [H*dk] fp32 or
+ *           NULL (zero), g_out [B*T, H*dk] fp32 = the [B, T, H, dk] gate of
+ *           gtr_gla_fwd.  logsigmoid uses the overflow-free form
+ *           min(u,0) - log1p(exp(-|u|)), so g <= 0 always.
+ *   Limits: 1 <= rank <= 64, d_model <= 4096, H*dk <= 4096, tau > 0 finite.
+ */
+GTR_API gtr_status_t gtr_gate_fwd(const void *x, int x_dtype, const float *w_down, const float *w_up,
+                          const float *bias, float *g_out, int B, int T, int d_model, int rank,
+                          int H, int dk, float tau, void *stream);
+
+/*
+ * Key-only GLA forward with the fused RMSNorm x SiLU output gate (GTR article
+ * 方法详解 §1 and §4; see the top of this file for the exact definition).
+ *   q, k [B,T,H,dk], v, outgate (= z), out [B,T,H,dv] in `dtype`; g [B,T,H,dk]
+ *   fp32 (log forget gate, expected <= 0; values > 0 are computed as given);
+ *   rms_w [dv] fp32 or NULL (all ones), shared by all heads.
+ *   dk, dv in {16, 32, 64, 128}; chunk (the chunk length C) in {16, 32, 64,
+ *   128}; the result does not depend on C beyond rounding.  T = grid_h*grid_w
+ *   must fit in an int.  `out` must not alias any input.
+ *   Workspace: fp32 segment states taken from a library-owned buffer cached
+ *   per (device, stream) and grown on demand with cudaMalloc (so the first call
+ *   for a shape must not happen during stream capture), or from the buffer
+ *   registered with gtr_gla_set_workspace.  Calls on one stream are ordered;
+ *   calls that share a registered workspace on different streams race.
+ */
+GTR_API gtr_status_t gtr_gla_fwd(const void *q, const void *k, const void *v, const float *g,
+                         const void *outgate, const float *rms_w, void *out, int B, int H,
+                         int grid_h, int grid_w, int dk, int dv, int dir, int chunk, int dtype,
+                         void *stream);
+
+/*
+ * gtr_gla_fwd that also records caller-created cudaEvent_t handles (any may be
+ * NULL) on `stream`: ev[0] before the summary kernel, ev[1] after it, ev[2]
+ * after the state scan, ev[3] after the output kernel.  For profiling only.
+ */
+GTR_API gtr_status_t gtr_gla_fwd_timed(const void *q, const void *k, const void *v, const float *g,
+                               const void *outgate, const float *rms_w, void *out, int B, int H,
+                               int grid_h, int grid_w, int dk, int dv, int dir, int chunk,
+                               int dtype, void *stream, void *const *ev);
+
+/*
+ * Chunk-boundary states, for testing the first two stages on their own: the
+ * state each chunk of `chunk` scan positions ends with,
+ *   states [B, H, ceil(T/chunk), dk, dv] fp32, entry c = S after scan position
+ *   min((c+1)*chunk, T) - 1 (GTR article 方法详解 §4, boundary states).
+ * Runs the summary and scan stages with one chunk per segment on `stream`.
+ */
+GTR_API gtr_status_t gtr_gla_chunk_states(const void *k, const void *v, const float *g, float *states,
+                                  int B, int H, int grid_h, int grid_w, int dk, int dv, int dir,
+                                  int chunk, int dtype, void *stream);
+
+/* Bytes of workspace gtr_gla_fwd needs for this problem on the current device
+ * (0 for an empty problem, (size_t)-1 for invalid arguments). */
+GTR_API size_t gtr_gla_workspace_bytes(int B, int H, int grid_h, int grid_w, int dk, int dv, int chunk,
+                               int dtype);
+
+/* Register a caller-owned device buffer as the workspace of the current device
+ * (ptr 256-byte aligned).  NULL releases it: calls go back to the
+ * library-owned buffers.  The caller keeps ownership and must keep the buffer
+ * alive while calls that use it are in flight. */
+GTR_API gtr_status_t gtr_gla_set_workspace(void *ptr, size_t bytes);
+
+/* Select the kernel family (gtr_path_t) of later gtr_gla_fwd calls in this
+ * process; GTR_ERR_UNSUPPORTED later if a forced path cannot run a shape. */
+GTR_API gtr_status_t gtr_gla_set_path(int path);
+
+/* The kernel family gtr_gla_fwd would use for this problem under the current
+ * setting (GTR_PATH_SIMT or GTR_PATH_TC), or a negative status. */
+GTR_API int gtr_gla_path_for(int B, int H, int grid_h, int grid_w, int dk, int dv, int chunk, int dtype);
+
+/*
+ * Device-side status of the current device: synchronises `stream`, returns
+ * GTR_OK if no kernel recorded a failed check since the last call, else
+ * GTR_ERR_DEVICE_CHECK, and clears the record.  If `counters` is not NULL it
+ * receives {status bits, chunks that took the exact-decay path of the
+ * tensor-core kernels} accumulated since the last call.
+ */
+GTR_API gtr_status_t gtr_last_device_status(void *stream, unsigned long long *counters);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GTR_GLA_H */

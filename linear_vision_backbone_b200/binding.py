@@ -1,0 +1,207 @@
+"""Thin ctypes binding of ``include/gtr_gla.h`` (argument marshalling only).
+
+Every step of the operator runs inside ``_build/libgtr_gla.so``; this module
+only checks torch tensors, passes their device pointers and the current CUDA
+stream through the C ABI, and turns status codes into exceptions.  There is no
+Python or CPU fallback: if the library is missing the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_build", "libgtr_gla.so")
+
+DTYPE_IDS = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
+DIR_IDS = {"LR": 0, "RL": 1, "TB": 2, "BT": 3, "ROTATE": 4}
+PATH_IDS = {"auto": 0, "simt": 1, "tc": 2}
+PATH_NAMES = {1: "simt", 2: "tc"}
+
+EXPORTS = (
+    "gtr_abi_version", "gtr_status_string", "gtr_gate_fwd", "gtr_gla_fwd", "gtr_gla_fwd_timed",
+    "gtr_gla_chunk_states", "gtr_gla_workspace_bytes", "gtr_gla_set_workspace",
+    "gtr_gla_set_path", "gtr_gla_path_for", "gtr_last_device_status",
+)
+
+_lock = threading.Lock()
+_lib = None
+
+
+class GtrError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn} failed: {msg} (status {status})")
+        self.status = status
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"CUDA library {path} is missing; build it with "
+                "`python -m linear_vision_backbone_b200.build` (there is no fallback)")
+        lib = ctypes.CDLL(path)
+        P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        sig = {
+            "gtr_abi_version": ([], I),
+            "gtr_status_string": ([I], ctypes.c_char_p),
+            "gtr_gate_fwd": ([P, I, P, P, P, P, I, I, I, I, I, I, F, P], I),
+            "gtr_gla_fwd": ([P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, P], I),
+            "gtr_gla_fwd_timed": ([P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, P, P], I),
+            "gtr_gla_chunk_states": ([P, P, P, P, I, I, I, I, I, I, I, I, I, P], I),
+            "gtr_gla_workspace_bytes": ([I, I, I, I, I, I, I, I], Z),
+            "gtr_gla_set_workspace": ([P, Z], I),
+            "gtr_gla_set_path": ([I], I),
+            "gtr_gla_path_for": ([I, I, I, I, I, I, I, I], I),
+            "gtr_last_device_status": ([P, P], I),
+        }
+        for name, (args, res) in sig.items():
+            fn = getattr(lib, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = lib
+        return lib
+
+
+def _check(fn: str, rc: int) -> None:
+    if rc != 0:
+        msg = load().gtr_status_string(rc).decode()
+        raise GtrError(fn, rc, msg)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype=None, shape=None) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def gate_fwd(x: torch.Tensor, w_down: torch.Tensor, w_up: torch.Tensor,
+             bias: Optional[torch.Tensor], H: int, dk: int, tau: float = 16.0,
+             out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """g = logsigmoid(x W_down W_up + bias) / tau as [B, T, H, dk] fp32 (``gtr_gate_fwd``)."""
+    _need(x, "x")
+    if x.dim() != 3:
+        raise ValueError("x must be [B, T, d_model]")
+    B, T, dm = x.shape
+    rank = w_down.shape[1]
+    _need(w_down, "w_down", torch.float32, (dm, rank))
+    _need(w_up, "w_up", torch.float32, (rank, H * dk))
+    if bias is not None:
+        _need(bias, "bias", torch.float32, (H * dk,))
+    if out is None:
+        out = torch.empty(B, T, H, dk, device=x.device, dtype=torch.float32)
+    _need(out, "out", torch.float32, (B, T, H, dk))
+    rc = load().gtr_gate_fwd(_ptr(x), DTYPE_IDS[x.dtype], _ptr(w_down), _ptr(w_up), _ptr(bias),
+                             _ptr(out), B, T, dm, rank, H, dk, float(tau), _stream(stream))
+    _check("gtr_gate_fwd", rc)
+    return out
+
+
+def _gla_check(q, k, v, g, z, w, out, grid_h, grid_w):
+    for name, t in (("q", q), ("k", k), ("v", v), ("z", z)):
+        _need(t, name, q.dtype)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if T != grid_h * grid_w:
+        raise ValueError(f"T={T} != grid_h*grid_w={grid_h * grid_w}")
+    _need(k, "k", q.dtype, (B, T, H, dk))
+    _need(v, "v", q.dtype, (B, T, H, dv))
+    _need(z, "z", q.dtype, (B, T, H, dv))
+    _need(g, "g", torch.float32, (B, T, H, dk))
+    if w is not None:
+        _need(w, "w", torch.float32, (dv,))
+    if out is None:
+        out = torch.empty(B, T, H, dv, device=q.device, dtype=q.dtype)
+    _need(out, "out", q.dtype, (B, T, H, dv))
+    return B, T, H, dk, dv, out
+
+
+def gla_fwd(q, k, v, g, z, w=None, *, grid_h: int, grid_w: int, direction: str = "LR",
+            chunk: int = 64, out: Optional[torch.Tensor] = None, stream=None,
+            events: Optional[Sequence] = None) -> torch.Tensor:
+    """y = RMSNorm(o) * w * SiLU(z) of the Key-only GLA (``gtr_gla_fwd``).
+
+    q, k: [B, T, H, dk]; v, z: [B, T, H, dv] (one dtype); g: [B, T, H, dk] fp32;
+    w: [dv] fp32 or None.  ``events`` (4 torch.cuda.Event or None) are recorded
+    around the three stages on the launch stream (``gtr_gla_fwd_timed``).
+    """
+    B, T, H, dk, dv, out = _gla_check(q, k, v, g, z, w, out, grid_h, grid_w)
+    lib = load()
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(z), _ptr(w), _ptr(out), B, H, grid_h, grid_w,
+            dk, dv, DIR_IDS[direction], int(chunk), DTYPE_IDS[q.dtype], _stream(stream))
+    if events is None:
+        _check("gtr_gla_fwd", lib.gtr_gla_fwd(*args))
+    else:
+        arr = (ctypes.c_void_p * 4)(*[None if e is None else e.cuda_event for e in events])
+        _check("gtr_gla_fwd_timed", lib.gtr_gla_fwd_timed(*args, arr))
+    return out
+
+
+def chunk_states(k, v, g, *, grid_h: int, grid_w: int, direction: str = "LR", chunk: int = 64,
+                 stream=None) -> torch.Tensor:
+    """State each chunk ends with: [B, H, ceil(T/chunk), dk, dv] fp32 (``gtr_gla_chunk_states``)."""
+    _need(k, "k")
+    B, T, H, dk = k.shape
+    dv = v.shape[-1]
+    _need(v, "v", k.dtype, (B, T, H, dv))
+    _need(g, "g", torch.float32, (B, T, H, dk))
+    nc = (T + chunk - 1) // chunk
+    st = torch.empty(B, H, nc, dk, dv, device=k.device, dtype=torch.float32)
+    rc = load().gtr_gla_chunk_states(_ptr(k), _ptr(v), _ptr(g), _ptr(st), B, H, grid_h, grid_w,
+                                     dk, dv, DIR_IDS[direction], int(chunk), DTYPE_IDS[k.dtype],
+                                     _stream(stream))
+    _check("gtr_gla_chunk_states", rc)
+    return st
+
+
+def set_path(path: str) -> None:
+    _check("gtr_gla_set_path", load().gtr_gla_set_path(PATH_IDS[path]))
+
+
+def path_for(B, H, grid_h, grid_w, dk, dv, chunk, dtype) -> str:
+    rc = load().gtr_gla_path_for(B, H, grid_h, grid_w, dk, dv, chunk, DTYPE_IDS[dtype])
+    if rc < 0:
+        _check("gtr_gla_path_for", rc)
+    return PATH_NAMES[rc]
+
+
+def workspace_bytes(B, H, grid_h, grid_w, dk, dv, chunk, dtype) -> int:
+    return int(load().gtr_gla_workspace_bytes(B, H, grid_h, grid_w, dk, dv, chunk, DTYPE_IDS[dtype]))
+
+
+def set_workspace(buf: Optional[torch.Tensor]) -> None:
+    if buf is None:
+        _check("gtr_gla_set_workspace", load().gtr_gla_set_workspace(None, 0))
+    else:
+        _need(buf, "workspace")
+        nbytes = buf.numel() * buf.element_size()
+        _check("gtr_gla_set_workspace", load().gtr_gla_set_workspace(_ptr(buf), nbytes))
+
+
+def device_status(stream=None):
+    """(status, exact_chunks): synchronises the stream and clears the device record."""
+    counters = (ctypes.c_ulonglong * 2)()
+    rc = load().gtr_last_device_status(_stream(stream), counters)
+    return rc, int(counters[0]), int(counters[1])

@@ -1,0 +1,390 @@
+// gtr_gla.cu -- the C ABI of include/gtr_gla.h and the host side of every
+// kernel launch.  Argument checks, the segment plan, workspace management and
+// the stage sequence K2 (summary) -> K3 (boundary scan) -> K4 (output) of the
+// chunkwise operator (GTR article, 方法详解 §4) live here; the kernels live in
+// the included .cuh files.  The whole library is this one translation unit.
+#include <atomic>
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "gtr_gla.h"
+#include "common.cuh"
+#include "gate_kernels.cuh"
+#include "simt_kernels.cuh"
+#include "scan_kernel.cuh"
+#include "tc_kernels.cuh"
+
+namespace {
+
+using namespace gtr;
+
+std::atomic<int> g_path_setting{GTR_PATH_AUTO};
+std::mutex g_mu;
+constexpr int kMaxDevices = 64;
+int g_sm_count[kMaxDevices];
+void* g_user_ws[kMaxDevices];
+size_t g_user_ws_bytes[kMaxDevices];
+std::map<std::pair<int, void*>, std::pair<void*, size_t>> g_ws;   // (device, stream) -> buffer
+
+bool valid_head_dim(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+bool valid_chunk(int c) { return c == 16 || c == 32 || c == 64 || c == 128; }
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+int current_device(int* dev) {
+  if (cudaGetDevice(dev) != cudaSuccess) return GTR_ERR_CUDA;
+  if (*dev < 0 || *dev >= kMaxDevices) return GTR_ERR_UNSUPPORTED;
+  return GTR_OK;
+}
+
+int sm_count(int dev) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_sm_count[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    g_sm_count[dev] = n;
+  }
+  return g_sm_count[dev];
+}
+
+// Plan of one gtr_gla_fwd call: chunk length, segment length (a run of
+// consecutive chunks one block of K2/K4 walks through) and workspace layout.
+struct Plan {
+  int B, H, gh, gw, T, dk, dv, dir, chunk, dtype;
+  int path;        // GTR_PATH_SIMT or GTR_PATH_TC
+  int nc;          // chunks per sequence
+  int seg_chunks;  // chunks per segment
+  int nseg;        // segments per sequence
+  int seg_len;     // scan positions per segment
+  size_t offL;     // byte offset of the log-decay array in the workspace
+  size_t ws_bytes;
+};
+
+// Segment length that balances the blocks over the resident slots: minimise
+// (rounds of resident blocks) x (chunks per block); on ties take the longer
+// segment, which moves fewer boundary states through memory.
+int plan_segments(long long bh, int nc, long long slots) {
+  int best = 1;
+  long long best_cost = -1;
+  const int mmax = nc < 65536 ? nc : 65536;
+  for (int m = 1; m <= mmax; ++m) {
+    const long long units = bh * ((nc + m - 1) / m);
+    const long long cost = ((units + slots - 1) / slots) * m;
+    if (best_cost < 0 || cost <= best_cost) { best_cost = cost; best = m; }
+  }
+  return best;
+}
+
+int check_gla_args(int B, int H, int gh, int gw, int dk, int dv, int dir, int chunk, int dtype) {
+  if (B < 0 || H < 0 || gh < 0 || gw < 0) return GTR_ERR_INVALID_ARG;
+  if (dir < 0 || dir > 4) return GTR_ERR_INVALID_ARG;
+  if (dtype < 0 || dtype > 2) return GTR_ERR_INVALID_ARG;
+  if (!valid_head_dim(dk) || !valid_head_dim(dv) || !valid_chunk(chunk)) return GTR_ERR_UNSUPPORTED;
+  const long long T = (long long)gh * gw;
+  if (T > 0x7fffffffLL) return GTR_ERR_INVALID_ARG;
+  // every element offset must fit in 63 bits with room to spare
+  const long long rows = (long long)B * T * H;
+  if (B > 0 && H > 0 && T > 0 && rows / ((long long)B * H) != T) return GTR_ERR_INVALID_ARG;
+  if (rows > (1LL << 46)) return GTR_ERR_INVALID_ARG;
+  return GTR_OK;
+}
+
+bool tc_supported(int dk, int dv, int chunk, int dtype) {
+  return tc_shape_supported(dk, dv, chunk, dtype);
+}
+
+int choose_path(int dk, int dv, int chunk, int dtype) {
+  const int setting = g_path_setting.load();
+  if (setting == GTR_PATH_SIMT) return GTR_PATH_SIMT;
+  if (setting == GTR_PATH_TC) return tc_supported(dk, dv, chunk, dtype) ? (int)GTR_PATH_TC : (int)GTR_ERR_UNSUPPORTED;
+  return tc_supported(dk, dv, chunk, dtype) ? (int)GTR_PATH_TC : (int)GTR_PATH_SIMT;
+}
+
+int make_plan(Plan* p, int dev, int B, int H, int gh, int gw, int dk, int dv, int dir, int chunk,
+              int dtype, int force_seg_chunks) {
+  p->B = B; p->H = H; p->gh = gh; p->gw = gw; p->T = gh * gw;
+  p->dk = dk; p->dv = dv; p->dir = dir; p->chunk = chunk; p->dtype = dtype;
+  const int path = choose_path(dk, dv, chunk, dtype);
+  if (path < 0) return path;
+  p->path = path;
+  p->nc = (p->T + chunk - 1) / chunk;
+  const long long bh = (long long)B * H;
+  const long long slots = (long long)sm_count(dev) * (path == GTR_PATH_TC ? tc_blocks_per_sm(dk, dv) : 4);
+  p->seg_chunks = force_seg_chunks > 0 ? force_seg_chunks : plan_segments(bh, p->nc, slots);
+  p->nseg = (p->nc + p->seg_chunks - 1) / p->seg_chunks;
+  p->seg_len = p->seg_chunks * chunk;
+  const size_t nS = (size_t)bh * p->nseg * dk * dv * sizeof(float);
+  p->offL = (nS + 255) & ~(size_t)255;
+  p->ws_bytes = p->offL + (size_t)bh * p->nseg * dk * sizeof(float);
+  return GTR_OK;
+}
+
+// Workspace of `bytes` for (device, stream): the registered caller buffer, or
+// a cached library buffer grown with cudaMalloc outside stream capture.
+int get_workspace(int dev, void* stream, size_t bytes, void** out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_user_ws[dev]) {
+    if (bytes > g_user_ws_bytes[dev]) return GTR_ERR_NO_MEMORY;
+    *out = g_user_ws[dev];
+    return GTR_OK;
+  }
+  auto key = std::make_pair(dev, stream);
+  auto it = g_ws.find(key);
+  if (it != g_ws.end() && it->second.second >= bytes) { *out = it->second.first; return GTR_OK; }
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing((cudaStream_t)stream, &cs) != cudaSuccess) return GTR_ERR_CUDA;
+  if (cs != cudaStreamCaptureStatusNone) return GTR_ERR_NO_MEMORY;
+  if (it != g_ws.end()) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return GTR_ERR_CUDA;
+    cudaFree(it->second.first);
+    g_ws.erase(it);
+  }
+  size_t want = bytes < ((size_t)1 << 20) ? ((size_t)1 << 20) : bytes + bytes / 4;
+  void* p = nullptr;
+  if (cudaMalloc(&p, want) != cudaSuccess) { (void)cudaGetLastError(); return GTR_ERR_NO_MEMORY; }
+  g_ws[key] = std::make_pair(p, want);
+  *out = p;
+  return GTR_OK;
+}
+
+int launch_status() {
+  return cudaGetLastError() == cudaSuccess ? GTR_OK : GTR_ERR_CUDA;
+}
+
+template <typename T, int ROWS>
+int launch_simt_rows(const Plan& p, const void* q, const void* k, const void* v, const float* g,
+                     const void* z, const float* w, void* out, float* wsS, float* wsL,
+                     cudaStream_t st, int stage) {
+  const dim3 grid(p.nseg, p.B * p.H);
+  if (stage == 0) {
+    const size_t smem = (size_t)simt_summary_smem_floats(p.dk, p.dv) * sizeof(float);
+    auto kern = gla_summary_simt<T, ROWS>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return GTR_ERR_CUDA;
+    kern<<<grid, kSimtThreads, smem, st>>>((const T*)k, (const T*)v, g, wsS, wsL, p.H, p.T, p.gh,
+                                           p.gw, p.dk, p.dv, p.dir, p.seg_len, p.nseg);
+  } else {
+    const size_t smem = (size_t)simt_output_smem_floats(p.dk, p.dv) * sizeof(float);
+    auto kern = gla_output_simt<T, ROWS>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return GTR_ERR_CUDA;
+    kern<<<grid, kSimtThreads, smem, st>>>((const T*)q, (const T*)k, (const T*)v, g, (const T*)z, w,
+                                           wsS, (T*)out, p.H, p.T, p.gh, p.gw, p.dk, p.dv, p.dir,
+                                           p.seg_len, p.nseg);
+  }
+  return launch_status();
+}
+
+template <typename T>
+int launch_simt(const Plan& p, const void* q, const void* k, const void* v, const float* g,
+                const void* z, const float* w, void* out, float* wsS, float* wsL, cudaStream_t st,
+                int stage) {
+  switch ((p.dk * p.dv) / kSimtThreads) {
+    case 1: return launch_simt_rows<T, 1>(p, q, k, v, g, z, w, out, wsS, wsL, st, stage);
+    case 2: return launch_simt_rows<T, 2>(p, q, k, v, g, z, w, out, wsS, wsL, st, stage);
+    case 4: return launch_simt_rows<T, 4>(p, q, k, v, g, z, w, out, wsS, wsL, st, stage);
+    case 8: return launch_simt_rows<T, 8>(p, q, k, v, g, z, w, out, wsS, wsL, st, stage);
+    case 16: return launch_simt_rows<T, 16>(p, q, k, v, g, z, w, out, wsS, wsL, st, stage);
+    case 32: return launch_simt_rows<T, 32>(p, q, k, v, g, z, w, out, wsS, wsL, st, stage);
+    case 64: return launch_simt_rows<T, 64>(p, q, k, v, g, z, w, out, wsS, wsL, st, stage);
+    default: return GTR_ERR_UNSUPPORTED;
+  }
+}
+
+// stage 0 = K2 summary, 1 = K4 output
+int launch_stage(const Plan& p, const void* q, const void* k, const void* v, const float* g,
+                 const void* z, const float* w, void* out, float* wsS, float* wsL, cudaStream_t st,
+                 int stage) {
+  if (p.path == GTR_PATH_TC)
+    return launch_tc(p.dtype, stage, q, k, v, g, z, w, out, wsS, wsL, p.B, p.H, p.T, p.gh, p.gw,
+                     p.dk, p.dv, p.dir, p.chunk, p.seg_chunks, p.nseg, st);
+  switch (p.dtype) {
+    case GTR_F32: return launch_simt<float>(p, q, k, v, g, z, w, out, wsS, wsL, st, stage);
+    case GTR_F16: return launch_simt<__half>(p, q, k, v, g, z, w, out, wsS, wsL, st, stage);
+    case GTR_BF16: return launch_simt<__nv_bfloat16>(p, q, k, v, g, z, w, out, wsS, wsL, st, stage);
+  }
+  return GTR_ERR_INVALID_ARG;
+}
+
+int launch_scan(const Plan& p, float* wsS, const float* wsL, int inclusive, cudaStream_t st) {
+  const long long total = (long long)p.B * p.H * p.dk * p.dv;
+  const long long blocks = (total + kScanThreads - 1) / kScanThreads;
+  gla_state_scan<<<(unsigned)blocks, kScanThreads, 0, st>>>(wsS, wsL, total, p.nseg, p.dk, p.dv,
+                                                           inclusive);
+  return launch_status();
+}
+
+int record(void* const* ev, int i, cudaStream_t st) {
+  if (ev && ev[i]) return cudaEventRecord((cudaEvent_t)ev[i], st) == cudaSuccess ? GTR_OK : GTR_ERR_CUDA;
+  return GTR_OK;
+}
+
+int gla_fwd_impl(const void* q, const void* k, const void* v, const float* g, const void* z,
+                 const float* w, void* out, int B, int H, int gh, int gw, int dk, int dv, int dir,
+                 int chunk, int dtype, void* stream, void* const* ev) {
+  int rc = check_gla_args(B, H, gh, gw, dk, dv, dir, chunk, dtype);
+  if (rc) return rc;
+  if (B == 0 || H == 0 || gh == 0 || gw == 0) return GTR_OK;
+  if (!q || !k || !v || !g || !z || !out) return GTR_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(z) ||
+      !aligned16(out) || (w && !aligned16(w)))
+    return GTR_ERR_ALIGNMENT;
+  int dev;
+  if ((rc = current_device(&dev))) return rc;
+  Plan p;
+  if ((rc = make_plan(&p, dev, B, H, gh, gw, dk, dv, dir, chunk, dtype, 0))) return rc;
+  void* ws = nullptr;
+  if ((rc = get_workspace(dev, stream, p.ws_bytes, &ws))) return rc;
+  float* wsS = (float*)ws;
+  float* wsL = (float*)((char*)ws + p.offL);
+  cudaStream_t st = (cudaStream_t)stream;
+  if ((rc = record(ev, 0, st))) return rc;
+  if ((rc = launch_stage(p, q, k, v, g, z, w, out, wsS, wsL, st, 0))) return rc;
+  if ((rc = record(ev, 1, st))) return rc;
+  if ((rc = launch_scan(p, wsS, wsL, 0, st))) return rc;
+  if ((rc = record(ev, 2, st))) return rc;
+  if ((rc = launch_stage(p, q, k, v, g, z, w, out, wsS, wsL, st, 1))) return rc;
+  return record(ev, 3, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int gtr_abi_version(void) { return GTR_ABI_VERSION; }
+
+const char* gtr_status_string(int status) {
+  switch (status) {
+    case GTR_OK: return "ok";
+    case GTR_ERR_INVALID_ARG: return "invalid argument";
+    case GTR_ERR_UNSUPPORTED: return "unsupported shape or option";
+    case GTR_ERR_ALIGNMENT: return "tensor pointer not 16-byte aligned";
+    case GTR_ERR_NO_MEMORY: return "workspace unavailable";
+    case GTR_ERR_CUDA: return "CUDA runtime or launch error";
+    case GTR_ERR_DEVICE_CHECK: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+gtr_status_t gtr_gate_fwd(const void* x, int x_dtype, const float* w_down, const float* w_up,
+                          const float* bias, float* g_out, int B, int T, int d_model, int rank,
+                          int H, int dk, float tau, void* stream) {
+  if (B < 0 || T < 0 || H < 0 || dk < 0 || d_model <= 0 || rank <= 0) return GTR_ERR_INVALID_ARG;
+  if (x_dtype < 0 || x_dtype > 2) return GTR_ERR_INVALID_ARG;
+  if (!(tau > 0.0f) || !(tau < 3.0e38f)) return GTR_ERR_INVALID_ARG;
+  if (rank > kGateMaxRank || d_model > 4096 || (long long)H * dk > 4096) return GTR_ERR_UNSUPPORTED;
+  const long long N = (long long)B * T;
+  if (N == 0 || H == 0 || dk == 0) return GTR_OK;
+  if (N > (1LL << 40)) return GTR_ERR_INVALID_ARG;
+  if (!x || !w_down || !w_up || !g_out) return GTR_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(g_out) || !aligned16(w_down) || !aligned16(w_up) ||
+      (bias && !aligned16(bias)))
+    return GTR_ERR_ALIGNMENT;
+  const int HD = H * dk;
+  const long long blocks = (N + kGateTok - 1) / kGateTok;
+  if (blocks > 0x7fffffffLL) return GTR_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  switch (x_dtype) {
+    case GTR_F32:
+      gate_proj_kernel<float><<<(unsigned)blocks, kGateThreads, 0, st>>>(
+          (const float*)x, w_down, w_up, bias, g_out, N, d_model, rank, HD, tau);
+      break;
+    case GTR_F16:
+      gate_proj_kernel<__half><<<(unsigned)blocks, kGateThreads, 0, st>>>(
+          (const __half*)x, w_down, w_up, bias, g_out, N, d_model, rank, HD, tau);
+      break;
+    default:
+      gate_proj_kernel<__nv_bfloat16><<<(unsigned)blocks, kGateThreads, 0, st>>>(
+          (const __nv_bfloat16*)x, w_down, w_up, bias, g_out, N, d_model, rank, HD, tau);
+      break;
+  }
+  return (gtr_status_t)launch_status();
+}
+
+gtr_status_t gtr_gla_fwd(const void* q, const void* k, const void* v, const float* g,
+                         const void* outgate, const float* rms_w, void* out, int B, int H,
+                         int grid_h, int grid_w, int dk, int dv, int dir, int chunk, int dtype,
+                         void* stream) {
+  return (gtr_status_t)gla_fwd_impl(q, k, v, g, outgate, rms_w, out, B, H, grid_h, grid_w, dk, dv,
+                                    dir, chunk, dtype, stream, nullptr);
+}
+
+gtr_status_t gtr_gla_fwd_timed(const void* q, const void* k, const void* v, const float* g,
+                               const void* outgate, const float* rms_w, void* out, int B, int H,
+                               int grid_h, int grid_w, int dk, int dv, int dir, int chunk,
+                               int dtype, void* stream, void* const* ev) {
+  return (gtr_status_t)gla_fwd_impl(q, k, v, g, outgate, rms_w, out, B, H, grid_h, grid_w, dk, dv,
+                                    dir, chunk, dtype, stream, ev);
+}
+
+gtr_status_t gtr_gla_chunk_states(const void* k, const void* v, const float* g, float* states,
+                                  int B, int H, int grid_h, int grid_w, int dk, int dv, int dir,
+                                  int chunk, int dtype, void* stream) {
+  int rc = check_gla_args(B, H, grid_h, grid_w, dk, dv, dir, chunk, dtype);
+  if (rc) return (gtr_status_t)rc;
+  if (B == 0 || H == 0 || grid_h == 0 || grid_w == 0) return GTR_OK;
+  if (!k || !v || !g || !states) return GTR_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(states)) return GTR_ERR_ALIGNMENT;
+  int dev;
+  if ((rc = current_device(&dev))) return (gtr_status_t)rc;
+  Plan p;
+  if ((rc = make_plan(&p, dev, B, H, grid_h, grid_w, dk, dv, dir, chunk, dtype, 1)))
+    return (gtr_status_t)rc;
+  void* ws = nullptr;
+  const size_t lbytes = (size_t)B * H * p.nseg * dk * sizeof(float);
+  if ((rc = get_workspace(dev, stream, lbytes, &ws))) return (gtr_status_t)rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  if ((rc = launch_stage(p, nullptr, k, v, g, nullptr, nullptr, nullptr, states, (float*)ws, st, 0)))
+    return (gtr_status_t)rc;
+  return (gtr_status_t)launch_scan(p, states, (const float*)ws, 1, st);
+}
+
+size_t gtr_gla_workspace_bytes(int B, int H, int grid_h, int grid_w, int dk, int dv, int chunk,
+                               int dtype) {
+  if (check_gla_args(B, H, grid_h, grid_w, dk, dv, 0, chunk, dtype)) return (size_t)-1;
+  if (B == 0 || H == 0 || grid_h == 0 || grid_w == 0) return 0;
+  int dev;
+  if (current_device(&dev)) return (size_t)-1;
+  Plan p;
+  if (make_plan(&p, dev, B, H, grid_h, grid_w, dk, dv, 0, chunk, dtype, 0)) return (size_t)-1;
+  return p.ws_bytes;
+}
+
+gtr_status_t gtr_gla_set_workspace(void* ptr, size_t bytes) {
+  int dev;
+  int rc = current_device(&dev);
+  if (rc) return (gtr_status_t)rc;
+  if (ptr && ((uintptr_t)ptr & 255u)) return GTR_ERR_ALIGNMENT;
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_user_ws[dev] = ptr;
+  g_user_ws_bytes[dev] = ptr ? bytes : 0;
+  return GTR_OK;
+}
+
+gtr_status_t gtr_gla_set_path(int path) {
+  if (path < GTR_PATH_AUTO || path > GTR_PATH_TC) return GTR_ERR_INVALID_ARG;
+  g_path_setting.store(path);
+  return GTR_OK;
+}
+
+int gtr_gla_path_for(int B, int H, int grid_h, int grid_w, int dk, int dv, int chunk, int dtype) {
+  int rc = check_gla_args(B, H, grid_h, grid_w, dk, dv, 0, chunk, dtype);
+  if (rc) return rc;
+  return choose_path(dk, dv, chunk, dtype);
+}
+
+gtr_status_t gtr_last_device_status(void* stream, unsigned long long* counters) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return GTR_ERR_CUDA;
+  unsigned int st = 0;
+  unsigned long long ex = 0;
+  const unsigned int zero = 0;
+  const unsigned long long zero64 = 0;
+  if (cudaMemcpyFromSymbol(&st, g_gtr_status, sizeof(st)) != cudaSuccess) return GTR_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&ex, g_gtr_exact_chunks, sizeof(ex)) != cudaSuccess) return GTR_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_gtr_status, &zero, sizeof(zero)) != cudaSuccess) return GTR_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_gtr_exact_chunks, &zero64, sizeof(zero64)) != cudaSuccess) return GTR_ERR_CUDA;
+  if (counters) { counters[0] = st; counters[1] = ex; }
+  return st ? GTR_ERR_DEVICE_CHECK : GTR_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,86 @@
+"""The C ABI library loads and exports every entry point of include/gtr_gla.h.
+
+CPU only: no call here launches work or touches a device.  Argument checks
+run before any CUDA call, so invalid arguments are rejected on any machine.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from linear_vision_backbone_b200 import binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gtr_gla.h")
+
+
+def header_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"GTR_API\s+[^;(]*?\b(gtr_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.load()
+
+
+def test_header_declares_the_abi():
+    syms = header_symbols()
+    assert set(syms) == set(binding.EXPORTS), syms
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", binding.LIB_PATH], check=True,
+                         capture_output=True, text=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    for s in header_symbols():
+        assert s in exported, s
+        assert getattr(lib, s) is not None
+    # nothing else leaks out of the library
+    assert {s for s in exported if s.startswith("gtr_")} == set(header_symbols())
+
+
+def test_version_and_status_strings(lib):
+    assert lib.gtr_abi_version() == 1
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert lib.gtr_status_string(code)
+    assert lib.gtr_status_string(12345) == b"unknown status"
+
+
+def test_invalid_arguments_rejected_before_any_launch(lib):
+    P = ctypes.c_void_p(16)
+    S = None
+    # bad direction, bad dtype, negative sizes, unsupported head dim / chunk
+    assert lib.gtr_gla_fwd(P, P, P, P, P, None, P, 1, 1, 4, 4, 64, 64, 7, 64, 1, S) == -1
+    assert lib.gtr_gla_fwd(P, P, P, P, P, None, P, 1, 1, 4, 4, 64, 64, 0, 64, 3, S) == -1
+    assert lib.gtr_gla_fwd(P, P, P, P, P, None, P, -1, 1, 4, 4, 64, 64, 0, 64, 1, S) == -1
+    assert lib.gtr_gla_fwd(P, P, P, P, P, None, P, 1, 1, 4, 4, 48, 64, 0, 64, 1, S) == -2
+    assert lib.gtr_gla_fwd(P, P, P, P, P, None, P, 1, 1, 4, 4, 64, 64, 0, 100, 1, S) == -2
+    # grid too large for an int
+    assert lib.gtr_gla_fwd(P, P, P, P, P, None, P, 1, 1, 65536, 65536, 64, 64, 0, 64, 1, S) == -1
+    # empty problems succeed without touching pointers or the device
+    assert lib.gtr_gla_fwd(None, None, None, None, None, None, None, 0, 6, 40, 40, 64, 64, 0, 64, 1, S) == 0
+    assert lib.gtr_gla_fwd(None, None, None, None, None, None, None, 1, 6, 0, 40, 64, 64, 0, 64, 1, S) == 0
+    # gate: bad rank, tau, dtype; rank above the limit is unsupported
+    assert lib.gtr_gate_fwd(P, 1, P, P, None, P, 1, 4, 384, 0, 6, 64, 16.0, S) == -1
+    assert lib.gtr_gate_fwd(P, 1, P, P, None, P, 1, 4, 384, 16, 6, 64, 0.0, S) == -1
+    assert lib.gtr_gate_fwd(P, 5, P, P, None, P, 1, 4, 384, 16, 6, 64, 16.0, S) == -1
+    assert lib.gtr_gate_fwd(P, 1, P, P, None, P, 1, 4, 384, 65, 6, 64, 16.0, S) == -2
+    assert lib.gtr_gate_fwd(None, 1, None, None, None, None, 0, 4, 384, 16, 6, 64, 16.0, S) == 0
+    assert lib.gtr_gla_set_path(9) == -1
+    assert lib.gtr_gla_workspace_bytes(1, 1, 4, 4, 48, 64, 64, 1) == ctypes.c_size_t(-1).value
+    assert lib.gtr_gla_workspace_bytes(0, 6, 40, 40, 64, 64, 64, 1) == 0
+
+
+def test_binding_refuses_a_missing_library(tmp_path):
+    with pytest.raises(RuntimeError, match="missing"):
+        # a fresh loader pointed at a path with no library fails loudly
+        saved = binding._lib
+        binding._lib = None
+        try:
+            binding.load(str(tmp_path / "nope.so"))
+        finally:
+            binding._lib = saved

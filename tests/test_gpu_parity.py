@@ -1,0 +1,265 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Every test runs the library on a B200 and compares, element by element, with
+the oracle on the same seeded inputs, under the rules of tests/parity.py.
+Workloads: the five of linear_vision_backbone_b200.inputs at full size (the
+launch configuration the benchmark times), plus ragged, degenerate and
+extreme-gate cases.
+"""
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_vision_backbone_b200 import binding, inputs
+from tests.parity import assert_close, compare
+
+pytestmark = pytest.mark.gpu
+
+DIRS = ("LR", "RL", "TB", "BT")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib(cuda_ok):
+    from linear_vision_backbone_b200 import build
+    build.build()
+    binding.load()
+    binding.set_path("auto")
+    yield
+    binding.set_path("auto")
+
+
+def _dev(t):
+    return t.cuda() if t is not None else None
+
+
+@functools.lru_cache(maxsize=None)
+def _workload_data(name, grid=None):
+    wl = inputs.WORKLOADS[name]
+    if grid is not None:
+        wl = wl.with_grid(grid)
+    return wl, inputs.make_inputs(wl)
+
+
+@functools.lru_cache(maxsize=None)
+def _oracle_gate(name, grid=None):
+    wl, d = _workload_data(name, grid)
+    return oracle.gate(d["x"], d["w_down"], d["w_up"], d["bias"], tau=wl.tau).reshape(
+        wl.B, wl.T, wl.H, wl.dk)
+
+
+@functools.lru_cache(maxsize=None)
+def _oracle_y(name, direction, grid=None):
+    wl, d = _workload_data(name, grid)
+    g = _oracle_gate(name, grid) if wl.recipe == "proj" else d["g"]
+    return oracle.gla_fwd(d["q"], d["k"], d["v"], g, d["z"], d["w"], gh=wl.gh, gw=wl.gw,
+                          direction=direction)
+
+
+def _gpu_step(wl, d, direction, chunk=None):
+    """The whole hot path on the GPU: gate projection (when the workload has
+    one) then the GLA forward, both through the C ABI."""
+    dv = {k: _dev(v) for k, v in d.items()}
+    if wl.recipe == "proj":
+        g = binding.gate_fwd(dv["x"], dv["w_down"], dv["w_up"], dv["bias"], wl.H, wl.dk, wl.tau)
+    else:
+        g = dv["g"]
+    y = binding.gla_fwd(dv["q"], dv["k"], dv["v"], g, dv["z"], dv["w"], grid_h=wl.gh, grid_w=wl.gw,
+                        direction=direction, chunk=chunk or wl.chunk)
+    torch.cuda.synchronize()
+    return y, g
+
+
+def _check_status():
+    rc, bits, _ = binding.device_status()
+    assert rc == 0 and bits == 0, (rc, bits)
+
+
+def test_tiny_fp32():
+    wl, d = _workload_data("tiny")
+    y, _ = _gpu_step(wl, d, "LR")
+    assert_close(y, _oracle_y("tiny", "LR"), torch.float32, "tiny")
+    _check_status()
+
+
+def test_gate_projection_640():
+    wl, d = _workload_data("640")
+    g = binding.gate_fwd(_dev(d["x"]), _dev(d["w_down"]), _dev(d["w_up"]), _dev(d["bias"]),
+                         wl.H, wl.dk, wl.tau)
+    ref = _oracle_gate("640")
+    got = g.double().cpu().numpy()
+    np.testing.assert_allclose(got, ref, rtol=1e-5, atol=1e-6)
+    assert np.all(got <= 0.0)
+
+
+def test_gate_projection_bf16_with_bias():
+    gen = torch.Generator().manual_seed(11)
+    x = torch.randn(3, 100, 384, generator=gen).to(torch.bfloat16)
+    wd = torch.randn(384, 16, generator=gen) / 384 ** 0.5
+    wu = torch.randn(16, 6 * 64, generator=gen) / 4
+    b = torch.randn(6 * 64, generator=gen) * 2
+    g = binding.gate_fwd(x.cuda(), wd.cuda(), wu.cuda(), b.cuda(), 6, 64, 16.0)
+    ref = oracle.gate(x, wd, wu, b, tau=16.0).reshape(3, 100, 6, 64)
+    np.testing.assert_allclose(g.double().cpu().numpy(), ref, rtol=1e-5, atol=1e-6)
+
+
+@pytest.mark.parametrize("direction", DIRS)
+def test_640_all_directions(direction):
+    wl, d = _workload_data("640")
+    y, _ = _gpu_step(wl, d, direction)
+    assert_close(y, _oracle_y("640", direction), torch.float16, f"640 {direction}")
+    _check_status()
+
+
+def test_640_batched_bf16_rotating_directions():
+    wl, d = _workload_data("640b8")
+    y, _ = _gpu_step(wl, d, "ROTATE")
+    assert_close(y, _oracle_y("640b8", "ROTATE"), torch.bfloat16, "640b8")
+    _check_status()
+
+
+@pytest.mark.parametrize("direction", ("TB", "BT"))
+def test_16k_strided_directions(direction):
+    wl, d = _workload_data("16k")
+    y, _ = _gpu_step(wl, d, direction)
+    assert_close(y, _oracle_y("16k", direction), torch.float16, f"16k {direction}")
+    _check_status()
+
+
+@pytest.mark.parametrize("grid", inputs.SWEEP_GRIDS)
+def test_scaling_sweep_bf16_d128(grid):
+    wl, d = _workload_data("sweep", grid)
+    y, _ = _gpu_step(wl, d, "LR")
+    assert_close(y, _oracle_y("sweep", "LR", grid), torch.bfloat16, f"sweep {grid}")
+    _check_status()
+
+
+def _run_custom(d, gh, gw, direction, chunk, dtype):
+    dv = {k: _dev(v) for k, v in d.items()}
+    y = binding.gla_fwd(dv["q"], dv["k"], dv["v"], dv["g"], dv["z"], dv["w"], grid_h=gh, grid_w=gw,
+                        direction=direction, chunk=chunk)
+    torch.cuda.synchronize()
+    ref = oracle.gla_fwd(d["q"], d["k"], d["v"], d["g"], d["z"], d["w"], gh=gh, gw=gw,
+                         direction=direction)
+    return y, ref
+
+
+@pytest.mark.parametrize("chunk", (16, 32, 64, 128))
+@pytest.mark.parametrize("direction", DIRS)
+def test_chunk_length_invariance_ragged_grid(chunk, direction):
+    gh, gw = 37, 29                                   # T = 1073: ragged for every chunk length
+    d = inputs.make_custom(2, 3, gh, gw, 64, 64, "f16", seed=21)
+    y, ref = _run_custom(d, gh, gw, direction, chunk, torch.float16)
+    assert_close(y, ref, torch.float16, f"chunk {chunk} {direction}")
+
+
+@pytest.mark.parametrize("path", ("simt", "auto"))
+@pytest.mark.parametrize("dtype", ("f16", "bf16"))
+def test_both_kernel_families(path, dtype):
+    gh, gw = 24, 40
+    d = inputs.make_custom(2, 4, gh, gw, 64, 64, dtype, seed=31, w_random=True)
+    binding.set_path(path)
+    try:
+        y, ref = _run_custom(d, gh, gw, "TB", 64, inputs.DTYPES[dtype])
+    finally:
+        binding.set_path("auto")
+    assert_close(y, ref, inputs.DTYPES[dtype], f"{path} {dtype}")
+
+
+@pytest.mark.parametrize("dk,dv,dtype", [(16, 16, "f32"), (32, 128, "bf16"), (128, 16, "f32"),
+                                         (64, 32, "f16"), (128, 128, "f16")])
+def test_head_dim_combinations(dk, dv, dtype):
+    gh, gw = 9, 23
+    d = inputs.make_custom(2, 2, gh, gw, dk, dv, dtype, seed=41, qk_std=dk ** -0.5)
+    for direction in ("LR", "BT"):
+        y, ref = _run_custom(d, gh, gw, direction, 32, inputs.DTYPES[dtype])
+        assert_close(y, ref, inputs.DTYPES[dtype], f"{dk}x{dv} {dtype} {direction}")
+
+
+@pytest.mark.parametrize("gh,gw", [(1, 1), (1, 5), (3, 1), (2, 3)])
+def test_tiny_and_degenerate_grids(gh, gw):
+    for dtype in ("f32", "f16"):
+        d = inputs.make_custom(3, 2, gh, gw, 64, 64, dtype, seed=51)
+        for direction in DIRS:
+            y, ref = _run_custom(d, gh, gw, direction, 16, inputs.DTYPES[dtype])
+            assert_close(y, ref, inputs.DTYPES[dtype], f"{gh}x{gw} {dtype} {direction}")
+
+
+def test_strong_decay_takes_the_exact_path():
+    # logsigmoid(N(-6, 1)) * 2 ~ -12 nats per token: the decay across one chunk
+    # far exceeds what a scaled operand can hold, so the tensor-core kernels
+    # must switch those chunks to the exact evaluation.
+    gh, gw = 16, 16
+    d = inputs.make_custom(1, 2, gh, gw, 64, 64, "f16", seed=61, g_mu=-6.0, g_scale=2.0)
+    binding.device_status()
+    y, ref = _run_custom(d, gh, gw, "LR", 64, torch.float16)
+    assert_close(y, ref, torch.float16, "strong decay")
+    rc, bits, exact = binding.device_status()
+    assert rc == 0 and bits == 0
+    if binding.path_for(1, 2, gh, gw, 64, 64, 64, torch.float16) == "tc":
+        assert exact > 0
+
+
+def test_zero_gate_long_memory():
+    gh, gw = 64, 64
+    d = inputs.make_custom(1, 2, gh, gw, 64, 64, "bf16", seed=71, qk_std=0.125)
+    d["g"] = torch.zeros_like(d["g"])
+    y, ref = _run_custom(d, gh, gw, "TB", 64, torch.bfloat16)
+    assert_close(y, ref, torch.bfloat16, "g = 0")
+
+
+@pytest.mark.parametrize("chunk", (16, 64, 128))
+@pytest.mark.parametrize("direction", ("LR", "BT"))
+def test_chunk_states_against_oracle(chunk, direction):
+    gh, gw = 20, 13
+    d = inputs.make_custom(2, 2, gh, gw, 64, 64, "f16", seed=81)
+    st = binding.chunk_states(_dev(d["k"]), _dev(d["v"]), _dev(d["g"]), grid_h=gh, grid_w=gw,
+                              direction=direction, chunk=chunk)
+    ref = oracle.chunk_states(d["k"], d["v"], d["g"], gh=gh, gw=gw, direction=direction, chunk=chunk)
+    got = st.double().cpu().numpy()
+    rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    assert rel < 1e-3, rel
+
+
+def test_output_stays_inside_its_buffer_and_inputs_untouched():
+    gh, gw = 11, 13
+    B, H, dk, dv = 2, 3, 64, 64
+    d = inputs.make_custom(B, H, gh, gw, dk, dv, "f16", seed=91)
+    n = B * gh * gw * H * dv
+    guard = 4096
+    for path in ("simt", "auto"):
+        binding.set_path(path)
+        try:
+            buf = torch.full((n + 2 * guard,), 7.0, dtype=torch.float16, device="cuda")
+            out = buf[guard:guard + n].view(B, gh * gw, H, dv)
+            dv_ = {k: _dev(v) for k, v in d.items()}
+            before = {k: v.clone() for k, v in dv_.items()}
+            binding.gla_fwd(dv_["q"], dv_["k"], dv_["v"], dv_["g"], dv_["z"], dv_["w"], grid_h=gh,
+                            grid_w=gw, direction="RL", chunk=32, out=out)
+            torch.cuda.synchronize()
+        finally:
+            binding.set_path("auto")
+        assert torch.all(buf[:guard] == 7.0) and torch.all(buf[guard + n:] == 7.0)
+        for k in before:
+            assert torch.equal(before[k], dv_[k]), k
+        ref = oracle.gla_fwd(d["q"], d["k"], d["v"], d["g"], d["z"], d["w"], gh=gh, gw=gw,
+                             direction="RL")
+        assert_close(out, ref, torch.float16, path)
+
+
+def test_empty_problem_and_argument_errors():
+    e = torch.empty(0, 40 * 40, 6, 64, dtype=torch.float16, device="cuda")
+    g = torch.empty(0, 40 * 40, 6, 64, dtype=torch.float32, device="cuda")
+    y = binding.gla_fwd(e, e, e, g, e, grid_h=40, grid_w=40)
+    assert y.shape == e.shape
+    # a tensor that starts 2 bytes past a 16-byte boundary
+    base = torch.zeros(1 + 1 * 16 * 2 * 64, dtype=torch.float16, device="cuda")
+    mis = base[1:].view(1, 16, 2, 64)
+    ok = torch.zeros(1, 16, 2, 64, dtype=torch.float16, device="cuda")
+    gg = torch.zeros(1, 16, 2, 64, dtype=torch.float32, device="cuda")
+    with pytest.raises(binding.GtrError) as ei:
+        binding.gla_fwd(mis, ok, ok, gg, ok, grid_h=4, grid_w=4)
+    assert ei.value.status == -3
+    _check_status()
