@@ -1,0 +1,509 @@
+"""Benchmark of the Key-only GLA hot path (gate projection + GLA forward).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 16k|640|640b8]
+    python bench.py --impl reference ...       # the fp64 CPU oracle, same workload
+
+One step = the whole hot path over one batch: gtr_gate_fwd (g from x) then
+gtr_gla_fwd (summary, boundary scan, output with the fused RMSNorm x SiLU
+epilogue), both through the C ABI.  Metric: token-heads per second,
+B*T*H per step, whole job (all ranks).
+
+Timing: inputs resident in HBM; four input sets rotate so that every step
+reads data that is not in L2 (the four sets together exceed the 126 MB L2).
+Each step is one CUDA graph replay (one graph per input set, captured once);
+K steps are timed with CUDA events on the launch stream, bracketed by a
+barrier and device synchronisation, max over ranks.  The graphs also hold
+CUDA events around every kernel, which give the per-kernel durations of the
+roofline entry.  nvidia-smi samples clocks during the timed region.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from linear_vision_backbone_b200 import inputs as gin  # noqa: E402
+
+N_SETS = 4
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.txt")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
+    ap.add_argument("--workload", default="16k", choices=("16k", "640", "640b8"))
+    ap.add_argument("--chunk", type=int, default=64)
+    ap.add_argument("--e2e-steps", type=int, default=40)
+    ap.add_argument("--no-secondary", action="store_true")
+    return ap.parse_args()
+
+
+def workload_text(wl: gin.Workload) -> str:
+    return (f"{wl.name}: B={wl.B}, {wl.gh}x{wl.gw} grid (T={wl.T}), H={wl.H}, dk=dv={wl.dk}, "
+            f"{wl.dtype}, scans {'/'.join(wl.dirs)}, gate rank {wl.rank} tau {wl.tau:g}, seed {wl.seed}")
+
+
+def step_dirs(wl):
+    return list(wl.dirs)
+
+
+def alg_bytes(wl, nseg, esz):
+    """Algorithmic bytes per launch of each kernel (unique reads + writes)."""
+    th = wl.token_heads
+    dk, dv = wl.dk, wl.dv
+    st = wl.B * wl.H * nseg * (dk * dv + dk) * 4
+    return {
+        "gate": wl.B * wl.T * wl.d_model * esz + th * dk * 4,
+        "summary": th * (dk * esz + dv * esz + dk * 4) + st,
+        "scan": 2 * st,
+        "output": th * (2 * dk * esz + 2 * dv * esz + dk * 4) + th * dv * esz + st,
+    }
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for ln in out.splitlines():
+            p = [x.strip() for x in ln.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                rows.append({"sm": float(p[1]), "max": float(p[2]), "power": float(p[3]),
+                             "hw": p[5], "hwt": p[6], "swt": p[7], "pcap": p[8]})
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        load = [r for r in rows if r["power"] > 200.0] or rows
+        reasons = set()
+        for r in load:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load),
+                "sm_max_mhz": max(r["max"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(load)}
+
+
+# ---------------------------------------------------------------- helpers
+def record_external(ev, stream):
+    """Record a torch event as an external event node when the stream is being
+    captured (a plain record inside capture is only a dependency, not a
+    timestamp), else as an ordinary record."""
+    from cuda.bindings import runtime as rt
+    err, status = rt.cudaStreamIsCapturing(stream.cuda_stream)
+    capturing = status == rt.cudaStreamCaptureStatus.cudaStreamCaptureStatusActive
+    if capturing:
+        (err,) = rt.cudaEventRecordWithFlags(ev.cuda_event, stream.cuda_stream,
+                                             rt.cudaEventRecordExternal)
+    else:
+        (err,) = rt.cudaEventRecord(ev.cuda_event, stream.cuda_stream)
+    assert err == rt.cudaError_t.cudaSuccess, err
+
+
+def event_ms(a, b) -> float:
+    """Elapsed ms between two recorded events, read through the CUDA runtime
+    (the events may have been recorded by the library or by graph replays)."""
+    from cuda.bindings import runtime as rt
+    err, ms = rt.cudaEventElapsedTime(a.cuda_event, b.cuda_event)
+    assert err == rt.cudaError_t.cudaSuccess, err
+    return float(ms)
+
+
+def read_peak():
+    try:
+        with open(PEAKS_FILE) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def read_traffic(kernel_name: str, src_hash: str):
+    """DRAM bytes per launch of a kernel from the committed ncu summary, if the
+    summary was taken on the current kernel source (matching hash)."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            for ln in f:
+                p = ln.split()
+                if len(p) >= 4 and p[0] == kernel_name and p[1] == src_hash:
+                    return float(p[2]), p[3]
+    except OSError:
+        pass
+    return None, None
+
+
+def kernel_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "linear_vision_backbone_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- CPU oracle
+def oracle_rate(wl, seconds=3.0, rows=32):
+    """Token-heads/s of the fp64 oracle (gate + GLA) on a bounded sample: every
+    head of the first `rows` grid rows of batch entry 0, repeated for about
+    `seconds`.  The oracle runs one (batch, head) sequence per OpenMP thread,
+    so it uses min(H, host cores) threads."""
+    import oracle
+    cores = os.cpu_count() or 1
+    used = min(oracle.set_threads(cores), wl.H)
+    d = gin.make_inputs(wl)
+    rows = max(1, min(wl.gh, rows))
+    T = rows * wl.gw
+    x = d["x"][:1, :T]
+    q, k, v, z = (d[n][:1, :T] for n in ("q", "k", "v", "z"))
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        g = oracle.gate(x, d["w_down"], d["w_up"], None, tau=wl.tau).reshape(1, T, wl.H, wl.dk)
+        oracle.gla_fwd(q, k, v, g, z, d["w"], gh=rows, gw=wl.gw, direction=wl.dirs[0])
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return {"value": n * T * wl.H / el, "unit": "token-heads/s", "cores": used, "kind": "oracle",
+            "sample": f"gate + GLA of all {wl.H} heads over the first {rows}x{wl.gw}={T} tokens of "
+                      f"the {wl.name} workload (batch entry 0), {n} repetitions in {el:.2f} s, fp64"}
+
+
+def run_reference(args, world, rank):
+    wl = gin.WORKLOADS[args.workload]
+    if rank != 0:
+        return
+    import oracle
+    oracle.set_threads(1)
+    d = gin.make_inputs(wl)
+    # bounded per-step sample: one head over 2 grid rows
+    rows = 2
+    T = rows * wl.gw
+    x = d["x"][:1, :T]
+    wu = d["w_up"][:, :wl.dk]
+    q, k, v, z = (d[n][:1, :T, 0:1] for n in ("q", "k", "v", "z"))
+
+    def step(i):
+        g = oracle.gate(x, d["w_down"], wu, None, tau=wl.tau).reshape(1, T, 1, wl.dk)
+        oracle.gla_fwd(q, k, v, g, z, d["w"], gh=rows, gw=wl.gw,
+                       direction=wl.dirs[i % len(wl.dirs)])
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    el = time.perf_counter() - t0
+    value = args.steps * T / el
+    sample = (f"per step: gate + GLA of 1 head over {rows}x{wl.gw}={T} tokens of the {wl.name} "
+              "workload (fp64 oracle, 1 thread)")
+    line = {
+        "impl": "reference", "metric": "GLA fwd token-heads/s (gate projection + Key-only GLA)",
+        "value": value, "unit": "token-heads/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_text(wl), "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "token-heads/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "token-heads/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU arm
+def run_ours(args, world, rank, local):
+    from linear_vision_backbone_b200 import binding, build
+    if not os.path.exists(binding.LIB_PATH):
+        build.build()
+    binding.load()
+    wl = gin.WORKLOADS[args.workload]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    host = gin.make_inputs(wl)
+    esz = host["q"].element_size()
+    dirs = step_dirs(wl)
+    # N_SETS device copies of the per-step tensors (activations + gate + output)
+    sets = []
+    for i in range(N_SETS):
+        s = {n: host[n].to(dev) for n in ("x", "q", "k", "v", "z")}
+        s["g"] = torch.empty(wl.B, wl.T, wl.H, wl.dk, device=dev, dtype=torch.float32)
+        s["out"] = torch.empty(wl.B, wl.T, wl.H, wl.dv, device=dev, dtype=host["q"].dtype)
+        sets.append(s)
+    params = {n: host[n].to(dev) for n in ("w_down", "w_up", "bias", "w")}
+    stream = torch.cuda.Stream(device=dev)
+    path = binding.path_for(wl.B, wl.H, wl.gh, wl.gw, wl.dk, wl.dv, args.chunk, host["q"].dtype)
+
+    def step(s, direction, evs=None):
+        if evs is not None:
+            record_external(evs[0], stream)
+        binding.gate_fwd(s["x"], params["w_down"], params["w_up"], params["bias"], wl.H, wl.dk,
+                         wl.tau, out=s["g"], stream=stream)
+        binding.gla_fwd(s["q"], s["k"], s["v"], s["g"], s["z"], params["w"], grid_h=wl.gh,
+                        grid_w=wl.gw, direction=direction, chunk=args.chunk, out=s["out"],
+                        stream=stream, events=None if evs is None else evs[1:])
+
+    # warm the library (workspace allocation happens outside capture)
+    with torch.cuda.stream(stream):
+        for i in range(N_SETS):
+            step(sets[i], dirs[i % len(dirs)])
+    stream.synchronize()
+
+    # one graph per input set, each holding kernel-boundary events
+    graphs, gevents = [], []
+    for i in range(N_SETS):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(sets[i], dirs[i % len(dirs)], evs)
+        graphs.append(g)
+        gevents.append(evs)
+    stream.synchronize()
+
+    for i in range(args.warmup):
+        with torch.cuda.stream(stream):
+            graphs[i % N_SETS].replay()
+    stream.synchronize()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_stop = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        t_start.record(stream)
+        for i in range(args.steps):
+            graphs[i % N_SETS].replay()
+        t_stop.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    ms = t_start.elapsed_time(t_stop)
+    ms_max = max_over_ranks(ms, world)
+
+    # per-kernel durations from the last replay of each graph
+    names = ("gate", "summary", "scan", "output")
+    per = {n: [] for n in names}
+    for evs in gevents:
+        for j, n in enumerate(names):
+            per[n].append(event_ms(evs[j], evs[j + 1]))
+    per_ms = {n: sum(v) / len(v) for n, v in per.items()}
+
+    # segment plan of this workload (for the state bytes)
+    nc = (wl.T + args.chunk - 1) // args.chunk
+    m = binding.segment_chunks(wl.B, wl.H, wl.gh, wl.gw, wl.dk, wl.dv, args.chunk, host["q"].dtype)
+    nseg = (nc + m - 1) // m
+    ab = alg_bytes(wl, nseg, esz)
+    dom = max(per_ms, key=lambda n: per_ms[n])
+    peak, peak_kind = read_peak()
+    achieved = ab[dom] / (per_ms[dom] * 1e-3) / 1e9
+    kname = {"gate": "gate_proj_kernel", "summary": "gla_summary", "scan": "gla_state_scan",
+             "output": "gla_output"}[dom]
+    traffic, _ = read_traffic(f"{kname}:{path}:{wl.name}", kernel_source_hash())
+
+    # e2e: host buffers, copies inside the timed region, through the public API
+    pinned = {n: host[n].pin_memory() for n in ("x", "q", "k", "v", "z")}
+    out_host = torch.empty(wl.B, wl.T, wl.H, wl.dv, dtype=host["q"].dtype).pin_memory()
+    s0 = sets[0]
+    h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+    d2h = out_host.numel() * out_host.element_size()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            for n in pinned:
+                s0[n].copy_(pinned[n], non_blocking=True)
+            step(s0, dirs[0])
+            out_host.copy_(s0["out"], non_blocking=True)
+    stream.synchronize()
+    barrier(world)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(args.e2e_steps):
+            for n in pinned:
+                s0[n].copy_(pinned[n], non_blocking=True)
+            step(s0, dirs[i % len(dirs)])
+            out_host.copy_(s0["out"], non_blocking=True)
+        e1.record(stream)
+    stream.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+
+    units = wl.token_heads
+    value = world * units * args.steps / (ms_max * 1e-3)
+    e2e_value = world * units * args.e2e_steps / (e2e_ms * 1e-3)
+
+    secondary = None
+    if not args.no_secondary and args.workload == "16k":
+        secondary = secondary_line(binding, dev)
+
+    if rank == 0:
+        cpu = oracle_rate(wl, seconds=2.0)
+        line = {
+            "metric": "GLA fwd token-heads/s (gate projection + Key-only GLA)",
+            "value": value, "unit": "token-heads/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32" if path == "simt" else "tf32/f32",
+            "data": "synthetic",
+            "config": {"workload": workload_text(wl), "chunk": args.chunk, "kernel_path": path,
+                       "l2": f"{N_SETS} rotating input sets, inputs larger than L2",
+                       "parallelism": f"replicas x{world} (independent (image, head) units)"},
+            "roofline": {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": peak,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": traffic, "alg_bytes": ab[dom],
+                         "kernel_ms": per_ms[dom]},
+            "kernels_ms": per_ms,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "token-heads/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": 4 * args.steps,
+            "clocks": clocks,
+        }
+        if secondary is not None:
+            line["secondary"] = secondary
+        print(json.dumps(line), flush=True)
+
+    for g in graphs:
+        del g
+    graphs.clear()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def secondary_line(binding, dev, steps=2000):
+    """The same step on the 640x640 workload (T = 1600), timed the same way."""
+    wl = gin.WORKLOADS["640"]
+    host = gin.make_inputs(wl)
+    sets = []
+    for i in range(8):
+        s = {n: host[n].to(dev) for n in ("x", "q", "k", "v", "z")}
+        s["g"] = torch.empty(wl.B, wl.T, wl.H, wl.dk, device=dev)
+        s["out"] = torch.empty_like(s["v"])
+        sets.append(s)
+    params = {n: host[n].to(dev) for n in ("w_down", "w_up", "bias", "w")}
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(s, direction):
+        binding.gate_fwd(s["x"], params["w_down"], params["w_up"], params["bias"], wl.H, wl.dk,
+                         wl.tau, out=s["g"], stream=stream)
+        binding.gla_fwd(s["q"], s["k"], s["v"], s["g"], s["z"], params["w"], grid_h=wl.gh,
+                        grid_w=wl.gw, direction=direction, chunk=64, out=s["out"], stream=stream)
+
+    with torch.cuda.stream(stream):
+        for i, s in enumerate(sets):
+            step(s, wl.dirs[i % 4])
+    stream.synchronize()
+    graphs = []
+    for i, s in enumerate(sets):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(s, wl.dirs[i % 4])
+        graphs.append(g)
+    # a 256 MB buffer written between replays keeps L2 cold for this small case
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for i in range(20):
+            graphs[i % 8].replay()
+        for i in range(steps):
+            flush.fill_(i & 255)
+            ev[i][0].record(stream)
+            graphs[i % 8].replay()
+            ev[i][1].record(stream)
+    stream.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in ev)
+    return {"workload": workload_text(wl), "value": wl.token_heads * steps / (ms * 1e-3),
+            "unit": "token-heads/s", "ms_per_step": ms / steps, "steps": steps,
+            "l2": "256 MiB buffer written between steps, outside the timed events"}
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args) if args.impl == "ours" else (
+        int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+        int(os.environ.get("LOCAL_RANK", "0")))
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -152,6 +152,12 @@ GTR_API gtr_status_t gtr_gla_chunk_states(const void *k, const void *v, const fl
 GTR_API size_t gtr_gla_workspace_bytes(int B, int H, int grid_h, int grid_w, int dk, int dv, int chunk,
                                int dtype);
 
+/* Chunks per segment of the plan gtr_gla_fwd would use for this problem on
+ * the current device (a segment is the run of consecutive chunks one block of
+ * the summary and output kernels walks through), or a negative status. */
+GTR_API int gtr_gla_segment_chunks(int B, int H, int grid_h, int grid_w, int dk, int dv, int chunk,
+                                   int dtype);
+
 /* Register a caller-owned device buffer as the workspace of the current device
  * (ptr 256-byte aligned).  NULL releases it: calls go back to the
  * library-owned buffers.  The caller keeps ownership and must keep the buffer

@@ -25,7 +25,7 @@ PATH_NAMES = {1: "simt", 2: "tc"}
 EXPORTS = (
     "gtr_abi_version", "gtr_status_string", "gtr_gate_fwd", "gtr_gla_fwd", "gtr_gla_fwd_timed",
     "gtr_gla_chunk_states", "gtr_gla_workspace_bytes", "gtr_gla_set_workspace",
-    "gtr_gla_set_path", "gtr_gla_path_for", "gtr_last_device_status",
+    "gtr_gla_set_path", "gtr_gla_path_for", "gtr_last_device_status", "gtr_gla_segment_chunks",
 )
 
 _lock = threading.Lock()
@@ -62,6 +62,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
             "gtr_gla_set_path": ([I], I),
             "gtr_gla_path_for": ([I, I, I, I, I, I, I, I], I),
             "gtr_last_device_status": ([P, P], I),
+            "gtr_gla_segment_chunks": ([I, I, I, I, I, I, I, I], I),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -189,6 +190,13 @@ def path_for(B, H, grid_h, grid_w, dk, dv, chunk, dtype) -> str:
 
 def workspace_bytes(B, H, grid_h, grid_w, dk, dv, chunk, dtype) -> int:
     return int(load().gtr_gla_workspace_bytes(B, H, grid_h, grid_w, dk, dv, chunk, DTYPE_IDS[dtype]))
+
+
+def segment_chunks(B, H, grid_h, grid_w, dk, dv, chunk, dtype) -> int:
+    rc = load().gtr_gla_segment_chunks(B, H, grid_h, grid_w, dk, dv, chunk, DTYPE_IDS[dtype])
+    if rc < 0:
+        _check("gtr_gla_segment_chunks", rc)
+    return rc
 
 
 def set_workspace(buf: Optional[torch.Tensor]) -> None:

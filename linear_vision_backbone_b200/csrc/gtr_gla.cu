@@ -51,6 +51,7 @@ int sm_count(int dev) {
 // consecutive chunks one block of K2/K4 walks through) and workspace layout.
 struct Plan {
   int B, H, gh, gw, T, dk, dv, dir, chunk, dtype;
+  int dev;
   int path;        // GTR_PATH_SIMT or GTR_PATH_TC
   int nc;          // chunks per sequence
   int seg_chunks;  // chunks per segment
@@ -102,7 +103,7 @@ int choose_path(int dk, int dv, int chunk, int dtype) {
 
 int make_plan(Plan* p, int dev, int B, int H, int gh, int gw, int dk, int dv, int dir, int chunk,
               int dtype, int force_seg_chunks) {
-  p->B = B; p->H = H; p->gh = gh; p->gw = gw; p->T = gh * gw;
+  p->B = B; p->H = H; p->gh = gh; p->gw = gw; p->T = gh * gw; p->dev = dev;
   p->dk = dk; p->dv = dv; p->dir = dir; p->chunk = chunk; p->dtype = dtype;
   const int path = choose_path(dk, dv, chunk, dtype);
   if (path < 0) return path;
@@ -151,23 +152,34 @@ int launch_status() {
   return cudaGetLastError() == cudaSuccess ? GTR_OK : GTR_ERR_CUDA;
 }
 
+// cudaFuncSetAttribute once per kernel instance and device.
+template <typename K>
+int ensure_smem(K kern, size_t smem, bool* done, int dev) {
+  if (done[dev]) return GTR_OK;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return GTR_ERR_CUDA;
+  done[dev] = true;
+  return GTR_OK;
+}
+
 template <typename T, int ROWS>
 int launch_simt_rows(const Plan& p, const void* q, const void* k, const void* v, const float* g,
                      const void* z, const float* w, void* out, float* wsS, float* wsL,
                      cudaStream_t st, int stage) {
   const dim3 grid(p.nseg, p.B * p.H);
   if (stage == 0) {
+    // at most kSimtBatch * 4 * 128 floats = 32 KB: no opt-in needed
     const size_t smem = (size_t)simt_summary_smem_floats(p.dk, p.dv) * sizeof(float);
     auto kern = gla_summary_simt<T, ROWS>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return GTR_ERR_CUDA;
     kern<<<grid, kSimtThreads, smem, st>>>((const T*)k, (const T*)v, g, wsS, wsL, p.H, p.T, p.gh,
                                            p.gw, p.dk, p.dv, p.dir, p.seg_len, p.nseg);
   } else {
     const size_t smem = (size_t)simt_output_smem_floats(p.dk, p.dv) * sizeof(float);
     auto kern = gla_output_simt<T, ROWS>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return GTR_ERR_CUDA;
+    // opt in once to the largest footprint any (dk, dv) of this instance can need
+    static bool done[kMaxDevices];
+    if (int rc = ensure_smem(kern, simt_output_smem_floats(128, 128) * sizeof(float), done, p.dev))
+      return rc;
     kern<<<grid, kSimtThreads, smem, st>>>((const T*)q, (const T*)k, (const T*)v, g, (const T*)z, w,
                                            wsS, (T*)out, p.H, p.T, p.gh, p.gw, p.dk, p.dv, p.dir,
                                            p.seg_len, p.nseg);
@@ -214,9 +226,16 @@ int launch_scan(const Plan& p, float* wsS, const float* wsL, int inclusive, cuda
   return launch_status();
 }
 
+// Record a caller event; inside stream capture it becomes an external event
+// node, so a replayed graph records real timestamps.
 int record(void* const* ev, int i, cudaStream_t st) {
-  if (ev && ev[i]) return cudaEventRecord((cudaEvent_t)ev[i], st) == cudaSuccess ? GTR_OK : GTR_ERR_CUDA;
-  return GTR_OK;
+  if (!ev || !ev[i]) return GTR_OK;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return GTR_ERR_CUDA;
+  const cudaError_t e = cs == cudaStreamCaptureStatusActive
+                            ? cudaEventRecordWithFlags((cudaEvent_t)ev[i], st, cudaEventRecordExternal)
+                            : cudaEventRecord((cudaEvent_t)ev[i], st);
+  return e == cudaSuccess ? GTR_OK : GTR_ERR_CUDA;
 }
 
 int gla_fwd_impl(const void* q, const void* k, const void* v, const float* g, const void* z,
@@ -348,6 +367,18 @@ size_t gtr_gla_workspace_bytes(int B, int H, int grid_h, int grid_w, int dk, int
   Plan p;
   if (make_plan(&p, dev, B, H, grid_h, grid_w, dk, dv, 0, chunk, dtype, 0)) return (size_t)-1;
   return p.ws_bytes;
+}
+
+int gtr_gla_segment_chunks(int B, int H, int grid_h, int grid_w, int dk, int dv, int chunk,
+                           int dtype) {
+  int rc = check_gla_args(B, H, grid_h, grid_w, dk, dv, 0, chunk, dtype);
+  if (rc) return rc;
+  if (B == 0 || H == 0 || grid_h == 0 || grid_w == 0) return 0;
+  int dev;
+  if ((rc = current_device(&dev))) return rc;
+  Plan p;
+  if ((rc = make_plan(&p, dev, B, H, grid_h, grid_w, dk, dv, 0, chunk, dtype, 0))) return rc;
+  return p.seg_chunks;
 }
 
 gtr_status_t gtr_gla_set_workspace(void* ptr, size_t bytes) {

@@ -1,17 +1,777 @@
-// tc_kernels.cuh -- tcgen05/TMEM path (placeholder until the tensor-core
-// kernels land; every shape reports unsupported so the SIMT path runs).
+// tc_kernels.cuh -- the tcgen05 / TMEM path of the Key-only GLA (sm_100a).
+//
+// Chunkwise evaluation (GTR article, 方法详解 §4 "硬件感知分块推理算子": chunk
+// summaries on tensor cores, a light sequential pass over boundary states,
+// chunk outputs with the scores kept on chip and the output gate fused into
+// the epilogue), for 16-bit q/k/v/z, fp32 gates, dk = dv = 64, chunk C = 64.
+//
+// One CTA (128 threads) walks a segment of consecutive chunks of one (batch,
+// head) sequence and carries the dk x dv state S in fp32 registers.  For chunk
+// c with in-chunk inclusive log-gate cumsum G_j (per key dim), G_m = G at the
+// middle position and Gam = G at the last one:
+//   q~_j = q_j e^{G_j - G_m},  k~_i = k_i e^{G_m - G_i},  k^_i = k_i e^{Gam - G_i}
+//   S'   = e^{G_m} S                                        (rows = key dims)
+//   o_j  = q~_j S' + sum_{i<=j} (q~_j . k~_i) v_i              -> RMSNorm x SiLU(z)
+//   S   <- e^{Gam} S + k^^T V
+// exp(G_j - G_i) = e^{G_j - G_m} e^{G_m - G_i} keeps both factors within
+// e^{+-span} of one, span = the chunk's own decay range.  A chunk whose span
+// exceeds kSpanMax nats, or whose gates rise above zero, evaluates its scores
+// exactly on CUDA cores instead (q~ = q e^{G_j}, S' = S,
+// P_ji = sum_d q_jd k_id e^{G_jd - G_id}).
+//
+// Data movement: every token's head vector is one contiguous 128-byte row (256
+// bytes for the fp32 gate), so the scan order is applied per token as the
+// source address of a 1-D bulk copy (cp.async.bulk, completion on an
+// mbarrier) into a double-buffered staging area; no transpose kernel runs and
+// reversed orders are just reversed addresses.  The next chunk's copies are in
+// flight while the current chunk computes.
+//
+// Tensor cores: tcgen05.mma kind::f16, M = 64, N = 64, K = 16 per
+// instruction, fp32 accumulators in tensor memory.  Every operand is a pair of
+// fp16 tiles (hi, lo) of a power-of-two-scaled fp32 value, multiplied as
+// hi*hi + hi*lo + lo*hi: products carry ~22 significant bits, the precision of
+// an fp32 evaluation for this operator's tolerance.
+//   cols [  0, 64)  q~ S'           A = q~ (K-major),  B = S' (MN-major)
+//   cols [ 64,128)  scores q~ k~^T  A = q~ (K-major),  B = k~ (K-major)
+//   cols [128,192)  P V             A = P  (K-major),  B = V  (MN-major)
+//   cols [192,256)  dS = k^^T V     A = k^ (MN-major), B = V  (MN-major)
+// An M = 64 accumulator puts row r in TMEM lane 32*(r/16) + r%16, so warp w
+// owns rows 16w..16w+15 in its lanes 0-15.  The masked scores P go back to
+// shared memory (K-major, two-term) for P V.  The epilogue reads whole rows,
+// so RMSNorm needs no cross-thread reduction.
 #pragma once
 #include "common.cuh"
 
 namespace gtr {
+namespace tc {
 
-inline bool tc_shape_supported(int, int, int, int) { return false; }
+constexpr int kC = 64;                 // chunk length
+constexpr int kD = 64;                 // head dim (dk = dv)
+constexpr int kThreads = 128;
+constexpr float kSpanMax = 20.0f;      // nats of in-chunk decay the scaled operands take
+constexpr unsigned long long kWaitNs = 500ull * 1000 * 1000;   // bounded waits: 0.5 s
+
+constexpr int kRaw16 = kC * kD * 2;    // one 16-bit staging tile: 8 KB
+constexpr int kRawG = kC * kD * 4;     // the fp32 gate tile: 16 KB
+constexpr int kTile = kC * kD * 2;     // one fp16 operand tile: 8 KB
+
+template <bool OUT> struct Layout {
+  static constexpr int kStage = OUT ? (4 * kRaw16 + kRawG) : (2 * kRaw16 + kRawG);
+  static constexpr int kOffK = 0, kOffV = kRaw16, kOffG = 2 * kRaw16;
+  static constexpr int kOffQ = 2 * kRaw16 + kRawG, kOffZ = 3 * kRaw16 + kRawG;
+  static constexpr int kOperands = 2 * kStage;
+  // tiles: V, k^ (hi, lo) [, q~ (hi, lo), k~ (hi, lo), S' (hi, lo)]
+  static constexpr int kTiles = OUT ? 9 : 3;
+  static constexpr int kMisc = kOperands + kTiles * kTile;
+  static constexpr int kMiscBytes = 6144;
+  static constexpr int kSmem = kMisc + kMiscBytes + 1024;      // + alignment slack
+  static constexpr int kTmemCols = OUT ? 256 : 64;
+  static constexpr int kColDS = OUT ? 192 : 0;
+  static constexpr uint32_t kTokenBytes = OUT ? (4 * kD * 2 + kD * 4) : (2 * kD * 2 + kD * 4);
+};
+
+// ------------------------------------------------------------------ PTX
+__device__ __forceinline__ uint32_t saddr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ unsigned long long globaltimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr(b)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(b)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ uint32_t mbar_try(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(saddr(b)), "r"(parity)
+      : "memory");
+  return ok;
+}
+// Wait for the phase with the given parity to complete; false after kWaitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity) {
+  if (mbar_try(b, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  while (!mbar_try(b, parity))
+    if (globaltimer() - t0 > kWaitNs) return false;
+  return true;
+}
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          saddr(dst)),
+      "l"(src), "r"(bytes), "r"(saddr(bar))
+      : "memory");
+}
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_before_sync() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_after_sync() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t cols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(saddr(dst)),
+               "r"(cols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols)
+               : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(saddr(bar))
+      : "memory");
+}
+// 32 lanes x 32 bit, 16 consecutive columns: thread t of warp w <- lane 32w+t.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ------------------------------------------------------- operand layouts
+// 16-bit operand tiles of 64 rows x 64 elements (128 bytes per row), layout
+// SWIZZLE_128B: atoms of 8 rows x 128 bytes, the 16-byte unit index XOR-ed
+// with the row's position in its atom.  The same physical layout serves a
+// K-major operand (rows = M or N, columns = K) and an MN-major one (rows = K,
+// columns = M or N); only the descriptor differs.
+__device__ __forceinline__ uint32_t sw16(int r, int c) {
+  return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + (((c >> 3) ^ (r & 7)) << 4) + (c & 7) * 2);
+}
+// tcgen05 shared-memory matrix descriptor (version 1): start address, leading
+// and stride byte offsets, layout type 2 = SWIZZLE_128B.
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+// K-major tile, K step s: 16 elements = 32 bytes into every row.
+__device__ __forceinline__ uint64_t kdesc(uint32_t base, int s) {
+  return sdesc(base + (uint32_t)(s * 32), 16, 1024);
+}
+// MN-major tile, K step s: 16 rows = two 8-row atoms 1024 bytes apart.
+__device__ __forceinline__ uint64_t mndesc(uint32_t base, int s) {
+  return sdesc(base + (uint32_t)(s * 2048), 8192, 1024);
+}
+// Instruction descriptor: kind::f16 with fp16 A and B, fp32 accumulate.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int a_mn, int b_mn) {
+  return (1u << 4) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+__device__ __forceinline__ void mma_f16(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                        uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// One 64x64x64 product: four K steps, accumulating onto the target unless it
+// starts the accumulator.
+__device__ __forceinline__ void mma_64(uint32_t d, uint32_t a, bool a_mn, uint32_t b, bool b_mn,
+                                       bool accumulate) {
+  const uint32_t id = idesc_f16(64, 64, a_mn, b_mn);
+#pragma unroll
+  for (int s = 0; s < 4; ++s)
+    mma_f16(d, a_mn ? mndesc(a, s) : kdesc(a, s), b_mn ? mndesc(b, s) : kdesc(b, s), id,
+            (accumulate || s > 0) ? 1u : 0u);
+}
+// (ah + al)(bh + bl) ~ ah bh + ah bl + al bh into d (fresh unless accumulate)
+__device__ __forceinline__ void mma_pair(uint32_t d, uint32_t ah, uint32_t al, bool a_mn,
+                                         uint32_t bh, uint32_t bl, bool b_mn, bool accumulate) {
+  mma_64(d, ah, a_mn, bh, b_mn, accumulate);
+  mma_64(d, ah, a_mn, bl, b_mn, true);
+  mma_64(d, al, a_mn, bh, b_mn, true);
+}
+
+// ------------------------------------------------- two-term fp16 operands
+// Every tensor-core operand is a pair (hi, lo) of fp16 tiles with
+// x * 2^e = hi + lo, hi = fp16(x 2^e), lo = fp16(x 2^e - hi): 22 significant
+// bits.  The power-of-two scale 2^e puts the largest magnitude of a row (or
+// column, or tile) in [2^14, 2^15), inside fp16's range; it is exact and is
+// undone on the fp32 accumulator.  Scales run along M or N, never along K, so
+// they factor out of every sum.
+__device__ __forceinline__ int scale_exp(float m) {
+  if (!(m > 0.f) || !(m <= 3.0e38f)) return 0;
+  const int ex = ((__float_as_int(m) >> 23) & 0xFF) - 127;
+  return max(-60, min(60, 14 - ex));
+}
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }
+__device__ __forceinline__ uint2 split4(float a, float b, float c, float d, uint2* lo) {
+  const __half2 h0 = __floats2half2_rn(a, b), h1 = __floats2half2_rn(c, d);
+  const float2 f0 = __half22float2(h0), f1 = __half22float2(h1);
+  const __half2 l0 = __floats2half2_rn(a - f0.x, b - f0.y), l1 = __floats2half2_rn(c - f1.x, d - f1.y);
+  uint2 hi;
+  memcpy(&hi.x, &h0, 4);
+  memcpy(&hi.y, &h1, 4);
+  memcpy(&lo->x, &l0, 4);
+  memcpy(&lo->y, &l1, 4);
+  return hi;
+}
+__device__ __forceinline__ uint2 half4(float a, float b, float c, float d) {
+  const __half2 h0 = __floats2half2_rn(a, b), h1 = __floats2half2_rn(c, d);
+  uint2 u;
+  memcpy(&u.x, &h0, 4);
+  memcpy(&u.y, &h1, 4);
+  return u;
+}
+// store one two-term group of 4 elements at byte offset `off` of (hi, lo) tiles
+__device__ __forceinline__ void put2(uint8_t* hi, uint8_t* lo, uint32_t off, float a, float b, float c,
+                                     float d) {
+  uint2 l;
+  const uint2 h = split4(a, b, c, d, &l);
+  *reinterpret_cast<uint2*>(hi + off) = h;
+  *reinterpret_cast<uint2*>(lo + off) = l;
+}
+// max over the 16 lanes of a half warp (one operand row in the builders)
+__device__ __forceinline__ float half_warp_max(float v) {
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float amax4(float a, float b, float c, float d) {
+  return fmaxf(fmaxf(fabsf(a), fabsf(b)), fmaxf(fabsf(c), fabsf(d)));
+}
+
+template <typename T> struct Vec4;
+template <> struct Vec4<__half> {
+  static __device__ __forceinline__ float4 from_bits(uint2 u) {
+    __half2 a, b;
+    memcpy(&a, &u.x, 4);
+    memcpy(&b, &u.y, 4);
+    const float2 fa = __half22float2(a), fb = __half22float2(b);
+    return make_float4(fa.x, fa.y, fb.x, fb.y);
+  }
+  static __device__ __forceinline__ float4 load(const void* p) {
+    return from_bits(*reinterpret_cast<const uint2*>(p));
+  }
+};
+template <> struct Vec4<__nv_bfloat16> {
+  static __device__ __forceinline__ float4 from_bits(uint2 u) {
+    __nv_bfloat162 a, b;
+    memcpy(&a, &u.x, 4);
+    memcpy(&b, &u.y, 4);
+    const float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    return make_float4(fa.x, fa.y, fb.x, fb.y);
+  }
+  static __device__ __forceinline__ float4 load(const void* p) {
+    return from_bits(*reinterpret_cast<const uint2*>(p));
+  }
+};
+template <typename T> __device__ __forceinline__ uint2 pack4(float a, float b, float c, float d);
+template <> __device__ __forceinline__ uint2 pack4<__half>(float a, float b, float c, float d) {
+  return half4(a, b, c, d);
+}
+template <> __device__ __forceinline__ uint2 pack4<__nv_bfloat16>(float a, float b, float c, float d) {
+  const __nv_bfloat162 x = __floats2bfloat162_rn(a, b), y = __floats2bfloat162_rn(c, d);
+  uint2 u;
+  memcpy(&u.x, &x, 4);
+  memcpy(&u.y, &y, 4);
+  return u;
+}
+
+struct Params {
+  const void* q; const void* k; const void* v; const float* g; const void* z; const float* w;
+  float* wsS; float* wsL; void* out;
+  int H, T, gh, gw, dir, seg_chunks, nseg;
+};
+
+struct Misc {                   // per-CTA scalars in shared memory
+  uint64_t full[2];             // staging stage filled
+  uint64_t mma;                 // MMA group committed
+  uint32_t tmem;                // tensor-memory base address
+  int abort;
+  float smax[4];                // per-warp max |S| of the carried state
+  float Gm[kD], Gam[kD], aG[kD], eK[kD], wv[kD];
+  float lo[2][kD], hi[2][kD], half0[kD], kmx[2][kD], vmx[2][kD];
+  float sev[kD], iev[kD];       // V column scales 2^e and 2^-e
+  float skh[kD], ikh[kD];       // k^ row (key dim) scales
+  float ieq[kC], iek[kC], iep[kC];   // inverse row scales of q~, k~, P
+};
+static_assert(sizeof(Misc) <= 6144, "Misc must fit its reserved bytes");
+
+// Issue the bulk copies of one chunk (warp 0): every token row of k, v, g (and
+// q, z for the output kernel), in scan order, into the staging stage.
+template <typename T, bool OUT>
+__device__ __forceinline__ void issue_chunk(const Params& p, uint8_t* stage, uint64_t* bar, int b,
+                                            int h, int d, int s0, int ntok, int lane) {
+  using L = Layout<OUT>;
+  if (lane == 0) mbar_expect_tx(bar, (uint32_t)ntok * L::kTokenBytes);
+  __syncwarp();
+  for (int j = lane; j < ntok; j += 32) {
+    const int t = scan_to_grid(d, s0 + j, p.T, p.gh, p.gw);
+    const size_t row = ((size_t)b * p.T + t) * p.H + h;
+    bulk_g2s(stage + L::kOffK + j * kD * 2, (const T*)p.k + row * kD, kD * 2, bar);
+    bulk_g2s(stage + L::kOffV + j * kD * 2, (const T*)p.v + row * kD, kD * 2, bar);
+    bulk_g2s(stage + L::kOffG + j * kD * 4, p.g + row * kD, kD * 4, bar);
+    if (OUT) {
+      bulk_g2s(stage + L::kOffQ + j * kD * 2, (const T*)p.q + row * kD, kD * 2, bar);
+      bulk_g2s(stage + L::kOffZ + j * kD * 2, (const T*)p.z + row * kD, kD * 2, bar);
+    }
+  }
+}
+
+// Column pass over the chunk (two threads per column, 32 tokens each): the
+// in-place inclusive cumsum of the gate tile, and the column maxima of |k| and
+// |v|.  Then per column d: G_m, Gam, e^{Gam}, e^{Gam-G_m}, the k^ and V
+// scales.  Returns true (block-uniform) if the chunk needs the exact scores:
+// its decay range exceeds kSpanMax or some gate sum rises above zero.
+template <typename T>
+__device__ __forceinline__ bool column_pass(float* G, const T* kst, const T* vst, Misc& m, int ntok,
+                                            int tid) {
+  const int dd = tid & 63, half = tid >> 6;
+  const int j0 = half * 32, j1 = min(j0 + 32, ntok);
+  float run = 0.f, lo = 3.0e38f, hi = -3.0e38f, km = 0.f, vm = 0.f;
+  for (int j = j0; j < j1; ++j) {
+    run += G[j * kD + dd];
+    G[j * kD + dd] = run;
+    lo = fminf(lo, run);
+    hi = fmaxf(hi, run);
+    km = fmaxf(km, fabsf(Elem<T>::to_f(kst[j * kD + dd])));
+    vm = fmaxf(vm, fabsf(Elem<T>::to_f(vst[j * kD + dd])));
+  }
+  if (half == 0) m.half0[dd] = run;
+  m.kmx[half][dd] = km;
+  m.vmx[half][dd] = vm;
+  __syncthreads();
+  if (half == 1 && j1 > j0) {
+    const float off = m.half0[dd];
+    for (int j = j0; j < j1; ++j) G[j * kD + dd] += off;
+    lo += off;
+    hi += off;
+  }
+  m.lo[half][dd] = lo;
+  m.hi[half][dd] = hi;
+  __syncthreads();
+  int irregular = 0;
+  if (tid < kD) {
+    const float gam = G[(ntok - 1) * kD + tid];
+    const float gm = G[((ntok - 1) >> 1) * kD + tid];
+    const float mn = fminf(m.lo[0][tid], m.lo[1][tid]), mx = fmaxf(m.hi[0][tid], m.hi[1][tid]);
+    m.Gam[tid] = gam;
+    m.Gm[tid] = gm;
+    m.aG[tid] = expf(gam);
+    m.eK[tid] = expf(gam - gm);
+    // k^_id = k_id e^{Gam_d - G_id} <= max_i |k_id| e^{Gam_d - min_i G_id}
+    const int ek = scale_exp(fmaxf(m.kmx[0][tid], m.kmx[1][tid]) * expf(gam - fminf(mn, 0.f)));
+    m.skh[tid] = pow2i(ek);
+    m.ikh[tid] = pow2i(-ek);
+    const int ev = scale_exp(fmaxf(m.vmx[0][tid], m.vmx[1][tid]));
+    m.sev[tid] = pow2i(ev);
+    m.iev[tid] = pow2i(-ev);
+    const float span = fmaxf(mx, 0.f) - fminf(mn, 0.f);
+    irregular = !(span <= kSpanMax) || mx > 0.f;
+  }
+  return __syncthreads_or(irregular) != 0;
+}
+
+// Max |S| over the block's state rows into m.smax (one value per warp).
+__device__ __forceinline__ void state_max(const float* S, bool owner, Misc& m, int warp, int lane) {
+  float mx = 0.f;
+  if (owner) {
+#pragma unroll
+    for (int c = 0; c < kD; ++c) mx = fmaxf(mx, fabsf(S[c]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if (lane == 0) m.smax[warp] = mx;
+}
+
+template <typename T, bool OUT>
+__global__ void __launch_bounds__(kThreads, 1)
+gla_tc(const Params p) {
+  using L = Layout<OUT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* stages = sm;
+  uint8_t* tiles = sm + L::kOperands;
+  uint8_t* VV = tiles;                       // V            (MN-major B), single fp16 tile
+  uint8_t* KHh = tiles + 1 * kTile;          // k^ hi / lo   (MN-major A)
+  uint8_t* KHl = tiles + 2 * kTile;
+  uint8_t* QTh = tiles + 3 * kTile;          // q~ hi / lo, then P (K-major A)   [OUT]
+  uint8_t* QTl = tiles + 4 * kTile;
+  uint8_t* KTh = tiles + 5 * kTile;          // k~ hi / lo   (K-major B)         [OUT]
+  uint8_t* KTl = tiles + 6 * kTile;
+  uint8_t* SPh = tiles + 7 * kTile;          // S' hi / lo   (MN-major B)        [OUT]
+  uint8_t* SPl = tiles + 8 * kTile;
+  Misc& m = *reinterpret_cast<Misc*>(sm + L::kMisc);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int seg = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / p.H, h = bh - b * p.H;
+  const int d = dir_of_batch(p.dir, b);
+  const int nc = (p.T + kC - 1) / kC;
+  const int c0 = seg * p.seg_chunks;
+  const int nch = min(nc, c0 + p.seg_chunks) - c0;
+  if (d < 0 || d > 3 || nch <= 0) {
+    if (tid == 0) gtr_flag(d < 0 || d > 3 ? kStatusBadDir : kStatusBadShape);
+    return;
+  }
+  const bool owner = lane < 16;          // this thread holds accumulator row 16*warp + lane
+  const int row = warp * 16 + lane;      // that row: a query token, or a key dim of S
+
+  // carried state: row `row` of S (key dim), 64 value columns
+  float S[kD];
+  if (OUT && owner) {
+    const float4* src = reinterpret_cast<const float4*>(
+        p.wsS + (((size_t)bh * p.nseg + seg) * kD + row) * kD);
+#pragma unroll
+    for (int c = 0; c < kD / 4; ++c) {
+      const float4 x = src[c];
+      S[4 * c] = x.x; S[4 * c + 1] = x.y; S[4 * c + 2] = x.z; S[4 * c + 3] = x.w;
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < kD; ++c) S[c] = 0.f;
+  }
+  if (OUT) state_max(S, owner, m, warp, lane);
+  if (tid == 0) {
+    mbar_init(&m.full[0], 1);
+    mbar_init(&m.full[1], 1);
+    mbar_init(&m.mma, 1);
+    mbar_fence_init();
+    m.abort = 0;
+  }
+  if (tid < kD) m.wv[tid] = (OUT && p.w) ? p.w[tid] : 1.0f;
+  if (warp == 0) {
+    tmem_alloc(&m.tmem, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_before_sync();
+  __syncthreads();
+  tc_after_sync();
+  const uint32_t tm = m.tmem;
+  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+
+  float lsum = 0.f;
+  uint32_t mma_phase = 0;
+  uint32_t outstanding = 1;               // bit s: stage s has copies in flight
+
+  if (warp == 0) {
+    const int s0 = c0 * kC;
+    issue_chunk<T, OUT>(p, stages, &m.full[0], b, h, d, s0, min(kC, p.T - s0), lane);
+  }
+
+  for (int it = 0; it < nch; ++it) {
+    const int st = it & 1;
+    uint8_t* stg = stages + st * L::kStage;
+    const int s0 = (c0 + it) * kC;
+    const int ntok = min(kC, p.T - s0);
+    if (it + 1 < nch) {
+      if (warp == 0) {
+        const int s1 = s0 + kC;
+        issue_chunk<T, OUT>(p, stages + (st ^ 1) * L::kStage, &m.full[st ^ 1], b, h, d, s1,
+                            min(kC, p.T - s1), lane);
+      }
+      outstanding |= 1u << (st ^ 1);
+    }
+    const bool ok = mbar_wait(&m.full[st], (it >> 1) & 1);
+    outstanding &= ~(1u << st);
+    if (__syncthreads_or(!ok)) {
+      if (tid == 0) gtr_flag(kStatusMbarTimeout);
+      m.abort = 1;
+      break;
+    }
+
+    float* G = reinterpret_cast<float*>(stg + L::kOffG);
+    const T* kst = reinterpret_cast<const T*>(stg + L::kOffK);
+    const T* vst = reinterpret_cast<const T*>(stg + L::kOffV);
+    const T* qst = reinterpret_cast<const T*>(stg + L::kOffQ);
+    const bool exact = column_pass<T>(G, kst, vst, m, ntok, tid) && OUT;
+
+    // ---- operand tiles; rows beyond ntok are zero.  Items: (row r, 4 columns
+    // cg..cg+3); a half warp covers one row, which makes per-row maxima cheap.
+#pragma unroll 2
+    for (int u = 0; u < 8; ++u) {
+      const int item = u * kThreads + tid;
+      const int r = item >> 4, cg = (item & 15) * 4;
+      const bool valid = r < ntok;
+      float4 kk = make_float4(0.f, 0.f, 0.f, 0.f), vv = kk, qq = kk;
+      if (valid) {
+        kk = Vec4<T>::load(kst + r * kD + cg);
+        vv = Vec4<T>::load(vst + r * kD + cg);
+        if (OUT) qq = Vec4<T>::load(qst + r * kD + cg);
+      }
+      const float4 gg = *reinterpret_cast<const float4*>(G + r * kD + cg);
+      const float4 ga = *reinterpret_cast<const float4*>(&m.Gam[cg]);
+      const uint32_t off = sw16(r, cg);
+      {   // V (column-scaled, one fp16 term: exact for 16-bit inputs)
+        const float4 sv = *reinterpret_cast<const float4*>(&m.sev[cg]);
+        *reinterpret_cast<uint2*>(VV + off) = half4(vv.x * sv.x, vv.y * sv.y, vv.z * sv.z, vv.w * sv.w);
+      }
+      {   // k^ = k e^{Gam - G} (key-dim scaled; rows = tokens = K of dS)
+        const float4 sk = *reinterpret_cast<const float4*>(&m.skh[cg]);
+        put2(KHh, KHl, off, kk.x * __expf(ga.x - gg.x) * sk.x, kk.y * __expf(ga.y - gg.y) * sk.y,
+             kk.z * __expf(ga.z - gg.z) * sk.z, kk.w * __expf(ga.w - gg.w) * sk.w);
+      }
+      if (OUT) {
+        const float4 gm = *reinterpret_cast<const float4*>(&m.Gm[cg]);
+        float q0, q1, q2, q3;
+        if (!exact) {
+          // k~ = k e^{G_m - G}, row (key token) scaled
+          const float a0 = kk.x * __expf(gm.x - gg.x), a1 = kk.y * __expf(gm.y - gg.y);
+          const float a2 = kk.z * __expf(gm.z - gg.z), a3 = kk.w * __expf(gm.w - gg.w);
+          const int ek = scale_exp(half_warp_max(amax4(a0, a1, a2, a3)));
+          const float s = pow2i(ek);
+          put2(KTh, KTl, off, a0 * s, a1 * s, a2 * s, a3 * s);
+          if (cg == 0) m.iek[r] = pow2i(-ek);
+          q0 = qq.x * __expf(gg.x - gm.x); q1 = qq.y * __expf(gg.y - gm.y);
+          q2 = qq.z * __expf(gg.z - gm.z); q3 = qq.w * __expf(gg.w - gm.w);
+        } else {   // exact chunk: q~ = q e^{G_j}
+          q0 = qq.x * __expf(gg.x); q1 = qq.y * __expf(gg.y);
+          q2 = qq.z * __expf(gg.z); q3 = qq.w * __expf(gg.w);
+        }
+        const int eq = scale_exp(half_warp_max(amax4(q0, q1, q2, q3)));
+        const float s = pow2i(eq);
+        put2(QTh, QTl, off, q0 * s, q1 * s, q2 * s, q3 * s);
+        if (cg == 0) m.ieq[r] = pow2i(-eq);
+      }
+    }
+    // S' = e^{G_m} S (S itself for an exact chunk), tile-scaled from max |S|
+    float inv_es = 1.f;
+    if (OUT) {
+      const float smx = fmaxf(fmaxf(m.smax[0], m.smax[1]), fmaxf(m.smax[2], m.smax[3]));
+      const int es = scale_exp(smx);
+      inv_es = pow2i(-es);
+      if (owner) {
+        const float sc = (exact ? 1.0f : __expf(m.Gm[row])) * pow2i(es);
+#pragma unroll
+        for (int c = 0; c < kD; c += 4)
+          put2(SPh, SPl, sw16(row, c), sc * S[c], sc * S[c + 1], sc * S[c + 2], sc * S[c + 3]);
+      }
+    }
+    fence_async_smem();
+    tc_before_sync();
+    __syncthreads();
+    tc_after_sync();
+
+    if (tid == 0) {
+      if (OUT) {
+        mma_pair(tm + 0, saddr(QTh), saddr(QTl), false, saddr(SPh), saddr(SPl), true, false);
+        if (!exact)
+          mma_pair(tm + 64, saddr(QTh), saddr(QTl), false, saddr(KTh), saddr(KTl), false, false);
+      }
+      mma_64(tm + L::kColDS, saddr(KHh), true, saddr(VV), true, false);
+      mma_64(tm + L::kColDS, saddr(KHl), true, saddr(VV), true, true);
+      mma_commit(&m.mma);
+    }
+    bool okm = mbar_wait(&m.mma, mma_phase);
+    mma_phase ^= 1;
+    if (__syncthreads_or(!okm)) {
+      if (tid == 0) gtr_flag(kStatusMbarTimeout);
+      m.abort = 1;
+      break;
+    }
+    tc_after_sync();
+
+    if (OUT) {
+      // ---- masked scores P (rows = queries j, columns = keys i), row-scaled, into QT
+      if (!exact) {
+        float sc[kC];
+#pragma unroll
+        for (int cb = 0; cb < 4; ++cb) tmem_ld16(tm + lane_base + 64 + cb * 16, sc + cb * 16);
+        tmem_ld_wait();
+        if (owner) {
+          const float iq = m.ieq[row];
+          float mx = 0.f;
+#pragma unroll
+          for (int i = 0; i < kC; ++i) {
+            sc[i] = (i <= row && row < ntok) ? sc[i] * iq * m.iek[i] : 0.f;
+            mx = fmaxf(mx, fabsf(sc[i]));
+          }
+          const int ep = scale_exp(mx);
+          const float s = pow2i(ep);
+          m.iep[row] = pow2i(-ep);
+#pragma unroll
+          for (int i = 0; i < kC; i += 4)
+            put2(QTh, QTl, sw16(row, i), sc[i] * s, sc[i + 1] * s, sc[i + 2] * s, sc[i + 3] * s);
+        }
+      } else {
+        // exact scores on CUDA cores: P_ji = sum_d q_jd k_id e^{G_jd - G_id}; two threads per row
+        if (tid == 0) atomicAdd(&g_gtr_exact_chunks, 1ull);
+        const int j = tid >> 1, ib = (tid & 1) * 32;
+        float acc[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) acc[e] = 0.f;
+        if (j < ntok) {
+          for (int dd = 0; dd < kD; ++dd) {
+            const float qj = Elem<T>::to_f(qst[j * kD + dd]);
+            const float gj = G[j * kD + dd];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int i = ib + e;
+              if (i <= j)
+                acc[e] = fmaf(qj * Elem<T>::to_f(kst[i * kD + dd]), expf(gj - G[i * kD + dd]), acc[e]);
+            }
+          }
+        }
+        float mx = 0.f;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, fabsf(acc[e]));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        const int ep = scale_exp(mx);
+        const float s = pow2i(ep);
+        if ((tid & 1) == 0) m.iep[j] = pow2i(-ep);
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          put2(QTh, QTl, sw16(j, ib + e), acc[e] * s, acc[e + 1] * s, acc[e + 2] * s, acc[e + 3] * s);
+      }
+      fence_async_smem();
+      tc_before_sync();
+      __syncthreads();
+      tc_after_sync();
+      if (tid == 0) {
+        mma_64(tm + 128, saddr(QTh), false, saddr(VV), true, false);
+        mma_64(tm + 128, saddr(QTl), false, saddr(VV), true, true);
+        mma_commit(&m.mma);
+      }
+      okm = mbar_wait(&m.mma, mma_phase);
+      mma_phase ^= 1;
+      if (__syncthreads_or(!okm)) {
+        if (tid == 0) gtr_flag(kStatusMbarTimeout);
+        m.abort = 1;
+        break;
+      }
+      tc_after_sync();
+
+      // ---- epilogue: o_j = q~_j S' + P_j V, then o_j / sqrt(mean o_j^2 + eps) * w * SiLU(z_j)
+      float o[kD], pv[kD];
+#pragma unroll
+      for (int cb = 0; cb < 4; ++cb) {
+        tmem_ld16(tm + lane_base + cb * 16, o + cb * 16);
+        tmem_ld16(tm + lane_base + 128 + cb * 16, pv + cb * 16);
+      }
+      tmem_ld_wait();
+      if (owner && row < ntok) {
+        const float a = m.ieq[row] * inv_es, bsc = m.iep[row];
+        float ss = 0.f;
+#pragma unroll
+        for (int c = 0; c < kD; ++c) {
+          o[c] = o[c] * a + pv[c] * bsc * m.iev[c];
+          ss = fmaf(o[c], o[c], ss);
+        }
+        const float inv = 1.0f / sqrtf(ss * (1.0f / kD) + kRmsEps);
+        const T* zr = reinterpret_cast<const T*>(stg + L::kOffZ) + row * kD;
+        const int t = scan_to_grid(d, s0 + row, p.T, p.gh, p.gw);
+        T* dst = reinterpret_cast<T*>(p.out) + (((size_t)b * p.T + t) * p.H + h) * kD;
+#pragma unroll
+        for (int c = 0; c < kD; c += 8) {
+          const uint4 zz = *reinterpret_cast<const uint4*>(zr + c);
+          const float4 z0 = Vec4<T>::from_bits(make_uint2(zz.x, zz.y));
+          const float4 z1 = Vec4<T>::from_bits(make_uint2(zz.z, zz.w));
+          const float4 w0 = *reinterpret_cast<const float4*>(&m.wv[c]);
+          const float4 w1 = *reinterpret_cast<const float4*>(&m.wv[c + 4]);
+          const uint2 lo = pack4<T>(o[c + 0] * inv * w0.x * silu_f(z0.x), o[c + 1] * inv * w0.y * silu_f(z0.y),
+                                    o[c + 2] * inv * w0.z * silu_f(z0.z), o[c + 3] * inv * w0.w * silu_f(z0.w));
+          const uint2 hi = pack4<T>(o[c + 4] * inv * w1.x * silu_f(z1.x), o[c + 5] * inv * w1.y * silu_f(z1.y),
+                                    o[c + 6] * inv * w1.z * silu_f(z1.z), o[c + 7] * inv * w1.w * silu_f(z1.w));
+          *reinterpret_cast<uint4*>(dst + c) = make_uint4(lo.x, lo.y, hi.x, hi.y);
+        }
+      }
+    }
+
+    // ---- state: S <- e^{Gam} S + dS (fp32 accumulation)
+    {
+      float ds[kD];
+#pragma unroll
+      for (int cb = 0; cb < 4; ++cb) tmem_ld16(tm + lane_base + L::kColDS + cb * 16, ds + cb * 16);
+      tmem_ld_wait();
+      if (owner) {
+        const float a = m.aG[row], ik = m.ikh[row];
+#pragma unroll
+        for (int c = 0; c < kD; ++c) S[c] = fmaf(a, S[c], ds[c] * ik * m.iev[c]);
+      }
+      if (OUT) state_max(S, owner, m, warp, lane);
+    }
+    if (!OUT && tid < kD) lsum += m.Gam[tid];
+    tc_before_sync();
+    __syncthreads();
+  }
+
+  if (m.abort) {
+    // let copies still in flight land before the block's shared memory is released
+    for (int s = 0; s < 2; ++s)
+      if (outstanding & (1u << s)) (void)mbar_wait(&m.full[s], 0);
+  } else if (!OUT) {
+    if (owner) {
+      float4* dst = reinterpret_cast<float4*>(p.wsS + (((size_t)bh * p.nseg + seg) * kD + row) * kD);
+#pragma unroll
+      for (int c = 0; c < kD / 4; ++c)
+        dst[c] = make_float4(S[4 * c], S[4 * c + 1], S[4 * c + 2], S[4 * c + 3]);
+    }
+    if (tid < kD) p.wsL[((size_t)bh * p.nseg + seg) * kD + tid] = lsum;
+  }
+  tc_before_sync();
+  __syncthreads();
+  tc_after_sync();
+  if (warp == 0) tmem_dealloc(tm, L::kTmemCols);
+}
+
+}  // namespace tc
+
+inline bool tc_shape_supported(int dk, int dv, int chunk, int dtype) {
+  return dk == tc::kD && dv == tc::kD && chunk == tc::kC && (dtype == kF16 || dtype == kBF16);
+}
 inline int tc_blocks_per_sm(int, int) { return 1; }
 
-inline int launch_tc(int, int, const void*, const void*, const void*, const float*, const void*,
-                     const float*, void*, float*, float*, int, int, int, int, int, int, int, int,
-                     int, int, int, cudaStream_t) {
-  return -2;
+template <typename T, bool OUT>
+inline int launch_tc_kernel(const tc::Params& p, int BH, cudaStream_t st, int dev) {
+  auto kern = tc::gla_tc<T, OUT>;
+  static bool done[64];
+  if (!done[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             tc::Layout<OUT>::kSmem) != cudaSuccess)
+      return -5;
+    done[dev] = true;
+  }
+  kern<<<dim3(p.nseg, BH), tc::kThreads, tc::Layout<OUT>::kSmem, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? 0 : -5;
+}
+
+// stage 0: segment summaries (K2); stage 1: segment outputs (K4)
+inline int launch_tc(int dtype, int stage, const void* q, const void* k, const void* v,
+                     const float* g, const void* z, const float* w, void* out, float* wsS,
+                     float* wsL, int B, int H, int T, int gh, int gw, int dk, int dv, int dir,
+                     int chunk, int seg_chunks, int nseg, cudaStream_t st) {
+  if (!tc_shape_supported(dk, dv, chunk, dtype)) return -2;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -5;
+  tc::Params p{q, k, v, g, z, w, wsS, wsL, out, H, T, gh, gw, dir, seg_chunks, nseg};
+  const int BH = B * H;
+  if (dtype == kF16)
+    return stage == 0 ? launch_tc_kernel<__half, false>(p, BH, st, dev)
+                      : launch_tc_kernel<__half, true>(p, BH, st, dev);
+  return stage == 0 ? launch_tc_kernel<__nv_bfloat16, false>(p, BH, st, dev)
+                    : launch_tc_kernel<__nv_bfloat16, true>(p, BH, st, dev);
 }
 
 }  // namespace gtr
