@@ -323,10 +323,14 @@ def run_ours(args, world, rank, local):
             step(sets[i], dirs[i % len(dirs)])
     stream.synchronize()
 
-    # one graph per input set, each holding kernel-boundary events
+    # one graph per input set, each holding kernel-boundary events (torch
+    # creates the CUDA event on its first record, so record each once first)
     graphs, gevents = [], []
     for i in range(N_SETS):
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        for e in evs:
+            e.record(stream)
+        stream.synchronize()
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             step(sets[i], dirs[i % len(dirs)], evs)

@@ -300,9 +300,45 @@ gtr_status_t gtr_gate_fwd(const void* x, int x_dtype, const float* w_down, const
       (bias && !aligned16(bias)))
     return GTR_ERR_ALIGNMENT;
   const int HD = H * dk;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (rank <= 16 && HD % 4 == 0 && HD <= kGate2MaxHD && (!bias || aligned16(bias))) {
+    // register-tiled kernel: one block per 64 tokens
+    const long long blocks = (N + kGate2Tok - 1) / kGate2Tok;
+    if (blocks > 0x7fffffffLL) return GTR_ERR_INVALID_ARG;
+    const size_t smem = gate_tiled_smem(HD);
+    int dev;
+    if (int rc = current_device(&dev)) return (gtr_status_t)rc;
+    const float inv_tau = 1.0f / tau;
+    switch (x_dtype) {
+      case GTR_F32: {
+        static bool done[kMaxDevices];
+        if (int rc = ensure_smem(gate_proj_tiled<float>, gate_tiled_smem(kGate2MaxHD), done, dev))
+          return (gtr_status_t)rc;
+        gate_proj_tiled<float><<<(unsigned)blocks, kGate2Threads, smem, st>>>(
+            (const float*)x, w_down, w_up, bias, g_out, N, d_model, rank, HD, inv_tau);
+        break;
+      }
+      case GTR_F16: {
+        static bool done[kMaxDevices];
+        if (int rc = ensure_smem(gate_proj_tiled<__half>, gate_tiled_smem(kGate2MaxHD), done, dev))
+          return (gtr_status_t)rc;
+        gate_proj_tiled<__half><<<(unsigned)blocks, kGate2Threads, smem, st>>>(
+            (const __half*)x, w_down, w_up, bias, g_out, N, d_model, rank, HD, inv_tau);
+        break;
+      }
+      default: {
+        static bool done[kMaxDevices];
+        if (int rc = ensure_smem(gate_proj_tiled<__nv_bfloat16>, gate_tiled_smem(kGate2MaxHD), done, dev))
+          return (gtr_status_t)rc;
+        gate_proj_tiled<__nv_bfloat16><<<(unsigned)blocks, kGate2Threads, smem, st>>>(
+            (const __nv_bfloat16*)x, w_down, w_up, bias, g_out, N, d_model, rank, HD, inv_tau);
+        break;
+      }
+    }
+    return (gtr_status_t)launch_status();
+  }
   const long long blocks = (N + kGateTok - 1) / kGateTok;
   if (blocks > 0x7fffffffLL) return GTR_ERR_INVALID_ARG;
-  cudaStream_t st = (cudaStream_t)stream;
   switch (x_dtype) {
     case GTR_F32:
       gate_proj_kernel<float><<<(unsigned)blocks, kGateThreads, 0, st>>>(

@@ -21,10 +21,13 @@
 //
 // Data movement: every token's head vector is one contiguous 128-byte row (256
 // bytes for the fp32 gate), so the scan order is applied per token as the
-// source address of a 1-D bulk copy (cp.async.bulk, completion on an
-// mbarrier) into a double-buffered staging area; no transpose kernel runs and
-// reversed orders are just reversed addresses.  The next chunk's copies are in
-// flight while the current chunk computes.
+// source address of 16-byte cp.async copies issued by all threads into a
+// staging area; no transpose kernel runs and reversed orders are just
+// reversed addresses.  The next chunk's q, k, v, g are fetched as soon as the
+// current chunk's operand tiles are built, and its z as soon as the current
+// epilogue is done, so the copies overlap the tensor-core work.  Two CTAs
+// share an SM (three for the summary kernel), which hides the latency of one
+// CTA's serial phases behind the others'.
 //
 // Tensor cores: tcgen05.mma kind::f16, M = 64, N = 64, K = 16 per
 // instruction, fp32 accumulators in tensor memory.  Every operand is a pair of
@@ -34,11 +37,14 @@
 //   cols [  0, 64)  q~ S'           A = q~ (K-major),  B = S' (MN-major)
 //   cols [ 64,128)  scores q~ k~^T  A = q~ (K-major),  B = k~ (K-major)
 //   cols [128,192)  P V             A = P  (K-major),  B = V  (MN-major)
-//   cols [192,256)  dS = k^^T V     A = k^ (MN-major), B = V  (MN-major)
-// An M = 64 accumulator puts row r in TMEM lane 32*(r/16) + r%16, so warp w
-// owns rows 16w..16w+15 in its lanes 0-15.  The masked scores P go back to
-// shared memory (K-major, two-term) for P V.  The epilogue reads whole rows,
-// so RMSNorm needs no cross-thread reduction.
+//   cols [192,256)  k~^T V          A = k~ (MN-major), B = V  (MN-major)
+// The state update uses k^ = diag(e^{Gam - G_m}) k~, a per-row factor of the
+// k~^T V accumulator, so one key tile serves both products (read K-major for
+// the scores and MN-major for the state).  An M = 64 accumulator puts row r in
+// TMEM lane 32*(r/16) + r%16, so warp w owns rows 16w..16w+15 in its lanes
+// 0-15.  The masked scores P go back to shared memory (K-major, two-term) for
+// P V.  The epilogue reads whole rows, so RMSNorm needs no cross-thread
+// reduction.
 #pragma once
 #include "common.cuh"
 
@@ -56,18 +62,18 @@ constexpr int kRawG = kC * kD * 4;     // the fp32 gate tile: 16 KB
 constexpr int kTile = kC * kD * 2;     // one fp16 operand tile: 8 KB
 
 template <bool OUT> struct Layout {
-  static constexpr int kStage = OUT ? (4 * kRaw16 + kRawG) : (2 * kRaw16 + kRawG);
+  // single staging area: k, v, g [, q, z]
   static constexpr int kOffK = 0, kOffV = kRaw16, kOffG = 2 * kRaw16;
   static constexpr int kOffQ = 2 * kRaw16 + kRawG, kOffZ = 3 * kRaw16 + kRawG;
-  static constexpr int kOperands = 2 * kStage;
-  // tiles: V, k^ (hi, lo) [, q~ (hi, lo), k~ (hi, lo), S' (hi, lo)]
-  static constexpr int kTiles = OUT ? 9 : 3;
-  static constexpr int kMisc = kOperands + kTiles * kTile;
-  static constexpr int kMiscBytes = 6144;
+  static constexpr int kStage = OUT ? (4 * kRaw16 + kRawG) : (2 * kRaw16 + kRawG);
+  // fp16 tiles: V, key tile (hi, lo) [, q~ (hi, lo), S' (hi, lo)]
+  static constexpr int kTiles = OUT ? 7 : 3;
+  static constexpr int kMisc = kStage + kTiles * kTile;        // 1024-aligned
+  static constexpr int kMiscBytes = 5632;
   static constexpr int kSmem = kMisc + kMiscBytes + 1024;      // + alignment slack
   static constexpr int kTmemCols = OUT ? 256 : 64;
   static constexpr int kColDS = OUT ? 192 : 0;
-  static constexpr uint32_t kTokenBytes = OUT ? (4 * kD * 2 + kD * 4) : (2 * kD * 2 + kD * 4);
+  static constexpr int kBlocksPerSM = OUT ? 2 : 3;
 };
 
 // ------------------------------------------------------------------ PTX
@@ -84,10 +90,6 @@ __device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
 }
 __device__ __forceinline__ void mbar_fence_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(b)), "r"(bytes)
-               : "memory");
 }
 __device__ __forceinline__ uint32_t mbar_try(uint64_t* b, uint32_t parity) {
   uint32_t ok;
@@ -108,12 +110,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity) {
     if (globaltimer() - t0 > kWaitNs) return false;
   return true;
 }
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          saddr(dst)),
-      "l"(src), "r"(bytes), "r"(saddr(bar))
-      : "memory");
+// 16-byte asynchronous global -> shared copy (L2 only), grouped by commit.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(saddr(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// wait until at most `pending` of this thread's committed groups are in flight
+__device__ __forceinline__ void cp_async_wait(int pending) {
+  if (pending) asm volatile("cp.async.wait_group 1;" ::: "memory");
+  else asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -305,52 +310,85 @@ struct Params {
   int H, T, gh, gw, dir, seg_chunks, nseg;
 };
 
-struct Misc {                   // per-CTA scalars in shared memory
-  uint64_t full[2];             // staging stage filled
-  uint64_t mma;                 // MMA group committed
+struct Misc {                   // per-CTA scalars in shared memory; every array that is read
+                                // as float4 is 16-byte aligned
+  uint64_t mma[2];              // [0] scores committed, [1] every product of the chunk committed
   uint32_t tmem;                // tensor-memory base address
-  int abort;
-  float smax[4];                // per-warp max |S| of the carried state
-  float Gm[kD], Gam[kD], aG[kD], eK[kD], wv[kD];
-  float lo[2][kD], hi[2][kD], half0[kD], kmx[2][kD], vmx[2][kD];
-  float sev[kD], iev[kD];       // V column scales 2^e and 2^-e
-  float skh[kD], ikh[kD];       // k^ row (key dim) scales
-  float ieq[kC], iek[kC], iep[kC];   // inverse row scales of q~, k~, P
+  int pad;
+  alignas(16) float smax[4];    // per-warp max |S| of the carried state
+  alignas(16) float kbound[2][2];   // per-warp max of the k~ [0] and k^ [1] bounds over key dims
+  alignas(16) float Gm[kD];
+  alignas(16) float Gam[kD];
+  alignas(16) float aG[kD];
+  alignas(16) float eK[kD];
+  alignas(16) float wv[kD];
+  alignas(16) float lo[2][kD];
+  alignas(16) float hi[2][kD];
+  alignas(16) float half0[kD];
+  alignas(16) float kmx[2][kD];
+  alignas(16) float vmx[2][kD];
+  alignas(16) float sev[kD];    // V column scales 2^e and 2^-e
+  alignas(16) float iev[kD];
+  alignas(16) float ieq[kC];    // inverse row scales of q~ and P
+  alignas(16) float iep[kC];
+  alignas(16) long long rows[kC];   // token rows (b*T + t)*H + h of the chunk being fetched
 };
-static_assert(sizeof(Misc) <= 6144, "Misc must fit its reserved bytes");
+static_assert(sizeof(Misc) <= 5632, "Misc must fit its reserved bytes");
+static_assert(offsetof(Misc, Gm) % 16 == 0 && offsetof(Misc, Gam) % 16 == 0 &&
+                  offsetof(Misc, wv) % 16 == 0 && offsetof(Misc, sev) % 16 == 0 &&
+                  offsetof(Misc, iev) % 16 == 0 && offsetof(Misc, eK) % 16 == 0,
+              "float4 reads of Misc arrays need 16-byte alignment");
 
-// Issue the bulk copies of one chunk (warp 0): every token row of k, v, g (and
-// q, z for the output kernel), in scan order, into the staging stage.
+// Token rows of the chunk starting at scan position s0 (threads 0..ntok-1).
+__device__ __forceinline__ void chunk_rows(const Params& p, Misc& m, int b, int h, int d, int s0,
+                                           int ntok, int tid) {
+  if (tid < ntok)
+    m.rows[tid] = ((long long)b * p.T + scan_to_grid(d, s0 + tid, p.T, p.gh, p.gw)) * p.H + h;
+}
+
+// Fetch k, v, g (and q for the output kernel) of a chunk: 16-byte pieces, the
+// 128-byte row of a token split over 8 consecutive threads.  One commit group.
 template <typename T, bool OUT>
-__device__ __forceinline__ void issue_chunk(const Params& p, uint8_t* stage, uint64_t* bar, int b,
-                                            int h, int d, int s0, int ntok, int lane) {
+__device__ __forceinline__ void fetch_kvqg(const Params& p, uint8_t* stg, const Misc& m, int ntok,
+                                           int tid) {
   using L = Layout<OUT>;
-  if (lane == 0) mbar_expect_tx(bar, (uint32_t)ntok * L::kTokenBytes);
-  __syncwarp();
-  for (int j = lane; j < ntok; j += 32) {
-    const int t = scan_to_grid(d, s0 + j, p.T, p.gh, p.gw);
-    const size_t row = ((size_t)b * p.T + t) * p.H + h;
-    bulk_g2s(stage + L::kOffK + j * kD * 2, (const T*)p.k + row * kD, kD * 2, bar);
-    bulk_g2s(stage + L::kOffV + j * kD * 2, (const T*)p.v + row * kD, kD * 2, bar);
-    bulk_g2s(stage + L::kOffG + j * kD * 4, p.g + row * kD, kD * 4, bar);
-    if (OUT) {
-      bulk_g2s(stage + L::kOffQ + j * kD * 2, (const T*)p.q + row * kD, kD * 2, bar);
-      bulk_g2s(stage + L::kOffZ + j * kD * 2, (const T*)p.z + row * kD, kD * 2, bar);
-    }
+  for (int o = tid; o < ntok * 8; o += kThreads) {
+    const int j = o >> 3, part = (o & 7) * 16;
+    const size_t src = (size_t)m.rows[j] * (kD * 2) + part;
+    cp_async16(stg + L::kOffK + j * 128 + part, (const uint8_t*)p.k + src);
+    cp_async16(stg + L::kOffV + j * 128 + part, (const uint8_t*)p.v + src);
+    if (OUT) cp_async16(stg + L::kOffQ + j * 128 + part, (const uint8_t*)p.q + src);
   }
+  for (int o = tid; o < ntok * 16; o += kThreads) {
+    const int j = o >> 4, part = (o & 15) * 16;
+    cp_async16(stg + L::kOffG + j * 256 + part, (const uint8_t*)p.g + (size_t)m.rows[j] * (kD * 4) + part);
+  }
+  cp_async_commit();
+}
+// Fetch z of a chunk (output kernel).  One commit group.
+__device__ __forceinline__ void fetch_z(const Params& p, uint8_t* stg, const Misc& m, int ntok,
+                                        int tid) {
+  using L = Layout<true>;
+  for (int o = tid; o < ntok * 8; o += kThreads) {
+    const int j = o >> 3, part = (o & 7) * 16;
+    cp_async16(stg + L::kOffZ + j * 128 + part, (const uint8_t*)p.z + (size_t)m.rows[j] * (kD * 2) + part);
+  }
+  cp_async_commit();
 }
 
 // Column pass over the chunk (two threads per column, 32 tokens each): the
 // in-place inclusive cumsum of the gate tile, and the column maxima of |k| and
-// |v|.  Then per column d: G_m, Gam, e^{Gam}, e^{Gam-G_m}, the k^ and V
-// scales.  Returns true (block-uniform) if the chunk needs the exact scores:
-// its decay range exceeds kSpanMax or some gate sum rises above zero.
-template <typename T>
+// |v|.  Then per column d: G_m, Gam, e^{Gam}, e^{Gam-G_m}, the V scales and
+// the bound of the k~ (output kernel) or k^ (summary kernel) column.  Returns
+// true (block-uniform) if the chunk needs the exact scores: its decay range
+// exceeds kSpanMax or some gate sum rises above zero.
+template <typename T, bool OUT>
 __device__ __forceinline__ bool column_pass(float* G, const T* kst, const T* vst, Misc& m, int ntok,
                                             int tid) {
   const int dd = tid & 63, half = tid >> 6;
   const int j0 = half * 32, j1 = min(j0 + 32, ntok);
   float run = 0.f, lo = 3.0e38f, hi = -3.0e38f, km = 0.f, vm = 0.f;
+#pragma unroll 4
   for (int j = j0; j < j1; ++j) {
     run += G[j * kD + dd];
     G[j * kD + dd] = run;
@@ -365,6 +403,7 @@ __device__ __forceinline__ bool column_pass(float* G, const T* kst, const T* vst
   __syncthreads();
   if (half == 1 && j1 > j0) {
     const float off = m.half0[dd];
+#pragma unroll 4
     for (int j = j0; j < j1; ++j) G[j * kD + dd] += off;
     lo += off;
     hi += off;
@@ -376,19 +415,28 @@ __device__ __forceinline__ bool column_pass(float* G, const T* kst, const T* vst
   if (tid < kD) {
     const float gam = G[(ntok - 1) * kD + tid];
     const float gm = G[((ntok - 1) >> 1) * kD + tid];
-    const float mn = fminf(m.lo[0][tid], m.lo[1][tid]), mx = fmaxf(m.hi[0][tid], m.hi[1][tid]);
+    const float mn = fminf(fminf(m.lo[0][tid], m.lo[1][tid]), 0.f);
+    const float mx = fmaxf(m.hi[0][tid], m.hi[1][tid]);
     m.Gam[tid] = gam;
     m.Gm[tid] = gm;
     m.aG[tid] = expf(gam);
     m.eK[tid] = expf(gam - gm);
-    // k^_id = k_id e^{Gam_d - G_id} <= max_i |k_id| e^{Gam_d - min_i G_id}
-    const int ek = scale_exp(fmaxf(m.kmx[0][tid], m.kmx[1][tid]) * expf(gam - fminf(mn, 0.f)));
-    m.skh[tid] = pow2i(ek);
-    m.ikh[tid] = pow2i(-ek);
     const int ev = scale_exp(fmaxf(m.vmx[0][tid], m.vmx[1][tid]));
     m.sev[tid] = pow2i(ev);
     m.iev[tid] = pow2i(-ev);
-    const float span = fmaxf(mx, 0.f) - fminf(mn, 0.f);
+    // |k~_id| <= max_i |k_id| e^{G_m,d - min_i G_id};  |k^_id| <= max_i |k_id| e^{Gam_d - min_i G_id}
+    const float km = fmaxf(m.kmx[0][tid], m.kmx[1][tid]);
+    float kb0 = km * expf(gm - mn), kb1 = km * expf(gam - mn);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      kb0 = fmaxf(kb0, __shfl_xor_sync(0xffffffffu, kb0, o));
+      kb1 = fmaxf(kb1, __shfl_xor_sync(0xffffffffu, kb1, o));
+    }
+    if ((tid & 31) == 0) {
+      m.kbound[0][tid >> 5] = kb0;
+      m.kbound[1][tid >> 5] = kb1;
+    }
+    const float span = fmaxf(mx, 0.f) - mn;
     irregular = !(span <= kSpanMax) || mx > 0.f;
   }
   return __syncthreads_or(irregular) != 0;
@@ -406,24 +454,29 @@ __device__ __forceinline__ void state_max(const float* S, bool owner, Misc& m, i
   if (lane == 0) m.smax[warp] = mx;
 }
 
+__device__ __forceinline__ float silu_fast(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
+
 template <typename T, bool OUT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, Layout<OUT>::kBlocksPerSM)
 gla_tc(const Params p) {
   using L = Layout<OUT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* stages = sm;
-  uint8_t* tiles = sm + L::kOperands;
-  uint8_t* VV = tiles;                       // V            (MN-major B), single fp16 tile
-  uint8_t* KHh = tiles + 1 * kTile;          // k^ hi / lo   (MN-major A)
-  uint8_t* KHl = tiles + 2 * kTile;
+  uint8_t* stg = sm;
+  uint8_t* tiles = sm + L::kStage;
+  uint8_t* VV = tiles;                       // V (MN-major B), one fp16 term
+  uint8_t* KTh = tiles + 1 * kTile;          // k~ (output) or k^ (summary), hi / lo
+  uint8_t* KTl = tiles + 2 * kTile;
   uint8_t* QTh = tiles + 3 * kTile;          // q~ hi / lo, then P (K-major A)   [OUT]
   uint8_t* QTl = tiles + 4 * kTile;
-  uint8_t* KTh = tiles + 5 * kTile;          // k~ hi / lo   (K-major B)         [OUT]
-  uint8_t* KTl = tiles + 6 * kTile;
-  uint8_t* SPh = tiles + 7 * kTile;          // S' hi / lo   (MN-major B)        [OUT]
-  uint8_t* SPl = tiles + 8 * kTile;
+  uint8_t* SPh = tiles + 5 * kTile;          // S' hi / lo   (MN-major B)        [OUT]
+  uint8_t* SPl = tiles + 6 * kTile;
   Misc& m = *reinterpret_cast<Misc*>(sm + L::kMisc);
+  float* G = reinterpret_cast<float*>(stg + L::kOffG);
+  const T* kst = reinterpret_cast<const T*>(stg + L::kOffK);
+  const T* vst = reinterpret_cast<const T*>(stg + L::kOffV);
+  const T* qst = reinterpret_cast<const T*>(stg + L::kOffQ);
+  const T* zst = reinterpret_cast<const T*>(stg + L::kOffZ);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int seg = blockIdx.x, bh = blockIdx.y;
@@ -437,7 +490,13 @@ gla_tc(const Params p) {
     return;
   }
   const bool owner = lane < 16;          // this thread holds accumulator row 16*warp + lane
-  const int row = warp * 16 + lane;      // that row: a query token, or a key dim of S
+  const int row = warp * 16 + (lane & 15);   // that row: a query token, or a key dim of S
+
+  // first chunk's copies go out before anything else
+  chunk_rows(p, m, b, h, d, c0 * kC, min(kC, p.T - c0 * kC), tid);
+  __syncthreads();
+  fetch_kvqg<T, OUT>(p, stg, m, min(kC, p.T - c0 * kC), tid);
+  if (OUT) fetch_z(p, stg, m, min(kC, p.T - c0 * kC), tid);
 
   // carried state: row `row` of S (key dim), 64 value columns
   float S[kD];
@@ -455,11 +514,9 @@ gla_tc(const Params p) {
   }
   if (OUT) state_max(S, owner, m, warp, lane);
   if (tid == 0) {
-    mbar_init(&m.full[0], 1);
-    mbar_init(&m.full[1], 1);
-    mbar_init(&m.mma, 1);
+    mbar_init(&m.mma[0], 1);
+    mbar_init(&m.mma[1], 1);
     mbar_fence_init();
-    m.abort = 0;
   }
   if (tid < kD) m.wv[tid] = (OUT && p.w) ? p.w[tid] : 1.0f;
   if (warp == 0) {
@@ -473,43 +530,26 @@ gla_tc(const Params p) {
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
 
   float lsum = 0.f;
-  uint32_t mma_phase = 0;
-  uint32_t outstanding = 1;               // bit s: stage s has copies in flight
-
-  if (warp == 0) {
-    const int s0 = c0 * kC;
-    issue_chunk<T, OUT>(p, stages, &m.full[0], b, h, d, s0, min(kC, p.T - s0), lane);
-  }
+  uint32_t ph0 = 0, ph1 = 0;
+  bool failed = false;
 
   for (int it = 0; it < nch; ++it) {
-    const int st = it & 1;
-    uint8_t* stg = stages + st * L::kStage;
     const int s0 = (c0 + it) * kC;
     const int ntok = min(kC, p.T - s0);
-    if (it + 1 < nch) {
-      if (warp == 0) {
-        const int s1 = s0 + kC;
-        issue_chunk<T, OUT>(p, stages + (st ^ 1) * L::kStage, &m.full[st ^ 1], b, h, d, s1,
-                            min(kC, p.T - s1), lane);
-      }
-      outstanding |= 1u << (st ^ 1);
-    }
-    const bool ok = mbar_wait(&m.full[st], (it >> 1) & 1);
-    outstanding &= ~(1u << st);
-    if (__syncthreads_or(!ok)) {
-      if (tid == 0) gtr_flag(kStatusMbarTimeout);
-      m.abort = 1;
-      break;
-    }
+    const bool more = it + 1 < nch;
+    const int s1 = s0 + kC;
+    const int ntok1 = more ? min(kC, p.T - s1) : 0;
 
-    float* G = reinterpret_cast<float*>(stg + L::kOffG);
-    const T* kst = reinterpret_cast<const T*>(stg + L::kOffK);
-    const T* vst = reinterpret_cast<const T*>(stg + L::kOffV);
-    const T* qst = reinterpret_cast<const T*>(stg + L::kOffQ);
-    const bool exact = column_pass<T>(G, kst, vst, m, ntok, tid) && OUT;
+    cp_async_wait(OUT ? 1 : 0);          // k, v, g (, q) of this chunk are in
+    __syncthreads();
+    const bool exact = column_pass<T, OUT>(G, kst, vst, m, ntok, tid) && OUT;
 
     // ---- operand tiles; rows beyond ntok are zero.  Items: (row r, 4 columns
     // cg..cg+3); a half warp covers one row, which makes per-row maxima cheap.
+    // the key tile holds k~ = k e^{G_m - G} for a regular output chunk, else k^ = k e^{Gam - G}
+    const bool tilde = OUT && !exact;
+    const int ekt = scale_exp(fmaxf(m.kbound[tilde ? 0 : 1][0], m.kbound[tilde ? 0 : 1][1]));
+    const float skt = pow2i(ekt);
 #pragma unroll 2
     for (int u = 0; u < 8; ++u) {
       const int item = u * kThreads + tid;
@@ -522,31 +562,21 @@ gla_tc(const Params p) {
         if (OUT) qq = Vec4<T>::load(qst + r * kD + cg);
       }
       const float4 gg = *reinterpret_cast<const float4*>(G + r * kD + cg);
-      const float4 ga = *reinterpret_cast<const float4*>(&m.Gam[cg]);
       const uint32_t off = sw16(r, cg);
-      {   // V (column-scaled, one fp16 term: exact for 16-bit inputs)
+      {   // V, column-scaled, one fp16 term (exact for 16-bit inputs)
         const float4 sv = *reinterpret_cast<const float4*>(&m.sev[cg]);
         *reinterpret_cast<uint2*>(VV + off) = half4(vv.x * sv.x, vv.y * sv.y, vv.z * sv.z, vv.w * sv.w);
       }
-      {   // k^ = k e^{Gam - G} (key-dim scaled; rows = tokens = K of dS)
-        const float4 sk = *reinterpret_cast<const float4*>(&m.skh[cg]);
-        put2(KHh, KHl, off, kk.x * __expf(ga.x - gg.x) * sk.x, kk.y * __expf(ga.y - gg.y) * sk.y,
-             kk.z * __expf(ga.z - gg.z) * sk.z, kk.w * __expf(ga.w - gg.w) * sk.w);
-      }
-      if (OUT) {
-        const float4 gm = *reinterpret_cast<const float4*>(&m.Gm[cg]);
+      // k~ = k e^{G_m - G} or k^ = k e^{Gam - G}, tile-scaled
+      const float4 gr = *reinterpret_cast<const float4*>(tilde ? &m.Gm[cg] : &m.Gam[cg]);
+      put2(KTh, KTl, off, kk.x * __expf(gr.x - gg.x) * skt, kk.y * __expf(gr.y - gg.y) * skt,
+           kk.z * __expf(gr.z - gg.z) * skt, kk.w * __expf(gr.w - gg.w) * skt);
+      if (OUT) {   // q~ = q e^{G - G_m} (exact chunk: q e^{G}), row-scaled
         float q0, q1, q2, q3;
         if (!exact) {
-          // k~ = k e^{G_m - G}, row (key token) scaled
-          const float a0 = kk.x * __expf(gm.x - gg.x), a1 = kk.y * __expf(gm.y - gg.y);
-          const float a2 = kk.z * __expf(gm.z - gg.z), a3 = kk.w * __expf(gm.w - gg.w);
-          const int ek = scale_exp(half_warp_max(amax4(a0, a1, a2, a3)));
-          const float s = pow2i(ek);
-          put2(KTh, KTl, off, a0 * s, a1 * s, a2 * s, a3 * s);
-          if (cg == 0) m.iek[r] = pow2i(-ek);
-          q0 = qq.x * __expf(gg.x - gm.x); q1 = qq.y * __expf(gg.y - gm.y);
-          q2 = qq.z * __expf(gg.z - gm.z); q3 = qq.w * __expf(gg.w - gm.w);
-        } else {   // exact chunk: q~ = q e^{G_j}
+          q0 = qq.x * __expf(gg.x - gr.x); q1 = qq.y * __expf(gg.y - gr.y);
+          q2 = qq.z * __expf(gg.z - gr.z); q3 = qq.w * __expf(gg.w - gr.w);
+        } else {
           q0 = qq.x * __expf(gg.x); q1 = qq.y * __expf(gg.y);
           q2 = qq.z * __expf(gg.z); q3 = qq.w * __expf(gg.w);
         }
@@ -569,43 +599,45 @@ gla_tc(const Params p) {
           put2(SPh, SPl, sw16(row, c), sc * S[c], sc * S[c + 1], sc * S[c + 2], sc * S[c + 3]);
       }
     }
+    if (more && !exact) chunk_rows(p, m, b, h, d, s1, ntok1, tid);
     fence_async_smem();
     tc_before_sync();
     __syncthreads();
     tc_after_sync();
 
+    // staging of this chunk is consumed (except z): fetch the next chunk now
+    if (more && !exact) fetch_kvqg<T, OUT>(p, stg, m, ntok1, tid);
+
     if (tid == 0) {
+      // q~ S' and the scores first: their commit frees the q~ tiles for P
       if (OUT) {
         mma_pair(tm + 0, saddr(QTh), saddr(QTl), false, saddr(SPh), saddr(SPl), true, false);
         if (!exact)
           mma_pair(tm + 64, saddr(QTh), saddr(QTl), false, saddr(KTh), saddr(KTl), false, false);
+        mma_commit(&m.mma[0]);
       }
-      mma_64(tm + L::kColDS, saddr(KHh), true, saddr(VV), true, false);
-      mma_64(tm + L::kColDS, saddr(KHl), true, saddr(VV), true, true);
-      mma_commit(&m.mma);
+      mma_64(tm + L::kColDS, saddr(KTh), true, saddr(VV), true, false);
+      mma_64(tm + L::kColDS, saddr(KTl), true, saddr(VV), true, true);
+      if (!OUT) mma_commit(&m.mma[1]);
     }
-    bool okm = mbar_wait(&m.mma, mma_phase);
-    mma_phase ^= 1;
-    if (__syncthreads_or(!okm)) {
-      if (tid == 0) gtr_flag(kStatusMbarTimeout);
-      m.abort = 1;
-      break;
-    }
-    tc_after_sync();
 
     if (OUT) {
       // ---- masked scores P (rows = queries j, columns = keys i), row-scaled, into QT
       if (!exact) {
+        const bool okm = mbar_wait(&m.mma[0], ph0);
+        ph0 ^= 1;
+        failed |= !okm;
+        tc_after_sync();
         float sc[kC];
 #pragma unroll
         for (int cb = 0; cb < 4; ++cb) tmem_ld16(tm + lane_base + 64 + cb * 16, sc + cb * 16);
         tmem_ld_wait();
         if (owner) {
-          const float iq = m.ieq[row];
+          const float f = m.ieq[row] * pow2i(-ekt);
           float mx = 0.f;
 #pragma unroll
           for (int i = 0; i < kC; ++i) {
-            sc[i] = (i <= row && row < ntok) ? sc[i] * iq * m.iek[i] : 0.f;
+            sc[i] = (i <= row && row < ntok) ? sc[i] * f : 0.f;
             mx = fmaxf(mx, fabsf(sc[i]));
           }
           const int ep = scale_exp(mx);
@@ -616,8 +648,12 @@ gla_tc(const Params p) {
             put2(QTh, QTl, sw16(row, i), sc[i] * s, sc[i + 1] * s, sc[i + 2] * s, sc[i + 3] * s);
         }
       } else {
-        // exact scores on CUDA cores: P_ji = sum_d q_jd k_id e^{G_jd - G_id}; two threads per row
+        // exact scores on CUDA cores: P_ji = sum_d q_jd k_id e^{G_jd - G_id}, two threads per
+        // row; q~ must stay intact until q~ S' is done
         if (tid == 0) atomicAdd(&g_gtr_exact_chunks, 1ull);
+        const bool okm = mbar_wait(&m.mma[0], ph0);
+        ph0 ^= 1;
+        failed |= !okm;
         const int j = tid >> 1, ib = (tid & 1) * 32;
         float acc[32];
 #pragma unroll
@@ -644,43 +680,45 @@ gla_tc(const Params p) {
 #pragma unroll
         for (int e = 0; e < 32; e += 4)
           put2(QTh, QTl, sw16(j, ib + e), acc[e] * s, acc[e + 1] * s, acc[e + 2] * s, acc[e + 3] * s);
+        if (more) chunk_rows(p, m, b, h, d, s1, ntok1, tid);
       }
+      cp_async_wait((more && !exact) ? 1 : 0);     // z of this chunk is in
       fence_async_smem();
       tc_before_sync();
-      __syncthreads();
+      if (__syncthreads_or(failed)) break;
       tc_after_sync();
+      if (exact && more) fetch_kvqg<T, OUT>(p, stg, m, ntok1, tid);
       if (tid == 0) {
         mma_64(tm + 128, saddr(QTh), false, saddr(VV), true, false);
         mma_64(tm + 128, saddr(QTl), false, saddr(VV), true, true);
-        mma_commit(&m.mma);
+        mma_commit(&m.mma[1]);
       }
-      okm = mbar_wait(&m.mma, mma_phase);
-      mma_phase ^= 1;
-      if (__syncthreads_or(!okm)) {
-        if (tid == 0) gtr_flag(kStatusMbarTimeout);
-        m.abort = 1;
-        break;
-      }
-      tc_after_sync();
+    }
+    failed |= !mbar_wait(&m.mma[1], ph1);
+    ph1 ^= 1;
+    tc_after_sync();
 
+    if (OUT) {
       // ---- epilogue: o_j = q~_j S' + P_j V, then o_j / sqrt(mean o_j^2 + eps) * w * SiLU(z_j)
-      float o[kD], pv[kD];
+      float o[kD];
+      float ss = 0.f;
+      const float a = m.ieq[row] * inv_es, bsc = m.iep[row];
 #pragma unroll
       for (int cb = 0; cb < 4; ++cb) {
+        float pv[16];
         tmem_ld16(tm + lane_base + cb * 16, o + cb * 16);
-        tmem_ld16(tm + lane_base + 128 + cb * 16, pv + cb * 16);
-      }
-      tmem_ld_wait();
-      if (owner && row < ntok) {
-        const float a = m.ieq[row] * inv_es, bsc = m.iep[row];
-        float ss = 0.f;
+        tmem_ld16(tm + lane_base + 128 + cb * 16, pv);
+        tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < kD; ++c) {
-          o[c] = o[c] * a + pv[c] * bsc * m.iev[c];
-          ss = fmaf(o[c], o[c], ss);
+        for (int c = 0; c < 16; ++c) {
+          const int cc = cb * 16 + c;
+          o[cc] = o[cc] * a + pv[c] * bsc * m.iev[cc];
+          ss = fmaf(o[cc], o[cc], ss);
         }
-        const float inv = 1.0f / sqrtf(ss * (1.0f / kD) + kRmsEps);
-        const T* zr = reinterpret_cast<const T*>(stg + L::kOffZ) + row * kD;
+      }
+      if (owner && row < ntok) {
+        const float inv = rsqrtf(ss * (1.0f / kD) + kRmsEps);
+        const T* zr = zst + row * kD;
         const int t = scan_to_grid(d, s0 + row, p.T, p.gh, p.gw);
         T* dst = reinterpret_cast<T*>(p.out) + (((size_t)b * p.T + t) * p.H + h) * kD;
 #pragma unroll
@@ -690,37 +728,41 @@ gla_tc(const Params p) {
           const float4 z1 = Vec4<T>::from_bits(make_uint2(zz.z, zz.w));
           const float4 w0 = *reinterpret_cast<const float4*>(&m.wv[c]);
           const float4 w1 = *reinterpret_cast<const float4*>(&m.wv[c + 4]);
-          const uint2 lo = pack4<T>(o[c + 0] * inv * w0.x * silu_f(z0.x), o[c + 1] * inv * w0.y * silu_f(z0.y),
-                                    o[c + 2] * inv * w0.z * silu_f(z0.z), o[c + 3] * inv * w0.w * silu_f(z0.w));
-          const uint2 hi = pack4<T>(o[c + 4] * inv * w1.x * silu_f(z1.x), o[c + 5] * inv * w1.y * silu_f(z1.y),
-                                    o[c + 6] * inv * w1.z * silu_f(z1.z), o[c + 7] * inv * w1.w * silu_f(z1.w));
+          const uint2 lo = pack4<T>(o[c + 0] * inv * w0.x * silu_fast(z0.x), o[c + 1] * inv * w0.y * silu_fast(z0.y),
+                                    o[c + 2] * inv * w0.z * silu_fast(z0.z), o[c + 3] * inv * w0.w * silu_fast(z0.w));
+          const uint2 hi = pack4<T>(o[c + 4] * inv * w1.x * silu_fast(z1.x), o[c + 5] * inv * w1.y * silu_fast(z1.y),
+                                    o[c + 6] * inv * w1.z * silu_fast(z1.z), o[c + 7] * inv * w1.w * silu_fast(z1.w));
           *reinterpret_cast<uint4*>(dst + c) = make_uint4(lo.x, lo.y, hi.x, hi.y);
         }
       }
     }
 
-    // ---- state: S <- e^{Gam} S + dS (fp32 accumulation)
+    // ---- state: S <- e^{Gam} S + diag(e^{Gam - G_m}) k~^T V   (summary: + k^^T V), fp32
     {
-      float ds[kD];
+      const float rs = (tilde ? m.eK[row] : 1.0f) * pow2i(-ekt);
+      const float a = m.aG[row];
 #pragma unroll
-      for (int cb = 0; cb < 4; ++cb) tmem_ld16(tm + lane_base + L::kColDS + cb * 16, ds + cb * 16);
-      tmem_ld_wait();
-      if (owner) {
-        const float a = m.aG[row], ik = m.ikh[row];
+      for (int cb = 0; cb < 4; ++cb) {
+        float ds[16];
+        tmem_ld16(tm + lane_base + L::kColDS + cb * 16, ds);
+        tmem_ld_wait();
+        if (owner) {
 #pragma unroll
-        for (int c = 0; c < kD; ++c) S[c] = fmaf(a, S[c], ds[c] * ik * m.iev[c]);
+          for (int c = 0; c < 16; ++c)
+            S[cb * 16 + c] = fmaf(a, S[cb * 16 + c], ds[c] * rs * m.iev[cb * 16 + c]);
+        }
       }
       if (OUT) state_max(S, owner, m, warp, lane);
     }
     if (!OUT && tid < kD) lsum += m.Gam[tid];
     tc_before_sync();
-    __syncthreads();
+    if (__syncthreads_or(failed)) break;
+    if (OUT && more) fetch_z(p, stg, m, ntok1, tid);     // z of this chunk is consumed
   }
 
-  if (m.abort) {
-    // let copies still in flight land before the block's shared memory is released
-    for (int s = 0; s < 2; ++s)
-      if (outstanding & (1u << s)) (void)mbar_wait(&m.full[s], 0);
+  cp_async_wait(0);                       // no copy may land after the block exits
+  if (failed) {
+    if (tid == 0) gtr_flag(kStatusMbarTimeout);
   } else if (!OUT) {
     if (owner) {
       float4* dst = reinterpret_cast<float4*>(p.wsS + (((size_t)bh * p.nseg + seg) * kD + row) * kD);
@@ -741,7 +783,7 @@ gla_tc(const Params p) {
 inline bool tc_shape_supported(int dk, int dv, int chunk, int dtype) {
   return dk == tc::kD && dv == tc::kD && chunk == tc::kC && (dtype == kF16 || dtype == kBF16);
 }
-inline int tc_blocks_per_sm(int, int) { return 1; }
+inline int tc_blocks_per_sm(int, int) { return tc::Layout<true>::kBlocksPerSM; }
 
 template <typename T, bool OUT>
 inline int launch_tc_kernel(const tc::Params& p, int BH, cudaStream_t st, int dev) {

@@ -105,6 +105,20 @@ def test_gate_projection_bf16_with_bias():
     np.testing.assert_allclose(g.double().cpu().numpy(), ref, rtol=1e-5, atol=1e-6)
 
 
+@pytest.mark.parametrize("rank,H,dk,dm", [(24, 6, 64, 384), (16, 3, 5, 100), (7, 2, 64, 300)])
+def test_gate_projection_other_shapes(rank, H, dk, dm):
+    # shapes outside the register-tiled kernel (rank > 16, H*dk not a multiple of 4) and a
+    # model width that is not a multiple of the staging slab
+    gen = torch.Generator().manual_seed(rank)
+    x = torch.randn(2, 77, dm, generator=gen).to(torch.float16)
+    wd = torch.randn(dm, rank, generator=gen) / dm ** 0.5
+    wu = torch.randn(rank, H * dk, generator=gen) / rank ** 0.5
+    b = torch.randn(H * dk, generator=gen)
+    g = binding.gate_fwd(x.cuda(), wd.cuda(), wu.cuda(), b.cuda(), H, dk, 4.0)
+    ref = oracle.gate(x, wd, wu, b, tau=4.0).reshape(2, 77, H, dk)
+    np.testing.assert_allclose(g.double().cpu().numpy(), ref, rtol=1e-5, atol=2e-6)
+
+
 @pytest.mark.parametrize("direction", DIRS)
 def test_640_all_directions(direction):
     wl, d = _workload_data("640")
