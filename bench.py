@@ -208,12 +208,19 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest value over all ranks (device timings: the slowest rank sets the time)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_value(units_per_rank: int, steps: int, ms_max: float, world: int) -> float:
+    """Whole-job throughput: the units every rank processed over the slowest rank's time."""
+    return world * units_per_rank * steps / (ms_max * 1e-3)
 
 
 # ---------------------------------------------------------------- CPU oracle
@@ -408,8 +415,8 @@ def run_ours(args, world, rank, local):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
 
     units = wl.token_heads
-    value = world * units * args.steps / (ms_max * 1e-3)
-    e2e_value = world * units * args.e2e_steps / (e2e_ms * 1e-3)
+    value = aggregate_value(units, args.steps, ms_max, world)
+    e2e_value = aggregate_value(units, args.e2e_steps, e2e_ms, world)
 
     secondary = None
     if not args.no_secondary and args.workload == "16k":

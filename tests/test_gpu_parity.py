@@ -84,6 +84,16 @@ def test_tiny_fp32():
     _check_status()
 
 
+def test_tiny_fp32_against_stored_oracle_values():
+    import json
+    import os
+    doc = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "tiny_oracle.json")))
+    stored = np.array([float.fromhex(v) for v in doc["y"]]).reshape(doc["shape"])
+    wl, d = _workload_data("tiny")
+    y, _ = _gpu_step(wl, d, "LR")
+    assert_close(y, stored, torch.float32, "tiny vs stored")
+
+
 def test_gate_projection_640():
     wl, d = _workload_data("640")
     g = binding.gate_fwd(_dev(d["x"]), _dev(d["w_down"]), _dev(d["w_up"]), _dev(d["bias"]),

@@ -303,3 +303,14 @@ def test_inputs_are_deterministic_and_shaped():
     t = inputs.make_inputs(inputs.WORKLOADS["tiny"])
     assert t["g"].dtype == torch.float32 and float(t["g"].max()) <= 0.0
     assert t["q"].dtype == torch.float32 and t["q"].shape == (1, 64, 1, 16)
+
+
+def test_oracle_reproduces_its_stored_tiny_output():
+    import json
+    import os
+    doc = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "tiny_oracle.json")))
+    wl = inputs.WORKLOADS["tiny"]
+    d = inputs.make_inputs(wl)
+    y = oracle.gla_fwd(d["q"], d["k"], d["v"], d["g"], d["z"], d["w"], gh=wl.gh, gw=wl.gw)
+    stored = np.array([float.fromhex(v) for v in doc["y"]]).reshape(doc["shape"])
+    np.testing.assert_allclose(y, stored, rtol=1e-13, atol=1e-15)
