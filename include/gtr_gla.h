@@ -127,6 +127,37 @@ GTR_API gtr_status_t gtr_gla_fwd(const void *q, const void *k, const void *v, co
                          void *stream);
 
 /*
+ * gtr_gla_fwd for callers that cannot allocate device memory while they run
+ * (the paper has no counterpart to this entry point).  Examples: a plugin
+ * inside an inference engine that forbids allocation once execution starts, a
+ * real-time loop whose memory footprint is fixed at start-up, or a process
+ * under a hard memory cap.  cudaMalloc can block on the device and fail when
+ * memory runs out, so such callers cannot use the workspace gtr_gla_fwd grows
+ * on demand.  Same arguments and result as gtr_gla_fwd; this call allocates
+ * nothing and calls no allocating routine.
+ *   Scratch: a static device array of GTR_NOALLOC_SCRATCH_BYTES (8 MiB) that
+ *   every GPU loading the library reserves until the process exits.  The
+ *   boundary states need B*H*nseg*(dk*dv + dk)*4 bytes; when the usual segment
+ *   plan needs more, longer segments are used (same result up to rounding).
+ *   If even one segment per sequence does not fit, i.e.
+ *   B*H*(dk*dv + dk)*4 + 256 > 8 MiB, the call returns GTR_ERR_NO_MEMORY and
+ *   launches nothing.
+ *   The first call on a device looks up the array's device address (once per
+ *   device, with that device current); make that first call before any stream
+ *   capture.
+ *   All calls share the one array and it keeps the last call's contents;
+ *   nothing in it needs to start at zero (every element is written before it
+ *   is read within a call).  Calls whose work overlaps on the GPU (other
+ *   streams, or other host threads) race on the array and give wrong results:
+ *   order them.
+ */
+#define GTR_NOALLOC_SCRATCH_BYTES (8u << 20)
+GTR_API gtr_status_t gtr_gla_fwd_noalloc(const void *q, const void *k, const void *v,
+                                         const float *g, const void *outgate, const float *rms_w,
+                                         void *out, int B, int H, int grid_h, int grid_w, int dk,
+                                         int dv, int dir, int chunk, int dtype, void *stream);
+
+/*
  * gtr_gla_fwd that also records caller-created cudaEvent_t handles (any may be
  * NULL) on `stream`: ev[0] before the summary kernel, ev[1] after it, ev[2]
  * after the state scan, ev[3] after the output kernel.  For profiling only.

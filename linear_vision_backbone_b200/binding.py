@@ -26,6 +26,7 @@ EXPORTS = (
     "gtr_abi_version", "gtr_status_string", "gtr_gate_fwd", "gtr_gla_fwd", "gtr_gla_fwd_timed",
     "gtr_gla_chunk_states", "gtr_gla_workspace_bytes", "gtr_gla_set_workspace",
     "gtr_gla_set_path", "gtr_gla_path_for", "gtr_last_device_status", "gtr_gla_segment_chunks",
+    "gtr_gla_fwd_noalloc",
 )
 
 _lock = threading.Lock()
@@ -63,6 +64,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
             "gtr_gla_path_for": ([I, I, I, I, I, I, I, I], I),
             "gtr_last_device_status": ([P, P], I),
             "gtr_gla_segment_chunks": ([I, I, I, I, I, I, I, I], I),
+            "gtr_gla_fwd_noalloc": ([P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, P], I),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -157,6 +159,19 @@ def gla_fwd(q, k, v, g, z, w=None, *, grid_h: int, grid_w: int, direction: str =
     else:
         arr = (ctypes.c_void_p * 4)(*[None if e is None else e.cuda_event for e in events])
         _check("gtr_gla_fwd_timed", lib.gtr_gla_fwd_timed(*args, arr))
+    return out
+
+
+def gla_fwd_noalloc(q, k, v, g, z, w=None, *, grid_h: int, grid_w: int, direction: str = "LR",
+                    chunk: int = 64, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """``gtr_gla_fwd_noalloc``: the result of :func:`gla_fwd` without any device allocation
+    by the library (its scratch is a fixed static device array; see include/gtr_gla.h).
+    Raises GtrError with status -4 when the problem needs more than that scratch."""
+    B, T, H, dk, dv, out = _gla_check(q, k, v, g, z, w, out, grid_h, grid_w)
+    rc = load().gtr_gla_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(z), _ptr(w), _ptr(out),
+                                    B, H, grid_h, grid_w, dk, dv, DIR_IDS[direction], int(chunk),
+                                    DTYPE_IDS[q.dtype], _stream(stream))
+    _check("gtr_gla_fwd_noalloc", rc)
     return out
 
 

@@ -266,6 +266,65 @@ int gla_fwd_impl(const void* q, const void* k, const void* v, const float* g, co
   return record(ev, 3, st);
 }
 
+// ---------------------------------------------------------------------------
+// Allocation-free variant of gtr_gla_fwd.  Its scratch (the segment states of
+// the summary and scan stages) is this file-scope device array instead of a
+// cudaMalloc'ed workspace.  Every GPU that loads the library reserves it until
+// the process exits.  Host code may not use the array's name as a device
+// pointer (on the host it names a stand-in object), so its device address is
+// looked up once per device with cudaGetSymbolAddress, with that device
+// current, and passed to the kernels.
+constexpr size_t kStaticScratchBytes = (size_t)8 << 20;   // 8 MiB per device
+static __device__ __align__(256) unsigned char g_gtr_static_scratch[kStaticScratchBytes];
+void* g_static_scratch_ptr[kMaxDevices];
+
+int static_scratch(int dev, void** out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_static_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_gtr_static_scratch) != cudaSuccess || !ptr) {
+      (void)cudaGetLastError();
+      return GTR_ERR_CUDA;
+    }
+    g_static_scratch_ptr[dev] = ptr;
+  }
+  *out = g_static_scratch_ptr[dev];
+  return GTR_OK;
+}
+
+int gla_fwd_noalloc_impl(const void* q, const void* k, const void* v, const float* g, const void* z,
+                         const float* w, void* out, int B, int H, int gh, int gw, int dk, int dv,
+                         int dir, int chunk, int dtype, void* stream) {
+  int rc = check_gla_args(B, H, gh, gw, dk, dv, dir, chunk, dtype);
+  if (rc) return rc;
+  if (B == 0 || H == 0 || gh == 0 || gw == 0) return GTR_OK;
+  if (!q || !k || !v || !g || !z || !out) return GTR_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(z) ||
+      !aligned16(out) || (w && !aligned16(w)))
+    return GTR_ERR_ALIGNMENT;
+  int dev;
+  if ((rc = current_device(&dev))) return rc;
+  Plan p;
+  if ((rc = make_plan(&p, dev, B, H, gh, gw, dk, dv, dir, chunk, dtype, 0))) return rc;
+  if (p.ws_bytes > kStaticScratchBytes) {
+    // fewer, longer segments until the boundary states fit the static scratch
+    const size_t per_seg = (size_t)B * H * ((size_t)dk * dv + dk) * sizeof(float);
+    const size_t max_nseg = (kStaticScratchBytes - 256) / per_seg;
+    if (max_nseg < 1) return GTR_ERR_NO_MEMORY;
+    const int seg = (int)((p.nc + max_nseg - 1) / max_nseg);
+    if ((rc = make_plan(&p, dev, B, H, gh, gw, dk, dv, dir, chunk, dtype, seg))) return rc;
+    if (p.ws_bytes > kStaticScratchBytes) return GTR_ERR_NO_MEMORY;
+  }
+  void* ws = nullptr;
+  if ((rc = static_scratch(dev, &ws))) return rc;
+  float* wsS = (float*)ws;
+  float* wsL = (float*)((char*)ws + p.offL);
+  cudaStream_t st = (cudaStream_t)stream;
+  if ((rc = launch_stage(p, q, k, v, g, z, w, out, wsS, wsL, st, 0))) return rc;
+  if ((rc = launch_scan(p, wsS, wsL, 0, st))) return rc;
+  return launch_stage(p, q, k, v, g, z, w, out, wsS, wsL, st, 1);
+}
+
 }  // namespace
 
 extern "C" {
@@ -362,6 +421,14 @@ gtr_status_t gtr_gla_fwd(const void* q, const void* k, const void* v, const floa
                          void* stream) {
   return (gtr_status_t)gla_fwd_impl(q, k, v, g, outgate, rms_w, out, B, H, grid_h, grid_w, dk, dv,
                                     dir, chunk, dtype, stream, nullptr);
+}
+
+gtr_status_t gtr_gla_fwd_noalloc(const void* q, const void* k, const void* v, const float* g,
+                                 const void* outgate, const float* rms_w, void* out, int B, int H,
+                                 int grid_h, int grid_w, int dk, int dv, int dir, int chunk,
+                                 int dtype, void* stream) {
+  return (gtr_status_t)gla_fwd_noalloc_impl(q, k, v, g, outgate, rms_w, out, B, H, grid_h, grid_w,
+                                            dk, dv, dir, chunk, dtype, stream);
 }
 
 gtr_status_t gtr_gla_fwd_timed(const void* q, const void* k, const void* v, const float* g,
