@@ -5,7 +5,7 @@
 // chunk outputs with the scores kept on chip and the output gate fused into
 // the epilogue), for 16-bit q/k/v/z, fp32 gates, dk = dv = 64, chunk C = 64.
 //
-// One CTA (128 threads) walks a segment of consecutive chunks of one (batch,
+// One CTA (256 threads) walks a segment of consecutive chunks of one (batch,
 // head) sequence and carries the dk x dv state S in fp32 registers.  For chunk
 // c with in-chunk inclusive log-gate cumsum G_j (per key dim), G_m = G at the
 // middle position and Gam = G at the last one:
@@ -25,9 +25,9 @@
 // staging area; no transpose kernel runs and reversed orders are just
 // reversed addresses.  The next chunk's q, k, v, g are fetched as soon as the
 // current chunk's operand tiles are built, and its z as soon as the current
-// epilogue is done, so the copies overlap the tensor-core work.  Two CTAs
-// share an SM (three for the summary kernel), which hides the latency of one
-// CTA's serial phases behind the others'.
+// epilogue is done, so the copies overlap the tensor-core work.  Two CTAs of
+// eight warps share an SM, which hides the latency of one CTA's serial phases
+// behind the other's.
 //
 // Tensor cores: tcgen05.mma kind::f16, M = 64, N = 64, K = 16 per
 // instruction, fp32 accumulators in tensor memory.  Every operand is a pair of
@@ -41,10 +41,11 @@
 // The state update uses k^ = diag(e^{Gam - G_m}) k~, a per-row factor of the
 // k~^T V accumulator, so one key tile serves both products (read K-major for
 // the scores and MN-major for the state).  An M = 64 accumulator puts row r in
-// TMEM lane 32*(r/16) + r%16, so warp w owns rows 16w..16w+15 in its lanes
-// 0-15.  The masked scores P go back to shared memory (K-major, two-term) for
-// P V.  The epilogue reads whole rows, so RMSNorm needs no cross-thread
-// reduction.
+// TMEM lane 32*(r/16) + r%16; warps w and w+4 read those 16 lanes of quadrant
+// w%4 with the 16x32bx2 shape, each thread taking 16 of the 64 columns, so the
+// row phases (S', P, epilogue, state) run four threads per row and combine row
+// maxima and sums with one shuffle and a two-warp named barrier.  The masked
+// scores P go back to shared memory (K-major, two-term) for P V.
 #pragma once
 #include "common.cuh"
 
@@ -53,7 +54,8 @@ namespace tc {
 
 constexpr int kC = 64;                 // chunk length
 constexpr int kD = 64;                 // head dim (dk = dv)
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
 constexpr float kSpanMax = 20.0f;      // nats of in-chunk decay the scaled operands take
 constexpr unsigned long long kWaitNs = 500ull * 1000 * 1000;   // bounded waits: 0.5 s
 
@@ -69,11 +71,11 @@ template <bool OUT> struct Layout {
   // fp16 tiles: V, key tile (hi, lo) [, q~ (hi, lo), S' (hi, lo)]
   static constexpr int kTiles = OUT ? 7 : 3;
   static constexpr int kMisc = kStage + kTiles * kTile;        // 1024-aligned
-  static constexpr int kMiscBytes = 5632;
+  static constexpr int kMiscBytes = 4608;
   static constexpr int kSmem = kMisc + kMiscBytes + 1024;      // + alignment slack
   static constexpr int kTmemCols = OUT ? 256 : 64;
   static constexpr int kColDS = OUT ? 192 : 0;
-  static constexpr int kBlocksPerSM = OUT ? 2 : 3;
+  static constexpr int kBlocksPerSM = 2;
 };
 
 // ------------------------------------------------------------------ PTX
@@ -91,14 +93,16 @@ __device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
 __device__ __forceinline__ void mbar_fence_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
+// One bounded probe of a phase; the thread may sleep in hardware for up to
+// 20 us while the phase is incomplete (fewer polling instructions).
 __device__ __forceinline__ uint32_t mbar_try(uint64_t* b, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(saddr(b)), "r"(parity)
+      : "r"(saddr(b)), "r"(parity), "r"(20000u)
       : "memory");
   return ok;
 }
@@ -158,6 +162,25 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
       : "r"(taddr));
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+// 16 lanes x 32 bit in two halves: thread t of warp w reads lane 32(w%4) + t%16
+// of the address's quadrant, columns [c, c+16) for t < 16 and [c+16, c+32) for
+// t >= 16 (c = the address's column).
+__device__ __forceinline__ void tmem_ld16x2(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], 16;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+// barrier over `count` threads (whole warps) on hardware barrier `id` (1..15)
+__device__ __forceinline__ void named_barrier(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
@@ -312,32 +335,46 @@ struct Params {
 
 struct Misc {                   // per-CTA scalars in shared memory; every array that is read
                                 // as float4 is 16-byte aligned
-  uint64_t mma[2];              // [0] scores committed, [1] every product of the chunk committed
+  uint64_t mma[2];              // [0] q~ S' and scores committed, [1] every product committed
   uint32_t tmem;                // tensor-memory base address
   int pad;
-  alignas(16) float smax[4];    // per-warp max |S| of the carried state
+  alignas(16) float smax[kWarps];   // per-warp max |S| of the carried state
   alignas(16) float kbound[2][2];   // per-warp max of the k~ [0] and k^ [1] bounds over key dims
   alignas(16) float Gm[kD];
   alignas(16) float Gam[kD];
   alignas(16) float aG[kD];
   alignas(16) float eK[kD];
   alignas(16) float wv[kD];
-  alignas(16) float lo[2][kD];
-  alignas(16) float hi[2][kD];
-  alignas(16) float half0[kD];
-  alignas(16) float kmx[2][kD];
-  alignas(16) float vmx[2][kD];
   alignas(16) float sev[kD];    // V column scales 2^e and 2^-e
   alignas(16) float iev[kD];
-  alignas(16) float ieq[kC];    // inverse row scales of q~ and P
-  alignas(16) float iep[kC];
+  // column statistics of the chunk: maxima of |k| and |v|, min and max of G
+  // (order-preserving int encodings, combined with shared-memory atomics)
+  alignas(16) int kmx[kD];
+  alignas(16) int vmx[kD];
+  alignas(16) int gmin[kD];
+  alignas(16) int gmax[kD];
+  union {
+    alignas(16) float part[4][kD];        // column pass: per-quarter gate sums
+    struct {
+      alignas(16) float ieq[kC];          // row phases: inverse row scales of q~ and P
+      alignas(16) float iep[kC];
+      alignas(16) float rowred[2][kC];    // row reductions across the two column halves
+    } r;
+  } u;
   alignas(16) long long rows[kC];   // token rows (b*T + t)*H + h of the chunk being fetched
 };
-static_assert(sizeof(Misc) <= 5632, "Misc must fit its reserved bytes");
+static_assert(sizeof(Misc) <= Layout<true>::kMiscBytes, "Misc must fit its reserved bytes");
 static_assert(offsetof(Misc, Gm) % 16 == 0 && offsetof(Misc, Gam) % 16 == 0 &&
                   offsetof(Misc, wv) % 16 == 0 && offsetof(Misc, sev) % 16 == 0 &&
                   offsetof(Misc, iev) % 16 == 0 && offsetof(Misc, eK) % 16 == 0,
               "float4 reads of Misc arrays need 16-byte alignment");
+
+// Order-preserving map of a float onto an int (for atomicMin / atomicMax).
+__device__ __forceinline__ int ord_enc(float f) {
+  const int i = __float_as_int(f);
+  return i >= 0 ? i : i ^ 0x7FFFFFFF;
+}
+__device__ __forceinline__ float ord_dec(int e) { return __int_as_float(e >= 0 ? e : e ^ 0x7FFFFFFF); }
 
 // Token rows of the chunk starting at scan position s0 (threads 0..ntok-1).
 __device__ __forceinline__ void chunk_rows(const Params& p, Misc& m, int b, int h, int d, int s0,
@@ -376,17 +413,26 @@ __device__ __forceinline__ void fetch_z(const Params& p, uint8_t* stg, const Mis
   cp_async_commit();
 }
 
-// Column pass over the chunk (two threads per column, 32 tokens each): the
+// Column pass over the chunk (four threads per column, 16 tokens each): the
 // in-place inclusive cumsum of the gate tile, and the column maxima of |k| and
 // |v|.  Then per column d: G_m, Gam, e^{Gam}, e^{Gam-G_m}, the V scales and
-// the bound of the k~ (output kernel) or k^ (summary kernel) column.  Returns
-// true (block-uniform) if the chunk needs the exact scores: its decay range
-// exceeds kSpanMax or some gate sum rises above zero.
-template <typename T, bool OUT>
+// the bounds of the k~ and k^ columns.  Returns true (block-uniform) if the
+// chunk needs the exact scores: its decay range exceeds kSpanMax or some gate
+// sum rises above zero.  m.kmx/vmx/gmin/gmax must hold their neutral values
+// (column_stats_reset) when it starts.
+__device__ __forceinline__ void column_stats_reset(Misc& m, int tid) {
+  if (tid < kD) {
+    m.kmx[tid] = 0;
+    m.vmx[tid] = 0;
+    m.gmin[tid] = ord_enc(0.0f);       // the running sum starts at 0 before the chunk
+    m.gmax[tid] = ord_enc(-3.0e38f);
+  }
+}
+template <typename T>
 __device__ __forceinline__ bool column_pass(float* G, const T* kst, const T* vst, Misc& m, int ntok,
                                             int tid) {
-  const int dd = tid & 63, half = tid >> 6;
-  const int j0 = half * 32, j1 = min(j0 + 32, ntok);
+  const int dd = tid & 63, qt = tid >> 6;
+  const int j0 = qt * 16, j1 = min(j0 + 16, ntok);
   float run = 0.f, lo = 3.0e38f, hi = -3.0e38f, km = 0.f, vm = 0.f;
 #pragma unroll 4
   for (int j = j0; j < j1; ++j) {
@@ -397,36 +443,36 @@ __device__ __forceinline__ bool column_pass(float* G, const T* kst, const T* vst
     km = fmaxf(km, fabsf(Elem<T>::to_f(kst[j * kD + dd])));
     vm = fmaxf(vm, fabsf(Elem<T>::to_f(vst[j * kD + dd])));
   }
-  if (half == 0) m.half0[dd] = run;
-  m.kmx[half][dd] = km;
-  m.vmx[half][dd] = vm;
+  m.u.part[qt][dd] = run;
+  atomicMax(&m.kmx[dd], __float_as_int(km));        // non-negative floats order as ints
+  atomicMax(&m.vmx[dd], __float_as_int(vm));
   __syncthreads();
-  if (half == 1 && j1 > j0) {
-    const float off = m.half0[dd];
+  float off = 0.f;
+  for (int q = 0; q < qt; ++q) off += m.u.part[q][dd];
+  if (qt > 0 && j1 > j0) {
 #pragma unroll 4
     for (int j = j0; j < j1; ++j) G[j * kD + dd] += off;
-    lo += off;
-    hi += off;
   }
-  m.lo[half][dd] = lo;
-  m.hi[half][dd] = hi;
+  if (j1 > j0) {
+    atomicMin(&m.gmin[dd], ord_enc(lo + off));
+    atomicMax(&m.gmax[dd], ord_enc(hi + off));
+  }
   __syncthreads();
   int irregular = 0;
   if (tid < kD) {
     const float gam = G[(ntok - 1) * kD + tid];
     const float gm = G[((ntok - 1) >> 1) * kD + tid];
-    const float mn = fminf(fminf(m.lo[0][tid], m.lo[1][tid]), 0.f);
-    const float mx = fmaxf(m.hi[0][tid], m.hi[1][tid]);
+    const float mn = ord_dec(m.gmin[tid]), mx = ord_dec(m.gmax[tid]);
+    const float km4 = __int_as_float(m.kmx[tid]), vm4 = __int_as_float(m.vmx[tid]);
     m.Gam[tid] = gam;
     m.Gm[tid] = gm;
     m.aG[tid] = expf(gam);
     m.eK[tid] = expf(gam - gm);
-    const int ev = scale_exp(fmaxf(m.vmx[0][tid], m.vmx[1][tid]));
+    const int ev = scale_exp(vm4);
     m.sev[tid] = pow2i(ev);
     m.iev[tid] = pow2i(-ev);
     // |k~_id| <= max_i |k_id| e^{G_m,d - min_i G_id};  |k^_id| <= max_i |k_id| e^{Gam_d - min_i G_id}
-    const float km = fmaxf(m.kmx[0][tid], m.kmx[1][tid]);
-    float kb0 = km * expf(gm - mn), kb1 = km * expf(gam - mn);
+    float kb0 = km4 * expf(gm - mn), kb1 = km4 * expf(gam - mn);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       kb0 = fmaxf(kb0, __shfl_xor_sync(0xffffffffu, kb0, o));
@@ -442,16 +488,20 @@ __device__ __forceinline__ bool column_pass(float* G, const T* kst, const T* vst
   return __syncthreads_or(irregular) != 0;
 }
 
-// Max |S| over the block's state rows into m.smax (one value per warp).
-__device__ __forceinline__ void state_max(const float* S, bool owner, Misc& m, int warp, int lane) {
-  float mx = 0.f;
-  if (owner) {
-#pragma unroll
-    for (int c = 0; c < kD; ++c) mx = fmaxf(mx, fabsf(S[c]));
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  if (lane == 0) m.smax[warp] = mx;
+// Max over the four threads that share an accumulator row: the other half of
+// the warp (lane ^ 16) and the same lanes of the partner warp (warp ^ 4),
+// through shared memory and a named barrier of those two warps.
+__device__ __forceinline__ float row_combine_max(float v, Misc& m, int row, int half, int qd, int lane) {
+  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+  if (lane < 16) m.u.r.rowred[half][row] = v;
+  named_barrier(1 + qd, 64);
+  return fmaxf(v, m.u.r.rowred[half ^ 1][row]);
+}
+__device__ __forceinline__ float row_combine_sum(float v, Misc& m, int row, int half, int qd, int lane) {
+  v += __shfl_xor_sync(0xffffffffu, v, 16);
+  if (lane < 16) m.u.r.rowred[half][row] = v;
+  named_barrier(1 + qd, 64);
+  return v + m.u.r.rowred[half ^ 1][row];
 }
 
 __device__ __forceinline__ float silu_fast(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
@@ -465,7 +515,7 @@ gla_tc(const Params p) {
   uint8_t* stg = sm;
   uint8_t* tiles = sm + L::kStage;
   uint8_t* VV = tiles;                       // V (MN-major B), one fp16 term
-  uint8_t* KTh = tiles + 1 * kTile;          // k~ (output) or k^ (summary), hi / lo
+  uint8_t* KTh = tiles + 1 * kTile;          // key tile: k~ or k^, hi / lo
   uint8_t* KTl = tiles + 2 * kTile;
   uint8_t* QTh = tiles + 3 * kTile;          // q~ hi / lo, then P (K-major A)   [OUT]
   uint8_t* QTl = tiles + 4 * kTile;
@@ -489,8 +539,14 @@ gla_tc(const Params p) {
     if (tid == 0) gtr_flag(d < 0 || d > 3 ? kStatusBadDir : kStatusBadShape);
     return;
   }
-  const bool owner = lane < 16;          // this thread holds accumulator row 16*warp + lane
-  const int row = warp * 16 + (lane & 15);   // that row: a query token, or a key dim of S
+  // Row phases: four threads per accumulator row.  Warp w reads TMEM lane
+  // quadrant qd = w % 4 (rows 16 qd .. 16 qd + 15) and column half w / 4; with
+  // the 16x32bx2 shape, lanes 0-15 take the first 16 columns of that half and
+  // lanes 16-31 the next 16, for the same 16 rows.
+  const int qd = warp & 3, half = warp >> 2;
+  const int row = qd * 16 + (lane & 15);
+  const int cbase = half * 32 + (lane >> 4) * 16;    // this thread's 16 columns
+  const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
 
   // first chunk's copies go out before anything else
   chunk_rows(p, m, b, h, d, c0 * kC, min(kC, p.T - c0 * kC), tid);
@@ -498,21 +554,29 @@ gla_tc(const Params p) {
   fetch_kvqg<T, OUT>(p, stg, m, min(kC, p.T - c0 * kC), tid);
   if (OUT) fetch_z(p, stg, m, min(kC, p.T - c0 * kC), tid);
 
-  // carried state: row `row` of S (key dim), 64 value columns
-  float S[kD];
-  if (OUT && owner) {
+  // carried state: S[row][cbase .. cbase + 15]
+  float S[16];
+  if (OUT) {
     const float4* src = reinterpret_cast<const float4*>(
-        p.wsS + (((size_t)bh * p.nseg + seg) * kD + row) * kD);
+        p.wsS + (((size_t)bh * p.nseg + seg) * kD + row) * kD + cbase);
 #pragma unroll
-    for (int c = 0; c < kD / 4; ++c) {
+    for (int c = 0; c < 4; ++c) {
       const float4 x = src[c];
       S[4 * c] = x.x; S[4 * c + 1] = x.y; S[4 * c + 2] = x.z; S[4 * c + 3] = x.w;
     }
   } else {
 #pragma unroll
-    for (int c = 0; c < kD; ++c) S[c] = 0.f;
+    for (int c = 0; c < 16; ++c) S[c] = 0.f;
   }
-  if (OUT) state_max(S, owner, m, warp, lane);
+  auto state_max = [&]() {
+    float mx = 0.f;
+#pragma unroll
+    for (int c = 0; c < 16; ++c) mx = fmaxf(mx, fabsf(S[c]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) m.smax[warp] = mx;
+  };
+  if (OUT) state_max();
   if (tid == 0) {
     mbar_init(&m.mma[0], 1);
     mbar_init(&m.mma[1], 1);
@@ -527,7 +591,6 @@ gla_tc(const Params p) {
   __syncthreads();
   tc_after_sync();
   const uint32_t tm = m.tmem;
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
 
   float lsum = 0.f;
   uint32_t ph0 = 0, ph1 = 0;
@@ -541,17 +604,19 @@ gla_tc(const Params p) {
     const int ntok1 = more ? min(kC, p.T - s1) : 0;
 
     cp_async_wait(OUT ? 1 : 0);          // k, v, g (, q) of this chunk are in
+    column_stats_reset(m, tid);
     __syncthreads();
-    const bool exact = column_pass<T, OUT>(G, kst, vst, m, ntok, tid) && OUT;
+    const bool exact = column_pass<T>(G, kst, vst, m, ntok, tid) && OUT;
 
     // ---- operand tiles; rows beyond ntok are zero.  Items: (row r, 4 columns
     // cg..cg+3); a half warp covers one row, which makes per-row maxima cheap.
-    // the key tile holds k~ = k e^{G_m - G} for a regular output chunk, else k^ = k e^{Gam - G}
+    // The key tile holds k~ = k e^{G_m - G} for a regular output chunk, else
+    // k^ = k e^{Gam - G}.
     const bool tilde = OUT && !exact;
     const int ekt = scale_exp(fmaxf(m.kbound[tilde ? 0 : 1][0], m.kbound[tilde ? 0 : 1][1]));
     const float skt = pow2i(ekt);
 #pragma unroll 2
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < (kC * kD / 4) / kThreads; ++u) {
       const int item = u * kThreads + tid;
       const int r = item >> 4, cg = (item & 15) * 4;
       const bool valid = r < ntok;
@@ -567,7 +632,6 @@ gla_tc(const Params p) {
         const float4 sv = *reinterpret_cast<const float4*>(&m.sev[cg]);
         *reinterpret_cast<uint2*>(VV + off) = half4(vv.x * sv.x, vv.y * sv.y, vv.z * sv.z, vv.w * sv.w);
       }
-      // k~ = k e^{G_m - G} or k^ = k e^{Gam - G}, tile-scaled
       const float4 gr = *reinterpret_cast<const float4*>(tilde ? &m.Gm[cg] : &m.Gam[cg]);
       put2(KTh, KTl, off, kk.x * __expf(gr.x - gg.x) * skt, kk.y * __expf(gr.y - gg.y) * skt,
            kk.z * __expf(gr.z - gg.z) * skt, kk.w * __expf(gr.w - gg.w) * skt);
@@ -583,21 +647,21 @@ gla_tc(const Params p) {
         const int eq = scale_exp(half_warp_max(amax4(q0, q1, q2, q3)));
         const float s = pow2i(eq);
         put2(QTh, QTl, off, q0 * s, q1 * s, q2 * s, q3 * s);
-        if (cg == 0) m.ieq[r] = pow2i(-eq);
+        if (cg == 0) m.u.r.ieq[r] = pow2i(-eq);
       }
     }
     // S' = e^{G_m} S (S itself for an exact chunk), tile-scaled from max |S|
     float inv_es = 1.f;
     if (OUT) {
-      const float smx = fmaxf(fmaxf(m.smax[0], m.smax[1]), fmaxf(m.smax[2], m.smax[3]));
+      float smx = 0.f;
+#pragma unroll
+      for (int w8 = 0; w8 < kWarps; ++w8) smx = fmaxf(smx, m.smax[w8]);
       const int es = scale_exp(smx);
       inv_es = pow2i(-es);
-      if (owner) {
-        const float sc = (exact ? 1.0f : __expf(m.Gm[row])) * pow2i(es);
+      const float sc = (exact ? 1.0f : __expf(m.Gm[row])) * pow2i(es);
 #pragma unroll
-        for (int c = 0; c < kD; c += 4)
-          put2(SPh, SPl, sw16(row, c), sc * S[c], sc * S[c + 1], sc * S[c + 2], sc * S[c + 3]);
-      }
+      for (int c = 0; c < 16; c += 4)
+        put2(SPh, SPl, sw16(row, cbase + c), sc * S[c], sc * S[c + 1], sc * S[c + 2], sc * S[c + 3]);
     }
     if (more && !exact) chunk_rows(p, m, b, h, d, s1, ntok1, tid);
     fence_async_smem();
@@ -622,48 +686,42 @@ gla_tc(const Params p) {
     }
 
     if (OUT) {
-      // ---- masked scores P (rows = queries j, columns = keys i), row-scaled, into QT
+      failed |= !mbar_wait(&m.mma[0], ph0);
+      ph0 ^= 1;
+      tc_after_sync();
       if (!exact) {
-        const bool okm = mbar_wait(&m.mma[0], ph0);
-        ph0 ^= 1;
-        failed |= !okm;
-        tc_after_sync();
-        float sc[kC];
-#pragma unroll
-        for (int cb = 0; cb < 4; ++cb) tmem_ld16(tm + lane_base + 64 + cb * 16, sc + cb * 16);
+        // ---- masked scores P (rows = queries j, columns = keys i), row-scaled, into QT
+        float sc[16];
+        tmem_ld16x2(tm + lane_base + 64 + half * 32, sc);
         tmem_ld_wait();
-        if (owner) {
-          const float f = m.ieq[row] * pow2i(-ekt);
-          float mx = 0.f;
+        const float f = m.u.r.ieq[row] * pow2i(-ekt);
+        float mx = 0.f;
 #pragma unroll
-          for (int i = 0; i < kC; ++i) {
-            sc[i] = (i <= row && row < ntok) ? sc[i] * f : 0.f;
-            mx = fmaxf(mx, fabsf(sc[i]));
-          }
-          const int ep = scale_exp(mx);
-          const float s = pow2i(ep);
-          m.iep[row] = pow2i(-ep);
-#pragma unroll
-          for (int i = 0; i < kC; i += 4)
-            put2(QTh, QTl, sw16(row, i), sc[i] * s, sc[i + 1] * s, sc[i + 2] * s, sc[i + 3] * s);
+        for (int c = 0; c < 16; ++c) {
+          const int i = cbase + c;
+          sc[c] = (i <= row && row < ntok) ? sc[c] * f : 0.f;
+          mx = fmaxf(mx, fabsf(sc[c]));
         }
-      } else {
-        // exact scores on CUDA cores: P_ji = sum_d q_jd k_id e^{G_jd - G_id}, two threads per
-        // row; q~ must stay intact until q~ S' is done
-        if (tid == 0) atomicAdd(&g_gtr_exact_chunks, 1ull);
-        const bool okm = mbar_wait(&m.mma[0], ph0);
-        ph0 ^= 1;
-        failed |= !okm;
-        const int j = tid >> 1, ib = (tid & 1) * 32;
-        float acc[32];
+        mx = row_combine_max(mx, m, row, half, qd, lane);
+        const int ep = scale_exp(mx);
+        const float s = pow2i(ep);
+        if (lane < 16 && half == 0) m.u.r.iep[row] = pow2i(-ep);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) acc[e] = 0.f;
+        for (int c = 0; c < 16; c += 4)
+          put2(QTh, QTl, sw16(row, cbase + c), sc[c] * s, sc[c + 1] * s, sc[c + 2] * s, sc[c + 3] * s);
+      } else {
+        // exact scores on CUDA cores: P_ji = sum_d q_jd k_id e^{G_jd - G_id}; four threads per row
+        if (tid == 0) atomicAdd(&g_gtr_exact_chunks, 1ull);
+        const int j = tid >> 2, ib = (tid & 3) * 16;
+        float acc[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) acc[e] = 0.f;
         if (j < ntok) {
           for (int dd = 0; dd < kD; ++dd) {
             const float qj = Elem<T>::to_f(qst[j * kD + dd]);
             const float gj = G[j * kD + dd];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
+            for (int e = 0; e < 16; ++e) {
               const int i = ib + e;
               if (i <= j)
                 acc[e] = fmaf(qj * Elem<T>::to_f(kst[i * kD + dd]), expf(gj - G[i * kD + dd]), acc[e]);
@@ -672,13 +730,14 @@ gla_tc(const Params p) {
         }
         float mx = 0.f;
 #pragma unroll
-        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, fabsf(acc[e]));
+        for (int e = 0; e < 16; ++e) mx = fmaxf(mx, fabsf(acc[e]));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
         const int ep = scale_exp(mx);
         const float s = pow2i(ep);
-        if ((tid & 1) == 0) m.iep[j] = pow2i(-ep);
+        if ((tid & 3) == 0) m.u.r.iep[j] = pow2i(-ep);
 #pragma unroll
-        for (int e = 0; e < 32; e += 4)
+        for (int e = 0; e < 16; e += 4)
           put2(QTh, QTl, sw16(j, ib + e), acc[e] * s, acc[e + 1] * s, acc[e + 2] * s, acc[e + 3] * s);
         if (more) chunk_rows(p, m, b, h, d, s1, ntok1, tid);
       }
@@ -700,34 +759,30 @@ gla_tc(const Params p) {
 
     if (OUT) {
       // ---- epilogue: o_j = q~_j S' + P_j V, then o_j / sqrt(mean o_j^2 + eps) * w * SiLU(z_j)
-      float o[kD];
+      float o[16], pv[16];
+      tmem_ld16x2(tm + lane_base + 0 + half * 32, o);
+      tmem_ld16x2(tm + lane_base + 128 + half * 32, pv);
+      tmem_ld_wait();
+      const float a = m.u.r.ieq[row] * inv_es, bsc = m.u.r.iep[row];
       float ss = 0.f;
-      const float a = m.ieq[row] * inv_es, bsc = m.iep[row];
 #pragma unroll
-      for (int cb = 0; cb < 4; ++cb) {
-        float pv[16];
-        tmem_ld16(tm + lane_base + cb * 16, o + cb * 16);
-        tmem_ld16(tm + lane_base + 128 + cb * 16, pv);
-        tmem_ld_wait();
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int cc = cb * 16 + c;
-          o[cc] = o[cc] * a + pv[c] * bsc * m.iev[cc];
-          ss = fmaf(o[cc], o[cc], ss);
-        }
+      for (int c = 0; c < 16; ++c) {
+        o[c] = o[c] * a + pv[c] * bsc * m.iev[cbase + c];
+        ss = fmaf(o[c], o[c], ss);
       }
-      if (owner && row < ntok) {
+      ss = row_combine_sum(ss, m, row, half, qd, lane);
+      if (row < ntok) {
         const float inv = rsqrtf(ss * (1.0f / kD) + kRmsEps);
-        const T* zr = zst + row * kD;
+        const T* zr = zst + row * kD + cbase;
         const int t = scan_to_grid(d, s0 + row, p.T, p.gh, p.gw);
-        T* dst = reinterpret_cast<T*>(p.out) + (((size_t)b * p.T + t) * p.H + h) * kD;
+        T* dst = reinterpret_cast<T*>(p.out) + (((size_t)b * p.T + t) * p.H + h) * kD + cbase;
 #pragma unroll
-        for (int c = 0; c < kD; c += 8) {
+        for (int c = 0; c < 16; c += 8) {
           const uint4 zz = *reinterpret_cast<const uint4*>(zr + c);
           const float4 z0 = Vec4<T>::from_bits(make_uint2(zz.x, zz.y));
           const float4 z1 = Vec4<T>::from_bits(make_uint2(zz.z, zz.w));
-          const float4 w0 = *reinterpret_cast<const float4*>(&m.wv[c]);
-          const float4 w1 = *reinterpret_cast<const float4*>(&m.wv[c + 4]);
+          const float4 w0 = *reinterpret_cast<const float4*>(&m.wv[cbase + c]);
+          const float4 w1 = *reinterpret_cast<const float4*>(&m.wv[cbase + c + 4]);
           const uint2 lo = pack4<T>(o[c + 0] * inv * w0.x * silu_fast(z0.x), o[c + 1] * inv * w0.y * silu_fast(z0.y),
                                     o[c + 2] * inv * w0.z * silu_fast(z0.z), o[c + 3] * inv * w0.w * silu_fast(z0.w));
           const uint2 hi = pack4<T>(o[c + 4] * inv * w1.x * silu_fast(z1.x), o[c + 5] * inv * w1.y * silu_fast(z1.y),
@@ -737,22 +792,16 @@ gla_tc(const Params p) {
       }
     }
 
-    // ---- state: S <- e^{Gam} S + diag(e^{Gam - G_m}) k~^T V   (summary: + k^^T V), fp32
+    // ---- state: S <- e^{Gam} S + diag(e^{Gam - G_m}) k~^T V   (or + k^^T V), fp32
     {
+      float ds[16];
+      tmem_ld16x2(tm + lane_base + L::kColDS + half * 32, ds);
+      tmem_ld_wait();
       const float rs = (tilde ? m.eK[row] : 1.0f) * pow2i(-ekt);
       const float a = m.aG[row];
 #pragma unroll
-      for (int cb = 0; cb < 4; ++cb) {
-        float ds[16];
-        tmem_ld16(tm + lane_base + L::kColDS + cb * 16, ds);
-        tmem_ld_wait();
-        if (owner) {
-#pragma unroll
-          for (int c = 0; c < 16; ++c)
-            S[cb * 16 + c] = fmaf(a, S[cb * 16 + c], ds[c] * rs * m.iev[cb * 16 + c]);
-        }
-      }
-      if (OUT) state_max(S, owner, m, warp, lane);
+      for (int c = 0; c < 16; ++c) S[c] = fmaf(a, S[c], ds[c] * rs * m.iev[cbase + c]);
+      if (OUT) state_max();
     }
     if (!OUT && tid < kD) lsum += m.Gam[tid];
     tc_before_sync();
@@ -764,12 +813,9 @@ gla_tc(const Params p) {
   if (failed) {
     if (tid == 0) gtr_flag(kStatusMbarTimeout);
   } else if (!OUT) {
-    if (owner) {
-      float4* dst = reinterpret_cast<float4*>(p.wsS + (((size_t)bh * p.nseg + seg) * kD + row) * kD);
+    float4* dst = reinterpret_cast<float4*>(p.wsS + (((size_t)bh * p.nseg + seg) * kD + row) * kD + cbase);
 #pragma unroll
-      for (int c = 0; c < kD / 4; ++c)
-        dst[c] = make_float4(S[4 * c], S[4 * c + 1], S[4 * c + 2], S[4 * c + 3]);
-    }
+    for (int c = 0; c < 4; ++c) dst[c] = make_float4(S[4 * c], S[4 * c + 1], S[4 * c + 2], S[4 * c + 3]);
     if (tid < kD) p.wsL[((size_t)bh * p.nseg + seg) * kD + tid] = lsum;
   }
   tc_before_sync();
