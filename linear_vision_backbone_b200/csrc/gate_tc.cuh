@@ -1,0 +1,319 @@
+// gate_tc.cuh -- K1 on tensor cores: the low-rank forget-gate projection
+//   g[n, j] = logsigmoid(sum_r (x[n,:] . W_down[:, r]) W_up[r, j] + b[j]) / tau
+// (GTR article, 方法详解 §1: a light low-rank projection with a temperature).
+//
+// One CTA (256 threads) per 128 tokens:
+//   * the x tile (128 rows x d_model, 16-bit, exact) arrives by 16-byte
+//     cp.async into a 128B-swizzled K-major tile;
+//   * W_down (rank 16) is split into terms of x's own type with a
+//     power-of-two scale per rank (fp16: hi + lo, bf16: hi + mid + lo), each
+//     thread holding its float4s in registers (all loads in flight at once),
+//     so x W_down is exact up to
+//     ~22-24 significant bits: low = sum_t x W_t (tcgen05.mma kind::f16,
+//     M = 128, N = 16, fp32 accumulators in TMEM);
+//   * low (fp32, per-row scaled) and W_up (per-column scaled) become two-term
+//     fp16 operands and u = low W_up is taken as hi*hi + hi*lo + lo*hi
+//     (M = 128, N = 64 per instruction);
+//   * the epilogue reads u from TMEM (thread = token row, warps 0-3 and 4-7
+//     on the two column halves), adds the bias and stores logsigmoid(u)/tau.
+// The scales are exact powers of two and are undone on the fp32 accumulators;
+// they run along M or N only, so they factor out of every sum.
+#pragma once
+#include <type_traits>
+
+#include "common.cuh"
+#include "gate_kernels.cuh"
+#include "tc_kernels.cuh"
+
+namespace gtr {
+namespace gate_tc {
+
+using tc::saddr;
+using tc::scale_exp;
+using tc::pow2i;
+
+constexpr int kM = 128;               // tokens per CTA
+constexpr int kThreads = 256;
+constexpr int kMaxDm = 384;           // d_model: multiple of 64, <= 384
+constexpr int kMaxHD = 448;           // H*dk: multiple of 64, <= 448
+constexpr int kRank = 16;             // the projection's N (rank <= 16, zero-padded)
+
+struct Layout {
+  static constexpr int kX = kM * kMaxDm * 2;               // x tile: 96 KB
+  static constexpr int kWd = kRank * kMaxDm * 2;           // one W_down term: 12 KB
+  static constexpr int kLow = kM * 128;                    // one low term (K = 16 of a 64-wide tile): 16 KB
+  static constexpr int kWu = kRank * kMaxHD * 2;           // one W_up term: 14 KB
+  static constexpr int kOffX = 0;
+  static constexpr int kOffWd = kOffX + kX;                // 3 terms
+  static constexpr int kOffLow = kOffWd + 3 * kWd;         // 2 terms
+  static constexpr int kOffWu = kOffLow + 2 * kLow;        // 2 terms
+  static constexpr int kOffMisc = kOffWu + 2 * kWu;
+  static constexpr int kMiscBytes = 5120;
+  static constexpr int kSmem = kOffMisc + kMiscBytes + 1024;
+};
+
+struct Misc {
+  uint64_t mma[2];
+  uint32_t tmem;
+  int pad;
+  alignas(16) float wd_s[kRank];     // W_down rank scales 2^e (and their inverses)
+  alignas(16) float wd_i[kRank];
+  alignas(16) float wu_i[kMaxHD];    // inverse W_up column scales
+  alignas(16) float low_i[kM];       // inverse row scales of low
+  alignas(16) float wd_part[kThreads / 32][kRank];   // per-warp |W_down| maxima per rank
+};
+static_assert(sizeof(Misc) <= Layout::kMiscBytes, "Misc must fit its reserved bytes");
+
+// K-major 16-bit tile (rows x K), 128B-swizzled atoms of 8 rows x 64 elements;
+// atom columns (64 K-elements) `rows`*128 bytes apart.
+__device__ __forceinline__ uint32_t swk(int r, int c, int rows) {
+  return (uint32_t)((c >> 6) * (rows * 128) + (r >> 3) * 1024 + (r & 7) * 128 +
+                    ((((c & 63) >> 3) ^ (r & 7)) << 4) + (c & 7) * 2);
+}
+// MN-major 16-bit tile (K rows x N), atoms of 8 K-rows x 64 N-elements; N atoms
+// `krows`*128 bytes apart.
+__device__ __forceinline__ uint32_t swmn(int k, int n, int krows) {
+  return (uint32_t)((n >> 6) * (krows * 128) + (k >> 3) * 1024 + (k & 7) * 128 +
+                    ((((n & 63) >> 3) ^ (k & 7)) << 4) + (n & 7) * 2);
+}
+__host__ __device__ constexpr uint32_t idesc16(int M, int N, int a_mn, int b_mn, int bf16) {
+  return (1u << 4) | ((uint32_t)bf16 << 7) | ((uint32_t)bf16 << 10) | ((uint32_t)a_mn << 15) |
+         ((uint32_t)b_mn << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+__device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr(dst)), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+
+template <typename T> struct Store16;
+template <> struct Store16<__half> {
+  static __device__ __forceinline__ void put(uint8_t* p, float v) { *reinterpret_cast<__half*>(p) = __float2half_rn(v); }
+  static __device__ __forceinline__ float back(float v) { return __half2float(__float2half_rn(v)); }
+};
+template <> struct Store16<__nv_bfloat16> {
+  static __device__ __forceinline__ void put(uint8_t* p, float v) {
+    *reinterpret_cast<__nv_bfloat16*>(p) = __float2bfloat16_rn(v);
+  }
+  static __device__ __forceinline__ float back(float v) { return __bfloat162float(__float2bfloat16_rn(v)); }
+};
+
+template <typename TX>
+__global__ void __launch_bounds__(kThreads, 1)
+gate_proj_tc(const TX* __restrict__ x, const float* __restrict__ w_down, const float* __restrict__ w_up,
+             const float* __restrict__ bias, float* __restrict__ g, long long N, int dm, int rank,
+             int HD, float inv_tau) {
+  constexpr bool kBf16 = std::is_same<TX, __nv_bfloat16>::value;
+  constexpr int kTerms = kBf16 ? 3 : 2;   // W_down terms in x's type
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* tX = sm + Layout::kOffX;
+  uint8_t* tWd = sm + Layout::kOffWd;
+  uint8_t* tLow = sm + Layout::kOffLow;
+  uint8_t* tWu = sm + Layout::kOffWu;
+  Misc& m = *reinterpret_cast<Misc*>(sm + Layout::kOffMisc);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long tok0 = (long long)blockIdx.x * kM;
+  const int ntok = (int)min((long long)kM, N - tok0);
+
+  // ---- x tile: 16-byte pieces into the swizzled K-major tile (rows beyond ntok zero-filled)
+  const int pieces = dm / 8;                      // 16-byte pieces per token row
+  for (int o = tid; o < kM * pieces; o += kThreads) {
+    const int r = o / pieces, c = (o - r * pieces) * 8;
+    const bool valid = r < ntok;
+    const TX* src = valid ? x + (tok0 + r) * dm + c : x;
+    cp_async16_zfill(tX + swk(r, c, kM), src, valid);
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+
+  if (tid == 0) {
+    tc::mbar_init(&m.mma[0], 1);
+    tc::mbar_init(&m.mma[1], 1);
+    tc::mbar_fence_init();
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(&m.tmem, 512);
+    tc::tmem_relinquish();
+  }
+  // ---- W_down [dm][16]: thread t holds the float4s t, t + 256, ... (ranks 4(t%4)..+3 of rows
+  // (t + 256i)/4), all loads in flight at once; the rank maxima reduce over the lanes with the
+  // same t%4 and then over the 8 warps.
+  constexpr int kWdVec = kMaxDm * kRank / 4 / kThreads;     // float4s per thread at most (6)
+  const int nwd = dm * kRank / 4;
+  float4 wd[kWdVec];
+  float4 wmx = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int i = 0; i < kWdVec; ++i) {
+    const int idx = tid + i * kThreads;
+    wd[i] = idx < nwd ? __ldg(reinterpret_cast<const float4*>(w_down) + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+    wmx = make_float4(fmaxf(wmx.x, fabsf(wd[i].x)), fmaxf(wmx.y, fabsf(wd[i].y)),
+                      fmaxf(wmx.z, fabsf(wd[i].z)), fmaxf(wmx.w, fabsf(wd[i].w)));
+  }
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    wmx.x = fmaxf(wmx.x, __shfl_xor_sync(0xffffffffu, wmx.x, o));
+    wmx.y = fmaxf(wmx.y, __shfl_xor_sync(0xffffffffu, wmx.y, o));
+    wmx.z = fmaxf(wmx.z, __shfl_xor_sync(0xffffffffu, wmx.z, o));
+    wmx.w = fmaxf(wmx.w, __shfl_xor_sync(0xffffffffu, wmx.w, o));
+  }
+  if (lane < 4) *reinterpret_cast<float4*>(&m.wd_part[warp][lane * 4]) = wmx;
+  // ---- W_up [16][HD]: thread t < HD/4 holds column quad t of all 16 ranks
+  const int nq = HD / 4;
+  float4 wu[kRank];
+  if (tid < nq) {
+#pragma unroll
+    for (int k = 0; k < kRank; ++k) wu[k] = __ldg(reinterpret_cast<const float4*>(w_up + (size_t)k * HD) + tid);
+  }
+  __syncthreads();
+  if (tid < kRank) {
+    float mx = 0.f;
+#pragma unroll
+    for (int w8 = 0; w8 < kThreads / 32; ++w8) mx = fmaxf(mx, m.wd_part[w8][tid]);
+    const int e = scale_exp(mx);
+    m.wd_s[tid] = pow2i(e);
+    m.wd_i[tid] = pow2i(-e);
+  }
+  if (tid < nq) {
+    float4 cm = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < kRank; ++k)
+      cm = make_float4(fmaxf(cm.x, fabsf(wu[k].x)), fmaxf(cm.y, fabsf(wu[k].y)),
+                       fmaxf(cm.z, fabsf(wu[k].z)), fmaxf(cm.w, fabsf(wu[k].w)));
+    const int e0 = scale_exp(cm.x), e1 = scale_exp(cm.y), e2 = scale_exp(cm.z), e3 = scale_exp(cm.w);
+    *reinterpret_cast<float4*>(&m.wu_i[4 * tid]) = make_float4(pow2i(-e0), pow2i(-e1), pow2i(-e2), pow2i(-e3));
+    const float s0 = pow2i(e0), s1 = pow2i(e1), s2 = pow2i(e2), s3 = pow2i(e3);
+    // W_up terms (B of stage 2, MN-major: rows = rank (K), columns = H*dk), fp16 hi + lo
+#pragma unroll
+    for (int k = 0; k < kRank; ++k) {
+      const uint32_t off = swmn(k, 4 * tid, kRank);
+      tc::put2(tWu, tWu + Layout::kWu, off, wu[k].x * s0, wu[k].y * s1, wu[k].z * s2, wu[k].w * s3);
+    }
+  }
+  __syncthreads();
+  // W_down^T terms (B of stage 1, K-major: rows = rank, columns = d_model)
+  {
+    const float4 sc = *reinterpret_cast<const float4*>(&m.wd_s[(tid & 3) * 4]);
+#pragma unroll
+    for (int i = 0; i < kWdVec; ++i) {
+      const int idx = tid + i * kThreads;
+      if (idx < nwd) {
+        const int c = idx >> 2, n0 = (idx & 3) * 4;
+        float w4[4] = {wd[i].x * sc.x, wd[i].y * sc.y, wd[i].z * sc.z, wd[i].w * sc.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t off = swk(n0 + e, c, kRank);
+          float w = w4[e];
+#pragma unroll
+          for (int t = 0; t < kTerms; ++t) {
+            Store16<TX>::put(tWd + t * Layout::kWd + off, w);
+            w -= Store16<TX>::back(w);
+          }
+        }
+      }
+    }
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  tc::fence_async_smem();
+  tc::tc_before_sync();
+  __syncthreads();
+  tc::tc_after_sync();
+  const uint32_t tm = m.tmem;
+
+  // ---- stage 1: low = x W_down  (TMEM columns 0..15)
+  if (tid == 0) {
+    const uint32_t id = idesc16(kM, kRank, 0, 0, kBf16 ? 1 : 0);
+    const int ksteps = dm / 16;
+    for (int t = 0; t < kTerms; ++t)
+      for (int s = 0; s < ksteps; ++s) {
+        const uint64_t a = tc::sdesc(saddr(tX) + (s >> 2) * (kM * 128) + (s & 3) * 32, 16, 1024);
+        const uint64_t b = tc::sdesc(saddr(tWd) + t * Layout::kWd + (s >> 2) * (kRank * 128) + (s & 3) * 32, 16, 1024);
+        tc::mma_f16(tm + 0, a, b, id, (t > 0 || s > 0) ? 1u : 0u);
+      }
+    tc::mma_commit(&m.mma[0]);
+  }
+  bool ok = tc::mbar_wait(&m.mma[0], 0);
+  tc::tc_after_sync();
+  // low row r (warps 0-3, thread = row) -> per-row scaled two-term fp16 A tile (K = 16)
+  if (warp < 4) {
+    float lw[16];
+    tc::tmem_ld16(tm + ((uint32_t)(warp * 32) << 16) + 0, lw);
+    tc::tmem_ld_wait();
+    const int r = warp * 32 + lane;
+    float mx = 0.f;
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      lw[c] *= m.wd_i[c];
+      mx = fmaxf(mx, fabsf(lw[c]));
+    }
+    const int e = scale_exp(mx);
+    const float s = pow2i(e);
+    m.low_i[r] = pow2i(-e);
+#pragma unroll
+    for (int c = 0; c < 16; c += 4)
+      tc::put2(tLow, tLow + Layout::kLow, swk(r, c, kM), lw[c] * s, lw[c + 1] * s, lw[c + 2] * s,
+               lw[c + 3] * s);
+  }
+  tc::fence_async_smem();
+  tc::tc_before_sync();
+  __syncthreads();
+  tc::tc_after_sync();
+
+  // ---- stage 2: u = low W_up  (TMEM columns 64 .. 64 + HD), 64 columns per instruction
+  if (tid == 0) {
+    const uint32_t id = idesc16(kM, 64, 0, 1, 0);
+    const uint64_t al = tc::sdesc(saddr(tLow), 16, 1024), all = tc::sdesc(saddr(tLow) + Layout::kLow, 16, 1024);
+    for (int nb = 0; nb < HD / 64; ++nb) {
+      const uint32_t ub = saddr(tWu) + nb * (kRank * 128);
+      const uint64_t bh = tc::sdesc(ub, kRank * 128, 1024), bl = tc::sdesc(ub + Layout::kWu, kRank * 128, 1024);
+      tc::mma_f16(tm + 64 + nb * 64, al, bh, id, 0u);
+      tc::mma_f16(tm + 64 + nb * 64, al, bl, id, 1u);
+      tc::mma_f16(tm + 64 + nb * 64, all, bh, id, 1u);
+    }
+    tc::mma_commit(&m.mma[1]);
+  }
+  ok &= tc::mbar_wait(&m.mma[1], 0);
+  tc::tc_after_sync();
+  if (!ok && tid == 0) gtr_flag(kStatusMbarTimeout);
+
+  // ---- epilogue: thread = token row (lane quadrant warp % 4), warps w and w + 4 take the
+  // two halves of the columns; g = logsigmoid(u + b) / tau
+  {
+    const int r = (warp & 3) * 32 + lane;
+    const int half = warp >> 2, ncol = HD / 2, c0 = half * ncol;
+    const float ri = m.low_i[r];
+    float* grow = g + (tok0 + r) * HD;
+    for (int cb = 0; cb < ncol; cb += 16) {
+      float u[16];
+      tc::tmem_ld16(tm + ((uint32_t)((warp & 3) * 32) << 16) + 64 + c0 + cb, u);
+      tc::tmem_ld_wait();
+      if (r < ntok) {
+#pragma unroll
+        for (int c = 0; c < 16; c += 4) {
+          const int j = c0 + cb + c;
+          const float4 bb = bias ? *reinterpret_cast<const float4*>(bias + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float4 ci = *reinterpret_cast<const float4*>(&m.wu_i[j]);
+          *reinterpret_cast<float4*>(grow + j) = make_float4(
+              logsigmoid_fast(fmaf(u[c + 0] * ri, ci.x, bb.x)) * inv_tau,
+              logsigmoid_fast(fmaf(u[c + 1] * ri, ci.y, bb.y)) * inv_tau,
+              logsigmoid_fast(fmaf(u[c + 2] * ri, ci.z, bb.z)) * inv_tau,
+              logsigmoid_fast(fmaf(u[c + 3] * ri, ci.w, bb.w)) * inv_tau);
+        }
+      }
+    }
+  }
+  tc::tc_before_sync();
+  __syncthreads();
+  tc::tc_after_sync();
+  if (warp == 0) tc::tmem_dealloc(tm, 512);
+}
+
+}  // namespace gate_tc
+
+// Shapes the tensor-core gate kernel takes: 16-bit x, d_model a multiple of 64
+// up to 384, rank 16, H*dk a multiple of 64 up to 448.
+inline bool gate_tc_supported(int x_dtype, int dm, int rank, int HD) {
+  return (x_dtype == kF16 || x_dtype == kBF16) && dm % 64 == 0 && dm <= gate_tc::kMaxDm &&
+         rank == gate_tc::kRank && HD % 64 == 0 && HD <= gate_tc::kMaxHD;
+}
+
+}  // namespace gtr

@@ -14,6 +14,7 @@
 #include "simt_kernels.cuh"
 #include "scan_kernel.cuh"
 #include "tc_kernels.cuh"
+#include "gate_tc.cuh"
 
 namespace {
 
@@ -360,6 +361,28 @@ gtr_status_t gtr_gate_fwd(const void* x, int x_dtype, const float* w_down, const
     return GTR_ERR_ALIGNMENT;
   const int HD = H * dk;
   cudaStream_t st = (cudaStream_t)stream;
+  if (gate_tc_supported(x_dtype, d_model, rank, HD) && (!bias || aligned16(bias))) {
+    // tensor-core kernel: one CTA per 128 tokens
+    const long long blocks = (N + gate_tc::kM - 1) / gate_tc::kM;
+    if (blocks > 0x7fffffffLL) return GTR_ERR_INVALID_ARG;
+    int dev;
+    if (int rc = current_device(&dev)) return (gtr_status_t)rc;
+    const float inv_tau = 1.0f / tau;
+    if (x_dtype == GTR_F16) {
+      static bool done[kMaxDevices];
+      if (int rc = ensure_smem(gate_tc::gate_proj_tc<__half>, gate_tc::Layout::kSmem, done, dev))
+        return (gtr_status_t)rc;
+      gate_tc::gate_proj_tc<__half><<<(unsigned)blocks, gate_tc::kThreads, gate_tc::Layout::kSmem, st>>>(
+          (const __half*)x, w_down, w_up, bias, g_out, N, d_model, rank, HD, inv_tau);
+    } else {
+      static bool done[kMaxDevices];
+      if (int rc = ensure_smem(gate_tc::gate_proj_tc<__nv_bfloat16>, gate_tc::Layout::kSmem, done, dev))
+        return (gtr_status_t)rc;
+      gate_tc::gate_proj_tc<__nv_bfloat16><<<(unsigned)blocks, gate_tc::kThreads, gate_tc::Layout::kSmem, st>>>(
+          (const __nv_bfloat16*)x, w_down, w_up, bias, g_out, N, d_model, rank, HD, inv_tau);
+    }
+    return (gtr_status_t)launch_status();
+  }
   if (rank <= 16 && HD % 4 == 0 && HD <= kGate2MaxHD && (!bias || aligned16(bias))) {
     // register-tiled kernel: one block per 64 tokens
     const long long blocks = (N + kGate2Tok - 1) / kGate2Tok;

@@ -10,15 +10,16 @@
 // where dS_s is the state segment s produces from a zero start and L_s its
 // summed log-gate.  The result overwrites dS in place (exclusive form: the
 // state each segment starts from) or, with `inclusive`, the state each segment
-// ends with.  Loads of a group of segments are issued before their stores, so
-// the dependent chain is only the FMA.
+// ends with.  The loads of a group of up to 32 segments are all issued before
+// any store, so one memory latency covers the whole group and the dependent
+// chain is only the FMA; blocks of 128 threads spread the pass over the SMs.
 #pragma once
 #include "common.cuh"
 
 namespace gtr {
 
-constexpr int kScanThreads = 256;
-constexpr int kScanGroup = 8;
+constexpr int kScanThreads = 128;
+constexpr int kScanGroup = 32;
 
 __global__ void __launch_bounds__(kScanThreads)
 gla_state_scan(float* __restrict__ wsS, const float* __restrict__ wsL, long long total, int nseg,

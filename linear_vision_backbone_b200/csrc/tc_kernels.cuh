@@ -43,10 +43,13 @@
 // the scores and MN-major for the state).  An M = 64 accumulator puts row r in
 // TMEM lane 32*(r/16) + r%16; warps w and w+4 read those 16 lanes of quadrant
 // w%4 with the 16x32bx2 shape, each thread taking 16 of the 64 columns, so the
-// row phases (S', P, epilogue, state) run four threads per row and combine row
-// maxima and sums with one shuffle and a two-warp named barrier.  The masked
-// scores P go back to shared memory (K-major, two-term) for P V.
+// row phases (S', P, epilogue, state) run four threads per row and combine the
+// RMSNorm row sums with one shuffle and a two-warp named barrier.  The masked
+// scores P go back to shared memory (K-major, two-term, a fixed 2^-22 shift)
+// for P V.
 #pragma once
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace gtr {
@@ -57,6 +60,7 @@ constexpr int kD = 64;                 // head dim (dk = dv)
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr float kSpanMax = 20.0f;      // nats of in-chunk decay the scaled operands take
+constexpr int kPShift = 22;            // masked scores enter P V as raw scores * 2^-22
 constexpr unsigned long long kWaitNs = 500ull * 1000 * 1000;   // bounded waits: 0.5 s
 
 constexpr int kRaw16 = kC * kD * 2;    // one 16-bit staging tile: 8 KB
@@ -441,7 +445,7 @@ __device__ __forceinline__ bool column_pass(float* G, const T* kst, const T* vst
     lo = fminf(lo, run);
     hi = fmaxf(hi, run);
     km = fmaxf(km, fabsf(Elem<T>::to_f(kst[j * kD + dd])));
-    vm = fmaxf(vm, fabsf(Elem<T>::to_f(vst[j * kD + dd])));
+    if (!std::is_same<T, __half>::value) vm = fmaxf(vm, fabsf(Elem<T>::to_f(vst[j * kD + dd])));
   }
   m.u.part[qt][dd] = run;
   atomicMax(&m.kmx[dd], __float_as_int(km));        // non-negative floats order as ints
@@ -468,7 +472,7 @@ __device__ __forceinline__ bool column_pass(float* G, const T* kst, const T* vst
     m.Gm[tid] = gm;
     m.aG[tid] = expf(gam);
     m.eK[tid] = expf(gam - gm);
-    const int ev = scale_exp(vm4);
+    const int ev = std::is_same<T, __half>::value ? 0 : scale_exp(vm4);
     m.sev[tid] = pow2i(ev);
     m.iev[tid] = pow2i(-ev);
     // |k~_id| <= max_i |k_id| e^{G_m,d - min_i G_id};  |k^_id| <= max_i |k_id| e^{Gam_d - min_i G_id}
@@ -488,15 +492,9 @@ __device__ __forceinline__ bool column_pass(float* G, const T* kst, const T* vst
   return __syncthreads_or(irregular) != 0;
 }
 
-// Max over the four threads that share an accumulator row: the other half of
+// Sum over the four threads that share an accumulator row: the other half of
 // the warp (lane ^ 16) and the same lanes of the partner warp (warp ^ 4),
 // through shared memory and a named barrier of those two warps.
-__device__ __forceinline__ float row_combine_max(float v, Misc& m, int row, int half, int qd, int lane) {
-  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-  if (lane < 16) m.u.r.rowred[half][row] = v;
-  named_barrier(1 + qd, 64);
-  return fmaxf(v, m.u.r.rowred[half ^ 1][row]);
-}
 __device__ __forceinline__ float row_combine_sum(float v, Misc& m, int row, int half, int qd, int lane) {
   v += __shfl_xor_sync(0xffffffffu, v, 16);
   if (lane < 16) m.u.r.rowred[half][row] = v;
@@ -628,7 +626,10 @@ gla_tc(const Params p) {
       }
       const float4 gg = *reinterpret_cast<const float4*>(G + r * kD + cg);
       const uint32_t off = sw16(r, cg);
-      {   // V, column-scaled, one fp16 term (exact for 16-bit inputs)
+      if (std::is_same<T, __half>::value) {   // V: fp16 input is already an exact operand
+        *reinterpret_cast<uint2*>(VV + off) =
+            valid ? *reinterpret_cast<const uint2*>(vst + r * kD + cg) : make_uint2(0u, 0u);
+      } else {   // bf16 V, column-scaled into fp16 (exact for all but tiny values)
         const float4 sv = *reinterpret_cast<const float4*>(&m.sev[cg]);
         *reinterpret_cast<uint2*>(VV + off) = half4(vv.x * sv.x, vv.y * sv.y, vv.z * sv.z, vv.w * sv.w);
       }
@@ -694,21 +695,19 @@ gla_tc(const Params p) {
         float sc[16];
         tmem_ld16x2(tm + lane_base + 64 + half * 32, sc);
         tmem_ld_wait();
-        const float f = m.u.r.ieq[row] * pow2i(-ekt);
-        float mx = 0.f;
+        // The raw scores carry the q~ row scale and the key-tile scale and stay below
+        // 64 * 2^15 * 2^15 = 2^36, so a fixed 2^-22 puts every row inside fp16's range;
+        // P V is decoded with the same factors.
+        const float f = pow2i(-kPShift);
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           const int i = cbase + c;
           sc[c] = (i <= row && row < ntok) ? sc[c] * f : 0.f;
-          mx = fmaxf(mx, fabsf(sc[c]));
         }
-        mx = row_combine_max(mx, m, row, half, qd, lane);
-        const int ep = scale_exp(mx);
-        const float s = pow2i(ep);
-        if (lane < 16 && half == 0) m.u.r.iep[row] = pow2i(-ep);
+        if (lane < 16 && half == 0) m.u.r.iep[row] = m.u.r.ieq[row] * pow2i(kPShift - ekt);
 #pragma unroll
         for (int c = 0; c < 16; c += 4)
-          put2(QTh, QTl, sw16(row, cbase + c), sc[c] * s, sc[c + 1] * s, sc[c + 2] * s, sc[c + 3] * s);
+          put2(QTh, QTl, sw16(row, cbase + c), sc[c], sc[c + 1], sc[c + 2], sc[c + 3]);
       } else {
         // exact scores on CUDA cores: P_ji = sum_d q_jd k_id e^{G_jd - G_id}; four threads per row
         if (tid == 0) atomicAdd(&g_gtr_exact_chunks, 1ull);
