@@ -429,7 +429,8 @@ def run_ours(args, world, rank, local):
             "value": value, "unit": "token-heads/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
-            "dtype": "f32" if path == "simt" else "tf32/f32",
+            # tensor-core path: two-term bf16 operands (hi + lo), fp32 accumulation
+            "dtype": "f32" if path == "simt" else "bf16x2/f32",
             "data": "synthetic",
             "config": {"workload": workload_text(wl), "chunk": args.chunk, "kernel_path": path,
                        "l2": f"{N_SETS} rotating input sets, inputs larger than L2",

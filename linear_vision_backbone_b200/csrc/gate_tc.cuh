@@ -29,8 +29,43 @@ namespace gtr {
 namespace gate_tc {
 
 using tc::saddr;
-using tc::scale_exp;
-using tc::pow2i;
+
+// Power-of-two operand scales: 2^e puts the magnitude m into [2^14, 2^15),
+// inside fp16's range; exact, and undone on the fp32 accumulator.
+__device__ __forceinline__ int scale_exp(float m) {
+  if (!(m > 0.f) || !(m <= 3.0e38f)) return 0;
+  const int ex = ((__float_as_int(m) >> 23) & 0xFF) - 127;
+  return max(-60, min(60, 14 - ex));
+}
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }
+// Two-term fp16 operand: x = hi + lo, hi = fp16(x), lo = fp16(x - hi); four
+// consecutive elements at byte offset `off` of the (hi, lo) tiles.
+__device__ __forceinline__ void put2(uint8_t* hi, uint8_t* lo, uint32_t off, float a, float b, float c,
+                                     float d) {
+  const __half2 h0 = __floats2half2_rn(a, b), h1 = __floats2half2_rn(c, d);
+  const float2 f0 = __half22float2(h0), f1 = __half22float2(h1);
+  const __half2 l0 = __floats2half2_rn(a - f0.x, b - f0.y), l1 = __floats2half2_rn(c - f1.x, d - f1.y);
+  uint2 H, L;
+  memcpy(&H.x, &h0, 4);
+  memcpy(&H.y, &h1, 4);
+  memcpy(&L.x, &l0, 4);
+  memcpy(&L.y, &l1, 4);
+  *reinterpret_cast<uint2*>(hi + off) = H;
+  *reinterpret_cast<uint2*>(lo + off) = L;
+}
+// 32 lanes x 32 bit, 16 consecutive columns: thread t of warp w <- lane 32w+t.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
 
 constexpr int kM = 128;               // tokens per CTA
 constexpr int kThreads = 256;
@@ -186,7 +221,7 @@ gate_proj_tc(const TX* __restrict__ x, const float* __restrict__ w_down, const f
 #pragma unroll
     for (int k = 0; k < kRank; ++k) {
       const uint32_t off = swmn(k, 4 * tid, kRank);
-      tc::put2(tWu, tWu + Layout::kWu, off, wu[k].x * s0, wu[k].y * s1, wu[k].z * s2, wu[k].w * s3);
+      put2(tWu, tWu + Layout::kWu, off, wu[k].x * s0, wu[k].y * s1, wu[k].z * s2, wu[k].w * s3);
     }
   }
   __syncthreads();
@@ -236,7 +271,7 @@ gate_proj_tc(const TX* __restrict__ x, const float* __restrict__ w_down, const f
   // low row r (warps 0-3, thread = row) -> per-row scaled two-term fp16 A tile (K = 16)
   if (warp < 4) {
     float lw[16];
-    tc::tmem_ld16(tm + ((uint32_t)(warp * 32) << 16) + 0, lw);
+    tmem_ld16(tm + ((uint32_t)(warp * 32) << 16) + 0, lw);
     tc::tmem_ld_wait();
     const int r = warp * 32 + lane;
     float mx = 0.f;
@@ -250,7 +285,7 @@ gate_proj_tc(const TX* __restrict__ x, const float* __restrict__ w_down, const f
     m.low_i[r] = pow2i(-e);
 #pragma unroll
     for (int c = 0; c < 16; c += 4)
-      tc::put2(tLow, tLow + Layout::kLow, swk(r, c, kM), lw[c] * s, lw[c + 1] * s, lw[c + 2] * s,
+      put2(tLow, tLow + Layout::kLow, swk(r, c, kM), lw[c] * s, lw[c + 1] * s, lw[c + 2] * s,
                lw[c + 3] * s);
   }
   tc::fence_async_smem();
@@ -284,7 +319,7 @@ gate_proj_tc(const TX* __restrict__ x, const float* __restrict__ w_down, const f
     float* grow = g + (tok0 + r) * HD;
     for (int cb = 0; cb < ncol; cb += 16) {
       float u[16];
-      tc::tmem_ld16(tm + ((uint32_t)((warp & 3) * 32) << 16) + 64 + c0 + cb, u);
+      tmem_ld16(tm + ((uint32_t)((warp & 3) * 32) << 16) + 64 + c0 + cb, u);
       tc::tmem_ld_wait();
       if (r < ntok) {
 #pragma unroll

@@ -58,7 +58,7 @@ struct Plan {
   int seg_chunks;  // chunks per segment
   int nseg;        // segments per sequence
   int seg_len;     // scan positions per segment
-  size_t offL;     // byte offset of the log-decay array in the workspace
+  size_t offA;     // byte offset of the segment decay factors in the workspace
   size_t ws_bytes;
 };
 
@@ -116,8 +116,8 @@ int make_plan(Plan* p, int dev, int B, int H, int gh, int gw, int dk, int dv, in
   p->nseg = (p->nc + p->seg_chunks - 1) / p->seg_chunks;
   p->seg_len = p->seg_chunks * chunk;
   const size_t nS = (size_t)bh * p->nseg * dk * dv * sizeof(float);
-  p->offL = (nS + 255) & ~(size_t)255;
-  p->ws_bytes = p->offL + (size_t)bh * p->nseg * dk * sizeof(float);
+  p->offA = (nS + 255) & ~(size_t)255;
+  p->ws_bytes = p->offA + (size_t)bh * p->nseg * dk * sizeof(float);
   return GTR_OK;
 }
 
@@ -165,14 +165,14 @@ int ensure_smem(K kern, size_t smem, bool* done, int dev) {
 
 template <typename T, int ROWS>
 int launch_simt_rows(const Plan& p, const void* q, const void* k, const void* v, const float* g,
-                     const void* z, const float* w, void* out, float* wsS, float* wsL,
+                     const void* z, const float* w, void* out, float* wsS, float* wsA,
                      cudaStream_t st, int stage) {
   const dim3 grid(p.nseg, p.B * p.H);
   if (stage == 0) {
     // at most kSimtBatch * 4 * 128 floats = 32 KB: no opt-in needed
     const size_t smem = (size_t)simt_summary_smem_floats(p.dk, p.dv) * sizeof(float);
     auto kern = gla_summary_simt<T, ROWS>;
-    kern<<<grid, kSimtThreads, smem, st>>>((const T*)k, (const T*)v, g, wsS, wsL, p.H, p.T, p.gh,
+    kern<<<grid, kSimtThreads, smem, st>>>((const T*)k, (const T*)v, g, wsS, wsA, p.H, p.T, p.gh,
                                            p.gw, p.dk, p.dv, p.dir, p.seg_len, p.nseg);
   } else {
     const size_t smem = (size_t)simt_output_smem_floats(p.dk, p.dv) * sizeof(float);
@@ -190,39 +190,39 @@ int launch_simt_rows(const Plan& p, const void* q, const void* k, const void* v,
 
 template <typename T>
 int launch_simt(const Plan& p, const void* q, const void* k, const void* v, const float* g,
-                const void* z, const float* w, void* out, float* wsS, float* wsL, cudaStream_t st,
+                const void* z, const float* w, void* out, float* wsS, float* wsA, cudaStream_t st,
                 int stage) {
   switch ((p.dk * p.dv) / kSimtThreads) {
-    case 1: return launch_simt_rows<T, 1>(p, q, k, v, g, z, w, out, wsS, wsL, st, stage);
-    case 2: return launch_simt_rows<T, 2>(p, q, k, v, g, z, w, out, wsS, wsL, st, stage);
-    case 4: return launch_simt_rows<T, 4>(p, q, k, v, g, z, w, out, wsS, wsL, st, stage);
-    case 8: return launch_simt_rows<T, 8>(p, q, k, v, g, z, w, out, wsS, wsL, st, stage);
-    case 16: return launch_simt_rows<T, 16>(p, q, k, v, g, z, w, out, wsS, wsL, st, stage);
-    case 32: return launch_simt_rows<T, 32>(p, q, k, v, g, z, w, out, wsS, wsL, st, stage);
-    case 64: return launch_simt_rows<T, 64>(p, q, k, v, g, z, w, out, wsS, wsL, st, stage);
+    case 1: return launch_simt_rows<T, 1>(p, q, k, v, g, z, w, out, wsS, wsA, st, stage);
+    case 2: return launch_simt_rows<T, 2>(p, q, k, v, g, z, w, out, wsS, wsA, st, stage);
+    case 4: return launch_simt_rows<T, 4>(p, q, k, v, g, z, w, out, wsS, wsA, st, stage);
+    case 8: return launch_simt_rows<T, 8>(p, q, k, v, g, z, w, out, wsS, wsA, st, stage);
+    case 16: return launch_simt_rows<T, 16>(p, q, k, v, g, z, w, out, wsS, wsA, st, stage);
+    case 32: return launch_simt_rows<T, 32>(p, q, k, v, g, z, w, out, wsS, wsA, st, stage);
+    case 64: return launch_simt_rows<T, 64>(p, q, k, v, g, z, w, out, wsS, wsA, st, stage);
     default: return GTR_ERR_UNSUPPORTED;
   }
 }
 
 // stage 0 = K2 summary, 1 = K4 output
 int launch_stage(const Plan& p, const void* q, const void* k, const void* v, const float* g,
-                 const void* z, const float* w, void* out, float* wsS, float* wsL, cudaStream_t st,
+                 const void* z, const float* w, void* out, float* wsS, float* wsA, cudaStream_t st,
                  int stage) {
   if (p.path == GTR_PATH_TC)
-    return launch_tc(p.dtype, stage, q, k, v, g, z, w, out, wsS, wsL, p.B, p.H, p.T, p.gh, p.gw,
+    return launch_tc(p.dtype, stage, q, k, v, g, z, w, out, wsS, wsA, p.B, p.H, p.T, p.gh, p.gw,
                      p.dk, p.dv, p.dir, p.chunk, p.seg_chunks, p.nseg, st);
   switch (p.dtype) {
-    case GTR_F32: return launch_simt<float>(p, q, k, v, g, z, w, out, wsS, wsL, st, stage);
-    case GTR_F16: return launch_simt<__half>(p, q, k, v, g, z, w, out, wsS, wsL, st, stage);
-    case GTR_BF16: return launch_simt<__nv_bfloat16>(p, q, k, v, g, z, w, out, wsS, wsL, st, stage);
+    case GTR_F32: return launch_simt<float>(p, q, k, v, g, z, w, out, wsS, wsA, st, stage);
+    case GTR_F16: return launch_simt<__half>(p, q, k, v, g, z, w, out, wsS, wsA, st, stage);
+    case GTR_BF16: return launch_simt<__nv_bfloat16>(p, q, k, v, g, z, w, out, wsS, wsA, st, stage);
   }
   return GTR_ERR_INVALID_ARG;
 }
 
-int launch_scan(const Plan& p, float* wsS, const float* wsL, int inclusive, cudaStream_t st) {
+int launch_scan(const Plan& p, float* wsS, const float* wsA, int inclusive, cudaStream_t st) {
   const long long total = (long long)p.B * p.H * p.dk * p.dv;
   const long long blocks = (total + kScanThreads - 1) / kScanThreads;
-  gla_state_scan<<<(unsigned)blocks, kScanThreads, 0, st>>>(wsS, wsL, total, p.nseg, p.dk, p.dv,
+  gla_state_scan<<<(unsigned)blocks, kScanThreads, 0, st>>>(wsS, wsA, total, p.nseg, p.dk, p.dv,
                                                            inclusive);
   return launch_status();
 }
@@ -256,14 +256,14 @@ int gla_fwd_impl(const void* q, const void* k, const void* v, const float* g, co
   void* ws = nullptr;
   if ((rc = get_workspace(dev, stream, p.ws_bytes, &ws))) return rc;
   float* wsS = (float*)ws;
-  float* wsL = (float*)((char*)ws + p.offL);
+  float* wsA = (float*)((char*)ws + p.offA);
   cudaStream_t st = (cudaStream_t)stream;
   if ((rc = record(ev, 0, st))) return rc;
-  if ((rc = launch_stage(p, q, k, v, g, z, w, out, wsS, wsL, st, 0))) return rc;
+  if ((rc = launch_stage(p, q, k, v, g, z, w, out, wsS, wsA, st, 0))) return rc;
   if ((rc = record(ev, 1, st))) return rc;
-  if ((rc = launch_scan(p, wsS, wsL, 0, st))) return rc;
+  if ((rc = launch_scan(p, wsS, wsA, 0, st))) return rc;
   if ((rc = record(ev, 2, st))) return rc;
-  if ((rc = launch_stage(p, q, k, v, g, z, w, out, wsS, wsL, st, 1))) return rc;
+  if ((rc = launch_stage(p, q, k, v, g, z, w, out, wsS, wsA, st, 1))) return rc;
   return record(ev, 3, st);
 }
 
@@ -319,11 +319,11 @@ int gla_fwd_noalloc_impl(const void* q, const void* k, const void* v, const floa
   void* ws = nullptr;
   if ((rc = static_scratch(dev, &ws))) return rc;
   float* wsS = (float*)ws;
-  float* wsL = (float*)((char*)ws + p.offL);
+  float* wsA = (float*)((char*)ws + p.offA);
   cudaStream_t st = (cudaStream_t)stream;
-  if ((rc = launch_stage(p, q, k, v, g, z, w, out, wsS, wsL, st, 0))) return rc;
-  if ((rc = launch_scan(p, wsS, wsL, 0, st))) return rc;
-  return launch_stage(p, q, k, v, g, z, w, out, wsS, wsL, st, 1);
+  if ((rc = launch_stage(p, q, k, v, g, z, w, out, wsS, wsA, st, 0))) return rc;
+  if ((rc = launch_scan(p, wsS, wsA, 0, st))) return rc;
+  return launch_stage(p, q, k, v, g, z, w, out, wsS, wsA, st, 1);
 }
 
 }  // namespace

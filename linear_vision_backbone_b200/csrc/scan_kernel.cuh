@@ -6,9 +6,10 @@
 // One thread per state element (b, h, i, j); consecutive threads own
 // consecutive j, so every load and store is a coalesced 128-byte line.  For
 // each (b, h) the segments are visited in scan order:
-//     S_in[0] = 0,   S_in[s+1] = exp(L_s[i]) * S_in[s] + dS_s[i][j]
-// where dS_s is the state segment s produces from a zero start and L_s its
-// summed log-gate.  The result overwrites dS in place (exclusive form: the
+//     S_in[0] = 0,   S_in[s+1] = A_s[i] * S_in[s] + dS_s[i][j]
+// where dS_s is the state segment s produces from a zero start and
+// A_s = exp(L_s) its decay factor (L_s = the segment's summed log-gate), both
+// written by the summary stage.  The result overwrites dS in place (exclusive form: the
 // state each segment starts from) or, with `inclusive`, the state each segment
 // ends with.  The loads of a group of up to 32 segments are all issued before
 // any store, so one memory latency covers the whole group and the dependent
@@ -22,7 +23,7 @@ constexpr int kScanThreads = 128;
 constexpr int kScanGroup = 32;
 
 __global__ void __launch_bounds__(kScanThreads)
-gla_state_scan(float* __restrict__ wsS, const float* __restrict__ wsL, long long total, int nseg,
+gla_state_scan(float* __restrict__ wsS, const float* __restrict__ wsA, long long total, int nseg,
                int dk, int dv, int inclusive) {
   const long long e = (long long)blockIdx.x * kScanThreads + threadIdx.x;
   if (e >= total) return;
@@ -31,7 +32,7 @@ gla_state_scan(float* __restrict__ wsS, const float* __restrict__ wsL, long long
   const int rem = (int)(e - bh * dkdv);
   const int i = rem / dv;
   float* p = wsS + (size_t)bh * nseg * dkdv + rem;
-  const float* L = wsL + (size_t)bh * nseg * dk + i;
+  const float* A = wsA + (size_t)bh * nseg * dk + i;
   float S = 0.f;
   for (int s0 = 0; s0 < nseg; s0 += kScanGroup) {
     const int n = min(kScanGroup, nseg - s0);
@@ -40,7 +41,7 @@ gla_state_scan(float* __restrict__ wsS, const float* __restrict__ wsL, long long
     for (int u = 0; u < kScanGroup; ++u) {
       if (u < n) {
         dS[u] = p[(size_t)(s0 + u) * dkdv];
-        a[u] = expf(L[(size_t)(s0 + u) * dk]);
+        a[u] = A[(size_t)(s0 + u) * dk];
       }
     }
 #pragma unroll

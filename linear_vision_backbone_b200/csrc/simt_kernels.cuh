@@ -37,7 +37,7 @@ __device__ __forceinline__ size_t token_row(int b, int t, int T_, int H, int h) 
 template <typename T, int ROWS>
 __global__ void __launch_bounds__(kSimtThreads)
 gla_summary_simt(const T* __restrict__ k, const T* __restrict__ v, const float* __restrict__ g,
-                 float* __restrict__ wsS, float* __restrict__ wsL, int H, int T_, int gh, int gw,
+                 float* __restrict__ wsS, float* __restrict__ wsA, int H, int T_, int gh, int gw,
                  int dk, int dv, int dir, int seg_len, int nseg) {
   extern __shared__ float sm[];
   float* ks = sm;                            // [batch][dk]
@@ -86,7 +86,7 @@ gla_summary_simt(const T* __restrict__ k, const T* __restrict__ v, const float* 
   float* outS = wsS + ((size_t)bh * nseg + seg) * dk * dv;
 #pragma unroll
   for (int r = 0; r < ROWS; ++r) outS[(size_t)(rg + r * nrg) * dv + j] = S[r];
-  if (tid < dk) wsL[((size_t)bh * nseg + seg) * dk + tid] = lsum;
+  if (tid < dk) wsA[((size_t)bh * nseg + seg) * dk + tid] = expf(lsum);   // segment decay factor
 }
 
 template <typename T, int ROWS>
