@@ -243,6 +243,15 @@ __device__ __forceinline__ void put4(uint8_t* H, uint8_t* L, uint32_t off, float
   *reinterpret_cast<uint2*>(L + off) = make_uint2(l0, l1);
 }
 
+// eight consecutive elements (16 bytes, one swizzle unit) at byte offset `off`
+__device__ __forceinline__ void put8(uint8_t* H, uint8_t* L, uint32_t off, const float* x) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) split2(x[2 * i], x[2 * i + 1], h[i], l[i]);
+  *reinterpret_cast<uint4*>(H + off) = make_uint4(h[0], h[1], h[2], h[3]);
+  *reinterpret_cast<uint4*>(L + off) = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
 template <typename T> struct Vec4;
 template <> struct Vec4<__half> {
   static __device__ __forceinline__ float4 from_bits(uint2 u) {
@@ -304,17 +313,6 @@ __device__ __forceinline__ void fetch16(uint8_t* dst, const void* src, const lon
     else *reinterpret_cast<uint4*>(dst + j * 128 + part) = make_uint4(0u, 0u, 0u, 0u);
   }
 }
-// The same pieces into a 128B-swizzled operand tile.
-__device__ __forceinline__ void fetch16_sw(uint8_t* tile, const void* src, const long long* rows,
-                                           int ntok, int tid) {
-#pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    const int o = tid + u * kThreads, j = o >> 3, part = o & 7;
-    uint8_t* dst = tile + sw_unit(j, part);
-    if (j < ntok) cp_async16(dst, (const uint8_t*)src + rows[j] * kRowBytes + part * 16);
-    else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
-  }
-}
 // The fp32 gate rows (256 bytes each); rows past ntok get a zero gate.
 __device__ __forceinline__ void fetch_g(uint8_t* dst, const float* g, const long long* rows, int ntok,
                                         int tid) {
@@ -325,26 +323,6 @@ __device__ __forceinline__ void fetch_g(uint8_t* dst, const float* g, const long
     else *reinterpret_cast<uint4*>(dst + j * 256 + part) = make_uint4(0u, 0u, 0u, 0u);
   }
 }
-// Split an fp16 V tile that fetch16_sw landed in L into bf16 (hi, lo) tiles,
-// in place; each thread converts exactly the pieces its own copies wrote.
-__device__ __forceinline__ void split_v_f16(uint8_t* H, uint8_t* L, int tid) {
-#pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    const int o = tid + u * kThreads;
-    const uint32_t off = sw_unit(o >> 3, o & 7);
-    const uint4 raw = *reinterpret_cast<const uint4*>(L + off);
-    const float4 a = Vec4<__half>::from_bits(make_uint2(raw.x, raw.y));
-    const float4 c = Vec4<__half>::from_bits(make_uint2(raw.z, raw.w));
-    uint32_t h0, l0, h1, l1, h2, l2, h3, l3;
-    split2(a.x, a.y, h0, l0);
-    split2(a.z, a.w, h1, l1);
-    split2(c.x, c.y, h2, l2);
-    split2(c.z, c.w, h3, l3);
-    *reinterpret_cast<uint4*>(H + off) = make_uint4(h0, h1, h2, h3);
-    *reinterpret_cast<uint4*>(L + off) = make_uint4(l0, l1, l2, l3);
-  }
-}
-
 // In-chunk inclusive cumsum of the gate tile, column dd, tokens 16 qt .. 16 qt
 // + 15 of this thread, in registers; the four threads of a column exchange
 // their partial sums once through `part` (one block barrier).  Returns the
@@ -368,7 +346,7 @@ __device__ __forceinline__ float silu_fast(float z) { return __fdividef(z, 1.0f 
 
 // ===================================================================== K4
 struct OutMisc {                  // per-CTA scalars; arrays read as float4 are 16-byte aligned
-  uint64_t mma[3];                // [0] q~ S' + scores, [1] + P V, [2] state increment
+  uint64_t mma[3];                // [0] q~ S' and scores (two arrivals), [1] + P V, [2] state increment
   uint32_t tmem;
   int pad;
   alignas(16) float red[4][kD];   // column-pass partial sums; epilogue row sums
@@ -380,8 +358,8 @@ struct OutMisc {                  // per-CTA scalars; arrays read as float4 are 
   alignas(16) long long rows[2][kC];   // token rows of the current / next chunk
 };
 struct OutLayout {
-  // staging (row-major): k, q, z, gate
-  static constexpr int kOffK = 0, kOffQ = kTile, kOffZ = 2 * kTile, kOffG = 3 * kTile;
+  // staging (row-major): k, q, v, gate of one chunk
+  static constexpr int kOffK = 0, kOffQ = kTile, kOffV = 2 * kTile, kOffG = 3 * kTile;
   // operand tiles (1024-aligned): VH VL QH QL KH KL SH SL
   static constexpr int kTiles = 3 * kTile + kGTile;
   static constexpr int kMisc = kTiles + 8 * kTile;
@@ -390,6 +368,15 @@ struct OutLayout {
   static constexpr int kBlocksPerSM = 2;
 };
 static_assert(OutLayout::kTiles % 1024 == 0, "operand tiles must be 1024-byte aligned");
+
+// The k, q, v, gate rows of a chunk into the output kernel's staging.
+__device__ __forceinline__ void fetch_chunk(uint8_t* sm, const Params& p, const long long* rows, int ntok,
+                                            int tid) {
+  fetch16(sm + OutLayout::kOffK, p.k, rows, ntok, tid);
+  fetch16(sm + OutLayout::kOffQ, p.q, rows, ntok, tid);
+  fetch16(sm + OutLayout::kOffV, p.v, rows, ntok, tid);
+  fetch_g(sm + OutLayout::kOffG, p.g, rows, ntok, tid);
+}
 static_assert(2 * (OutLayout::kSmem + 1024) <= 228 * 1024, "two output CTAs must share an SM");
 
 // Sum over the four threads that share an accumulator row: the other half of
@@ -412,7 +399,7 @@ gla_out_tc(const Params p) {
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const T* kst = reinterpret_cast<const T*>(sm + L::kOffK);
   const T* qst = reinterpret_cast<const T*>(sm + L::kOffQ);
-  const T* zst = reinterpret_cast<const T*>(sm + L::kOffZ);
+  const T* vst = reinterpret_cast<const T*>(sm + L::kOffV);
   float* G = reinterpret_cast<float*>(sm + L::kOffG);
   uint8_t* VH = sm + L::kTiles;
   uint8_t* VL = VH + kTile;
@@ -444,18 +431,12 @@ gla_out_tc(const Params p) {
   const int dd = tid & 63, qt = tid >> 6;
   const int rb = tid >> 4, cg = (tid & 15) * 4;
 
-  // chunk 0: its k, q, g / V / z copies go out first, as three groups
+  // chunk 0's copies go out first
   {
     const int ntok0 = min(kC, p.T - c0 * kC);
     chunk_rows(p, m.rows[0], b, h, d, c0 * kC, ntok0, tid);
     __syncthreads();
-    fetch16(sm + L::kOffK, p.k, m.rows[0], ntok0, tid);
-    fetch16(sm + L::kOffQ, p.q, m.rows[0], ntok0, tid);
-    fetch_g(sm + L::kOffG, p.g, m.rows[0], ntok0, tid);
-    cp_async_commit();
-    fetch16_sw(kV2 ? VL : VH, p.v, m.rows[0], ntok0, tid);
-    cp_async_commit();
-    fetch16(sm + L::kOffZ, p.z, m.rows[0], ntok0, tid);
+    fetch_chunk(sm, p, m.rows[0], ntok0, tid);
     cp_async_commit();
   }
   // carried state: S[row][cbase .. cbase + 15], from the boundary scan
@@ -470,7 +451,7 @@ gla_out_tc(const Params p) {
     }
   }
   if (tid == 0) {
-    mbar_init(&m.mma[0], 1);
+    mbar_init(&m.mma[0], 2);
     mbar_init(&m.mma[1], 1);
     mbar_init(&m.mma[2], 1);
     mbar_fence_init();
@@ -480,7 +461,7 @@ gla_out_tc(const Params p) {
     tmem_alloc(&m.tmem, L::kTmemCols);
     tmem_relinquish();
   }
-  cp_async_wait<2>();                     // chunk 0's k, q, g
+  cp_async_wait<0>();                     // chunk 0's k, q, v, g
   tc_before_sync();
   __syncthreads();
   tc_after_sync();
@@ -491,9 +472,9 @@ gla_out_tc(const Params p) {
 
   uint32_t ph0 = 0, ph1 = 0, ph2 = 0;
   bool failed = false;
-  // cp.async groups per chunk, in order: next k, q, g (after the tiles, or
-  // after P for an exact chunk; the other of the two is empty), next V (once
-  // this chunk's products are done), next z (after the epilogue).
+  // The next chunk's k, q, v, g are copied once this chunk's tiles are built
+  // (after P for an exact chunk, whose scores still read the staging); z goes
+  // straight to registers, requested two phases before the epilogue uses it.
   for (int it = 0; it < nch; ++it) {
     const int par = it & 1;
     const int s0 = (c0 + it) * kC;
@@ -548,32 +529,57 @@ gla_out_tc(const Params p) {
       }
       // S' = e^{G_m} S, or S for an exact chunk
       const float sc = tilde ? __expf(m.Gm[row]) : 1.0f;
+      float sp[16];
 #pragma unroll
-      for (int c = 0; c < 16; c += 4)
-        put4(SH, SL, sw16(row, cbase + c), sc * S[c], sc * S[c + 1], sc * S[c + 2], sc * S[c + 3]);
+      for (int c = 0; c < 16; ++c) sp[c] = sc * S[c];
+      put8(SH, SL, sw16(row, cbase), sp);
+      put8(SH, SL, sw16(row, cbase + 8), sp + 8);
     }
-    cp_async_wait<1>();                   // this chunk's V (pending after this: its z)
-    if (kV2) split_v_f16(VH, VL, tid);
+    // V from staging: fp16 as two bf16 terms, bf16 as it is
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int r = rb + 16 * u;
+      const uint32_t off = sw16(r, cg);
+      if (kV2) {
+        const float4 vv = Vec4<T>::load(vst + r * kD + cg);
+        put4(VH, VL, off, vv.x, vv.y, vv.z, vv.w);
+      } else {
+        *reinterpret_cast<uint2*>(VH + off) = *reinterpret_cast<const uint2*>(vst + r * kD + cg);
+      }
+    }
     if (more) chunk_rows(p, m.rows[par ^ 1], b, h, d, s1, ntok1, tid);
     fence_async_smem();
     tc_before_sync();
     __syncthreads();
     tc_after_sync();
 
+    // Two issuing threads: a single thread issues one MMA per ~60 cycles
+    // whatever its size, so independent products go out from two warps and
+    // the tensor pipe interleaves them.  Warp 0 owns o (q~ S', later P V),
+    // warp 4 the score columns (scores, later the state increment); each
+    // thread's own MMAs execute in issue order.  P overwrites q~, so mma[0]
+    // completes only when both threads' products are done.
     if (tid == 0) {
-      const uint64_t qh = desc_k(QH), ql = desc_k(QL);
-      mma_terms<kStepK, kStepMN>(tm + 0, qh, ql, desc_mn(SH), desc_mn(SL), true, kIdQS, false);
+      mma_terms<kStepK, kStepMN>(tm + 0, desc_k(QH), desc_k(QL), desc_mn(SH), desc_mn(SL), true, kIdQS,
+                                 false);
+      mma_commit(&m.mma[0]);
+    }
+    if (tid == 128) {
       if (tilde)
-        mma_terms<kStepK, kStepK>(tm + 64, qh, ql, desc_k(KH), desc_k(KL), true, kIdQK, false);
+        mma_terms<kStepK, kStepK>(tm + 64, desc_k(QH), desc_k(QL), desc_k(KH), desc_k(KL), true, kIdQK,
+                                  false);
       mma_commit(&m.mma[0]);
     }
     // the staging of k, q, g is consumed unless an exact chunk still reads it
-    if (more && tilde) {
-      fetch16(sm + L::kOffK, p.k, m.rows[par ^ 1], ntok1, tid);
-      fetch16(sm + L::kOffQ, p.q, m.rows[par ^ 1], ntok1, tid);
-      fetch_g(sm + L::kOffG, p.g, m.rows[par ^ 1], ntok1, tid);
-    }
+    if (more && tilde) fetch_chunk(sm, p, m.rows[par ^ 1], ntok1, tid);
     cp_async_commit();
+    // this chunk's z for the epilogue: 16 elements of the thread's row
+    uint4 zz0 = make_uint4(0u, 0u, 0u, 0u), zz1 = zz0;
+    if (row < ntok) {
+      const uint4* zp = reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.z) + m.rows[par][row] * kD + cbase);
+      zz0 = __ldg(zp);
+      zz1 = __ldg(zp + 1);
+    }
 
     failed |= !mbar_wait(&m.mma[0], ph0);
     ph0 ^= 1;
@@ -585,9 +591,8 @@ gla_out_tc(const Params p) {
       tmem_ld_wait();
 #pragma unroll
       for (int c = 0; c < 16; ++c) sc[c] = cbase + c <= row ? sc[c] : 0.f;
-#pragma unroll
-      for (int c = 0; c < 16; c += 4)
-        put4(QH, QL, sw16(row, cbase + c), sc[c], sc[c + 1], sc[c + 2], sc[c + 3]);
+      put8(QH, QL, sw16(row, cbase), sc);
+      put8(QH, QL, sw16(row, cbase + 8), sc + 8);
     } else {
       // exact scores on CUDA cores: P_ji = sum_d q_jd k_id e^{G_jd - G_id}; four threads per row
       if (tid == 0) atomicAdd(&g_gtr_exact_chunks, 1ull);
@@ -610,22 +615,20 @@ gla_out_tc(const Params p) {
       for (int e = 0; e < 16; e += 4)
         put4(QH, QL, sw16(j, ib + e), acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
     }
-    cp_async_wait<1>();                   // this chunk's z (pending after this: the next k, q, g)
     fence_async_smem();
     tc_before_sync();
     if (__syncthreads_or(failed)) break;
     tc_after_sync();
-    if (more && exact) {
-      fetch16(sm + L::kOffK, p.k, m.rows[par ^ 1], ntok1, tid);
-      fetch16(sm + L::kOffQ, p.q, m.rows[par ^ 1], ntok1, tid);
-      fetch_g(sm + L::kOffG, p.g, m.rows[par ^ 1], ntok1, tid);
-    }
+    if (more && exact) fetch_chunk(sm, p, m.rows[par ^ 1], ntok1, tid);
     cp_async_commit();
     if (tid == 0) {
-      const uint64_t vh = desc_mn(VH), vl = desc_mn(VL);
-      mma_terms<kStepK, kStepMN>(tm + 0, desc_k(QH), desc_k(QL), vh, vl, kV2, kIdQS, true);
+      mma_terms<kStepK, kStepMN>(tm + 0, desc_k(QH), desc_k(QL), desc_mn(VH), desc_mn(VL), kV2, kIdQS,
+                                 true);
       mma_commit(&m.mma[1]);
-      mma_terms<kStepMN, kStepMN>(tm + 64, desc_mn(KH), desc_mn(KL), vh, vl, kV2, kIdKV, false);
+    }
+    if (tid == 128) {
+      mma_terms<kStepMN, kStepMN>(tm + 64, desc_mn(KH), desc_mn(KL), desc_mn(VH), desc_mn(VL), kV2,
+                                  kIdKV, false);
       mma_commit(&m.mma[2]);
     }
 
@@ -643,11 +646,10 @@ gla_out_tc(const Params p) {
       ss = row_combine_sum(ss, m.red, row, half, qd, lane);
       if (row < ntok) {
         const float inv = rsqrtf(ss * (1.0f / kD) + kRmsEps);
-        const T* zr = zst + row * kD + cbase;
         T* dst = reinterpret_cast<T*>(p.out) + m.rows[par][row] * kD + cbase;
 #pragma unroll
         for (int c = 0; c < 16; c += 8) {
-          const uint4 zz = *reinterpret_cast<const uint4*>(zr + c);
+          const uint4 zz = c == 0 ? zz0 : zz1;
           const float4 z0 = Vec4<T>::from_bits(make_uint2(zz.x, zz.y));
           const float4 z1 = Vec4<T>::from_bits(make_uint2(zz.z, zz.w));
           const float4 w0 = *reinterpret_cast<const float4*>(&m.wv[cbase + c]);
@@ -665,8 +667,6 @@ gla_out_tc(const Params p) {
     failed |= !mbar_wait(&m.mma[2], ph2);
     ph2 ^= 1;
     tc_after_sync();
-    if (more) fetch16_sw(kV2 ? VL : VH, p.v, m.rows[par ^ 1], ntok1, tid);   // V tile is free
-    cp_async_commit();
     {
       float ds[16];
       tmem_ld16x2(tm + lane_base + 64 + half * 32, ds);
@@ -675,12 +675,10 @@ gla_out_tc(const Params p) {
 #pragma unroll
       for (int c = 0; c < 16; ++c) S[c] = fmaf(a, S[c], f * ds[c]);
     }
-    cp_async_wait<1>();                   // the next k, q, g (pending after this: its V)
+    cp_async_wait<0>();                   // the next chunk's k, q, v, g
     tc_before_sync();
     if (__syncthreads_or(failed)) break;
     tc_after_sync();
-    if (more) fetch16(sm + L::kOffZ, p.z, m.rows[par ^ 1], ntok1, tid);   // z is consumed
-    cp_async_commit();
   }
 
   cp_async_wait<0>();                     // no copy may land after the block exits
@@ -707,7 +705,7 @@ struct SumLayout {
   static constexpr int kTiles = 2 * kStage;
   static constexpr int kMisc = kTiles + 4 * kTile;
   static constexpr int kSmem = kMisc + (int)sizeof(SumMisc) + 1024;
-  static constexpr int kTmemCols = 64;
+  static constexpr int kTmemCols = 128;   // two accumulators, summed at the end
   static constexpr int kBlocksPerSM = 2;
 };
 static_assert(SumLayout::kTiles % 1024 == 0, "operand tiles must be 1024-byte aligned");
@@ -755,7 +753,7 @@ gla_sum_tc(const Params p) {
   fetch_g(sm + L::kOffG, p.g, m.rows[0], ntok_first, tid);
   cp_async_commit();
   if (tid == 0) {
-    mbar_init(&m.mma, 1);
+    mbar_init(&m.mma, 2);
     mbar_fence_init();
   }
   if (warp == 0) {
@@ -824,9 +822,15 @@ gla_sum_tc(const Params p) {
     tc_before_sync();
     if (__syncthreads_or(failed)) break;
     tc_after_sync();
+    // two issuing threads (one MMA per ~60 cycles each): k^hi V into columns
+    // [0, 64), k^lo V into [64, 128)
     if (tid == 0) {
-      mma_terms<kStepMN, kStepMN>(tm, desc_mn(KH), desc_mn(KL), desc_mn(VH), desc_mn(VL), kV2, kIdKV,
-                                  it > 0);
+      mma_k64<kStepMN, kStepMN>(tm, desc_mn(KH), desc_mn(VH), kIdKV, it > 0);
+      if (kV2) mma_k64<kStepMN, kStepMN>(tm, desc_mn(KH), desc_mn(VL), kIdKV, true);
+      mma_commit(&m.mma);
+    }
+    if (tid == 128) {
+      mma_k64<kStepMN, kStepMN>(tm + 64, desc_mn(KL), desc_mn(VH), kIdKV, it > 0);
       mma_commit(&m.mma);
     }
   }
@@ -834,9 +838,12 @@ gla_sum_tc(const Params p) {
   tc_after_sync();
   cp_async_wait<0>();
   if (!failed) {
-    float ds[16];
+    float ds[16], dl[16];
     tmem_ld16x2(tm + lane_base + half * 32, ds);
+    tmem_ld16x2(tm + lane_base + 64 + half * 32, dl);
     tmem_ld_wait();
+#pragma unroll
+    for (int c = 0; c < 16; ++c) ds[c] += dl[c];
     float4* dst = reinterpret_cast<float4*>(p.wsS + (((size_t)bh * p.nseg + seg) * kD + row) * kD + cbase);
 #pragma unroll
     for (int c = 0; c < 4; ++c) dst[c] = make_float4(ds[4 * c], ds[4 * c + 1], ds[4 * c + 2], ds[4 * c + 3]);
