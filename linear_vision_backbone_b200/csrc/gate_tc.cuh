@@ -2,20 +2,23 @@
 //   g[n, j] = logsigmoid(sum_r (x[n,:] . W_down[:, r]) W_up[r, j] + b[j]) / tau
 // (GTR article, 方法详解 §1: a light low-rank projection with a temperature).
 //
-// One CTA (256 threads) per 128 tokens:
-//   * the x tile (128 rows x d_model, 16-bit, exact) arrives by 16-byte
-//     cp.async into a 128B-swizzled K-major tile;
+// One CTA (256 threads) per tile of up to 128 tokens (the host sizes tiles so
+// that there is about one per SM):
+//   * the x tile (16-bit, exact) arrives by 16-byte cp.async into a
+//     128B-swizzled K-major tile (M = 128 rows, rows past the tile zeroed);
 //   * W_down (rank 16) is split into terms of x's own type with a
 //     power-of-two scale per rank (fp16: hi + lo, bf16: hi + mid + lo), each
-//     thread holding its float4s in registers (all loads in flight at once),
-//     so x W_down is exact up to
-//     ~22-24 significant bits: low = sum_t x W_t (tcgen05.mma kind::f16,
-//     M = 128, N = 16, fp32 accumulators in TMEM);
+//     thread holding its float4s in registers (all loads in flight at once);
+//     the terms sit side by side along N, so one tcgen05.mma kind::f16 per
+//     K step (M = 128, N = 16 x terms) gives every x W_t, summed when read:
+//     x W_down exact up to ~22-24 significant bits;
 //   * low (fp32, per-row scaled) and W_up (per-column scaled) become two-term
 //     fp16 operands and u = low W_up is taken as hi*hi + hi*lo + lo*hi
 //     (M = 128, N = 64 per instruction);
 //   * the epilogue reads u from TMEM (thread = token row, warps 0-3 and 4-7
-//     on the two column halves), adds the bias and stores logsigmoid(u)/tau.
+//     on the two halves of each 64-column slab), adds the bias, forms
+//     logsigmoid(u)/tau into a shared-memory slab (the x tile's space, free
+//     by then) and writes each slab out with coalesced 16-byte stores.
 // The scales are exact powers of two and are undone on the fp32 accumulators;
 // they run along M or N only, so they factor out of every sum.
 #pragma once
@@ -84,6 +87,8 @@ struct Layout {
   static constexpr int kOffWu = kOffLow + 2 * kLow;        // 2 terms
   static constexpr int kOffMisc = kOffWu + 2 * kWu;
   static constexpr int kMiscBytes = 5120;
+  static constexpr int kSlabPitch = 64 * 4 + 16;           // staged g row: 64 floats + bank padding
+  static constexpr int kSlab = kM * kSlabPitch;             // two slabs fit in the x tile's space
   static constexpr int kSmem = kOffMisc + kMiscBytes + 1024;
 };
 
@@ -96,8 +101,10 @@ struct Misc {
   alignas(16) float wu_i[kMaxHD];    // inverse W_up column scales
   alignas(16) float low_i[kM];       // inverse row scales of low
   alignas(16) float wd_part[kThreads / 32][kRank];   // per-warp |W_down| maxima per rank
+  alignas(16) float bias[kMaxHD];
 };
 static_assert(sizeof(Misc) <= Layout::kMiscBytes, "Misc must fit its reserved bytes");
+static_assert(2 * Layout::kSlab <= Layout::kX, "two g slabs must fit in the x tile");
 
 // K-major 16-bit tile (rows x K), 128B-swizzled atoms of 8 rows x 64 elements;
 // atom columns (64 K-elements) `rows`*128 bytes apart.
@@ -137,7 +144,7 @@ template <typename TX>
 __global__ void __launch_bounds__(kThreads, 1)
 gate_proj_tc(const TX* __restrict__ x, const float* __restrict__ w_down, const float* __restrict__ w_up,
              const float* __restrict__ bias, float* __restrict__ g, long long N, int dm, int rank,
-             int HD, float inv_tau) {
+             int HD, float inv_tau, int tpc) {
   constexpr bool kBf16 = std::is_same<TX, __nv_bfloat16>::value;
   constexpr int kTerms = kBf16 ? 3 : 2;   // W_down terms in x's type
   extern __shared__ uint8_t smem_raw[];
@@ -148,8 +155,8 @@ gate_proj_tc(const TX* __restrict__ x, const float* __restrict__ w_down, const f
   uint8_t* tWu = sm + Layout::kOffWu;
   Misc& m = *reinterpret_cast<Misc*>(sm + Layout::kOffMisc);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const long long tok0 = (long long)blockIdx.x * kM;
-  const int ntok = (int)min((long long)kM, N - tok0);
+  const long long tok0 = (long long)blockIdx.x * tpc;
+  const int ntok = (int)min((long long)tpc, N - tok0);
 
   // ---- x tile: 16-byte pieces into the swizzled K-major tile (rows beyond ntok zero-filled)
   const int pieces = dm / 8;                      // 16-byte pieces per token row
@@ -170,6 +177,7 @@ gate_proj_tc(const TX* __restrict__ x, const float* __restrict__ w_down, const f
     tc::tmem_alloc(&m.tmem, 512);
     tc::tmem_relinquish();
   }
+  for (int j = tid; j < HD; j += kThreads) m.bias[j] = bias ? __ldg(bias + j) : 0.f;
   // ---- W_down [dm][16]: thread t holds the float4s t, t + 256, ... (ranks 4(t%4)..+3 of rows
   // (t + 256i)/4), all loads in flight at once; the rank maxima reduce over the lanes with the
   // same t%4 and then over the 8 warps.
@@ -225,7 +233,7 @@ gate_proj_tc(const TX* __restrict__ x, const float* __restrict__ w_down, const f
     }
   }
   __syncthreads();
-  // W_down^T terms (B of stage 1, K-major: rows = rank, columns = d_model)
+  // W_down^T terms (B of stage 1, K-major: row t * 16 + rank for term t, columns = d_model)
   {
     const float4 sc = *reinterpret_cast<const float4*>(&m.wd_s[(tid & 3) * 4]);
 #pragma unroll
@@ -236,11 +244,10 @@ gate_proj_tc(const TX* __restrict__ x, const float* __restrict__ w_down, const f
         float w4[4] = {wd[i].x * sc.x, wd[i].y * sc.y, wd[i].z * sc.z, wd[i].w * sc.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const uint32_t off = swk(n0 + e, c, kRank);
           float w = w4[e];
 #pragma unroll
           for (int t = 0; t < kTerms; ++t) {
-            Store16<TX>::put(tWd + t * Layout::kWd + off, w);
+            Store16<TX>::put(tWd + swk(t * kRank + n0 + e, c, kTerms * kRank), w);
             w -= Store16<TX>::back(w);
           }
         }
@@ -254,25 +261,32 @@ gate_proj_tc(const TX* __restrict__ x, const float* __restrict__ w_down, const f
   tc::tc_after_sync();
   const uint32_t tm = m.tmem;
 
-  // ---- stage 1: low = x W_down  (TMEM columns 0..15)
+  // ---- stage 1: x W_t for every term t at once (TMEM columns 16 t .. 16 t + 15)
   if (tid == 0) {
-    const uint32_t id = idesc16(kM, kRank, 0, 0, kBf16 ? 1 : 0);
+    constexpr int kN1 = kTerms * kRank;
+    const uint32_t id = idesc16(kM, kN1, 0, 0, kBf16 ? 1 : 0);
     const int ksteps = dm / 16;
-    for (int t = 0; t < kTerms; ++t)
-      for (int s = 0; s < ksteps; ++s) {
-        const uint64_t a = tc::sdesc(saddr(tX) + (s >> 2) * (kM * 128) + (s & 3) * 32, 16, 1024);
-        const uint64_t b = tc::sdesc(saddr(tWd) + t * Layout::kWd + (s >> 2) * (kRank * 128) + (s & 3) * 32, 16, 1024);
-        tc::mma_f16(tm + 0, a, b, id, (t > 0 || s > 0) ? 1u : 0u);
-      }
+    for (int s = 0; s < ksteps; ++s) {
+      const uint64_t a = tc::sdesc(saddr(tX) + (s >> 2) * (kM * 128) + (s & 3) * 32, 16, 1024);
+      const uint64_t b = tc::sdesc(saddr(tWd) + (s >> 2) * (kN1 * 128) + (s & 3) * 32, 16, 1024);
+      tc::mma_f16(tm + 0, a, b, id, s > 0 ? 1u : 0u);
+    }
     tc::mma_commit(&m.mma[0]);
   }
   bool ok = tc::mbar_wait(&m.mma[0], 0);
   tc::tc_after_sync();
   // low row r (warps 0-3, thread = row) -> per-row scaled two-term fp16 A tile (K = 16)
   if (warp < 4) {
-    float lw[16];
+    float lw[16], lt[16];
     tmem_ld16(tm + ((uint32_t)(warp * 32) << 16) + 0, lw);
     tc::tmem_ld_wait();
+#pragma unroll
+    for (int t = 1; t < kTerms; ++t) {
+      tmem_ld16(tm + ((uint32_t)(warp * 32) << 16) + t * kRank, lt);
+      tc::tmem_ld_wait();
+#pragma unroll
+      for (int c = 0; c < 16; ++c) lw[c] += lt[c];
+    }
     const int r = warp * 32 + lane;
     float mx = 0.f;
 #pragma unroll
@@ -310,30 +324,39 @@ gate_proj_tc(const TX* __restrict__ x, const float* __restrict__ w_down, const f
   tc::tc_after_sync();
   if (!ok && tid == 0) gtr_flag(kStatusMbarTimeout);
 
-  // ---- epilogue: thread = token row (lane quadrant warp % 4), warps w and w + 4 take the
-  // two halves of the columns; g = logsigmoid(u + b) / tau
+  // ---- epilogue, one 64-column slab of u at a time: thread = token row (TMEM
+  // lane quadrant warp % 4), warps w and w + 4 on the slab's two 32-column
+  // halves; g = logsigmoid(u + b) / tau goes to a shared-memory slab (two
+  // alternate, so one barrier per slab), which all threads then write out
+  // with coalesced 16-byte stores (16 threads per 256-byte row piece).
   {
-    const int r = (warp & 3) * 32 + lane;
-    const int half = warp >> 2, ncol = HD / 2, c0 = half * ncol;
+    const int q = warp & 3, hf = warp >> 2;
+    const int r = q * 32 + lane;
     const float ri = m.low_i[r];
-    float* grow = g + (tok0 + r) * HD;
-    for (int cb = 0; cb < ncol; cb += 16) {
-      float u[16];
-      tmem_ld16(tm + ((uint32_t)((warp & 3) * 32) << 16) + 64 + c0 + cb, u);
+    const uint32_t tq = tm + ((uint32_t)(q * 32) << 16) + 64 + 32 * hf;
+    const int nslab = HD / 64;
+    for (int j = 0; j < nslab; ++j) {
+      uint8_t* slab = tX + (j & 1) * Layout::kSlab;
+      float u[32];
+      tmem_ld16(tq + 64 * j, u);
+      tmem_ld16(tq + 64 * j + 16, u + 16);
       tc::tmem_ld_wait();
-      if (r < ntok) {
+      const int cb = 64 * j + 32 * hf;
 #pragma unroll
-        for (int c = 0; c < 16; c += 4) {
-          const int j = c0 + cb + c;
-          const float4 bb = bias ? *reinterpret_cast<const float4*>(bias + j) : make_float4(0.f, 0.f, 0.f, 0.f);
-          const float4 ci = *reinterpret_cast<const float4*>(&m.wu_i[j]);
-          *reinterpret_cast<float4*>(grow + j) = make_float4(
-              logsigmoid_fast(fmaf(u[c + 0] * ri, ci.x, bb.x)) * inv_tau,
-              logsigmoid_fast(fmaf(u[c + 1] * ri, ci.y, bb.y)) * inv_tau,
-              logsigmoid_fast(fmaf(u[c + 2] * ri, ci.z, bb.z)) * inv_tau,
-              logsigmoid_fast(fmaf(u[c + 3] * ri, ci.w, bb.w)) * inv_tau);
-        }
+      for (int c = 0; c < 32; c += 4) {
+        const float4 bb = *reinterpret_cast<const float4*>(&m.bias[cb + c]);
+        const float4 ci = *reinterpret_cast<const float4*>(&m.wu_i[cb + c]);
+        *reinterpret_cast<float4*>(slab + r * Layout::kSlabPitch + (32 * hf + c) * 4) = make_float4(
+            logsigmoid_fast(fmaf(u[c + 0] * ri, ci.x, bb.x)) * inv_tau,
+            logsigmoid_fast(fmaf(u[c + 1] * ri, ci.y, bb.y)) * inv_tau,
+            logsigmoid_fast(fmaf(u[c + 2] * ri, ci.z, bb.z)) * inv_tau,
+            logsigmoid_fast(fmaf(u[c + 3] * ri, ci.w, bb.w)) * inv_tau);
       }
+      __syncthreads();
+      const int piece = tid & 15;
+      for (int rr = tid >> 4; rr < ntok; rr += kThreads / 16)
+        *reinterpret_cast<float4*>(g + (tok0 + rr) * HD + 64 * j + piece * 4) =
+            *reinterpret_cast<const float4*>(slab + rr * Layout::kSlabPitch + piece * 16);
     }
   }
   tc::tc_before_sync();
@@ -345,7 +368,13 @@ gate_proj_tc(const TX* __restrict__ x, const float* __restrict__ w_down, const f
 }  // namespace gate_tc
 
 // Shapes the tensor-core gate kernel takes: 16-bit x, d_model a multiple of 64
-// up to 384, rank 16, H*dk a multiple of 64 up to 448.
+// up to 384, rank 16, H*dk a multiple of 64 up to 448.  Tokens per CTA: about
+// N / #SMs rounded up to a multiple of 16, at most 128.
+inline int gate_tc_tile(long long N, int sms) {
+  long long t = (N + sms - 1) / (sms > 0 ? sms : 1);
+  t = (t + 15) / 16 * 16;
+  return (int)(t < 16 ? 16 : t > gate_tc::kM ? gate_tc::kM : t);
+}
 inline bool gate_tc_supported(int x_dtype, int dm, int rank, int HD) {
   return (x_dtype == kF16 || x_dtype == kBF16) && dm % 64 == 0 && dm <= gate_tc::kMaxDm &&
          rank == gate_tc::kRank && HD % 64 == 0 && HD <= gate_tc::kMaxHD;

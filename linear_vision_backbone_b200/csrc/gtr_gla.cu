@@ -362,24 +362,25 @@ gtr_status_t gtr_gate_fwd(const void* x, int x_dtype, const float* w_down, const
   const int HD = H * dk;
   cudaStream_t st = (cudaStream_t)stream;
   if (gate_tc_supported(x_dtype, d_model, rank, HD) && (!bias || aligned16(bias))) {
-    // tensor-core kernel: one CTA per 128 tokens
-    const long long blocks = (N + gate_tc::kM - 1) / gate_tc::kM;
-    if (blocks > 0x7fffffffLL) return GTR_ERR_INVALID_ARG;
+    // tensor-core kernel: about one tile of tokens per SM
     int dev;
     if (int rc = current_device(&dev)) return (gtr_status_t)rc;
+    const int tpc = gate_tc_tile(N, sm_count(dev));
+    const long long blocks = (N + tpc - 1) / tpc;
+    if (blocks > 0x7fffffffLL) return GTR_ERR_INVALID_ARG;
     const float inv_tau = 1.0f / tau;
     if (x_dtype == GTR_F16) {
       static bool done[kMaxDevices];
       if (int rc = ensure_smem(gate_tc::gate_proj_tc<__half>, gate_tc::Layout::kSmem, done, dev))
         return (gtr_status_t)rc;
       gate_tc::gate_proj_tc<__half><<<(unsigned)blocks, gate_tc::kThreads, gate_tc::Layout::kSmem, st>>>(
-          (const __half*)x, w_down, w_up, bias, g_out, N, d_model, rank, HD, inv_tau);
+          (const __half*)x, w_down, w_up, bias, g_out, N, d_model, rank, HD, inv_tau, tpc);
     } else {
       static bool done[kMaxDevices];
       if (int rc = ensure_smem(gate_tc::gate_proj_tc<__nv_bfloat16>, gate_tc::Layout::kSmem, done, dev))
         return (gtr_status_t)rc;
       gate_tc::gate_proj_tc<__nv_bfloat16><<<(unsigned)blocks, gate_tc::kThreads, gate_tc::Layout::kSmem, st>>>(
-          (const __nv_bfloat16*)x, w_down, w_up, bias, g_out, N, d_model, rank, HD, inv_tau);
+          (const __nv_bfloat16*)x, w_down, w_up, bias, g_out, N, d_model, rank, HD, inv_tau, tpc);
     }
     return (gtr_status_t)launch_status();
   }
