@@ -158,6 +158,17 @@ gate_proj_tc(const TX* __restrict__ x, const float* __restrict__ w_down, const f
   const long long tok0 = (long long)blockIdx.x * tpc;
   const int ntok = (int)min((long long)tpc, N - tok0);
 
+  if (tid == 0) {
+    tc::mbar_init(&m.mma[0], 1);
+    tc::mbar_init(&m.mma[1], 1);
+    tc::mbar_fence_init();
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(&m.tmem, 512);
+    tc::tmem_relinquish();
+  }
+  pdl_wait();                                     // x and the weights may come from the previous kernel
+  pdl_trigger();
   // ---- x tile: 16-byte pieces into the swizzled K-major tile (rows beyond ntok zero-filled)
   const int pieces = dm / 8;                      // 16-byte pieces per token row
   for (int o = tid; o < kM * pieces; o += kThreads) {
@@ -168,15 +179,6 @@ gate_proj_tc(const TX* __restrict__ x, const float* __restrict__ w_down, const f
   }
   asm volatile("cp.async.commit_group;" ::: "memory");
 
-  if (tid == 0) {
-    tc::mbar_init(&m.mma[0], 1);
-    tc::mbar_init(&m.mma[1], 1);
-    tc::mbar_fence_init();
-  }
-  if (warp == 0) {
-    tc::tmem_alloc(&m.tmem, 512);
-    tc::tmem_relinquish();
-  }
   for (int j = tid; j < HD; j += kThreads) m.bias[j] = bias ? __ldg(bias + j) : 0.f;
   // ---- W_down [dm][16]: thread t holds the float4s t, t + 256, ... (ranks 4(t%4)..+3 of rows
   // (t + 256i)/4), all loads in flight at once; the rank maxima reduce over the lanes with the

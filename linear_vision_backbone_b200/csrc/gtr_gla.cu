@@ -222,9 +222,10 @@ int launch_stage(const Plan& p, const void* q, const void* k, const void* v, con
 int launch_scan(const Plan& p, float* wsS, const float* wsA, int inclusive, cudaStream_t st) {
   const long long total = (long long)p.B * p.H * p.dk * p.dv;
   const long long blocks = (total + kScanThreads - 1) / kScanThreads;
-  gla_state_scan<<<(unsigned)blocks, kScanThreads, 0, st>>>(wsS, wsA, total, p.nseg, p.dk, p.dv,
-                                                           inclusive);
-  return launch_status();
+  return launch_pdl(gla_state_scan, dim3((unsigned)blocks), dim3(kScanThreads), 0, st, wsS,
+                    (const float*)wsA, total, p.nseg, p.dk, p.dv, inclusive) == 0
+             ? GTR_OK
+             : GTR_ERR_CUDA;
 }
 
 // Record a caller event; inside stream capture it becomes an external event
@@ -373,14 +374,18 @@ gtr_status_t gtr_gate_fwd(const void* x, int x_dtype, const float* w_down, const
       static bool done[kMaxDevices];
       if (int rc = ensure_smem(gate_tc::gate_proj_tc<__half>, gate_tc::Layout::kSmem, done, dev))
         return (gtr_status_t)rc;
-      gate_tc::gate_proj_tc<__half><<<(unsigned)blocks, gate_tc::kThreads, gate_tc::Layout::kSmem, st>>>(
-          (const __half*)x, w_down, w_up, bias, g_out, N, d_model, rank, HD, inv_tau, tpc);
+      if (launch_pdl(gate_tc::gate_proj_tc<__half>, dim3((unsigned)blocks), dim3(gate_tc::kThreads),
+                     gate_tc::Layout::kSmem, st, (const __half*)x, w_down, w_up, bias, g_out, N,
+                     d_model, rank, HD, inv_tau, tpc))
+        return GTR_ERR_CUDA;
     } else {
       static bool done[kMaxDevices];
       if (int rc = ensure_smem(gate_tc::gate_proj_tc<__nv_bfloat16>, gate_tc::Layout::kSmem, done, dev))
         return (gtr_status_t)rc;
-      gate_tc::gate_proj_tc<__nv_bfloat16><<<(unsigned)blocks, gate_tc::kThreads, gate_tc::Layout::kSmem, st>>>(
-          (const __nv_bfloat16*)x, w_down, w_up, bias, g_out, N, d_model, rank, HD, inv_tau, tpc);
+      if (launch_pdl(gate_tc::gate_proj_tc<__nv_bfloat16>, dim3((unsigned)blocks),
+                     dim3(gate_tc::kThreads), gate_tc::Layout::kSmem, st, (const __nv_bfloat16*)x,
+                     w_down, w_up, bias, g_out, N, d_model, rank, HD, inv_tau, tpc))
+        return GTR_ERR_CUDA;
     }
     return (gtr_status_t)launch_status();
   }

@@ -25,6 +25,8 @@ constexpr int kScanGroup = 32;
 __global__ void __launch_bounds__(kScanThreads)
 gla_state_scan(float* __restrict__ wsS, const float* __restrict__ wsA, long long total, int nseg,
                int dk, int dv, int inclusive) {
+  pdl_wait();                             // the summaries are complete
+  pdl_trigger();
   const long long e = (long long)blockIdx.x * kScanThreads + threadIdx.x;
   if (e >= total) return;
   const int dkdv = dk * dv;

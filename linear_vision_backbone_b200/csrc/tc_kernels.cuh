@@ -439,6 +439,13 @@ gla_out_tc(const Params p) {
     fetch_chunk(sm, p, m.rows[0], ntok0, tid);
     cp_async_commit();
   }
+  if (tid < kD) m.wv[tid] = p.w ? p.w[tid] : 1.0f;
+  // Launched programmatically after the boundary scan, this block may start
+  // while the scan runs: q, k, v, g, z and w were complete before the summary
+  // stage passed its own wait (the scan starts its dependents only after
+  // that), so chunk 0 is fetched above; the boundary states need the wait.
+  pdl_wait();
+  pdl_trigger();
   // carried state: S[row][cbase .. cbase + 15], from the boundary scan
   float S[16];
   {
@@ -456,7 +463,6 @@ gla_out_tc(const Params p) {
     mbar_init(&m.mma[2], 1);
     mbar_fence_init();
   }
-  if (tid < kD) m.wv[tid] = p.w ? p.w[tid] : 1.0f;
   if (warp == 0) {
     tmem_alloc(&m.tmem, L::kTmemCols);
     tmem_relinquish();
@@ -748,6 +754,8 @@ gla_sum_tc(const Params p) {
   chunk_rows(p, m.rows[0], b, h, d, clast * kC, ntok_first, tid);
   if (nch > 1) chunk_rows(p, m.rows[1], b, h, d, (clast - 1) * kC, kC, tid);
   __syncthreads();
+  pdl_wait();                             // k, v, g may come from the previous kernel
+  pdl_trigger();
   fetch16(sm + L::kOffK, p.k, m.rows[0], ntok_first, tid);
   fetch16(sm + L::kOffV, p.v, m.rows[0], ntok_first, tid);
   fetch_g(sm + L::kOffG, p.g, m.rows[0], ntok_first, tid);
@@ -872,8 +880,7 @@ inline int launch_tc_kernel(K kern, int smem, const tc::Params& p, int BH, cudaS
       return -5;
     done[dev] = true;
   }
-  kern<<<dim3(p.nseg, BH), tc::kThreads, smem, st>>>(p);
-  return cudaGetLastError() == cudaSuccess ? 0 : -5;
+  return launch_pdl(kern, dim3(p.nseg, BH), dim3(tc::kThreads), smem, st, p);
 }
 
 // stage 0: segment summaries (K2); stage 1: segment outputs (K4)
