@@ -317,11 +317,13 @@ def run_ours(args, world, rank, local):
     stream = torch.cuda.Stream(device=dev)
     path = binding.path_for(wl.B, wl.H, wl.gh, wl.gw, wl.dk, wl.dv, args.chunk, host["q"].dtype)
 
+    gate = make_gate(binding, wl, params, host["x"].dtype)
+    torch.cuda.synchronize()
+
     def step(s, direction, evs=None):
         if evs is not None:
             record_external(evs[0], stream)
-        binding.gate_fwd(s["x"], params["w_down"], params["w_up"], params["bias"], wl.H, wl.dk,
-                         wl.tau, out=s["g"], stream=stream)
+        gate(s["x"], s["g"], stream)
         binding.gla_fwd(s["q"], s["k"], s["v"], s["g"], s["z"], params["w"], grid_h=wl.gh,
                         grid_w=wl.gw, direction=direction, chunk=args.chunk, out=s["out"],
                         stream=stream, events=None if evs is None else evs[1:])
@@ -480,6 +482,27 @@ def run_ours(args, world, rank, local):
         dist.destroy_process_group()
 
 
+def make_gate(binding, wl, params, x_dtype):
+    """The gate projection of a step.  The weights are static, so for the
+    tensor-core gate they are packed once here (outside any timed region) and
+    every step runs the packed forward; other shapes run gtr_gate_fwd."""
+    rank = params["w_down"].shape[1]
+    hd = wl.H * wl.dk
+    if (x_dtype in (torch.float16, torch.bfloat16) and rank == 16 and wl.d_model % 64 == 0
+            and wl.d_model <= 384 and hd % 64 == 0 and hd <= 448):
+        packed = binding.gate_pack(params["w_down"], params["w_up"], x_dtype, wl.H, wl.dk)
+
+        def gate(x, out, stream):
+            binding.gate_fwd_packed(x, packed, params["bias"], rank, wl.H, wl.dk, wl.tau,
+                                    out=out, stream=stream)
+        return gate
+
+    def gate(x, out, stream):
+        binding.gate_fwd(x, params["w_down"], params["w_up"], params["bias"], wl.H, wl.dk,
+                         wl.tau, out=out, stream=stream)
+    return gate
+
+
 def secondary_line(binding, dev, steps=2000):
     """The same step on the 640x640 workload (T = 1600), timed the same way."""
     wl = gin.WORKLOADS["640"]
@@ -492,10 +515,11 @@ def secondary_line(binding, dev, steps=2000):
         sets.append(s)
     params = {n: host[n].to(dev) for n in ("w_down", "w_up", "bias", "w")}
     stream = torch.cuda.Stream(device=dev)
+    gate = make_gate(binding, wl, params, host["x"].dtype)
+    torch.cuda.synchronize()
 
     def step(s, direction):
-        binding.gate_fwd(s["x"], params["w_down"], params["w_up"], params["bias"], wl.H, wl.dk,
-                         wl.tau, out=s["g"], stream=stream)
+        gate(s["x"], s["g"], stream)
         binding.gla_fwd(s["q"], s["k"], s["v"], s["g"], s["z"], params["w"], grid_h=wl.gh,
                         grid_w=wl.gw, direction=direction, chunk=64, out=s["out"], stream=stream)
 

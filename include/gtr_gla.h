@@ -101,10 +101,41 @@ GTR_API const char *gtr_status_string(int status);
  *           gtr_gla_fwd.  logsigmoid uses the overflow-free form
  *           min(u,0) - log1p(exp(-|u|)), so g <= 0 always.
  *   Limits: 1 <= rank <= 64, d_model <= 4096, H*dk <= 4096, tau > 0 finite.
+ *   For 16-bit x with the tensor-core shapes (see gtr_gate_pack) it packs the
+ *   weights into a buffer cached per (device, stream) -- allocated with
+ *   cudaMalloc by the first such call on a stream, which must not happen
+ *   during stream capture -- and runs gtr_gate_fwd_packed.
  */
 GTR_API gtr_status_t gtr_gate_fwd(const void *x, int x_dtype, const float *w_down, const float *w_up,
                           const float *bias, float *g_out, int B, int T, int d_model, int rank,
                           int H, int dk, float tau, void *stream);
+
+/*
+ * Packed gate weights for the tensor-core gate kernel.  The weights of a
+ * model are fixed while it runs, so their preparation (splitting W_down and
+ * W_up into the power-of-two-scaled multi-term 16-bit operand tiles the
+ * kernel multiplies, in its shared-memory byte layout) can be done once and
+ * reused by every gtr_gate_fwd_packed call.
+ *   gtr_gate_packed_bytes: size of a packed weight buffer.
+ *   gtr_gate_pack: w_down [d_model, 16] and w_up [16, H*dk] fp32 (as in
+ *     gtr_gate_fwd) -> `packed`, a caller-owned device buffer of at least
+ *     gtr_gate_packed_bytes() bytes, 16-byte aligned, written asynchronously
+ *     on `stream`.  x_dtype (GTR_F16 or GTR_BF16) is the type of the x it
+ *     will multiply.  Shapes: rank 16, d_model a multiple of 64 up to 384,
+ *     H*dk a multiple of 64 up to 448; others return GTR_ERR_UNSUPPORTED.
+ *   gtr_gate_fwd_packed: gtr_gate_fwd with packed weights (made for the same
+ *     x_dtype, d_model, rank, H, dk); additionally B*T < 2^31.
+ *   Errors: GTR_ERR_INVALID_ARG (NULL pointer, bad sizes), GTR_ERR_UNSUPPORTED
+ *   (shape), GTR_ERR_NO_MEMORY (packed_bytes too small), GTR_ERR_ALIGNMENT,
+ *   GTR_ERR_CUDA (launch or tensor-map failure).
+ */
+GTR_API size_t gtr_gate_packed_bytes(void);
+GTR_API gtr_status_t gtr_gate_pack(const float *w_down, const float *w_up, int x_dtype, int d_model,
+                           int rank, int H, int dk, void *packed, size_t packed_bytes,
+                           void *stream);
+GTR_API gtr_status_t gtr_gate_fwd_packed(const void *x, int x_dtype, const void *packed,
+                                 const float *bias, float *g_out, int B, int T, int d_model,
+                                 int rank, int H, int dk, float tau, void *stream);
 
 /*
  * Key-only GLA forward with the fused RMSNorm x SiLU output gate (GTR article

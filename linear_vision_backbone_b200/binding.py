@@ -26,7 +26,7 @@ EXPORTS = (
     "gtr_abi_version", "gtr_status_string", "gtr_gate_fwd", "gtr_gla_fwd", "gtr_gla_fwd_timed",
     "gtr_gla_chunk_states", "gtr_gla_workspace_bytes", "gtr_gla_set_workspace",
     "gtr_gla_set_path", "gtr_gla_path_for", "gtr_last_device_status", "gtr_gla_segment_chunks",
-    "gtr_gla_fwd_noalloc",
+    "gtr_gla_fwd_noalloc", "gtr_gate_packed_bytes", "gtr_gate_pack", "gtr_gate_fwd_packed",
 )
 
 _lock = threading.Lock()
@@ -65,6 +65,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
             "gtr_last_device_status": ([P, P], I),
             "gtr_gla_segment_chunks": ([I, I, I, I, I, I, I, I], I),
             "gtr_gla_fwd_noalloc": ([P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, P], I),
+            "gtr_gate_packed_bytes": ([], Z),
+            "gtr_gate_pack": ([P, P, I, I, I, I, I, P, Z, P], I),
+            "gtr_gate_fwd_packed": ([P, I, P, P, P, I, I, I, I, I, I, F, P], I),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -119,6 +122,42 @@ def gate_fwd(x: torch.Tensor, w_down: torch.Tensor, w_up: torch.Tensor,
     rc = load().gtr_gate_fwd(_ptr(x), DTYPE_IDS[x.dtype], _ptr(w_down), _ptr(w_up), _ptr(bias),
                              _ptr(out), B, T, dm, rank, H, dk, float(tau), _stream(stream))
     _check("gtr_gate_fwd", rc)
+    return out
+
+
+def gate_pack(w_down: torch.Tensor, w_up: torch.Tensor, x_dtype: torch.dtype, H: int, dk: int,
+              out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Packed gate weights for ``gate_fwd_packed`` (``gtr_gate_pack``): a uint8 device tensor."""
+    dm, rank = w_down.shape
+    _need(w_down, "w_down", torch.float32, (dm, rank))
+    _need(w_up, "w_up", torch.float32, (rank, H * dk))
+    nbytes = int(load().gtr_gate_packed_bytes())
+    if out is None:
+        out = torch.empty(nbytes, device=w_down.device, dtype=torch.uint8)
+    rc = load().gtr_gate_pack(_ptr(w_down), _ptr(w_up), DTYPE_IDS[x_dtype], dm, rank, H, dk,
+                              _ptr(out), out.numel(), _stream(stream))
+    _check("gtr_gate_pack", rc)
+    return out
+
+
+def gate_fwd_packed(x: torch.Tensor, packed: torch.Tensor, bias: Optional[torch.Tensor], rank: int,
+                    H: int, dk: int, tau: float = 16.0, out: Optional[torch.Tensor] = None,
+                    stream=None) -> torch.Tensor:
+    """``gate_fwd`` with weights packed by ``gate_pack`` (``gtr_gate_fwd_packed``)."""
+    _need(x, "x")
+    if x.dim() != 3:
+        raise ValueError("x must be [B, T, d_model]")
+    B, T, dm = x.shape
+    if packed.dtype != torch.uint8 or packed.device != x.device:
+        raise ValueError("packed must be a uint8 tensor on x's device")
+    if bias is not None:
+        _need(bias, "bias", torch.float32, (H * dk,))
+    if out is None:
+        out = torch.empty(B, T, H, dk, device=x.device, dtype=torch.float32)
+    _need(out, "out", torch.float32, (B, T, H, dk))
+    rc = load().gtr_gate_fwd_packed(_ptr(x), DTYPE_IDS[x.dtype], _ptr(packed), _ptr(bias), _ptr(out),
+                                    B, T, dm, rank, H, dk, float(tau), _stream(stream))
+    _check("gtr_gate_fwd_packed", rc)
     return out
 
 

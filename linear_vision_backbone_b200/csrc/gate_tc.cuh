@@ -2,26 +2,34 @@
 //   g[n, j] = logsigmoid(sum_r (x[n,:] . W_down[:, r]) W_up[r, j] + b[j]) / tau
 // (GTR article, 方法详解 §1: a light low-rank projection with a temperature).
 //
-// One CTA (256 threads) per tile of up to 128 tokens (the host sizes tiles so
-// that there is about one per SM):
-//   * the x tile (16-bit, exact) arrives by 16-byte cp.async into a
-//     128B-swizzled K-major tile (M = 128 rows, rows past the tile zeroed);
-//   * W_down (rank 16) is split into terms of x's own type with a
-//     power-of-two scale per rank (fp16: hi + lo, bf16: hi + mid + lo), each
-//     thread holding its float4s in registers (all loads in flight at once);
-//     the terms sit side by side along N, so one tcgen05.mma kind::f16 per
-//     K step (M = 128, N = 16 x terms) gives every x W_t, summed when read:
-//     x W_down exact up to ~22-24 significant bits;
-//   * low (fp32, per-row scaled) and W_up (per-column scaled) become two-term
-//     fp16 operands and u = low W_up is taken as hi*hi + hi*lo + lo*hi
-//     (M = 128, N = 64 per instruction);
-//   * the epilogue reads u from TMEM (thread = token row, warps 0-3 and 4-7
-//     on the two halves of each 64-column slab), adds the bias, forms
-//     logsigmoid(u)/tau into a shared-memory slab (the x tile's space, free
-//     by then) and writes each slab out with coalesced 16-byte stores.
+// Two kernels.
+//   gate_pack_tc  -- once per weight set: splits W_down and W_up into the
+//     operand tiles the forward kernel multiplies, in their shared-memory
+//     byte layout ("packed weights"), with the power-of-two scales:
+//       * W_down (rank 16) into terms of x's own type with a scale per rank
+//         (fp16: hi + lo, bf16: hi + mid + lo), the terms side by side along
+//         N, K-major: x W_down is exact up to ~22-24 significant bits;
+//       * W_up into two fp16 terms (hi + lo) with a scale per column, MN-major.
+//   gate_fwd_tc -- one CTA (512 threads) per tile of up to 128 tokens (about
+//     one tile per SM):
+//       * TMA (tensor map, 128B swizzle) loads the x tile straight into the
+//         K-major operand layout (rows past the tensor read as zero), and bulk
+//         copies bring the packed weights;
+//       * stage 1: one tcgen05.mma kind::f16 per K step (M = 128, N = 16 x
+//         terms) gives every x W_t; their sum, per-row scaled, becomes a
+//         two-term fp16 operand `low`;
+//       * stage 2: u = low W_up as hi*hi + hi*lo + lo*hi (N = 64 per
+//         instruction), fp32 in TMEM;
+//       * epilogue, one 64-column slab at a time: thread = token row (TMEM lane
+//         quadrant warp % 4), warps w, w+4, w+8, w+12 on the slab's four
+//         16-column quarters; logsigmoid(u + b)/tau goes into a 128B-swizzled
+//         shared-memory slab (the x tile's space, free by then) that TMA
+//         stores to g, so the stores cost the warps nothing.
 // The scales are exact powers of two and are undone on the fp32 accumulators;
 // they run along M or N only, so they factor out of every sum.
 #pragma once
+#include <cuda.h>
+
 #include <type_traits>
 
 #include "common.cuh"
@@ -56,7 +64,7 @@ __device__ __forceinline__ void put2(uint8_t* hi, uint8_t* lo, uint32_t off, flo
   *reinterpret_cast<uint2*>(hi + off) = H;
   *reinterpret_cast<uint2*>(lo + off) = L;
 }
-// 32 lanes x 32 bit, 16 consecutive columns: thread t of warp w <- lane 32w+t.
+// 32 lanes x 32 bit, 16 consecutive columns: thread t of warp w <- lane 32(w%4)+t.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
   uint32_t r[16];
   asm volatile(
@@ -70,11 +78,47 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-constexpr int kM = 128;               // tokens per CTA
-constexpr int kThreads = 256;
+// TMA: tiled 2-D copies through a tensor map (coordinates: x = innermost
+// element index, y = row), and their completion.
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3}], [%4];" ::"r"(saddr(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(saddr(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_store_2d(const void* map, int x, int y, const void* src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(map),
+               "r"(x), "r"(y), "r"(saddr(src))
+               : "memory");
+}
+// Untiled bulk copy global -> shared (16-byte aligned, size a multiple of 16).
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          saddr(dst)),
+      "l"(src), "r"(bytes), "r"(saddr(bar))
+      : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until at most N committed bulk stores still read shared memory / are in flight
+template <int N> __device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+template <int N> __device__ __forceinline__ void bulk_wait() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+
+constexpr int kM = 128;               // rows of the MMA tile (tokens per CTA <= kM)
+constexpr int kThreads = 512;
+constexpr int kPackThreads = 256;
 constexpr int kMaxDm = 384;           // d_model: multiple of 64, <= 384
 constexpr int kMaxHD = 448;           // H*dk: multiple of 64, <= 448
-constexpr int kRank = 16;             // the projection's N (rank <= 16, zero-padded)
+constexpr int kRank = 16;             // the projection's N (rank 16)
 
 struct Layout {
   static constexpr int kX = kM * kMaxDm * 2;               // x tile: 96 KB
@@ -86,25 +130,38 @@ struct Layout {
   static constexpr int kOffLow = kOffWd + 3 * kWd;         // 2 terms
   static constexpr int kOffWu = kOffLow + 2 * kLow;        // 2 terms
   static constexpr int kOffMisc = kOffWu + 2 * kWu;
-  static constexpr int kMiscBytes = 5120;
-  static constexpr int kSlabPitch = 64 * 4 + 16;           // staged g row: 64 floats + bank padding
-  static constexpr int kSlab = kM * kSlabPitch;             // two slabs fit in the x tile's space
+  static constexpr int kMiscBytes = 6144;
   static constexpr int kSmem = kOffMisc + kMiscBytes + 1024;
+  static constexpr int kHalfSlab = kM * 128;               // 32 fp32 columns x 128 rows, 128B-swizzled
 };
+// Packed weights in global memory: the W_down and W_up term regions in their
+// shared-memory byte layout, then the inverse scales (W_down per rank, W_up
+// per column).
+struct Pack {
+  static constexpr int kOffWd = 0;
+  static constexpr int kWdBytes = 3 * Layout::kWd;
+  static constexpr int kOffWu = kOffWd + kWdBytes;
+  static constexpr int kWuBytes = 2 * Layout::kWu;
+  static constexpr int kOffScale = kOffWu + kWuBytes;
+  static constexpr int kScaleBytes = (kRank + kMaxHD) * 4;
+  static constexpr int kBytes = kOffScale + kScaleBytes;
+  static constexpr int kSmem = kBytes + 1024;                // the pack kernel's image + alignment slack
+};
+static_assert(Pack::kBytes % 16 == 0 && Pack::kScaleBytes % 16 == 0, "bulk copies move 16-byte multiples");
 
 struct Misc {
   uint64_t mma[2];
+  uint64_t ld;                       // the x tile and the packed weights
   uint32_t tmem;
   int pad;
-  alignas(16) float wd_s[kRank];     // W_down rank scales 2^e (and their inverses)
-  alignas(16) float wd_i[kRank];
-  alignas(16) float wu_i[kMaxHD];    // inverse W_up column scales
+  alignas(16) float wd_i[kRank];     // inverse W_down rank scales; wu_i follows (one bulk copy)
+  float wu_i[kMaxHD];                // inverse W_up column scales
   alignas(16) float low_i[kM];       // inverse row scales of low
-  alignas(16) float wd_part[kThreads / 32][kRank];   // per-warp |W_down| maxima per rank
   alignas(16) float bias[kMaxHD];
 };
 static_assert(sizeof(Misc) <= Layout::kMiscBytes, "Misc must fit its reserved bytes");
-static_assert(2 * Layout::kSlab <= Layout::kX, "two g slabs must fit in the x tile");
+static_assert(offsetof(Misc, wu_i) == offsetof(Misc, wd_i) + kRank * 4, "scales are one block");
+static_assert(4 * Layout::kHalfSlab <= Layout::kX, "two staged slabs must fit in the x tile");
 
 // K-major 16-bit tile (rows x K), 128B-swizzled atoms of 8 rows x 64 elements;
 // atom columns (64 K-elements) `rows`*128 bytes apart.
@@ -122,11 +179,6 @@ __host__ __device__ constexpr uint32_t idesc16(int M, int N, int a_mn, int b_mn,
   return (1u << 4) | ((uint32_t)bf16 << 7) | ((uint32_t)bf16 << 10) | ((uint32_t)a_mn << 15) |
          ((uint32_t)b_mn << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
-__device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr(dst)), "l"(src),
-               "r"(valid ? 16 : 0)
-               : "memory");
-}
 
 template <typename T> struct Store16;
 template <> struct Store16<__half> {
@@ -140,56 +192,34 @@ template <> struct Store16<__nv_bfloat16> {
   static __device__ __forceinline__ float back(float v) { return __bfloat162float(__float2bfloat16_rn(v)); }
 };
 
+// ------------------------------------------------------------- weight pack
 template <typename TX>
-__global__ void __launch_bounds__(kThreads, 1)
-gate_proj_tc(const TX* __restrict__ x, const float* __restrict__ w_down, const float* __restrict__ w_up,
-             const float* __restrict__ bias, float* __restrict__ g, long long N, int dm, int rank,
-             int HD, float inv_tau, int tpc) {
-  constexpr bool kBf16 = std::is_same<TX, __nv_bfloat16>::value;
-  constexpr int kTerms = kBf16 ? 3 : 2;   // W_down terms in x's type
+__global__ void __launch_bounds__(kPackThreads, 1)
+gate_pack_tc(const float* __restrict__ w_down, const float* __restrict__ w_up, int dm, int HD,
+             uint8_t* __restrict__ pack) {
+  constexpr int kTerms = std::is_same<TX, __nv_bfloat16>::value ? 3 : 2;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* tX = sm + Layout::kOffX;
-  uint8_t* tWd = sm + Layout::kOffWd;
-  uint8_t* tLow = sm + Layout::kOffLow;
-  uint8_t* tWu = sm + Layout::kOffWu;
-  Misc& m = *reinterpret_cast<Misc*>(sm + Layout::kOffMisc);
+  uint8_t* img = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);   // Pack::kBytes
+  uint8_t* tWd = img + Pack::kOffWd;
+  uint8_t* tWu = img + Pack::kOffWu;
+  float* wd_i = reinterpret_cast<float*>(img + Pack::kOffScale);
+  float* wu_i = wd_i + kRank;
+  __shared__ float wd_part[kPackThreads / 32][kRank];
+  __shared__ float wd_s[kRank];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const long long tok0 = (long long)blockIdx.x * tpc;
-  const int ntok = (int)min((long long)tpc, N - tok0);
-
-  if (tid == 0) {
-    tc::mbar_init(&m.mma[0], 1);
-    tc::mbar_init(&m.mma[1], 1);
-    tc::mbar_fence_init();
-  }
-  if (warp == 0) {
-    tc::tmem_alloc(&m.tmem, 512);
-    tc::tmem_relinquish();
-  }
-  pdl_wait();                                     // x and the weights may come from the previous kernel
+  pdl_wait();                                     // the weights may come from the previous kernel
   pdl_trigger();
-  // ---- x tile: 16-byte pieces into the swizzled K-major tile (rows beyond ntok zero-filled)
-  const int pieces = dm / 8;                      // 16-byte pieces per token row
-  for (int o = tid; o < kM * pieces; o += kThreads) {
-    const int r = o / pieces, c = (o - r * pieces) * 8;
-    const bool valid = r < ntok;
-    const TX* src = valid ? x + (tok0 + r) * dm + c : x;
-    cp_async16_zfill(tX + swk(r, c, kM), src, valid);
-  }
-  asm volatile("cp.async.commit_group;" ::: "memory");
-
-  for (int j = tid; j < HD; j += kThreads) m.bias[j] = bias ? __ldg(bias + j) : 0.f;
-  // ---- W_down [dm][16]: thread t holds the float4s t, t + 256, ... (ranks 4(t%4)..+3 of rows
-  // (t + 256i)/4), all loads in flight at once; the rank maxima reduce over the lanes with the
-  // same t%4 and then over the 8 warps.
-  constexpr int kWdVec = kMaxDm * kRank / 4 / kThreads;     // float4s per thread at most (6)
+  // zero the image (regions beyond d_model / H*dk are never read, but are copied)
+  for (int o = tid; o < Pack::kBytes / 16; o += kPackThreads)
+    reinterpret_cast<uint4*>(img)[o] = make_uint4(0u, 0u, 0u, 0u);
+  // W_down [dm][16]: thread t holds float4s t, t + 256, ... (ranks 4(t%4)..+3 of rows (t+256i)/4)
+  constexpr int kWdVec = kMaxDm * kRank / 4 / kPackThreads;
   const int nwd = dm * kRank / 4;
   float4 wd[kWdVec];
   float4 wmx = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
   for (int i = 0; i < kWdVec; ++i) {
-    const int idx = tid + i * kThreads;
+    const int idx = tid + i * kPackThreads;
     wd[i] = idx < nwd ? __ldg(reinterpret_cast<const float4*>(w_down) + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
     wmx = make_float4(fmaxf(wmx.x, fabsf(wd[i].x)), fmaxf(wmx.y, fabsf(wd[i].y)),
                       fmaxf(wmx.z, fabsf(wd[i].z)), fmaxf(wmx.w, fabsf(wd[i].w)));
@@ -201,49 +231,45 @@ gate_proj_tc(const TX* __restrict__ x, const float* __restrict__ w_down, const f
     wmx.z = fmaxf(wmx.z, __shfl_xor_sync(0xffffffffu, wmx.z, o));
     wmx.w = fmaxf(wmx.w, __shfl_xor_sync(0xffffffffu, wmx.w, o));
   }
-  if (lane < 4) *reinterpret_cast<float4*>(&m.wd_part[warp][lane * 4]) = wmx;
-  // ---- W_up [16][HD]: thread t < HD/4 holds column quad t of all 16 ranks
-  const int nq = HD / 4;
-  float4 wu[kRank];
-  if (tid < nq) {
-#pragma unroll
-    for (int k = 0; k < kRank; ++k) wu[k] = __ldg(reinterpret_cast<const float4*>(w_up + (size_t)k * HD) + tid);
-  }
-  __syncthreads();
+  if (lane < 4) *reinterpret_cast<float4*>(&wd_part[warp][lane * 4]) = wmx;
+  __syncthreads();                                // also orders the zeroing before the writes below
   if (tid < kRank) {
     float mx = 0.f;
 #pragma unroll
-    for (int w8 = 0; w8 < kThreads / 32; ++w8) mx = fmaxf(mx, m.wd_part[w8][tid]);
+    for (int w8 = 0; w8 < kPackThreads / 32; ++w8) mx = fmaxf(mx, wd_part[w8][tid]);
     const int e = scale_exp(mx);
-    m.wd_s[tid] = pow2i(e);
-    m.wd_i[tid] = pow2i(-e);
+    wd_s[tid] = pow2i(e);
+    wd_i[tid] = pow2i(-e);
   }
-  if (tid < nq) {
+  // W_up [16][HD]: thread t < HD/4 handles column quad t of all 16 ranks; fp16 hi + lo,
+  // per-column scales (B of stage 2, MN-major: rows = rank (K), columns = H*dk)
+  for (int qd = tid; qd < HD / 4; qd += kPackThreads) {
+    float4 wu[kRank];
+#pragma unroll
+    for (int k = 0; k < kRank; ++k) wu[k] = __ldg(reinterpret_cast<const float4*>(w_up + (size_t)k * HD) + qd);
     float4 cm = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int k = 0; k < kRank; ++k)
       cm = make_float4(fmaxf(cm.x, fabsf(wu[k].x)), fmaxf(cm.y, fabsf(wu[k].y)),
                        fmaxf(cm.z, fabsf(wu[k].z)), fmaxf(cm.w, fabsf(wu[k].w)));
     const int e0 = scale_exp(cm.x), e1 = scale_exp(cm.y), e2 = scale_exp(cm.z), e3 = scale_exp(cm.w);
-    *reinterpret_cast<float4*>(&m.wu_i[4 * tid]) = make_float4(pow2i(-e0), pow2i(-e1), pow2i(-e2), pow2i(-e3));
+    *reinterpret_cast<float4*>(&wu_i[4 * qd]) = make_float4(pow2i(-e0), pow2i(-e1), pow2i(-e2), pow2i(-e3));
     const float s0 = pow2i(e0), s1 = pow2i(e1), s2 = pow2i(e2), s3 = pow2i(e3);
-    // W_up terms (B of stage 2, MN-major: rows = rank (K), columns = H*dk), fp16 hi + lo
 #pragma unroll
-    for (int k = 0; k < kRank; ++k) {
-      const uint32_t off = swmn(k, 4 * tid, kRank);
-      put2(tWu, tWu + Layout::kWu, off, wu[k].x * s0, wu[k].y * s1, wu[k].z * s2, wu[k].w * s3);
-    }
+    for (int k = 0; k < kRank; ++k)
+      put2(tWu, tWu + Layout::kWu, swmn(k, 4 * qd, kRank), wu[k].x * s0, wu[k].y * s1, wu[k].z * s2,
+           wu[k].w * s3);
   }
   __syncthreads();
   // W_down^T terms (B of stage 1, K-major: row t * 16 + rank for term t, columns = d_model)
   {
-    const float4 sc = *reinterpret_cast<const float4*>(&m.wd_s[(tid & 3) * 4]);
+    const float4 sc = *reinterpret_cast<const float4*>(&wd_s[(tid & 3) * 4]);
 #pragma unroll
     for (int i = 0; i < kWdVec; ++i) {
-      const int idx = tid + i * kThreads;
+      const int idx = tid + i * kPackThreads;
       if (idx < nwd) {
         const int c = idx >> 2, n0 = (idx & 3) * 4;
-        float w4[4] = {wd[i].x * sc.x, wd[i].y * sc.y, wd[i].z * sc.z, wd[i].w * sc.w};
+        const float w4[4] = {wd[i].x * sc.x, wd[i].y * sc.y, wd[i].z * sc.z, wd[i].w * sc.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           float w = w4[e];
@@ -256,10 +282,57 @@ gate_proj_tc(const TX* __restrict__ x, const float* __restrict__ w_down, const f
       }
     }
   }
-  asm volatile("cp.async.wait_group 0;" ::: "memory");
-  tc::fence_async_smem();
+  __syncthreads();
+  for (int o = tid; o < Pack::kBytes / 16; o += kPackThreads)
+    reinterpret_cast<uint4*>(pack)[o] = reinterpret_cast<const uint4*>(img)[o];
+}
+
+// --------------------------------------------------------------- forward
+// tmx: x as [N rows][dm] 16-bit, box 64 x 128, 128B swizzle.  tmg: g as
+// [N rows][HD] fp32, box 32 x tpc, 128B swizzle.
+template <typename TX>
+__global__ void __launch_bounds__(kThreads, 1)
+gate_fwd_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmg,
+            const uint8_t* __restrict__ pack, const float* __restrict__ bias, int dm, int HD,
+            float inv_tau, int tpc) {
+  constexpr bool kBf16 = std::is_same<TX, __nv_bfloat16>::value;
+  constexpr int kTerms = kBf16 ? 3 : 2;   // W_down terms in x's type
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* tX = sm + Layout::kOffX;
+  uint8_t* tWd = sm + Layout::kOffWd;
+  uint8_t* tLow = sm + Layout::kOffLow;
+  uint8_t* tWu = sm + Layout::kOffWu;
+  Misc& m = *reinterpret_cast<Misc*>(sm + Layout::kOffMisc);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tok0 = blockIdx.x * tpc;
+
+  if (tid == 0) {
+    tc::mbar_init(&m.ld, 1);
+    tc::mbar_init(&m.mma[0], 1);
+    tc::mbar_init(&m.mma[1], 1);
+    tc::mbar_fence_init();
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(&m.tmem, 512);
+    tc::tmem_relinquish();
+  }
   tc::tc_before_sync();
   __syncthreads();
+  tc::tc_after_sync();
+  pdl_wait();                                     // x and the packed weights may come from the previous kernel
+  pdl_trigger();
+  const int natoms = dm / 64;
+  if (tid == 0) {
+    mbar_expect_tx(&m.ld, (uint32_t)(natoms * (kM * 128) + Pack::kWdBytes + Pack::kWuBytes + Pack::kScaleBytes));
+    for (int a = 0; a < natoms; ++a) tma_load_2d(tX + a * (kM * 128), &tmx, a * 64, tok0, &m.ld);
+    bulk_g2s(tWd, pack + Pack::kOffWd, Pack::kWdBytes, &m.ld);
+    bulk_g2s(tWu, pack + Pack::kOffWu, Pack::kWuBytes, &m.ld);
+    bulk_g2s(&m.wd_i[0], pack + Pack::kOffScale, Pack::kScaleBytes, &m.ld);
+  }
+  for (int j = tid; j < HD; j += kThreads) m.bias[j] = bias ? __ldg(bias + j) : 0.f;
+  __syncthreads();
+  bool ok = tc::mbar_wait(&m.ld, 0);
   tc::tc_after_sync();
   const uint32_t tm = m.tmem;
 
@@ -275,7 +348,7 @@ gate_proj_tc(const TX* __restrict__ x, const float* __restrict__ w_down, const f
     }
     tc::mma_commit(&m.mma[0]);
   }
-  bool ok = tc::mbar_wait(&m.mma[0], 0);
+  ok &= tc::mbar_wait(&m.mma[0], 0);
   tc::tc_after_sync();
   // low row r (warps 0-3, thread = row) -> per-row scaled two-term fp16 A tile (K = 16)
   if (warp < 4) {
@@ -302,7 +375,7 @@ gate_proj_tc(const TX* __restrict__ x, const float* __restrict__ w_down, const f
 #pragma unroll
     for (int c = 0; c < 16; c += 4)
       put2(tLow, tLow + Layout::kLow, swk(r, c, kM), lw[c] * s, lw[c + 1] * s, lw[c + 2] * s,
-               lw[c + 3] * s);
+           lw[c + 3] * s);
   }
   tc::fence_async_smem();
   tc::tc_before_sync();
@@ -324,42 +397,49 @@ gate_proj_tc(const TX* __restrict__ x, const float* __restrict__ w_down, const f
   }
   ok &= tc::mbar_wait(&m.mma[1], 0);
   tc::tc_after_sync();
+  ok = __syncthreads_and(ok) != 0;                // block-uniform: the epilogue has barriers
   if (!ok && tid == 0) gtr_flag(kStatusMbarTimeout);
 
   // ---- epilogue, one 64-column slab of u at a time: thread = token row (TMEM
-  // lane quadrant warp % 4), warps w and w + 4 on the slab's two 32-column
-  // halves; g = logsigmoid(u + b) / tau goes to a shared-memory slab (two
-  // alternate, so one barrier per slab), which all threads then write out
-  // with coalesced 16-byte stores (16 threads per 256-byte row piece).
-  {
-    const int q = warp & 3, hf = warp >> 2;
+  // lane quadrant warp % 4), warp w on the slab's 16-column quarter w / 4.  Each
+  // slab is staged as two 32-column halves (128-byte rows, 16-byte units XOR-ed
+  // with row % 8: the TMA 128B swizzle) and TMA-stored; two slabs alternate.
+  if (ok) {
+    const int q = warp & 3, qp = warp >> 2;
     const int r = q * 32 + lane;
     const float ri = m.low_i[r];
-    const uint32_t tq = tm + ((uint32_t)(q * 32) << 16) + 64 + 32 * hf;
+    const uint32_t tq = tm + ((uint32_t)(q * 32) << 16) + 64 + 16 * qp;
     const int nslab = HD / 64;
     for (int j = 0; j < nslab; ++j) {
-      uint8_t* slab = tX + (j & 1) * Layout::kSlab;
-      float u[32];
+      uint8_t* slab = tX + (j & 1) * (2 * Layout::kHalfSlab);
+      // the store issued from this buffer two slabs ago has read it
+      if (tid == 0 && j >= 2) bulk_wait_read<1>();
+      __syncthreads();
+      float u[16];
       tmem_ld16(tq + 64 * j, u);
-      tmem_ld16(tq + 64 * j + 16, u + 16);
       tc::tmem_ld_wait();
-      const int cb = 64 * j + 32 * hf;
+      const int cb = 64 * j + 16 * qp;
+      uint8_t* half = slab + (qp >> 1) * Layout::kHalfSlab + r * 128;
 #pragma unroll
-      for (int c = 0; c < 32; c += 4) {
+      for (int c = 0; c < 16; c += 4) {
         const float4 bb = *reinterpret_cast<const float4*>(&m.bias[cb + c]);
         const float4 ci = *reinterpret_cast<const float4*>(&m.wu_i[cb + c]);
-        *reinterpret_cast<float4*>(slab + r * Layout::kSlabPitch + (32 * hf + c) * 4) = make_float4(
+        const int unit = (qp & 1) * 4 + (c >> 2);
+        *reinterpret_cast<float4*>(half + ((unit ^ (r & 7)) << 4)) = make_float4(
             logsigmoid_fast(fmaf(u[c + 0] * ri, ci.x, bb.x)) * inv_tau,
             logsigmoid_fast(fmaf(u[c + 1] * ri, ci.y, bb.y)) * inv_tau,
             logsigmoid_fast(fmaf(u[c + 2] * ri, ci.z, bb.z)) * inv_tau,
             logsigmoid_fast(fmaf(u[c + 3] * ri, ci.w, bb.w)) * inv_tau);
       }
+      tc::fence_async_smem();                     // these writes, then the TMA engine's reads
       __syncthreads();
-      const int piece = tid & 15;
-      for (int rr = tid >> 4; rr < ntok; rr += kThreads / 16)
-        *reinterpret_cast<float4*>(g + (tok0 + rr) * HD + 64 * j + piece * 4) =
-            *reinterpret_cast<const float4*>(slab + rr * Layout::kSlabPitch + piece * 16);
+      if (tid == 0) {
+        tma_store_2d(&tmg, 64 * j, tok0, slab);
+        tma_store_2d(&tmg, 64 * j + 32, tok0, slab + Layout::kHalfSlab);
+        bulk_commit();
+      }
     }
+    if (tid == 0) bulk_wait<0>();                 // every store done before the block ends
   }
   tc::tc_before_sync();
   __syncthreads();
@@ -369,17 +449,17 @@ gate_proj_tc(const TX* __restrict__ x, const float* __restrict__ w_down, const f
 
 }  // namespace gate_tc
 
-// Shapes the tensor-core gate kernel takes: 16-bit x, d_model a multiple of 64
-// up to 384, rank 16, H*dk a multiple of 64 up to 448.  Tokens per CTA: about
-// N / #SMs rounded up to a multiple of 16, at most 128.
+// Shapes the tensor-core gate kernels take: 16-bit x, d_model a multiple of 64
+// up to 384, rank 16, H*dk a multiple of 64 up to 448.
+inline bool gate_tc_supported(int x_dtype, int dm, int rank, int HD) {
+  return (x_dtype == kF16 || x_dtype == kBF16) && dm % 64 == 0 && dm <= gate_tc::kMaxDm &&
+         rank == gate_tc::kRank && HD % 64 == 0 && HD <= gate_tc::kMaxHD;
+}
+// Tokens per CTA: about N / #SMs rounded up to a multiple of 16, at most 128.
 inline int gate_tc_tile(long long N, int sms) {
   long long t = (N + sms - 1) / (sms > 0 ? sms : 1);
   t = (t + 15) / 16 * 16;
   return (int)(t < 16 ? 16 : t > gate_tc::kM ? gate_tc::kM : t);
-}
-inline bool gate_tc_supported(int x_dtype, int dm, int rank, int HD) {
-  return (x_dtype == kF16 || x_dtype == kBF16) && dm % 64 == 0 && dm <= gate_tc::kMaxDm &&
-         rank == gate_tc::kRank && HD % 64 == 0 && HD <= gate_tc::kMaxHD;
 }
 
 }  // namespace gtr

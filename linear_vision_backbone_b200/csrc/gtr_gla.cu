@@ -153,6 +153,8 @@ int launch_status() {
   return cudaGetLastError() == cudaSuccess ? GTR_OK : GTR_ERR_CUDA;
 }
 
+
+
 // cudaFuncSetAttribute once per kernel instance and device.
 template <typename K>
 int ensure_smem(K kern, size_t smem, bool* done, int dev) {
@@ -160,6 +162,105 @@ int ensure_smem(K kern, size_t smem, bool* done, int dev) {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return GTR_ERR_CUDA;
   done[dev] = true;
+  return GTR_OK;
+}
+
+// ---- TMA tensor maps (encoded on the host through the driver entry point)
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled() {
+  static std::atomic<EncodeTiledFn> fn{nullptr};
+  EncodeTiledFn f = fn.load();
+  if (!f) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess && p) {
+      f = (EncodeTiledFn)p;
+      fn.store(f);
+    } else {
+      (void)cudaGetLastError();
+    }
+  }
+  return f;
+}
+// 2-D row-major tensor [rows][cols] with the given row pitch, box box_cols x
+// box_rows, 128-byte swizzle, out-of-range elements read as zero.
+int tmap_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, unsigned long long rows,
+            unsigned long long cols, unsigned long long pitch_bytes, unsigned box_cols, unsigned box_rows) {
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) return GTR_ERR_CUDA;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {pitch_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? GTR_OK : GTR_ERR_CUDA;
+}
+
+// ---- tensor-core gate: weight packing and the forward pass
+int gate_pack_launch(int x_dtype, const float* w_down, const float* w_up, int dm, int HD, void* pack,
+                     cudaStream_t st, int dev) {
+  static bool done_h[kMaxDevices], done_b[kMaxDevices];
+  if (x_dtype == GTR_F16) {
+    if (int rc = ensure_smem(gate_tc::gate_pack_tc<__half>, gate_tc::Pack::kSmem, done_h, dev)) return rc;
+    return launch_pdl(gate_tc::gate_pack_tc<__half>, dim3(1), dim3(gate_tc::kPackThreads),
+                      gate_tc::Pack::kSmem, st, w_down, w_up, dm, HD, (uint8_t*)pack)
+               ? GTR_ERR_CUDA
+               : GTR_OK;
+  }
+  if (int rc = ensure_smem(gate_tc::gate_pack_tc<__nv_bfloat16>, gate_tc::Pack::kSmem, done_b, dev)) return rc;
+  return launch_pdl(gate_tc::gate_pack_tc<__nv_bfloat16>, dim3(1), dim3(gate_tc::kPackThreads),
+                    gate_tc::Pack::kSmem, st, w_down, w_up, dm, HD, (uint8_t*)pack)
+             ? GTR_ERR_CUDA
+             : GTR_OK;
+}
+int gate_fwd_packed_launch(int x_dtype, const void* x, const void* pack, const float* bias, float* g,
+                           long long N, int dm, int HD, float tau, cudaStream_t st, int dev) {
+  const int tpc = gate_tc_tile(N, sm_count(dev));
+  const long long blocks = (N + tpc - 1) / tpc;
+  CUtensorMap tmx, tmg;
+  const CUtensorMapDataType xdt =
+      x_dtype == GTR_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (int rc = tmap_2d(&tmx, xdt, x, (unsigned long long)N, (unsigned long long)dm,
+                       (unsigned long long)dm * 2, 64, gate_tc::kM))
+    return rc;
+  if (int rc = tmap_2d(&tmg, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, g, (unsigned long long)N,
+                       (unsigned long long)HD, (unsigned long long)HD * 4, 32, (unsigned)tpc))
+    return rc;
+  const float inv_tau = 1.0f / tau;
+  static bool done_h[kMaxDevices], done_b[kMaxDevices];
+  if (x_dtype == GTR_F16) {
+    if (int rc = ensure_smem(gate_tc::gate_fwd_tc<__half>, gate_tc::Layout::kSmem, done_h, dev)) return rc;
+    return launch_pdl(gate_tc::gate_fwd_tc<__half>, dim3((unsigned)blocks), dim3(gate_tc::kThreads),
+                      gate_tc::Layout::kSmem, st, tmx, tmg, (const uint8_t*)pack, bias, dm, HD, inv_tau, tpc)
+               ? GTR_ERR_CUDA
+               : GTR_OK;
+  }
+  if (int rc = ensure_smem(gate_tc::gate_fwd_tc<__nv_bfloat16>, gate_tc::Layout::kSmem, done_b, dev)) return rc;
+  return launch_pdl(gate_tc::gate_fwd_tc<__nv_bfloat16>, dim3((unsigned)blocks), dim3(gate_tc::kThreads),
+                    gate_tc::Layout::kSmem, st, tmx, tmg, (const uint8_t*)pack, bias, dm, HD, inv_tau, tpc)
+             ? GTR_ERR_CUDA
+             : GTR_OK;
+}
+// Per-(device, stream) buffer for the packed weights gtr_gate_fwd makes each call.
+std::map<std::pair<int, void*>, void*> g_pack_ws;
+int pack_workspace(int dev, void* stream, void** out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto key = std::make_pair(dev, stream);
+  auto it = g_pack_ws.find(key);
+  if (it != g_pack_ws.end()) { *out = it->second; return GTR_OK; }
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing((cudaStream_t)stream, &cs) != cudaSuccess) return GTR_ERR_CUDA;
+  if (cs != cudaStreamCaptureStatusNone) return GTR_ERR_NO_MEMORY;
+  void* p = nullptr;
+  if (cudaMalloc(&p, gate_tc::Pack::kBytes) != cudaSuccess) { (void)cudaGetLastError(); return GTR_ERR_NO_MEMORY; }
+  g_pack_ws[key] = p;
+  *out = p;
   return GTR_OK;
 }
 
@@ -362,32 +463,15 @@ gtr_status_t gtr_gate_fwd(const void* x, int x_dtype, const float* w_down, const
     return GTR_ERR_ALIGNMENT;
   const int HD = H * dk;
   cudaStream_t st = (cudaStream_t)stream;
-  if (gate_tc_supported(x_dtype, d_model, rank, HD) && (!bias || aligned16(bias))) {
-    // tensor-core kernel: about one tile of tokens per SM
+  if (gate_tc_supported(x_dtype, d_model, rank, HD) && N < (1LL << 31)) {
+    // tensor-core kernels: pack the weights into this stream's buffer, then
+    // the forward pass (about one tile of tokens per SM)
     int dev;
     if (int rc = current_device(&dev)) return (gtr_status_t)rc;
-    const int tpc = gate_tc_tile(N, sm_count(dev));
-    const long long blocks = (N + tpc - 1) / tpc;
-    if (blocks > 0x7fffffffLL) return GTR_ERR_INVALID_ARG;
-    const float inv_tau = 1.0f / tau;
-    if (x_dtype == GTR_F16) {
-      static bool done[kMaxDevices];
-      if (int rc = ensure_smem(gate_tc::gate_proj_tc<__half>, gate_tc::Layout::kSmem, done, dev))
-        return (gtr_status_t)rc;
-      if (launch_pdl(gate_tc::gate_proj_tc<__half>, dim3((unsigned)blocks), dim3(gate_tc::kThreads),
-                     gate_tc::Layout::kSmem, st, (const __half*)x, w_down, w_up, bias, g_out, N,
-                     d_model, rank, HD, inv_tau, tpc))
-        return GTR_ERR_CUDA;
-    } else {
-      static bool done[kMaxDevices];
-      if (int rc = ensure_smem(gate_tc::gate_proj_tc<__nv_bfloat16>, gate_tc::Layout::kSmem, done, dev))
-        return (gtr_status_t)rc;
-      if (launch_pdl(gate_tc::gate_proj_tc<__nv_bfloat16>, dim3((unsigned)blocks),
-                     dim3(gate_tc::kThreads), gate_tc::Layout::kSmem, st, (const __nv_bfloat16*)x,
-                     w_down, w_up, bias, g_out, N, d_model, rank, HD, inv_tau, tpc))
-        return GTR_ERR_CUDA;
-    }
-    return (gtr_status_t)launch_status();
+    void* pack = nullptr;
+    if (int rc = pack_workspace(dev, stream, &pack)) return (gtr_status_t)rc;
+    if (int rc = gate_pack_launch(x_dtype, w_down, w_up, d_model, HD, pack, st, dev)) return (gtr_status_t)rc;
+    return (gtr_status_t)gate_fwd_packed_launch(x_dtype, x, pack, bias, g_out, N, d_model, HD, tau, st, dev);
   }
   if (rank <= 16 && HD % 4 == 0 && HD <= kGate2MaxHD && (!bias || aligned16(bias))) {
     // register-tiled kernel: one block per 64 tokens
@@ -442,6 +526,43 @@ gtr_status_t gtr_gate_fwd(const void* x, int x_dtype, const float* w_down, const
       break;
   }
   return (gtr_status_t)launch_status();
+}
+
+size_t gtr_gate_packed_bytes(void) { return (size_t)gate_tc::Pack::kBytes; }
+
+gtr_status_t gtr_gate_pack(const float* w_down, const float* w_up, int x_dtype, int d_model, int rank,
+                           int H, int dk, void* packed, size_t packed_bytes, void* stream) {
+  if (H <= 0 || dk <= 0 || d_model <= 0 || rank <= 0) return GTR_ERR_INVALID_ARG;
+  if (x_dtype < 0 || x_dtype > 2) return GTR_ERR_INVALID_ARG;
+  const long long HD = (long long)H * dk;
+  if (HD > 4096 || !gate_tc_supported(x_dtype, d_model, rank, (int)HD)) return GTR_ERR_UNSUPPORTED;
+  if (!w_down || !w_up || !packed) return GTR_ERR_INVALID_ARG;
+  if (packed_bytes < (size_t)gate_tc::Pack::kBytes) return GTR_ERR_NO_MEMORY;
+  if (!aligned16(w_down) || !aligned16(w_up) || !aligned16(packed)) return GTR_ERR_ALIGNMENT;
+  int dev;
+  if (int rc = current_device(&dev)) return (gtr_status_t)rc;
+  return (gtr_status_t)gate_pack_launch(x_dtype, w_down, w_up, d_model, (int)HD, packed,
+                                        (cudaStream_t)stream, dev);
+}
+
+gtr_status_t gtr_gate_fwd_packed(const void* x, int x_dtype, const void* packed, const float* bias,
+                                 float* g_out, int B, int T, int d_model, int rank, int H, int dk,
+                                 float tau, void* stream) {
+  if (B < 0 || T < 0 || H <= 0 || dk <= 0 || d_model <= 0 || rank <= 0) return GTR_ERR_INVALID_ARG;
+  if (x_dtype < 0 || x_dtype > 2) return GTR_ERR_INVALID_ARG;
+  if (!(tau > 0.0f) || !(tau < 3.0e38f)) return GTR_ERR_INVALID_ARG;
+  const long long HD = (long long)H * dk;
+  if (HD > 4096 || !gate_tc_supported(x_dtype, d_model, rank, (int)HD)) return GTR_ERR_UNSUPPORTED;
+  const long long N = (long long)B * T;
+  if (N == 0) return GTR_OK;
+  if (N >= (1LL << 31)) return GTR_ERR_UNSUPPORTED;
+  if (!x || !packed || !g_out) return GTR_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(packed) || !aligned16(g_out) || (bias && !aligned16(bias)))
+    return GTR_ERR_ALIGNMENT;
+  int dev;
+  if (int rc = current_device(&dev)) return (gtr_status_t)rc;
+  return (gtr_status_t)gate_fwd_packed_launch(x_dtype, x, packed, bias, g_out, N, d_model, (int)HD, tau,
+                                              (cudaStream_t)stream, dev);
 }
 
 gtr_status_t gtr_gla_fwd(const void* q, const void* k, const void* v, const float* g,

@@ -70,6 +70,19 @@ def test_invalid_arguments_rejected_before_any_launch(lib):
     assert lib.gtr_gate_fwd(P, 5, P, P, None, P, 1, 4, 384, 16, 6, 64, 16.0, S) == -1
     assert lib.gtr_gate_fwd(P, 1, P, P, None, P, 1, 4, 384, 65, 6, 64, 16.0, S) == -2
     assert lib.gtr_gate_fwd(None, 1, None, None, None, None, 0, 4, 384, 16, 6, 64, 16.0, S) == 0
+    # packed gate: shapes outside the tensor-core kernel, NULL buffers, short buffers
+    nb = lib.gtr_gate_packed_bytes()
+    assert nb > 0 and nb % 16 == 0
+    assert lib.gtr_gate_pack(P, P, 1, 384, 8, 6, 64, P, nb, S) == -2       # rank 8
+    assert lib.gtr_gate_pack(P, P, 1, 100, 16, 6, 64, P, nb, S) == -2      # d_model % 64
+    assert lib.gtr_gate_pack(P, P, 0, 384, 16, 6, 64, P, nb, S) == -2      # fp32 x
+    assert lib.gtr_gate_pack(P, P, 1, 384, 16, 8, 64, P, nb, S) == -2      # H*dk > 448
+    assert lib.gtr_gate_pack(None, P, 1, 384, 16, 6, 64, P, nb, S) == -1
+    assert lib.gtr_gate_pack(P, P, 1, 384, 16, 6, 64, P, nb - 16, S) == -4
+    assert lib.gtr_gate_fwd_packed(P, 1, P, None, P, 1, 4, 384, 16, 6, 64, 0.0, S) == -1
+    assert lib.gtr_gate_fwd_packed(P, 2, P, None, P, 1, 4, 384, 16, 6, 48, 16.0, S) == -2
+    assert lib.gtr_gate_fwd_packed(None, 1, P, None, P, 1, 4, 384, 16, 6, 64, 16.0, S) == -1
+    assert lib.gtr_gate_fwd_packed(None, 1, None, None, None, 0, 4, 384, 16, 6, 64, 16.0, S) == 0
     assert lib.gtr_gla_set_path(9) == -1
     assert lib.gtr_gla_workspace_bytes(1, 1, 4, 4, 48, 64, 64, 1) == ctypes.c_size_t(-1).value
     assert lib.gtr_gla_workspace_bytes(0, 6, 40, 40, 64, 64, 64, 1) == 0

@@ -115,6 +115,31 @@ def test_gate_projection_bf16_with_bias():
     np.testing.assert_allclose(g.double().cpu().numpy(), ref, rtol=1e-5, atol=1e-6)
 
 
+@pytest.mark.parametrize("dtype,B,T,dm,H,bias", [
+    (torch.float16, 1, 1600, 384, 6, False),    # the 640x640 workload's shapes
+    (torch.bfloat16, 3, 100, 384, 6, True),     # bf16 x, three W_down terms, bias
+    (torch.float16, 1, 5, 64, 1, True),         # fewer tokens than one tile, smallest width
+    (torch.float16, 2, 777, 192, 7, True),      # ragged last tile, H*dk = 448 (the largest)
+])
+def test_gate_packed_weights(dtype, B, T, dm, H, bias):
+    # the tensor-core gate with weights packed once: against the oracle, and identical to
+    # gtr_gate_fwd (which packs per call and runs the same kernels)
+    gen = torch.Generator().manual_seed(T + dm)
+    x = torch.randn(B, T, dm, generator=gen).to(dtype)
+    wd = torch.randn(dm, 16, generator=gen) / dm ** 0.5
+    wu = torch.randn(16, H * 64, generator=gen) / 4
+    b = torch.randn(H * 64, generator=gen) if bias else None
+    xd, wdd, wud = x.cuda(), wd.cuda(), wu.cuda()
+    bd = b.cuda() if bias else None
+    packed = binding.gate_pack(wdd, wud, dtype, H, 64)
+    g = binding.gate_fwd_packed(xd, packed, bd, 16, H, 64, 16.0)
+    g2 = binding.gate_fwd(xd, wdd, wud, bd, H, 64, 16.0)
+    ref = oracle.gate(x, wd, wu, b, tau=16.0).reshape(B, T, H, 64)
+    np.testing.assert_allclose(g.double().cpu().numpy(), ref, rtol=1e-5, atol=1e-6)
+    assert torch.equal(g, g2)
+    assert np.all(g.cpu().numpy() <= 0.0)
+
+
 @pytest.mark.parametrize("rank,H,dk,dm", [(24, 6, 64, 384), (16, 3, 5, 100), (7, 2, 64, 300)])
 def test_gate_projection_other_shapes(rank, H, dk, dm):
     # shapes outside the register-tiled kernel (rank > 16, H*dk not a multiple of 4) and a
