@@ -401,8 +401,7 @@ def run_ours(args, world, rank, local):
 
     # segment plan of this workload (for the state bytes)
     nc = (wl.T + args.chunk - 1) // args.chunk
-    m = binding.segment_chunks(wl.B, wl.H, wl.gh, wl.gw, wl.dk, wl.dv, args.chunk, host["q"].dtype)
-    nseg = (nc + m - 1) // m
+    nseg = binding.segment_count(wl.B, wl.H, wl.gh, wl.gw, wl.dk, wl.dv, args.chunk, host["q"].dtype)
     ab = alg_bytes(wl, nseg, esz)
     dom = max(per_ms, key=lambda n: per_ms[n])
     peak, peak_kind = read_peak()

@@ -214,9 +214,14 @@ GTR_API gtr_status_t gtr_gla_chunk_states(const void *k, const void *v, const fl
 GTR_API size_t gtr_gla_workspace_bytes(int B, int H, int grid_h, int grid_w, int dk, int dv, int chunk,
                                int dtype);
 
-/* Chunks per segment of the plan gtr_gla_fwd would use for this problem on
- * the current device (a segment is the run of consecutive chunks one block of
- * the summary and output kernels walks through), or a negative status. */
+/* The segment plan gtr_gla_fwd would use for this problem on the current
+ * device.  A segment is the run of consecutive chunks one block of the summary
+ * and output kernels walks through; segment s of n covers chunks
+ * [s*nc/n, (s+1)*nc/n) of the sequence's nc chunks (an even split).
+ * gtr_gla_segment_chunks: chunks in the longest segment; gtr_gla_segment_count:
+ * segments per sequence.  0 for an empty problem, or a negative status. */
+GTR_API int gtr_gla_segment_count(int B, int H, int grid_h, int grid_w, int dk, int dv, int chunk,
+                                  int dtype);
 GTR_API int gtr_gla_segment_chunks(int B, int H, int grid_h, int grid_w, int dk, int dv, int chunk,
                                    int dtype);
 

@@ -27,6 +27,7 @@ EXPORTS = (
     "gtr_gla_chunk_states", "gtr_gla_workspace_bytes", "gtr_gla_set_workspace",
     "gtr_gla_set_path", "gtr_gla_path_for", "gtr_last_device_status", "gtr_gla_segment_chunks",
     "gtr_gla_fwd_noalloc", "gtr_gate_packed_bytes", "gtr_gate_pack", "gtr_gate_fwd_packed",
+    "gtr_gla_segment_count",
 )
 
 _lock = threading.Lock()
@@ -64,6 +65,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
             "gtr_gla_path_for": ([I, I, I, I, I, I, I, I], I),
             "gtr_last_device_status": ([P, P], I),
             "gtr_gla_segment_chunks": ([I, I, I, I, I, I, I, I], I),
+            "gtr_gla_segment_count": ([I, I, I, I, I, I, I, I], I),
             "gtr_gla_fwd_noalloc": ([P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, P], I),
             "gtr_gate_packed_bytes": ([], Z),
             "gtr_gate_pack": ([P, P, I, I, I, I, I, P, Z, P], I),
@@ -250,6 +252,13 @@ def segment_chunks(B, H, grid_h, grid_w, dk, dv, chunk, dtype) -> int:
     rc = load().gtr_gla_segment_chunks(B, H, grid_h, grid_w, dk, dv, chunk, DTYPE_IDS[dtype])
     if rc < 0:
         _check("gtr_gla_segment_chunks", rc)
+    return rc
+
+
+def segment_count(B, H, grid_h, grid_w, dk, dv, chunk, dtype) -> int:
+    rc = load().gtr_gla_segment_count(B, H, grid_h, grid_w, dk, dv, chunk, DTYPE_IDS[dtype])
+    if rc < 0:
+        _check("gtr_gla_segment_count", rc)
     return rc
 
 

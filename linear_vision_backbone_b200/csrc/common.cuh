@@ -26,6 +26,12 @@ enum StatusBits : unsigned {
   kStatusMbarTimeout = 8u,   // a bounded mbarrier wait ran out
 };
 
+// Segment s of nseg covers chunks [first(s), first(s + 1)) of a sequence of
+// nc chunks: an even split, lengths differing by at most one chunk.
+__host__ __device__ __forceinline__ int seg_first_chunk(int s, int nc, int nseg) {
+  return (int)(((long long)s * nc) / nseg);
+}
+
 // Direction of batch entry b (GTR_ROTATE_BATCH cycles LR, RL, TB, BT).
 __device__ __forceinline__ int dir_of_batch(int dir, int b) { return dir == kRotate ? (b & 3) : dir; }
 

@@ -161,7 +161,7 @@ struct Misc {
 };
 static_assert(sizeof(Misc) <= Layout::kMiscBytes, "Misc must fit its reserved bytes");
 static_assert(offsetof(Misc, wu_i) == offsetof(Misc, wd_i) + kRank * 4, "scales are one block");
-static_assert(4 * Layout::kHalfSlab <= Layout::kX, "two staged slabs must fit in the x tile");
+static_assert(6 * Layout::kHalfSlab <= Layout::kX, "three staged slabs must fit in the x tile");
 
 // K-major 16-bit tile (rows x K), 128B-swizzled atoms of 8 rows x 64 elements;
 // atom columns (64 K-elements) `rows`*128 bytes apart.
@@ -403,7 +403,10 @@ gate_fwd_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUt
   // ---- epilogue, one 64-column slab of u at a time: thread = token row (TMEM
   // lane quadrant warp % 4), warp w on the slab's 16-column quarter w / 4.  Each
   // slab is staged as two 32-column halves (128-byte rows, 16-byte units XOR-ed
-  // with row % 8: the TMA 128B swizzle) and TMA-stored; two slabs alternate.
+  // with row % 8: the TMA 128B swizzle) and TMA-stored.  Three slab buffers
+  // rotate, so the one barrier per slab also covers buffer reuse: before it,
+  // the issuing thread waits until the store of two slabs ago has read its
+  // buffer, which is the buffer the next slab fills.
   if (ok) {
     const int q = warp & 3, qp = warp >> 2;
     const int r = q * 32 + lane;
@@ -411,10 +414,7 @@ gate_fwd_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUt
     const uint32_t tq = tm + ((uint32_t)(q * 32) << 16) + 64 + 16 * qp;
     const int nslab = HD / 64;
     for (int j = 0; j < nslab; ++j) {
-      uint8_t* slab = tX + (j & 1) * (2 * Layout::kHalfSlab);
-      // the store issued from this buffer two slabs ago has read it
-      if (tid == 0 && j >= 2) bulk_wait_read<1>();
-      __syncthreads();
+      uint8_t* slab = tX + (j % 3) * (2 * Layout::kHalfSlab);
       float u[16];
       tmem_ld16(tq + 64 * j, u);
       tc::tmem_ld_wait();
@@ -432,6 +432,7 @@ gate_fwd_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUt
             logsigmoid_fast(fmaf(u[c + 3] * ri, ci.w, bb.w)) * inv_tau);
       }
       tc::fence_async_smem();                     // these writes, then the TMA engine's reads
+      if (tid == 0 && j >= 2) bulk_wait_read<1>();   // slab j - 2's store has read buffer (j + 1) % 3
       __syncthreads();
       if (tid == 0) {
         tma_store_2d(&tmg, 64 * j, tok0, slab);

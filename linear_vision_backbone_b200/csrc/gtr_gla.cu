@@ -48,23 +48,23 @@ int sm_count(int dev) {
   return g_sm_count[dev];
 }
 
-// Plan of one gtr_gla_fwd call: chunk length, segment length (a run of
-// consecutive chunks one block of K2/K4 walks through) and workspace layout.
+// Plan of one gtr_gla_fwd call: chunk length, segments (runs of consecutive
+// chunks one block of K2/K4 walks through; segment s of nseg covers chunks
+// [s nc / nseg, (s+1) nc / nseg)) and workspace layout.
 struct Plan {
   int B, H, gh, gw, T, dk, dv, dir, chunk, dtype;
   int dev;
   int path;        // GTR_PATH_SIMT or GTR_PATH_TC
   int nc;          // chunks per sequence
-  int seg_chunks;  // chunks per segment
   int nseg;        // segments per sequence
-  int seg_len;     // scan positions per segment
+  int seg_chunks;  // chunks in the longest segment
   size_t offA;     // byte offset of the segment decay factors in the workspace
   size_t ws_bytes;
 };
 
-// Segment length that balances the blocks over the resident slots: minimise
-// (rounds of resident blocks) x (chunks per block); on ties take the longer
-// segment, which moves fewer boundary states through memory.
+// Segment length for the multi-wave case: minimise (rounds of resident
+// blocks) x (chunks per block); on ties take the longer segment, which moves
+// fewer boundary states through memory.
 int plan_segments(long long bh, int nc, long long slots) {
   int best = 1;
   long long best_cost = -1;
@@ -73,6 +73,40 @@ int plan_segments(long long bh, int nc, long long slots) {
     const long long units = bh * ((nc + m - 1) / m);
     const long long cost = ((units + slots - 1) / slots) * m;
     if (best_cost < 0 || cost <= best_cost) { best_cost = cost; best = m; }
+  }
+  return best;
+}
+
+// Segments per sequence when every block fits in one wave of `per_sm` blocks
+// per SM.  Block L = bh * nseg + seg is taken to share an SM with blocks
+// L +- sms (the order in which a single wave fills the SMs); a block alone on
+// its SM walks a chunk in time 1 and two co-resident blocks each take
+// kPairCost (measured for the tensor-core output kernel: about 6.9 us against
+// 4.0 us per chunk), so an SM holding blocks of a <= b chunks finishes at
+// kPairCost a + (b - a).  Minimise the slowest SM; ties to fewer segments.
+// Returns 0 when no split fits one wave.
+int plan_nseg_one_wave(long long bh, int nc, int sms, int per_sm) {
+  constexpr double kPairCost = 1.725;
+  if (per_sm != 2 || bh <= 0 || sms <= 0) return 0;
+  const long long slots = (long long)sms * per_sm;
+  int best = 0;
+  double best_cost = 0.0;
+  for (int nseg = 1; nseg <= nc && bh * nseg <= slots; ++nseg) {
+    const long long n = bh * nseg;
+    double cost = 0.0;
+    for (long long sm = 0; sm < sms && sm < n; ++sm) {
+      const int s1 = (int)(sm % nseg);
+      const int a = seg_first_chunk(s1 + 1, nc, nseg) - seg_first_chunk(s1, nc, nseg);
+      double t = a;
+      if (sm + sms < n) {
+        const int s2 = (int)((sm + sms) % nseg);
+        const int b = seg_first_chunk(s2 + 1, nc, nseg) - seg_first_chunk(s2, nc, nseg);
+        const int lo = a < b ? a : b, hi = a < b ? b : a;
+        t = kPairCost * lo + (hi - lo);
+      }
+      if (t > cost) cost = t;
+    }
+    if (best == 0 || cost < best_cost - 1e-9) { best = nseg; best_cost = cost; }
   }
   return best;
 }
@@ -103,7 +137,7 @@ int choose_path(int dk, int dv, int chunk, int dtype) {
 }
 
 int make_plan(Plan* p, int dev, int B, int H, int gh, int gw, int dk, int dv, int dir, int chunk,
-              int dtype, int force_seg_chunks) {
+              int dtype, int force_nseg) {
   p->B = B; p->H = H; p->gh = gh; p->gw = gw; p->T = gh * gw; p->dev = dev;
   p->dk = dk; p->dv = dv; p->dir = dir; p->chunk = chunk; p->dtype = dtype;
   const int path = choose_path(dk, dv, chunk, dtype);
@@ -111,10 +145,18 @@ int make_plan(Plan* p, int dev, int B, int H, int gh, int gw, int dk, int dv, in
   p->path = path;
   p->nc = (p->T + chunk - 1) / chunk;
   const long long bh = (long long)B * H;
-  const long long slots = (long long)sm_count(dev) * (path == GTR_PATH_TC ? tc_blocks_per_sm(dk, dv) : 4);
-  p->seg_chunks = force_seg_chunks > 0 ? force_seg_chunks : plan_segments(bh, p->nc, slots);
-  p->nseg = (p->nc + p->seg_chunks - 1) / p->seg_chunks;
-  p->seg_len = p->seg_chunks * chunk;
+  const int per_sm = path == GTR_PATH_TC ? tc_blocks_per_sm(dk, dv) : 4;
+  const long long slots = (long long)sm_count(dev) * per_sm;
+  if (force_nseg > 0) {
+    p->nseg = force_nseg < p->nc ? force_nseg : p->nc;
+  } else {
+    p->nseg = plan_nseg_one_wave(bh, p->nc, sm_count(dev), per_sm);
+    if (p->nseg == 0) {
+      const int m = plan_segments(bh, p->nc, slots);
+      p->nseg = (p->nc + m - 1) / m;
+    }
+  }
+  p->seg_chunks = (p->nc + p->nseg - 1) / p->nseg;
   const size_t nS = (size_t)bh * p->nseg * dk * dv * sizeof(float);
   p->offA = (nS + 255) & ~(size_t)255;
   p->ws_bytes = p->offA + (size_t)bh * p->nseg * dk * sizeof(float);
@@ -274,7 +316,7 @@ int launch_simt_rows(const Plan& p, const void* q, const void* k, const void* v,
     const size_t smem = (size_t)simt_summary_smem_floats(p.dk, p.dv) * sizeof(float);
     auto kern = gla_summary_simt<T, ROWS>;
     kern<<<grid, kSimtThreads, smem, st>>>((const T*)k, (const T*)v, g, wsS, wsA, p.H, p.T, p.gh,
-                                           p.gw, p.dk, p.dv, p.dir, p.seg_len, p.nseg);
+                                           p.gw, p.dk, p.dv, p.dir, p.chunk, p.nseg);
   } else {
     const size_t smem = (size_t)simt_output_smem_floats(p.dk, p.dv) * sizeof(float);
     auto kern = gla_output_simt<T, ROWS>;
@@ -284,7 +326,7 @@ int launch_simt_rows(const Plan& p, const void* q, const void* k, const void* v,
       return rc;
     kern<<<grid, kSimtThreads, smem, st>>>((const T*)q, (const T*)k, (const T*)v, g, (const T*)z, w,
                                            wsS, (T*)out, p.H, p.T, p.gh, p.gw, p.dk, p.dv, p.dir,
-                                           p.seg_len, p.nseg);
+                                           p.chunk, p.nseg);
   }
   return launch_status();
 }
@@ -311,7 +353,7 @@ int launch_stage(const Plan& p, const void* q, const void* k, const void* v, con
                  int stage) {
   if (p.path == GTR_PATH_TC)
     return launch_tc(p.dtype, stage, q, k, v, g, z, w, out, wsS, wsA, p.B, p.H, p.T, p.gh, p.gw,
-                     p.dk, p.dv, p.dir, p.chunk, p.seg_chunks, p.nseg, st);
+                     p.dk, p.dv, p.dir, p.chunk, p.nseg, st);
   switch (p.dtype) {
     case GTR_F32: return launch_simt<float>(p, q, k, v, g, z, w, out, wsS, wsA, st, stage);
     case GTR_F16: return launch_simt<__half>(p, q, k, v, g, z, w, out, wsS, wsA, st, stage);
@@ -414,8 +456,8 @@ int gla_fwd_noalloc_impl(const void* q, const void* k, const void* v, const floa
     const size_t per_seg = (size_t)B * H * ((size_t)dk * dv + dk) * sizeof(float);
     const size_t max_nseg = (kStaticScratchBytes - 256) / per_seg;
     if (max_nseg < 1) return GTR_ERR_NO_MEMORY;
-    const int seg = (int)((p.nc + max_nseg - 1) / max_nseg);
-    if ((rc = make_plan(&p, dev, B, H, gh, gw, dk, dv, dir, chunk, dtype, seg))) return rc;
+    const int nseg = (int)(max_nseg < (size_t)p.nc ? max_nseg : (size_t)p.nc);
+    if ((rc = make_plan(&p, dev, B, H, gh, gw, dk, dv, dir, chunk, dtype, nseg))) return rc;
     if (p.ws_bytes > kStaticScratchBytes) return GTR_ERR_NO_MEMORY;
   }
   void* ws = nullptr;
@@ -600,7 +642,8 @@ gtr_status_t gtr_gla_chunk_states(const void* k, const void* v, const float* g, 
   int dev;
   if ((rc = current_device(&dev))) return (gtr_status_t)rc;
   Plan p;
-  if ((rc = make_plan(&p, dev, B, H, grid_h, grid_w, dk, dv, dir, chunk, dtype, 1)))
+  // one chunk per segment: the scan then gives the state after every chunk
+  if ((rc = make_plan(&p, dev, B, H, grid_h, grid_w, dk, dv, dir, chunk, dtype, 0x7fffffff)))
     return (gtr_status_t)rc;
   void* ws = nullptr;
   const size_t lbytes = (size_t)B * H * p.nseg * dk * sizeof(float);
@@ -632,6 +675,17 @@ int gtr_gla_segment_chunks(int B, int H, int grid_h, int grid_w, int dk, int dv,
   Plan p;
   if ((rc = make_plan(&p, dev, B, H, grid_h, grid_w, dk, dv, 0, chunk, dtype, 0))) return rc;
   return p.seg_chunks;
+}
+
+int gtr_gla_segment_count(int B, int H, int grid_h, int grid_w, int dk, int dv, int chunk, int dtype) {
+  int rc = check_gla_args(B, H, grid_h, grid_w, dk, dv, 0, chunk, dtype);
+  if (rc) return rc;
+  if (B == 0 || H == 0 || grid_h == 0 || grid_w == 0) return 0;
+  int dev;
+  if ((rc = current_device(&dev))) return rc;
+  Plan p;
+  if ((rc = make_plan(&p, dev, B, H, grid_h, grid_w, dk, dv, 0, chunk, dtype, 0))) return rc;
+  return p.nseg;
 }
 
 gtr_status_t gtr_gla_set_workspace(void* ptr, size_t bytes) {

@@ -38,7 +38,7 @@ template <typename T, int ROWS>
 __global__ void __launch_bounds__(kSimtThreads)
 gla_summary_simt(const T* __restrict__ k, const T* __restrict__ v, const float* __restrict__ g,
                  float* __restrict__ wsS, float* __restrict__ wsA, int H, int T_, int gh, int gw,
-                 int dk, int dv, int dir, int seg_len, int nseg) {
+                 int dk, int dv, int dir, int chunk, int nseg) {
   extern __shared__ float sm[];
   float* ks = sm;                            // [batch][dk]
   float* as = ks + kSimtBatch * dk;          // [batch][dk]  exp(g)
@@ -50,7 +50,9 @@ gla_summary_simt(const T* __restrict__ k, const T* __restrict__ v, const float* 
   if (d < 0 || d > 3) { if (threadIdx.x == 0) gtr_flag(kStatusBadDir); return; }
   const int tid = threadIdx.x;
   const int nrg = kSimtThreads / dv, j = tid % dv, rg = tid / dv;
-  const int s0 = seg * seg_len, s1 = min(T_, s0 + seg_len);
+  const int nc = (T_ + chunk - 1) / chunk;
+  const int s0 = seg_first_chunk(seg, nc, nseg) * chunk;
+  const int s1 = min(T_, seg_first_chunk(seg + 1, nc, nseg) * chunk);
   float S[ROWS];
 #pragma unroll
   for (int r = 0; r < ROWS; ++r) S[r] = 0.f;
@@ -94,7 +96,7 @@ __global__ void __launch_bounds__(kSimtThreads)
 gla_output_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                 const float* __restrict__ g, const T* __restrict__ z, const float* __restrict__ w,
                 const float* __restrict__ wsS, T* __restrict__ out, int H, int T_, int gh, int gw,
-                int dk, int dv, int dir, int seg_len, int nseg) {
+                int dk, int dv, int dir, int chunk, int nseg) {
   extern __shared__ float sm[];
   const int nrg = kSimtThreads / dv;
   float* qs = sm;                            // [batch][dk]
@@ -109,7 +111,9 @@ gla_output_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __res
   if (d < 0 || d > 3) { if (threadIdx.x == 0) gtr_flag(kStatusBadDir); return; }
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int j = tid % dv, rg = tid / dv;
-  const int s0 = seg * seg_len, s1 = min(T_, s0 + seg_len);
+  const int nc = (T_ + chunk - 1) / chunk;
+  const int s0 = seg_first_chunk(seg, nc, nseg) * chunk;
+  const int s1 = min(T_, seg_first_chunk(seg + 1, nc, nseg) * chunk);
   const float* inS = wsS + ((size_t)bh * nseg + seg) * dk * dv;
   float S[ROWS];
 #pragma unroll

@@ -292,7 +292,7 @@ template <> __device__ __forceinline__ uint2 pack4<__nv_bfloat16>(float a, float
 struct Params {
   const void* q; const void* k; const void* v; const float* g; const void* z; const float* w;
   float* wsS; float* wsA; void* out;
-  int H, T, gh, gw, dir, seg_chunks, nseg;
+  int H, T, gh, gw, dir, nseg;
 };
 
 // ------------------------------------------------------------- fetching
@@ -416,8 +416,8 @@ gla_out_tc(const Params p) {
   const int b = bh / p.H, h = bh - b * p.H;
   const int d = dir_of_batch(p.dir, b);
   const int nc = (p.T + kC - 1) / kC;
-  const int c0 = seg * p.seg_chunks;
-  const int nch = min(nc, c0 + p.seg_chunks) - c0;
+  const int c0 = seg_first_chunk(seg, nc, p.nseg);
+  const int nch = seg_first_chunk(seg + 1, nc, p.nseg) - c0;
   if (d < 0 || d > 3 || nch <= 0) {
     if (tid == 0) gtr_flag(d < 0 || d > 3 ? kStatusBadDir : kStatusBadShape);
     return;
@@ -735,8 +735,8 @@ gla_sum_tc(const Params p) {
   const int b = bh / p.H, h = bh - b * p.H;
   const int d = dir_of_batch(p.dir, b);
   const int nc = (p.T + kC - 1) / kC;
-  const int c0 = seg * p.seg_chunks;
-  const int nch = min(nc, c0 + p.seg_chunks) - c0;
+  const int c0 = seg_first_chunk(seg, nc, p.nseg);
+  const int nch = seg_first_chunk(seg + 1, nc, p.nseg) - c0;
   if (d < 0 || d > 3 || nch <= 0) {
     if (tid == 0) gtr_flag(d < 0 || d > 3 ? kStatusBadDir : kStatusBadShape);
     return;
@@ -895,11 +895,11 @@ inline int launch_tc_typed(int stage, const tc::Params& p, int BH, cudaStream_t 
 inline int launch_tc(int dtype, int stage, const void* q, const void* k, const void* v,
                      const float* g, const void* z, const float* w, void* out, float* wsS,
                      float* wsA, int B, int H, int T, int gh, int gw, int dk, int dv, int dir,
-                     int chunk, int seg_chunks, int nseg, cudaStream_t st) {
+                     int chunk, int nseg, cudaStream_t st) {
   if (!tc_shape_supported(dk, dv, chunk, dtype)) return -2;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -5;
-  const tc::Params p{q, k, v, g, z, w, wsS, wsA, out, H, T, gh, gw, dir, seg_chunks, nseg};
+  const tc::Params p{q, k, v, g, z, w, wsS, wsA, out, H, T, gh, gw, dir, nseg};
   const int BH = B * H;
   return dtype == kF16 ? launch_tc_typed<__half>(stage, p, BH, st, dev)
                        : launch_tc_typed<__nv_bfloat16>(stage, p, BH, st, dev);
