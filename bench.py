@@ -406,8 +406,8 @@ def run_ours(args, world, rank, local):
     dom = max(per_ms, key=lambda n: per_ms[n])
     peak, peak_kind = read_peak()
     achieved = ab[dom] / (per_ms[dom] * 1e-3) / 1e9
-    kname = {"gate": "gate_proj_kernel", "summary": "gla_summary", "scan": "gla_state_scan",
-             "output": "gla_output"}[dom]
+    kname = {"gate": "gate_fwd_tc", "summary": "gla_sum_tc", "scan": "gla_state_scan",
+             "output": "gla_out_tc"}[dom]
     traffic, _ = read_traffic(f"{kname}:{path}:{wl.name}", kernel_source_hash())
 
     # e2e: host buffers, copies inside the timed region, through the public API
