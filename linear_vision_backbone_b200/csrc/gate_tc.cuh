@@ -49,6 +49,17 @@ __device__ __forceinline__ int scale_exp(float m) {
   return max(-60, min(60, 14 - ex));
 }
 __device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }
+// logsigmoid(u) / tau = (min(u, 0) - ln(1 + e^{-|u|})) / tau, the exponential
+// and the logarithm (as log2, scaled by ln2_tau = ln 2 / tau) by the hardware
+// approximations.  1 + e^{-|u|} is formed in fp32, so the log term carries an
+// absolute error below 1e-7 (it rounds to zero once e^{-|u|} is under fp32's
+// resolution at one); both terms are <= 0, so the result is too.
+__device__ __forceinline__ float logsigmoid_over_tau(float u, float inv_tau, float ln2_tau) {
+  const float e = tc::ex2(-fabsf(u) * 1.4426950408889634f);
+  float l;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(l) : "f"(1.0f + e));
+  return fmaf(-l, ln2_tau, fminf(u, 0.0f) * inv_tau);
+}
 // Two-term fp16 operand: x = hi + lo, hi = fp16(x), lo = fp16(x - hi); four
 // consecutive elements at byte offset `off` of the (hi, lo) tiles.
 __device__ __forceinline__ void put2(uint8_t* hi, uint8_t* lo, uint32_t off, float a, float b, float c,
@@ -408,6 +419,7 @@ gate_fwd_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUt
   // the issuing thread waits until the store of two slabs ago has read its
   // buffer, which is the buffer the next slab fills.
   if (ok) {
+    const float ln2_tau = 0.6931471805599453f * inv_tau;
     const int q = warp & 3, qp = warp >> 2;
     const int r = q * 32 + lane;
     const float ri = m.low_i[r];
@@ -426,10 +438,10 @@ gate_fwd_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUt
         const float4 ci = *reinterpret_cast<const float4*>(&m.wu_i[cb + c]);
         const int unit = (qp & 1) * 4 + (c >> 2);
         *reinterpret_cast<float4*>(half + ((unit ^ (r & 7)) << 4)) = make_float4(
-            logsigmoid_fast(fmaf(u[c + 0] * ri, ci.x, bb.x)) * inv_tau,
-            logsigmoid_fast(fmaf(u[c + 1] * ri, ci.y, bb.y)) * inv_tau,
-            logsigmoid_fast(fmaf(u[c + 2] * ri, ci.z, bb.z)) * inv_tau,
-            logsigmoid_fast(fmaf(u[c + 3] * ri, ci.w, bb.w)) * inv_tau);
+            logsigmoid_over_tau(fmaf(u[c + 0] * ri, ci.x, bb.x), inv_tau, ln2_tau),
+            logsigmoid_over_tau(fmaf(u[c + 1] * ri, ci.y, bb.y), inv_tau, ln2_tau),
+            logsigmoid_over_tau(fmaf(u[c + 2] * ri, ci.z, bb.z), inv_tau, ln2_tau),
+            logsigmoid_over_tau(fmaf(u[c + 3] * ri, ci.w, bb.w), inv_tau, ln2_tau));
       }
       tc::fence_async_smem();                     // these writes, then the TMA engine's reads
       if (tid == 0 && j >= 2) bulk_wait_read<1>();   // slab j - 2's store has read buffer (j + 1) % 3

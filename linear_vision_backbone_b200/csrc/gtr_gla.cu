@@ -244,6 +244,63 @@ int tmap_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, unsigned
   return r == CUDA_SUCCESS ? GTR_OK : GTR_ERR_CUDA;
 }
 
+// Tensor map of a [B, T, H, D] row-major tensor (element size es bytes,
+// D = 64) for box loads of one chunk of one head: orientation 0 views it as
+// (D, H, T, B), box (64, 1, 64, 1); orientation 1 as (D, H, gw, gh, B), box
+// (64, 1, 1, 64, 1), a run of 64 grid rows in one column.
+int tmap_chunk(CUtensorMap* map, CUtensorMapDataType dt, int es, const void* base, const Plan& p, int orient,
+               bool swizzle) {
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) return GTR_ERR_CUDA;
+  const cuuint64_t D = 64, es_ = (cuuint64_t)es;
+  const cuuint64_t tok = (cuuint64_t)p.H * D * es_;   // bytes per token
+  CUresult r;
+  if (orient == 0) {
+    const cuuint64_t dims[4] = {D, (cuuint64_t)p.H, (cuuint64_t)p.T, (cuuint64_t)p.B};
+    const cuuint64_t strides[3] = {D * es_, tok, tok * (cuuint64_t)p.T};
+    const cuuint32_t box[4] = {64, 1, 64, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    r = enc(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  } else {
+    const cuuint64_t dims[5] = {D, (cuuint64_t)p.H, (cuuint64_t)p.gw, (cuuint64_t)p.gh, (cuuint64_t)p.B};
+    const cuuint64_t strides[4] = {D * es_, tok, tok * (cuuint64_t)p.gw, tok * (cuuint64_t)p.T};
+    const cuuint32_t box[5] = {64, 1, 1, 64, 1};
+    const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    r = enc(map, dt, 5, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  }
+  return r == CUDA_SUCCESS ? GTR_OK : GTR_ERR_CUDA;
+}
+// The output stage's tensor maps, when every chunk it reads is one box:
+// 16-byte aligned bases, and for the column orders (TB, BT) 64 | gh so that
+// no chunk crosses a grid column.  Returns false to gather with cp.async.
+bool out_stage_maps(const Plan& p, const void* q, const void* k, const void* v, const float* g,
+                    tc::Maps* maps) {
+  for (const void* a : {q, k, v, (const void*)g})
+    if (((uintptr_t)a & 15) != 0) return false;
+  bool orient[2] = {false, false};
+  for (int b = 0; b < (p.dir == kRotate ? (p.B < 4 ? p.B : 4) : 1); ++b) {
+    const int d = p.dir == kRotate ? b : p.dir;
+    orient[d == kTB || d == kBT] = true;
+  }
+  if (orient[1] && p.gh % 64 != 0) return false;
+  if (p.T >= (1 << 30) || p.B >= (1 << 30)) return false;
+  const CUtensorMapDataType dt = p.dtype == GTR_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  *maps = tc::Maps{};
+  for (int o = 0; o < 2; ++o) {
+    if (!orient[o]) continue;
+    if (tmap_chunk(&maps->t[o][tc::kMapQ], dt, 2, q, p, o, false) ||
+        tmap_chunk(&maps->t[o][tc::kMapK], dt, 2, k, p, o, false) ||
+        tmap_chunk(&maps->t[o][tc::kMapV], dt, 2, v, p, o, true) ||
+        tmap_chunk(&maps->t[o][tc::kMapG], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, g, p, o, false))
+      return false;
+  }
+  return true;
+}
+
 // ---- tensor-core gate: weight packing and the forward pass
 int gate_pack_launch(int x_dtype, const float* w_down, const float* w_up, int dm, int HD, void* pack,
                      cudaStream_t st, int dev) {
@@ -351,9 +408,12 @@ int launch_simt(const Plan& p, const void* q, const void* k, const void* v, cons
 int launch_stage(const Plan& p, const void* q, const void* k, const void* v, const float* g,
                  const void* z, const float* w, void* out, float* wsS, float* wsA, cudaStream_t st,
                  int stage) {
-  if (p.path == GTR_PATH_TC)
+  if (p.path == GTR_PATH_TC) {
+    tc::Maps maps;
+    const bool boxes = stage == 1 && out_stage_maps(p, q, k, v, g, &maps);
     return launch_tc(p.dtype, stage, q, k, v, g, z, w, out, wsS, wsA, p.B, p.H, p.T, p.gh, p.gw,
-                     p.dk, p.dv, p.dir, p.chunk, p.nseg, st);
+                     p.dk, p.dv, p.dir, p.chunk, p.nseg, boxes ? &maps : nullptr, st);
+  }
   switch (p.dtype) {
     case GTR_F32: return launch_simt<float>(p, q, k, v, g, z, w, out, wsS, wsA, st, stage);
     case GTR_F16: return launch_simt<__half>(p, q, k, v, g, z, w, out, wsS, wsA, st, stage);
@@ -364,7 +424,7 @@ int launch_stage(const Plan& p, const void* q, const void* k, const void* v, con
 
 int launch_scan(const Plan& p, float* wsS, const float* wsA, int inclusive, cudaStream_t st) {
   const long long total = (long long)p.B * p.H * p.dk * p.dv;
-  const long long blocks = (total + kScanThreads - 1) / kScanThreads;
+  const long long blocks = (total + 31) / 32;   // 32 elements per block
   return launch_pdl(gla_state_scan, dim3((unsigned)blocks), dim3(kScanThreads), 0, st, wsS,
                     (const float*)wsA, total, p.nseg, p.dk, p.dv, inclusive) == 0
              ? GTR_OK

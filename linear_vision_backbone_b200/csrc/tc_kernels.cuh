@@ -51,6 +51,8 @@
 // chunk are zero-filled when the chunk is fetched (a zero gate repeats the
 // last cumsum), so no later phase tests them.
 #pragma once
+#include <cuda.h>
+
 #include <type_traits>
 
 #include "common.cuh"
@@ -104,6 +106,30 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity) {
   while (!mbar_try(b, parity))
     if (globaltimer() - t0 > kWaitNs) return false;
   return true;
+}
+// One arrival that also expects `bytes` of asynchronous copies on the barrier.
+__device__ __forceinline__ void mbar_arrive_tx(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(b)), "r"(bytes)
+               : "memory");
+}
+// Tensor-map box loads (global -> shared), completing on an mbarrier.  The
+// innermost coordinate is always 0 here (16-byte aligned); the others may be
+// negative or past the end, which reads zeros.
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
+      "%4, %5}], [%6];" ::"r"(saddr(dst)),
+      "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(saddr(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
+                                            int c4, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
+      "%4, %5, %6}], [%7];" ::"r"(saddr(dst)),
+      "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(saddr(bar))
+      : "memory");
 }
 // 16-byte asynchronous global -> shared copy (L2 only), grouped by commit.
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
@@ -252,6 +278,14 @@ __device__ __forceinline__ void put8(uint8_t* H, uint8_t* L, uint32_t off, const
   *reinterpret_cast<uint4*>(L + off) = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
+// two consecutive elements (4 bytes) at byte offset `off` of the (hi, lo) tiles
+__device__ __forceinline__ void put2x(uint8_t* H, uint8_t* L, uint32_t off, float a, float b) {
+  uint32_t h, l;
+  split2(a, b, h, l);
+  *reinterpret_cast<uint32_t*>(H + off) = h;
+  *reinterpret_cast<uint32_t*>(L + off) = l;
+}
+
 template <typename T> struct Vec4;
 template <> struct Vec4<__half> {
   static __device__ __forceinline__ float4 from_bits(uint2 u) {
@@ -277,6 +311,12 @@ template <> struct Vec4<__nv_bfloat16> {
     return from_bits(*reinterpret_cast<const uint2*>(p));
   }
 };
+// two consecutive 16-bit elements as floats
+__device__ __forceinline__ float2 ld2(const __half* p) { return __half22float2(*reinterpret_cast<const __half2*>(p)); }
+__device__ __forceinline__ float2 ld2(const __nv_bfloat16* p) {
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+}
+
 template <typename T> __device__ __forceinline__ uint2 pack4(float a, float b, float c, float d);
 template <> __device__ __forceinline__ uint2 pack4<__half>(float a, float b, float c, float d) {
   const __half2 x = __floats2half2_rn(a, b), y = __floats2half2_rn(c, d);
@@ -293,24 +333,65 @@ struct Params {
   const void* q; const void* k; const void* v; const float* g; const void* z; const float* w;
   float* wsS; float* wsA; void* out;
   int H, T, gh, gw, dir, nseg;
+  int tma;                        // 1: chunks arrive by tensor-map loads (Maps valid)
+};
+// Tensor maps of q, k, v, g ([B, T, H, D] row-major) for box loads of one
+// chunk of one head: [0] the token order, dims (D, H, T, B), box (64, 1, 64,
+// 1); [1] the grid columns, dims (D, H, gw, gh, B), box (64, 1, 1, 64, 1)
+// (valid when 64 divides gh).  A reversed scan loads the same box and walks
+// it backwards.  q, k, g are plain row-major boxes; v lands in the
+// SWIZZLE_128B operand layout.
+enum { kMapQ = 0, kMapK = 1, kMapV = 2, kMapG = 3 };
+struct Maps {
+  CUtensorMap t[2][4];
 };
 
 // ------------------------------------------------------------- fetching
+// Scan order -> box: orientation (0 token order, 1 grid columns) and whether
+// the chunk's box is walked backwards.
+__device__ __forceinline__ int dir_orient(int d) { return d == kTB || d == kBT; }
+__device__ __forceinline__ bool dir_reversed(int d) { return d == kRL || d == kBT; }
+// Box loads of the chunk at scan position s0: q, k (row-major), v (operand
+// layout, at vdst), g (row-major fp32), all completing on `bar`.  Box row j
+// holds scan position s0 + j, or s0 + 63 - j for a reversed scan (whose
+// last, ragged chunk then starts at a negative token and reads zeros there).
+__device__ __forceinline__ void tma_chunk(const Params& p, const Maps& mp, uint8_t* kdst, uint8_t* qdst,
+                                          uint8_t* vdst, uint8_t* gdst, uint64_t* bar, int d, int b, int h,
+                                          int s0) {
+  const int t0 = dir_reversed(d) ? p.T - s0 - kC : s0;   // first scan position of the box, in its order
+  mbar_arrive_tx(bar, 3 * kTile + kGTile);
+  if (!dir_orient(d)) {
+    const CUtensorMap* m = mp.t[0];
+    tma_load_4d(kdst, m + kMapK, 0, h, t0, b, bar);
+    tma_load_4d(qdst, m + kMapQ, 0, h, t0, b, bar);
+    tma_load_4d(vdst, m + kMapV, 0, h, t0, b, bar);
+    tma_load_4d(gdst, m + kMapG, 0, h, t0, b, bar);
+  } else {
+    const CUtensorMap* m = mp.t[1];
+    const int col = t0 / p.gh, r0 = t0 - col * p.gh;   // whole chunks: t0 >= 0, r0 + 64 <= gh
+    tma_load_5d(kdst, m + kMapK, 0, h, col, r0, b, bar);
+    tma_load_5d(qdst, m + kMapQ, 0, h, col, r0, b, bar);
+    tma_load_5d(vdst, m + kMapV, 0, h, col, r0, b, bar);
+    tma_load_5d(gdst, m + kMapG, 0, h, col, r0, b, bar);
+  }
+}
 // Token rows (b*T + t)*H + h of the chunk starting at scan position s0.
 __device__ __forceinline__ void chunk_rows(const Params& p, long long* rows, int b, int h, int d,
                                            int s0, int ntok, int tid) {
   if (tid < ntok) rows[tid] = ((long long)b * p.T + scan_to_grid(d, s0 + tid, p.T, p.gh, p.gw)) * p.H + h;
 }
-// A 16-bit tensor's rows of the chunk into a row-major staging tile (row j at
-// byte j * 128): 16-byte pieces, piece o = (row o / 8, part o % 8); rows past
-// ntok are zeroed.
+// A 16-bit tensor's rows of the chunk into a 64 x 64 tile: row-major (row j
+// at byte j * 128) or, with kSw, in the SWIZZLE_128B operand layout.  16-byte
+// pieces, piece o = (row o / 8, unit o % 8); rows past ntok are zeroed.
+template <bool kSw = false>
 __device__ __forceinline__ void fetch16(uint8_t* dst, const void* src, const long long* rows, int ntok,
                                         int tid) {
 #pragma unroll
   for (int u = 0; u < 2; ++u) {
     const int o = tid + u * kThreads, j = o >> 3, part = (o & 7) * 16;
-    if (j < ntok) cp_async16(dst + j * 128 + part, (const uint8_t*)src + rows[j] * kRowBytes + part);
-    else *reinterpret_cast<uint4*>(dst + j * 128 + part) = make_uint4(0u, 0u, 0u, 0u);
+    uint8_t* to = dst + (kSw ? sw_unit(j, o & 7) : (uint32_t)(j * 128 + part));
+    if (j < ntok) cp_async16(to, (const uint8_t*)src + rows[j] * kRowBytes + part);
+    else *reinterpret_cast<uint4*>(to) = make_uint4(0u, 0u, 0u, 0u);
   }
 }
 // The fp32 gate rows (256 bytes each); rows past ntok get a zero gate.
@@ -346,21 +427,22 @@ __device__ __forceinline__ float silu_fast(float z) { return __fdividef(z, 1.0f 
 
 // ===================================================================== K4
 struct OutMisc {                  // per-CTA scalars; arrays read as float4 are 16-byte aligned
-  uint64_t mma[3];                // [0] q~ S' and scores (two arrivals), [1] + P V, [2] state increment
+  uint64_t mma[3];                // [0] q~ S and scores (two arrivals), [1] + P V, [2] state increment
+  uint64_t ld;                    // a chunk's box loads
   uint32_t tmem;
   int pad;
-  alignas(16) float red[4][kD];   // column-pass partial sums; epilogue row sums
-  alignas(16) float Gm[kD];
+  alignas(16) float part[kWarps][kD];   // cumsum partials: tokens 8 w .. 8 w + 7, per dim
+  alignas(16) float red[2][kD];   // epilogue row sums
   alignas(16) float Gam[kD];
   alignas(16) float aG[kD];       // e^{Gam}: state decay over the chunk
-  alignas(16) float eK[kD];       // e^{Gam - G_m}: row factor of k~^T V
   alignas(16) float wv[kD];       // RMSNorm weight
   alignas(16) long long rows[2][kC];   // token rows of the current / next chunk
 };
 struct OutLayout {
-  // staging (row-major): k, q, v, gate of one chunk
+  // staging: k, q (row-major), v (operand layout), gate (row-major fp32)
   static constexpr int kOffK = 0, kOffQ = kTile, kOffV = 2 * kTile, kOffG = 3 * kTile;
-  // operand tiles (1024-aligned): VH VL QH QL KH KL SH SL
+  // operand tiles (1024-aligned): VH VL QH QL KH KL SH SL.  A bf16 v read in
+  // scan order lands directly in VH / VL, alternately by chunk parity.
   static constexpr int kTiles = 3 * kTile + kGTile;
   static constexpr int kMisc = kTiles + 8 * kTile;
   static constexpr int kSmem = kMisc + (int)sizeof(OutMisc) + 1024;   // + alignment slack
@@ -369,12 +451,13 @@ struct OutLayout {
 };
 static_assert(OutLayout::kTiles % 1024 == 0, "operand tiles must be 1024-byte aligned");
 
-// The k, q, v, gate rows of a chunk into the output kernel's staging.
-__device__ __forceinline__ void fetch_chunk(uint8_t* sm, const Params& p, const long long* rows, int ntok,
-                                            int tid) {
+// The k, q, gate rows of a chunk into the output kernel's staging (cp.async),
+// v into `vdst` in the operand layout.
+__device__ __forceinline__ void fetch_chunk(uint8_t* sm, uint8_t* vdst, const Params& p, const long long* rows,
+                                            int ntok, int tid) {
   fetch16(sm + OutLayout::kOffK, p.k, rows, ntok, tid);
   fetch16(sm + OutLayout::kOffQ, p.q, rows, ntok, tid);
-  fetch16(sm + OutLayout::kOffV, p.v, rows, ntok, tid);
+  fetch16<true>(vdst, p.v, rows, ntok, tid);
   fetch_g(sm + OutLayout::kOffG, p.g, rows, ntok, tid);
 }
 static_assert(2 * (OutLayout::kSmem + 1024) <= 228 * 1024, "two output CTAs must share an SM");
@@ -392,14 +475,13 @@ __device__ __forceinline__ float row_combine_sum(float v, float (*red)[kD], int 
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads, OutLayout::kBlocksPerSM)
-gla_out_tc(const Params p) {
+gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
   using L = OutLayout;
   constexpr bool kV2 = std::is_same<T, __half>::value;   // fp16 V: two bf16 terms
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const T* kst = reinterpret_cast<const T*>(sm + L::kOffK);
   const T* qst = reinterpret_cast<const T*>(sm + L::kOffQ);
-  const T* vst = reinterpret_cast<const T*>(sm + L::kOffV);
   float* G = reinterpret_cast<float*>(sm + L::kOffG);
   uint8_t* VH = sm + L::kTiles;
   uint8_t* VL = VH + kTile;
@@ -407,7 +489,7 @@ gla_out_tc(const Params p) {
   uint8_t* QL = VH + 3 * kTile;
   uint8_t* KH = VH + 4 * kTile;       // k~ or k^: K-major B of the scores, MN-major A of k^T V
   uint8_t* KL = VH + 5 * kTile;
-  uint8_t* SH = VH + 6 * kTile;       // S' (MN-major B)
+  uint8_t* SH = VH + 6 * kTile;       // S (MN-major B)
   uint8_t* SL = VH + 7 * kTile;
   OutMisc& m = *reinterpret_cast<OutMisc*>(sm + L::kMisc);
 
@@ -422,21 +504,42 @@ gla_out_tc(const Params p) {
     if (tid == 0) gtr_flag(d < 0 || d > 3 ? kStatusBadDir : kStatusBadShape);
     return;
   }
+  const bool tma = p.tma != 0;
+  // staging row of scan offset i: box loads of a reversed scan hold the chunk backwards
+  const int rmask = (tma && dir_reversed(d)) ? kC - 1 : 0;
+  // a bf16 v in scan order is the operand tile itself (double-buffered by
+  // chunk parity); otherwise it is staged and converted by the builder
+  const bool vdirect = !kV2 && rmask == 0;
+  auto vtile = [&](int it) -> uint8_t* { return vdirect ? ((it & 1) ? VL : VH) : sm + L::kOffV; };
+  auto fetch = [&](int it, int s, int ntk, const long long* rws) {
+    if (tma) {
+      if (tid == 32) tma_chunk(p, mp, sm + L::kOffK, sm + L::kOffQ, vtile(it), sm + L::kOffG, &m.ld, d, b, h, s);
+    } else {
+      fetch_chunk(sm, vtile(it), p, rws, ntk, tid);
+    }
+  };
   // row phases: quadrant qd, column half, 16 columns from cbase of accumulator row `row`
   const int qd = warp & 3, half = warp >> 2;
   const int row = qd * 16 + (lane & 15);
   const int cbase = half * 32 + (lane >> 4) * 16;
   const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
-  // column pass: column dd, tokens 16 qt ..; tile build: rows rb + 16 u, columns cg .. cg + 3
-  const int dd = tid & 63, qt = tid >> 6;
-  const int rb = tid >> 4, cg = (tid & 15) * 4;
+  // cumsum and tile build: dims 2 lane, 2 lane + 1 of scan offsets 8 warp ..
+  // 8 warp + 7, so every shared-memory access of a warp covers one whole row
+  const int dc = 2 * lane, tb = 8 * warp;
 
+  if (tid == 0) {
+    mbar_init(&m.mma[0], 2);
+    mbar_init(&m.mma[1], 1);
+    mbar_init(&m.mma[2], 1);
+    mbar_init(&m.ld, 1);
+    mbar_fence_init();
+  }
   // chunk 0's copies go out first
   {
     const int ntok0 = min(kC, p.T - c0 * kC);
     chunk_rows(p, m.rows[0], b, h, d, c0 * kC, ntok0, tid);
     __syncthreads();
-    fetch_chunk(sm, p, m.rows[0], ntok0, tid);
+    fetch(0, c0 * kC, ntok0, m.rows[0]);
     cp_async_commit();
   }
   if (tid < kD) m.wv[tid] = p.w ? p.w[tid] : 1.0f;
@@ -457,30 +560,24 @@ gla_out_tc(const Params p) {
       S[4 * c] = x.x; S[4 * c + 1] = x.y; S[4 * c + 2] = x.z; S[4 * c + 3] = x.w;
     }
   }
-  if (tid == 0) {
-    mbar_init(&m.mma[0], 2);
-    mbar_init(&m.mma[1], 1);
-    mbar_init(&m.mma[2], 1);
-    mbar_fence_init();
-  }
   if (warp == 0) {
     tmem_alloc(&m.tmem, L::kTmemCols);
     tmem_relinquish();
   }
-  cp_async_wait<0>();                     // chunk 0's k, q, v, g
+  cp_async_wait<0>();                     // chunk 0's k, q, v, g (copied by this thread)
   tc_before_sync();
   __syncthreads();
   tc_after_sync();
   const uint32_t tm = m.tmem;
-  constexpr uint32_t kIdQS = idesc_bf16(0, 1);   // A K-major, B MN-major: q~ S', P V
+  constexpr uint32_t kIdQS = idesc_bf16(0, 1);   // A K-major, B MN-major: q~ S, P V
   constexpr uint32_t kIdQK = idesc_bf16(0, 0);   // both K-major: q~ k~^T
   constexpr uint32_t kIdKV = idesc_bf16(1, 1);   // both MN-major: k~^T V
 
-  uint32_t ph0 = 0, ph1 = 0, ph2 = 0;
-  bool failed = false;
-  // The next chunk's k, q, v, g are copied once this chunk's tiles are built
-  // (after P for an exact chunk, whose scores still read the staging); z goes
-  // straight to registers, requested two phases before the epilogue uses it.
+  uint32_t ph0 = 0, ph1 = 0, ph2 = 0, phl = 0;
+  bool failed = false, ld_pending = tma;
+  // The next chunk's k, q, v, g are requested once this chunk's tiles are
+  // built (after P for an exact chunk, whose scores still read the staging);
+  // z goes straight to registers, requested two phases before the epilogue.
   for (int it = 0; it < nch; ++it) {
     const int par = it & 1;
     const int s0 = (c0 + it) * kC;
@@ -488,80 +585,88 @@ gla_out_tc(const Params p) {
     const bool more = it + 1 < nch;
     const int s1 = s0 + kC;
     const int ntok1 = more ? min(kC, p.T - s1) : 0;
+    uint8_t* const Vh = vdirect ? vtile(it) : VH;
+    uint8_t* const Vl = vdirect ? Vh : VL;      // VL is read only for a two-term (fp16) v
+    if (tma) {
+      failed |= !mbar_wait(&m.ld, phl);
+      phl ^= 1;
+      ld_pending = false;
+    }
 
-    // ---- column pass: G in place; G_m, Gam; exact test per element
-    float gv[16];
-    column_cumsum(G, gv, &m.red[0][0], dd, qt);
+    // ---- in-chunk cumsum G: eight scan offsets in registers, then the
+    // partial sums of the warps before this one (one block barrier)
+    float2 gc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      gc[i] = *reinterpret_cast<const float2*>(G + ((tb + i) ^ rmask) * kD + dc);
+      if (i) { gc[i].x += gc[i - 1].x; gc[i].y += gc[i - 1].y; }
+    }
+    *reinterpret_cast<float2*>(&m.part[warp][dc]) = gc[7];
+    __syncthreads();
+    {
+      float2 off = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int w = 0; w < kWarps - 1; ++w)
+        if (w < warp) {
+          const float2 pp = *reinterpret_cast<const float2*>(&m.part[w][dc]);
+          off.x += pp.x; off.y += pp.y;
+        }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { gc[i].x += off.x; gc[i].y += off.y; }
+    }
     int bad = 0;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      G[(qt * 16 + i) * kD + dd] = gv[i];
-      bad |= !(gv[i] <= 0.f && gv[i] >= -kSpanMax);
-    }
-    {
-      const int mid = (ntok - 1) >> 1;
-      if (qt == (mid >> 4)) m.Gm[dd] = G[mid * kD + dd];   // this thread's own store
-      if (qt == 3) m.Gam[dd] = gv[15];
-    }
-    // with G in [-kSpanMax, 0] everywhere every column's span is within bounds
-    const bool exact = __syncthreads_or(bad) != 0;
-    const bool tilde = !exact;
-    if (tid < kD) {
-      const float gm = m.Gm[tid], gam = m.Gam[tid];
-      m.aG[tid] = expf(gam);
-      m.eK[tid] = expf(gam - gm);
+    for (int i = 0; i < 8; ++i)
+      bad |= !(gc[i].x <= 0.f && gc[i].x >= -kSpanMax && gc[i].y <= 0.f && gc[i].y >= -kSpanMax);
+    if (warp == kWarps - 1) {
+      *reinterpret_cast<float2*>(&m.Gam[dc]) = gc[7];
+      *reinterpret_cast<float2*>(&m.aG[dc]) = make_float2(expf(gc[7].x), expf(gc[7].y));
     }
 
-    // ---- operand tiles (rows past ntok are zero: their q, k were zero-filled)
+    // ---- operand tiles, referenced to the chunk start: q~ = q e^{G}, k~ = k e^{-G}
+    // (rows past ntok are zero: their q, k were zero-filled).  All eight rows
+    // are loaded before any tile is written: the stores could alias the
+    // staging as far as the compiler knows, so interleaving them with the
+    // loads would serialise every row on the shared-memory latency.
     {
-      const float4 gr = *reinterpret_cast<const float4*>(tilde ? &m.Gm[cg] : &m.Gam[cg]);
-      const float r0 = gr.x * kLog2e, r1 = gr.y * kLog2e, r2 = gr.z * kLog2e, r3 = gr.w * kLog2e;
+      uint32_t qr[8], kr[8], vr[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int r = rb + 16 * u;
-        const float4 kk = Vec4<T>::load(kst + r * kD + cg);
-        const float4 qq = Vec4<T>::load(qst + r * kD + cg);
-        const float4 gg = *reinterpret_cast<const float4*>(G + r * kD + cg);
-        // x = (G - reference) log2 e: key factor 2^-x; query factor 2^x, or e^{G} for an exact chunk
-        const float x0 = fmaf(gg.x, kLog2e, -r0), x1 = fmaf(gg.y, kLog2e, -r1);
-        const float x2 = fmaf(gg.z, kLog2e, -r2), x3 = fmaf(gg.w, kLog2e, -r3);
-        const uint32_t off = sw16(r, cg);
-        put4(KH, KL, off, kk.x * ex2(-x0), kk.y * ex2(-x1), kk.z * ex2(-x2), kk.w * ex2(-x3));
-        if (tilde)
-          put4(QH, QL, off, qq.x * ex2(x0), qq.y * ex2(x1), qq.z * ex2(x2), qq.w * ex2(x3));
-        else
-          put4(QH, QL, off, qq.x * ex2(gg.x * kLog2e), qq.y * ex2(gg.y * kLog2e),
-               qq.z * ex2(gg.z * kLog2e), qq.w * ex2(gg.w * kLog2e));
+      for (int i = 0; i < 8; ++i) {
+        const int rs = (tb + i) ^ rmask;
+        qr[i] = *reinterpret_cast<const uint32_t*>(qst + rs * kD + dc);
+        kr[i] = *reinterpret_cast<const uint32_t*>(kst + rs * kD + dc);
+        vr[i] = vdirect ? 0u : *reinterpret_cast<const uint32_t*>(sm + L::kOffV + sw16(rs, dc));
       }
-      // S' = e^{G_m} S, or S for an exact chunk
-      const float sc = tilde ? __expf(m.Gm[row]) : 1.0f;
-      float sp[16];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) sp[c] = sc * S[c];
-      put8(SH, SL, sw16(row, cbase), sp);
-      put8(SH, SL, sw16(row, cbase + 8), sp + 8);
-    }
-    // V from staging: fp16 as two bf16 terms, bf16 as it is
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int r = rb + 16 * u;
-      const uint32_t off = sw16(r, cg);
-      if (kV2) {
-        const float4 vv = Vec4<T>::load(vst + r * kD + cg);
-        put4(VH, VL, off, vv.x, vv.y, vv.z, vv.w);
-      } else {
-        *reinterpret_cast<uint2*>(VH + off) = *reinterpret_cast<const uint2*>(vst + r * kD + cg);
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t off = sw16(tb + i, dc);
+        const float2 qq = ld2(reinterpret_cast<const T*>(&qr[i])), kk = ld2(reinterpret_cast<const T*>(&kr[i]));
+        const float x0 = gc[i].x * kLog2e, x1 = gc[i].y * kLog2e;
+        put2x(QH, QL, off, qq.x * ex2(x0), qq.y * ex2(x1));
+        put2x(KH, KL, off, kk.x * ex2(-x0), kk.y * ex2(-x1));
+        if (!vdirect) {
+          if (kV2) {
+            const float2 vv = ld2(reinterpret_cast<const T*>(&vr[i]));
+            put2x(VH, VL, off, vv.x, vv.y);
+          } else {
+            *reinterpret_cast<uint32_t*>(VH + off) = vr[i];
+          }
+        }
       }
     }
+    put8(SH, SL, sw16(row, cbase), S);
+    put8(SH, SL, sw16(row, cbase + 8), S + 8);
     if (more) chunk_rows(p, m.rows[par ^ 1], b, h, d, s1, ntok1, tid);
     fence_async_smem();
     tc_before_sync();
-    __syncthreads();
+    // with G in [-kSpanMax, 0] everywhere no factor leaves [e^{-kSpanMax}, e^{kSpanMax}]
+    const bool exact = __syncthreads_or(bad) != 0;
+    const bool tilde = !exact;
     tc_after_sync();
 
     // Two issuing threads: a single thread issues one MMA per ~60 cycles
     // whatever its size, so independent products go out from two warps and
-    // the tensor pipe interleaves them.  Warp 0 owns o (q~ S', later P V),
+    // the tensor pipe interleaves them.  Warp 0 owns o (q~ S, later P V),
     // warp 4 the score columns (scores, later the state increment); each
     // thread's own MMAs execute in issue order.  P overwrites q~, so mma[0]
     // completes only when both threads' products are done.
@@ -576,9 +681,25 @@ gla_out_tc(const Params p) {
                                   false);
       mma_commit(&m.mma[0]);
     }
-    // the staging of k, q, g is consumed unless an exact chunk still reads it
-    if (more && tilde) fetch_chunk(sm, p, m.rows[par ^ 1], ntok1, tid);
+    // the staging of k, q, v, g is consumed unless an exact chunk still reads it
+    if (more && tilde) {
+      fetch(it + 1, s1, ntok1, m.rows[par ^ 1]);
+      ld_pending = tma;
+    }
     cp_async_commit();
+    if (exact) {
+      // the CUDA-core scores read G (scan order) from the staging; the key
+      // tile becomes k^ = k e^{Gam - G}, the state update S <- e^{Gam} S + k^^T V
+      const float2 gam = *reinterpret_cast<const float2*>(&m.Gam[dc]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = tb + i;
+        *reinterpret_cast<float2*>(G + r * kD + dc) = gc[i];
+        const float2 kk = ld2(kst + (r ^ rmask) * kD + dc);
+        put2x(KH, KL, sw16(r, dc), kk.x * expf(gam.x - gc[i].x), kk.y * expf(gam.y - gc[i].y));
+      }
+      __syncthreads();
+    }
     // this chunk's z for the epilogue: 16 elements of the thread's row
     uint4 zz0 = make_uint4(0u, 0u, 0u, 0u), zz1 = zz0;
     if (row < ntok) {
@@ -607,13 +728,15 @@ gla_out_tc(const Params p) {
 #pragma unroll
       for (int e = 0; e < 16; ++e) acc[e] = 0.f;
       if (j < ntok) {
+        const T* qj_row = qst + (j ^ rmask) * kD;
         for (int x = 0; x < kD; ++x) {
-          const float qj = Elem<T>::to_f(qst[j * kD + x]);
+          const float qj = Elem<T>::to_f(qj_row[x]);
           const float gj = G[j * kD + x];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int i = ib + e;
-            if (i <= j) acc[e] = fmaf(qj * Elem<T>::to_f(kst[i * kD + x]), expf(gj - G[i * kD + x]), acc[e]);
+            if (i <= j)
+              acc[e] = fmaf(qj * Elem<T>::to_f(kst[(i ^ rmask) * kD + x]), expf(gj - G[i * kD + x]), acc[e]);
           }
         }
       }
@@ -625,17 +748,34 @@ gla_out_tc(const Params p) {
     tc_before_sync();
     if (__syncthreads_or(failed)) break;
     tc_after_sync();
-    if (more && exact) fetch_chunk(sm, p, m.rows[par ^ 1], ntok1, tid);
+    if (more && exact) {
+      fetch(it + 1, s1, ntok1, m.rows[par ^ 1]);
+      ld_pending = tma;
+    }
     cp_async_commit();
     if (tid == 0) {
-      mma_terms<kStepK, kStepMN>(tm + 0, desc_k(QH), desc_k(QL), desc_mn(VH), desc_mn(VL), kV2, kIdQS,
+      mma_terms<kStepK, kStepMN>(tm + 0, desc_k(QH), desc_k(QL), desc_mn(Vh), desc_mn(Vl), kV2, kIdQS,
                                  true);
       mma_commit(&m.mma[1]);
     }
     if (tid == 128) {
-      mma_terms<kStepMN, kStepMN>(tm + 64, desc_mn(KH), desc_mn(KL), desc_mn(VH), desc_mn(VL), kV2,
+      mma_terms<kStepMN, kStepMN>(tm + 64, desc_mn(KH), desc_mn(KL), desc_mn(Vh), desc_mn(Vl), kV2,
                                   kIdKV, false);
       mma_commit(&m.mma[2]);
+    }
+    // the output gate w * SiLU(z) while P V and the increment run
+    float wz[16];
+#pragma unroll
+    for (int c = 0; c < 16; c += 8) {
+      const uint4 zz = c == 0 ? zz0 : zz1;
+      const float4 z0 = Vec4<T>::from_bits(make_uint2(zz.x, zz.y));
+      const float4 z1 = Vec4<T>::from_bits(make_uint2(zz.z, zz.w));
+      const float4 w0 = *reinterpret_cast<const float4*>(&m.wv[cbase + c]);
+      const float4 w1 = *reinterpret_cast<const float4*>(&m.wv[cbase + c + 4]);
+      wz[c + 0] = w0.x * silu_fast(z0.x); wz[c + 1] = w0.y * silu_fast(z0.y);
+      wz[c + 2] = w0.z * silu_fast(z0.z); wz[c + 3] = w0.w * silu_fast(z0.w);
+      wz[c + 4] = w1.x * silu_fast(z1.x); wz[c + 5] = w1.y * silu_fast(z1.y);
+      wz[c + 6] = w1.z * silu_fast(z1.z); wz[c + 7] = w1.w * silu_fast(z1.w);
     }
 
     // ---- epilogue: o_j / sqrt(mean o_j^2 + eps) * w * SiLU(z_j), stored at the token's grid row
@@ -655,21 +795,16 @@ gla_out_tc(const Params p) {
         T* dst = reinterpret_cast<T*>(p.out) + m.rows[par][row] * kD + cbase;
 #pragma unroll
         for (int c = 0; c < 16; c += 8) {
-          const uint4 zz = c == 0 ? zz0 : zz1;
-          const float4 z0 = Vec4<T>::from_bits(make_uint2(zz.x, zz.y));
-          const float4 z1 = Vec4<T>::from_bits(make_uint2(zz.z, zz.w));
-          const float4 w0 = *reinterpret_cast<const float4*>(&m.wv[cbase + c]);
-          const float4 w1 = *reinterpret_cast<const float4*>(&m.wv[cbase + c + 4]);
-          const uint2 lo = pack4<T>(o[c + 0] * inv * w0.x * silu_fast(z0.x), o[c + 1] * inv * w0.y * silu_fast(z0.y),
-                                    o[c + 2] * inv * w0.z * silu_fast(z0.z), o[c + 3] * inv * w0.w * silu_fast(z0.w));
-          const uint2 hi = pack4<T>(o[c + 4] * inv * w1.x * silu_fast(z1.x), o[c + 5] * inv * w1.y * silu_fast(z1.y),
-                                    o[c + 6] * inv * w1.z * silu_fast(z1.z), o[c + 7] * inv * w1.w * silu_fast(z1.w));
+          const uint2 lo = pack4<T>(o[c + 0] * inv * wz[c + 0], o[c + 1] * inv * wz[c + 1],
+                                    o[c + 2] * inv * wz[c + 2], o[c + 3] * inv * wz[c + 3]);
+          const uint2 hi = pack4<T>(o[c + 4] * inv * wz[c + 4], o[c + 5] * inv * wz[c + 5],
+                                    o[c + 6] * inv * wz[c + 6], o[c + 7] * inv * wz[c + 7]);
           *reinterpret_cast<uint4*>(dst + c) = make_uint4(lo.x, lo.y, hi.x, hi.y);
         }
       }
     }
 
-    // ---- state: S <- e^{Gam} S + diag(e^{Gam - G_m}) k~^T V  (or + k^^T V)
+    // ---- state: S <- e^{Gam} (S + k~^T V), or e^{Gam} S + k^^T V for an exact chunk
     failed |= !mbar_wait(&m.mma[2], ph2);
     ph2 ^= 1;
     tc_after_sync();
@@ -677,17 +812,18 @@ gla_out_tc(const Params p) {
       float ds[16];
       tmem_ld16x2(tm + lane_base + 64 + half * 32, ds);
       tmem_ld_wait();
-      const float f = tilde ? m.eK[row] : 1.0f, a = m.aG[row];
+      const float a = m.aG[row];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) S[c] = fmaf(a, S[c], f * ds[c]);
+      for (int c = 0; c < 16; ++c) S[c] = tilde ? a * (S[c] + ds[c]) : fmaf(a, S[c], ds[c]);
     }
-    cp_async_wait<0>();                   // the next chunk's k, q, v, g
+    cp_async_wait<0>();                   // the next chunk's copies made by this thread
     tc_before_sync();
     if (__syncthreads_or(failed)) break;
     tc_after_sync();
   }
 
   cp_async_wait<0>();                     // no copy may land after the block exits
+  if (ld_pending && !mbar_wait(&m.ld, phl)) failed = true;
   if (failed && tid == 0) gtr_flag(kStatusMbarTimeout);
   tc_before_sync();
   __syncthreads();
@@ -872,37 +1008,42 @@ inline bool tc_shape_supported(int dk, int dv, int chunk, int dtype) {
 }
 inline int tc_blocks_per_sm(int, int) { return tc::OutLayout::kBlocksPerSM; }
 
-template <typename K>
-inline int launch_tc_kernel(K kern, int smem, const tc::Params& p, int BH, cudaStream_t st, bool* done,
-                            int dev) {
+template <typename K, typename... Args>
+inline int launch_tc_kernel(K kern, int smem, int nseg, int BH, cudaStream_t st, bool* done, int dev,
+                            const Args&... args) {
   if (!done[dev]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return -5;
     done[dev] = true;
   }
-  return launch_pdl(kern, dim3(p.nseg, BH), dim3(tc::kThreads), smem, st, p);
+  return launch_pdl(kern, dim3(nseg, BH), dim3(tc::kThreads), smem, st, args...);
 }
 
 // stage 0: segment summaries (K2); stage 1: segment outputs (K4)
 template <typename T>
-inline int launch_tc_typed(int stage, const tc::Params& p, int BH, cudaStream_t st, int dev) {
+inline int launch_tc_typed(int stage, const tc::Params& p, const tc::Maps& mp, int BH, cudaStream_t st,
+                           int dev) {
   static bool done_sum[64], done_out[64];
   if (stage == 0)
-    return launch_tc_kernel(tc::gla_sum_tc<T>, tc::SumLayout::kSmem, p, BH, st, done_sum, dev);
-  return launch_tc_kernel(tc::gla_out_tc<T>, tc::OutLayout::kSmem, p, BH, st, done_out, dev);
+    return launch_tc_kernel(tc::gla_sum_tc<T>, tc::SumLayout::kSmem, p.nseg, BH, st, done_sum, dev, p);
+  return launch_tc_kernel(tc::gla_out_tc<T>, tc::OutLayout::kSmem, p.nseg, BH, st, done_out, dev, p, mp);
 }
 
+// `maps`: tensor maps of q, k, v, g for the output stage's box loads, or
+// null (the chunks are then gathered with cp.async).
 inline int launch_tc(int dtype, int stage, const void* q, const void* k, const void* v,
                      const float* g, const void* z, const float* w, void* out, float* wsS,
                      float* wsA, int B, int H, int T, int gh, int gw, int dk, int dv, int dir,
-                     int chunk, int nseg, cudaStream_t st) {
+                     int chunk, int nseg, const tc::Maps* maps, cudaStream_t st) {
   if (!tc_shape_supported(dk, dv, chunk, dtype)) return -2;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -5;
-  const tc::Params p{q, k, v, g, z, w, wsS, wsA, out, H, T, gh, gw, dir, nseg};
+  const tc::Params p{q, k, v, g, z, w, wsS, wsA, out, H, T, gh, gw, dir, nseg, maps ? 1 : 0};
+  static const tc::Maps kNoMaps{};
+  const tc::Maps& mp = maps ? *maps : kNoMaps;
   const int BH = B * H;
-  return dtype == kF16 ? launch_tc_typed<__half>(stage, p, BH, st, dev)
-                       : launch_tc_typed<__nv_bfloat16>(stage, p, BH, st, dev);
+  return dtype == kF16 ? launch_tc_typed<__half>(stage, p, mp, BH, st, dev)
+                       : launch_tc_typed<__nv_bfloat16>(stage, p, mp, BH, st, dev);
 }
 
 }  // namespace gtr

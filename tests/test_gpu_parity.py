@@ -251,6 +251,43 @@ def test_strong_decay_takes_the_exact_path():
         assert exact > 0
 
 
+@pytest.mark.parametrize("dtype", ("f16", "bf16"))
+@pytest.mark.parametrize("direction", DIRS + ("ROTATE",))
+def test_box_loaded_chunks_every_order(dtype, direction):
+    # 64 divides gh, so every scan order's chunk of one head is a single
+    # tensor-map box: the token order for LR / RL, a grid column for TB / BT
+    # (reversed orders walk the box backwards).  B = 4 gives ROTATE all four.
+    gh, gw = 64, 24
+    d = inputs.make_custom(4, 2, gh, gw, 64, 64, dtype, seed=23, w_random=True)
+    y, ref = _run_custom(d, gh, gw, direction, 64, inputs.DTYPES[dtype])
+    assert_close(y, ref, inputs.DTYPES[dtype], f"boxes {dtype} {direction}")
+    _check_status()
+
+
+@pytest.mark.parametrize("dtype", ("f16", "bf16"))
+def test_ragged_reversed_box(dtype):
+    # RL over T = 1073: the last chunk's box starts before token 0 and reads zeros there
+    gh, gw = 37, 29
+    d = inputs.make_custom(2, 3, gh, gw, 64, 64, dtype, seed=27)
+    y, ref = _run_custom(d, gh, gw, "RL", 64, inputs.DTYPES[dtype])
+    assert_close(y, ref, inputs.DTYPES[dtype], f"ragged RL {dtype}")
+    _check_status()
+
+
+@pytest.mark.parametrize("direction", ("RL", "BT"))
+def test_strong_decay_reversed_boxes(direction):
+    # exact chunks read the staged q, k backwards and rewrite the gate cumsum in scan order
+    gh, gw = 64, 4
+    d = inputs.make_custom(1, 2, gh, gw, 64, 64, "bf16", seed=63, g_mu=-6.0, g_scale=2.0)
+    binding.device_status()
+    y, ref = _run_custom(d, gh, gw, direction, 64, torch.bfloat16)
+    assert_close(y, ref, torch.bfloat16, f"strong decay {direction}")
+    rc, bits, exact = binding.device_status()
+    assert rc == 0 and bits == 0
+    if binding.path_for(1, 2, gh, gw, 64, 64, 64, torch.bfloat16) == "tc":
+        assert exact > 0
+
+
 def test_zero_gate_long_memory():
     gh, gw = 64, 64
     d = inputs.make_custom(1, 2, gh, gw, 64, 64, "bf16", seed=71, qk_std=0.125)
@@ -267,6 +304,19 @@ def test_chunk_states_against_oracle(chunk, direction):
     st = binding.chunk_states(_dev(d["k"]), _dev(d["v"]), _dev(d["g"]), grid_h=gh, grid_w=gw,
                               direction=direction, chunk=chunk)
     ref = oracle.chunk_states(d["k"], d["v"], d["g"], gh=gh, gw=gw, direction=direction, chunk=chunk)
+    got = st.double().cpu().numpy()
+    rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    assert rel < 1e-3, rel
+
+
+def test_chunk_states_many_segments():
+    # 320 chunks: the boundary scan splits each element's segments into ranges
+    # longer than it keeps in registers and re-reads them for its second pass
+    gh, gw = 64, 80
+    d = inputs.make_custom(1, 2, gh, gw, 64, 64, "bf16", seed=83)
+    st = binding.chunk_states(_dev(d["k"]), _dev(d["v"]), _dev(d["g"]), grid_h=gh, grid_w=gw,
+                              direction="TB", chunk=16)
+    ref = oracle.chunk_states(d["k"], d["v"], d["g"], gh=gh, gw=gw, direction="TB", chunk=16)
     got = st.double().cpu().numpy()
     rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
     assert rel < 1e-3, rel
