@@ -274,11 +274,11 @@ int tmap_chunk(CUtensorMap* map, CUtensorMapDataType dt, int es, const void* bas
   }
   return r == CUDA_SUCCESS ? GTR_OK : GTR_ERR_CUDA;
 }
-// The output stage's tensor maps, when every chunk it reads is one box:
-// 16-byte aligned bases, and for the column orders (TB, BT) 64 | gh so that
-// no chunk crosses a grid column.  Returns false to gather with cp.async.
-bool out_stage_maps(const Plan& p, const void* q, const void* k, const void* v, const float* g,
-                    tc::Maps* maps) {
+// Tensor maps of q (when given; the summary stage reads none), k, v, g, when
+// every chunk of one head is one box: 16-byte aligned bases, and for the
+// column orders (TB, BT) 64 | gh so that no chunk crosses a grid column.
+// Returns false to gather with cp.async.
+bool chunk_maps(const Plan& p, const void* q, const void* k, const void* v, const float* g, tc::Maps* maps) {
   for (const void* a : {q, k, v, (const void*)g})
     if (((uintptr_t)a & 15) != 0) return false;
   bool orient[2] = {false, false};
@@ -292,7 +292,7 @@ bool out_stage_maps(const Plan& p, const void* q, const void* k, const void* v, 
   *maps = tc::Maps{};
   for (int o = 0; o < 2; ++o) {
     if (!orient[o]) continue;
-    if (tmap_chunk(&maps->t[o][tc::kMapQ], dt, 2, q, p, o, false) ||
+    if ((q && tmap_chunk(&maps->t[o][tc::kMapQ], dt, 2, q, p, o, false)) ||
         tmap_chunk(&maps->t[o][tc::kMapK], dt, 2, k, p, o, false) ||
         tmap_chunk(&maps->t[o][tc::kMapV], dt, 2, v, p, o, true) ||
         tmap_chunk(&maps->t[o][tc::kMapG], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, g, p, o, false))
@@ -410,7 +410,7 @@ int launch_stage(const Plan& p, const void* q, const void* k, const void* v, con
                  int stage) {
   if (p.path == GTR_PATH_TC) {
     tc::Maps maps;
-    const bool boxes = stage == 1 && out_stage_maps(p, q, k, v, g, &maps);
+    const bool boxes = chunk_maps(p, stage == 1 ? q : nullptr, k, v, g, &maps);
     return launch_tc(p.dtype, stage, q, k, v, g, z, w, out, wsS, wsA, p.B, p.H, p.T, p.gh, p.gw,
                      p.dk, p.dv, p.dir, p.chunk, p.nseg, boxes ? &maps : nullptr, st);
   }

@@ -25,9 +25,11 @@ namespace gtr {
 
 constexpr int kScanParts = 4;
 constexpr int kScanThreads = 32 * kScanParts;
-constexpr int kScanReg = 16;
+constexpr int kScanReg = 12;
 
-__global__ void __launch_bounds__(kScanThreads)
+// at most 64 registers: eight blocks per SM, so a 16k-token, 6-head problem
+// (768 blocks) is resident in one wave
+__global__ void __launch_bounds__(kScanThreads, 8)
 gla_state_scan(float* __restrict__ wsS, const float* __restrict__ wsA, long long total, int nseg,
                int dk, int dv, int inclusive) {
   __shared__ float mapP[kScanParts][32], mapR[kScanParts][32];

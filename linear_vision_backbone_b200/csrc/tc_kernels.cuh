@@ -355,25 +355,24 @@ __device__ __forceinline__ bool dir_reversed(int d) { return d == kRL || d == kB
 // layout, at vdst), g (row-major fp32), all completing on `bar`.  Box row j
 // holds scan position s0 + j, or s0 + 63 - j for a reversed scan (whose
 // last, ragged chunk then starts at a negative token and reads zeros there).
+__device__ __forceinline__ void tma_box(const Params& p, const Maps& mp, int which, void* dst, uint64_t* bar,
+                                        int d, int b, int h, int s0) {
+  const int t0 = dir_reversed(d) ? p.T - s0 - kC : s0;   // first scan position of the box, in its order
+  if (!dir_orient(d)) {
+    tma_load_4d(dst, &mp.t[0][which], 0, h, t0, b, bar);
+  } else {
+    const int col = t0 / p.gh, r0 = t0 - col * p.gh;   // whole chunks: t0 >= 0, r0 + 64 <= gh
+    tma_load_5d(dst, &mp.t[1][which], 0, h, col, r0, b, bar);
+  }
+}
 __device__ __forceinline__ void tma_chunk(const Params& p, const Maps& mp, uint8_t* kdst, uint8_t* qdst,
                                           uint8_t* vdst, uint8_t* gdst, uint64_t* bar, int d, int b, int h,
                                           int s0) {
-  const int t0 = dir_reversed(d) ? p.T - s0 - kC : s0;   // first scan position of the box, in its order
   mbar_arrive_tx(bar, 3 * kTile + kGTile);
-  if (!dir_orient(d)) {
-    const CUtensorMap* m = mp.t[0];
-    tma_load_4d(kdst, m + kMapK, 0, h, t0, b, bar);
-    tma_load_4d(qdst, m + kMapQ, 0, h, t0, b, bar);
-    tma_load_4d(vdst, m + kMapV, 0, h, t0, b, bar);
-    tma_load_4d(gdst, m + kMapG, 0, h, t0, b, bar);
-  } else {
-    const CUtensorMap* m = mp.t[1];
-    const int col = t0 / p.gh, r0 = t0 - col * p.gh;   // whole chunks: t0 >= 0, r0 + 64 <= gh
-    tma_load_5d(kdst, m + kMapK, 0, h, col, r0, b, bar);
-    tma_load_5d(qdst, m + kMapQ, 0, h, col, r0, b, bar);
-    tma_load_5d(vdst, m + kMapV, 0, h, col, r0, b, bar);
-    tma_load_5d(gdst, m + kMapG, 0, h, col, r0, b, bar);
-  }
+  tma_box(p, mp, kMapK, kdst, bar, d, b, h, s0);
+  tma_box(p, mp, kMapQ, qdst, bar, d, b, h, s0);
+  tma_box(p, mp, kMapV, vdst, bar, d, b, h, s0);
+  tma_box(p, mp, kMapG, gdst, bar, d, b, h, s0);
 }
 // Token rows (b*T + t)*H + h of the chunk starting at scan position s0.
 __device__ __forceinline__ void chunk_rows(const Params& p, long long* rows, int b, int h, int d,
@@ -834,13 +833,14 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
 // ===================================================================== K2
 struct SumMisc {
   uint64_t mma;
+  uint64_t ld[2];                 // box loads into staging buffer 0 / 1
   uint32_t tmem;
-  int pad;
-  alignas(16) float part[4][kD];
-  alignas(16) long long rows[2][kC];
+  int waited, fetched, issued;    // steps whose loads were consumed / issued, products issued
+  alignas(16) float part[kWarps][kD];   // cumsum partials: tokens 8 w .. 8 w + 7, per dim
+  alignas(16) long long rows[2][kC];    // token rows (cp.async gathers only)
 };
 struct SumLayout {
-  // two staging buffers of k (8 KB), v (8 KB), gate (16 KB)
+  // two staging buffers of k (8 KB, row-major), v (8 KB, operand layout), gate (16 KB)
   static constexpr int kOffK = 0, kOffV = kTile, kOffG = 2 * kTile;
   static constexpr int kStage = 2 * kTile + kGTile;
   // operand tiles (1024-aligned): KH KL VH VL
@@ -849,13 +849,16 @@ struct SumLayout {
   static constexpr int kSmem = kMisc + (int)sizeof(SumMisc) + 1024;
   static constexpr int kTmemCols = 128;   // two accumulators, summed at the end
   static constexpr int kBlocksPerSM = 2;
+  // eight warps build the tiles; a ninth issues the MMAs and the box loads, so
+  // the builders go on to the next chunk while the tensor pipe works
+  static constexpr int kThreadsAll = kThreads + 32;
 };
 static_assert(SumLayout::kTiles % 1024 == 0, "operand tiles must be 1024-byte aligned");
 static_assert(2 * (SumLayout::kSmem + 1024) <= 228 * 1024, "two summary CTAs must share an SM");
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads, SumLayout::kBlocksPerSM)
-gla_sum_tc(const Params p) {
+__global__ void __launch_bounds__(SumLayout::kThreadsAll, SumLayout::kBlocksPerSM)
+gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
   using L = SumLayout;
   constexpr bool kV2 = std::is_same<T, __half>::value;
   extern __shared__ uint8_t smem_raw[];
@@ -877,29 +880,59 @@ gla_sum_tc(const Params p) {
     if (tid == 0) gtr_flag(d < 0 || d > 3 ? kStatusBadDir : kStatusBadShape);
     return;
   }
+  const bool tma = p.tma != 0;
+  const int rmask = (tma && dir_reversed(d)) ? kC - 1 : 0;   // staging row of scan offset i: i ^ rmask
+  const bool vdirect = !kV2 && rmask == 0;                    // a bf16 v in scan order is the B operand as staged
+  // final accumulator read: quadrant qd, column half, 16 columns from cbase of row `row`
   const int qd = warp & 3, half = warp >> 2;
   const int row = qd * 16 + (lane & 15);
   const int cbase = half * 32 + (lane >> 4) * 16;
   const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
-  const int dd = tid & 63, qt = tid >> 6;
-  const int rb = tid >> 4, cg = (tid & 15) * 4;
-  // step it handles chunk c0 + nch - 1 - it; only the first one can be ragged
+  // cumsum and tile build: dims 2 lane, 2 lane + 1 of scan offsets 8 warp .. 8 warp + 7
+  const int dc = 2 * lane, tb = 8 * warp;
+  // step `it` handles chunk c0 + nch - 1 - it (last to first); only the first can be ragged
   const int clast = c0 + nch - 1;
-  const int ntok_first = min(kC, p.T - clast * kC);
+  auto stage = [&](int it) -> uint8_t* { return sm + (it & 1) * L::kStage; };
+  // step it's k, v (v in the operand layout), g into stage(it)
+  auto fetch = [&](int it) {
+    const int s0 = (clast - it) * kC;
+    uint8_t* st = stage(it);
+    if (tma) {
+      if (tid == kThreads) {
+        uint64_t* bar = &m.ld[it & 1];
+        mbar_arrive_tx(bar, 2 * kTile + kGTile);
+        tma_box(p, mp, kMapK, st + L::kOffK, bar, d, b, h, s0);
+        tma_box(p, mp, kMapV, st + L::kOffV, bar, d, b, h, s0);
+        tma_box(p, mp, kMapG, st + L::kOffG, bar, d, b, h, s0);
+      }
+    } else {
+      const int ntok = min(kC, p.T - s0);
+      fetch16(st + L::kOffK, p.k, m.rows[it & 1], ntok, tid);
+      fetch16<true>(st + L::kOffV, p.v, m.rows[it & 1], ntok, tid);
+      fetch_g(st + L::kOffG, p.g, m.rows[it & 1], ntok, tid);
+      cp_async_commit();
+    }
+  };
 
-  chunk_rows(p, m.rows[0], b, h, d, clast * kC, ntok_first, tid);
-  if (nch > 1) chunk_rows(p, m.rows[1], b, h, d, (clast - 1) * kC, kC, tid);
-  __syncthreads();
-  pdl_wait();                             // k, v, g may come from the previous kernel
-  pdl_trigger();
-  fetch16(sm + L::kOffK, p.k, m.rows[0], ntok_first, tid);
-  fetch16(sm + L::kOffV, p.v, m.rows[0], ntok_first, tid);
-  fetch_g(sm + L::kOffG, p.g, m.rows[0], ntok_first, tid);
-  cp_async_commit();
+  const bool control = tid >= kThreads;   // warp 8
   if (tid == 0) {
-    mbar_init(&m.mma, 2);
+    mbar_init(&m.mma, 1);
+    mbar_init(&m.ld[0], 1);
+    mbar_init(&m.ld[1], 1);
     mbar_fence_init();
   }
+  if (!tma) {
+    chunk_rows(p, m.rows[0], b, h, d, clast * kC, min(kC, p.T - clast * kC), tid);
+    if (nch > 1) chunk_rows(p, m.rows[1], b, h, d, (clast - 1) * kC, kC, tid);
+  }
+  __syncthreads();
+  pdl_wait();                             // g comes from the previous kernel
+  pdl_trigger();
+  if (tma || !control) {
+    fetch(0);
+    if (nch > 1) fetch(1);
+  }
+  int fetched = nch > 1 ? 1 : 0, waited = -1;   // box loads issued / consumed, by step
   if (warp == 0) {
     tmem_alloc(&m.tmem, L::kTmemCols);
     tmem_relinquish();
@@ -910,78 +943,131 @@ gla_sum_tc(const Params p) {
   const uint32_t tm = m.tmem;
   constexpr uint32_t kIdKV = idesc_bf16(1, 1);
 
-  float R = 0.f;              // summed log-gate of column dd over the chunks already seen
   uint32_t ph = 0;
   bool failed = false;
-  for (int it = 0; it < nch; ++it) {
-    const int buf = it & 1;
-    uint8_t* st = sm + buf * L::kStage;
-    // the next chunk (toward the segment start) into the other buffer; always full
-    if (it + 1 < nch) {
-      uint8_t* nx = sm + (buf ^ 1) * L::kStage;
-      fetch16(nx + L::kOffK, p.k, m.rows[buf ^ 1], kC, tid);
-      fetch16(nx + L::kOffV, p.v, m.rows[buf ^ 1], kC, tid);
-      fetch_g(nx + L::kOffG, p.g, m.rows[buf ^ 1], kC, tid);
+  int issued = -1;
+  if (control) {
+    // ---- control warp: products of each chunk once the builders have its
+    // tiles, then (box loads) the chunk after next into the buffer they read
+    for (int it = 0; it < nch; ++it) {
+      tc_before_sync();
+      if (__syncthreads_or(failed)) {                 // the builders' barrier B
+        failed = true;
+        break;
+      }
+      tc_after_sync();
+      uint8_t* const Vb = vdirect ? stage(it) + L::kOffV : VH;
+      if (tid == kThreads) {
+        // k^hi V into columns [0, 64), k^lo V into [64, 128)
+        mma_k64<kStepMN, kStepMN>(tm, desc_mn(KH), desc_mn(Vb), kIdKV, it > 0);
+        mma_k64<kStepMN, kStepMN>(tm + 64, desc_mn(KL), desc_mn(Vb), kIdKV, it > 0);
+        if (kV2) mma_k64<kStepMN, kStepMN>(tm, desc_mn(KH), desc_mn(VL), kIdKV, true);
+        mma_commit(&m.mma);
+      }
+      issued = it;
+      if (tma && it + 2 < nch) {
+        if (!mbar_wait(&m.mma, (uint32_t)it & 1u)) failed = true;
+        tc_after_sync();
+        fetch(it + 2);
+        fetched = it + 2;
+      }
+      __syncwarp();
     }
-    cp_async_commit();
-    cp_async_wait<1>();                   // this chunk's copies
-    __syncthreads();
-
-    // ---- weights e^{R + Gam - G_s} in place of the gates
-    float* Gw = reinterpret_cast<float*>(st + L::kOffG);
-    float gv[16];
-    const float tot = column_cumsum(Gw, gv, &m.part[0][0], dd, qt);
-    const float base = R + tot;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) Gw[(qt * 16 + i) * kD + dd] = ex2((base - gv[i]) * kLog2e);
-    R = base;
-    if (it + 2 < nch) chunk_rows(p, m.rows[buf], b, h, d, (clast - it - 2) * kC, kC, tid);
-    __syncthreads();
-    if (it > 0) {                         // the previous chunk's products have read the tiles
-      failed |= !mbar_wait(&m.mma, ph);
-      ph ^= 1;
-    }
-    tc_after_sync();
-
-    // ---- operand tiles: k^ = k * weight (two terms), V
-    {
+  } else {
+    // R: summed log-gate, per dim, of the chunks already seen (the segment's tail)
+    float2 R = make_float2(0.f, 0.f);
+    for (int it = 0; it < nch; ++it) {
+      uint8_t* st = stage(it);
       const T* kst = reinterpret_cast<const T*>(st + L::kOffK);
-      const T* vst = reinterpret_cast<const T*>(st + L::kOffV);
+      const float* G = reinterpret_cast<const float*>(st + L::kOffG);
+      if (tma) {
+        failed |= !mbar_wait(&m.ld[it & 1], (uint32_t)(it >> 1) & 1u);
+        waited = it;
+      } else {
+        if (it == 0 && nch > 1) cp_async_wait<1>();
+        else cp_async_wait<0>();
+        named_barrier(1, kThreads);
+      }
+      // rows of the next chunk (cp.async gathers; that buffer's gather is long done)
+      if (!tma && it >= 1 && it + 1 < nch) chunk_rows(p, m.rows[(it + 1) & 1], b, h, d, (clast - it - 1) * kC, kC, tid);
+
+      // ---- in-chunk cumsum G (eight scan offsets in registers), the partial
+      // sums of the other warps, and the chunk total Gam
+      float2 gc[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int r = rb + 16 * u;
-        const float4 kk = Vec4<T>::load(kst + r * kD + cg);
-        const float4 ww = *reinterpret_cast<const float4*>(Gw + r * kD + cg);
-        const uint32_t off = sw16(r, cg);
-        put4(KH, KL, off, kk.x * ww.x, kk.y * ww.y, kk.z * ww.z, kk.w * ww.w);
-        if (kV2) {
-          const float4 vv = Vec4<T>::load(vst + r * kD + cg);
-          put4(VH, VL, off, vv.x, vv.y, vv.z, vv.w);
-        } else {
-          *reinterpret_cast<uint2*>(VH + off) = *reinterpret_cast<const uint2*>(vst + r * kD + cg);
+      for (int i = 0; i < 8; ++i) {
+        gc[i] = *reinterpret_cast<const float2*>(G + ((tb + i) ^ rmask) * kD + dc);
+        if (i) { gc[i].x += gc[i - 1].x; gc[i].y += gc[i - 1].y; }
+      }
+      *reinterpret_cast<float2*>(&m.part[warp][dc]) = gc[7];
+      named_barrier(1, kThreads);
+      float2 off = make_float2(0.f, 0.f), tot = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const float2 pp = *reinterpret_cast<const float2*>(&m.part[w][dc]);
+        if (w < warp) { off.x += pp.x; off.y += pp.y; }
+        tot.x += pp.x; tot.y += pp.y;
+      }
+      // weights e^{R + Gam - G_s}: the decay from token s to the segment end
+      const float2 base = make_float2(R.x + tot.x - off.x, R.y + tot.y - off.y);
+      R.x += tot.x; R.y += tot.y;
+      uint32_t kr[8], vr[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int rs = (tb + i) ^ rmask;
+        kr[i] = *reinterpret_cast<const uint32_t*>(kst + rs * kD + dc);
+        vr[i] = vdirect ? 0u : *reinterpret_cast<const uint32_t*>(st + L::kOffV + sw16(rs, dc));
+      }
+      if (it > 0) {                       // the previous chunk's products have read the tiles
+        failed |= !mbar_wait(&m.mma, ph);
+        ph ^= 1;
+      }
+      tc_after_sync();
+      if (!tma && it >= 1 && it + 1 < nch) fetch(it + 1);   // into the buffer those products read
+
+      // ---- operand tiles: k^ = k * weight (two terms), V
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t o = sw16(tb + i, dc);
+        const float2 kk = ld2(reinterpret_cast<const T*>(&kr[i]));
+        put2x(KH, KL, o, kk.x * ex2((base.x - gc[i].x) * kLog2e), kk.y * ex2((base.y - gc[i].y) * kLog2e));
+        if (!vdirect) {
+          if (kV2) {
+            const float2 vv = ld2(reinterpret_cast<const T*>(&vr[i]));
+            put2x(VH, VL, o, vv.x, vv.y);
+          } else {
+            *reinterpret_cast<uint32_t*>(VH + o) = vr[i];
+          }
         }
       }
+      fence_async_smem();
+      tc_before_sync();
+      if (__syncthreads_or(failed)) {                 // barrier B: the control warp issues
+        failed = true;
+        break;
+      }
+      tc_after_sync();
     }
-    fence_async_smem();
-    tc_before_sync();
-    if (__syncthreads_or(failed)) break;
-    tc_after_sync();
-    // two issuing threads (one MMA per ~60 cycles each): k^hi V into columns
-    // [0, 64), k^lo V into [64, 128)
-    if (tid == 0) {
-      mma_k64<kStepMN, kStepMN>(tm, desc_mn(KH), desc_mn(VH), kIdKV, it > 0);
-      if (kV2) mma_k64<kStepMN, kStepMN>(tm, desc_mn(KH), desc_mn(VL), kIdKV, true);
-      mma_commit(&m.mma);
-    }
-    if (tid == 128) {
-      mma_k64<kStepMN, kStepMN>(tm + 64, desc_mn(KL), desc_mn(VH), kIdKV, it > 0);
-      mma_commit(&m.mma);
-    }
+    if (warp == 0)
+      *reinterpret_cast<float2*>(&m.part[0][dc]) = R;  // the segment's summed log-gate
   }
-  if (!failed) failed = !mbar_wait(&m.mma, ph);
+  // Drain: the last issued products, then box loads issued but not consumed
+  // (only after an early exit), before TMEM and shared memory are released.
+  if (tid == kThreads) {
+    m.issued = issued;
+    m.fetched = fetched;
+  }
+  if (tid == 0) m.waited = waited;
+  failed = __syncthreads_or(failed) != 0;
+  const int last = m.issued;
+  if (last >= 0 && !mbar_wait(&m.mma, (uint32_t)last & 1u)) failed = true;
   tc_after_sync();
   cp_async_wait<0>();
-  if (!failed) {
+  if (tma && tid == 0)
+    for (int x = m.waited + 1; x <= m.fetched; ++x)
+      if (!mbar_wait(&m.ld[x & 1], (uint32_t)(x >> 1) & 1u)) failed = true;
+  failed = __syncthreads_or(failed) != 0;
+  if (!failed && !control) {
     float ds[16], dl[16];
     tmem_ld16x2(tm + lane_base + half * 32, ds);
     tmem_ld16x2(tm + lane_base + 64 + half * 32, dl);
@@ -991,8 +1077,11 @@ gla_sum_tc(const Params p) {
     float4* dst = reinterpret_cast<float4*>(p.wsS + (((size_t)bh * p.nseg + seg) * kD + row) * kD + cbase);
 #pragma unroll
     for (int c = 0; c < 4; ++c) dst[c] = make_float4(ds[4 * c], ds[4 * c + 1], ds[4 * c + 2], ds[4 * c + 3]);
-    if (qt == 0) p.wsA[((size_t)bh * p.nseg + seg) * kD + dd] = expf(R);
-  } else if (tid == 0) {
+    if (warp == 0) {
+      const float2 R = *reinterpret_cast<const float2*>(&m.part[0][dc]);
+      *reinterpret_cast<float2*>(p.wsA + ((size_t)bh * p.nseg + seg) * kD + dc) = make_float2(expf(R.x), expf(R.y));
+    }
+  } else if (failed && tid == 0) {
     gtr_flag(kStatusMbarTimeout);
   }
   tc_before_sync();
@@ -1009,14 +1098,14 @@ inline bool tc_shape_supported(int dk, int dv, int chunk, int dtype) {
 inline int tc_blocks_per_sm(int, int) { return tc::OutLayout::kBlocksPerSM; }
 
 template <typename K, typename... Args>
-inline int launch_tc_kernel(K kern, int smem, int nseg, int BH, cudaStream_t st, bool* done, int dev,
-                            const Args&... args) {
+inline int launch_tc_kernel(K kern, int smem, int threads, int nseg, int BH, cudaStream_t st, bool* done,
+                            int dev, const Args&... args) {
   if (!done[dev]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return -5;
     done[dev] = true;
   }
-  return launch_pdl(kern, dim3(nseg, BH), dim3(tc::kThreads), smem, st, args...);
+  return launch_pdl(kern, dim3(nseg, BH), dim3(threads), smem, st, args...);
 }
 
 // stage 0: segment summaries (K2); stage 1: segment outputs (K4)
@@ -1025,8 +1114,10 @@ inline int launch_tc_typed(int stage, const tc::Params& p, const tc::Maps& mp, i
                            int dev) {
   static bool done_sum[64], done_out[64];
   if (stage == 0)
-    return launch_tc_kernel(tc::gla_sum_tc<T>, tc::SumLayout::kSmem, p.nseg, BH, st, done_sum, dev, p);
-  return launch_tc_kernel(tc::gla_out_tc<T>, tc::OutLayout::kSmem, p.nseg, BH, st, done_out, dev, p, mp);
+    return launch_tc_kernel(tc::gla_sum_tc<T>, tc::SumLayout::kSmem, tc::SumLayout::kThreadsAll, p.nseg, BH, st,
+                            done_sum, dev, p, mp);
+  return launch_tc_kernel(tc::gla_out_tc<T>, tc::OutLayout::kSmem, tc::kThreads, p.nseg, BH, st, done_out, dev,
+                          p, mp);
 }
 
 // `maps`: tensor maps of q, k, v, g for the output stage's box loads, or

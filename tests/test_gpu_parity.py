@@ -328,7 +328,7 @@ def test_output_stays_inside_its_buffer_and_inputs_untouched():
     d = inputs.make_custom(B, H, gh, gw, dk, dv, "f16", seed=91)
     n = B * gh * gw * H * dv
     guard = 4096
-    for path in ("simt", "auto"):
+    for path, chunk in (("simt", 32), ("auto", 32), ("auto", 64)):
         binding.set_path(path)
         try:
             buf = torch.full((n + 2 * guard,), 7.0, dtype=torch.float16, device="cuda")
@@ -336,7 +336,7 @@ def test_output_stays_inside_its_buffer_and_inputs_untouched():
             dv_ = {k: _dev(v) for k, v in d.items()}
             before = {k: v.clone() for k, v in dv_.items()}
             binding.gla_fwd(dv_["q"], dv_["k"], dv_["v"], dv_["g"], dv_["z"], dv_["w"], grid_h=gh,
-                            grid_w=gw, direction="RL", chunk=32, out=out)
+                            grid_w=gw, direction="RL", chunk=chunk, out=out)
             torch.cuda.synchronize()
         finally:
             binding.set_path("auto")
