@@ -178,13 +178,20 @@ def read_traffic(kernel_name: str, src_hash: str):
 
 
 def kernel_source_hash():
+    """Hash of the CUDA sources with comments and blank space removed, so that
+    a figure measured on a kernel stays attached to it through comment edits."""
     import hashlib
+    import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "linear_vision_backbone_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode())
-            h.update(f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        text = " ".join(text.split())
+        h.update(name.encode())
+        h.update(text.encode())
     return h.hexdigest()[:12]
 
 

@@ -40,16 +40,20 @@
 // its chunks last to first keeping R, the summed log-gate of the chunks
 // already seen, so every weight e^{R + Gam_c - G_s} is known when its chunk is
 // built (and is at most one for non-positive gates); all chunks accumulate
-// into one TMEM accumulator and no state passes through registers.  Its
-// staging is double-buffered: the next chunk's copies are in flight while the
-// current one is built.
+// into one TMEM accumulator and no state passes through registers.  Eight
+// warps build the tiles; a ninth issues the products and the chunk loads, so
+// the builders move on while the tensor pipe works.  Staging is double-
+// buffered two chunks ahead.
 //
 // Data movement: every token's head vector is one contiguous 128-byte row (256
-// bytes for the fp32 gate), so the scan order is applied per token as the
-// source address of 16-byte cp.async copies; no transpose kernel runs and
-// reversed orders are reversed addresses.  Rows past the end of a ragged last
-// chunk are zero-filled when the chunk is fetched (a zero gate repeats the
-// last cumsum), so no later phase tests them.
+// bytes for the fp32 gate) of a [B, T, H, D] tensor, so one head's chunk is a
+// tensor-map box: 64 consecutive tokens in scan order LR / RL, 64 consecutive
+// grid rows of one column in TB / BT (when 64 divides the grid height).  A
+// reversed scan loads the same box and walks its rows backwards.  Other
+// shapes gather the chunk per token with 16-byte cp.async copies (the scan
+// order in the source address).  No transpose kernel runs.  Rows past the end
+// of a ragged last chunk are zero-filled (a zero gate repeats the last
+// cumsum), so no later phase tests them.
 #pragma once
 #include <cuda.h>
 
