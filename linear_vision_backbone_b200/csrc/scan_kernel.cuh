@@ -27,6 +27,20 @@ constexpr int kScanParts = 4;
 constexpr int kScanThreads = 32 * kScanParts;
 constexpr int kScanReg = 12;
 
+// Pass 1 / pass 2 over `n` segments held in registers (n <= kScanReg); the
+// full-window case is unrolled without predicates.
+template <bool kFull>
+__device__ __forceinline__ void scan_window(const float* pd, const float* pa, int n, int dkdv, int dk, float (&dS)[kScanReg],
+                                            float (&a)[kScanReg]) {
+#pragma unroll
+  for (int u = 0; u < kScanReg; ++u) {
+    if (kFull || u < n) {
+      dS[u] = pd[u * dkdv];
+      a[u] = pa[u * dk];
+    }
+  }
+}
+
 // at most 64 registers: eight blocks per SM, so a 16k-token, 6-head problem
 // (768 blocks) is resident in one wave
 __global__ void __launch_bounds__(kScanThreads, 8)
@@ -36,64 +50,64 @@ gla_state_scan(float* __restrict__ wsS, const float* __restrict__ wsA, long long
   pdl_wait();                             // the summaries are complete
   pdl_trigger();
   const int lane = threadIdx.x & 31, part = threadIdx.x >> 5;
-  const long long e = (long long)blockIdx.x * 32 + lane;
-  const bool live = e < total;
+  // 32 elements per block; dk * dv is a multiple of 32, so a block stays in one (b, h)
   const int dkdv = dk * dv;
-  const long long bh = live ? e / dkdv : 0;
-  const int rem = live ? (int)(e - bh * dkdv) : 0;
+  const int per_bh = dkdv >> 5;
+  const long long bh = blockIdx.x / per_bh;
+  const int rem = (int)(blockIdx.x - bh * per_bh) * 32 + lane;
+  const bool live = (long long)blockIdx.x * 32 + lane < total;
   const int i = rem / dv;
-  float* p = wsS + (size_t)bh * nseg * dkdv + rem;
-  const float* A = wsA + (size_t)bh * nseg * dk + i;
   const int len = (nseg + kScanParts - 1) / kScanParts;
   const int sa = min(nseg, part * len), sb = min(nseg, sa + len);
+  const int n = sb - sa;
+  // this range's first segment; offsets within a (b, h) fit in 32 bits (nseg dk dv < 2^31)
+  float* p = wsS + (size_t)bh * nseg * dkdv + (size_t)sa * dkdv + rem;
+  const float* A = wsA + (size_t)bh * nseg * dk + (size_t)sa * dk + i;
 
   // pass 1: this range as one map S -> P S + R
   float dS[kScanReg], a[kScanReg];
   float P = 1.f, R = 0.f;
-  for (int s0 = sa; s0 < sb; s0 += kScanReg) {
-    const int n = min(kScanReg, sb - s0);
+  if (live) {
+    for (int s0 = 0; s0 < n; s0 += kScanReg) {
+      const int m = min(kScanReg, n - s0);
+      if (m == kScanReg) scan_window<true>(p + s0 * dkdv, A + s0 * dk, m, dkdv, dk, dS, a);
+      else scan_window<false>(p + s0 * dkdv, A + s0 * dk, m, dkdv, dk, dS, a);
 #pragma unroll
-    for (int u = 0; u < kScanReg; ++u) {
-      if (u < n && live) {
-        dS[u] = p[(size_t)(s0 + u) * dkdv];
-        a[u] = A[(size_t)(s0 + u) * dk];
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kScanReg; ++u) {
-      if (u < n && live) {
-        R = fmaf(a[u], R, dS[u]);
-        P *= a[u];
+      for (int u = 0; u < kScanReg; ++u) {
+        if (u < m) {
+          R = fmaf(a[u], R, dS[u]);
+          P *= a[u];
+        }
       }
     }
   }
   mapP[part][lane] = P;
   mapR[part][lane] = R;
   __syncthreads();
+  if (!live) return;
   // the state entering this range
   float S = 0.f;
   for (int r = 0; r < part; ++r) S = fmaf(mapP[r][lane], S, mapR[r][lane]);
-  if (!live) return;
 
-  // pass 2: the states, from registers when the range is one group
-  for (int s0 = sa; s0 < sb; s0 += kScanReg) {
-    const int n = min(kScanReg, sb - s0);
-    if (sb - sa > kScanReg) {
+  // pass 2: the states, from registers when the range is one window
+  for (int s0 = 0; s0 < n; s0 += kScanReg) {
+    const int m = min(kScanReg, n - s0);
+    if (n > kScanReg) scan_window<false>(p + s0 * dkdv, A + s0 * dk, m, dkdv, dk, dS, a);
+    float* q = p + s0 * dkdv;
+    if (inclusive) {
 #pragma unroll
-      for (int u = 0; u < kScanReg; ++u) {
-        if (u < n) {
-          dS[u] = p[(size_t)(s0 + u) * dkdv];
-          a[u] = A[(size_t)(s0 + u) * dk];
+      for (int u = 0; u < kScanReg; ++u)
+        if (u < m) {
+          S = fmaf(a[u], S, dS[u]);
+          q[u * dkdv] = S;
         }
-      }
-    }
+    } else {
 #pragma unroll
-    for (int u = 0; u < kScanReg; ++u) {
-      if (u < n) {
-        if (!inclusive) p[(size_t)(s0 + u) * dkdv] = S;
-        S = fmaf(a[u], S, dS[u]);
-        if (inclusive) p[(size_t)(s0 + u) * dkdv] = S;
-      }
+      for (int u = 0; u < kScanReg; ++u)
+        if (u < m) {
+          q[u * dkdv] = S;
+          S = fmaf(a[u], S, dS[u]);
+        }
     }
   }
 }
