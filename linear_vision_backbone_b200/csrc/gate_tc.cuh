@@ -365,11 +365,11 @@ gate_fwd_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUt
   if (warp < 4) {
     float lw[16], lt[16];
     tmem_ld16(tm + ((uint32_t)(warp * 32) << 16) + 0, lw);
-    tc::tmem_ld_wait();
+    tc::tmem_ld_wait(lw);
 #pragma unroll
     for (int t = 1; t < kTerms; ++t) {
       tmem_ld16(tm + ((uint32_t)(warp * 32) << 16) + t * kRank, lt);
-      tc::tmem_ld_wait();
+      tc::tmem_ld_wait(lt);
 #pragma unroll
       for (int c = 0; c < 16; ++c) lw[c] += lt[c];
     }
@@ -425,11 +425,8 @@ gate_fwd_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUt
     const float ri = m.low_i[r];
     const uint32_t tq = tm + ((uint32_t)(q * 32) << 16) + 64 + 16 * qp;
     const int nslab = HD / 64;
-    for (int j = 0; j < nslab; ++j) {
+    auto emit = [&](int j, const float* u) {
       uint8_t* slab = tX + (j % 3) * (2 * Layout::kHalfSlab);
-      float u[16];
-      tmem_ld16(tq + 64 * j, u);
-      tc::tmem_ld_wait();
       const int cb = 64 * j + 16 * qp;
       uint8_t* half = slab + (qp >> 1) * Layout::kHalfSlab + r * 128;
 #pragma unroll
@@ -450,6 +447,19 @@ gate_fwd_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUt
         tma_store_2d(&tmg, 64 * j, tok0, slab);
         tma_store_2d(&tmg, 64 * j + 32, tok0, slab + Layout::kHalfSlab);
         bulk_commit();
+      }
+    };
+    // the next slab's TMEM columns are requested before this one is formed
+    float ua[16], ub[16];
+    tmem_ld16(tq, ua);
+    for (int j = 0; j < nslab; j += 2) {
+      tc::tmem_ld_wait(ua);                       // slab j in ua
+      if (j + 1 < nslab) tmem_ld16(tq + 64 * (j + 1), ub);
+      emit(j, ua);
+      if (j + 1 < nslab) {
+        tc::tmem_ld_wait(ub);                     // slab j + 1 in ub
+        if (j + 2 < nslab) tmem_ld16(tq + 64 * (j + 2), ua);
+        emit(j + 1, ub);
       }
     }
     if (tid == 0) bulk_wait<0>();                 // every store done before the block ends

@@ -185,8 +185,16 @@ __device__ __forceinline__ void tmem_ld16x2(uint32_t taddr, float* v) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
-__device__ __forceinline__ void tmem_ld_wait() {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+// Wait for this thread's tcgen05.ld, tied to the 16 registers of the load so
+// that no use of them can be scheduled before it (the compiler does not know
+// the load is asynchronous).
+__device__ __forceinline__ void tmem_ld_wait(float (&v)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]),
+                 "+f"(v[7]), "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]), "+f"(v[12]), "+f"(v[13]),
+                 "+f"(v[14]), "+f"(v[15])
+               :
+               : "memory");
 }
 // barrier over `count` threads (whole warps) on hardware barrier `id` (1..15)
 __device__ __forceinline__ void named_barrier(int id, int count) {
@@ -718,7 +726,7 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
       // ---- masked scores P (rows = queries j, columns = keys i) into the q~ tiles
       float sc[16];
       tmem_ld16x2(tm + lane_base + 64 + half * 32, sc);
-      tmem_ld_wait();
+      tmem_ld_wait(sc);
 #pragma unroll
       for (int c = 0; c < 16; ++c) sc[c] = cbase + c <= row ? sc[c] : 0.f;
       put8(QH, QL, sw16(row, cbase), sc);
@@ -788,7 +796,7 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
     {
       float o[16];
       tmem_ld16x2(tm + lane_base + half * 32, o);
-      tmem_ld_wait();
+      tmem_ld_wait(o);
       float ss = 0.f;
 #pragma unroll
       for (int c = 0; c < 16; ++c) ss = fmaf(o[c], o[c], ss);
@@ -814,7 +822,7 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
     {
       float ds[16];
       tmem_ld16x2(tm + lane_base + 64 + half * 32, ds);
-      tmem_ld_wait();
+      tmem_ld_wait(ds);
       const float a = m.aG[row];
 #pragma unroll
       for (int c = 0; c < 16; ++c) S[c] = tilde ? a * (S[c] + ds[c]) : fmaf(a, S[c], ds[c]);
@@ -1075,7 +1083,8 @@ gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
     float ds[16], dl[16];
     tmem_ld16x2(tm + lane_base + half * 32, ds);
     tmem_ld16x2(tm + lane_base + 64 + half * 32, dl);
-    tmem_ld_wait();
+    tmem_ld_wait(ds);
+    tmem_ld_wait(dl);
 #pragma unroll
     for (int c = 0; c < 16; ++c) ds[c] += dl[c];
     float4* dst = reinterpret_cast<float4*>(p.wsS + (((size_t)bh * p.nseg + seg) * kD + row) * kD + cbase);
