@@ -8,27 +8,36 @@
 // Operands.  Every tensor-core operand is a pair of bf16 tiles (hi, lo) of an
 // fp32 value, hi = bf16(x), lo = bf16(x - hi), multiplied as
 // hi*hi' + hi*lo' + lo*hi' (tcgen05.mma kind::f16 with bf16 inputs, fp32
-// accumulators in tensor memory, M = N = 64, K = 16 per instruction).  A
+// accumulators in tensor memory, M = 64, N = 64 or 128, K = 16 per
+// instruction).  A
 // product carries about 16 significant bits, 32 times finer than a tf32
 // operand, and bf16 has fp32's exponent range, so no operand needs a scale
 // and products of different operands add in one accumulator.  A bf16 V is
 // used as it is (one term); an fp16 V is exactly hi + lo.
 //
 // Output kernel (gla_out_tc).  One CTA (256 threads) walks a segment of
-// consecutive chunks of one (batch, head) sequence and carries the dk x dv
-// state S in fp32 registers.  For chunk c with in-chunk inclusive log-gate
-// cumsum G_j (per key dim), G_m = G at the middle position and Gam = G at the
-// last one:
-//   q~_j = q_j e^{G_j - G_m},  k~_i = k_i e^{G_m - G_i},  S' = e^{G_m} S
-//   o_j  = q~_j S' + sum_{i<=j} (q~_j . k~_i) v_i              -> RMSNorm x SiLU(z)
-//   S   <- e^{Gam} S + diag(e^{Gam - G_m}) k~^T V
-// exp(G_j - G_i) = e^{G_j - G_m} e^{G_m - G_i} keeps both factors within
-// e^{+-span} of one, span = the chunk's own decay range.  A chunk whose span
-// exceeds kSpanMax nats, or whose gates rise above zero, evaluates its scores
-// exactly on CUDA cores instead (q~ = q e^{G}, key tile k^ = k e^{Gam - G},
-// S' = S, P_ji = sum_d q_jd k_id e^{G_jd - G_id}).
-// Tensor memory (128 columns): [0, 64) o = q~ S', then += P V; [64, 128) the
-// scores q~ k~^T, then (once P has been read out) the increment k~^T V.
+// consecutive chunks of one (batch, head) sequence and carries the state in
+// fp32 registers, transposed (S^T, rows dv).  For chunk c with in-chunk
+// inclusive log-gate cumsum G_j (per key dim) and Gam = G at its last
+// position, the factors are referenced to the chunk start:
+//   q~_j = q_j e^{G_j},  k~_i = k_i e^{-G_i}
+//   o_j  = q~_j S + sum_{i<=j} (q~_j . k~_i) v_i              -> RMSNorm x SiLU(z)
+//   S^T <- (S^T + V^T k~) diag(e^{Gam})
+// With every G_j in [-kSpanMax, 0] both factors stay within e^{kSpanMax} of
+// one (bf16 has fp32's exponent range), and each product q~_jd k~_id equals
+// q_jd k_id e^{G_jd - G_id} to the operands' precision, so the unmasked
+// scores carry no cancellation.  A chunk with a gate cumsum outside that
+// range evaluates its scores exactly on CUDA cores instead (key tile
+// k^ = k e^{Gam - G}, P_ji = sum_d q_jd k_id e^{G_jd - G_id},
+// S^T <- S^T diag(e^{Gam}) + V^T k^).  The cumsum, the exact-chunk test and
+// the operand build run as one pass: each warp takes eight tokens, each lane
+// two dims, so every shared-memory access of a warp is one whole 128-byte row.
+// An MMA instruction costs about the same for N = 128 as for N = 64, so o and
+// the scores come from one N = 128 product q~ [S^T; k~]^T (the state tile
+// and the key tile adjacent in shared memory, K-major).
+// Tensor memory (128 columns): [0, 64) o = q~ S, then += P V; [64, 128) the
+// scores q~ k~^T, then (once P has been read out) the increment (V^T k~)^T
+// with rows dv, matching the transposed state.
 // Row phases (P, epilogue, state) run four threads per accumulator row: warp w
 // reads the 16 TMEM lanes of quadrant w % 4 that an M = 64 accumulator uses
 // (row r -> lane 32 (r / 16) + r % 16) with the 16x32bx2 shape, half w / 4 of
@@ -228,10 +237,11 @@ __device__ __forceinline__ uint64_t desc_k(const void* tile) { return sdesc(sadd
 // MN-major tile: a K step of 16 rows is two 8-row atoms, 2048 bytes.
 __device__ __forceinline__ uint64_t desc_mn(const void* tile) { return sdesc(saddr(tile), 8192, 1024); }
 constexpr uint32_t kStepK = 32 >> 4, kStepMN = 2048 >> 4;   // descriptor address units per K step
-// Instruction descriptor: kind::f16 with bf16 A and B, fp32 accumulate, M = N = 64.
-__host__ __device__ constexpr uint32_t idesc_bf16(int a_mn, int b_mn) {
+// Instruction descriptor: kind::f16 with bf16 A and B, fp32 accumulate, M = 64,
+// N = n (64 unless given).
+__host__ __device__ constexpr uint32_t idesc_bf16(int a_mn, int b_mn, int n = 64) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
-         ((uint32_t)(64 >> 3) << 17) | ((uint32_t)(64 >> 4) << 24);
+         ((uint32_t)(n >> 3) << 17) | ((uint32_t)(64 >> 4) << 24);
 }
 // One tcgen05.mma kind::f16 instruction; the instruction descriptor selects
 // fp16 or bf16 operands.
@@ -257,6 +267,14 @@ __device__ __forceinline__ void mma_terms(uint32_t d, uint64_t ah, uint64_t al, 
   mma_k64<SA, SB>(d, ah, bh, id, acc);
   if (b_two) mma_k64<SA, SB>(d, ah, bl, id, true);
   mma_k64<SA, SB>(d, al, bh, id, true);
+}
+// The same with the optional second term on A: a bh + a bl for a one-term A.
+template <uint32_t SA, uint32_t SB>
+__device__ __forceinline__ void mma_terms_a(uint32_t d, uint64_t ah, uint64_t al, uint64_t bh,
+                                            uint64_t bl, bool a_two, uint32_t id, bool acc) {
+  mma_k64<SA, SB>(d, ah, bh, id, acc);
+  mma_k64<SA, SB>(d, ah, bl, id, true);
+  if (a_two) mma_k64<SA, SB>(d, al, bh, id, true);
 }
 
 // --------------------------------------------------- two-term bf16 operands
@@ -438,7 +456,7 @@ __device__ __forceinline__ float silu_fast(float z) { return __fdividef(z, 1.0f 
 
 // ===================================================================== K4
 struct OutMisc {                  // per-CTA scalars; arrays read as float4 are 16-byte aligned
-  uint64_t mma[3];                // [0] q~ S and scores (two arrivals), [1] + P V, [2] state increment
+  uint64_t mma[3];                // [0] q~ S and the scores, [1] + P V, [2] state increment
   uint64_t ld;                    // a chunk's box loads
   uint32_t tmem;
   int pad;
@@ -452,8 +470,10 @@ struct OutMisc {                  // per-CTA scalars; arrays read as float4 are 
 struct OutLayout {
   // staging: k, q (row-major), v (operand layout), gate (row-major fp32)
   static constexpr int kOffK = 0, kOffQ = kTile, kOffV = 2 * kTile, kOffG = 3 * kTile;
-  // operand tiles (1024-aligned): VH VL QH QL KH KL SH SL.  A bf16 v read in
-  // scan order lands directly in VH / VL, alternately by chunk parity.
+  // operand tiles (1024-aligned): VH VL QH QL SH KH SL KL.  The state tile
+  // S^T and the key tile are adjacent, so that [S^T; k~] is one 128-row
+  // K-major B operand.  A bf16 v read in scan order lands directly in VH / VL,
+  // alternately by chunk parity.
   static constexpr int kTiles = 3 * kTile + kGTile;
   static constexpr int kMisc = kTiles + 8 * kTile;
   static constexpr int kSmem = kMisc + (int)sizeof(OutMisc) + 1024;   // + alignment slack
@@ -498,10 +518,10 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
   uint8_t* VL = VH + kTile;
   uint8_t* QH = VH + 2 * kTile;       // q~, then P (K-major A)
   uint8_t* QL = VH + 3 * kTile;
-  uint8_t* KH = VH + 4 * kTile;       // k~ or k^: K-major B of the scores, MN-major A of k^T V
-  uint8_t* KL = VH + 5 * kTile;
-  uint8_t* SH = VH + 6 * kTile;       // S (MN-major B)
-  uint8_t* SL = VH + 7 * kTile;
+  uint8_t* SH = VH + 4 * kTile;       // S^T, rows dv: rows 0-63 of the K-major B [S^T; k~]
+  uint8_t* KH = VH + 5 * kTile;       // k~ or k^: rows 64-127 of that B; MN-major B of V^T k~
+  uint8_t* SL = VH + 6 * kTile;
+  uint8_t* KL = VH + 7 * kTile;
   OutMisc& m = *reinterpret_cast<OutMisc*>(sm + L::kMisc);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -539,7 +559,7 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
   const int dc = 2 * lane, tb = 8 * warp;
 
   if (tid == 0) {
-    mbar_init(&m.mma[0], 2);
+    mbar_init(&m.mma[0], 1);
     mbar_init(&m.mma[1], 1);
     mbar_init(&m.mma[2], 1);
     mbar_init(&m.ld, 1);
@@ -560,16 +580,13 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
   // that), so chunk 0 is fetched above; the boundary states need the wait.
   pdl_wait();
   pdl_trigger();
-  // carried state: S[row][cbase .. cbase + 15], from the boundary scan
+  // carried state, transposed: S[c] = S^T[row][cbase + c] = S[cbase + c][row]
+  // (row a dv index), from the boundary scan's [dk][dv] states
   float S[16];
   {
-    const float4* src = reinterpret_cast<const float4*>(
-        p.wsS + (((size_t)bh * p.nseg + seg) * kD + row) * kD + cbase);
+    const float* src = p.wsS + ((size_t)bh * p.nseg + seg) * kD * kD + (size_t)cbase * kD + row;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const float4 x = src[c];
-      S[4 * c] = x.x; S[4 * c + 1] = x.y; S[4 * c + 2] = x.z; S[4 * c + 3] = x.w;
-    }
+    for (int c = 0; c < 16; ++c) S[c] = src[c * kD];
   }
   if (warp == 0) {
     tmem_alloc(&m.tmem, L::kTmemCols);
@@ -580,9 +597,10 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
   __syncthreads();
   tc_after_sync();
   const uint32_t tm = m.tmem;
-  constexpr uint32_t kIdQS = idesc_bf16(0, 1);   // A K-major, B MN-major: q~ S, P V
-  constexpr uint32_t kIdQK = idesc_bf16(0, 0);   // both K-major: q~ k~^T
-  constexpr uint32_t kIdKV = idesc_bf16(1, 1);   // both MN-major: k~^T V
+  constexpr uint32_t kIdQSK = idesc_bf16(0, 0, 128);   // both K-major, N = 128: q~ [S^T; k~]^T
+  constexpr uint32_t kIdQS = idesc_bf16(0, 0);          // both K-major: q~ S (an exact chunk)
+  constexpr uint32_t kIdPV = idesc_bf16(0, 1);          // A K-major, B MN-major: P V
+  constexpr uint32_t kIdVK = idesc_bf16(1, 1);          // both MN-major: V^T k~
 
   uint32_t ph0 = 0, ph1 = 0, ph2 = 0, phl = 0;
   bool failed = false, ld_pending = tma;
@@ -675,20 +693,16 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
     const bool tilde = !exact;
     tc_after_sync();
 
-    // Two issuing threads: a single thread issues one MMA per ~60 cycles
-    // whatever its size, so independent products go out from two warps and
-    // the tensor pipe interleaves them.  Warp 0 owns o (q~ S, later P V),
-    // warp 4 the score columns (scores, later the state increment); each
-    // thread's own MMAs execute in issue order.  P overwrites q~, so mma[0]
-    // completes only when both threads' products are done.
+    // An MMA instruction costs about as much for N = 128 as for N = 64, so o
+    // and the scores come from one N = 128 product q~ [S^T; k~]^T (o alone for
+    // an exact chunk), issued by warp 0; later warp 0 adds P V onto o and warp
+    // 4 forms the state increment, each thread's MMAs in issue order.
     if (tid == 0) {
-      mma_terms<kStepK, kStepMN>(tm + 0, desc_k(QH), desc_k(QL), desc_mn(SH), desc_mn(SL), true, kIdQS,
-                                 false);
-      mma_commit(&m.mma[0]);
-    }
-    if (tid == 128) {
       if (tilde)
-        mma_terms<kStepK, kStepK>(tm + 64, desc_k(QH), desc_k(QL), desc_k(KH), desc_k(KL), true, kIdQK,
+        mma_terms<kStepK, kStepK>(tm + 0, desc_k(QH), desc_k(QL), desc_k(SH), desc_k(SL), true, kIdQSK,
+                                  false);
+      else
+        mma_terms<kStepK, kStepK>(tm + 0, desc_k(QH), desc_k(QL), desc_k(SH), desc_k(SL), true, kIdQS,
                                   false);
       mma_commit(&m.mma[0]);
     }
@@ -765,13 +779,14 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
     }
     cp_async_commit();
     if (tid == 0) {
-      mma_terms<kStepK, kStepMN>(tm + 0, desc_k(QH), desc_k(QL), desc_mn(Vh), desc_mn(Vl), kV2, kIdQS,
+      mma_terms<kStepK, kStepMN>(tm + 0, desc_k(QH), desc_k(QL), desc_mn(Vh), desc_mn(Vl), kV2, kIdPV,
                                  true);
       mma_commit(&m.mma[1]);
     }
     if (tid == 128) {
-      mma_terms<kStepMN, kStepMN>(tm + 64, desc_mn(KH), desc_mn(KL), desc_mn(Vh), desc_mn(Vl), kV2,
-                                  kIdKV, false);
+      // (V^T k~)^T rows dv: A = V read MN-major, B = the key tile read MN-major
+      mma_terms_a<kStepMN, kStepMN>(tm + 64, desc_mn(Vh), desc_mn(Vl), desc_mn(KH), desc_mn(KL), kV2,
+                                    kIdVK, false);
       mma_commit(&m.mma[2]);
     }
     // the output gate w * SiLU(z) while P V and the increment run
@@ -815,7 +830,8 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
       }
     }
 
-    // ---- state: S <- e^{Gam} (S + k~^T V), or e^{Gam} S + k^^T V for an exact chunk
+    // ---- state, transposed: S^T <- (S^T + V^T k~) diag(e^{Gam}), or
+    // S^T diag(e^{Gam}) + V^T k^ for an exact chunk
     failed |= !mbar_wait(&m.mma[2], ph2);
     ph2 ^= 1;
     tc_after_sync();
@@ -823,9 +839,14 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
       float ds[16];
       tmem_ld16x2(tm + lane_base + 64 + half * 32, ds);
       tmem_ld_wait(ds);
-      const float a = m.aG[row];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) S[c] = tilde ? a * (S[c] + ds[c]) : fmaf(a, S[c], ds[c]);
+      for (int c = 0; c < 16; c += 4) {
+        const float4 a = *reinterpret_cast<const float4*>(&m.aG[cbase + c]);
+        S[c + 0] = tilde ? a.x * (S[c + 0] + ds[c + 0]) : fmaf(a.x, S[c + 0], ds[c + 0]);
+        S[c + 1] = tilde ? a.y * (S[c + 1] + ds[c + 1]) : fmaf(a.y, S[c + 1], ds[c + 1]);
+        S[c + 2] = tilde ? a.z * (S[c + 2] + ds[c + 2]) : fmaf(a.z, S[c + 2], ds[c + 2]);
+        S[c + 3] = tilde ? a.w * (S[c + 3] + ds[c + 3]) : fmaf(a.w, S[c + 3], ds[c + 3]);
+      }
     }
     cp_async_wait<0>();                   // the next chunk's copies made by this thread
     tc_before_sync();
