@@ -120,6 +120,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity) {
     if (globaltimer() - t0 > kWaitNs) return false;
   return true;
 }
+// One plain arrival.
+__device__ __forceinline__ void mbar_arrive_one(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(saddr(b)) : "memory");
+}
 // One arrival that also expects `bytes` of asynchronous copies on the barrier.
 __device__ __forceinline__ void mbar_arrive_tx(uint64_t* b, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(b)), "r"(bytes)
@@ -208,6 +212,19 @@ __device__ __forceinline__ void tmem_ld_wait(float (&v)[16]) {
 // barrier over `count` threads (whole warps) on hardware barrier `id` (1..15)
 __device__ __forceinline__ void named_barrier(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+// The same barrier, also OR-ing a predicate across its threads.
+__device__ __forceinline__ bool named_barrier_or(int id, int count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %3, 0;\n\t"
+      "barrier.cta.red.or.pred q, %1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(id), "r"(count), "r"((uint32_t)pred)
+      : "memory");
+  return r != 0;
 }
 // 2^x by the hardware approximation (ex2.approx, flush-to-zero)
 __device__ __forceinline__ float ex2(float x) {
@@ -455,9 +472,10 @@ __device__ __forceinline__ float column_cumsum(const float* G, float (&gv)[16], 
 __device__ __forceinline__ float silu_fast(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
 // ===================================================================== K4
-struct OutMisc {                  // per-CTA scalars; arrays read as float4 are 16-byte aligned
+struct OutMisc {                  // per-chain scalars; arrays read as float4 are 16-byte aligned
   uint64_t mma[3];                // [0] q~ S and the scores, [1] + P V, [2] state increment
   uint64_t ld;                    // a chunk's box loads
+  uint64_t built;                 // this chain has built a chunk's tiles (the other chain's turn)
   uint32_t tmem;
   int pad;
   alignas(16) float part[kWarps][kD];   // cumsum partials: tokens 8 w .. 8 w + 7, per dim
@@ -468,7 +486,9 @@ struct OutMisc {                  // per-CTA scalars; arrays read as float4 are 
   alignas(16) long long rows[2][kC];   // token rows of the current / next chunk
 };
 struct OutLayout {
-  // staging: k, q (row-major), v (operand layout), gate (row-major fp32)
+  // Two chains per CTA (warps 0-7 and 8-15), each with the layout below at
+  // offset kChain * chain.  Staging: k, q (row-major), v (operand layout),
+  // gate (row-major fp32).
   static constexpr int kOffK = 0, kOffQ = kTile, kOffV = 2 * kTile, kOffG = 3 * kTile;
   // operand tiles (1024-aligned): VH VL QH QL SH KH SL KL.  The state tile
   // S^T and the key tile are adjacent, so that [S^T; k~] is one 128-row
@@ -476,9 +496,11 @@ struct OutLayout {
   // alternately by chunk parity.
   static constexpr int kTiles = 3 * kTile + kGTile;
   static constexpr int kMisc = kTiles + 8 * kTile;
-  static constexpr int kSmem = kMisc + (int)sizeof(OutMisc) + 1024;   // + alignment slack
-  static constexpr int kTmemCols = 128;
-  static constexpr int kBlocksPerSM = 2;
+  static constexpr int kChain = (kMisc + (int)sizeof(OutMisc) + 1023) & ~1023;
+  static constexpr int kSmem = 2 * kChain + 1024;   // + alignment slack
+  static constexpr int kTmemCols = 256;             // 128 per chain
+  static constexpr int kThreadsAll = 2 * kThreads;
+  static constexpr int kChainsPerSM = 2;
 };
 static_assert(OutLayout::kTiles % 1024 == 0, "operand tiles must be 1024-byte aligned");
 
@@ -491,26 +513,37 @@ __device__ __forceinline__ void fetch_chunk(uint8_t* sm, uint8_t* vdst, const Pa
   fetch16<true>(vdst, p.v, rows, ntok, tid);
   fetch_g(sm + OutLayout::kOffG, p.g, rows, ntok, tid);
 }
-static_assert(2 * (OutLayout::kSmem + 1024) <= 228 * 1024, "two output CTAs must share an SM");
+static_assert(OutLayout::kSmem <= 227 * 1024, "the two-chain output CTA must fit one SM");
 
 // Sum over the four threads that share an accumulator row: the other half of
 // the warp (lane ^ 16) and the same lanes of the partner warp (warp ^ 4),
-// through shared memory and a named barrier of those two warps.
-__device__ __forceinline__ float row_combine_sum(float v, float (*red)[kD], int row, int half, int qd,
+// through shared memory and a named barrier (`bar`) of those two warps.
+__device__ __forceinline__ float row_combine_sum(float v, float (*red)[kD], int row, int half, int bar,
                                                  int lane) {
   v += __shfl_xor_sync(0xffffffffu, v, 16);
   if (lane < 16) red[half][row] = v;
-  named_barrier(1 + qd, 64);
+  named_barrier(bar, 64);
   return v + red[half ^ 1][row];
 }
 
+// Two chains per CTA: warps 0-7 walk segment 2 blockIdx.x, warps 8-15 segment
+// 2 blockIdx.x + 1, each with its own shared memory, TMEM columns and
+// barriers (chain barrier 1 + 5 g over 256 threads, row-pair barriers
+// 2 + 5 g + qd).  Their tile-build phases alternate (chain 0 builds chunk i
+// after chain 1 has built chunk i - 1, chain 1 builds chunk i after chain 0
+// has built chunk i), so each chain's build overlaps the other's MMAs, P and
+// epilogue instead of contending with its build.
 template <typename T>
-__global__ void __launch_bounds__(kThreads, OutLayout::kBlocksPerSM)
+__global__ void __launch_bounds__(OutLayout::kThreadsAll, 1)
 gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
   using L = OutLayout;
   constexpr bool kV2 = std::is_same<T, __half>::value;   // fp16 V: two bf16 terms
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const int chain = threadIdx.x >> 8;
+  uint8_t* const sm0 = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sm = sm0 + chain * L::kChain;
+  OutMisc& m_other = *reinterpret_cast<OutMisc*>(sm0 + (chain ^ 1) * L::kChain + L::kMisc);
+  const int bar_all = 1 + 5 * chain, bar_pair = 2 + 5 * chain;
   const T* kst = reinterpret_cast<const T*>(sm + L::kOffK);
   const T* qst = reinterpret_cast<const T*>(sm + L::kOffQ);
   float* G = reinterpret_cast<float*>(sm + L::kOffG);
@@ -524,16 +557,21 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
   uint8_t* KL = VH + 7 * kTile;
   OutMisc& m = *reinterpret_cast<OutMisc*>(sm + L::kMisc);
 
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int seg = blockIdx.x, bh = blockIdx.y;
+  const int tid = threadIdx.x & (kThreads - 1), warp = tid >> 5, lane = tid & 31;
+  const int seg = 2 * blockIdx.x + chain, bh = blockIdx.y;
   const int b = bh / p.H, h = bh - b * p.H;
   const int d = dir_of_batch(p.dir, b);
   const int nc = (p.T + kC - 1) / kC;
-  const int c0 = seg_first_chunk(seg, nc, p.nseg);
-  const int nch = seg_first_chunk(seg + 1, nc, p.nseg) - c0;
-  if (d < 0 || d > 3 || nch <= 0) {
-    if (tid == 0) gtr_flag(d < 0 || d > 3 ? kStatusBadDir : kStatusBadShape);
-    return;
+  // chunks of each chain (a chain past the last segment has none)
+  auto chunks_of = [&](int sg) {
+    return sg < p.nseg ? seg_first_chunk(sg + 1, nc, p.nseg) - seg_first_chunk(sg, nc, p.nseg) : 0;
+  };
+  const int c0 = seg < p.nseg ? seg_first_chunk(seg, nc, p.nseg) : 0;
+  int nch = chunks_of(seg);
+  const int nch_other = (d < 0 || d > 3) ? 0 : chunks_of(seg ^ 1);
+  if (d < 0 || d > 3) {
+    if (tid == 0) gtr_flag(kStatusBadDir);
+    nch = 0;
   }
   const bool tma = p.tma != 0;
   // staging row of scan offset i: box loads of a reversed scan hold the chunk backwards
@@ -563,13 +601,14 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
     mbar_init(&m.mma[1], 1);
     mbar_init(&m.mma[2], 1);
     mbar_init(&m.ld, 1);
+    mbar_init(&m.built, 1);
     mbar_fence_init();
   }
   // chunk 0's copies go out first
-  {
+  if (nch > 0) {
     const int ntok0 = min(kC, p.T - c0 * kC);
     chunk_rows(p, m.rows[0], b, h, d, c0 * kC, ntok0, tid);
-    __syncthreads();
+    named_barrier(bar_all, kThreads);
     fetch(0, c0 * kC, ntok0, m.rows[0]);
     cp_async_commit();
   }
@@ -583,27 +622,28 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
   // carried state, transposed: S[c] = S^T[row][cbase + c] = S[cbase + c][row]
   // (row a dv index), from the boundary scan's [dk][dv] states
   float S[16];
-  {
+  if (nch > 0) {
     const float* src = p.wsS + ((size_t)bh * p.nseg + seg) * kD * kD + (size_t)cbase * kD + row;
 #pragma unroll
     for (int c = 0; c < 16; ++c) S[c] = src[c * kD];
   }
-  if (warp == 0) {
-    tmem_alloc(&m.tmem, L::kTmemCols);
+  OutMisc& m0 = *reinterpret_cast<OutMisc*>(sm0 + L::kMisc);
+  if (threadIdx.x < 32) {
+    tmem_alloc(&m0.tmem, L::kTmemCols);
     tmem_relinquish();
   }
   cp_async_wait<0>();                     // chunk 0's k, q, v, g (copied by this thread)
   tc_before_sync();
-  __syncthreads();
+  __syncthreads();                        // both chains: their barriers and the TMEM columns
   tc_after_sync();
-  const uint32_t tm = m.tmem;
+  const uint32_t tm = m0.tmem + 128u * (uint32_t)chain;
   constexpr uint32_t kIdQSK = idesc_bf16(0, 0, 128);   // both K-major, N = 128: q~ [S^T; k~]^T
   constexpr uint32_t kIdQS = idesc_bf16(0, 0);          // both K-major: q~ S (an exact chunk)
   constexpr uint32_t kIdPV = idesc_bf16(0, 1);          // A K-major, B MN-major: P V
   constexpr uint32_t kIdVK = idesc_bf16(1, 1);          // both MN-major: V^T k~
 
   uint32_t ph0 = 0, ph1 = 0, ph2 = 0, phl = 0;
-  bool failed = false, ld_pending = tma;
+  bool failed = false, ld_pending = tma && nch > 0;   // chunk 0's boxes
   // The next chunk's k, q, v, g are requested once this chunk's tiles are
   // built (after P for an exact chunk, whose scores still read the staging);
   // z goes straight to registers, requested two phases before the epilogue.
@@ -616,6 +656,11 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
     const int ntok1 = more ? min(kC, p.T - s1) : 0;
     uint8_t* const Vh = vdirect ? vtile(it) : VH;
     uint8_t* const Vl = vdirect ? Vh : VL;      // VL is read only for a two-term (fp16) v
+    // this chain's turn to build: chain 0 after the other's chunk it - 1, chain 1 after its chunk it
+    {
+      const int j = chain == 0 ? it - 1 : it;
+      if (j >= 0 && j < nch_other) failed |= !mbar_wait(&m_other.built, (uint32_t)j & 1u);
+    }
     if (tma) {
       failed |= !mbar_wait(&m.ld, phl);
       phl ^= 1;
@@ -631,7 +676,7 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
       if (i) { gc[i].x += gc[i - 1].x; gc[i].y += gc[i - 1].y; }
     }
     *reinterpret_cast<float2*>(&m.part[warp][dc]) = gc[7];
-    __syncthreads();
+    named_barrier(bar_all, kThreads);
     {
       float2 off = make_float2(0.f, 0.f);
 #pragma unroll
@@ -689,9 +734,10 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
     fence_async_smem();
     tc_before_sync();
     // with G in [-kSpanMax, 0] everywhere no factor leaves [e^{-kSpanMax}, e^{kSpanMax}]
-    const bool exact = __syncthreads_or(bad) != 0;
+    const bool exact = named_barrier_or(bar_all, kThreads, bad != 0);
     const bool tilde = !exact;
     tc_after_sync();
+    if (tid == 0) mbar_arrive_one(&m.built);   // the other chain may build now
 
     // An MMA instruction costs about as much for N = 128 as for N = 64, so o
     // and the scores come from one N = 128 product q~ [S^T; k~]^T (o alone for
@@ -723,7 +769,7 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
         const float2 kk = ld2(kst + (r ^ rmask) * kD + dc);
         put2x(KH, KL, sw16(r, dc), kk.x * expf(gam.x - gc[i].x), kk.y * expf(gam.y - gc[i].y));
       }
-      __syncthreads();
+      named_barrier(bar_all, kThreads);
     }
     // this chunk's z for the epilogue: 16 elements of the thread's row
     uint4 zz0 = make_uint4(0u, 0u, 0u, 0u), zz1 = zz0;
@@ -771,7 +817,7 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
     }
     fence_async_smem();
     tc_before_sync();
-    if (__syncthreads_or(failed)) break;
+    if (named_barrier_or(bar_all, kThreads, failed)) { failed = true; break; }
     tc_after_sync();
     if (more && exact) {
       fetch(it + 1, s1, ntok1, m.rows[par ^ 1]);
@@ -815,7 +861,7 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
       float ss = 0.f;
 #pragma unroll
       for (int c = 0; c < 16; ++c) ss = fmaf(o[c], o[c], ss);
-      ss = row_combine_sum(ss, m.red, row, half, qd, lane);
+      ss = row_combine_sum(ss, m.red, row, half, bar_pair + qd, lane);
       if (row < ntok) {
         const float inv = rsqrtf(ss * (1.0f / kD) + kRmsEps);
         T* dst = reinterpret_cast<T*>(p.out) + m.rows[par][row] * kD + cbase;
@@ -850,17 +896,20 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
     }
     cp_async_wait<0>();                   // the next chunk's copies made by this thread
     tc_before_sync();
-    if (__syncthreads_or(failed)) break;
+    if (named_barrier_or(bar_all, kThreads, failed)) { failed = true; break; }
     tc_after_sync();
   }
+  // after an early exit the other chain may still wait for this one's turns
+  if (failed && tid == 0)
+    for (int j = 0; j < 2; ++j) mbar_arrive_one(&m.built);
 
   cp_async_wait<0>();                     // no copy may land after the block exits
   if (ld_pending && !mbar_wait(&m.ld, phl)) failed = true;
   if (failed && tid == 0) gtr_flag(kStatusMbarTimeout);
   tc_before_sync();
-  __syncthreads();
+  __syncthreads();                        // both chains
   tc_after_sync();
-  if (warp == 0) tmem_dealloc(tm, L::kTmemCols);
+  if (threadIdx.x < 32) tmem_dealloc(m0.tmem, L::kTmemCols);
 }
 
 // ===================================================================== K2
@@ -1129,7 +1178,8 @@ gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
 inline bool tc_shape_supported(int dk, int dv, int chunk, int dtype) {
   return dk == tc::kD && dv == tc::kD && chunk == tc::kC && (dtype == kF16 || dtype == kBF16);
 }
-inline int tc_blocks_per_sm(int, int) { return tc::OutLayout::kBlocksPerSM; }
+// segments resident per SM (the output kernel's chains; the summary kernel's blocks)
+inline int tc_blocks_per_sm(int, int) { return tc::OutLayout::kChainsPerSM; }
 
 template <typename K, typename... Args>
 inline int launch_tc_kernel(K kern, int smem, int threads, int nseg, int BH, cudaStream_t st, bool* done,
@@ -1150,8 +1200,8 @@ inline int launch_tc_typed(int stage, const tc::Params& p, const tc::Maps& mp, i
   if (stage == 0)
     return launch_tc_kernel(tc::gla_sum_tc<T>, tc::SumLayout::kSmem, tc::SumLayout::kThreadsAll, p.nseg, BH, st,
                             done_sum, dev, p, mp);
-  return launch_tc_kernel(tc::gla_out_tc<T>, tc::OutLayout::kSmem, tc::kThreads, p.nseg, BH, st, done_out, dev,
-                          p, mp);
+  return launch_tc_kernel(tc::gla_out_tc<T>, tc::OutLayout::kSmem, tc::OutLayout::kThreadsAll, (p.nseg + 1) / 2,
+                          BH, st, done_out, dev, p, mp);
 }
 
 // `maps`: tensor maps of q, k, v, g for the output stage's box loads, or
