@@ -35,9 +35,12 @@
 // An MMA instruction costs about the same for N = 128 as for N = 64, so o and
 // the scores come from one N = 128 product q~ [S^T; k~]^T (the state tile
 // and the key tile adjacent in shared memory, K-major).
-// Tensor memory (128 columns): [0, 64) o = q~ S, then += P V; [64, 128) the
-// scores q~ k~^T, then (once P has been read out) the increment (V^T k~)^T
-// with rows dv, matching the transposed state.
+// Tensor memory (256 columns per chain): [0, 64) o = q~ S, then += P V;
+// [64, 128) the scores q~ k~^T, then (once P has been read out) the
+// increment (V^T k~)^T with rows dv, matching the transposed state;
+// [128, 192) the masked two-term P, written back from registers as the
+// tensor-memory A operand of P V (no shared-memory round trip; an exact
+// chunk's CUDA-core P goes through the q~ tiles instead).
 // Row phases (P, epilogue, state) run four threads per accumulator row: warp w
 // reads the 16 TMEM lanes of quadrant w % 4 that an M = 64 accumulator uses
 // (row r -> lane 32 (r / 16) + r % 16) with the 16x32bx2 shape, half w / 4 of
@@ -209,6 +212,16 @@ __device__ __forceinline__ void tmem_ld_wait(float (&v)[16]) {
                :
                : "memory");
 }
+// 16 lanes x 32 bit in two halves, eight columns each (the store counterpart
+// of tmem_ld16x2 at half the width): thread t of warp w writes lane
+// 32(w%4) + t%16, columns [c, c+8) for t < 16 and [c+8, c+16) for t >= 16.
+__device__ __forceinline__ void tmem_st8x2(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.16x32bx2.x8.b32 [%0], 8, {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 // barrier over `count` threads (whole warps) on hardware barrier `id` (1..15)
 __device__ __forceinline__ void named_barrier(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
@@ -270,6 +283,31 @@ __device__ __forceinline__ void mma_f16(uint32_t d, uint64_t a, uint64_t b, uint
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
       "l"(a), "l"(b), "r"(idesc), "r"(acc)
       : "memory");
+}
+// One tcgen05.mma kind::f16 with A in tensor memory (M = 64: row r in lane
+// 32 (r / 16) + r % 16, two 16-bit elements per 32-bit column, the even one
+// in the low half; a K = 16 step is 8 columns).
+__device__ __forceinline__ void mma_f16_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                           uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// d += (ah + al)(bh + bl) ~ ah bh + ah bl + al bh over K = 64, A in tensor memory
+template <uint32_t SB>
+__device__ __forceinline__ void mma_terms_ts(uint32_t d, uint32_t ah, uint32_t al, uint64_t bh, uint64_t bl,
+                                             bool b_two, uint32_t id) {
+#pragma unroll
+  for (uint32_t s = 0; s < 4; ++s) mma_f16_ts(d, ah + 8 * s, bh + s * SB, id, 1u);
+  if (b_two) {
+#pragma unroll
+    for (uint32_t s = 0; s < 4; ++s) mma_f16_ts(d, ah + 8 * s, bl + s * SB, id, 1u);
+  }
+#pragma unroll
+  for (uint32_t s = 0; s < 4; ++s) mma_f16_ts(d, al + 8 * s, bh + s * SB, id, 1u);
 }
 // d (+)= A B over K = 64: four K = 16 instructions.
 template <uint32_t SA, uint32_t SB>
@@ -498,7 +536,8 @@ struct OutLayout {
   static constexpr int kMisc = kTiles + 8 * kTile;
   static constexpr int kChain = (kMisc + (int)sizeof(OutMisc) + 1023) & ~1023;
   static constexpr int kSmem = 2 * kChain + 1024;   // + alignment slack
-  static constexpr int kTmemCols = 256;             // 128 per chain
+  // per chain: o [0, 64), scores / increment [64, 128), P hi [128, 160), P lo [160, 192)
+  static constexpr int kTmemCols = 512;             // 256 per chain
   static constexpr int kThreadsAll = 2 * kThreads;
   static constexpr int kChainsPerSM = 2;
 };
@@ -636,7 +675,7 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
   tc_before_sync();
   __syncthreads();                        // both chains: their barriers and the TMEM columns
   tc_after_sync();
-  const uint32_t tm = m0.tmem + 128u * (uint32_t)chain;
+  const uint32_t tm = m0.tmem + 256u * (uint32_t)chain;
   constexpr uint32_t kIdQSK = idesc_bf16(0, 0, 128);   // both K-major, N = 128: q~ [S^T; k~]^T
   constexpr uint32_t kIdQS = idesc_bf16(0, 0);          // both K-major: q~ S (an exact chunk)
   constexpr uint32_t kIdPV = idesc_bf16(0, 1);          // A K-major, B MN-major: P V
@@ -789,8 +828,13 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
       tmem_ld_wait(sc);
 #pragma unroll
       for (int c = 0; c < 16; ++c) sc[c] = cbase + c <= row ? sc[c] : 0.f;
-      put8(QH, QL, sw16(row, cbase), sc);
-      put8(QH, QL, sw16(row, cbase + 8), sc + 8);
+      // two-term P straight back into tensor memory: the A operand of P V
+      uint32_t ph[8], pl[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) split2(sc[2 * e], sc[2 * e + 1], ph[e], pl[e]);
+      tmem_st8x2(tm + lane_base + 128 + half * 16, ph);
+      tmem_st8x2(tm + lane_base + 160 + half * 16, pl);
+      tmem_st_wait();
     } else {
       // exact scores on CUDA cores: P_ji = sum_d q_jd k_id e^{G_jd - G_id}; four threads per row
       if (tid == 0) atomicAdd(&g_gtr_exact_chunks, 1ull);
@@ -825,8 +869,11 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
     }
     cp_async_commit();
     if (tid == 0) {
-      mma_terms<kStepK, kStepMN>(tm + 0, desc_k(QH), desc_k(QL), desc_mn(Vh), desc_mn(Vl), kV2, kIdPV,
-                                 true);
+      if (tilde)
+        mma_terms_ts<kStepMN>(tm + 0, tm + 128, tm + 160, desc_mn(Vh), desc_mn(Vl), kV2, kIdPV);
+      else   // an exact chunk's P is in the q~ tiles
+        mma_terms<kStepK, kStepMN>(tm + 0, desc_k(QH), desc_k(QL), desc_mn(Vh), desc_mn(Vl), kV2, kIdPV,
+                                   true);
       mma_commit(&m.mma[1]);
     }
     if (tid == 128) {
