@@ -162,7 +162,8 @@ static_assert(Pack::kBytes % 16 == 0 && Pack::kScaleBytes % 16 == 0, "bulk copie
 
 struct Misc {
   uint64_t mma[2];
-  uint64_t ld;                       // the x tile and the packed weights
+  uint64_t ld;                       // the packed weights
+  uint64_t ldx[kMaxDm / 64];         // the x tile, one 64-column atom each
   uint32_t tmem;
   int pad;
   alignas(16) float wd_i[kRank];     // inverse W_down rank scales; wu_i follows (one bulk copy)
@@ -320,6 +321,7 @@ gate_fwd_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUt
 
   if (tid == 0) {
     tc::mbar_init(&m.ld, 1);
+    for (int a = 0; a < kMaxDm / 64; ++a) tc::mbar_init(&m.ldx[a], 1);
     tc::mbar_init(&m.mma[0], 1);
     tc::mbar_init(&m.mma[1], 1);
     tc::mbar_fence_init();
@@ -335,30 +337,41 @@ gate_fwd_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUt
   pdl_trigger();
   const int natoms = dm / 64;
   if (tid == 0) {
-    mbar_expect_tx(&m.ld, (uint32_t)(natoms * (kM * 128) + Pack::kWdBytes + Pack::kWuBytes + Pack::kScaleBytes));
-    for (int a = 0; a < natoms; ++a) tma_load_2d(tX + a * (kM * 128), &tmx, a * 64, tok0, &m.ld);
+    // the weights first (shared by every block, mostly from L2), then the x
+    // atoms, each on its own barrier so stage 1 starts with the first
+    mbar_expect_tx(&m.ld, (uint32_t)(Pack::kWdBytes + Pack::kWuBytes + Pack::kScaleBytes));
     bulk_g2s(tWd, pack + Pack::kOffWd, Pack::kWdBytes, &m.ld);
     bulk_g2s(tWu, pack + Pack::kOffWu, Pack::kWuBytes, &m.ld);
     bulk_g2s(&m.wd_i[0], pack + Pack::kOffScale, Pack::kScaleBytes, &m.ld);
+    for (int a = 0; a < natoms; ++a) {
+      mbar_expect_tx(&m.ldx[a], (uint32_t)(kM * 128));
+      tma_load_2d(tX + a * (kM * 128), &tmx, a * 64, tok0, &m.ldx[a]);
+    }
   }
   for (int j = tid; j < HD; j += kThreads) m.bias[j] = bias ? __ldg(bias + j) : 0.f;
   __syncthreads();
-  bool ok = tc::mbar_wait(&m.ld, 0);
-  tc::tc_after_sync();
   const uint32_t tm = m.tmem;
+  bool ok = true;
 
-  // ---- stage 1: x W_t for every term t at once (TMEM columns 16 t .. 16 t + 15)
+  // ---- stage 1: x W_t for every term t at once (TMEM columns 16 t .. 16 t + 15),
+  // each 64-column atom of x as soon as it has landed
   if (tid == 0) {
     constexpr int kN1 = kTerms * kRank;
     const uint32_t id = idesc16(kM, kN1, 0, 0, kBf16 ? 1 : 0);
-    const int ksteps = dm / 16;
-    for (int s = 0; s < ksteps; ++s) {
-      const uint64_t a = tc::sdesc(saddr(tX) + (s >> 2) * (kM * 128) + (s & 3) * 32, 16, 1024);
-      const uint64_t b = tc::sdesc(saddr(tWd) + (s >> 2) * (kN1 * 128) + (s & 3) * 32, 16, 1024);
-      tc::mma_f16(tm + 0, a, b, id, s > 0 ? 1u : 0u);
+    ok &= tc::mbar_wait(&m.ld, 0);
+    for (int at = 0; at < natoms; ++at) {
+      ok &= tc::mbar_wait(&m.ldx[at], 0);
+      tc::tc_after_sync();
+      for (int s = 4 * at; s < 4 * at + 4; ++s) {
+        const uint64_t a = tc::sdesc(saddr(tX) + (s >> 2) * (kM * 128) + (s & 3) * 32, 16, 1024);
+        const uint64_t b = tc::sdesc(saddr(tWd) + (s >> 2) * (kN1 * 128) + (s & 3) * 32, 16, 1024);
+        tc::mma_f16(tm + 0, a, b, id, s > 0 ? 1u : 0u);
+      }
     }
     tc::mma_commit(&m.mma[0]);
   }
+  // every thread reads the weight scales below: the weights' barrier, then stage 1's
+  ok &= tc::mbar_wait(&m.ld, 0);
   ok &= tc::mbar_wait(&m.mma[0], 0);
   tc::tc_after_sync();
   // low row r (warps 0-3, thread = row) -> per-row scaled two-term fp16 A tile (K = 16)
