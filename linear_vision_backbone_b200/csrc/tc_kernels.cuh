@@ -1023,16 +1023,20 @@ gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
   const int clast = c0 + nch - 1;
   auto stage = [&](int it) -> uint8_t* { return sm + (it & 1) * L::kStage; };
   // step it's k, v (v in the operand layout), g into stage(it)
-  auto fetch = [&](int it) {
+  // (the box loads of k and v may be issued apart from g's: `parts` 1 = k, v;
+  // 2 = g; 3 = all; the barrier expects all three from the first part)
+  auto fetch = [&](int it, int parts = 3) {
     const int s0 = (clast - it) * kC;
     uint8_t* st = stage(it);
     if (tma) {
       if (tid == kThreads) {
         uint64_t* bar = &m.ld[it & 1];
-        mbar_arrive_tx(bar, 2 * kTile + kGTile);
-        tma_box(p, mp, kMapK, st + L::kOffK, bar, d, b, h, s0);
-        tma_box(p, mp, kMapV, st + L::kOffV, bar, d, b, h, s0);
-        tma_box(p, mp, kMapG, st + L::kOffG, bar, d, b, h, s0);
+        if (parts & 1) {
+          mbar_arrive_tx(bar, 2 * kTile + kGTile);
+          tma_box(p, mp, kMapK, st + L::kOffK, bar, d, b, h, s0);
+          tma_box(p, mp, kMapV, st + L::kOffV, bar, d, b, h, s0);
+        }
+        if (parts & 2) tma_box(p, mp, kMapG, st + L::kOffG, bar, d, b, h, s0);
       }
     } else {
       const int ntok = min(kC, p.T - s0);
@@ -1055,9 +1059,18 @@ gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
     if (nch > 1) chunk_rows(p, m.rows[1], b, h, d, (clast - 1) * kC, kC, tid);
   }
   __syncthreads();
-  pdl_wait();                             // g comes from the previous kernel
+  // k and v are inputs: their first boxes go out before the wait; g comes
+  // from the previous kernel
+  if (tma) {
+    fetch(0, 1);
+    if (nch > 1) fetch(1, 1);
+  }
+  pdl_wait();
   pdl_trigger();
-  if (tma || !control) {
+  if (tma) {
+    fetch(0, 2);
+    if (nch > 1) fetch(1, 2);
+  } else if (!control) {
     fetch(0);
     if (nch > 1) fetch(1);
   }
