@@ -288,6 +288,17 @@ def test_strong_decay_reversed_boxes(direction):
         assert exact > 0
 
 
+@pytest.mark.parametrize("B,H,gh,gw", [(4, 80, 8, 8), (2, 160, 16, 16), (1, 320, 64, 2)])
+def test_many_sequences_multi_wave(B, H, gh, gw):
+    # more (image, head) sequences than two per SM: the segment plan goes
+    # multi-wave and the output CTAs' second chains idle wherever a sequence
+    # has an odd number of segments
+    d = inputs.make_custom(B, H, gh, gw, 64, 64, "f16", seed=29, qk_std=0.5)
+    y, ref = _run_custom(d, gh, gw, "BT", 64, torch.float16)
+    assert_close(y, ref, torch.float16, f"{B}x{H} {gh}x{gw}")
+    _check_status()
+
+
 def test_zero_gate_long_memory():
     gh, gw = 64, 64
     d = inputs.make_custom(1, 2, gh, gw, 64, 64, "bf16", seed=71, qk_std=0.125)
