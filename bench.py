@@ -233,7 +233,7 @@ def aggregate_value(units_per_rank: int, steps: int, ms_max: float, world: int) 
 
 
 # ---------------------------------------------------------------- CPU oracle
-def oracle_rate(wl, seconds=3.0, rows=32):
+def oracle_rate(wl, seconds=10.0, rows=32):
     """Token-heads/s of the fp64 oracle (gate + GLA) on a bounded sample: every
     head of the first `rows` grid rows of batch entry 0, repeated for about
     `seconds`.  The oracle runs one (batch, head) sequence per OpenMP thread,
@@ -452,7 +452,7 @@ def run_ours(args, world, rank, local):
         secondary = secondary_line(binding, dev)
 
     if rank == 0:
-        cpu = oracle_rate(wl, seconds=2.0)
+        cpu = oracle_rate(wl, seconds=10.0)
         line = {
             "metric": "GLA fwd token-heads/s (gate projection + Key-only GLA)",
             "value": value, "unit": "token-heads/s", "n_gpus": world, "steps": args.steps,
