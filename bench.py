@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--chunk", type=int, default=64)
     ap.add_argument("--e2e-steps", type=int, default=40)
     ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--fused", action="store_true",
+                    help="time gtr_gla_fwd_gated (gate second half inside the summary kernel)")
     return ap.parse_args()
 
 
@@ -64,14 +66,17 @@ def step_dirs(wl):
     return list(wl.dirs)
 
 
-def alg_bytes(wl, nseg, esz):
-    """Algorithmic bytes per launch of each kernel (unique reads + writes)."""
+def alg_bytes(wl, nseg, esz, fused=False):
+    """Algorithmic bytes per launch of each kernel (unique reads + writes).
+    fused: the gate kernel writes the rank-16 rows x W_down (fp32) and the
+    summary kernel reads them and writes g."""
     th = wl.token_heads
     dk, dv = wl.dk, wl.dv
     st = wl.B * wl.H * nseg * (dk * dv + dk) * 4
+    low = wl.B * wl.T * wl.rank * 4
     return {
-        "gate": wl.B * wl.T * wl.d_model * esz + th * dk * 4,
-        "summary": th * (dk * esz + dv * esz + dk * 4) + st,
+        "gate": wl.B * wl.T * wl.d_model * esz + (low if fused else th * dk * 4),
+        "summary": th * (dk * esz + dv * esz + dk * 4) + st + (low if fused else 0),
         "scan": 2 * st,
         "output": th * (2 * dk * esz + 2 * dv * esz + dk * 4) + th * dv * esz + st,
     }
@@ -324,16 +329,8 @@ def run_ours(args, world, rank, local):
     stream = torch.cuda.Stream(device=dev)
     path = binding.path_for(wl.B, wl.H, wl.gh, wl.gw, wl.dk, wl.dv, args.chunk, host["q"].dtype)
 
-    gate = make_gate(binding, wl, params, host["x"].dtype)
+    step, fused = make_step(binding, wl, params, host["x"].dtype, args.chunk, stream, args.fused)
     torch.cuda.synchronize()
-
-    def step(s, direction, evs=None):
-        if evs is not None:
-            record_external(evs[0], stream)
-        gate(s["x"], s["g"], stream)
-        binding.gla_fwd(s["q"], s["k"], s["v"], s["g"], s["z"], params["w"], grid_h=wl.gh,
-                        grid_w=wl.gw, direction=direction, chunk=args.chunk, out=s["out"],
-                        stream=stream, events=None if evs is None else evs[1:])
 
     # warm the library (workspace allocation happens outside capture)
     with torch.cuda.stream(stream):
@@ -409,12 +406,12 @@ def run_ours(args, world, rank, local):
     # segment plan of this workload (for the state bytes)
     nc = (wl.T + args.chunk - 1) // args.chunk
     nseg = binding.segment_count(wl.B, wl.H, wl.gh, wl.gw, wl.dk, wl.dv, args.chunk, host["q"].dtype)
-    ab = alg_bytes(wl, nseg, esz)
+    ab = alg_bytes(wl, nseg, esz, fused)
     dom = max(per_ms, key=lambda n: per_ms[n])
     peak, peak_kind = read_peak()
     achieved = ab[dom] / (per_ms[dom] * 1e-3) / 1e9
-    kname = {"gate": "gate_fwd_tc", "summary": "gla_sum_tc", "scan": "gla_state_scan",
-             "output": "gla_out_tc"}[dom]
+    kname = {"gate": "gate_low_tc" if fused else "gate_fwd_tc", "summary": "gla_sum_tc",
+             "scan": "gla_state_scan", "output": "gla_out_tc"}[dom]
     traffic, _ = read_traffic(f"{kname}:{path}:{wl.name}", kernel_source_hash())
 
     # e2e: host buffers, copies inside the timed region, through the public API
@@ -462,6 +459,8 @@ def run_ours(args, world, rank, local):
             "dtype": "f32" if path == "simt" else "bf16x2/f32",
             "data": "synthetic",
             "config": {"workload": workload_text(wl), "chunk": args.chunk, "kernel_path": path,
+                       "step_call": ("gtr_gla_fwd_gated" if fused
+                                     else "gtr_gate_fwd_packed + gtr_gla_fwd"),
                        "l2": f"{N_SETS} rotating input sets, inputs larger than L2",
                        "parallelism": f"replicas x{world} (independent (image, head) units)",
                        "timing": "value from plain graph replays; kernels_ms and the roofline "
@@ -488,25 +487,52 @@ def run_ours(args, world, rank, local):
         dist.destroy_process_group()
 
 
-def make_gate(binding, wl, params, x_dtype):
-    """The gate projection of a step.  The weights are static, so for the
-    tensor-core gate they are packed once here (outside any timed region) and
-    every step runs the packed forward; other shapes run gtr_gate_fwd."""
+def make_step(binding, wl, params, x_dtype, chunk, stream, fused=False):
+    """One step of the hot path: the gate projection then the GLA forward.
+    The weights are static, so for the tensor-core gate shapes they are packed
+    once here (outside any timed region) and every step runs
+    gtr_gate_fwd_packed and gtr_gla_fwd, or with `fused` one
+    gtr_gla_fwd_gated call (the gate's second half inside the summary
+    kernel; measured slower on the 16k step); other shapes run gtr_gate_fwd
+    and gtr_gla_fwd.  `evs` (5 events): before the gate, after each of the
+    four kernels.  Returns (step, fused)."""
     rank = params["w_down"].shape[1]
     hd = wl.H * wl.dk
-    if (x_dtype in (torch.float16, torch.bfloat16) and rank == 16 and wl.d_model % 64 == 0
-            and wl.d_model <= 384 and hd % 64 == 0 and hd <= 448):
+    packable = (x_dtype in (torch.float16, torch.bfloat16) and rank == 16 and wl.d_model % 64 == 0
+                and wl.d_model <= 384 and hd % 64 == 0 and hd <= 448)
+    if packable and not fused:
         packed = binding.gate_pack(params["w_down"], params["w_up"], x_dtype, wl.H, wl.dk)
 
-        def gate(x, out, stream):
-            binding.gate_fwd_packed(x, packed, params["bias"], rank, wl.H, wl.dk, wl.tau,
-                                    out=out, stream=stream)
-        return gate
+        def step(s, direction, evs=None):
+            if evs is not None:
+                record_external(evs[0], stream)
+            binding.gate_fwd_packed(s["x"], packed, params["bias"], rank, wl.H, wl.dk, wl.tau,
+                                    out=s["g"], stream=stream)
+            binding.gla_fwd(s["q"], s["k"], s["v"], s["g"], s["z"], params["w"], grid_h=wl.gh,
+                            grid_w=wl.gw, direction=direction, chunk=chunk, out=s["out"],
+                            stream=stream, events=None if evs is None else evs[1:])
+        return step, False
+    if packable:
+        packed = binding.gate_pack(params["w_down"], params["w_up"], x_dtype, wl.H, wl.dk)
 
-    def gate(x, out, stream):
-        binding.gate_fwd(x, params["w_down"], params["w_up"], params["bias"], wl.H, wl.dk,
-                         wl.tau, out=out, stream=stream)
-    return gate
+        def step(s, direction, evs=None):
+            if evs is not None:
+                record_external(evs[0], stream)
+            binding.gla_fwd_gated(s["x"], packed, params["bias"], s["q"], s["k"], s["v"], s["z"],
+                                  params["w"], tau=wl.tau, grid_h=wl.gh, grid_w=wl.gw,
+                                  direction=direction, chunk=chunk, g_out=s["g"], out=s["out"],
+                                  stream=stream, events=None if evs is None else [None] + evs[1:])
+        return step, True
+
+    def step(s, direction, evs=None):
+        if evs is not None:
+            record_external(evs[0], stream)
+        binding.gate_fwd(s["x"], params["w_down"], params["w_up"], params["bias"], wl.H, wl.dk,
+                         wl.tau, out=s["g"], stream=stream)
+        binding.gla_fwd(s["q"], s["k"], s["v"], s["g"], s["z"], params["w"], grid_h=wl.gh,
+                        grid_w=wl.gw, direction=direction, chunk=chunk, out=s["out"],
+                        stream=stream, events=None if evs is None else evs[1:])
+    return step, False
 
 
 def secondary_line(binding, dev, steps=2000):
@@ -521,13 +547,8 @@ def secondary_line(binding, dev, steps=2000):
         sets.append(s)
     params = {n: host[n].to(dev) for n in ("w_down", "w_up", "bias", "w")}
     stream = torch.cuda.Stream(device=dev)
-    gate = make_gate(binding, wl, params, host["x"].dtype)
+    step, _ = make_step(binding, wl, params, host["x"].dtype, 64, stream)
     torch.cuda.synchronize()
-
-    def step(s, direction):
-        gate(s["x"], s["g"], stream)
-        binding.gla_fwd(s["q"], s["k"], s["v"], s["g"], s["z"], params["w"], grid_h=wl.gh,
-                        grid_w=wl.gw, direction=direction, chunk=64, out=s["out"], stream=stream)
 
     with torch.cuda.stream(stream):
         for i, s in enumerate(sets):

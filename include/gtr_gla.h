@@ -199,6 +199,46 @@ GTR_API gtr_status_t gtr_gla_fwd_timed(const void *q, const void *k, const void 
                                int dtype, void *stream, void *const *ev);
 
 /*
+ * Gate projection and GLA forward of one token mixer in one call:
+ *     g_out = logsigmoid(x W_down W_up + bias) / tau        (as gtr_gate_fwd_packed)
+ *     out   = gtr_gla_fwd(q, k, v, g_out, outgate, rms_w)
+ * (GTR article 方法详解 §1, the low-rank key-side gate, and §4).
+ *   x [B, T, d_model] in x_dtype; `packed`: W_down and W_up from gtr_gate_pack
+ *   for this x_dtype, d_model, rank, H, dk (so the shapes gtr_gate_pack takes);
+ *   bias [H*dk] fp32 or NULL; tau > 0.  q, k, v, outgate, rms_w, out, the sizes,
+ *   dir, chunk and dtype as in gtr_gla_fwd; g_out [B, T, H, dk] fp32 receives g
+ *   (the output stage reads it back; it must not alias another argument).
+ *   Where gtr_gla_fwd takes its tensor-core path (dk = dv = 64, chunk 64, 16-bit
+ *   dtype) the gate is split at its rank-16 bottleneck: one kernel writes
+ *   x W_down ([B*T, 16] fp32, 64 bytes per token, in the workspace, which
+ *   therefore grows by B*T*64 bytes), and the summary kernel forms g chunk by
+ *   chunk from it, so the gate costs no pass of its own over g.  g_out and
+ *   out equal those of gtr_gate_fwd_packed followed by gtr_gla_fwd up to
+ *   rounding.  Other shapes run exactly those two calls.
+ *   Errors as gtr_gate_fwd_packed and gtr_gla_fwd; B*T must be below 2^31.
+ */
+GTR_API gtr_status_t gtr_gla_fwd_gated(const void *x, int x_dtype, const void *packed,
+                                       const float *bias, int d_model, int rank, float tau,
+                                       const void *q, const void *k, const void *v,
+                                       const void *outgate, const float *rms_w, float *g_out,
+                                       void *out, int B, int H, int grid_h, int grid_w, int dk,
+                                       int dv, int dir, int chunk, int dtype, void *stream);
+
+/*
+ * gtr_gla_fwd_gated that also records caller-created cudaEvent_t handles (any
+ * may be NULL) on `stream`: ev[0] before the gate kernel, ev[1] after it, ev[2]
+ * after the summary kernel, ev[3] after the state scan, ev[4] after the output
+ * kernel.  For profiling only.
+ */
+GTR_API gtr_status_t gtr_gla_fwd_gated_timed(const void *x, int x_dtype, const void *packed,
+                                             const float *bias, int d_model, int rank, float tau,
+                                             const void *q, const void *k, const void *v,
+                                             const void *outgate, const float *rms_w,
+                                             float *g_out, void *out, int B, int H, int grid_h,
+                                             int grid_w, int dk, int dv, int dir, int chunk,
+                                             int dtype, void *stream, void *const *ev);
+
+/*
  * Chunk-boundary states, for testing the first two stages on their own: the
  * state each chunk of `chunk` scan positions ends with,
  *   states [B, H, ceil(T/chunk), dk, dv] fp32, entry c = S after scan position

@@ -27,7 +27,7 @@ EXPORTS = (
     "gtr_gla_chunk_states", "gtr_gla_workspace_bytes", "gtr_gla_set_workspace",
     "gtr_gla_set_path", "gtr_gla_path_for", "gtr_last_device_status", "gtr_gla_segment_chunks",
     "gtr_gla_fwd_noalloc", "gtr_gate_packed_bytes", "gtr_gate_pack", "gtr_gate_fwd_packed",
-    "gtr_gla_segment_count",
+    "gtr_gla_segment_count", "gtr_gla_fwd_gated", "gtr_gla_fwd_gated_timed",
 )
 
 _lock = threading.Lock()
@@ -70,6 +70,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
             "gtr_gate_packed_bytes": ([], Z),
             "gtr_gate_pack": ([P, P, I, I, I, I, I, P, Z, P], I),
             "gtr_gate_fwd_packed": ([P, I, P, P, P, I, I, I, I, I, I, F, P], I),
+            "gtr_gla_fwd_gated": ([P, I, P, P, I, I, F, P, P, P, P, P, P, P,
+                                   I, I, I, I, I, I, I, I, I, P], I),
+            "gtr_gla_fwd_gated_timed": ([P, I, P, P, I, I, F, P, P, P, P, P, P, P,
+                                         I, I, I, I, I, I, I, I, I, P, P], I),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -201,6 +205,43 @@ def gla_fwd(q, k, v, g, z, w=None, *, grid_h: int, grid_w: int, direction: str =
         arr = (ctypes.c_void_p * 4)(*[None if e is None else e.cuda_event for e in events])
         _check("gtr_gla_fwd_timed", lib.gtr_gla_fwd_timed(*args, arr))
     return out
+
+
+def gla_fwd_gated(x, packed, bias, q, k, v, z, w=None, *, tau: float, grid_h: int, grid_w: int,
+                  direction: str = "LR", chunk: int = 64, rank: int = 16,
+                  g_out: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                  stream=None, events: Optional[Sequence] = None):
+    """Gate projection and GLA forward in one call (``gtr_gla_fwd_gated``).
+
+    x: [B, T, d_model] 16-bit; packed: ``gate_pack(w_down, w_up, x.dtype, H, dk)``;
+    bias: [H*dk] fp32 or None; q, k, v, z, w as in :func:`gla_fwd`.  Returns
+    (out, g_out) with g_out = logsigmoid(x W_down W_up + bias)/tau [B, T, H, dk]
+    fp32.  ``events`` (5 torch.cuda.Event or None) are recorded before the gate
+    and after each of its four kernels (``gtr_gla_fwd_gated_timed``).
+    """
+    _need(x, "x")
+    if x.dim() != 3:
+        raise ValueError("x must be [B, T, d_model]")
+    if packed.dtype != torch.uint8 or packed.device != x.device:
+        raise ValueError("packed must be a uint8 tensor on x's device")
+    B, T, H, dk = q.shape
+    if g_out is None:
+        g_out = torch.empty(B, T, H, dk, device=q.device, dtype=torch.float32)
+    B, T, H, dk, dv, out = _gla_check(q, k, v, g_out, z, w, out, grid_h, grid_w)
+    if tuple(x.shape[:2]) != (B, T):
+        raise ValueError(f"x must be [B={B}, T={T}, d_model], got {tuple(x.shape)}")
+    if bias is not None:
+        _need(bias, "bias", torch.float32, (H * dk,))
+    lib = load()
+    args = (_ptr(x), DTYPE_IDS[x.dtype], _ptr(packed), _ptr(bias), x.shape[2], int(rank), float(tau),
+            _ptr(q), _ptr(k), _ptr(v), _ptr(z), _ptr(w), _ptr(g_out), _ptr(out), B, H, grid_h, grid_w,
+            dk, dv, DIR_IDS[direction], int(chunk), DTYPE_IDS[q.dtype], _stream(stream))
+    if events is None:
+        _check("gtr_gla_fwd_gated", lib.gtr_gla_fwd_gated(*args))
+    else:
+        arr = (ctypes.c_void_p * 5)(*[None if e is None else e.cuda_event for e in events])
+        _check("gtr_gla_fwd_gated_timed", lib.gtr_gla_fwd_gated_timed(*args, arr))
+    return out, g_out
 
 
 def gla_fwd_noalloc(q, k, v, g, z, w=None, *, grid_h: int, grid_w: int, direction: str = "LR",

@@ -41,25 +41,14 @@ namespace gate_tc {
 
 using tc::saddr;
 
-// Power-of-two operand scales: 2^e puts the magnitude m into [2^14, 2^15),
-// inside fp16's range; exact, and undone on the fp32 accumulator.
-__device__ __forceinline__ int scale_exp(float m) {
-  if (!(m > 0.f) || !(m <= 3.0e38f)) return 0;
-  const int ex = ((__float_as_int(m) >> 23) & 0xFF) - 127;
-  return max(-60, min(60, 14 - ex));
-}
-__device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }
-// logsigmoid(u) / tau = (min(u, 0) - ln(1 + e^{-|u|})) / tau, the exponential
-// and the logarithm (as log2, scaled by ln2_tau = ln 2 / tau) by the hardware
-// approximations.  1 + e^{-|u|} is formed in fp32, so the log term carries an
-// absolute error below 1e-7 (it rounds to zero once e^{-|u|} is under fp32's
-// resolution at one); both terms are <= 0, so the result is too.
-__device__ __forceinline__ float logsigmoid_over_tau(float u, float inv_tau, float ln2_tau) {
-  const float e = tc::ex2(-fabsf(u) * 1.4426950408889634f);
-  float l;
-  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(l) : "f"(1.0f + e));
-  return fmaf(-l, ln2_tau, fminf(u, 0.0f) * inv_tau);
-}
+using tc::logsigmoid_over_tau;
+using tc::pow2i;
+using tc::scale_exp;
+using tc::bulk_g2s;
+using tc::bulk_commit;
+using tc::bulk_wait;
+using tc::bulk_wait_read;
+
 // Two-term fp16 operand: x = hi + lo, hi = fp16(x), lo = fp16(x - hi); four
 // consecutive elements at byte offset `off` of the (hi, lo) tiles.
 __device__ __forceinline__ void put2(uint8_t* hi, uint8_t* lo, uint32_t off, float a, float b, float c,
@@ -103,27 +92,10 @@ __device__ __forceinline__ void tma_store_2d(const void* map, int x, int y, cons
                "r"(x), "r"(y), "r"(saddr(src))
                : "memory");
 }
-// Untiled bulk copy global -> shared (16-byte aligned, size a multiple of 16).
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          saddr(dst)),
-      "l"(src), "r"(bytes), "r"(saddr(bar))
-      : "memory");
-}
 __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(bar)), "r"(bytes)
                : "memory");
 }
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// wait until at most N committed bulk stores still read shared memory / are in flight
-template <int N> __device__ __forceinline__ void bulk_wait_read() {
-  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
-template <int N> __device__ __forceinline__ void bulk_wait() {
-  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
-}
-
 constexpr int kM = 128;               // rows of the MMA tile (tokens per CTA <= kM)
 constexpr int kThreads = 512;
 constexpr int kPackThreads = 256;
@@ -481,6 +453,108 @@ gate_fwd_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUt
   __syncthreads();
   tc::tc_after_sync();
   if (warp == 0) tc::tmem_dealloc(tm, 512);
+}
+
+// --------------------------------------------------- rank-16 rows only
+// The gate's first half for a summary stage that forms g itself: low = x
+// W_down [N, 16] fp32 (the stage-1 product of gate_fwd_tc, its terms summed
+// and the rank scales undone), one tile of up to 128 tokens per CTA.  One
+// thread per token row writes its 64 bytes.
+constexpr int kLowThreads = 128;
+struct LowLayout {
+  static constexpr int kOffX = 0;
+  static constexpr int kOffWd = kOffX + Layout::kX;
+  static constexpr int kOffMisc = kOffWd + 3 * Layout::kWd;
+  static constexpr int kSmem = kOffMisc + (int)sizeof(Misc) + 1024;
+};
+static_assert(LowLayout::kOffWd % 1024 == 0, "operand tiles must be 1024-byte aligned");
+
+template <typename TX>
+__global__ void __launch_bounds__(kLowThreads, 1)
+gate_low_tc(const __grid_constant__ CUtensorMap tmx, const uint8_t* __restrict__ pack, int dm,
+            float* __restrict__ low, long long N, int tpc) {
+  constexpr bool kBf16 = std::is_same<TX, __nv_bfloat16>::value;
+  constexpr int kTerms = kBf16 ? 3 : 2;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* tX = sm + LowLayout::kOffX;
+  uint8_t* tWd = sm + LowLayout::kOffWd;
+  Misc& m = *reinterpret_cast<Misc*>(sm + LowLayout::kOffMisc);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long tok0 = (long long)blockIdx.x * tpc;
+
+  if (tid == 0) {
+    tc::mbar_init(&m.ld, 1);
+    for (int a = 0; a < kMaxDm / 64; ++a) tc::mbar_init(&m.ldx[a], 1);
+    tc::mbar_init(&m.mma[0], 1);
+    tc::mbar_fence_init();
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(&m.tmem, 64);
+    tc::tmem_relinquish();
+  }
+  tc::tc_before_sync();
+  __syncthreads();
+  tc::tc_after_sync();
+  pdl_wait();                                     // x and the packed weights may come from the previous kernel
+  pdl_trigger();
+  const int natoms = dm / 64;
+  if (tid == 0) {
+    mbar_expect_tx(&m.ld, (uint32_t)(kTerms * Layout::kWd + kRank * 4));
+    bulk_g2s(tWd, pack + Pack::kOffWd, kTerms * Layout::kWd, &m.ld);   // the terms' rows side by side
+    bulk_g2s(&m.wd_i[0], pack + Pack::kOffScale, kRank * 4, &m.ld);
+    for (int a = 0; a < natoms; ++a) {
+      mbar_expect_tx(&m.ldx[a], (uint32_t)(kM * 128));
+      tma_load_2d(tX + a * (kM * 128), &tmx, a * 64, (int)tok0, &m.ldx[a]);
+    }
+  }
+  __syncthreads();
+  const uint32_t tm = m.tmem;
+  bool ok = true;
+  if (tid == 0) {
+    constexpr int kN1 = kTerms * kRank;
+    const uint32_t id = idesc16(kM, kN1, 0, 0, kBf16 ? 1 : 0);
+    ok &= tc::mbar_wait(&m.ld, 0);
+    for (int at = 0; at < natoms; ++at) {
+      ok &= tc::mbar_wait(&m.ldx[at], 0);
+      tc::tc_after_sync();
+      for (int s = 4 * at; s < 4 * at + 4; ++s) {
+        const uint64_t a = tc::sdesc(saddr(tX) + (s >> 2) * (kM * 128) + (s & 3) * 32, 16, 1024);
+        const uint64_t b = tc::sdesc(saddr(tWd) + (s >> 2) * (kN1 * 128) + (s & 3) * 32, 16, 1024);
+        tc::mma_f16(tm + 0, a, b, id, s > 0 ? 1u : 0u);
+      }
+    }
+    tc::mma_commit(&m.mma[0]);
+  }
+  ok &= tc::mbar_wait(&m.ld, 0);
+  ok &= tc::mbar_wait(&m.mma[0], 0);
+  tc::tc_after_sync();
+  {
+    float lw[16], lt[16];
+    tmem_ld16(tm + ((uint32_t)(warp * 32) << 16) + 0, lw);
+    tc::tmem_ld_wait(lw);
+#pragma unroll
+    for (int t = 1; t < kTerms; ++t) {
+      tmem_ld16(tm + ((uint32_t)(warp * 32) << 16) + t * kRank, lt);
+      tc::tmem_ld_wait(lt);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) lw[c] += lt[c];
+    }
+    const int r = warp * 32 + lane;
+    if (ok && r < tpc && tok0 + r < N) {
+      float4* dst = reinterpret_cast<float4*>(low + (tok0 + r) * kRank);
+#pragma unroll
+      for (int c = 0; c < 16; c += 4)
+        dst[c / 4] = make_float4(lw[c] * m.wd_i[c], lw[c + 1] * m.wd_i[c + 1], lw[c + 2] * m.wd_i[c + 2],
+                                 lw[c + 3] * m.wd_i[c + 3]);
+    }
+  }
+  ok = __syncthreads_and(ok) != 0;
+  if (!ok && tid == 0) gtr_flag(kStatusMbarTimeout);
+  tc::tc_before_sync();
+  __syncthreads();
+  tc::tc_after_sync();
+  if (warp == 0) tc::tmem_dealloc(tm, 64);
 }
 
 }  // namespace gate_tc

@@ -245,28 +245,30 @@ int tmap_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, unsigned
 }
 
 // Tensor map of a [B, T, H, D] row-major tensor (element size es bytes,
-// D = 64) for box loads of one chunk of one head: orientation 0 views it as
-// (D, H, T, B), box (64, 1, 64, 1); orientation 1 as (D, H, gw, gh, B), box
-// (64, 1, 1, 64, 1), a run of 64 grid rows in one column.
+// D = 64, or D = 16 with H = 1 for the rank-16 gate rows) for box loads of one
+// chunk of one head: orientation 0 views it as (D, H, T, B), box (D, 1, 64,
+// 1); orientation 1 as (D, H, gw, gh, B), box (D, 1, 1, 64, 1), a run of 64
+// grid rows in one column.
 int tmap_chunk(CUtensorMap* map, CUtensorMapDataType dt, int es, const void* base, const Plan& p, int orient,
-               bool swizzle) {
+               bool swizzle, int D_ = 64, int H_ = -1, int box_inner = 0) {
   EncodeTiledFn enc = encode_tiled();
   if (!enc) return GTR_ERR_CUDA;
-  const cuuint64_t D = 64, es_ = (cuuint64_t)es;
-  const cuuint64_t tok = (cuuint64_t)p.H * D * es_;   // bytes per token
+  const cuuint64_t D = (cuuint64_t)D_, es_ = (cuuint64_t)es;
+  const cuuint64_t H = (cuuint64_t)(H_ < 0 ? p.H : H_);
+  const cuuint64_t tok = H * D * es_;   // bytes per token
   CUresult r;
   if (orient == 0) {
-    const cuuint64_t dims[4] = {D, (cuuint64_t)p.H, (cuuint64_t)p.T, (cuuint64_t)p.B};
+    const cuuint64_t dims[4] = {D, H, (cuuint64_t)p.T, (cuuint64_t)p.B};
     const cuuint64_t strides[3] = {D * es_, tok, tok * (cuuint64_t)p.T};
-    const cuuint32_t box[4] = {64, 1, 64, 1};
+    const cuuint32_t box[4] = {(cuuint32_t)(box_inner ? box_inner : D_), 1, 64, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     r = enc(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
             swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   } else {
-    const cuuint64_t dims[5] = {D, (cuuint64_t)p.H, (cuuint64_t)p.gw, (cuuint64_t)p.gh, (cuuint64_t)p.B};
+    const cuuint64_t dims[5] = {D, H, (cuuint64_t)p.gw, (cuuint64_t)p.gh, (cuuint64_t)p.B};
     const cuuint64_t strides[4] = {D * es_, tok, tok * (cuuint64_t)p.gw, tok * (cuuint64_t)p.T};
-    const cuuint32_t box[5] = {64, 1, 1, 64, 1};
+    const cuuint32_t box[5] = {(cuuint32_t)(box_inner ? box_inner : D_), 1, 1, 64, 1};
     const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
     r = enc(map, dt, 5, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
             swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
@@ -278,8 +280,12 @@ int tmap_chunk(CUtensorMap* map, CUtensorMapDataType dt, int es, const void* bas
 // every chunk of one head is one box: 16-byte aligned bases, and for the
 // column orders (TB, BT) 64 | gh so that no chunk crosses a grid column.
 // Returns false to gather with cp.async.
-bool chunk_maps(const Plan& p, const void* q, const void* k, const void* v, const float* g, tc::Maps* maps) {
-  for (const void* a : {q, k, v, (const void*)g})
+// With `low` (the gate's rank-16 rows) the g map is replaced by low's map and
+// g may be null; `g_store` adds the store map of the g the summary kernel
+// writes (32-column boxes, SWIZZLE_128B).
+bool chunk_maps(const Plan& p, const void* q, const void* k, const void* v, const float* g, tc::Maps* maps,
+                const float* low = nullptr, const float* g_store = nullptr) {
+  for (const void* a : {q, k, v, (const void*)g, (const void*)low, (const void*)g_store})
     if (((uintptr_t)a & 15) != 0) return false;
   bool orient[2] = {false, false};
   for (int b = 0; b < (p.dir == kRotate ? (p.B < 4 ? p.B : 4) : 1); ++b) {
@@ -295,7 +301,11 @@ bool chunk_maps(const Plan& p, const void* q, const void* k, const void* v, cons
     if ((q && tmap_chunk(&maps->t[o][tc::kMapQ], dt, 2, q, p, o, false)) ||
         tmap_chunk(&maps->t[o][tc::kMapK], dt, 2, k, p, o, false) ||
         tmap_chunk(&maps->t[o][tc::kMapV], dt, 2, v, p, o, true) ||
-        tmap_chunk(&maps->t[o][tc::kMapG], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, g, p, o, false))
+        (g && tmap_chunk(&maps->t[o][tc::kMapG], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, g, p, o, false)) ||
+        (low && tmap_chunk(&maps->t[o][tc::kMapL], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, low, p, o, false,
+                           tc::kLowRank, 1)) ||
+        (g_store && tmap_chunk(&maps->t[o][tc::kMapGS], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, g_store, p, o, true,
+                               64, -1, 32)))
       return false;
   }
   return true;
@@ -343,6 +353,31 @@ int gate_fwd_packed_launch(int x_dtype, const void* x, const void* pack, const f
   if (int rc = ensure_smem(gate_tc::gate_fwd_tc<__nv_bfloat16>, gate_tc::Layout::kSmem, done_b, dev)) return rc;
   return launch_pdl(gate_tc::gate_fwd_tc<__nv_bfloat16>, dim3((unsigned)blocks), dim3(gate_tc::kThreads),
                     gate_tc::Layout::kSmem, st, tmx, tmg, (const uint8_t*)pack, bias, dm, HD, inv_tau, tpc)
+             ? GTR_ERR_CUDA
+             : GTR_OK;
+}
+// The gate's rank-16 rows low = x W_down [N, 16] fp32 (packed weights).
+int gate_low_launch(int x_dtype, const void* x, const void* pack, float* low, long long N, int dm,
+                    cudaStream_t st, int dev) {
+  const int tpc = gate_tc_tile(N, sm_count(dev));
+  const long long blocks = (N + tpc - 1) / tpc;
+  CUtensorMap tmx;
+  const CUtensorMapDataType xdt =
+      x_dtype == GTR_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (int rc = tmap_2d(&tmx, xdt, x, (unsigned long long)N, (unsigned long long)dm,
+                       (unsigned long long)dm * 2, 64, gate_tc::kM))
+    return rc;
+  static bool done_h[kMaxDevices], done_b[kMaxDevices];
+  if (x_dtype == GTR_F16) {
+    if (int rc = ensure_smem(gate_tc::gate_low_tc<__half>, gate_tc::LowLayout::kSmem, done_h, dev)) return rc;
+    return launch_pdl(gate_tc::gate_low_tc<__half>, dim3((unsigned)blocks), dim3(gate_tc::kLowThreads),
+                      gate_tc::LowLayout::kSmem, st, tmx, (const uint8_t*)pack, dm, low, N, tpc)
+               ? GTR_ERR_CUDA
+               : GTR_OK;
+  }
+  if (int rc = ensure_smem(gate_tc::gate_low_tc<__nv_bfloat16>, gate_tc::LowLayout::kSmem, done_b, dev)) return rc;
+  return launch_pdl(gate_tc::gate_low_tc<__nv_bfloat16>, dim3((unsigned)blocks), dim3(gate_tc::kLowThreads),
+                    gate_tc::LowLayout::kSmem, st, tmx, (const uint8_t*)pack, dm, low, N, tpc)
              ? GTR_ERR_CUDA
              : GTR_OK;
 }
@@ -469,6 +504,66 @@ int gla_fwd_impl(const void* q, const void* k, const void* v, const float* g, co
   if ((rc = record(ev, 2, st))) return rc;
   if ((rc = launch_stage(p, q, k, v, g, z, w, out, wsS, wsA, st, 1))) return rc;
   return record(ev, 3, st);
+}
+
+// Gate projection + GLA forward (gtr_gla_fwd_gated).  On the tensor-core path
+// the gate is split at its rank-16 bottleneck: a short kernel writes low = x
+// W_down ([N, 16] fp32, in the workspace), and the summary kernel forms g =
+// logsigmoid(low W_up + b)/tau per chunk as it needs it, writing g_out for the
+// output kernel; no separate pass over g runs.  Otherwise the gate kernel and
+// gtr_gla_fwd run one after the other.  Events (profiling): ev[0] before the
+// gate, ev[1] after it, ev[2] after the summary, ev[3] after the scan, ev[4]
+// after the output kernel.
+int gla_fwd_gated_impl(const void* x, int x_dtype, const void* packed, const float* bias, int d_model,
+                       int rank, float tau, const void* q, const void* k, const void* v, const void* z,
+                       const float* w, float* g_out, void* out, int B, int H, int gh, int gw, int dk, int dv,
+                       int dir, int chunk, int dtype, void* stream, void* const* ev) {
+  int rc = check_gla_args(B, H, gh, gw, dk, dv, dir, chunk, dtype);
+  if (rc) return rc;
+  if (x_dtype < 0 || x_dtype > 2 || d_model <= 0 || rank <= 0) return GTR_ERR_INVALID_ARG;
+  if (!(tau > 0.0f) || !(tau < 3.0e38f)) return GTR_ERR_INVALID_ARG;
+  const long long HD = (long long)H * dk;
+  if (HD > 4096 || !gate_tc_supported(x_dtype, d_model, rank, (int)HD)) return GTR_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0 || gh == 0 || gw == 0) return GTR_OK;
+  const long long N = (long long)B * gh * gw;
+  if (N >= (1LL << 31)) return GTR_ERR_UNSUPPORTED;
+  if (!x || !packed || !q || !k || !v || !z || !g_out || !out) return GTR_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(packed) || (bias && !aligned16(bias)) || !aligned16(q) || !aligned16(k) ||
+      !aligned16(v) || !aligned16(z) || !aligned16(g_out) || !aligned16(out) || (w && !aligned16(w)))
+    return GTR_ERR_ALIGNMENT;
+  int dev;
+  if ((rc = current_device(&dev))) return rc;
+  Plan p;
+  if ((rc = make_plan(&p, dev, B, H, gh, gw, dk, dv, dir, chunk, dtype, 0))) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  if ((rc = record(ev, 0, st))) return rc;
+  if (p.path != GTR_PATH_TC) {
+    if ((rc = gate_fwd_packed_launch(x_dtype, x, packed, bias, g_out, N, d_model, (int)HD, tau, st, dev)))
+      return rc;
+    if ((rc = record(ev, 1, st))) return rc;
+    void* ev4[4] = {nullptr, ev ? ev[2] : nullptr, ev ? ev[3] : nullptr, ev ? ev[4] : nullptr};
+    return gla_fwd_impl(q, k, v, g_out, z, w, out, B, H, gh, gw, dk, dv, dir, chunk, dtype, stream, ev4);
+  }
+  const size_t offL = (p.ws_bytes + 255) & ~(size_t)255;
+  void* ws = nullptr;
+  if ((rc = get_workspace(dev, stream, offL + (size_t)N * tc::kLowRank * sizeof(float), &ws))) return rc;
+  float* wsS = (float*)ws;
+  float* wsA = (float*)((char*)ws + p.offA);
+  float* low = (float*)((char*)ws + offL);
+  if ((rc = gate_low_launch(x_dtype, x, packed, low, N, d_model, st, dev))) return rc;
+  if ((rc = record(ev, 1, st))) return rc;
+  tc::Maps maps;
+  const bool boxes = chunk_maps(p, nullptr, k, v, nullptr, &maps, low, g_out);
+  const uint8_t* pk = (const uint8_t*)packed;
+  if (launch_tc_gated_sum(p.dtype, k, v, low, pk + gate_tc::Pack::kOffWu, gate_tc::Layout::kWu,
+                          (const float*)(pk + gate_tc::Pack::kOffScale) + gate_tc::kRank, bias, 1.0f / tau,
+                          g_out, wsS, wsA, B, H, p.T, gh, gw, dir, p.nseg, boxes ? &maps : nullptr, st))
+    return GTR_ERR_CUDA;
+  if ((rc = record(ev, 2, st))) return rc;
+  if ((rc = launch_scan(p, wsS, wsA, 0, st))) return rc;
+  if ((rc = record(ev, 3, st))) return rc;
+  if ((rc = launch_stage(p, q, k, v, g_out, z, w, out, wsS, wsA, st, 1))) return rc;
+  return record(ev, 4, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -689,6 +784,26 @@ gtr_status_t gtr_gla_fwd_timed(const void* q, const void* k, const void* v, cons
                                int dtype, void* stream, void* const* ev) {
   return (gtr_status_t)gla_fwd_impl(q, k, v, g, outgate, rms_w, out, B, H, grid_h, grid_w, dk, dv,
                                     dir, chunk, dtype, stream, ev);
+}
+
+gtr_status_t gtr_gla_fwd_gated(const void* x, int x_dtype, const void* packed, const float* bias,
+                               int d_model, int rank, float tau, const void* q, const void* k,
+                               const void* v, const void* outgate, const float* rms_w, float* g_out,
+                               void* out, int B, int H, int grid_h, int grid_w, int dk, int dv, int dir,
+                               int chunk, int dtype, void* stream) {
+  return (gtr_status_t)gla_fwd_gated_impl(x, x_dtype, packed, bias, d_model, rank, tau, q, k, v, outgate,
+                                          rms_w, g_out, out, B, H, grid_h, grid_w, dk, dv, dir, chunk,
+                                          dtype, stream, nullptr);
+}
+
+gtr_status_t gtr_gla_fwd_gated_timed(const void* x, int x_dtype, const void* packed, const float* bias,
+                                     int d_model, int rank, float tau, const void* q, const void* k,
+                                     const void* v, const void* outgate, const float* rms_w, float* g_out,
+                                     void* out, int B, int H, int grid_h, int grid_w, int dk, int dv,
+                                     int dir, int chunk, int dtype, void* stream, void* const* ev) {
+  return (gtr_status_t)gla_fwd_gated_impl(x, x_dtype, packed, bias, d_model, rank, tau, q, k, v, outgate,
+                                          rms_w, g_out, out, B, H, grid_h, grid_w, dk, dv, dir, chunk,
+                                          dtype, stream, ev);
 }
 
 gtr_status_t gtr_gla_chunk_states(const void* k, const void* v, const float* g, float* states,

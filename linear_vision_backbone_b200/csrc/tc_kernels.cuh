@@ -151,6 +151,30 @@ __device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, i
       "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(saddr(bar))
       : "memory");
 }
+// Tiled tensor-map stores shared -> global (bulk-group completion).  The
+// innermost coordinate must be 16-byte aligned and no coordinate negative.
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void* src, int c0, int c1, int c2,
+                                             int c3) {
+  asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3, %4}], [%5];" ::"l"(
+                   map),
+               "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(saddr(src))
+               : "memory");
+}
+__device__ __forceinline__ void tma_store_5d(const CUtensorMap* map, const void* src, int c0, int c1, int c2,
+                                             int c3, int c4) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3, %4, %5}], [%6];" ::"l"(map),
+      "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(saddr(src))
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until at most N committed bulk stores still read shared memory / are in flight
+template <int N> __device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+template <int N> __device__ __forceinline__ void bulk_wait() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
 // 16-byte asynchronous global -> shared copy (L2 only), grouped by commit.
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(saddr(dst)), "l"(src) : "memory");
@@ -246,6 +270,44 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Power-of-two operand scales: 2^e puts the magnitude m into [2^14, 2^15),
+// inside fp16's range; exact, and undone on the fp32 accumulator.
+__device__ __forceinline__ int scale_exp(float m) {
+  if (!(m > 0.f) || !(m <= 3.0e38f)) return 0;
+  const int ex = ((__float_as_int(m) >> 23) & 0xFF) - 127;
+  return max(-60, min(60, 14 - ex));
+}
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }
+// logsigmoid(u) / tau = (min(u, 0) - ln(1 + e^{-|u|})) / tau, the exponential
+// and the logarithm (as log2, scaled by ln2_tau = ln 2 / tau) by the hardware
+// approximations.  1 + e^{-|u|} is formed in fp32, so the log term carries an
+// absolute error below 1e-7 (it rounds to zero once e^{-|u|} is under fp32's
+// resolution at one); both terms are <= 0, so the result is too.
+__device__ __forceinline__ float logsigmoid_over_tau(float u, float inv_tau, float ln2_tau) {
+  const float e = ex2(-fabsf(u) * 1.4426950408889634f);
+  float l;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(l) : "f"(1.0f + e));
+  return fmaf(-l, ln2_tau, fminf(u, 0.0f) * inv_tau);
+}
+// Two-term fp16 value pairs: x = hi + lo, hi = fp16(x), lo = fp16(x - hi),
+// two consecutive elements per 32-bit word.
+__device__ __forceinline__ void split2h(float a, float b, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(a, b);
+  const float2 f = __half22float2(h);
+  const __half2 l = __floats2half2_rn(a - f.x, b - f.y);
+  memcpy(&hi, &h, 4);
+  memcpy(&lo, &l, 4);
+}
+// Untiled bulk copy global -> shared (16-byte aligned, size a multiple of 16),
+// completing on `bar` (which must expect the bytes).
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          saddr(dst)),
+      "l"(src), "r"(bytes), "r"(saddr(bar))
+      : "memory");
+}
+
 // ------------------------------------------------------- operand layouts
 // 16-bit operand tiles of 64 rows x 64 elements (128 bytes per row), layout
 // SWIZZLE_128B: atoms of 8 rows x 128 bytes, the 16-byte unit index XOR-ed
@@ -272,6 +334,11 @@ constexpr uint32_t kStepK = 32 >> 4, kStepMN = 2048 >> 4;   // descriptor addres
 __host__ __device__ constexpr uint32_t idesc_bf16(int a_mn, int b_mn, int n = 64) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
          ((uint32_t)(n >> 3) << 17) | ((uint32_t)(64 >> 4) << 24);
+}
+// The same with fp16 A and B.
+__host__ __device__ constexpr uint32_t idesc_f16(int a_mn, int b_mn, int n = 64) {
+  return (1u << 4) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) | ((uint32_t)(n >> 3) << 17) |
+         ((uint32_t)(64 >> 4) << 24);
 }
 // One tcgen05.mma kind::f16 instruction; the instruction descriptor selects
 // fp16 or bf16 operands.
@@ -419,6 +486,14 @@ struct Params {
   float* wsS; float* wsA; void* out;
   int H, T, gh, gw, dir, nseg;
   int tma;                        // 1: chunks arrive by tensor-map loads (Maps valid)
+  // Summary stage with the gate's second half in-kernel (gla_sum_tc<T, true>):
+  // the rank-16 rows low = x W_down [B, T, 16] fp32, the packed W_up terms
+  // (two fp16 tiles of 16 x H*dk, MN-major, `wu_term` bytes apart, head h's
+  // 64 columns a 2 KB block at 2048 h), their inverse column scales, the bias
+  // (or null) and 1/tau; the kernel writes g to `g_out`.
+  const float* low; const uint8_t* wu; const float* wu_scale; const float* gbias; float* g_out;
+  int wu_term;
+  float inv_tau;
 };
 // Tensor maps of q, k, v, g ([B, T, H, D] row-major) for box loads of one
 // chunk of one head: [0] the token order, dims (D, H, T, B), box (64, 1, 64,
@@ -426,9 +501,12 @@ struct Params {
 // (valid when 64 divides gh).  A reversed scan loads the same box and walks
 // it backwards.  q, k, g are plain row-major boxes; v lands in the
 // SWIZZLE_128B operand layout.
-enum { kMapQ = 0, kMapK = 1, kMapV = 2, kMapG = 3 };
+// [.][kMapL]: the rank-16 rows low [B, T, 16] fp32 as dims (16, 1, T, B) /
+// (16, 1, gw, gh, B), box 16 x 64 tokens (head coordinate 0).  [.][kMapGS]:
+// g_out for stores, box 32 x 64 (one 128-byte half of each row), SWIZZLE_128B.
+enum { kMapQ = 0, kMapK = 1, kMapV = 2, kMapG = 3, kMapL = 4, kMapGS = 5 };
 struct Maps {
-  CUtensorMap t[2][4];
+  CUtensorMap t[2][6];
 };
 
 // ------------------------------------------------------------- fetching
@@ -448,6 +526,19 @@ __device__ __forceinline__ void tma_box(const Params& p, const Maps& mp, int whi
   } else {
     const int col = t0 / p.gh, r0 = t0 - col * p.gh;   // whole chunks: t0 >= 0, r0 + 64 <= gh
     tma_load_5d(dst, &mp.t[1][which], 0, h, col, r0, b, bar);
+  }
+}
+// Store counterpart of tma_box (box rows in the same order), at column x of
+// the rows; not for a reversed scan's ragged chunk (its box starts before
+// token 0, and a store may not start at a negative coordinate).
+__device__ __forceinline__ void tma_store_box(const Params& p, const Maps& mp, int which, const void* src, int d,
+                                              int b, int h, int s0, int x) {
+  const int t0 = dir_reversed(d) ? p.T - s0 - kC : s0;
+  if (!dir_orient(d)) {
+    tma_store_4d(&mp.t[0][which], src, x, h, t0, b);
+  } else {
+    const int col = t0 / p.gh, r0 = t0 - col * p.gh;
+    tma_store_5d(&mp.t[1][which], src, x, h, col, r0, b);
   }
 }
 __device__ __forceinline__ void tma_chunk(const Params& p, const Maps& mp, uint8_t* kdst, uint8_t* qdst,
@@ -960,35 +1051,79 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
 }
 
 // ===================================================================== K2
+constexpr int kLowRank = 16;                   // rank of the gate projection
+constexpr int kLowTile = kC * kLowRank * 4;    // a chunk's fp32 rank-16 rows: 4 KB
 struct SumMisc {
   uint64_t mma;
   uint64_t ld[2];                 // box loads into staging buffer 0 / 1
+  uint64_t umma;                  // gate: the chunk's u = low W_up product
+  uint64_t wl;                    // gate: W_up tiles, column scales, bias
+  uint64_t gready;                // gate: the chunk's g tile is staged (one arrival per builder warp)
   uint32_t tmem;
   int waited, fetched, issued;    // steps whose loads were consumed / issued, products issued
   alignas(16) float part[kWarps][kD];   // cumsum partials: tokens 8 w .. 8 w + 7, per dim
   alignas(16) long long rows[2][kC];    // token rows (cp.async gathers only)
+  alignas(16) float ri[kC];       // gate: inverse row scales of the staged low rows
+  alignas(16) float ci[kD];       // gate: inverse W_up column scales of this head
+  alignas(16) float gb[kD];       // gate: bias of this head
 };
-struct SumLayout {
-  // two staging buffers of k (8 KB, row-major), v (8 KB, operand layout), gate (16 KB)
+template <bool kGate>
+struct SumLayoutT {
+  // two staging buffers of k (8 KB, row-major), v (8 KB, operand layout) and
+  // the gate: g (16 KB, fp32 rows) or, with the gate in-kernel, the rank-16
+  // rows low (4 KB)
   static constexpr int kOffK = 0, kOffV = kTile, kOffG = 2 * kTile;
-  static constexpr int kStage = 2 * kTile + kGTile;
-  // operand tiles (1024-aligned): KH KL VH VL
-  static constexpr int kTiles = 2 * kStage;
-  static constexpr int kMisc = kTiles + 4 * kTile;
+  static constexpr int kStage = 2 * kTile + (kGate ? kLowTile : kGTile);
+  // gate in-kernel: the chunk's g (fp32 rows, 16-byte units XOR-ed with
+  // row % 16), single-buffered
+  static constexpr int kOffGT = 2 * kStage;
+  // operand tiles (1024-aligned): KH KL VH VL; then, gate in-kernel, the A
+  // tile of low (fp16 hi in K columns 0-15, lo in 16-31) and the two B tiles
+  // of W_up (16 x 64, MN-major, 2 KB each)
+  static constexpr int kTiles = kOffGT + (kGate ? kGTile : 0);
+  static constexpr int kOffAU = kTiles + 4 * kTile;
+  static constexpr int kOffBU = kOffAU + (kGate ? kTile : 0);
+  static constexpr int kMisc = kOffBU + (kGate ? 2 * 2048 : 0);
   static constexpr int kSmem = kMisc + (int)sizeof(SumMisc) + 1024;
-  static constexpr int kTmemCols = 128;   // two accumulators, summed at the end
+  // [0, 128) two accumulators, summed at the end; gate: [128, 192) u
+  static constexpr int kTmemCols = kGate ? 256 : 128;
   static constexpr int kBlocksPerSM = 2;
   // eight warps build the tiles; a ninth issues the MMAs and the box loads, so
   // the builders go on to the next chunk while the tensor pipe works
   static constexpr int kThreadsAll = kThreads + 32;
+  static_assert(kTiles % 1024 == 0 && kStage % 1024 == 0 && kOffAU % 1024 == 0 && kOffBU % 1024 == 0,
+                "operand tiles and swizzled boxes must be 1024-byte aligned");
+  static_assert(2 * (kSmem + 1024) <= 228 * 1024, "two summary CTAs must share an SM");
 };
-static_assert(SumLayout::kTiles % 1024 == 0, "operand tiles must be 1024-byte aligned");
-static_assert(2 * (SumLayout::kSmem + 1024) <= 228 * 1024, "two summary CTAs must share an SM");
+using SumLayout = SumLayoutT<false>;
 
-template <typename T>
-__global__ void __launch_bounds__(SumLayout::kThreadsAll, SumLayout::kBlocksPerSM)
+// The staged low rows of a chunk (64 bytes each), gathered with cp.async;
+// rows past ntok are zeroed.  `rows` are token rows (b T + t) H + h.
+__device__ __forceinline__ void fetch_low(uint8_t* dst, const float* low, const long long* rows, int ntok,
+                                          int H, int tid) {
+  const int j = tid >> 2, part = (tid & 3) * 16;
+  if (j < ntok) cp_async16(dst + j * 64 + part, (const uint8_t*)low + (rows[j] / H) * 64 + part);
+  else *reinterpret_cast<uint4*>(dst + j * 64 + part) = make_uint4(0u, 0u, 0u, 0u);
+}
+// Byte offset of fp32 element (row, col) of a 64 x 64 tile kept as two
+// SWIZZLE_128B halves (columns 0-31, 32-63; 128-byte rows, 16-byte units
+// XOR-ed with row % 8): the layout a tensor-map store of 32-column boxes
+// reads, and conflict-free for a row per thread and for a row per warp.
+__device__ __forceinline__ uint32_t gt_off(int row, int col) {
+  return (uint32_t)((col >> 5) * 8192 + row * 128 + (((((col & 31) >> 2) ^ (row & 7))) << 4) + (col & 3) * 4);
+}
+
+// kGate: the gate's second half runs here (GTR article, 方法详解 §1, the
+// low-rank gate): per chunk the rank-16 rows low of its tokens become a
+// scaled two-term fp16 A tile, u = low W_up comes from three MMAs (hi*hi +
+// hi*lo + lo*hi, as in the gate kernel), and g = logsigmoid(u + b)/tau is
+// formed from TMEM (thread = token row, 16 dims), written to g_out for the
+// output stage and staged for the cumsum.  Scan positions past the sequence
+// get g = 0.
+template <typename T, bool kGate>
+__global__ void __launch_bounds__(SumLayoutT<kGate>::kThreadsAll, SumLayoutT<kGate>::kBlocksPerSM)
 gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
-  using L = SumLayout;
+  using L = SumLayoutT<kGate>;
   constexpr bool kV2 = std::is_same<T, __half>::value;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -996,6 +1131,9 @@ gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
   uint8_t* KL = KH + kTile;
   uint8_t* VH = KH + 2 * kTile;       // V (MN-major B)
   uint8_t* VL = KH + 3 * kTile;
+  uint8_t* GT = sm + L::kOffGT;       // gate: the chunk's g
+  uint8_t* AU = sm + L::kOffAU;       // gate: low (A)
+  uint8_t* BU = sm + L::kOffBU;       // gate: W_up hi, lo (B)
   SumMisc& m = *reinterpret_cast<SumMisc*>(sm + L::kMisc);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1012,7 +1150,8 @@ gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
   const bool tma = p.tma != 0;
   const int rmask = (tma && dir_reversed(d)) ? kC - 1 : 0;   // staging row of scan offset i: i ^ rmask
   const bool vdirect = !kV2 && rmask == 0;                    // a bf16 v in scan order is the B operand as staged
-  // final accumulator read: quadrant qd, column half, 16 columns from cbase of row `row`
+  // final accumulator read (and, gate, the u read): quadrant qd, column half,
+  // 16 columns from cbase of row `row`
   const int qd = warp & 3, half = warp >> 2;
   const int row = qd * 16 + (lane & 15);
   const int cbase = half * 32 + (lane >> 4) * 16;
@@ -1022,9 +1161,10 @@ gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
   // step `it` handles chunk c0 + nch - 1 - it (last to first); only the first can be ragged
   const int clast = c0 + nch - 1;
   auto stage = [&](int it) -> uint8_t* { return sm + (it & 1) * L::kStage; };
-  // step it's k, v (v in the operand layout), g into stage(it)
-  // (the box loads of k and v may be issued apart from g's: `parts` 1 = k, v;
-  // 2 = g; 3 = all; the barrier expects all three from the first part)
+  // step it's k, v (v in the operand layout), gate rows into stage(it)
+  // (the box loads of k and v may be issued apart from the gate's: `parts`
+  // 1 = k, v; 2 = g or low; 3 = all; the barrier expects all three from the
+  // first part)
   auto fetch = [&](int it, int parts = 3) {
     const int s0 = (clast - it) * kC;
     uint8_t* st = stage(it);
@@ -1032,17 +1172,21 @@ gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
       if (tid == kThreads) {
         uint64_t* bar = &m.ld[it & 1];
         if (parts & 1) {
-          mbar_arrive_tx(bar, 2 * kTile + kGTile);
+          mbar_arrive_tx(bar, 2 * kTile + (kGate ? kLowTile : kGTile));
           tma_box(p, mp, kMapK, st + L::kOffK, bar, d, b, h, s0);
           tma_box(p, mp, kMapV, st + L::kOffV, bar, d, b, h, s0);
         }
-        if (parts & 2) tma_box(p, mp, kMapG, st + L::kOffG, bar, d, b, h, s0);
+        if (parts & 2) {
+          if (kGate) tma_box(p, mp, kMapL, st + L::kOffG, bar, d, b, 0, s0);
+          else tma_box(p, mp, kMapG, st + L::kOffG, bar, d, b, h, s0);
+        }
       }
     } else {
       const int ntok = min(kC, p.T - s0);
       fetch16(st + L::kOffK, p.k, m.rows[it & 1], ntok, tid);
       fetch16<true>(st + L::kOffV, p.v, m.rows[it & 1], ntok, tid);
-      fetch_g(st + L::kOffG, p.g, m.rows[it & 1], ntok, tid);
+      if (kGate) fetch_low(st + L::kOffG, p.low, m.rows[it & 1], ntok, p.H, tid);
+      else fetch_g(st + L::kOffG, p.g, m.rows[it & 1], ntok, tid);
       cp_async_commit();
     }
   };
@@ -1052,6 +1196,9 @@ gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
     mbar_init(&m.mma, 1);
     mbar_init(&m.ld[0], 1);
     mbar_init(&m.ld[1], 1);
+    mbar_init(&m.umma, 1);
+    mbar_init(&m.wl, 1);
+    mbar_init(&m.gready, kWarps);
     mbar_fence_init();
   }
   if (!tma) {
@@ -1059,8 +1206,8 @@ gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
     if (nch > 1) chunk_rows(p, m.rows[1], b, h, d, (clast - 1) * kC, kC, tid);
   }
   __syncthreads();
-  // k and v are inputs: their first boxes go out before the wait; g comes
-  // from the previous kernel
+  // k and v are inputs: their first boxes go out before the wait; the gate
+  // rows come from the previous kernel
   if (tma) {
     fetch(0, 1);
     if (nch > 1) fetch(1, 1);
@@ -1074,6 +1221,15 @@ gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
     fetch(0);
     if (nch > 1) fetch(1);
   }
+  if (kGate && tid == kThreads) {
+    // this head's W_up terms (2 KB each), column scales and bias
+    mbar_arrive_tx(&m.wl, 2 * 2048 + 256 + (p.gbias ? 256 : 0));
+    bulk_g2s(BU, p.wu + 2048 * h, 2048, &m.wl);
+    bulk_g2s(BU + 2048, p.wu + p.wu_term + 2048 * h, 2048, &m.wl);
+    bulk_g2s(m.ci, p.wu_scale + kD * h, 256, &m.wl);
+    if (p.gbias) bulk_g2s(m.gb, p.gbias + kD * h, 256, &m.wl);
+  }
+  if (kGate && !p.gbias && tid < kD) m.gb[tid] = 0.f;
   int fetched = nch > 1 ? 1 : 0, waited = -1;   // box loads issued / consumed, by step
   if (warp == 0) {
     tmem_alloc(&m.tmem, L::kTmemCols);
@@ -1084,6 +1240,15 @@ gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
   tc_after_sync();
   const uint32_t tm = m.tmem;
   constexpr uint32_t kIdKV = idesc_bf16(1, 1);
+  constexpr uint32_t kIdU = idesc_f16(0, 1);     // A K-major, B MN-major
+  // gate: u = low W_up into columns [128, 192), hi*hi + hi*lo + lo*hi
+  auto issue_u = [&]() {
+    const uint64_t ah = desc_k(AU), bhi = desc_mn(BU), blo = desc_mn(BU + 2048);
+    mma_f16(tm + 128, ah, bhi, kIdU, 0u);
+    mma_f16(tm + 128, ah, blo, kIdU, 1u);
+    mma_f16(tm + 128, ah + kStepK, bhi, kIdU, 1u);
+    mma_commit(&m.umma);
+  };
 
   uint32_t ph = 0;
   bool failed = false;
@@ -1092,6 +1257,19 @@ gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
     // ---- control warp: products of each chunk once the builders have its
     // tiles, then (box loads) the chunk after next into the buffer they read
     for (int it = 0; it < nch; ++it) {
+      if (kGate) {
+        // the chunk's g tile out by two tensor-map stores (not for gathered
+        // loads or a reversed scan's ragged chunk: the builders store those),
+        // read out of shared memory before barrier B frees the tile
+        const int s0 = (clast - it) * kC;
+        if (!mbar_wait(&m.gready, (uint32_t)it & 1u)) failed = true;
+        if (tid == kThreads && !failed && tma && !(rmask && s0 + kC > p.T)) {
+          tma_store_box(p, mp, kMapGS, GT, d, b, h, s0, 0);
+          tma_store_box(p, mp, kMapGS, GT + 8192, d, b, h, s0, 32);
+          bulk_commit();
+          bulk_wait_read<0>();
+        }
+      }
       tc_before_sync();
       if (__syncthreads_or(failed)) {                 // the builders' barrier B
         failed = true;
@@ -1100,6 +1278,7 @@ gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
       tc_after_sync();
       uint8_t* const Vb = vdirect ? stage(it) + L::kOffV : VH;
       if (tid == kThreads) {
+        if (kGate && it + 1 < nch) issue_u();   // chunk it + 1's gate product (its A tile is built)
         // k^hi V into columns [0, 64), k^lo V into [64, 128)
         mma_k64<kStepMN, kStepMN>(tm, desc_mn(KH), desc_mn(Vb), kIdKV, it > 0);
         mma_k64<kStepMN, kStepMN>(tm + 64, desc_mn(KL), desc_mn(Vb), kIdKV, it > 0);
@@ -1116,29 +1295,117 @@ gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
       __syncwarp();
     }
   } else {
-    // R: summed log-gate, per dim, of the chunks already seen (the segment's tail)
-    float2 R = make_float2(0.f, 0.f);
-    for (int it = 0; it < nch; ++it) {
-      uint8_t* st = stage(it);
-      const T* kst = reinterpret_cast<const T*>(st + L::kOffK);
-      const float* G = reinterpret_cast<const float*>(st + L::kOffG);
+    // gate: the A tile of chunk `it`'s low rows (row tid / 4, ranks 4 (tid %
+    // 4) .. + 3; a power-of-two scale per row over the four threads of the
+    // row).  Chunk it + 1's tile is built before barrier B of chunk it and
+    // the control warp issues its product ahead of chunk it's k^T V products,
+    // so u is ready when chunk it + 1 starts.
+    int u_issued = 0, u_waited = 0;
+    auto gate_tile = [&](int it) {
+      const float* lw = reinterpret_cast<const float*>(stage(it) + L::kOffG);
+      const int r = tid >> 2, k0 = (tid & 3) * 4;
+      const float4 l = *reinterpret_cast<const float4*>(lw + r * kLowRank + k0);
+      float mx = fmaxf(fmaxf(fabsf(l.x), fabsf(l.y)), fmaxf(fabsf(l.z), fabsf(l.w)));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      const int e = scale_exp(mx);
+      const float sc = pow2i(e);
+      if ((tid & 3) == 0) m.ri[r] = pow2i(-e);
+      uint32_t h0, h1, l0, l1;
+      split2h(l.x * sc, l.y * sc, h0, l0);
+      split2h(l.z * sc, l.w * sc, h1, l1);
+      *reinterpret_cast<uint2*>(AU + sw16(r, k0)) = make_uint2(h0, h1);
+      *reinterpret_cast<uint2*>(AU + sw16(r, kLowRank + k0)) = make_uint2(l0, l1);
+      fence_async_smem();
+    };
+    // the loads of chunk `it` have landed (box loads: its barrier; gathers:
+    // every cp.async group of this thread, then the builders' barrier)
+    auto wait_loads = [&](int it) {
       if (tma) {
         failed |= !mbar_wait(&m.ld[it & 1], (uint32_t)(it >> 1) & 1u);
-        waited = it;
+        waited = it > waited ? it : waited;
       } else {
         if (it == 0 && nch > 1) cp_async_wait<1>();
         else cp_async_wait<0>();
         named_barrier(1, kThreads);
       }
+    };
+    if (kGate) {
+      failed |= !mbar_wait(&m.wl, 0);
+      wait_loads(0);
+      gate_tile(0);
+      tc_before_sync();
+      named_barrier(1, kThreads);
+      if (tid == 0) {
+        tc_after_sync();
+        issue_u();
+      }
+      u_issued = 1;
+    }
+    // gate: chunk it's g goes out by two tensor-map stores of the staged
+    // tile, except with gathered loads or where the box would start before
+    // token 0 (a reversed scan's ragged chunk): then each warp stores its rows
+    const bool gt_tma = tma;
+    // R: summed log-gate, per dim, of the chunks already seen (the segment's tail)
+    float2 R = make_float2(0.f, 0.f);
+    for (int it = 0; it < nch; ++it) {
+      uint8_t* st = stage(it);
+      const T* kst = reinterpret_cast<const T*>(st + L::kOffK);
+      const float* G = reinterpret_cast<const float*>(kGate ? GT : st + L::kOffG);
+      const int s0 = (clast - it) * kC;   // first scan position of the chunk
+      wait_loads(it);
       // rows of the next chunk (cp.async gathers; that buffer's gather is long done)
       if (!tma && it >= 1 && it + 1 < nch) chunk_rows(p, m.rows[(it + 1) & 1], b, h, d, (clast - it - 1) * kC, kC, tid);
+
+      if (kGate) {
+        // ---- g of this chunk from u (thread = token row `row`, dims cbase ..
+        // cbase + 15), staged for the cumsum; scan positions past the
+        // sequence get g = 0
+        if (!mbar_wait(&m.umma, (uint32_t)u_waited & 1u)) failed = true;
+        ++u_waited;
+        tc_after_sync();
+        float u[16];
+        tmem_ld16x2(tm + lane_base + 128 + half * 32, u);
+        tmem_ld_wait(u);
+        const bool valid = s0 + (row ^ rmask) < p.T;
+        const float ri = m.ri[row];
+        const float inv_tau = p.inv_tau, ln2_tau = 0.6931471805599453f * p.inv_tau;
+        float gv[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          gv[c] = valid ? logsigmoid_over_tau(fmaf(u[c] * ri, m.ci[cbase + c], m.gb[cbase + c]), inv_tau, ln2_tau)
+                        : 0.f;
+#pragma unroll
+        for (int c = 0; c < 16; c += 4)
+          *reinterpret_cast<float4*>(GT + gt_off(row, cbase + c)) = make_float4(gv[c], gv[c + 1], gv[c + 2], gv[c + 3]);
+        fence_async_smem();               // the tile, then the tensor-map stores' reads
+        __syncwarp();
+        if (lane == 0) mbar_arrive_one(&m.gready);   // the control warp stores it
+        tc_before_sync();
+        named_barrier(1, kThreads);
+      }
 
       // ---- in-chunk cumsum G (eight scan offsets in registers), the partial
       // sums of the other warps, and the chunk total Gam
       float2 gc[8];
+      // gate: each warp writes g of its eight scan positions to g_out, one
+      // whole 256-byte row per position (box loads: consecutive positions of
+      // a chunk are `gstep` grid indices apart)
+      const bool gst = kGate && !(gt_tma && !(rmask && s0 + kC > p.T));   // this chunk's g by the warps
+      long long grow = 0, gstep = 0;
+      if (gst && tma) {
+        grow = (long long)b * p.T + scan_to_grid(d, min(s0 + tb, p.T - 1), p.T, p.gh, p.gw);
+        gstep = d == kLR ? 1 : d == kRL ? -1 : d == kTB ? p.gw : -p.gw;
+      }
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        gc[i] = *reinterpret_cast<const float2*>(G + ((tb + i) ^ rmask) * kD + dc);
+        const int rg = (tb + i) ^ rmask;
+        gc[i] = kGate ? *reinterpret_cast<const float2*>(GT + gt_off(rg, dc))
+                      : *reinterpret_cast<const float2*>(G + rg * kD + dc);
+        if (gst && s0 + tb + i < p.T) {
+          const long long tr = tma ? (grow + gstep * i) * p.H + h : m.rows[it & 1][tb + i];
+          *reinterpret_cast<float2*>(p.g_out + tr * kD + dc) = gc[i];
+        }
         if (i) { gc[i].x += gc[i - 1].x; gc[i].y += gc[i - 1].y; }
       }
       *reinterpret_cast<float2*>(&m.part[warp][dc]) = gc[7];
@@ -1182,6 +1449,10 @@ gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
           }
         }
       }
+      if (kGate && it + 1 < nch) {        // the next chunk's gate tile
+        wait_loads(it + 1);
+        gate_tile(it + 1);
+      }
       fence_async_smem();
       tc_before_sync();
       if (__syncthreads_or(failed)) {                 // barrier B: the control warp issues
@@ -1189,9 +1460,14 @@ gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
         break;
       }
       tc_after_sync();
+      if (kGate && it + 1 < nch) ++u_issued;
     }
     if (warp == 0)
       *reinterpret_cast<float2*>(&m.part[0][dc]) = R;  // the segment's summed log-gate
+    // a gate product not waited for (early exit) completes before tensor
+    // memory is released
+    if (kGate && tid == 0 && u_issued > u_waited) (void)mbar_wait(&m.umma, (uint32_t)(u_issued - 1) & 1u);
+
   }
   // Drain: the last issued products, then box loads issued but not consumed
   // (only after an early exit), before TMEM and shared memory are released.
@@ -1208,6 +1484,10 @@ gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
   if (tma && tid == 0)
     for (int x = m.waited + 1; x <= m.fetched; ++x)
       if (!mbar_wait(&m.ld[x & 1], (uint32_t)(x >> 1) & 1u)) failed = true;
+  if (kGate && tid == kThreads) {
+    (void)mbar_wait(&m.wl, 0);                    // the weight copies have landed
+    bulk_wait<0>();                               // every g store is complete
+  }
   failed = __syncthreads_or(failed) != 0;
   if (!failed && !control) {
     float ds[16], dl[16];
@@ -1256,10 +1536,13 @@ inline int launch_tc_kernel(K kern, int smem, int threads, int nseg, int BH, cud
 template <typename T>
 inline int launch_tc_typed(int stage, const tc::Params& p, const tc::Maps& mp, int BH, cudaStream_t st,
                            int dev) {
-  static bool done_sum[64], done_out[64];
+  static bool done_sum[64], done_out[64], done_gsum[64];
   if (stage == 0)
-    return launch_tc_kernel(tc::gla_sum_tc<T>, tc::SumLayout::kSmem, tc::SumLayout::kThreadsAll, p.nseg, BH, st,
-                            done_sum, dev, p, mp);
+    return launch_tc_kernel(tc::gla_sum_tc<T, false>, tc::SumLayout::kSmem, tc::SumLayout::kThreadsAll, p.nseg,
+                            BH, st, done_sum, dev, p, mp);
+  if (stage == 2)   // summary with the gate's second half in-kernel
+    return launch_tc_kernel(tc::gla_sum_tc<T, true>, tc::SumLayoutT<true>::kSmem,
+                            tc::SumLayoutT<true>::kThreadsAll, p.nseg, BH, st, done_gsum, dev, p, mp);
   return launch_tc_kernel(tc::gla_out_tc<T>, tc::OutLayout::kSmem, tc::OutLayout::kThreadsAll, (p.nseg + 1) / 2,
                           BH, st, done_out, dev, p, mp);
 }
@@ -1279,6 +1562,33 @@ inline int launch_tc(int dtype, int stage, const void* q, const void* k, const v
   const int BH = B * H;
   return dtype == kF16 ? launch_tc_typed<__half>(stage, p, mp, BH, st, dev)
                        : launch_tc_typed<__nv_bfloat16>(stage, p, mp, BH, st, dev);
+}
+
+// The summary stage with the gate's second half in-kernel (stage 2 of
+// launch_tc_typed): low [B, T, 16] fp32, the packed W_up terms (`wu`,
+// `wu_term` bytes apart), their inverse column scales, bias (or null), 1/tau;
+// writes g_out [B, T, H, 64] fp32 and the segment states.  `maps` must hold
+// the k, v and low maps when not null.
+inline int launch_tc_gated_sum(int dtype, const void* k, const void* v, const float* low, const uint8_t* wu,
+                               int wu_term, const float* wu_scale, const float* gbias, float inv_tau,
+                               float* g_out, float* wsS, float* wsA, int B, int H, int T, int gh, int gw,
+                               int dir, int nseg, const tc::Maps* maps, cudaStream_t st) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -5;
+  tc::Params p{nullptr, k, v, nullptr, nullptr, nullptr, wsS, wsA, nullptr, H, T, gh, gw, dir, nseg,
+               maps ? 1 : 0};
+  p.low = low;
+  p.wu = wu;
+  p.wu_scale = wu_scale;
+  p.gbias = gbias;
+  p.g_out = g_out;
+  p.wu_term = wu_term;
+  p.inv_tau = inv_tau;
+  static const tc::Maps kNoMaps{};
+  const tc::Maps& mp = maps ? *maps : kNoMaps;
+  const int BH = B * H;
+  return dtype == kF16 ? launch_tc_typed<__half>(2, p, mp, BH, st, dev)
+                       : launch_tc_typed<__nv_bfloat16>(2, p, mp, BH, st, dev);
 }
 
 }  // namespace gtr

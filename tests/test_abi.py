@@ -97,3 +97,27 @@ def test_binding_refuses_a_missing_library(tmp_path):
             binding.load(str(tmp_path / "nope.so"))
         finally:
             binding._lib = saved
+
+
+def test_gated_call_rejects_invalid_arguments_before_any_launch(lib):
+    P = ctypes.c_void_p(16)
+    S = None
+    F = ctypes.c_float
+
+    def call(x=P, xdt=1, packed=P, bias=None, dm=384, rank=16, tau=16.0, q=P, g=P, out=P, B=1, H=6,
+             gh=8, gw=8, dk=64, dv=64, dir_=0, chunk=64, dtype=1):
+        return lib.gtr_gla_fwd_gated(x, xdt, packed, bias, dm, rank, F(tau), q, P, P, P, None, g, out,
+                                     B, H, gh, gw, dk, dv, dir_, chunk, dtype, S)
+
+    assert call(dir_=9) == -1                       # GLA arguments as gtr_gla_fwd
+    assert call(dk=48) == -2
+    assert call(tau=0.0) == -1                      # gate arguments as gtr_gate_fwd_packed
+    assert call(xdt=7) == -1
+    assert call(rank=8) == -2                       # only the packed (tensor-core) gate shapes
+    assert call(dm=100) == -2
+    assert call(xdt=0) == -2                        # fp32 x has no packed weights
+    assert call(B=0, x=None, packed=None, q=None, g=None, out=None) == 0   # empty problem
+    assert call(packed=None) == -1
+    assert call(g=None) == -1
+    assert call(x=ctypes.c_void_p(24)) == -3        # 16-byte alignment
+    assert call(g=ctypes.c_void_p(40)) == -3
