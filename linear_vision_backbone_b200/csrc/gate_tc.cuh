@@ -97,7 +97,8 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
                : "memory");
 }
 constexpr int kM = 128;               // rows of the MMA tile (tokens per CTA <= kM)
-constexpr int kThreads = 512;
+constexpr int kThreads = 512;         // stages and epilogue: 16 warps
+constexpr int kThreadsAll = kThreads + 32;   // + a warp that issues the g stores
 constexpr int kPackThreads = 256;
 constexpr int kMaxDm = 384;           // d_model: multiple of 64, <= 384
 constexpr int kMaxHD = 448;           // H*dk: multiple of 64, <= 448
@@ -134,6 +135,8 @@ static_assert(Pack::kBytes % 16 == 0 && Pack::kScaleBytes % 16 == 0, "bulk copie
 
 struct Misc {
   uint64_t mma[2];
+  uint64_t sfull[3];                 // epilogue slab buffer b staged (one arrival per epilogue warp)
+  uint64_t sfree[3];                 // its tensor-map stores have read it
   uint64_t ld;                       // the packed weights
   uint64_t ldx[kMaxDm / 64];         // the x tile, one 64-column atom each
   uint32_t tmem;
@@ -275,7 +278,7 @@ gate_pack_tc(const float* __restrict__ w_down, const float* __restrict__ w_up, i
 // tmx: x as [N rows][dm] 16-bit, box 64 x 128, 128B swizzle.  tmg: g as
 // [N rows][HD] fp32, box 32 x tpc, 128B swizzle.
 template <typename TX>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreadsAll, 1)
 gate_fwd_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmg,
             const uint8_t* __restrict__ pack, const float* __restrict__ bias, int dm, int HD,
             float inv_tau, int tpc) {
@@ -296,6 +299,10 @@ gate_fwd_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUt
     for (int a = 0; a < kMaxDm / 64; ++a) tc::mbar_init(&m.ldx[a], 1);
     tc::mbar_init(&m.mma[0], 1);
     tc::mbar_init(&m.mma[1], 1);
+    for (int b = 0; b < 3; ++b) {
+      tc::mbar_init(&m.sfull[b], kThreads / 32);
+      tc::mbar_init(&m.sfree[b], 1);
+    }
     tc::mbar_fence_init();
   }
   if (warp == 0) {
@@ -399,56 +406,66 @@ gate_fwd_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUt
   // ---- epilogue, one 64-column slab of u at a time: thread = token row (TMEM
   // lane quadrant warp % 4), warp w on the slab's 16-column quarter w / 4.  Each
   // slab is staged as two 32-column halves (128-byte rows, 16-byte units XOR-ed
-  // with row % 8: the TMA 128B swizzle) and TMA-stored.  Three slab buffers
-  // rotate, so the one barrier per slab also covers buffer reuse: before it,
-  // the issuing thread waits until the store of two slabs ago has read its
-  // buffer, which is the buffer the next slab fills.
+  // with row % 8: the TMA 128B swizzle) in one of three rotating buffers; each
+  // warp signals its part on the buffer's `sfull` barrier, and a seventeenth
+  // warp issues the two tensor-map stores of a full slab and signals `sfree`
+  // once they have read the buffer, which the warps wait for before staging
+  // the slab three later there.  No block barrier runs between slabs.
   if (ok) {
-    const float ln2_tau = 0.6931471805599453f * inv_tau;
-    const int q = warp & 3, qp = warp >> 2;
-    const int r = q * 32 + lane;
-    const float ri = m.low_i[r];
-    const uint32_t tq = tm + ((uint32_t)(q * 32) << 16) + 64 + 16 * qp;
     const int nslab = HD / 64;
-    auto emit = [&](int j, const float* u) {
-      uint8_t* slab = tX + (j % 3) * (2 * Layout::kHalfSlab);
-      const int cb = 64 * j + 16 * qp;
-      uint8_t* half = slab + (qp >> 1) * Layout::kHalfSlab + r * 128;
+    if (warp < kThreads / 32) {
+      const float ln2_tau = 0.6931471805599453f * inv_tau;
+      const int q = warp & 3, qp = warp >> 2;
+      const int r = q * 32 + lane;
+      const float ri = m.low_i[r];
+      const uint32_t tq = tm + ((uint32_t)(q * 32) << 16) + 64 + 16 * qp;
+      auto emit = [&](int j, const float* u) {
+        uint8_t* slab = tX + (j % 3) * (2 * Layout::kHalfSlab);
+        if (j >= 3) ok &= tc::mbar_wait(&m.sfree[j % 3], (uint32_t)((j / 3) - 1) & 1u);
+        const int cb = 64 * j + 16 * qp;
+        uint8_t* half = slab + (qp >> 1) * Layout::kHalfSlab + r * 128;
 #pragma unroll
-      for (int c = 0; c < 16; c += 4) {
-        const float4 bb = *reinterpret_cast<const float4*>(&m.bias[cb + c]);
-        const float4 ci = *reinterpret_cast<const float4*>(&m.wu_i[cb + c]);
-        const int unit = (qp & 1) * 4 + (c >> 2);
-        *reinterpret_cast<float4*>(half + ((unit ^ (r & 7)) << 4)) = make_float4(
-            logsigmoid_over_tau(fmaf(u[c + 0] * ri, ci.x, bb.x), inv_tau, ln2_tau),
-            logsigmoid_over_tau(fmaf(u[c + 1] * ri, ci.y, bb.y), inv_tau, ln2_tau),
-            logsigmoid_over_tau(fmaf(u[c + 2] * ri, ci.z, bb.z), inv_tau, ln2_tau),
-            logsigmoid_over_tau(fmaf(u[c + 3] * ri, ci.w, bb.w), inv_tau, ln2_tau));
+        for (int c = 0; c < 16; c += 4) {
+          const float4 bb = *reinterpret_cast<const float4*>(&m.bias[cb + c]);
+          const float4 ci = *reinterpret_cast<const float4*>(&m.wu_i[cb + c]);
+          const int unit = (qp & 1) * 4 + (c >> 2);
+          const float2 g01 = tc::logsigmoid_over_tau2(fmaf(u[c + 0] * ri, ci.x, bb.x),
+                                                      fmaf(u[c + 1] * ri, ci.y, bb.y), inv_tau, ln2_tau);
+          const float2 g23 = tc::logsigmoid_over_tau2(fmaf(u[c + 2] * ri, ci.z, bb.z),
+                                                      fmaf(u[c + 3] * ri, ci.w, bb.w), inv_tau, ln2_tau);
+          *reinterpret_cast<float4*>(half + ((unit ^ (r & 7)) << 4)) = make_float4(g01.x, g01.y, g23.x, g23.y);
+        }
+        tc::fence_async_smem();                   // these writes, then the TMA engine's reads
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive_one(&m.sfull[j % 3]);
+      };
+      // the next slab's TMEM columns are requested before this one is formed
+      float ua[16], ub[16];
+      tmem_ld16(tq, ua);
+      for (int j = 0; j < nslab; j += 2) {
+        tc::tmem_ld_wait(ua);                     // slab j in ua
+        if (j + 1 < nslab) tmem_ld16(tq + 64 * (j + 1), ub);
+        emit(j, ua);
+        if (j + 1 < nslab) {
+          tc::tmem_ld_wait(ub);                   // slab j + 1 in ub
+          if (j + 2 < nslab) tmem_ld16(tq + 64 * (j + 2), ua);
+          emit(j + 1, ub);
+        }
       }
-      tc::fence_async_smem();                     // these writes, then the TMA engine's reads
-      if (tid == 0 && j >= 2) bulk_wait_read<1>();   // slab j - 2's store has read buffer (j + 1) % 3
-      __syncthreads();
-      if (tid == 0) {
+    } else if (lane == 0) {
+      for (int j = 0; j < nslab; ++j) {
+        uint8_t* slab = tX + (j % 3) * (2 * Layout::kHalfSlab);
+        ok &= tc::mbar_wait(&m.sfull[j % 3], (uint32_t)(j / 3) & 1u);
         tma_store_2d(&tmg, 64 * j, tok0, slab);
         tma_store_2d(&tmg, 64 * j + 32, tok0, slab + Layout::kHalfSlab);
         bulk_commit();
+        bulk_wait_read<0>();
+        tc::mbar_arrive_one(&m.sfree[j % 3]);
       }
-    };
-    // the next slab's TMEM columns are requested before this one is formed
-    float ua[16], ub[16];
-    tmem_ld16(tq, ua);
-    for (int j = 0; j < nslab; j += 2) {
-      tc::tmem_ld_wait(ua);                       // slab j in ua
-      if (j + 1 < nslab) tmem_ld16(tq + 64 * (j + 1), ub);
-      emit(j, ua);
-      if (j + 1 < nslab) {
-        tc::tmem_ld_wait(ub);                     // slab j + 1 in ub
-        if (j + 2 < nslab) tmem_ld16(tq + 64 * (j + 2), ua);
-        emit(j + 1, ub);
-      }
+      bulk_wait<0>();                             // every store done before the block ends
     }
-    if (tid == 0) bulk_wait<0>();                 // every store done before the block ends
   }
+  if (__syncthreads_or(!ok) && tid == 0) gtr_flag(kStatusMbarTimeout);
   tc::tc_before_sync();
   __syncthreads();
   tc::tc_after_sync();

@@ -345,13 +345,13 @@ int gate_fwd_packed_launch(int x_dtype, const void* x, const void* pack, const f
   static bool done_h[kMaxDevices], done_b[kMaxDevices];
   if (x_dtype == GTR_F16) {
     if (int rc = ensure_smem(gate_tc::gate_fwd_tc<__half>, gate_tc::Layout::kSmem, done_h, dev)) return rc;
-    return launch_pdl(gate_tc::gate_fwd_tc<__half>, dim3((unsigned)blocks), dim3(gate_tc::kThreads),
+    return launch_pdl(gate_tc::gate_fwd_tc<__half>, dim3((unsigned)blocks), dim3(gate_tc::kThreadsAll),
                       gate_tc::Layout::kSmem, st, tmx, tmg, (const uint8_t*)pack, bias, dm, HD, inv_tau, tpc)
                ? GTR_ERR_CUDA
                : GTR_OK;
   }
   if (int rc = ensure_smem(gate_tc::gate_fwd_tc<__nv_bfloat16>, gate_tc::Layout::kSmem, done_b, dev)) return rc;
-  return launch_pdl(gate_tc::gate_fwd_tc<__nv_bfloat16>, dim3((unsigned)blocks), dim3(gate_tc::kThreads),
+  return launch_pdl(gate_tc::gate_fwd_tc<__nv_bfloat16>, dim3((unsigned)blocks), dim3(gate_tc::kThreadsAll),
                     gate_tc::Layout::kSmem, st, tmx, tmg, (const uint8_t*)pack, bias, dm, HD, inv_tau, tpc)
              ? GTR_ERR_CUDA
              : GTR_OK;
