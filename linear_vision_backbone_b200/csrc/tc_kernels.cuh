@@ -640,6 +640,12 @@ __device__ __forceinline__ float column_cumsum(const float* G, float (&gv)[16], 
   return ((p0 + p1) + p2) + p3;
 }
 
+// 32-byte store (st.global.v8, sm_100); `p` must be 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void* p, uint4 a, uint4 b) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a.x), "r"(a.y), "r"(a.z),
+               "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+               : "memory");
+}
 __device__ __forceinline__ float silu_fast(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
 // ===================================================================== K4
@@ -746,6 +752,7 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
     nch = 0;
   }
   const bool tma = p.tma != 0;
+  const bool out32 = ((uintptr_t)p.out & 31) == 0;
   // staging row of scan offset i: box loads of a reversed scan hold the chunk backwards
   const int rmask = (tma && dir_reversed(d)) ? kC - 1 : 0;
   // a bf16 v in scan order is the operand tile itself (double-buffered by
@@ -1045,13 +1052,21 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
       if (row < ntok) {
         const float inv = rsqrtf(ss * (1.0f / kD) + kRmsEps);
         T* dst = reinterpret_cast<T*>(p.out) + m.rows[par][row] * kD + cbase;
+        uint4 y8[2];
 #pragma unroll
         for (int c = 0; c < 16; c += 8) {
           const uint2 lo = pack4<T>(o[c + 0] * inv * wz[c + 0], o[c + 1] * inv * wz[c + 1],
                                     o[c + 2] * inv * wz[c + 2], o[c + 3] * inv * wz[c + 3]);
           const uint2 hi = pack4<T>(o[c + 4] * inv * wz[c + 4], o[c + 5] * inv * wz[c + 5],
                                     o[c + 6] * inv * wz[c + 6], o[c + 7] * inv * wz[c + 7]);
-          *reinterpret_cast<uint4*>(dst + c) = make_uint4(lo.x, lo.y, hi.x, hi.y);
+          y8[c >> 3] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+        }
+        // the row's 32 bytes: one whole sector per thread when `out` is 32-byte aligned
+        if (out32) {
+          st_global_v8(dst, y8[0], y8[1]);
+        } else {
+          reinterpret_cast<uint4*>(dst)[0] = y8[0];
+          reinterpret_cast<uint4*>(dst)[1] = y8[1];
         }
       }
     }
