@@ -473,6 +473,13 @@ __device__ __forceinline__ void put8(uint8_t* H, uint8_t* L, uint32_t off, const
 }
 
 // two consecutive elements (4 bytes) at byte offset `off` of the (hi, lo) tiles
+// the same in fp16 terms
+__device__ __forceinline__ void put2h(uint8_t* H, uint8_t* L, uint32_t off, float a, float b) {
+  uint32_t h, l;
+  split2h(a, b, h, l);
+  *reinterpret_cast<uint32_t*>(H + off) = h;
+  *reinterpret_cast<uint32_t*>(L + off) = l;
+}
 __device__ __forceinline__ void put2x(uint8_t* H, uint8_t* L, uint32_t off, float a, float b) {
   uint32_t h, l;
   split2(a, b, h, l);
@@ -1111,7 +1118,7 @@ gla_out_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
 constexpr int kLowRank = 16;                   // rank of the gate projection
 constexpr int kLowTile = kC * kLowRank * 4;    // a chunk's fp32 rank-16 rows: 4 KB
 struct SumMisc {
-  uint64_t mma;
+  uint64_t mma[2];                // the k^T V products of even / odd steps
   uint64_t ld[2];                 // box loads into staging buffer 0 / 1
   uint64_t umma;                  // gate: the chunk's u = low W_up product
   uint64_t wl;                    // gate: W_up tiles, column scales, bias
@@ -1134,9 +1141,10 @@ struct SumLayoutT {
   // gate in-kernel: the chunk's g (fp32 rows, 16-byte units XOR-ed with
   // row % 16), single-buffered
   static constexpr int kOffGT = 2 * kStage;
-  // operand tiles (1024-aligned): KH KL VH VL; then, gate in-kernel, the A
-  // tile of low (fp16 hi in K columns 0-15, lo in 16-31) and the two B tiles
-  // of W_up (16 x 64, MN-major, 2 KB each)
+  // operand tiles (1024-aligned): the two-term key tile k^ (hi, lo) of even
+  // and odd steps; then, gate in-kernel, the A tile of low (fp16 hi in K
+  // columns 0-15, lo in 16-31) and the two B tiles of W_up (16 x 64,
+  // MN-major, 2 KB each)
   static constexpr int kTiles = kOffGT + (kGate ? kGTile : 0);
   static constexpr int kOffAU = kTiles + 4 * kTile;
   static constexpr int kOffBU = kOffAU + (kGate ? kTile : 0);
@@ -1184,10 +1192,8 @@ gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
   constexpr bool kV2 = std::is_same<T, __half>::value;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* KH = sm + L::kTiles;       // k^ (MN-major A)
-  uint8_t* KL = KH + kTile;
-  uint8_t* VH = KH + 2 * kTile;       // V (MN-major B)
-  uint8_t* VL = KH + 3 * kTile;
+  // k^ (MN-major A) of step it: hi at ktile(it), lo kTile after it
+  auto ktile = [&](int it) -> uint8_t* { return sm + L::kTiles + (it & 1) * 2 * kTile; };
   uint8_t* GT = sm + L::kOffGT;       // gate: the chunk's g
   uint8_t* AU = sm + L::kOffAU;       // gate: low (A)
   uint8_t* BU = sm + L::kOffBU;       // gate: W_up hi, lo (B)
@@ -1206,7 +1212,11 @@ gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
   }
   const bool tma = p.tma != 0;
   const int rmask = (tma && dir_reversed(d)) ? kC - 1 : 0;   // staging row of scan offset i: i ^ rmask
-  const bool vdirect = !kV2 && rmask == 0;                    // a bf16 v in scan order is the B operand as staged
+  // The contraction over the chunk's tokens does not depend on their order,
+  // so the key tile keeps the staging's row order and the staged v (operand
+  // layout) is the B operand as it is, in its own type: an fp16 v with fp16
+  // key terms, a bf16 v with bf16 ones.  Every weight e^{R + Gam - G_s} is at
+  // most one, so the fp16 terms of k^ never overflow.
   // final accumulator read (and, gate, the u read): quadrant qd, column half,
   // 16 columns from cbase of row `row`
   const int qd = warp & 3, half = warp >> 2;
@@ -1250,7 +1260,8 @@ gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
 
   const bool control = tid >= kThreads;   // warp 8
   if (tid == 0) {
-    mbar_init(&m.mma, 1);
+    mbar_init(&m.mma[0], 1);
+    mbar_init(&m.mma[1], 1);
     mbar_init(&m.ld[0], 1);
     mbar_init(&m.ld[1], 1);
     mbar_init(&m.umma, 1);
@@ -1296,7 +1307,7 @@ gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
   __syncthreads();
   tc_after_sync();
   const uint32_t tm = m.tmem;
-  constexpr uint32_t kIdKV = idesc_bf16(1, 1);
+  constexpr uint32_t kIdKV = kV2 ? idesc_f16(1, 1) : idesc_bf16(1, 1);   // both MN-major
   constexpr uint32_t kIdU = idesc_f16(0, 1);     // A K-major, B MN-major
   // gate: u = low W_up into columns [128, 192), hi*hi + hi*lo + lo*hi
   auto issue_u = [&]() {
@@ -1307,7 +1318,6 @@ gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
     mma_commit(&m.umma);
   };
 
-  uint32_t ph = 0;
   bool failed = false;
   int issued = -1;
   if (control) {
@@ -1333,18 +1343,17 @@ gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
         break;
       }
       tc_after_sync();
-      uint8_t* const Vb = vdirect ? stage(it) + L::kOffV : VH;
+      uint8_t* const Vb = stage(it) + L::kOffV;
       if (tid == kThreads) {
         if (kGate && it + 1 < nch) issue_u();   // chunk it + 1's gate product (its A tile is built)
         // k^hi V into columns [0, 64), k^lo V into [64, 128)
-        mma_k64<kStepMN, kStepMN>(tm, desc_mn(KH), desc_mn(Vb), kIdKV, it > 0);
-        mma_k64<kStepMN, kStepMN>(tm + 64, desc_mn(KL), desc_mn(Vb), kIdKV, it > 0);
-        if (kV2) mma_k64<kStepMN, kStepMN>(tm, desc_mn(KH), desc_mn(VL), kIdKV, true);
-        mma_commit(&m.mma);
+        mma_k64<kStepMN, kStepMN>(tm, desc_mn(ktile(it)), desc_mn(Vb), kIdKV, it > 0);
+        mma_k64<kStepMN, kStepMN>(tm + 64, desc_mn(ktile(it) + kTile), desc_mn(Vb), kIdKV, it > 0);
+        mma_commit(&m.mma[it & 1]);
       }
       issued = it;
       if (tma && it + 2 < nch) {
-        if (!mbar_wait(&m.mma, (uint32_t)it & 1u)) failed = true;
+        if (!mbar_wait(&m.mma[it & 1], (uint32_t)(it >> 1) & 1u)) failed = true;
         tc_after_sync();
         fetch(it + 2);
         fetched = it + 2;
@@ -1481,34 +1490,28 @@ gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
       // weights e^{R + Gam - G_s}: the decay from token s to the segment end
       const float2 base = make_float2(R.x + tot.x - off.x, R.y + tot.y - off.y);
       R.x += tot.x; R.y += tot.y;
-      uint32_t kr[8], vr[8];
+      uint32_t kr[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int rs = (tb + i) ^ rmask;
-        kr[i] = *reinterpret_cast<const uint32_t*>(kst + rs * kD + dc);
-        vr[i] = vdirect ? 0u : *reinterpret_cast<const uint32_t*>(st + L::kOffV + sw16(rs, dc));
-      }
-      if (it > 0) {                       // the previous chunk's products have read the tiles
-        failed |= !mbar_wait(&m.mma, ph);
-        ph ^= 1;
+      for (int i = 0; i < 8; ++i)
+        kr[i] = *reinterpret_cast<const uint32_t*>(kst + ((tb + i) ^ rmask) * kD + dc);
+      if (it >= 2) {                      // step it - 2's products have read this key tile
+        failed |= !mbar_wait(&m.mma[it & 1], (uint32_t)((it - 2) >> 1) & 1u);
       }
       tc_after_sync();
-      if (!tma && it >= 1 && it + 1 < nch) fetch(it + 1);   // into the buffer those products read
+      if (!tma && it >= 1 && it + 1 < nch) {   // into the buffer step it - 1's products read
+        failed |= !mbar_wait(&m.mma[(it - 1) & 1], (uint32_t)((it - 1) >> 1) & 1u);
+        fetch(it + 1);
+      }
 
-      // ---- operand tiles: k^ = k * weight (two terms), V
+      // ---- key tile k^ = k * weight (two terms), rows in the staging's order
+      uint8_t* const KH = ktile(it);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const uint32_t o = sw16(tb + i, dc);
+        const uint32_t o = sw16((tb + i) ^ rmask, dc);
         const float2 kk = ld2(reinterpret_cast<const T*>(&kr[i]));
-        put2x(KH, KL, o, kk.x * ex2((base.x - gc[i].x) * kLog2e), kk.y * ex2((base.y - gc[i].y) * kLog2e));
-        if (!vdirect) {
-          if (kV2) {
-            const float2 vv = ld2(reinterpret_cast<const T*>(&vr[i]));
-            put2x(VH, VL, o, vv.x, vv.y);
-          } else {
-            *reinterpret_cast<uint32_t*>(VH + o) = vr[i];
-          }
-        }
+        const float wa = ex2((base.x - gc[i].x) * kLog2e), wb = ex2((base.y - gc[i].y) * kLog2e);
+        if (kV2) put2h(KH, KH + kTile, o, kk.x * wa, kk.y * wb);
+        else put2x(KH, KH + kTile, o, kk.x * wa, kk.y * wb);
       }
       if (kGate && it + 1 < nch) {        // the next chunk's gate tile
         wait_loads(it + 1);
@@ -1539,7 +1542,7 @@ gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
   if (tid == 0) m.waited = waited;
   failed = __syncthreads_or(failed) != 0;
   const int last = m.issued;
-  if (last >= 0 && !mbar_wait(&m.mma, (uint32_t)last & 1u)) failed = true;
+  if (last >= 0 && !mbar_wait(&m.mma[last & 1], (uint32_t)(last >> 1) & 1u)) failed = true;
   tc_after_sync();
   cp_async_wait<0>();
   if (tma && tid == 0)
