@@ -5,15 +5,17 @@
 // chunk outputs with the scores kept on chip and the output gate fused into
 // the epilogue), for 16-bit q/k/v/z, fp32 gates, dk = dv = 64, chunk C = 64.
 //
-// Operands.  Every tensor-core operand is a pair of bf16 tiles (hi, lo) of an
-// fp32 value, hi = bf16(x), lo = bf16(x - hi), multiplied as
-// hi*hi' + hi*lo' + lo*hi' (tcgen05.mma kind::f16 with bf16 inputs, fp32
-// accumulators in tensor memory, M = 64, N = 64 or 128, K = 16 per
-// instruction).  A
-// product carries about 16 significant bits, 32 times finer than a tf32
-// operand, and bf16 has fp32's exponent range, so no operand needs a scale
-// and products of different operands add in one accumulator.  A bf16 V is
-// used as it is (one term); an fp16 V is exactly hi + lo.
+// Operands.  In the output kernel every tensor-core operand is a pair of bf16
+// tiles (hi, lo) of an fp32 value, hi = bf16(x), lo = bf16(x - hi),
+// multiplied as hi*hi' + hi*lo' + lo*hi' (tcgen05.mma kind::f16 with bf16
+// inputs, fp32 accumulators in tensor memory, M = 64, N = 64 or 128, K = 16
+// per instruction).  A product carries about 16 significant bits, 32 times
+// finer than a tf32 operand, and bf16 has fp32's exponent range, so no
+// operand needs a scale and products of different operands add in one
+// accumulator.  A bf16 V is used as it is (one term); an fp16 V is exactly
+// hi + lo.  The summary kernel's key operand is bounded by |k| (its weights
+// are at most one), so there it is a pair of fp16 tiles when the inputs are
+// fp16 (22 significant bits), and v is the second operand as it is.
 //
 // Output kernel (gla_out_tc).  One CTA (256 threads) walks a segment of
 // consecutive chunks of one (batch, head) sequence and carries the state in
