@@ -281,7 +281,7 @@ template <typename TX>
 __global__ void __launch_bounds__(kThreadsAll, 1)
 gate_fwd_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmg,
             const uint8_t* __restrict__ pack, const float* __restrict__ bias, int dm, int HD,
-            float inv_tau, int tpc) {
+            float inv_tau, int tpc, int spb) {
   constexpr bool kBf16 = std::is_same<TX, __nv_bfloat16>::value;
   constexpr int kTerms = kBf16 ? 3 : 2;   // W_down terms in x's type
   extern __shared__ uint8_t smem_raw[];
@@ -293,6 +293,9 @@ gate_fwd_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUt
   Misc& m = *reinterpret_cast<Misc*>(sm + Layout::kOffMisc);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tok0 = blockIdx.x * tpc;
+  // this block's 64-column slabs of g: [j0, j1) (blockIdx.y splits the
+  // columns when there are few token tiles)
+  const int j0 = blockIdx.y * spb, j1 = min(HD / 64, j0 + spb);
 
   if (tid == 0) {
     tc::mbar_init(&m.ld, 1);
@@ -389,7 +392,7 @@ gate_fwd_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUt
   if (tid == 0) {
     const uint32_t id = idesc16(kM, 64, 0, 1, 0);
     const uint64_t al = tc::sdesc(saddr(tLow), 16, 1024), all = tc::sdesc(saddr(tLow) + Layout::kLow, 16, 1024);
-    for (int nb = 0; nb < HD / 64; ++nb) {
+    for (int nb = j0; nb < j1; ++nb) {
       const uint32_t ub = saddr(tWu) + nb * (kRank * 128);
       const uint64_t bh = tc::sdesc(ub, kRank * 128, 1024), bl = tc::sdesc(ub + Layout::kWu, kRank * 128, 1024);
       tc::mma_f16(tm + 64 + nb * 64, al, bh, id, 0u);
@@ -412,17 +415,17 @@ gate_fwd_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUt
   // once they have read the buffer, which the warps wait for before staging
   // the slab three later there.  No block barrier runs between slabs.
   if (ok) {
-    const int nslab = HD / 64;
+    const int nslab = j1 - j0;                    // slabs j0 + l, l < nslab
     if (warp < kThreads / 32) {
       const float ln2_tau = 0.6931471805599453f * inv_tau;
       const int q = warp & 3, qp = warp >> 2;
       const int r = q * 32 + lane;
       const float ri = m.low_i[r];
       const uint32_t tq = tm + ((uint32_t)(q * 32) << 16) + 64 + 16 * qp;
-      auto emit = [&](int j, const float* u) {
-        uint8_t* slab = tX + (j % 3) * (2 * Layout::kHalfSlab);
-        if (j >= 3) ok &= tc::mbar_wait(&m.sfree[j % 3], (uint32_t)((j / 3) - 1) & 1u);
-        const int cb = 64 * j + 16 * qp;
+      auto emit = [&](int l, const float* u) {
+        uint8_t* slab = tX + (l % 3) * (2 * Layout::kHalfSlab);
+        if (l >= 3) ok &= tc::mbar_wait(&m.sfree[l % 3], (uint32_t)((l / 3) - 1) & 1u);
+        const int cb = 64 * (j0 + l) + 16 * qp;
         uint8_t* half = slab + (qp >> 1) * Layout::kHalfSlab + r * 128;
 #pragma unroll
         for (int c = 0; c < 16; c += 4) {
@@ -437,30 +440,30 @@ gate_fwd_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUt
         }
         tc::fence_async_smem();                   // these writes, then the TMA engine's reads
         __syncwarp();
-        if (lane == 0) tc::mbar_arrive_one(&m.sfull[j % 3]);
+        if (lane == 0) tc::mbar_arrive_one(&m.sfull[l % 3]);
       };
       // the next slab's TMEM columns are requested before this one is formed
       float ua[16], ub[16];
-      tmem_ld16(tq, ua);
+      tmem_ld16(tq + 64 * j0, ua);
       for (int j = 0; j < nslab; j += 2) {
         tc::tmem_ld_wait(ua);                     // slab j in ua
-        if (j + 1 < nslab) tmem_ld16(tq + 64 * (j + 1), ub);
+        if (j + 1 < nslab) tmem_ld16(tq + 64 * (j0 + j + 1), ub);
         emit(j, ua);
         if (j + 1 < nslab) {
           tc::tmem_ld_wait(ub);                   // slab j + 1 in ub
-          if (j + 2 < nslab) tmem_ld16(tq + 64 * (j + 2), ua);
+          if (j + 2 < nslab) tmem_ld16(tq + 64 * (j0 + j + 2), ua);
           emit(j + 1, ub);
         }
       }
     } else if (lane == 0) {
-      for (int j = 0; j < nslab; ++j) {
-        uint8_t* slab = tX + (j % 3) * (2 * Layout::kHalfSlab);
-        ok &= tc::mbar_wait(&m.sfull[j % 3], (uint32_t)(j / 3) & 1u);
-        tma_store_2d(&tmg, 64 * j, tok0, slab);
-        tma_store_2d(&tmg, 64 * j + 32, tok0, slab + Layout::kHalfSlab);
+      for (int l = 0; l < nslab; ++l) {
+        uint8_t* slab = tX + (l % 3) * (2 * Layout::kHalfSlab);
+        ok &= tc::mbar_wait(&m.sfull[l % 3], (uint32_t)(l / 3) & 1u);
+        tma_store_2d(&tmg, 64 * (j0 + l), tok0, slab);
+        tma_store_2d(&tmg, 64 * (j0 + l) + 32, tok0, slab + Layout::kHalfSlab);
         bulk_commit();
         bulk_wait_read<0>();
-        tc::mbar_arrive_one(&m.sfree[j % 3]);
+        tc::mbar_arrive_one(&m.sfree[l % 3]);
       }
       bulk_wait<0>();                             // every store done before the block ends
     }
@@ -587,6 +590,23 @@ inline int gate_tc_tile(long long N, int sms) {
   long long t = (N + sms - 1) / (sms > 0 ? sms : 1);
   t = (t + 15) / 16 * 16;
   return (int)(t < 16 ? 16 : t > gate_tc::kM ? gate_tc::kM : t);
+}
+// The forward kernel's grid: (token tiles of *tpc tokens) x (column blocks of
+// *spb 64-column slabs).  A block's epilogue time grows with its slabs, not
+// with its tokens (its warps cover all 128 TMEM lanes), so when the token
+// tiles of 128 times the slabs fit on the SMs, the columns are split too,
+// one slab per block.
+inline void gate_tc_grid(long long N, int HD, int sms, int* tpc, int* spb, long long* rows, int* cols) {
+  const int nslab = HD / 64;
+  if (sms > 0 && (N + gate_tc::kM - 1) / gate_tc::kM * nslab <= sms) {
+    *tpc = gate_tc_tile(N * nslab, sms);        // about N nslab / #SMs tokens per block
+    *spb = 1;
+  } else {
+    *tpc = gate_tc_tile(N, sms);
+    *spb = nslab;
+  }
+  *rows = (N + *tpc - 1) / *tpc;
+  *cols = (nslab + *spb - 1) / *spb;
 }
 
 }  // namespace gtr

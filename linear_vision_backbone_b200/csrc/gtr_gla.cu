@@ -330,8 +330,9 @@ int gate_pack_launch(int x_dtype, const float* w_down, const float* w_up, int dm
 }
 int gate_fwd_packed_launch(int x_dtype, const void* x, const void* pack, const float* bias, float* g,
                            long long N, int dm, int HD, float tau, cudaStream_t st, int dev) {
-  const int tpc = gate_tc_tile(N, sm_count(dev));
-  const long long blocks = (N + tpc - 1) / tpc;
+  int tpc, spb, cols;
+  long long blocks;
+  gate_tc_grid(N, HD, sm_count(dev), &tpc, &spb, &blocks, &cols);
   CUtensorMap tmx, tmg;
   const CUtensorMapDataType xdt =
       x_dtype == GTR_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -345,14 +346,14 @@ int gate_fwd_packed_launch(int x_dtype, const void* x, const void* pack, const f
   static bool done_h[kMaxDevices], done_b[kMaxDevices];
   if (x_dtype == GTR_F16) {
     if (int rc = ensure_smem(gate_tc::gate_fwd_tc<__half>, gate_tc::Layout::kSmem, done_h, dev)) return rc;
-    return launch_pdl(gate_tc::gate_fwd_tc<__half>, dim3((unsigned)blocks), dim3(gate_tc::kThreadsAll),
-                      gate_tc::Layout::kSmem, st, tmx, tmg, (const uint8_t*)pack, bias, dm, HD, inv_tau, tpc)
+    return launch_pdl(gate_tc::gate_fwd_tc<__half>, dim3((unsigned)blocks, (unsigned)cols), dim3(gate_tc::kThreadsAll),
+                      gate_tc::Layout::kSmem, st, tmx, tmg, (const uint8_t*)pack, bias, dm, HD, inv_tau, tpc, spb)
                ? GTR_ERR_CUDA
                : GTR_OK;
   }
   if (int rc = ensure_smem(gate_tc::gate_fwd_tc<__nv_bfloat16>, gate_tc::Layout::kSmem, done_b, dev)) return rc;
-  return launch_pdl(gate_tc::gate_fwd_tc<__nv_bfloat16>, dim3((unsigned)blocks), dim3(gate_tc::kThreadsAll),
-                    gate_tc::Layout::kSmem, st, tmx, tmg, (const uint8_t*)pack, bias, dm, HD, inv_tau, tpc)
+  return launch_pdl(gate_tc::gate_fwd_tc<__nv_bfloat16>, dim3((unsigned)blocks, (unsigned)cols), dim3(gate_tc::kThreadsAll),
+                    gate_tc::Layout::kSmem, st, tmx, tmg, (const uint8_t*)pack, bias, dm, HD, inv_tau, tpc, spb)
              ? GTR_ERR_CUDA
              : GTR_OK;
 }
