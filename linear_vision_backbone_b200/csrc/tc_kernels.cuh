@@ -1563,9 +1563,19 @@ gla_sum_tc(const __grid_constant__ Params p, const __grid_constant__ Maps mp) {
     tmem_ld_wait(dl);
 #pragma unroll
     for (int c = 0; c < 16; ++c) ds[c] += dl[c];
-    float4* dst = reinterpret_cast<float4*>(p.wsS + (((size_t)bh * p.nseg + seg) * kD + row) * kD + cbase);
+    float* dst = p.wsS + (((size_t)bh * p.nseg + seg) * kD + row) * kD + cbase;
+    uint4 w4[4];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) dst[c] = make_float4(ds[4 * c], ds[4 * c + 1], ds[4 * c + 2], ds[4 * c + 3]);
+    for (int c = 0; c < 4; ++c)
+      w4[c] = make_uint4(__float_as_uint(ds[4 * c]), __float_as_uint(ds[4 * c + 1]), __float_as_uint(ds[4 * c + 2]),
+                         __float_as_uint(ds[4 * c + 3]));
+    if (((uintptr_t)p.wsS & 31) == 0) {           // whole 32-byte sectors (the row's 64 bytes)
+      st_global_v8(dst, w4[0], w4[1]);
+      st_global_v8(dst + 8, w4[2], w4[3]);
+    } else {                                      // a caller's states buffer: 16-byte alignment only
+#pragma unroll
+      for (int c = 0; c < 4; ++c) reinterpret_cast<uint4*>(dst)[c] = w4[c];
+    }
     if (warp == 0) {
       const float2 R = *reinterpret_cast<const float2*>(&m.part[0][dc]);
       *reinterpret_cast<float2*>(p.wsA + ((size_t)bh * p.nseg + seg) * kD + dc) = make_float2(expf(R.x), expf(R.y));

@@ -333,6 +333,31 @@ def test_chunk_states_many_segments():
     assert rel < 1e-3, rel
 
 
+def test_chunk_states_into_a_16_byte_aligned_buffer():
+    # the summary kernel writes whole 32-byte sectors when its state buffer
+    # allows it; a caller's buffer that is only 16-byte aligned takes 16-byte stores
+    import ctypes
+    gh, gw = 64, 4
+    B, H = 1, 2
+    d = inputs.make_custom(B, H, gh, gw, 64, 64, "f16", seed=85)
+    k, v, g = _dev(d["k"]), _dev(d["v"]), _dev(d["g"])
+    nc = gh * gw // 64
+    n = B * H * nc * 64 * 64
+    buf = torch.full((n + 8,), 3.0, dtype=torch.float32, device="cuda")
+    view = buf[4:4 + n]                     # 16 bytes past a 256-byte boundary
+    assert view.data_ptr() % 32 == 16
+    rc = binding.load().gtr_gla_chunk_states(
+        ctypes.c_void_p(k.data_ptr()), ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(g.data_ptr()),
+        ctypes.c_void_p(view.data_ptr()), B, H, gh, gw, 64, 64, 2, 64, 1,
+        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert float(buf[:4].sub(3.0).abs().max()) == 0.0 and float(buf[4 + n:].sub(3.0).abs().max()) == 0.0
+    ref = binding.chunk_states(k, v, g, grid_h=gh, grid_w=gw, direction="TB", chunk=64)
+    torch.cuda.synchronize()
+    assert torch.equal(view.view_as(ref), ref)
+
+
 @pytest.mark.parametrize("guard", (4096, 4104))
 def test_output_stays_inside_its_buffer_and_inputs_untouched(guard):
     # guard 4104 fp16 elements: `out` is 16-byte but not 32-byte aligned (the
