@@ -239,6 +239,27 @@ GTR_API gtr_status_t gtr_gla_fwd_gated_timed(const void *x, int x_dtype, const v
                                              int dtype, void *stream, void *const *ev);
 
 /*
+ * The token mixer's projections on either side of the GLA (GTR article
+ * 方法详解 §1: q, k, v and the output gate z are linear maps of the block input
+ * x, and the mixer output is mapped back to the model width).  Plain dense
+ * GEMMs with fp32 accumulation, run by cuBLAS, which the library loads with
+ * dlopen at the first call (GTR_ERR_UNSUPPORTED if it cannot be loaded); make
+ * the first call on a device outside stream capture.  16-bit dtype only
+ * (GTR_F16 or GTR_BF16; GTR_F32 is GTR_ERR_UNSUPPORTED); every pointer a
+ * device pointer, 16-byte aligned, row-major.
+ *   gtr_mixer_in_proj: x [B*T, d_model], w_in [d_model, 2 H dk + 2 H dv] whose
+ *     column blocks are W_q | W_k | W_v | W_z -> q = x W_q, k = x W_k ([B, T, H,
+ *     dk]), v = x W_v, z = x W_z ([B, T, H, dv]), rounded to dtype.
+ *   gtr_mixer_out_proj: out [N, d_out] = y [N, d_in] w_out [d_in, d_out].
+ *   Sizes of zero are an empty problem (GTR_OK, nothing launched).
+ */
+GTR_API gtr_status_t gtr_mixer_in_proj(const void *x, const void *w_in, void *q, void *k, void *v,
+                                       void *z, int B, int T, int d_model, int H, int dk, int dv,
+                                       int dtype, void *stream);
+GTR_API gtr_status_t gtr_mixer_out_proj(const void *y, const void *w_out, void *out, long long N,
+                                        int d_in, int d_out, int dtype, void *stream);
+
+/*
  * Chunk-boundary states, for testing the first two stages on their own: the
  * state each chunk of `chunk` scan positions ends with,
  *   states [B, H, ceil(T/chunk), dk, dv] fp32, entry c = S after scan position

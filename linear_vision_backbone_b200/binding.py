@@ -27,7 +27,8 @@ EXPORTS = (
     "gtr_gla_chunk_states", "gtr_gla_workspace_bytes", "gtr_gla_set_workspace",
     "gtr_gla_set_path", "gtr_gla_path_for", "gtr_last_device_status", "gtr_gla_segment_chunks",
     "gtr_gla_fwd_noalloc", "gtr_gate_packed_bytes", "gtr_gate_pack", "gtr_gate_fwd_packed",
-    "gtr_gla_segment_count", "gtr_gla_fwd_gated", "gtr_gla_fwd_gated_timed",
+    "gtr_gla_segment_count", "gtr_gla_fwd_gated", "gtr_gla_fwd_gated_timed", "gtr_mixer_in_proj",
+    "gtr_mixer_out_proj",
 )
 
 _lock = threading.Lock()
@@ -74,6 +75,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                    I, I, I, I, I, I, I, I, I, P], I),
             "gtr_gla_fwd_gated_timed": ([P, I, P, P, I, I, F, P, P, P, P, P, P, P,
                                          I, I, I, I, I, I, I, I, I, P, P], I),
+            "gtr_mixer_in_proj": ([P, P, P, P, P, P, I, I, I, I, I, I, I, P], I),
+            "gtr_mixer_out_proj": ([P, P, P, ctypes.c_longlong, I, I, I, P], I),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -242,6 +245,44 @@ def gla_fwd_gated(x, packed, bias, q, k, v, z, w=None, *, tau: float, grid_h: in
         arr = (ctypes.c_void_p * 5)(*[None if e is None else e.cuda_event for e in events])
         _check("gtr_gla_fwd_gated_timed", lib.gtr_gla_fwd_gated_timed(*args, arr))
     return out, g_out
+
+
+def mixer_in_proj(x, w_in, H: int, dk: int, dv: Optional[int] = None, stream=None):
+    """q, k, v, z = x W_q, x W_k, x W_v, x W_z (``gtr_mixer_in_proj``).
+
+    x: [B, T, d_model] 16-bit; w_in: [d_model, 2 H dk + 2 H dv] of x's dtype,
+    column blocks W_q | W_k | W_v | W_z.  Returns q, k [B, T, H, dk] and v, z
+    [B, T, H, dv] in x's dtype."""
+    dv = dk if dv is None else dv
+    _need(x, "x")
+    if x.dim() != 3:
+        raise ValueError("x must be [B, T, d_model]")
+    B, T, dm = x.shape
+    _need(w_in, "w_in", x.dtype, (dm, 2 * H * dk + 2 * H * dv))
+    q = torch.empty(B, T, H, dk, device=x.device, dtype=x.dtype)
+    k = torch.empty_like(q)
+    v = torch.empty(B, T, H, dv, device=x.device, dtype=x.dtype)
+    z = torch.empty_like(v)
+    rc = load().gtr_mixer_in_proj(_ptr(x), _ptr(w_in), _ptr(q), _ptr(k), _ptr(v), _ptr(z), B, T, dm, H, dk,
+                                  dv, DTYPE_IDS[x.dtype], _stream(stream))
+    _check("gtr_mixer_in_proj", rc)
+    return q, k, v, z
+
+
+def mixer_out_proj(y, w_out, stream=None):
+    """out = y w_out (``gtr_mixer_out_proj``): y [..., d_in], w_out [d_in, d_out], one 16-bit dtype."""
+    _need(y, "y")
+    d_in = y.shape[-1]
+    _need(w_out, "w_out", y.dtype)
+    if w_out.dim() != 2 or w_out.shape[0] != d_in:
+        raise ValueError(f"w_out must be [{d_in}, d_out]")
+    d_out = w_out.shape[1]
+    out = torch.empty(*y.shape[:-1], d_out, device=y.device, dtype=y.dtype)
+    N = y.numel() // d_in if d_in else 0
+    rc = load().gtr_mixer_out_proj(_ptr(y), _ptr(w_out), _ptr(out), N, d_in, d_out, DTYPE_IDS[y.dtype],
+                                   _stream(stream))
+    _check("gtr_mixer_out_proj", rc)
+    return out
 
 
 def gla_fwd_noalloc(q, k, v, g, z, w=None, *, grid_h: int, grid_w: int, direction: str = "LR",

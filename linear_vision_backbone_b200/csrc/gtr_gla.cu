@@ -15,6 +15,7 @@
 #include "scan_kernel.cuh"
 #include "tc_kernels.cuh"
 #include "gate_tc.cuh"
+#include "mixer_proj.cuh"
 
 namespace {
 
@@ -805,6 +806,52 @@ gtr_status_t gtr_gla_fwd_gated_timed(const void* x, int x_dtype, const void* pac
   return (gtr_status_t)gla_fwd_gated_impl(x, x_dtype, packed, bias, d_model, rank, tau, q, k, v, outgate,
                                           rms_w, g_out, out, B, H, grid_h, grid_w, dk, dv, dir, chunk,
                                           dtype, stream, ev);
+}
+
+gtr_status_t gtr_mixer_in_proj(const void* x, const void* w_in, void* q, void* k, void* v, void* z, int B, int T,
+                               int d_model, int H, int dk, int dv, int dtype, void* stream) {
+  if (B < 0 || T < 0 || H < 0 || dk < 0 || dv < 0 || d_model < 0) return GTR_ERR_INVALID_ARG;
+  if (dtype < 0 || dtype > 2) return GTR_ERR_INVALID_ARG;
+  const long long N = (long long)B * T, n_q = (long long)H * dk, n_v = (long long)H * dv;
+  if (N == 0 || n_q + n_v == 0 || d_model == 0) return GTR_OK;
+  if (dtype == GTR_F32) return GTR_ERR_UNSUPPORTED;
+  if (N >= (1LL << 31) || 2 * (n_q + n_v) >= (1LL << 31)) return GTR_ERR_INVALID_ARG;
+  if (!x || !w_in || !q || !k || !v || !z) return GTR_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_in) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(z))
+    return GTR_ERR_ALIGNMENT;
+  int dev;
+  if (int rc = current_device(&dev)) return (gtr_status_t)rc;
+  const cudaDataType dt = dtype == GTR_F16 ? CUDA_R_16F : CUDA_R_16BF;
+  const int ldw = (int)(2 * (n_q + n_v));
+  const char* W = (const char*)w_in;
+  cudaStream_t st = (cudaStream_t)stream;
+  // column blocks of W: q | k | v | z
+  const long long off[4] = {0, n_q, 2 * n_q, 2 * n_q + n_v};
+  const long long width[4] = {n_q, n_q, n_v, n_v};
+  void* outs[4] = {q, k, v, z};
+  for (int i = 0; i < 4; ++i) {
+    if (width[i] == 0) continue;
+    if (int rc = blas_gemm_rowmajor(dev, st, dt, x, d_model, W + off[i] * 2, ldw, outs[i], (int)width[i], (int)N,
+                                    d_model, (int)width[i]))
+      return (gtr_status_t)rc;
+  }
+  return GTR_OK;
+}
+
+gtr_status_t gtr_mixer_out_proj(const void* y, const void* w_out, void* out, long long N, int d_in, int d_out,
+                                int dtype, void* stream) {
+  if (N < 0 || d_in < 0 || d_out < 0) return GTR_ERR_INVALID_ARG;
+  if (dtype < 0 || dtype > 2) return GTR_ERR_INVALID_ARG;
+  if (N == 0 || d_in == 0 || d_out == 0) return GTR_OK;
+  if (dtype == GTR_F32) return GTR_ERR_UNSUPPORTED;
+  if (N >= (1LL << 31)) return GTR_ERR_INVALID_ARG;
+  if (!y || !w_out || !out) return GTR_ERR_INVALID_ARG;
+  if (!aligned16(y) || !aligned16(w_out) || !aligned16(out)) return GTR_ERR_ALIGNMENT;
+  int dev;
+  if (int rc = current_device(&dev)) return (gtr_status_t)rc;
+  const cudaDataType dt = dtype == GTR_F16 ? CUDA_R_16F : CUDA_R_16BF;
+  return (gtr_status_t)blas_gemm_rowmajor(dev, (cudaStream_t)stream, dt, y, d_in, w_out, d_out, out, d_out, (int)N,
+                                          d_in, d_out);
 }
 
 gtr_status_t gtr_gla_chunk_states(const void* k, const void* v, const float* g, float* states,

@@ -1,0 +1,78 @@
+// mixer_proj.cuh -- the token mixer's input and output projections, the steps
+// on either side of the GLA (GTR article, 方法详解 §1: q, k, v and the output
+// gate z are linear maps of the block input x; the mixer's output is mapped
+// back to the model width).  Both are plain dense GEMMs,
+//     C[N, n] = X[N, K] W[K, n]        (X, W, C row-major, one 16-bit type),
+// run by cuBLAS with fp32 accumulation.  cuBLAS is loaded with dlopen at the
+// first call, so the rest of the library neither links nor needs it.
+#pragma once
+#include <dlfcn.h>
+
+#include <mutex>
+
+#include <cublas_v2.h>
+
+namespace gtr {
+
+using BlasCreateFn = cublasStatus_t (*)(cublasHandle_t*);
+using BlasSetStreamFn = cublasStatus_t (*)(cublasHandle_t, cudaStream_t);
+using BlasGemmExFn = cublasStatus_t (*)(cublasHandle_t, cublasOperation_t, cublasOperation_t, int, int, int,
+                                        const void*, const void*, cudaDataType, int, const void*, cudaDataType,
+                                        int, const void*, void*, cudaDataType, int, cublasComputeType_t,
+                                        cublasGemmAlgo_t);
+struct BlasApi {
+  bool tried = false;
+  void* lib = nullptr;
+  BlasCreateFn create = nullptr;
+  BlasSetStreamFn set_stream = nullptr;
+  BlasGemmExFn gemm = nullptr;
+  cublasHandle_t handle[64] = {};
+};
+
+inline BlasApi& blas_api() {
+  static BlasApi api;
+  return api;
+}
+inline std::mutex& blas_mutex() {
+  static std::mutex mu;
+  return mu;
+}
+
+// The cuBLAS entry points, loaded once; false when the library is missing.
+inline bool blas_load(BlasApi& a) {
+  if (a.tried) return a.gemm != nullptr;
+  a.tried = true;
+  for (const char* name : {"libcublas.so.12", "libcublas.so"}) {
+    a.lib = dlopen(name, RTLD_NOW | RTLD_LOCAL);
+    if (a.lib) break;
+  }
+  if (!a.lib) return false;
+  a.create = (BlasCreateFn)dlsym(a.lib, "cublasCreate_v2");
+  a.set_stream = (BlasSetStreamFn)dlsym(a.lib, "cublasSetStream_v2");
+  a.gemm = (BlasGemmExFn)dlsym(a.lib, "cublasGemmEx");
+  if (!a.create || !a.set_stream || !a.gemm) a.gemm = nullptr;
+  return a.gemm != nullptr;
+}
+
+// C[N, n] = X[N, K] W[K, n] on `st`: X with row stride ldx, W with row stride
+// ldw (a column block of a wider weight matrix), C with row stride ldc, all
+// 16-bit of type `dt` (CUDA_R_16F / CUDA_R_16BF), fp32 accumulation.  In
+// cuBLAS's column-major terms this is C^T = W^T X^T.  Returns a gtr status.
+inline int blas_gemm_rowmajor(int dev, cudaStream_t st, cudaDataType dt, const void* X, int ldx, const void* W,
+                              int ldw, void* C, int ldc, int N, int K, int n) {
+  std::lock_guard<std::mutex> lk(blas_mutex());
+  BlasApi& a = blas_api();
+  if (!blas_load(a)) return -2;   // GTR_ERR_UNSUPPORTED
+  if (dev < 0 || dev >= 64) return -2;
+  if (!a.handle[dev] && a.create(&a.handle[dev]) != CUBLAS_STATUS_SUCCESS) {
+    a.handle[dev] = nullptr;
+    return -5;                    // GTR_ERR_CUDA
+  }
+  if (a.set_stream(a.handle[dev], st) != CUBLAS_STATUS_SUCCESS) return -5;
+  const float one = 1.0f, zero = 0.0f;
+  const cublasStatus_t r = a.gemm(a.handle[dev], CUBLAS_OP_N, CUBLAS_OP_N, n, N, K, &one, W, dt, ldw, X, dt, ldx,
+                                  &zero, C, dt, ldc, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
+  return r == CUBLAS_STATUS_SUCCESS ? 0 : -5;
+}
+
+}  // namespace gtr

@@ -143,6 +143,13 @@ def gla_fwd(q, k, v, g, z, w=None, *, gh: int, gw: int, direction: str = "LR",
     return (y, o) if return_o else y
 
 
+def linear(x, w) -> np.ndarray:
+    """x W in fp64 (the token mixer's projections, GTR article 方法详解 §1):
+    x [..., K], w [K, n] -> [..., n].  A plain matrix product."""
+    x64, w64 = _f64(x), _f64(w)
+    return np.matmul(x64, w64)
+
+
 def chunk_states(k, v, g, *, gh: int, gw: int, direction: str = "LR", chunk: int = 64) -> np.ndarray:
     """State after each chunk of ``chunk`` scan positions: [B, H, ceil(T/chunk), dk, dv]."""
     k, v, g = (_f64(a) for a in (k, v, g))

@@ -121,3 +121,21 @@ def test_gated_call_rejects_invalid_arguments_before_any_launch(lib):
     assert call(g=None) == -1
     assert call(x=ctypes.c_void_p(24)) == -3        # 16-byte alignment
     assert call(g=ctypes.c_void_p(40)) == -3
+
+
+def test_mixer_projections_reject_invalid_arguments(lib):
+    P = ctypes.c_void_p(16)
+    S = None
+    # in-projection: negative sizes, bad dtype, fp32 unsupported, empty, nulls, alignment
+    assert lib.gtr_mixer_in_proj(P, P, P, P, P, P, -1, 4, 384, 6, 64, 64, 1, S) == -1
+    assert lib.gtr_mixer_in_proj(P, P, P, P, P, P, 1, 4, 384, 6, 64, 64, 3, S) == -1
+    assert lib.gtr_mixer_in_proj(P, P, P, P, P, P, 1, 4, 384, 6, 64, 64, 0, S) == -2
+    assert lib.gtr_mixer_in_proj(None, None, None, None, None, None, 0, 4, 384, 6, 64, 64, 1, S) == 0
+    assert lib.gtr_mixer_in_proj(P, None, P, P, P, P, 1, 4, 384, 6, 64, 64, 1, S) == -1
+    assert lib.gtr_mixer_in_proj(ctypes.c_void_p(24), P, P, P, P, P, 1, 4, 384, 6, 64, 64, 1, S) == -3
+    # out-projection
+    assert lib.gtr_mixer_out_proj(P, P, P, -1, 384, 384, 1, S) == -1
+    assert lib.gtr_mixer_out_proj(P, P, P, 4, 384, 384, 0, S) == -2
+    assert lib.gtr_mixer_out_proj(None, None, None, 0, 384, 384, 1, S) == 0
+    assert lib.gtr_mixer_out_proj(P, P, None, 4, 384, 384, 1, S) == -1
+    assert lib.gtr_mixer_out_proj(P, ctypes.c_void_p(40), P, 4, 384, 384, 2, S) == -3

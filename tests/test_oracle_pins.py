@@ -314,3 +314,17 @@ def test_oracle_reproduces_its_stored_tiny_output():
     y = oracle.gla_fwd(d["q"], d["k"], d["v"], d["g"], d["z"], d["w"], gh=wl.gh, gw=wl.gw)
     stored = np.array([float.fromhex(v) for v in doc["y"]]).reshape(doc["shape"])
     np.testing.assert_allclose(y, stored, rtol=1e-13, atol=1e-15)
+
+
+def test_linear_is_the_matrix_product():
+    # the projections' oracle against the definition of the product, summed term by term
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((3, 4, 5))
+    w = rng.standard_normal((5, 7))
+    got = oracle.linear(x, w)
+    ref = np.zeros((3, 4, 7))
+    for a in range(3):
+        for b in range(4):
+            for j in range(7):
+                ref[a, b, j] = sum(x[a, b, i] * w[i, j] for i in range(5))
+    np.testing.assert_allclose(got, ref, rtol=1e-13, atol=1e-13)
