@@ -466,8 +466,10 @@ def run_ours(args, world, rank, local):
     e2e_value = aggregate_value(units, args.e2e_steps, e2e_ms, world)
 
     secondary = None
+    mixer = None
     if not args.no_secondary and args.workload == "16k":
         secondary = secondary_line(binding, dev)
+        mixer = mixer_line(binding, dev, wl, host)
 
     if rank == 0:
         cpu = oracle_rate(wl, seconds=10.0)
@@ -501,6 +503,8 @@ def run_ours(args, world, rank, local):
         }
         if secondary is not None:
             line["secondary"] = secondary
+        if mixer is not None:
+            line["mixer"] = mixer
         print(json.dumps(line), flush=True)
 
     graphs.clear()
@@ -556,6 +560,80 @@ def make_step(binding, wl, params, x_dtype, chunk, stream, fused=False):
                         grid_w=wl.gw, direction=direction, chunk=chunk, out=s["out"],
                         stream=stream, events=None if evs is None else evs[1:])
     return step, False
+
+
+def mixer_line(binding, dev, wl, host, steps=200):
+    """The token mixer around the timed step (the next row of the hot path):
+    the input projection x -> q, k, v, z and the output projection y W_o as
+    cuBLAS GEMMs (16-bit, fp32 accumulation, random weights of the workload's
+    shapes), each timed alone on graphs, and the whole mixer step (input
+    projection, gate, GLA, output projection).  Tensor-bound: FLOP/s against
+    the measured bf16 GEMM peak."""
+    dt = host["q"].dtype
+    H, dk, dm = wl.H, wl.dk, wl.d_model
+    gen = torch.Generator().manual_seed(7)
+    w_in = (torch.randn(dm, 4 * H * dk, generator=gen) / dm ** 0.5).to(dt).to(dev)
+    w_o = (torch.randn(H * dk, dm, generator=gen) / (H * dk) ** 0.5).to(dt).to(dev)
+    x = host["x"].to(dev)
+    params = {n: host[n].to(dev) for n in ("w_down", "w_up", "bias", "w")}
+    stream = torch.cuda.Stream(device=dev)
+    step, _ = make_step(binding, wl, params, x.dtype, 64, stream)
+    buf = {}
+
+    def in_proj():
+        buf["q"], buf["k"], buf["v"], buf["z"] = binding.mixer_in_proj(x, w_in, H, dk, stream=stream)
+
+    def out_proj():
+        buf["o"] = binding.mixer_out_proj(buf["y"], w_o, stream=stream)
+
+    def whole():
+        in_proj()
+        s = {"x": x, "q": buf["q"], "k": buf["k"], "v": buf["v"], "z": buf["z"], "g": buf["g"],
+             "out": buf["out"]}
+        step(s, wl.dirs[0])
+        buf["y"] = buf["out"].reshape(wl.B, wl.T, H * dk)
+        out_proj()
+
+    with torch.cuda.stream(stream):
+        in_proj()
+        buf["g"] = torch.empty(wl.B, wl.T, H, dk, device=dev)
+        buf["out"] = torch.empty_like(buf["v"])
+        buf["y"] = buf["out"].reshape(wl.B, wl.T, H * dk)
+        out_proj()
+        whole()
+    stream.synchronize()
+
+    def time_graph(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            for _ in range(10):
+                g.replay()
+            a.record(stream)
+            for _ in range(steps):
+                g.replay()
+            b.record(stream)
+        stream.synchronize()
+        return a.elapsed_time(b) / steps
+
+    ms_in, ms_out, ms_all = time_graph(in_proj), time_graph(out_proj), time_graph(whole)
+    n_tok = wl.B * wl.T
+    fl_in, fl_out = 2.0 * n_tok * dm * 4 * H * dk, 2.0 * n_tok * H * dk * dm
+    try:
+        peak = float(json.load(open(PEAKS_FILE))["bf16_tflops"])
+        kind = "measured"
+    except (OSError, KeyError, ValueError):
+        peak, kind = 1590.0, "fallback"
+    return {"workload": workload_text(wl), "gemm": "cuBLAS (cublasGemmEx, fp32 accumulation)",
+            "in_proj": {"ms": ms_in, "tflops": fl_in / (ms_in * 1e-3) / 1e12,
+                        "frac": fl_in / (ms_in * 1e-3) / 1e12 / peak},
+            "out_proj": {"ms": ms_out, "tflops": fl_out / (ms_out * 1e-3) / 1e12,
+                         "frac": fl_out / (ms_out * 1e-3) / 1e12 / peak},
+            "peak_tflops": peak, "peak_kind": kind,
+            "mixer_step_ms": ms_all, "mixer_token_heads_per_s": wl.token_heads / (ms_all * 1e-3),
+            "l2": "warm (one input set; weights and activations fit L2 at 16k only partly)"}
 
 
 def secondary_line(binding, dev, steps=2000):
