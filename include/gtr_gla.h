@@ -249,7 +249,9 @@ GTR_API gtr_status_t gtr_gla_fwd_gated_timed(const void *x, int x_dtype, const v
  * device pointer, 16-byte aligned, row-major.
  *   gtr_mixer_in_proj: x [B*T, d_model], w_in [d_model, 2 H dk + 2 H dv] whose
  *     column blocks are W_q | W_k | W_v | W_z -> q = x W_q, k = x W_k ([B, T, H,
- *     dk]), v = x W_v, z = x W_z ([B, T, H, dv]), rounded to dtype.
+ *     dk]), v = x W_v, z = x W_z ([B, T, H, dv]), rounded to dtype.  When dk ==
+ *     dv and q, k, v, z lie at equal, non-overlapping distances in memory (one
+ *     [4, B, T, H, dk] buffer) the four products are one batched call.
  *   gtr_mixer_out_proj: out [N, d_out] = y [N, d_in] w_out [d_in, d_out].
  *   Sizes of zero are an empty problem (GTR_OK, nothing launched).
  */

@@ -259,10 +259,13 @@ def mixer_in_proj(x, w_in, H: int, dk: int, dv: Optional[int] = None, stream=Non
         raise ValueError("x must be [B, T, d_model]")
     B, T, dm = x.shape
     _need(w_in, "w_in", x.dtype, (dm, 2 * H * dk + 2 * H * dv))
-    q = torch.empty(B, T, H, dk, device=x.device, dtype=x.dtype)
-    k = torch.empty_like(q)
-    v = torch.empty(B, T, H, dv, device=x.device, dtype=x.dtype)
-    z = torch.empty_like(v)
+    if dv == dk:   # one buffer: the four outputs equally spaced (one batched product)
+        q, k, v, z = torch.empty(4, B, T, H, dk, device=x.device, dtype=x.dtype).unbind(0)
+    else:
+        q = torch.empty(B, T, H, dk, device=x.device, dtype=x.dtype)
+        k = torch.empty_like(q)
+        v = torch.empty(B, T, H, dv, device=x.device, dtype=x.dtype)
+        z = torch.empty_like(v)
     rc = load().gtr_mixer_in_proj(_ptr(x), _ptr(w_in), _ptr(q), _ptr(k), _ptr(v), _ptr(z), B, T, dm, H, dk,
                                   dv, DTYPE_IDS[x.dtype], _stream(stream))
     _check("gtr_mixer_in_proj", rc)

@@ -825,7 +825,13 @@ gtr_status_t gtr_mixer_in_proj(const void* x, const void* w_in, void* q, void* k
   const int ldw = (int)(2 * (n_q + n_v));
   const char* W = (const char*)w_in;
   cudaStream_t st = (cudaStream_t)stream;
-  // column blocks of W: q | k | v | z
+  // column blocks of W: q | k | v | z.  Four equal blocks whose outputs lie
+  // equally spaced in memory go out as one strided-batched product.
+  const long long gap = (const char*)k - (const char*)q;
+  if (n_q == n_v && gap > 0 && gap % 2 == 0 && (const char*)v - (const char*)k == gap &&
+      (const char*)z - (const char*)v == gap && gap >= N * n_q * 2)
+    return (gtr_status_t)blas_gemm_rowmajor(dev, st, dt, x, d_model, W, ldw, q, (int)n_q, (int)N, d_model,
+                                            (int)n_q, 4, n_q, gap / 2);
   const long long off[4] = {0, n_q, 2 * n_q, 2 * n_q + n_v};
   const long long width[4] = {n_q, n_q, n_v, n_v};
   void* outs[4] = {q, k, v, z};

@@ -20,12 +20,17 @@ using BlasGemmExFn = cublasStatus_t (*)(cublasHandle_t, cublasOperation_t, cubla
                                         const void*, const void*, cudaDataType, int, const void*, cudaDataType,
                                         int, const void*, void*, cudaDataType, int, cublasComputeType_t,
                                         cublasGemmAlgo_t);
+using BlasGemmBatchFn = cublasStatus_t (*)(cublasHandle_t, cublasOperation_t, cublasOperation_t, int, int, int,
+                                            const void*, const void*, cudaDataType, int, long long, const void*,
+                                            cudaDataType, int, long long, const void*, void*, cudaDataType, int,
+                                            long long, int, cublasComputeType_t, cublasGemmAlgo_t);
 struct BlasApi {
   bool tried = false;
   void* lib = nullptr;
   BlasCreateFn create = nullptr;
   BlasSetStreamFn set_stream = nullptr;
   BlasGemmExFn gemm = nullptr;
+  BlasGemmBatchFn gemm_batch = nullptr;
   cublasHandle_t handle[64] = {};
 };
 
@@ -50,16 +55,20 @@ inline bool blas_load(BlasApi& a) {
   a.create = (BlasCreateFn)dlsym(a.lib, "cublasCreate_v2");
   a.set_stream = (BlasSetStreamFn)dlsym(a.lib, "cublasSetStream_v2");
   a.gemm = (BlasGemmExFn)dlsym(a.lib, "cublasGemmEx");
-  if (!a.create || !a.set_stream || !a.gemm) a.gemm = nullptr;
+  a.gemm_batch = (BlasGemmBatchFn)dlsym(a.lib, "cublasGemmStridedBatchedEx");
+  if (!a.create || !a.set_stream || !a.gemm || !a.gemm_batch) a.gemm = nullptr;
   return a.gemm != nullptr;
 }
 
 // C[N, n] = X[N, K] W[K, n] on `st`: X with row stride ldx, W with row stride
 // ldw (a column block of a wider weight matrix), C with row stride ldc, all
 // 16-bit of type `dt` (CUDA_R_16F / CUDA_R_16BF), fp32 accumulation.  In
-// cuBLAS's column-major terms this is C^T = W^T X^T.  Returns a gtr status.
+// cuBLAS's column-major terms this is C^T = W^T X^T.  With batch > 1, `batch`
+// such products with the same X, W and C advanced by w_step and c_step
+// elements (one strided-batched call).  Returns a gtr status.
 inline int blas_gemm_rowmajor(int dev, cudaStream_t st, cudaDataType dt, const void* X, int ldx, const void* W,
-                              int ldw, void* C, int ldc, int N, int K, int n) {
+                              int ldw, void* C, int ldc, int N, int K, int n, int batch = 1, long long w_step = 0,
+                              long long c_step = 0) {
   std::lock_guard<std::mutex> lk(blas_mutex());
   BlasApi& a = blas_api();
   if (!blas_load(a)) return -2;   // GTR_ERR_UNSUPPORTED
@@ -70,8 +79,11 @@ inline int blas_gemm_rowmajor(int dev, cudaStream_t st, cudaDataType dt, const v
   }
   if (a.set_stream(a.handle[dev], st) != CUBLAS_STATUS_SUCCESS) return -5;
   const float one = 1.0f, zero = 0.0f;
-  const cublasStatus_t r = a.gemm(a.handle[dev], CUBLAS_OP_N, CUBLAS_OP_N, n, N, K, &one, W, dt, ldw, X, dt, ldx,
-                                  &zero, C, dt, ldc, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
+  const cublasStatus_t r =
+      batch == 1 ? a.gemm(a.handle[dev], CUBLAS_OP_N, CUBLAS_OP_N, n, N, K, &one, W, dt, ldw, X, dt, ldx, &zero, C,
+                          dt, ldc, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT)
+                 : a.gemm_batch(a.handle[dev], CUBLAS_OP_N, CUBLAS_OP_N, n, N, K, &one, W, dt, ldw, w_step, X, dt,
+                                ldx, 0, &zero, C, dt, ldc, c_step, batch, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
   return r == CUBLAS_STATUS_SUCCESS ? 0 : -5;
 }
 
