@@ -386,6 +386,36 @@ def test_output_stays_inside_its_buffer_and_inputs_untouched(guard):
         assert_close(out, ref, torch.float16, path)
 
 
+def test_registered_workspace_too_small_then_large_enough():
+    # a caller-registered workspace that is too small is reported (no launch, status -4)
+    # and one of exactly gtr_gla_workspace_bytes serves the call; releasing it returns
+    # the library to its own buffers
+    gh, gw = 40, 40
+    d = inputs.make_custom(1, 6, gh, gw, 64, 64, "f16", seed=97)
+    dv = {k: _dev(v) for k, v in d.items()}
+    args = (dv["q"], dv["k"], dv["v"], dv["g"], dv["z"], dv["w"])
+    ref = binding.gla_fwd(*args, grid_h=gh, grid_w=gw, direction="TB")
+    need = binding.workspace_bytes(1, 6, gh, gw, 64, 64, 64, torch.float16)
+    assert need > 256
+    small = torch.empty(256, dtype=torch.uint8, device="cuda")
+    exact = torch.empty(need, dtype=torch.uint8, device="cuda")
+    try:
+        binding.set_workspace(small)
+        with pytest.raises(binding.GtrError) as ei:
+            binding.gla_fwd(*args, grid_h=gh, grid_w=gw, direction="TB")
+        assert ei.value.status == -4
+        binding.set_workspace(exact)
+        y = binding.gla_fwd(*args, grid_h=gh, grid_w=gw, direction="TB")
+        torch.cuda.synchronize()
+    finally:
+        binding.set_workspace(None)
+    assert torch.equal(y, ref)
+    y2 = binding.gla_fwd(*args, grid_h=gh, grid_w=gw, direction="TB")
+    torch.cuda.synchronize()
+    assert torch.equal(y2, ref)
+    _check_status()
+
+
 def test_empty_problem_and_argument_errors():
     e = torch.empty(0, 40 * 40, 6, 64, dtype=torch.float16, device="cuda")
     g = torch.empty(0, 40 * 40, 6, 64, dtype=torch.float32, device="cuda")
