@@ -622,7 +622,8 @@ def mixer_line(binding, dev, wl, host, steps=200):
     n_tok = wl.B * wl.T
     fl_in, fl_out = 2.0 * n_tok * dm * 4 * H * dk, 2.0 * n_tok * H * dk * dm
     try:
-        peak = float(json.load(open(PEAKS_FILE))["bf16_tflops"])
+        with open(PEAKS_FILE) as f:
+            peak = float(json.load(f)["bf16_tflops"])
         kind = "measured"
     except (OSError, KeyError, ValueError):
         peak, kind = 1590.0, "fallback"

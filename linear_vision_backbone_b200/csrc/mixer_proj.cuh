@@ -24,6 +24,8 @@ using BlasGemmBatchFn = cublasStatus_t (*)(cublasHandle_t, cublasOperation_t, cu
                                             const void*, const void*, cudaDataType, int, long long, const void*,
                                             cudaDataType, int, long long, const void*, void*, cudaDataType, int,
                                             long long, int, cublasComputeType_t, cublasGemmAlgo_t);
+// One cuBLAS handle per device, created at its first projection call and kept
+// for the life of the process (the library has no teardown entry point).
 struct BlasApi {
   bool tried = false;
   void* lib = nullptr;
