@@ -17,11 +17,17 @@ Functions (each cites the page passage it follows in ``gla_oracle.c``):
 * :func:`chunk_states` -- the state after every chunk of scan positions (GTR
   article, 方法详解 §4, the boundary states of the chunkwise operator).
 * :func:`scan_index` -- the grid index visited at a scan position.
+* :func:`linear` -- the token mixer's projections, a plain matrix product.
+* :func:`dwconv2d`, :func:`sswiglu_mix`, :func:`sswiglu` -- the Spatial SwiGLU
+  feed-forward block: SiLU(gate) times the depthwise-convolved value branch on
+  the token grid, between two projections (GTR article, 方法详解 §2), in
+  numpy fp64.
 
 Pins: every function here is checked in ``tests/test_oracle_pins.py`` against
 results fixed independently of it (the quadratic masked form, plain causal
 linear attention at g = 0, the memoryless limit, T = 1, explicit grid flips and
-transposes, closed forms of the gate).
+transposes, closed forms of the gate, scipy's 2-D correlation and brute-force
+loops for the depthwise convolution).
 """
 from __future__ import annotations
 
@@ -162,3 +168,57 @@ def chunk_states(k, v, g, *, gh: int, gw: int, direction: str = "LR", chunk: int
     if rc != 0:
         raise ValueError(f"oracle_gla_chunk_states_f64 rejected its arguments (rc={rc})")
     return st
+
+
+def silu(a) -> np.ndarray:
+    """SiLU(a) = a * sigmoid(a) in fp64, written so that neither branch overflows."""
+    a = _f64(a)
+    e = np.exp(-np.abs(a))
+    return np.where(a >= 0, a / (1.0 + e), a * e / (1.0 + e))
+
+
+def dwconv2d(val, weight, bias=None, *, gh: int, gw: int) -> np.ndarray:
+    """Depthwise 2-D cross-correlation of a channels-last token grid, fp64.
+
+    val [B, gh*gw, C] (token t = row * gw + column), weight [k, k, C] (odd k),
+    bias [C] or None -> [B, gh*gw, C] with
+        out[b, y, x, c] = bias[c] + sum_{i,j} weight[i, j, c] * val[b, y+i-r, x+j-r, c],
+    r = k // 2, and val = 0 outside the grid ("same" size, zero padding).  This
+    is the local mixing of the S-SwiGLU value branch after it is laid out as the
+    2-D token grid (GTR article, 方法详解 §2, Spatial SwiGLU).  Written as the k*k
+    shifted copies of the zero-padded grid, summed tap by tap."""
+    v = _f64(val)
+    w = _f64(weight)
+    B, T, C = v.shape
+    k = w.shape[0]
+    if T != gh * gw or w.shape != (k, k, C) or k % 2 != 1:
+        raise ValueError("dwconv2d: shapes")
+    r = k // 2
+    grid = v.reshape(B, gh, gw, C)
+    pad = np.zeros((B, gh + 2 * r, gw + 2 * r, C))
+    pad[:, r:r + gh, r:r + gw] = grid
+    out = np.zeros((B, gh, gw, C))
+    for i in range(k):
+        for j in range(k):
+            out += w[i, j] * pad[:, i:i + gh, j:j + gw]
+    if bias is not None:
+        out += _f64(bias)
+    return out.reshape(B, T, C)
+
+
+def sswiglu_mix(u, weight, bias=None, *, gh: int, gw: int) -> np.ndarray:
+    """The S-SwiGLU hidden activation from the expanded tokens, fp64 (GTR
+    article, 方法详解 §2): u [B, T, 2C] holds the gate branch in its first C
+    channels and the value branch in the last C; the value branch is mixed on
+    the token grid by the depthwise convolution and multiplied by SiLU of the
+    gate branch: h = SiLU(u_gate) * dwconv2d(u_value) -> [B, T, C]."""
+    u = _f64(u)
+    C = u.shape[-1] // 2
+    return silu(u[..., :C]) * dwconv2d(u[..., C:], weight, bias, gh=gh, gw=gw)
+
+
+def sswiglu(x, w_in, weight, bias, w_out, *, gh: int, gw: int) -> np.ndarray:
+    """The S-SwiGLU feed-forward block in fp64 (GTR article, 方法详解 §2): the
+    expansion x W_in -> [gate | value], the grid-mixed gated product h, and the
+    projection back h W_out.  x [B, T, Cm], w_in [Cm, 2C], w_out [C, Cm]."""
+    return linear(sswiglu_mix(linear(x, w_in), weight, bias, gh=gh, gw=gw), w_out)
