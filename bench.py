@@ -183,13 +183,18 @@ def read_traffic(kernel_name: str, src_hash: str):
 
 
 def kernel_source_hash():
-    """Hash of the CUDA sources with comments and blank space removed, so that
-    a figure measured on a kernel stays attached to it through comment edits."""
+    """Hash of the CUDA sources the gate + GLA step is compiled from (the
+    translation unit gtr_gla.cu and the headers beside it; another .cu file is
+    its own translation unit and cannot change these kernels), with comments and
+    blank space removed, so that a figure measured on a kernel stays attached
+    to it through comment edits."""
     import hashlib
     import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "linear_vision_backbone_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
+        if name.endswith(".cu") and name != "gtr_gla.cu":
+            continue
         with open(os.path.join(csrc, name), encoding="utf-8") as f:
             text = f.read()
         text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
@@ -467,9 +472,11 @@ def run_ours(args, world, rank, local):
 
     secondary = None
     mixer = None
+    ffn = None
     if not args.no_secondary and args.workload == "16k":
         secondary = secondary_line(binding, dev)
         mixer = mixer_line(binding, dev, wl, host)
+        ffn = sswiglu_line(binding, dev, wl)
 
     if rank == 0:
         cpu = oracle_rate(wl, seconds=10.0)
@@ -505,6 +512,8 @@ def run_ours(args, world, rank, local):
             line["secondary"] = secondary
         if mixer is not None:
             line["mixer"] = mixer
+        if ffn is not None:
+            line["sswiglu"] = ffn
         print(json.dumps(line), flush=True)
 
     graphs.clear()
@@ -635,6 +644,72 @@ def mixer_line(binding, dev, wl, host, steps=200):
             "peak_tflops": peak, "peak_kind": kind,
             "mixer_step_ms": ms_all, "mixer_token_heads_per_s": wl.token_heads / (ms_all * 1e-3),
             "l2": "warm (one input set; weights and activations fit L2 at 16k only partly)"}
+
+
+SSWIGLU_HIDDEN = 1024
+
+
+def sswiglu_bytes(B, T, C):
+    """Algorithmic bytes of one S-SwiGLU mixing launch (16-bit activations):
+    u read once (2C channels), h written once (C channels), fp32 taps and bias."""
+    return B * T * (2 * C + C) * 2 + (9 * C + C) * 4
+
+
+def sswiglu_line(binding, dev, wl, steps=200):
+    """The Spatial SwiGLU block on the workload's token grid (hidden width 1024,
+    random weights): the mixing kernel alone (HBM-bound; two input sets
+    alternate, 200 MB together, more than L2) with its achieved GB/s against
+    the measured copy bandwidth, and the whole block (two cuBLAS projections and
+    the mixing kernel) on warm buffers."""
+    B, gh, gw, dm, C = wl.B, wl.gh, wl.gw, wl.d_model, SSWIGLU_HIDDEN
+    T = gh * gw
+    gen = torch.Generator().manual_seed(23)
+    x = torch.randn(B, T, dm, generator=gen).half().to(dev)
+    w_in = (torch.randn(dm, 2 * C, generator=gen) / dm ** 0.5).half().to(dev)
+    w_out = (torch.randn(C, dm, generator=gen) / C ** 0.5).half().to(dev)
+    cw = (torch.randn(3, 3, C, generator=gen) / 3.0).float().to(dev)
+    cb = (torch.randn(C, generator=gen) * 0.1).float().to(dev)
+    sets = [(torch.randn(B, T, 2 * C, device=dev).half(), torch.empty(B, T, C, device=dev, dtype=torch.half))
+            for _ in range(2)]
+    stream = torch.cuda.Stream(device=dev)
+
+    def mix():
+        for u, h in sets:
+            binding.sswiglu_mix(u, cw, cb, grid_h=gh, grid_w=gw, out=h, stream=stream)
+
+    def block():
+        binding.sswiglu_fwd(x, w_in, cw, cb, w_out, grid_h=gh, grid_w=gw, scratch=sets[0], stream=stream)
+
+    with torch.cuda.stream(stream):
+        mix()
+        block()
+    stream.synchronize()
+
+    def time_graph(fn, reps):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            for _ in range(10):
+                g.replay()
+            a.record(stream)
+            for _ in range(reps):
+                g.replay()
+            b.record(stream)
+        stream.synchronize()
+        return a.elapsed_time(b) / reps
+
+    ms_mix = time_graph(mix, steps) / len(sets)
+    ms_block = time_graph(block, steps)
+    peak, kind = read_peak()
+    ab = sswiglu_bytes(B, T, C)
+    gbs = ab / (ms_mix * 1e-3) / 1e9
+    return {"workload": f"{B}x{gh}x{gw} tokens, d_model {dm}, hidden {C}, 3x3 depthwise, fp16",
+            "mix_kernel": "sswiglu_mix_kernel", "mix_ms": ms_mix, "mix_alg_bytes": ab,
+            "mix_gbs": gbs, "peak_gbs": peak, "peak_kind": kind, "mix_frac": gbs / peak,
+            "block_ms": ms_block, "block_tokens_per_s": B * T / (ms_block * 1e-3),
+            "l2": "mix: two alternating input sets (200 MB); block: warm"}
 
 
 def secondary_line(binding, dev, steps=2000):

@@ -262,6 +262,42 @@ GTR_API gtr_status_t gtr_mixer_out_proj(const void *y, const void *w_out, void *
                                         int d_in, int d_out, int dtype, void *stream);
 
 /*
+ * The Spatial SwiGLU feed-forward block of a GTR layer (GTR article, 方法详解
+ * §2, Spatial SwiGLU): the channel expansion u = x W_in holds a gate branch and
+ * a value branch; the value branch, laid out as the 2-D token grid, is mixed by
+ * a depthwise convolution with zero padding (output grid = input grid); the
+ * result is multiplied by SiLU of the gate branch and projected back:
+ *     h[b,y,x,c] = SiLU(u[b,y,x,c]) * (bias[c] + sum_{i,j} conv_w[i,j,c] * u[b,y+i-1,x+j-1,C+c]),
+ *     y_out = h W_out.
+ * The pages leave the kernel size blank; ksize must be 3 (other odd sizes are
+ * GTR_ERR_UNSUPPORTED, even or non-positive ones GTR_ERR_INVALID_ARG).
+ * Tokens are in grid order, t = row * grid_w + column.  dtype GTR_F16 or
+ * GTR_BF16 for every activation and projection weight (GTR_F32 is
+ * GTR_ERR_UNSUPPORTED); C (the hidden width) a multiple of 8, else
+ * GTR_ERR_UNSUPPORTED.  Every pointer is a device pointer, 16-byte aligned
+ * (GTR_ERR_ALIGNMENT otherwise), owned by the caller; the call launches on
+ * `stream` and returns without synchronising.  Sizes of zero are an empty
+ * problem (GTR_OK, nothing launched).
+ *   gtr_sswiglu_mix: u [B, T, 2C] (gate channels [0, C), value channels [C, 2C)),
+ *     conv_w [3, 3, C] fp32 (tap (i, j) = kernel row i, column j), conv_b [C]
+ *     fp32 or NULL (no bias) -> h [B, T, C], fp32 arithmetic, rounded once to
+ *     dtype.  One kernel; h must not overlap u.
+ *   gtr_sswiglu_fwd: x [B*T, d_model], w_in [d_model, 2C], w_out [C, d_model]
+ *     -> y [B*T, d_model]; u [B*T, 2C] and h [B*T, C] are caller-provided
+ *     scratch that receive the expansion and the hidden activation.  The two
+ *     projections are cuBLAS GEMMs with fp32 accumulation (loaded as for
+ *     gtr_mixer_in_proj; make the first call on a device outside stream
+ *     capture).  C = 0 writes y = 0.
+ */
+GTR_API gtr_status_t gtr_sswiglu_mix(const void *u, const float *conv_w, const float *conv_b, void *h,
+                                     int B, int grid_h, int grid_w, int C, int ksize, int dtype,
+                                     void *stream);
+GTR_API gtr_status_t gtr_sswiglu_fwd(const void *x, const void *w_in, const float *conv_w,
+                                     const float *conv_b, const void *w_out, void *u, void *h, void *y,
+                                     int B, int grid_h, int grid_w, int d_model, int C, int ksize,
+                                     int dtype, void *stream);
+
+/*
  * Chunk-boundary states, for testing the first two stages on their own: the
  * state each chunk of `chunk` scan positions ends with,
  *   states [B, H, ceil(T/chunk), dk, dv] fp32, entry c = S after scan position

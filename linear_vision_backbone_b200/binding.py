@@ -28,7 +28,7 @@ EXPORTS = (
     "gtr_gla_set_path", "gtr_gla_path_for", "gtr_last_device_status", "gtr_gla_segment_chunks",
     "gtr_gla_fwd_noalloc", "gtr_gate_packed_bytes", "gtr_gate_pack", "gtr_gate_fwd_packed",
     "gtr_gla_segment_count", "gtr_gla_fwd_gated", "gtr_gla_fwd_gated_timed", "gtr_mixer_in_proj",
-    "gtr_mixer_out_proj",
+    "gtr_mixer_out_proj", "gtr_sswiglu_mix", "gtr_sswiglu_fwd",
 )
 
 _lock = threading.Lock()
@@ -77,6 +77,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                          I, I, I, I, I, I, I, I, I, P, P], I),
             "gtr_mixer_in_proj": ([P, P, P, P, P, P, I, I, I, I, I, I, I, P], I),
             "gtr_mixer_out_proj": ([P, P, P, ctypes.c_longlong, I, I, I, P], I),
+            "gtr_sswiglu_mix": ([P, P, P, P, I, I, I, I, I, I, P], I),
+            "gtr_sswiglu_fwd": ([P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P], I),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -286,6 +288,63 @@ def mixer_out_proj(y, w_out, stream=None):
                                    _stream(stream))
     _check("gtr_mixer_out_proj", rc)
     return out
+
+
+def _conv_check(conv_w, conv_b, C: int, ksize: int = 3):
+    _need(conv_w, "conv_w", torch.float32, (ksize, ksize, C))
+    if conv_b is not None:
+        _need(conv_b, "conv_b", torch.float32, (C,))
+
+
+def sswiglu_mix(u, conv_w, conv_b=None, *, grid_h: int, grid_w: int, out=None, stream=None):
+    """The Spatial SwiGLU hidden activation (``gtr_sswiglu_mix``): u [B, T, 2C]
+    16-bit (gate channels first, value channels last, T = grid_h * grid_w in
+    grid order), conv_w [3, 3, C] fp32, conv_b [C] fp32 or None ->
+    h = SiLU(u_gate) * (depthwise 3x3 convolution of u_value on the grid + conv_b)
+    as [B, T, C] in u's dtype."""
+    _need(u, "u")
+    if u.dim() != 3 or u.shape[1] != grid_h * grid_w or u.shape[2] % 2:
+        raise ValueError("u must be [B, grid_h * grid_w, 2C]")
+    B, T, C2 = u.shape
+    C = C2 // 2
+    _conv_check(conv_w, conv_b, C, conv_w.shape[0] if conv_w.dim() == 3 else 3)
+    if out is None:
+        out = torch.empty(B, T, C, device=u.device, dtype=u.dtype)
+    _need(out, "out", u.dtype, (B, T, C))
+    rc = load().gtr_sswiglu_mix(_ptr(u), _ptr(conv_w), _ptr(conv_b), _ptr(out), B, grid_h, grid_w, C,
+                                conv_w.shape[0], DTYPE_IDS[u.dtype], _stream(stream))
+    _check("gtr_sswiglu_mix", rc)
+    return out
+
+
+def sswiglu_fwd(x, w_in, conv_w, conv_b, w_out, *, grid_h: int, grid_w: int, scratch=None, stream=None):
+    """The Spatial SwiGLU block (``gtr_sswiglu_fwd``): x [B, T, d_model] 16-bit,
+    w_in [d_model, 2C] and w_out [C, d_model] of x's dtype, conv_w [3, 3, C] and
+    conv_b [C] fp32 -> y [B, T, d_model].  ``scratch`` is an optional (u, h)
+    pair of [B, T, 2C] and [B, T, C] tensors that receive the expansion and the
+    hidden activation; they are allocated when not given."""
+    _need(x, "x")
+    if x.dim() != 3 or x.shape[1] != grid_h * grid_w:
+        raise ValueError("x must be [B, grid_h * grid_w, d_model]")
+    B, T, dm = x.shape
+    _need(w_in, "w_in", x.dtype)
+    if w_in.dim() != 2 or w_in.shape[0] != dm or w_in.shape[1] % 2:
+        raise ValueError(f"w_in must be [{dm}, 2C]")
+    C = w_in.shape[1] // 2
+    _need(w_out, "w_out", x.dtype, (C, dm))
+    _conv_check(conv_w, conv_b, C, conv_w.shape[0] if conv_w.dim() == 3 else 3)
+    if scratch is None:
+        scratch = (torch.empty(B, T, 2 * C, device=x.device, dtype=x.dtype),
+                   torch.empty(B, T, C, device=x.device, dtype=x.dtype))
+    u, h = scratch
+    _need(u, "u", x.dtype, (B, T, 2 * C))
+    _need(h, "h", x.dtype, (B, T, C))
+    y = torch.empty(B, T, dm, device=x.device, dtype=x.dtype)
+    rc = load().gtr_sswiglu_fwd(_ptr(x), _ptr(w_in), _ptr(conv_w), _ptr(conv_b), _ptr(w_out), _ptr(u), _ptr(h),
+                                _ptr(y), B, grid_h, grid_w, dm, C, conv_w.shape[0], DTYPE_IDS[x.dtype],
+                                _stream(stream))
+    _check("gtr_sswiglu_fwd", rc)
+    return y
 
 
 def gla_fwd_noalloc(q, k, v, g, z, w=None, *, grid_h: int, grid_w: int, direction: str = "LR",

@@ -2,7 +2,8 @@
 
     python -m linear_vision_backbone_b200.build
 
-compiles ``csrc/gtr_gla.cu`` (the whole library is one translation unit) into
+compiles the translation units ``csrc/*.cu`` (``gtr_gla.cu``: the gate and the
+GLA with their projections; ``sswiglu.cu``: the Spatial SwiGLU block) into
 ``_build/libgtr_gla.so`` next to this file.  The library exports only the
 ``extern "C"`` entry points declared in ``include/gtr_gla.h``.
 """
@@ -47,7 +48,7 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     nvcc = os.environ.get("NVCC", "nvcc")
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = [nvcc, *NVCC_FLAGS, *extra, "-I", INCLUDE, "-I", CSRC,
-           os.path.join(CSRC, "gtr_gla.cu"), "-o", tmp]
+           *sorted(glob.glob(os.path.join(CSRC, "*.cu"))), "-o", tmp]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)

@@ -139,3 +139,30 @@ def test_mixer_projections_reject_invalid_arguments(lib):
     assert lib.gtr_mixer_out_proj(None, None, None, 0, 384, 384, 1, S) == 0
     assert lib.gtr_mixer_out_proj(P, P, None, 4, 384, 384, 1, S) == -1
     assert lib.gtr_mixer_out_proj(P, ctypes.c_void_p(40), P, 4, 384, 384, 2, S) == -3
+
+
+def test_sswiglu_rejects_invalid_arguments(lib):
+    P = ctypes.c_void_p(16)
+    S = None
+    mix = lib.gtr_sswiglu_mix
+    # u, conv_w, conv_b, h, B, gh, gw, C, ksize, dtype, stream
+    assert mix(P, P, P, P, -1, 4, 4, 64, 3, 1, S) == -1             # negative size
+    assert mix(P, P, P, P, 1, 4, 4, 64, 3, 5, S) == -1              # bad dtype
+    assert mix(P, P, P, P, 1, 4, 4, 64, 4, 1, S) == -1              # even kernel
+    assert mix(P, P, P, P, 1, 4, 4, 64, 0, 1, S) == -1
+    assert mix(P, P, P, P, 1, 4, 4, 64, 5, 1, S) == -2              # only 3 x 3
+    assert mix(P, P, P, P, 1, 4, 4, 64, 3, 0, S) == -2              # fp32
+    assert mix(P, P, P, P, 1, 4, 4, 60, 3, 1, S) == -2              # C not a multiple of 8
+    assert mix(None, None, None, None, 0, 4, 4, 64, 3, 1, S) == 0   # empty
+    assert mix(None, None, None, None, 1, 4, 4, 0, 3, 2, S) == 0
+    assert mix(P, None, P, P, 1, 4, 4, 64, 3, 1, S) == -1           # null weights
+    assert mix(P, P, P, None, 1, 4, 4, 64, 3, 1, S) == -1
+    assert mix(ctypes.c_void_p(24), P, None, P, 1, 4, 4, 64, 3, 1, S) == -3
+    assert mix(P, P, ctypes.c_void_p(20), P, 1, 4, 4, 64, 3, 2, S) == -3
+    fwd = lib.gtr_sswiglu_fwd
+    # x, w_in, conv_w, conv_b, w_out, u, h, y, B, gh, gw, d_model, C, ksize, dtype, stream
+    assert fwd(P, P, P, P, P, P, P, P, 1, 4, 4, -384, 1024, 3, 1, S) == -1
+    assert fwd(P, P, P, P, P, P, P, P, 1, 4, 4, 384, 1024, 3, 0, S) == -2
+    assert fwd(None, None, None, None, None, None, None, None, 1, 4, 4, 0, 1024, 3, 1, S) == 0
+    assert fwd(P, P, P, P, P, P, None, P, 1, 4, 4, 384, 1024, 3, 1, S) == -1
+    assert fwd(P, P, P, P, P, P, P, ctypes.c_void_p(8), 1, 4, 4, 384, 1024, 3, 1, S) == -3
