@@ -85,3 +85,9 @@ def test_kernel_source_hash_ignores_comments(tmp_path, monkeypatch):
     (csrc / "a.cuh").write_text("int f() { return 2; }\n")
     assert bench.kernel_source_hash() != h1
     assert os.path.isdir(csrc)
+
+
+def test_sswiglu_algorithmic_bytes():
+    # u read once (2C channels), h written once (C channels), 16-bit; fp32 taps (9 C) and bias (C)
+    assert bench.sswiglu_bytes(1, 16384, 1024) == 16384 * 3 * 1024 * 2 + 10 * 1024 * 4
+    assert bench.sswiglu_bytes(2, 10, 8) == 2 * 10 * 24 * 2 + 80 * 4
