@@ -1,6 +1,6 @@
 // common.cuh -- element types, scan-order index maps and device status shared
-// by the kernels of the Key-only GLA library.  Everything in this library is a
-// single translation unit (gtr_gla.cu) so device globals need no relocatable
+// by the kernels of the Key-only GLA library.  Every kernel that uses them is
+// in one translation unit (gtr_gla.cu), so device globals need no relocatable
 // device code.
 #pragma once
 

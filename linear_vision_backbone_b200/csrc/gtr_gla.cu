@@ -2,7 +2,8 @@
 // kernel launch.  Argument checks, the segment plan, workspace management and
 // the stage sequence K2 (summary) -> K3 (boundary scan) -> K4 (output) of the
 // chunkwise operator (GTR article, 方法详解 §4) live here; the kernels live in
-// the included .cuh files.  The whole library is this one translation unit.
+// the included .cuh files, all in this one translation unit (the Spatial
+// SwiGLU block is the library's other one, sswiglu.cu).
 #include <atomic>
 #include <map>
 #include <mutex>
