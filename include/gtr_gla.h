@@ -281,7 +281,7 @@ GTR_API gtr_status_t gtr_mixer_out_proj(const void *y, const void *w_out, void *
  *   gtr_sswiglu_mix: u [B, T, 2C] (gate channels [0, C), value channels [C, 2C)),
  *     conv_w [3, 3, C] fp32 (tap (i, j) = kernel row i, column j), conv_b [C]
  *     fp32 or NULL (no bias) -> h [B, T, C], fp32 arithmetic, rounded once to
- *     dtype.  One kernel; h must not overlap u.
+ *     dtype.  One kernel; an h that overlaps u is GTR_ERR_INVALID_ARG.
  *   gtr_sswiglu_fwd: x [B*T, d_model], w_in [d_model, 2C], w_out [C, d_model]
  *     -> y [B*T, d_model]; u [B*T, 2C] and h [B*T, C] are caller-provided
  *     scratch that receive the expansion and the hidden activation.  The two

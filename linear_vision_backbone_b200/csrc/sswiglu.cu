@@ -252,6 +252,12 @@ GTR_API gtr_status_t gtr_sswiglu_mix(const void* u, const float* conv_w, const f
   if (!u || !conv_w || !h) return GTR_ERR_INVALID_ARG;
   if (!aligned16(u) || !aligned16(conv_w) || !aligned16(h) || (conv_b && !aligned16(conv_b)))
     return GTR_ERR_ALIGNMENT;
+  {  // h is written while u is still being read by other blocks: the two must not overlap
+    const uintptr_t u0 = (uintptr_t)u, h0 = (uintptr_t)h;
+    const uintptr_t tok = (uintptr_t)B * grid_h * grid_w;
+    const uintptr_t u1 = u0 + tok * 2 * C * 2, h1 = h0 + tok * C * 2;
+    if (u0 < h1 && h0 < u1) return GTR_ERR_INVALID_ARG;
+  }
   const cudaStream_t st = (cudaStream_t)stream;
   rc = dtype == GTR_F16 ? mix_launch<__half>(u, conv_w, conv_b, h, B, grid_h, grid_w, C, st)
                         : mix_launch<__nv_bfloat16>(u, conv_w, conv_b, h, B, grid_h, grid_w, C, st);

@@ -159,6 +159,11 @@ def test_sswiglu_rejects_invalid_arguments(lib):
     assert mix(P, P, P, None, 1, 4, 4, 64, 3, 1, S) == -1
     assert mix(ctypes.c_void_p(24), P, None, P, 1, 4, 4, 64, 3, 1, S) == -3
     assert mix(P, P, ctypes.c_void_p(20), P, 1, 4, 4, 64, 3, 2, S) == -3
+    # h overlapping u (u spans 1*4*4*128*2 = 4096 bytes from 4096): rejected before any launch
+    U = ctypes.c_void_p(4096)
+    assert mix(U, P, None, ctypes.c_void_p(4096 + 4080), 1, 4, 4, 64, 3, 1, S) == -1
+    assert mix(U, P, None, ctypes.c_void_p(4096 - 2048 + 16), 1, 4, 4, 64, 3, 1, S) == -1
+    assert mix(U, P, None, U, 1, 4, 4, 64, 3, 1, S) == -1
     fwd = lib.gtr_sswiglu_fwd
     # x, w_in, conv_w, conv_b, w_out, u, h, y, B, gh, gw, d_model, C, ksize, dtype, stream
     assert fwd(P, P, P, P, P, P, P, P, 1, 4, 4, -384, 1024, 3, 1, S) == -1
