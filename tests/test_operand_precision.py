@@ -1,0 +1,104 @@
+"""The numeric design of the tensor-core GLA path, checked on the CPU.
+
+The chunk outputs are computed from chunk-start-referenced factors
+q~ = q e^{G}, k~ = k e^{-G} (G the in-chunk gate cumsum; GTR article, 方法详解
+§4, chunkwise operator), every tensor-core operand split into two bf16 terms
+hi = bf16(x), lo = bf16(x - hi) and multiplied as hi hi' + hi lo' + lo hi' with
+fp32 results.  These tests restate that arithmetic in numpy on one head of the
+16k workload and hold it to the parity rules of tests/parity.py against the
+fp64 oracle, at the kernel's chunk of 64 tokens and at 128.  They also check
+that the workload's gates keep every chunk inside the factorised range (the
+exact-chunk test's 20 nats).  They test the design's precision budget, not the
+CUDA code, which tests/test_gpu_parity.py compares with the oracle directly.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_vision_backbone_b200 import inputs
+from tests.parity import compare
+
+SPAN_MAX = 20.0   # nats of in-chunk decay the factorised scores take
+
+
+def _bf16(x):
+    return torch.from_numpy(np.ascontiguousarray(x)).float().to(torch.bfloat16).double().numpy()
+
+
+def _two_terms(x):
+    x32 = x.astype(np.float32).astype(np.float64)
+    hi = _bf16(x32)
+    return hi, _bf16(x32 - hi)
+
+
+def _product(a, b):
+    """(a_hi + a_lo)(b_hi + b_lo) without the lo lo term, rounded to fp32."""
+    return (a[0] @ b[0] + a[0] @ b[1] + a[1] @ b[0]).astype(np.float32).astype(np.float64)
+
+
+def _t(pair):
+    return pair[0].T, pair[1].T
+
+
+@pytest.fixture(scope="module")
+def head():
+    wl = inputs.WORKLOADS["16k"]
+    d = inputs.make_inputs(wl)
+    g = oracle.gate(d["x"], d["w_down"], d["w_up"], d["bias"], tau=wl.tau).reshape(1, wl.T, wl.H, wl.dk)
+    return wl, d, g
+
+
+def _emulate(q, k, v, z, g, w, chunk, key_terms=2):
+    n = q.shape[0]
+    S = np.zeros((q.shape[1], v.shape[1]))
+    o = np.zeros((n, v.shape[1]))
+    for c0 in range(0, n, chunk):
+        sl = slice(c0, c0 + chunk)
+        G = np.cumsum(g[sl], axis=0).astype(np.float32).astype(np.float64)
+        qt, kt = _two_terms(q[sl] * np.exp(G)), _two_terms(k[sl] * np.exp(-G))
+        if key_terms == 1:
+            kt = (kt[0], np.zeros_like(kt[1]))
+        vt = _two_terms(v[sl])
+        P = np.tril(_product(qt, _t(kt)))
+        o[sl] = _product(qt, _two_terms(S)) + _product(_two_terms(P), vt)
+        S = ((S + _product(_t(kt), vt)) * np.exp(G[-1])[:, None]).astype(np.float32).astype(np.float64)
+    rms = np.sqrt(np.mean(o ** 2, axis=-1, keepdims=True) + 1e-5)
+    return o / rms * w * (z / (1.0 + np.exp(-z)))
+
+
+def _head_case(head, n=4096, h=2):
+    wl, d, g = head
+    idx = np.array([oracle.scan_index("TB", s, wl.gh, wl.gw) for s in range(n)])
+    q, k, v, z = (d[name][0, idx, h].double().numpy() for name in ("q", "k", "v", "z"))
+    gg = g[0, idx, h].astype(np.float32).astype(np.float64)
+    w = d["w"].double().numpy()
+    one = lambda a: a.reshape(1, n, 1, -1)
+    ref = oracle.gla_fwd(one(q), one(k), one(v), one(gg), one(z), w, gh=1, gw=n, direction="LR")[0, :, 0]
+    return (q, k, v, z, gg, w), ref
+
+
+@pytest.mark.parametrize("chunk", (64, 128))
+def test_two_term_operands_meet_the_parity_bound(head, chunk):
+    args, ref = _head_case(head)
+    r = compare(torch.from_numpy(_emulate(*args, chunk)).half(), ref, torch.float16)
+    assert r["ok"] and r["worst_over_bound"] < 0.8 and r["rel_l2"] < 1e-4, r
+
+
+def test_one_term_keys_would_not(head):
+    # the reason for the key's second term: one bf16 term of k~ misses the bound
+    args, ref = _head_case(head)
+    r = compare(torch.from_numpy(_emulate(*args, 64, key_terms=1)).half(), ref, torch.float16)
+    assert not r["ok"] and r["worst_over_bound"] > 1.5, r
+
+
+@pytest.mark.parametrize("chunk", (64, 128))
+def test_workload_gates_stay_inside_the_factorised_range(head, chunk):
+    wl, _, g = head
+    grid = g[0].reshape(wl.gh, wl.gw, wl.H, wl.dk)
+    tb = grid.transpose(1, 0, 2, 3).reshape(wl.T, wl.H, wl.dk)        # down each column
+    for seq in (tb, tb[::-1]):
+        nc = wl.T // chunk
+        G = np.cumsum(seq[: nc * chunk].reshape(nc, chunk, wl.H, wl.dk), axis=1)
+        assert G.max() <= 0.0
+        assert -G.min() < SPAN_MAX / 2
