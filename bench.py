@@ -66,20 +66,46 @@ def step_dirs(wl):
     return list(wl.dirs)
 
 
-def alg_bytes(wl, nseg, esz, fused=False):
-    """Algorithmic bytes per launch of each kernel (unique reads + writes).
-    fused: the gate kernel writes the rank-16 rows x W_down (fp32) and the
-    summary kernel reads them and writes g."""
+def alg_bytes(wl, esz, fused=False):
+    """Algorithmic bytes per launch of each kernel: the unique reads and writes
+    of the operator's own tensors, without the workspace (boundary states).
+    Per token-head at dk = dv = 64 with 16-bit tensors: output kernel q, k, v,
+    z, out (2 x 64 bytes each) and g (4 x 64) = 896 bytes; summary kernel k, v,
+    g = 512 bytes; the boundary scan touches only the workspace (0).  fused:
+    the gate kernel writes the rank-16 rows x W_down (fp32) and the summary
+    kernel reads them and writes g."""
     th = wl.token_heads
     dk, dv = wl.dk, wl.dv
-    st = wl.B * wl.H * nseg * (dk * dv + dk) * 4
     low = wl.B * wl.T * wl.rank * 4
     return {
         "gate": wl.B * wl.T * wl.d_model * esz + (low if fused else th * dk * 4),
-        "summary": th * (dk * esz + dv * esz + dk * 4) + st + (low if fused else 0),
-        "scan": 2 * st,
-        "output": th * (2 * dk * esz + 2 * dv * esz + dk * 4) + th * dv * esz + st,
+        "summary": th * (dk * esz + dv * esz + dk * 4) + (low if fused else 0),
+        "scan": 0,
+        "output": th * (2 * dk * esz + 2 * dv * esz + dk * 4) + th * dv * esz,
     }
+
+
+def workspace_bytes(wl, nstates):
+    """Bytes of boundary-state traffic per launch (workspace, not algorithmic):
+    the summary kernel writes each of the `nstates` states (dk x dv fp32 and a
+    dk decay vector), the scan reads and rewrites them, the output kernel reads
+    them."""
+    st = wl.B * wl.H * nstates * (wl.dk * wl.dv + wl.dk) * 4
+    return {"gate": 0, "summary": st, "scan": 2 * st, "output": st}
+
+
+def host_cpu():
+    """Core count and CPU model of the host the CPU baseline runs on."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"host_cores": os.cpu_count(), "cpu_model": model}
 
 
 # ---------------------------------------------------------------- clocks
@@ -266,6 +292,7 @@ def oracle_rate(wl, seconds=10.0, rows=32):
         if el >= seconds:
             break
     return {"value": n * T * wl.H / el, "unit": "token-heads/s", "cores": used, "kind": "oracle",
+            **host_cpu(),
             "sample": f"gate + GLA of all {wl.H} heads over the first {rows}x{wl.gw}={T} tokens of "
                       f"the {wl.name} workload (batch entry 0), {n} repetitions in {el:.2f} s, fp64"}
 
@@ -305,7 +332,7 @@ def run_reference(args, world, rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": workload_text(wl), "sample": sample},
         "cpu_baseline": {"value": value, "unit": "token-heads/s", "cores": 1, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, **host_cpu()},
         "e2e": {"value": value, "unit": "token-heads/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -411,7 +438,8 @@ def run_ours(args, world, rank, local):
     # segment plan of this workload (for the state bytes)
     nc = (wl.T + args.chunk - 1) // args.chunk
     nseg = binding.segment_count(wl.B, wl.H, wl.gh, wl.gw, wl.dk, wl.dv, args.chunk, host["q"].dtype)
-    ab = alg_bytes(wl, nseg, esz, fused)
+    ab = alg_bytes(wl, esz, fused)
+    wsb = workspace_bytes(wl, nseg)
     dom = max(per_ms, key=lambda n: per_ms[n])
     peak, peak_kind = read_peak()
     achieved = ab[dom] / (per_ms[dom] * 1e-3) / 1e9
@@ -471,10 +499,12 @@ def run_ours(args, world, rank, local):
     e2e_value = aggregate_value(units, args.e2e_steps, e2e_ms, world)
 
     secondary = None
+    others = None
     mixer = None
     ffn = None
     if not args.no_secondary and args.workload == "16k":
         secondary = secondary_line(binding, dev)
+        others = configs_lines(binding, dev)
         mixer = mixer_line(binding, dev, wl, host)
         ffn = sswiglu_line(binding, dev, wl)
 
@@ -498,7 +528,7 @@ def run_ours(args, world, rank, local):
             "roofline": {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": traffic, "alg_bytes": ab[dom],
-                         "kernel_ms": per_ms[dom]},
+                         "workspace_bytes": wsb[dom], "kernel_ms": per_ms[dom]},
             "kernels_ms": per_ms,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "token-heads/s", "h2d_bytes_per_step": h2d,
@@ -510,6 +540,8 @@ def run_ours(args, world, rank, local):
         }
         if secondary is not None:
             line["secondary"] = secondary
+        if others is not None:
+            line["configs"] = others
         if mixer is not None:
             line["mixer"] = mixer
         if ffn is not None:
@@ -712,48 +744,99 @@ def sswiglu_line(binding, dev, wl, steps=200):
             "l2": "mix: two alternating input sets (200 MB); block: warm"}
 
 
-def secondary_line(binding, dev, steps=2000):
-    """The same step on the 640x640 workload (T = 1600), timed the same way."""
-    wl = gin.WORKLOADS["640"]
+def step_alg_bytes(wl):
+    """Algorithmic bytes of one whole step (gate projection when the workload
+    has one, then the GLA): per token-head q, k, v, z, out in the storage
+    dtype and g in fp32, plus, with the gate, x once (d_model values per token)
+    and the g write."""
+    esz = inputs_esz(wl)
+    th = wl.token_heads
+    gla = th * ((2 * wl.dk + 3 * wl.dv) * esz + wl.dk * 4)
+    if wl.recipe != "proj":
+        return gla
+    return gla + wl.B * wl.T * wl.d_model * esz + th * wl.dk * 4
+
+
+def inputs_esz(wl):
+    return {"f32": 4, "f16": 2, "bf16": 2}[wl.dtype]
+
+
+def config_line(binding, dev, wl, steps=200, nsets=8):
+    """One workload timed as the headline step is: a CUDA graph per input set
+    (gate projection + GLA for the projected workloads, GLA alone for the ones
+    whose gates are drawn directly), a 256 MiB buffer written between steps
+    (outside the timed events) so that every step starts with a cold L2, and
+    the step's algorithmic bytes over its time against the measured copy
+    bandwidth."""
     host = gin.make_inputs(wl)
+    nsets = max(1, min(nsets, (1 << 30) // max(1, sum(t.numel() * t.element_size()
+                                                       for t in host.values()))))
     sets = []
-    for i in range(8):
-        s = {n: host[n].to(dev) for n in ("x", "q", "k", "v", "z")}
-        s["g"] = torch.empty(wl.B, wl.T, wl.H, wl.dk, device=dev)
+    for i in range(nsets):
+        s = {n: host[n].to(dev) for n in host if n not in ("w_down", "w_up", "bias", "w")}
+        if "g" not in s:
+            s["g"] = torch.empty(wl.B, wl.T, wl.H, wl.dk, device=dev)
         s["out"] = torch.empty_like(s["v"])
         sets.append(s)
-    params = {n: host[n].to(dev) for n in ("w_down", "w_up", "bias", "w")}
     stream = torch.cuda.Stream(device=dev)
-    step, _ = make_step(binding, wl, params, host["x"].dtype, 64, stream)
-    torch.cuda.synchronize()
+    if wl.recipe == "proj":
+        params = {n: host[n].to(dev) for n in ("w_down", "w_up", "bias", "w")}
+        step, _ = make_step(binding, wl, params, host["x"].dtype, wl.chunk, stream)
+    else:
+        w = host["w"].to(dev)
 
+        def step(s, direction, evs=None):
+            binding.gla_fwd(s["q"], s["k"], s["v"], s["g"], s["z"], w, grid_h=wl.gh, grid_w=wl.gw,
+                            direction=direction, chunk=wl.chunk, out=s["out"], stream=stream)
+    torch.cuda.synchronize()
+    dirs = list(wl.dirs)
     with torch.cuda.stream(stream):
         for i, s in enumerate(sets):
-            step(s, wl.dirs[i % 4])
+            step(s, dirs[i % len(dirs)])
     stream.synchronize()
     graphs = []
     for i, s in enumerate(sets):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            step(s, wl.dirs[i % 4])
+            step(s, dirs[i % len(dirs)])
         graphs.append(g)
-    # a 256 MB buffer written between replays keeps L2 cold for this small case
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(steps)]
     with torch.cuda.stream(stream):
-        for i in range(20):
-            graphs[i % 8].replay()
+        for i in range(min(20, steps)):
+            graphs[i % nsets].replay()
         for i in range(steps):
             flush.fill_(i & 255)
             ev[i][0].record(stream)
-            graphs[i % 8].replay()
+            graphs[i % nsets].replay()
             ev[i][1].record(stream)
     stream.synchronize()
-    ms = sum(a.elapsed_time(b) for a, b in ev)
-    return {"workload": workload_text(wl), "value": wl.token_heads * steps / (ms * 1e-3),
-            "unit": "token-heads/s", "ms_per_step": ms / steps, "steps": steps,
-            "l2": "256 MiB buffer written between steps, outside the timed events"}
+    ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    peak, kind = read_peak()
+    ab = step_alg_bytes(wl)
+    gbs = ab / (ms * 1e-3) / 1e9
+    return {"workload": workload_text(wl), "value": wl.token_heads / (ms * 1e-3),
+            "unit": "token-heads/s", "ms_per_step": ms, "steps": steps,
+            "kernel_path": binding.path_for(wl.B, wl.H, wl.gh, wl.gw, wl.dk, wl.dv, wl.chunk,
+                                            host["q"].dtype),
+            "step_alg_bytes": ab, "achieved_gbs": gbs, "peak_gbs": peak, "peak_kind": kind,
+            "frac": gbs / peak, "l2": "256 MiB buffer written between steps, outside the timed events"}
+
+
+def secondary_line(binding, dev, steps=2000):
+    """The same step on the 640x640 workload (T = 1600), timed the same way."""
+    return config_line(binding, dev, gin.WORKLOADS["640"], steps=steps)
+
+
+def configs_lines(binding, dev):
+    """Every other workload: the batched 640x640 case and the d = 128 sweep."""
+    out = {"640b8": config_line(binding, dev, gin.WORKLOADS["640b8"], steps=500),
+           "tiny": config_line(binding, dev, gin.WORKLOADS["tiny"], steps=500)}
+    for gsz in gin.SWEEP_GRIDS:
+        wl = gin.WORKLOADS["sweep"].with_grid(gsz)
+        out[f"sweep-{gsz}"] = config_line(binding, dev, wl, steps=100 if gsz >= 128 else 300)
+    return out
 
 
 def main():

@@ -15,6 +15,7 @@
 #include "simt_kernels.cuh"
 #include "scan_kernel.cuh"
 #include "tc_kernels.cuh"
+#include "pipe_kernels.cuh"
 #include "gate_tc.cuh"
 #include "mixer_proj.cuh"
 
@@ -57,6 +58,7 @@ struct Plan {
   int B, H, gh, gw, T, dk, dv, dir, chunk, dtype;
   int dev;
   int path;        // GTR_PATH_SIMT or GTR_PATH_TC
+  int pipe;        // 1: the chunk-parallel tensor-core pipeline (a state per chunk)
   int nc;          // chunks per sequence
   int nseg;        // segments per sequence
   int seg_chunks;  // chunks in the longest segment
@@ -138,15 +140,27 @@ int choose_path(int dk, int dv, int chunk, int dtype) {
   return tc_supported(dk, dv, chunk, dtype) ? (int)GTR_PATH_TC : (int)GTR_PATH_SIMT;
 }
 
+// `legacy`: the segment-walking tensor-core kernels (the gate-fused call);
+// otherwise tensor-core shapes run the chunk-parallel pipeline, whose
+// workspace holds one state tile (16 KB) and one decay vector per chunk.
 int make_plan(Plan* p, int dev, int B, int H, int gh, int gw, int dk, int dv, int dir, int chunk,
-              int dtype, int force_nseg) {
+              int dtype, int force_nseg, bool legacy = false, int force_path = 0) {
   p->B = B; p->H = H; p->gh = gh; p->gw = gw; p->T = gh * gw; p->dev = dev;
   p->dk = dk; p->dv = dv; p->dir = dir; p->chunk = chunk; p->dtype = dtype;
-  const int path = choose_path(dk, dv, chunk, dtype);
+  const int path = force_path ? force_path : choose_path(dk, dv, chunk, dtype);
   if (path < 0) return path;
   p->path = path;
   p->nc = (p->T + chunk - 1) / chunk;
   const long long bh = (long long)B * H;
+  p->pipe = path == GTR_PATH_TC && !legacy;
+  if (p->pipe) {
+    if (bh * p->nc >= (1LL << 31)) return GTR_ERR_UNSUPPORTED;   // work items are counted in an int
+    p->nseg = p->nc;
+    p->seg_chunks = 1;
+    p->offA = ((size_t)bh * p->nc * tc::kStateTile + 255) & ~(size_t)255;
+    p->ws_bytes = p->offA + (size_t)bh * p->nc * dk * sizeof(float);
+    return GTR_OK;
+  }
   const int per_sm = path == GTR_PATH_TC ? tc_blocks_per_sm(dk, dv) : 4;
   const long long slots = (long long)sm_count(dev) * per_sm;
   if (force_nseg > 0) {
@@ -469,6 +483,50 @@ int launch_scan(const Plan& p, float* wsS, const float* wsA, int inclusive, cuda
              : GTR_ERR_CUDA;
 }
 
+// ---- the chunk-parallel tensor-core pipeline (pipe_kernels.cuh)
+template <typename T>
+int launch_pipe_typed(int stage, const tc::PipeParams& pp, const tc::Maps& mp, cudaStream_t st, int dev) {
+  static bool done_sum[kMaxDevices], done_out[kMaxDevices];
+  const long long total = (long long)pp.nbh * pp.nc;
+  const unsigned grid = (unsigned)(total < sm_count(dev) ? total : sm_count(dev));
+  if (stage == 0) {
+    if (int rc = ensure_smem(tc::gla_sum_pipe<T>, tc::kSumPipeSmem, done_sum, dev)) return rc;
+    return launch_pdl(tc::gla_sum_pipe<T>, dim3(grid), dim3(tc::kPipeThreads), tc::kSumPipeSmem, st, pp, mp)
+               ? GTR_ERR_CUDA
+               : GTR_OK;
+  }
+  if (int rc = ensure_smem(tc::gla_out_pipe<T>, tc::kOutPipeSmem, done_out, dev)) return rc;
+  return launch_pdl(tc::gla_out_pipe<T>, dim3(grid), dim3(tc::kPipeThreads), tc::kOutPipeSmem, st, pp, mp)
+             ? GTR_ERR_CUDA
+             : GTR_OK;
+}
+
+// One stage of the pipeline for sequences bh0 .. bh0 + nbh - 1: 0 = chunk
+// summaries, 1 = chunk scan (into `states`, inclusive fp32, when given), 2 =
+// chunk outputs.  `stb` / `ab`: the state tiles and decay factors of those
+// sequences.
+int launch_pipe(const Plan& p, int stage, const void* q, const void* k, const void* v, const float* g,
+                const void* z, const float* w, void* out, uint8_t* stb, float* ab, float* states, int bh0,
+                int nbh, cudaStream_t st) {
+  tc::PipeParams pp{q, k, v, g, z, w, stb, ab, out, states, p.H, p.T, p.gh, p.gw, p.dir, p.nc, bh0, nbh, 0};
+  if (stage == 1)
+    return launch_pdl(tc::gla_chunk_scan, dim3((unsigned)nbh * 64u), dim3(tc::kChunkScanThreads), 0, st, pp)
+               ? GTR_ERR_CUDA
+               : GTR_OK;
+  tc::Maps maps;
+  pp.tma = chunk_maps(p, stage == 2 ? q : nullptr, k, v, g, &maps) ? 1 : 0;
+  static const tc::Maps kNoMaps{};
+  const tc::Maps& mp = pp.tma ? maps : kNoMaps;
+  const int s = stage == 0 ? 0 : 1;
+  return p.dtype == GTR_F16 ? launch_pipe_typed<__half>(s, pp, mp, st, p.dev)
+                            : launch_pipe_typed<__nv_bfloat16>(s, pp, mp, st, p.dev);
+}
+
+// The three stages for sequences bh0 .. bh0 + nbh - 1 with their state tiles
+// at `ws` (events as gtr_gla_fwd_timed; null when not wanted).
+int run_pipe(const Plan& p, const void* q, const void* k, const void* v, const float* g, const void* z,
+             const float* w, void* out, void* ws, int bh0, int nbh, cudaStream_t st, void* const* ev);
+
 // Record a caller event; inside stream capture it becomes an external event
 // node, so a replayed graph records real timestamps.
 int record(void* const* ev, int i, cudaStream_t st) {
@@ -479,6 +537,21 @@ int record(void* const* ev, int i, cudaStream_t st) {
                             ? cudaEventRecordWithFlags((cudaEvent_t)ev[i], st, cudaEventRecordExternal)
                             : cudaEventRecord((cudaEvent_t)ev[i], st);
   return e == cudaSuccess ? GTR_OK : GTR_ERR_CUDA;
+}
+
+int run_pipe(const Plan& p, const void* q, const void* k, const void* v, const float* g, const void* z,
+             const float* w, void* out, void* ws, int bh0, int nbh, cudaStream_t st, void* const* ev) {
+  // the group's tiles, then its decay factors (256-byte aligned)
+  uint8_t* stb = (uint8_t*)ws;
+  float* ab = (float*)((char*)ws + (((size_t)nbh * p.nc * tc::kStateTile + 255) & ~(size_t)255));
+  int rc;
+  if ((rc = record(ev, 0, st))) return rc;
+  if ((rc = launch_pipe(p, 0, q, k, v, g, z, w, out, stb, ab, nullptr, bh0, nbh, st))) return rc;
+  if ((rc = record(ev, 1, st))) return rc;
+  if ((rc = launch_pipe(p, 1, q, k, v, g, z, w, out, stb, ab, nullptr, bh0, nbh, st))) return rc;
+  if ((rc = record(ev, 2, st))) return rc;
+  if ((rc = launch_pipe(p, 2, q, k, v, g, z, w, out, stb, ab, nullptr, bh0, nbh, st))) return rc;
+  return record(ev, 3, st);
 }
 
 int gla_fwd_impl(const void* q, const void* k, const void* v, const float* g, const void* z,
@@ -497,9 +570,10 @@ int gla_fwd_impl(const void* q, const void* k, const void* v, const float* g, co
   if ((rc = make_plan(&p, dev, B, H, gh, gw, dk, dv, dir, chunk, dtype, 0))) return rc;
   void* ws = nullptr;
   if ((rc = get_workspace(dev, stream, p.ws_bytes, &ws))) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (p.pipe) return run_pipe(p, q, k, v, g, z, w, out, ws, 0, B * H, st, ev);
   float* wsS = (float*)ws;
   float* wsA = (float*)((char*)ws + p.offA);
-  cudaStream_t st = (cudaStream_t)stream;
   if ((rc = record(ev, 0, st))) return rc;
   if ((rc = launch_stage(p, q, k, v, g, z, w, out, wsS, wsA, st, 0))) return rc;
   if ((rc = record(ev, 1, st))) return rc;
@@ -537,7 +611,7 @@ int gla_fwd_gated_impl(const void* x, int x_dtype, const void* packed, const flo
   int dev;
   if ((rc = current_device(&dev))) return rc;
   Plan p;
-  if ((rc = make_plan(&p, dev, B, H, gh, gw, dk, dv, dir, chunk, dtype, 0))) return rc;
+  if ((rc = make_plan(&p, dev, B, H, gh, gw, dk, dv, dir, chunk, dtype, 0, true))) return rc;
   cudaStream_t st = (cudaStream_t)stream;
   if ((rc = record(ev, 0, st))) return rc;
   if (p.path != GTR_PATH_TC) {
@@ -609,20 +683,38 @@ int gla_fwd_noalloc_impl(const void* q, const void* k, const void* v, const floa
   if ((rc = current_device(&dev))) return rc;
   Plan p;
   if ((rc = make_plan(&p, dev, B, H, gh, gw, dk, dv, dir, chunk, dtype, 0))) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (p.pipe) {
+    // the tensor-core pipeline keeps a state per chunk: as many sequences per
+    // round of its three kernels as the static scratch holds
+    const size_t per_seq = (size_t)p.nc * (tc::kStateTile + dk * sizeof(float));
+    const size_t group = (kStaticScratchBytes - 256) / per_seq;
+    if (group >= 1) {
+      void* ws = nullptr;
+      if ((rc = static_scratch(dev, &ws))) return rc;
+      const int nbh = B * H;
+      for (int bh0 = 0; bh0 < nbh; bh0 += (int)group) {
+        const int n = nbh - bh0 < (int)group ? nbh - bh0 : (int)group;
+        if ((rc = run_pipe(p, q, k, v, g, z, w, out, ws, bh0, n, st, nullptr))) return rc;
+      }
+      return GTR_OK;
+    }
+    // a sequence longer than that runs the segment-walking SIMT kernels
+    if ((rc = make_plan(&p, dev, B, H, gh, gw, dk, dv, dir, chunk, dtype, 0, false, GTR_PATH_SIMT))) return rc;
+  }
   if (p.ws_bytes > kStaticScratchBytes) {
     // fewer, longer segments until the boundary states fit the static scratch
     const size_t per_seg = (size_t)B * H * ((size_t)dk * dv + dk) * sizeof(float);
     const size_t max_nseg = (kStaticScratchBytes - 256) / per_seg;
     if (max_nseg < 1) return GTR_ERR_NO_MEMORY;
     const int nseg = (int)(max_nseg < (size_t)p.nc ? max_nseg : (size_t)p.nc);
-    if ((rc = make_plan(&p, dev, B, H, gh, gw, dk, dv, dir, chunk, dtype, nseg))) return rc;
+    if ((rc = make_plan(&p, dev, B, H, gh, gw, dk, dv, dir, chunk, dtype, nseg, false, p.path))) return rc;
     if (p.ws_bytes > kStaticScratchBytes) return GTR_ERR_NO_MEMORY;
   }
   void* ws = nullptr;
   if ((rc = static_scratch(dev, &ws))) return rc;
   float* wsS = (float*)ws;
   float* wsA = (float*)((char*)ws + p.offA);
-  cudaStream_t st = (cudaStream_t)stream;
   if ((rc = launch_stage(p, q, k, v, g, z, w, out, wsS, wsA, st, 0))) return rc;
   if ((rc = launch_scan(p, wsS, wsA, 0, st))) return rc;
   return launch_stage(p, q, k, v, g, z, w, out, wsS, wsA, st, 1);
@@ -875,10 +967,21 @@ gtr_status_t gtr_gla_chunk_states(const void* k, const void* v, const float* g, 
   // one chunk per segment: the scan then gives the state after every chunk
   if ((rc = make_plan(&p, dev, B, H, grid_h, grid_w, dk, dv, dir, chunk, dtype, 0x7fffffff)))
     return (gtr_status_t)rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (p.pipe) {
+    // the pipeline's summary kernel, then its scan in inclusive fp32 mode
+    void* ws = nullptr;
+    if ((rc = get_workspace(dev, stream, p.ws_bytes, &ws))) return (gtr_status_t)rc;
+    uint8_t* stb = (uint8_t*)ws;
+    float* ab = (float*)((char*)ws + p.offA);
+    if ((rc = launch_pipe(p, 0, nullptr, k, v, g, nullptr, nullptr, nullptr, stb, ab, nullptr, 0, B * H, st)))
+      return (gtr_status_t)rc;
+    return (gtr_status_t)launch_pipe(p, 1, nullptr, k, v, g, nullptr, nullptr, nullptr, stb, ab, states, 0,
+                                     B * H, st);
+  }
   void* ws = nullptr;
   const size_t lbytes = (size_t)B * H * p.nseg * dk * sizeof(float);
   if ((rc = get_workspace(dev, stream, lbytes, &ws))) return (gtr_status_t)rc;
-  cudaStream_t st = (cudaStream_t)stream;
   if ((rc = launch_stage(p, nullptr, k, v, g, nullptr, nullptr, nullptr, states, (float*)ws, st, 0)))
     return (gtr_status_t)rc;
   return (gtr_status_t)launch_scan(p, states, (const float*)ws, 1, st);

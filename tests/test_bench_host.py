@@ -9,22 +9,44 @@ from linear_vision_backbone_b200 import inputs
 
 def test_algorithmic_bytes_of_the_16k_step():
     wl = inputs.WORKLOADS["16k"]
-    nseg = 48
     th = 16384 * 6
-    st = 6 * nseg * (64 * 64 + 64) * 4
-    ab = bench.alg_bytes(wl, nseg, 2)
-    # K4: q, k, v, z (2 bytes x 64 each), g (4 x 64), out (2 x 64) per token-head, plus states
-    assert ab["output"] == th * (4 * 128 + 256 + 128) + st
-    # K2: k, v, g per token-head plus states; K3 reads and writes the states
-    assert ab["summary"] == th * (128 + 128 + 256) + st
-    assert ab["scan"] == 2 * st
+    ab = bench.alg_bytes(wl, 2)
+    # K4: q, k, v, z (2 bytes x 64 each), g (4 x 64), out (2 x 64) per token-head: 896 bytes
+    assert ab["output"] == th * 896
+    # K2: k, v, g per token-head; K3 touches only the workspace
+    assert ab["summary"] == th * (128 + 128 + 256)
+    assert ab["scan"] == 0
     # K1: x once (384 x 2 bytes per token) and g written
     assert ab["gate"] == 16384 * 384 * 2 + th * 256
     # the fused gate: rank-16 rows instead of g in K1, read by K2 (which then writes g)
-    fused = bench.alg_bytes(wl, nseg, 2, fused=True)
+    fused = bench.alg_bytes(wl, 2, fused=True)
     assert fused["gate"] == 16384 * 384 * 2 + 16384 * 16 * 4
     assert fused["summary"] == ab["summary"] + 16384 * 16 * 4
     assert fused["output"] == ab["output"]
+    # boundary states are workspace traffic, reported apart from the algorithmic bytes
+    ws = bench.workspace_bytes(wl, 256)
+    st = 6 * 256 * (64 * 64 + 64) * 4
+    assert ws == {"gate": 0, "summary": st, "scan": 2 * st, "output": st}
+
+
+def test_whole_step_algorithmic_bytes_of_every_workload():
+    # gate + GLA at d = 64, 16-bit: 896 + 384 bytes per token-head (x is 384 x 2 / 6 heads)
+    wl = inputs.WORKLOADS["16k"]
+    assert bench.step_alg_bytes(wl) == wl.token_heads * (896 + 384)
+    wl = inputs.WORKLOADS["640b8"]
+    assert bench.step_alg_bytes(wl) == 8 * 1600 * 6 * (896 + 384)
+    # GLA alone (gates drawn directly): d = 128 bf16 is 5 x 256 + 512 = 1792 bytes
+    wl = inputs.WORKLOADS["sweep"].with_grid(64)
+    assert bench.step_alg_bytes(wl) == 4096 * 4 * 1792
+    # fp32 d = 16: 5 x 64 + 64 = 384 bytes
+    wl = inputs.WORKLOADS["tiny"]
+    assert bench.step_alg_bytes(wl) == 64 * 384
+
+
+def test_host_cpu_record():
+    h = bench.host_cpu()
+    assert h["host_cores"] == os.cpu_count()
+    assert "cpu_model" in h
 
 
 def test_whole_job_value_counts_every_rank():

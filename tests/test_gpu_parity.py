@@ -307,6 +307,21 @@ def test_zero_gate_long_memory():
     assert_close(y, ref, torch.bfloat16, "g = 0")
 
 
+def _states_close(st, ref):
+    """fp32 chunk-boundary states against the fp64 oracle, element by element:
+    |got - ref| <= 1e-4 (|ref| + RMS(ref)).  The states are sums of fp32
+    products over up to a few thousand tokens; the tensor-core summary's key
+    operand carries 22 (fp16 terms) or 16 (bf16 terms) significant bits, so
+    its per-element error stays well inside 1e-4 of the state's scale."""
+    got = st.double().cpu().numpy()
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.all(np.isfinite(got))
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    bound = 1e-4 * (np.abs(ref) + rms)
+    worst = float(np.max(np.abs(got - ref) / bound))
+    assert worst <= 1.0, worst
+
+
 @pytest.mark.parametrize("chunk", (16, 64, 128))
 @pytest.mark.parametrize("direction", ("LR", "BT"))
 def test_chunk_states_against_oracle(chunk, direction):
@@ -315,9 +330,7 @@ def test_chunk_states_against_oracle(chunk, direction):
     st = binding.chunk_states(_dev(d["k"]), _dev(d["v"]), _dev(d["g"]), grid_h=gh, grid_w=gw,
                               direction=direction, chunk=chunk)
     ref = oracle.chunk_states(d["k"], d["v"], d["g"], gh=gh, gw=gw, direction=direction, chunk=chunk)
-    got = st.double().cpu().numpy()
-    rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
-    assert rel < 1e-3, rel
+    _states_close(st, ref)
 
 
 def test_chunk_states_many_segments():
@@ -328,9 +341,7 @@ def test_chunk_states_many_segments():
     st = binding.chunk_states(_dev(d["k"]), _dev(d["v"]), _dev(d["g"]), grid_h=gh, grid_w=gw,
                               direction="TB", chunk=16)
     ref = oracle.chunk_states(d["k"], d["v"], d["g"], gh=gh, gw=gw, direction="TB", chunk=16)
-    got = st.double().cpu().numpy()
-    rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
-    assert rel < 1e-3, rel
+    _states_close(st, ref)
 
 
 def test_chunk_states_into_a_16_byte_aligned_buffer():
