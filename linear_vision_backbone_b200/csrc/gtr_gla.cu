@@ -140,6 +140,31 @@ int choose_path(int dk, int dv, int chunk, int dtype) {
   return tc_supported(dk, dv, chunk, dtype) ? (int)GTR_PATH_TC : (int)GTR_PATH_SIMT;
 }
 
+// Workspace of the tensor-core pipeline for nbh sequences of nc chunks in
+// nseg segments: chunk increments (a 16 KB state tile per chunk), chunk
+// decay factors (64 fp32), segment states (a tile per segment), segment
+// decay factors; each region 256-byte aligned.
+struct PipeWs {
+  uint8_t* dS; float* a; uint8_t* segS; float* segA;
+};
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+size_t pipe_ws_bytes(long long nbh, int nc, int nseg) {
+  return align256((size_t)nbh * nc * tc::kStateTile) + align256((size_t)nbh * nc * 64 * sizeof(float)) +
+         align256((size_t)nbh * nseg * tc::kStateTile) + (size_t)nbh * nseg * 64 * sizeof(float);
+}
+PipeWs pipe_ws(void* base, long long nbh, int nc, int nseg) {
+  PipeWs w;
+  char* b = (char*)base;
+  w.dS = (uint8_t*)b;
+  b += align256((size_t)nbh * nc * tc::kStateTile);
+  w.a = (float*)b;
+  b += align256((size_t)nbh * nc * 64 * sizeof(float));
+  w.segS = (uint8_t*)b;
+  b += align256((size_t)nbh * nseg * tc::kStateTile);
+  w.segA = (float*)b;
+  return w;
+}
+
 // `legacy`: the segment-walking tensor-core kernels (the gate-fused call);
 // otherwise tensor-core shapes run the chunk-parallel pipeline, whose
 // workspace holds one state tile (16 KB) and one decay vector per chunk.
@@ -154,11 +179,14 @@ int make_plan(Plan* p, int dev, int B, int H, int gh, int gw, int dk, int dv, in
   const long long bh = (long long)B * H;
   p->pipe = path == GTR_PATH_TC && !legacy;
   if (p->pipe) {
-    if (bh * p->nc >= (1LL << 31)) return GTR_ERR_UNSUPPORTED;   // work items are counted in an int
-    p->nseg = p->nc;
-    p->seg_chunks = 1;
-    p->offA = ((size_t)bh * p->nc * tc::kStateTile + 255) & ~(size_t)255;
-    p->ws_bytes = p->offA + (size_t)bh * p->nc * dk * sizeof(float);
+    if (bh * p->nc >= (1LL << 31)) return GTR_ERR_UNSUPPORTED;   // chunks are counted in an int
+    // one segment per CTA when the sequences leave SMs over; a CTA walks
+    // several segments otherwise
+    const long long per = sm_count(dev) / (bh > 0 ? bh : 1);
+    p->nseg = (int)(per < 1 ? 1 : (per > p->nc ? p->nc : per));
+    p->seg_chunks = (p->nc + p->nseg - 1) / p->nseg;
+    p->offA = 0;
+    p->ws_bytes = pipe_ws_bytes(bh, p->nc, p->nseg);
     return GTR_OK;
   }
   const int per_sm = path == GTR_PATH_TC ? tc_blocks_per_sm(dk, dv) : 4;
@@ -300,7 +328,7 @@ int tmap_chunk(CUtensorMap* map, CUtensorMapDataType dt, int es, const void* bas
 // g may be null; `g_store` adds the store map of the g the summary kernel
 // writes (32-column boxes, SWIZZLE_128B).
 bool chunk_maps(const Plan& p, const void* q, const void* k, const void* v, const float* g, tc::Maps* maps,
-                const float* low = nullptr, const float* g_store = nullptr) {
+                const float* low = nullptr, const float* g_store = nullptr, bool swizzle_qk = false) {
   for (const void* a : {q, k, v, (const void*)g, (const void*)low, (const void*)g_store})
     if (((uintptr_t)a & 15) != 0) return false;
   bool orient[2] = {false, false};
@@ -314,8 +342,8 @@ bool chunk_maps(const Plan& p, const void* q, const void* k, const void* v, cons
   *maps = tc::Maps{};
   for (int o = 0; o < 2; ++o) {
     if (!orient[o]) continue;
-    if ((q && tmap_chunk(&maps->t[o][tc::kMapQ], dt, 2, q, p, o, false)) ||
-        tmap_chunk(&maps->t[o][tc::kMapK], dt, 2, k, p, o, false) ||
+    if ((q && tmap_chunk(&maps->t[o][tc::kMapQ], dt, 2, q, p, o, swizzle_qk)) ||
+        tmap_chunk(&maps->t[o][tc::kMapK], dt, 2, k, p, o, swizzle_qk) ||
         tmap_chunk(&maps->t[o][tc::kMapV], dt, 2, v, p, o, true) ||
         (g && tmap_chunk(&maps->t[o][tc::kMapG], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, g, p, o, false)) ||
         (low && tmap_chunk(&maps->t[o][tc::kMapL], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, low, p, o, false,
@@ -483,12 +511,12 @@ int launch_scan(const Plan& p, float* wsS, const float* wsA, int inclusive, cuda
              : GTR_ERR_CUDA;
 }
 
-// ---- the chunk-parallel tensor-core pipeline (pipe_kernels.cuh)
+// ---- the tensor-core pipeline (pipe_kernels.cuh)
 template <typename T>
 int launch_pipe_typed(int stage, const tc::PipeParams& pp, const tc::Maps& mp, cudaStream_t st, int dev) {
   static bool done_sum[kMaxDevices], done_out[kMaxDevices];
-  const long long total = (long long)pp.nbh * pp.nc;
-  const unsigned grid = (unsigned)(total < sm_count(dev) ? total : sm_count(dev));
+  const long long segs = (long long)pp.nbh * pp.nseg;
+  const unsigned grid = (unsigned)(segs < sm_count(dev) ? segs : sm_count(dev));
   if (stage == 0) {
     if (int rc = ensure_smem(tc::gla_sum_pipe<T>, tc::kSumPipeSmem, done_sum, dev)) return rc;
     return launch_pdl(tc::gla_sum_pipe<T>, dim3(grid), dim3(tc::kPipeThreads), tc::kSumPipeSmem, st, pp, mp)
@@ -501,20 +529,25 @@ int launch_pipe_typed(int stage, const tc::PipeParams& pp, const tc::Maps& mp, c
              : GTR_OK;
 }
 
-// One stage of the pipeline for sequences bh0 .. bh0 + nbh - 1: 0 = chunk
-// summaries, 1 = chunk scan (into `states`, inclusive fp32, when given), 2 =
-// chunk outputs.  `stb` / `ab`: the state tiles and decay factors of those
-// sequences.
+// The affine scan over `n` state tiles per sequence for nbh sequences (see
+// gla_tile_scan): in place (entering states) or, with `states`, inclusive fp32.
+int launch_tile_scan(uint8_t* tiles, const float* a, float* states, int n, int nbh, cudaStream_t st) {
+  const tc::ScanParams sp{tiles, a, states, n, states ? 1 : 0};
+  return launch_pdl(tc::gla_tile_scan, dim3((unsigned)nbh * 64u), dim3(tc::kTileScanThreads), 0, st, sp)
+             ? GTR_ERR_CUDA
+             : GTR_OK;
+}
+
+// One stage of the pipeline for sequences bh0 .. bh0 + nbh - 1 with their
+// workspace `w`: 0 = chunk summaries (and segment maps), 1 = scan over the
+// segments, 2 = chunk outputs.
 int launch_pipe(const Plan& p, int stage, const void* q, const void* k, const void* v, const float* g,
-                const void* z, const float* w, void* out, uint8_t* stb, float* ab, float* states, int bh0,
-                int nbh, cudaStream_t st) {
-  tc::PipeParams pp{q, k, v, g, z, w, stb, ab, out, states, p.H, p.T, p.gh, p.gw, p.dir, p.nc, bh0, nbh, 0};
-  if (stage == 1)
-    return launch_pdl(tc::gla_chunk_scan, dim3((unsigned)nbh * 64u), dim3(tc::kChunkScanThreads), 0, st, pp)
-               ? GTR_ERR_CUDA
-               : GTR_OK;
+                const void* z, const float* w, void* out, const PipeWs& ws, int bh0, int nbh, cudaStream_t st) {
+  if (stage == 1) return launch_tile_scan(ws.segS, ws.segA, nullptr, p.nseg, nbh, st);
+  tc::PipeParams pp{q, k, v, g, z, w, ws.dS, ws.a, ws.segS, ws.segA, out,
+                    p.H, p.T, p.gh, p.gw, p.dir, p.nc, p.nseg, bh0, nbh, 0};
   tc::Maps maps;
-  pp.tma = chunk_maps(p, stage == 2 ? q : nullptr, k, v, g, &maps) ? 1 : 0;
+  pp.tma = chunk_maps(p, stage == 2 ? q : nullptr, k, v, g, &maps, nullptr, nullptr, true) ? 1 : 0;
   static const tc::Maps kNoMaps{};
   const tc::Maps& mp = pp.tma ? maps : kNoMaps;
   const int s = stage == 0 ? 0 : 1;
@@ -522,8 +555,8 @@ int launch_pipe(const Plan& p, int stage, const void* q, const void* k, const vo
                             : launch_pipe_typed<__nv_bfloat16>(s, pp, mp, st, p.dev);
 }
 
-// The three stages for sequences bh0 .. bh0 + nbh - 1 with their state tiles
-// at `ws` (events as gtr_gla_fwd_timed; null when not wanted).
+// The three stages for sequences bh0 .. bh0 + nbh - 1 with their workspace at
+// `ws` (events as gtr_gla_fwd_timed; null when not wanted).
 int run_pipe(const Plan& p, const void* q, const void* k, const void* v, const float* g, const void* z,
              const float* w, void* out, void* ws, int bh0, int nbh, cudaStream_t st, void* const* ev);
 
@@ -541,16 +574,14 @@ int record(void* const* ev, int i, cudaStream_t st) {
 
 int run_pipe(const Plan& p, const void* q, const void* k, const void* v, const float* g, const void* z,
              const float* w, void* out, void* ws, int bh0, int nbh, cudaStream_t st, void* const* ev) {
-  // the group's tiles, then its decay factors (256-byte aligned)
-  uint8_t* stb = (uint8_t*)ws;
-  float* ab = (float*)((char*)ws + (((size_t)nbh * p.nc * tc::kStateTile + 255) & ~(size_t)255));
+  const PipeWs pw = pipe_ws(ws, nbh, p.nc, p.nseg);
   int rc;
   if ((rc = record(ev, 0, st))) return rc;
-  if ((rc = launch_pipe(p, 0, q, k, v, g, z, w, out, stb, ab, nullptr, bh0, nbh, st))) return rc;
+  if ((rc = launch_pipe(p, 0, q, k, v, g, z, w, out, pw, bh0, nbh, st))) return rc;
   if ((rc = record(ev, 1, st))) return rc;
-  if ((rc = launch_pipe(p, 1, q, k, v, g, z, w, out, stb, ab, nullptr, bh0, nbh, st))) return rc;
+  if ((rc = launch_pipe(p, 1, q, k, v, g, z, w, out, pw, bh0, nbh, st))) return rc;
   if ((rc = record(ev, 2, st))) return rc;
-  if ((rc = launch_pipe(p, 2, q, k, v, g, z, w, out, stb, ab, nullptr, bh0, nbh, st))) return rc;
+  if ((rc = launch_pipe(p, 2, q, k, v, g, z, w, out, pw, bh0, nbh, st))) return rc;
   return record(ev, 3, st);
 }
 
@@ -685,10 +716,10 @@ int gla_fwd_noalloc_impl(const void* q, const void* k, const void* v, const floa
   if ((rc = make_plan(&p, dev, B, H, gh, gw, dk, dv, dir, chunk, dtype, 0))) return rc;
   cudaStream_t st = (cudaStream_t)stream;
   if (p.pipe) {
-    // the tensor-core pipeline keeps a state per chunk: as many sequences per
-    // round of its three kernels as the static scratch holds
-    const size_t per_seq = (size_t)p.nc * (tc::kStateTile + dk * sizeof(float));
-    const size_t group = (kStaticScratchBytes - 256) / per_seq;
+    // the tensor-core pipeline keeps a state tile per chunk and per segment:
+    // as many sequences per round of its three kernels as the static scratch holds
+    const size_t per_seq = ((size_t)p.nc + p.nseg) * (tc::kStateTile + dk * sizeof(float));
+    const size_t group = (kStaticScratchBytes - 4 * 256) / per_seq;
     if (group >= 1) {
       void* ws = nullptr;
       if ((rc = static_scratch(dev, &ws))) return rc;
@@ -969,15 +1000,14 @@ gtr_status_t gtr_gla_chunk_states(const void* k, const void* v, const float* g, 
     return (gtr_status_t)rc;
   cudaStream_t st = (cudaStream_t)stream;
   if (p.pipe) {
-    // the pipeline's summary kernel, then its scan in inclusive fp32 mode
+    // the pipeline's summary kernel, then the scan over its chunk increments
+    // in inclusive fp32 mode
     void* ws = nullptr;
     if ((rc = get_workspace(dev, stream, p.ws_bytes, &ws))) return (gtr_status_t)rc;
-    uint8_t* stb = (uint8_t*)ws;
-    float* ab = (float*)((char*)ws + p.offA);
-    if ((rc = launch_pipe(p, 0, nullptr, k, v, g, nullptr, nullptr, nullptr, stb, ab, nullptr, 0, B * H, st)))
+    const PipeWs pw = pipe_ws(ws, (long long)B * H, p.nc, p.nseg);
+    if ((rc = launch_pipe(p, 0, nullptr, k, v, g, nullptr, nullptr, nullptr, pw, 0, B * H, st)))
       return (gtr_status_t)rc;
-    return (gtr_status_t)launch_pipe(p, 1, nullptr, k, v, g, nullptr, nullptr, nullptr, stb, ab, states, 0,
-                                     B * H, st);
+    return (gtr_status_t)launch_tile_scan(pw.dS, pw.a, states, p.nc, B * H, st);
   }
   void* ws = nullptr;
   const size_t lbytes = (size_t)B * H * p.nseg * dk * sizeof(float);

@@ -1,41 +1,48 @@
-// pipe_kernels.cuh -- the chunk-parallel tcgen05 path of the Key-only GLA
-// (sm_100a): 16-bit q/k/v/z, fp32 gates, dk = dv = 64, chunk C = 64.
+// pipe_kernels.cuh -- the tcgen05 path of the Key-only GLA (sm_100a): 16-bit
+// q/k/v/z, fp32 gates, dk = dv = 64, chunk C = 64.
 //
 // The three stages of the GTR article's chunkwise operator (方法详解 §4
 // "硬件感知分块推理算子": chunk summaries on tensor cores, a light sequential
-// pass over the chunk-boundary states with coalesced accesses, chunk outputs
-// with the scores kept on chip and the output gate fused into the epilogue),
-// each a kernel over independent work items:
+// pass over boundary states with coalesced accesses, chunk outputs with the
+// scores kept on chip and the output gate fused into the epilogue):
 //
-//   gla_sum_pipe   one item per (sequence, chunk): the chunk's own state
-//                  increment dS_c^T = V^T k^ (k^_j = k_j e^{Gam - G_j}, the
-//                  decay from token j to the chunk end, at most one) and its
-//                  decay factor a_c = e^{Gam}.
-//   gla_chunk_scan the sequential pass: S_c = a_c (.) S_{c-1} + dS_c over the
-//                  chunks of each sequence, per state element, writing the
-//                  state each chunk starts from as the two-term bf16 operand
-//                  tiles the output kernel multiplies.
-//   gla_out_pipe   one item per (sequence, chunk): o = q~ S + mask(q~ k~^T) V
-//                  (q~ = q e^{G}, k~ = k e^{-G}, referenced to the chunk start),
-//                  RMSNorm x w x SiLU(z), stored at the tokens' grid rows.
+//   gla_sum_pipe   per chunk c of a sequence: its state increment
+//                  dS_c^T = V^T k^ (k^_j = k_j e^{Gam - G_j}, the decay from
+//                  token j to the chunk end, at most one) and decay factor
+//                  a_c = e^{Gam}; per segment (a run of consecutive chunks one
+//                  CTA walks): the segment's own map S -> A S + R.
+//   gla_tile_scan  the sequential pass over the segments of each sequence
+//                  (S_in of segment s+1 = A_s (.) S_in + R_s), per state
+//                  element; the same kernel over chunks gives the state after
+//                  every chunk (gtr_gla_chunk_states).
+//   gla_out_pipe   per chunk, in segment order: o = q~ S + mask(q~ k~^T) V
+//                  (q~ = q e^{G}, k~ = k e^{-G}, referenced to the chunk
+//                  start), RMSNorm x w x SiLU(z), stored at the tokens' grid
+//                  rows.  The state entering each chunk is carried in fp32
+//                  registers by the builder warps, S_c = a_c (.) S_{c-1} +
+//                  dS_c, from the segment's entering state, so the only
+//                  sequential step inside a segment is elementwise.
 //
-// Nothing is sequential inside the summary and output kernels, so each is a
-// persistent warp-specialised pipeline: one CTA per SM walks its items
-// (blockIdx.x, + gridDim.x, ...) with a loader warp (tensor-map box loads or
-// cp.async gathers), an MMA warp (one thread issues every tcgen05.mma), eight
-// builder warps (in-chunk cumsum and operand tiles) and four epilogue warps
-// (tensor memory -> registers -> global), hand-offs on mbarriers, and two or
-// four slots of shared and tensor memory so that consecutive items overlap.
+// The summary and output kernels are persistent warp-specialised pipelines:
+// one CTA per SM walks its segments (blockIdx.x, + gridDim.x, ...) chunk by
+// chunk with a loader warp (tensor-map box loads or cp.async gathers), an MMA
+// warp (one thread issues every tcgen05.mma), eight builder warps (in-chunk
+// cumsum, operand tiles, state) and four epilogue warps (tensor memory ->
+// registers -> global), hand-offs on mbarriers, and several slots of shared
+// and tensor memory so that consecutive chunks overlap.
 //
-// State tiles.  For chunk c of sequence bh the workspace holds 16 KB at
-// ((bh * nc) + c) * 16384: two 8 KB halves in the SWIZZLE_128B K-major
-// operand layout of a 64 x 64 16-bit tile whose rows are the value dims j and
-// whose columns are the key dims i (S^T).  The summary kernel writes dS^T in
-// fp32 into the same 16 KB: the 8 values (j, 8u .. 8u+7) of swizzle unit
-// (j, u) go 4 to the first half's unit and 4 to the second half's, so the
-// scan reads and rewrites each unit in place (the bf16 hi term of the 8
-// values into the first half, the lo term into the second), one thread per
-// unit, with no other thread touching it.
+// Staging order.  A chunk's tokens arrive in box order (a reversed scan's box
+// holds the chunk backwards); every operand tile keeps that row order, the
+// builders convert q and k to their operand terms in place, V is the B
+// operand of P V as loaded, and the causal mask compares scan positions
+// (row r of the box is scan offset r ^ rmask), so no tile is ever reordered.
+//
+// State tiles (workspace).  A 64 x 64 fp32 state S^T (rows: value dim j,
+// columns: key dim i) is kept in 16 KB as two 8 KB halves laid out like the
+// SWIZZLE_128B K-major operand tile: the 8 values (j, 8u .. 8u+7) of swizzle
+// unit (j, u) sit 4 in the first half's 16-byte unit and 4 in the second's.
+// The builders read such a tile and write the bf16 terms hi, lo of the same
+// unit to the S^T operand tiles, one thread per unit.
 #pragma once
 #include "tc_kernels.cuh"
 
@@ -67,31 +74,57 @@ __device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, uin
                : "memory");
 }
 
-// Parameters of the pipelined kernels.  Items run over nbh sequences (bh0 ..
-// bh0 + nbh - 1 of the B*H in the tensors) times nc chunks.
-struct PipeParams {
-  const void* q; const void* k; const void* v; const float* g; const void* z; const float* w;
-  uint8_t* st;          // state tiles, 16 KB per (sequence, chunk)
-  float* a;             // chunk decay factors e^{Gam}, 64 per (sequence, chunk)
-  void* out;
-  float* states;        // chunk scan, inclusive fp32 mode: [nbh, nc, 64, 64] (else null)
-  int H, T, gh, gw, dir, nc, bh0, nbh;
-  int tma;              // 1: chunks arrive by tensor-map box loads (Maps valid)
-};
-
-constexpr int kStateTile = 2 * kTile;     // 16 KB per chunk state
+constexpr int kStateTile = 2 * kTile;     // 16 KB per fp32 state tile
 constexpr int kPipeThreads = 14 * 32;     // loader, MMA, 8 builder warps, 4 epilogue warps
 constexpr int kWarpLoad = 0, kWarpMma = 1, kWarpBuild0 = 2, kWarpEpi0 = 10;
 constexpr int kBarBuild = 1, kBarEpi = 2;  // named barriers: builders (256), epilogue warps (128)
 
-// One work item: chunk c of sequence bh (batch b, head h), scan direction d.
-struct Item {
-  int bhl, c, b, h, d, s0, ntok, rmask;
+// Parameters of the summary and output kernels.  Work runs over nbh
+// sequences (bh0 .. bh0 + nbh - 1 of the B*H in the tensors), each split into
+// nseg segments of consecutive chunks (segment s covers chunks
+// [s nc / nseg, (s+1) nc / nseg)).
+struct PipeParams {
+  const void* q; const void* k; const void* v; const float* g; const void* z; const float* w;
+  uint8_t* dS;          // chunk increments, a state tile per (sequence, chunk)
+  float* a;             // chunk decay factors e^{Gam}, 64 per (sequence, chunk)
+  uint8_t* segS;        // segment maps' R, then (after the scan) the states entering the segments
+  float* segA;          // segment decay factors, 64 per (sequence, segment)
+  void* out;
+  int H, T, gh, gw, dir, nc, nseg, bh0, nbh;
+  int tma;              // 1: chunks arrive by tensor-map box loads (Maps valid)
 };
-__device__ __forceinline__ Item pipe_item(const PipeParams& p, int idx) {
+
+// One work item: chunk c of sequence bh (batch b, head h), scan direction d,
+// in segment sg; first / last: the segment's first / last chunk.
+struct Item {
+  int bhl, sg, c, b, h, d, s0, ntok, rmask;
+  bool first, last;
+};
+__device__ __forceinline__ int seg_len(const PipeParams& p, int s) {
+  return seg_first_chunk(s + 1, p.nc, p.nseg) - seg_first_chunk(s, p.nc, p.nseg);
+}
+// Chunks this CTA walks.
+__device__ __forceinline__ int cta_items(const PipeParams& p) {
+  int n = 0;
+  for (int sg = blockIdx.x; sg < p.nbh * p.nseg; sg += gridDim.x) n += seg_len(p, sg % p.nseg);
+  return n;
+}
+// The CTA's n-th chunk.
+__device__ __forceinline__ Item item_at(const PipeParams& p, int n) {
   Item it;
-  it.bhl = idx / p.nc;
-  it.c = idx - it.bhl * p.nc;
+  for (int sg = blockIdx.x;; sg += gridDim.x) {
+    const int bhl = sg / p.nseg, s = sg - bhl * p.nseg;
+    const int c0 = seg_first_chunk(s, p.nc, p.nseg), len = seg_first_chunk(s + 1, p.nc, p.nseg) - c0;
+    if (n < len) {
+      it.bhl = bhl;
+      it.sg = sg;
+      it.c = c0 + n;
+      it.first = n == 0;
+      it.last = n == len - 1;
+      break;
+    }
+    n -= len;
+  }
   const int bh = p.bh0 + it.bhl;
   it.b = bh / p.H;
   it.h = bh - it.b * p.H;
@@ -105,16 +138,11 @@ __device__ __forceinline__ Item pipe_item(const PipeParams& p, int idx) {
 __device__ __forceinline__ long long item_row(const PipeParams& p, const Item& it, int j) {
   return ((long long)it.b * p.T + scan_to_grid(it.d, it.s0 + j, p.T, p.gh, p.gw)) * p.H + it.h;
 }
-// Items of this CTA: blockIdx.x, blockIdx.x + gridDim.x, ...
-__device__ __forceinline__ int pipe_count(int total) {
-  return total > (int)blockIdx.x ? (total - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
-}
-__device__ __forceinline__ int pipe_index(int n) { return (int)blockIdx.x + n * (int)gridDim.x; }
 
 // Gathered chunk rows (no box layout): lane l copies scan offsets l and l + 32
-// of the 16-bit tensors in `which` (bit 0 q, 1 k, 2 v) and of the gate, 16
-// bytes per cp.async; offsets past ntok read zeros.  q, k land row-major, v in
-// the SWIZZLE_128B operand layout; completes on `bar` (an arrive per lane).
+// of the 16-bit tensors in `which` (bit 0 q, 1 k, 2 v) into the SWIZZLE_128B
+// operand layout and of the gate (row-major fp32), 16 bytes per cp.async;
+// offsets past ntok read zeros.  Completes on `bar` (an arrive per lane).
 __device__ __forceinline__ void gather_chunk(const PipeParams& p, const Item& it, int lane, unsigned which,
                                              uint8_t* qdst, uint8_t* kdst, uint8_t* vdst, uint8_t* gdst,
                                              uint64_t* bar) {
@@ -126,9 +154,10 @@ __device__ __forceinline__ void gather_chunk(const PipeParams& p, const Item& it
     const uint32_t nb = ok ? 16u : 0u;
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-      if (which & 1u) cp_async16_zfill(qdst + j * 128 + u * 16, (const uint8_t*)p.q + row * kRowBytes + u * 16, nb);
-      if (which & 2u) cp_async16_zfill(kdst + j * 128 + u * 16, (const uint8_t*)p.k + row * kRowBytes + u * 16, nb);
-      if (which & 4u) cp_async16_zfill(vdst + sw_unit(j, u), (const uint8_t*)p.v + row * kRowBytes + u * 16, nb);
+      const uint32_t o = sw_unit(j, u);
+      if (which & 1u) cp_async16_zfill(qdst + o, (const uint8_t*)p.q + row * kRowBytes + u * 16, nb);
+      if (which & 2u) cp_async16_zfill(kdst + o, (const uint8_t*)p.k + row * kRowBytes + u * 16, nb);
+      if (which & 4u) cp_async16_zfill(vdst + o, (const uint8_t*)p.v + row * kRowBytes + u * 16, nb);
     }
 #pragma unroll
     for (int u = 0; u < 16; ++u)
@@ -148,10 +177,10 @@ __device__ __forceinline__ void box_load(const PipeParams& p, const Maps& mp, in
   }
 }
 
-// In-chunk inclusive cumsum of the staged gate (scan order) for the builder
-// thread's eight scan offsets tb .. tb+7 and dims dc, dc+1: gc[i] = G at
-// offset tb + i; returns the chunk total Gam.  `part` holds the warps'
-// partial sums; one builder barrier.
+// In-chunk inclusive cumsum of the staged gate for the builder thread's eight
+// scan offsets tb .. tb+7 and dims dc, dc+1 (gate row of scan offset i: i ^
+// rmask): gc[i] = G at offset tb + i; returns the chunk total Gam.  `part`
+// holds the warps' partial sums; one builder barrier.
 __device__ __forceinline__ float2 chunk_cumsum(const float* G, float2 (&gc)[8], float (*part)[kD], int bw,
                                                int tb, int dc, int rmask) {
 #pragma unroll
@@ -173,23 +202,38 @@ __device__ __forceinline__ float2 chunk_cumsum(const float* G, float2 (&gc)[8], 
   return tot;
 }
 
+// 8 fp32 values of unit (j, u) of a state tile
+__device__ __forceinline__ void tile_load8(const uint8_t* t, int j, int u, float* x) {
+  const uint32_t o = sw_unit(j, u);
+  const float4 a = *reinterpret_cast<const float4*>(t + o);
+  const float4 b = *reinterpret_cast<const float4*>(t + kTile + o);
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+__device__ __forceinline__ void tile_store8(uint8_t* t, int j, int u, const float* x) {
+  const uint32_t o = sw_unit(j, u);
+  *reinterpret_cast<float4*>(t + o) = make_float4(x[0], x[1], x[2], x[3]);
+  *reinterpret_cast<float4*>(t + kTile + o) = make_float4(x[4], x[5], x[6], x[7]);
+}
+
 // =========================================================== summary (K2)
 struct SumPipeLayout {
   static constexpr int kSlots = 4;
-  // per slot: k (row-major), v (operand layout), k^ hi, lo (operand layout), gate (fp32 rows)
-  static constexpr int kOffK = 0, kOffV = kTile, kOffKH = 2 * kTile, kOffKL = 3 * kTile, kOffG = 4 * kTile;
-  static constexpr int kSlot = 4 * kTile + kGTile;
+  // per slot: k (operand layout; its bf16 / fp16 hi term k^ written in
+  // place), k^ lo, v (operand layout), gate (fp32 rows)
+  static constexpr int kOffKH = 0, kOffKL = kTile, kOffV = 2 * kTile, kOffG = 3 * kTile;
+  static constexpr int kSlot = 3 * kTile + kGTile;
   static constexpr int kMisc = kSlots * kSlot;
   static constexpr int kTmemCols = 256;   // 64 per slot
 };
 struct SumPipeMisc {
   uint64_t full[SumPipeLayout::kSlots];    // the item's k, v, g have landed
-  uint64_t built[SumPipeLayout::kSlots];   // k^ tiles written
-  uint64_t mma[SumPipeLayout::kSlots];     // dS^T product complete (slot's tiles free)
-  uint64_t tfree[SumPipeLayout::kSlots];   // accumulator read out
+  uint64_t built[SumPipeLayout::kSlots];   // k^ tiles and the decay factors written
+  uint64_t mma[SumPipeLayout::kSlots];     // dS^T product complete
+  uint64_t tfree[SumPipeLayout::kSlots];   // accumulator read out (the slot is free)
   uint32_t tmem;
   int abort;
   alignas(16) float part[kWarps][kD];
+  alignas(16) float ac[SumPipeLayout::kSlots][kD];   // the item's e^{Gam}
 };
 constexpr int kSumPipeSmem = SumPipeLayout::kMisc + (int)sizeof(SumPipeMisc) + 1024;
 static_assert(kSumPipeSmem <= 227 * 1024, "summary pipeline must fit one SM");
@@ -204,8 +248,7 @@ gla_sum_pipe(const __grid_constant__ PipeParams p, const __grid_constant__ Maps 
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   SumPipeMisc& m = *reinterpret_cast<SumPipeMisc*>(sm + L::kMisc);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int total = p.nbh * p.nc;
-  const int nit = pipe_count(total);
+  const int nit = cta_items(p);
   const bool tma = p.tma != 0;
 
   if (threadIdx.x == 0) {
@@ -230,15 +273,17 @@ gla_sum_pipe(const __grid_constant__ PipeParams p, const __grid_constant__ Maps 
 
   if (warp == kWarpLoad) {
     // ---- loader: k and v are inputs, their first boxes go out before the
-    // dependency wait; the gate comes from the previous kernel
+    // dependency wait; the gate comes from the previous kernel.  A slot is
+    // refilled once its accumulator has been read out (everything of the
+    // slot's previous item is then complete).
     int issued = 0;
     const int pre = min(nit, NS);
     if (tma && lane == 0) {
       for (int n = 0; n < pre; ++n) {
-        const Item it = pipe_item(p, pipe_index(n));
+        const Item it = item_at(p, n);
         uint8_t* sl = sm + n * L::kSlot;
         mbar_arrive_tx(&m.full[n], 2 * kTile + kGTile);
-        box_load(p, mp, kMapK, sl + L::kOffK, &m.full[n], it);
+        box_load(p, mp, kMapK, sl + L::kOffKH, &m.full[n], it);
         box_load(p, mp, kMapV, sl + L::kOffV, &m.full[n], it);
       }
     }
@@ -247,10 +292,10 @@ gla_sum_pipe(const __grid_constant__ PipeParams p, const __grid_constant__ Maps 
     for (int n = 0; n < nit; ++n) {
       const int s = n % NS, use = n / NS;
       uint8_t* sl = sm + s * L::kSlot;
-      const Item it = pipe_item(p, pipe_index(n));
+      const Item it = item_at(p, n);
       if (n >= NS) {
         bool ok = true;
-        if (lane == 0) ok = mbar_wait(&m.mma[s], (uint32_t)(use - 1) & 1u);
+        if (lane == 0) ok = mbar_wait(&m.tfree[s], (uint32_t)(use - 1) & 1u);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) { failed = true; break; }
       }
@@ -258,13 +303,13 @@ gla_sum_pipe(const __grid_constant__ PipeParams p, const __grid_constant__ Maps 
         if (lane == 0) {
           if (n >= pre) {
             mbar_arrive_tx(&m.full[s], 2 * kTile + kGTile);
-            box_load(p, mp, kMapK, sl + L::kOffK, &m.full[s], it);
+            box_load(p, mp, kMapK, sl + L::kOffKH, &m.full[s], it);
             box_load(p, mp, kMapV, sl + L::kOffV, &m.full[s], it);
           }
           box_load(p, mp, kMapG, sl + L::kOffG, &m.full[s], it);
         }
       } else {
-        gather_chunk(p, it, lane, 6u, nullptr, sl + L::kOffK, sl + L::kOffV, sl + L::kOffG, &m.full[s]);
+        gather_chunk(p, it, lane, 6u, nullptr, sl + L::kOffKH, sl + L::kOffV, sl + L::kOffG, &m.full[s]);
       }
       issued = n + 1;
       // (items before `pre` had their k, v boxes issued before the wait: their
@@ -276,6 +321,7 @@ gla_sum_pipe(const __grid_constant__ PipeParams p, const __grid_constant__ Maps 
       for (int n = max(0, issued - NS); n < issued; ++n)
         if (!mbar_wait(&m.full[n % NS], (uint32_t)(n / NS) & 1u)) failed = true;
     if (!tma) cp_async_wait<0>();
+    if (failed && lane == 0) m.abort = 1;
   } else if (warp == kWarpMma) {
     constexpr uint32_t kIdVK = kH ? idesc_f16(1, 1) : idesc_bf16(1, 1);   // both MN-major
     int issued = 0;
@@ -284,7 +330,6 @@ gla_sum_pipe(const __grid_constant__ PipeParams p, const __grid_constant__ Maps 
         const int s = n % NS, use = n / NS;
         uint8_t* sl = sm + s * L::kSlot;
         if (!mbar_wait(&m.built[s], (uint32_t)use & 1u)) { failed = true; break; }
-        if (use > 0 && !mbar_wait(&m.tfree[s], (uint32_t)(use - 1) & 1u)) { failed = true; break; }
         tc_after_sync();
         // dS^T = V^T k^ (rows dv, columns dk): A = V, B = k^ hi then lo, both MN-major
         const uint32_t d = tm + 64u * (uint32_t)s;
@@ -294,73 +339,92 @@ gla_sum_pipe(const __grid_constant__ PipeParams p, const __grid_constant__ Maps 
         issued = n + 1;
       }
       if (issued > 0 && !mbar_wait(&m.mma[(issued - 1) % NS], (uint32_t)((issued - 1) / NS) & 1u)) failed = true;
+      if (failed) m.abort = 1;
     }
   } else if (warp < kWarpEpi0) {
-    // ---- builders: cumsum, weights e^{Gam - G_j}, k^ two-term (rows in the
-    // staging order, which V shares, so no reordering in any scan order)
+    // ---- builders: cumsum, weights e^{Gam - G_j}, k^ = k e^{Gam - G} as two
+    // terms (fp16 for fp16 inputs, bf16 for bf16), rows in the staging order
+    // V shares, so no reordering in any scan order
     pdl_wait();
     pdl_trigger();
     const int bt = threadIdx.x - 32 * kWarpBuild0, bw = bt >> 5;
     const int dc = 2 * lane, tb = 8 * bw;
+    float2 segA = make_float2(1.f, 1.f);  // the segment's decay so far (builder warp 0)
     for (int n = 0; n < nit; ++n) {
       const int s = n % NS, use = n / NS;
       uint8_t* sl = sm + s * L::kSlot;
-      const Item it = pipe_item(p, pipe_index(n));
+      const Item it = item_at(p, n);
       failed |= !mbar_wait(&m.full[s], (uint32_t)use & 1u);
       if (named_barrier_or(kBarBuild, kThreads, failed || aborted(&m.abort))) { failed = true; break; }
       float2 gc[8];
       const float2 tot = chunk_cumsum(reinterpret_cast<const float*>(sl + L::kOffG), gc, m.part, bw, tb, dc,
                                       it.rmask);
-      const T* kst = reinterpret_cast<const T*>(sl + L::kOffK);
       uint8_t* KH = sl + L::kOffKH;
+      uint32_t kr[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) kr[i] = *reinterpret_cast<const uint32_t*>(KH + sw16((tb + i) ^ it.rmask, dc));
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const int rs = (tb + i) ^ it.rmask;
-        const uint32_t o = sw16(rs, dc);
-        const float2 kk = ld2(kst + rs * kD + dc);
+        const uint32_t o = sw16((tb + i) ^ it.rmask, dc);
+        const float2 kk = ld2(reinterpret_cast<const T*>(&kr[i]));
         const float wa = ex2((tot.x - gc[i].x) * kLog2e), wb = ex2((tot.y - gc[i].y) * kLog2e);
         if (kH) put2h(KH, KH + kTile, o, kk.x * wa, kk.y * wb);
         else put2x(KH, KH + kTile, o, kk.x * wa, kk.y * wb);
       }
-      if (bw == 0)
-        *reinterpret_cast<float2*>(p.a + ((size_t)it.bhl * p.nc + it.c) * kD + dc) =
-            make_float2(expf(tot.x), expf(tot.y));
+      if (bw == 0) {
+        const float2 ea = make_float2(expf(tot.x), expf(tot.y));
+        *reinterpret_cast<float2*>(&m.ac[s][dc]) = ea;
+        *reinterpret_cast<float2*>(p.a + ((size_t)it.bhl * p.nc + it.c) * kD + dc) = ea;
+        segA = it.first ? ea : make_float2(segA.x * ea.x, segA.y * ea.y);
+        if (it.last) *reinterpret_cast<float2*>(p.segA + (size_t)it.sg * kD + dc) = segA;
+      }
       fence_async_smem();
       named_barrier(kBarBuild, kThreads);   // tiles written; partials read
       if (bt == 0) mbar_arrive_one(&m.built[s]);
     }
     if (failed && bt == 0) m.abort = 1;
   } else {
-    // ---- epilogue warps: dS^T from tensor memory into the state tile
+    // ---- epilogue warps: dS^T from tensor memory into the chunk's state
+    // tile, and the segment's map S -> A S + R accumulated in registers
+    // (thread: row `row`, key dims c0 .. c0+15 and c1 .. c1+15)
     pdl_wait();
     pdl_trigger();
     const int qd = warp & 3;
     const int row = qd * 16 + (lane & 15), ch = lane >> 4;
+    const int c0 = 16 * ch, c1 = 32 + 16 * ch;
     const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
+    float R[32];
     for (int n = 0; n < nit; ++n) {
       const int s = n % NS, use = n / NS;
-      const Item it = pipe_item(p, pipe_index(n));
+      const Item it = item_at(p, n);
       failed |= !mbar_wait(&m.mma[s], (uint32_t)use & 1u);
+      failed |= !mbar_wait(&m.built[s], (uint32_t)use & 1u);   // the decay factors in m.ac
       if (named_barrier_or(kBarEpi, 128, failed || aborted(&m.abort))) { failed = true; break; }
       tc_after_sync();
-      float v0[16], v1[16];
-      tmem_ld16x2(tm + 64u * (uint32_t)s + lane_base, v0);
-      tmem_ld16x2(tm + 64u * (uint32_t)s + lane_base + 32, v1);
-      tmem_ld_wait(v0);
-      tmem_ld_wait(v1);
+      float v[32];
+      tmem_ld16x2(tm + 64u * (uint32_t)s + lane_base, v);
+      tmem_ld16x2(tm + 64u * (uint32_t)s + lane_base + 32, v + 16);
+      tmem_ld_wait(*reinterpret_cast<float(*)[16]>(v));
+      tmem_ld_wait(*reinterpret_cast<float(*)[16]>(v + 16));
       tc_before_sync();
       named_barrier(kBarEpi, 128);
       if (warp == kWarpEpi0 && lane == 0) mbar_arrive_one(&m.tfree[s]);
-      // columns (key dims) ch*16 .. +15 from v0 and 32 + ch*16 .. +15 from v1:
-      // units u = 2 ch, 2 ch + 1, 4 + 2 ch, 5 + 2 ch of row `row`
-      uint8_t* dst = p.st + ((size_t)it.bhl * p.nc + it.c) * kStateTile;
+      // units 2ch, 2ch + 1 (columns c0 ..) and 4 + 2ch, 5 + 2ch (columns c1 ..)
+      uint8_t* dst = p.dS + ((size_t)it.bhl * p.nc + it.c) * kStateTile;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float* x = q < 2 ? v0 + 8 * q : v1 + 8 * (q - 2);
-        const int u = (q < 2 ? 0 : 4) + 2 * ch + (q & 1);
-        const uint32_t o = sw_unit(row, u);
-        *reinterpret_cast<float4*>(dst + o) = make_float4(x[0], x[1], x[2], x[3]);
-        *reinterpret_cast<float4*>(dst + kTile + o) = make_float4(x[4], x[5], x[6], x[7]);
+      for (int q = 0; q < 4; ++q) tile_store8(dst, row, (q < 2 ? 0 : 4) + 2 * ch + (q & 1), v + 8 * q);
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) {
+        const float4 ea = *reinterpret_cast<const float4*>(&m.ac[s][(e < 16 ? c0 : c1 - 16) + e]);
+        R[e] = it.first ? v[e] : fmaf(ea.x, R[e], v[e]);
+        R[e + 1] = it.first ? v[e + 1] : fmaf(ea.y, R[e + 1], v[e + 1]);
+        R[e + 2] = it.first ? v[e + 2] : fmaf(ea.z, R[e + 2], v[e + 2]);
+        R[e + 3] = it.first ? v[e + 3] : fmaf(ea.w, R[e + 3], v[e + 3]);
+      }
+      if (it.last) {
+        uint8_t* sdst = p.segS + (size_t)it.sg * kStateTile;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tile_store8(sdst, row, (q < 2 ? 0 : 4) + 2 * ch + (q & 1), R + 8 * q);
       }
     }
     if (failed && threadIdx.x == 32 * kWarpEpi0) m.abort = 1;
@@ -372,104 +436,129 @@ gla_sum_pipe(const __grid_constant__ PipeParams p, const __grid_constant__ Maps 
   if (warp == kWarpLoad) tmem_dealloc(tm, L::kTmemCols);
 }
 
-// ======================================================= chunk scan (K3)
-// Block = one (sequence, value dim j): 8 units u (key dims 8u .. 8u+7) x 32
-// ranges of consecutive chunks.  Each thread reduces its range to an affine
-// map S -> P (.) S + R, the ranges exchange maps through shared memory, and
-// each replays its range from the composed entering state, writing the state
-// each chunk starts from (two-term bf16, in place) or, in inclusive fp32 mode,
-// the state each chunk ends with into p.states.
+// ====================================================== tile scan (K3)
+// For every sequence and state element, the affine recurrence over the
+// sequence's n items (segments, or chunks):
+//     S_0 = 0,   S_{m+1} = a_m (.) S_m + R_m      (a_m per key dim i)
+// `inclusive` = 0: S_m (the state entering item m) overwrites R_m in place;
+// 1: S_{m+1} (the state after item m) goes to states[nbh, n, 64 (i), 64 (j)]
+// fp32.  Block = one (sequence, value dim j): 8 units u (key dims 8u .. 8u+7)
+// x 32 ranges of consecutive items.  Each thread reduces its range to a map
+// S -> P (.) S + Q, warp u scans the 32 ranges' maps with shuffles, and each
+// range replays its items from the composed entering state.
+struct ScanParams {
+  uint8_t* st;          // [nbh][n] state tiles (R_m)
+  const float* a;       // [nbh][n][64]
+  float* states;        // inclusive output or null
+  int n, inclusive;
+};
 constexpr int kScanRanges = 32;
-constexpr int kChunkScanThreads = 8 * kScanRanges;
-constexpr int kScanWin = 4;
+constexpr int kTileScanThreads = 8 * kScanRanges;
+constexpr int kScanWin = 2;
 
-__global__ void __launch_bounds__(kChunkScanThreads)
-gla_chunk_scan(const __grid_constant__ PipeParams p) {
-  __shared__ float4 mapP[kScanRanges][8][2], mapR[kScanRanges][8][2];
+__global__ void __launch_bounds__(kTileScanThreads, 3)
+gla_tile_scan(const __grid_constant__ ScanParams p) {
+  // [range][unit]: first the ranges' maps (P, Q), then the state entering each range
+  __shared__ float4 mapP[kScanRanges][8][2], mapQ[kScanRanges][8][2];
   pdl_wait();
   pdl_trigger();
   const int u = threadIdx.x & 7, part = threadIdx.x >> 3;
   const int bhl = blockIdx.x >> 6, j = blockIdx.x & 63;
-  const int len = (p.nc + kScanRanges - 1) / kScanRanges;
-  const int ca = min(p.nc, part * len), cb = min(p.nc, ca + len);
-  uint8_t* base = p.st + (size_t)bhl * p.nc * kStateTile;
-  const float* abase = p.a + (size_t)bhl * p.nc * kD + 8 * u;
-  const uint32_t o = sw_unit(j, u);
+  const int len = (p.n + kScanRanges - 1) / kScanRanges;
+  const int ca = min(p.n, part * len), cb = min(p.n, ca + len);
+  uint8_t* base = p.st + (size_t)bhl * p.n * kStateTile;
+  const float* abase = p.a + (size_t)bhl * p.n * kD + 8 * u;
 
-  float P[8], R[8];
+  float P[8], Q[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) { P[e] = 1.f; R[e] = 0.f; }
+  for (int e = 0; e < 8; ++e) { P[e] = 1.f; Q[e] = 0.f; }
   for (int c0 = ca; c0 < cb; c0 += kScanWin) {
-    float4 d[kScanWin][2], a[kScanWin][2];
+    float d[kScanWin][8], a[kScanWin][8];
 #pragma unroll
     for (int w = 0; w < kScanWin; ++w) {
       if (c0 + w < cb) {
-        const uint8_t* t = base + (size_t)(c0 + w) * kStateTile;
-        d[w][0] = *reinterpret_cast<const float4*>(t + o);
-        d[w][1] = *reinterpret_cast<const float4*>(t + kTile + o);
-        a[w][0] = *reinterpret_cast<const float4*>(abase + (size_t)(c0 + w) * kD);
-        a[w][1] = *reinterpret_cast<const float4*>(abase + (size_t)(c0 + w) * kD + 4);
+        tile_load8(base + (size_t)(c0 + w) * kStateTile, j, u, d[w]);
+        const float4 a0 = *reinterpret_cast<const float4*>(abase + (size_t)(c0 + w) * kD);
+        const float4 a1 = *reinterpret_cast<const float4*>(abase + (size_t)(c0 + w) * kD + 4);
+        a[w][0] = a0.x; a[w][1] = a0.y; a[w][2] = a0.z; a[w][3] = a0.w;
+        a[w][4] = a1.x; a[w][5] = a1.y; a[w][6] = a1.z; a[w][7] = a1.w;
       }
     }
 #pragma unroll
     for (int w = 0; w < kScanWin; ++w) {
       if (c0 + w < cb) {
-        const float dd[8] = {d[w][0].x, d[w][0].y, d[w][0].z, d[w][0].w, d[w][1].x, d[w][1].y, d[w][1].z, d[w][1].w};
-        const float aa[8] = {a[w][0].x, a[w][0].y, a[w][0].z, a[w][0].w, a[w][1].x, a[w][1].y, a[w][1].z, a[w][1].w};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) { R[e] = fmaf(aa[e], R[e], dd[e]); P[e] *= aa[e]; }
+        for (int e = 0; e < 8; ++e) { Q[e] = fmaf(a[w][e], Q[e], d[w][e]); P[e] *= a[w][e]; }
       }
     }
   }
   mapP[part][u][0] = make_float4(P[0], P[1], P[2], P[3]);
   mapP[part][u][1] = make_float4(P[4], P[5], P[6], P[7]);
-  mapR[part][u][0] = make_float4(R[0], R[1], R[2], R[3]);
-  mapR[part][u][1] = make_float4(R[4], R[5], R[6], R[7]);
+  mapQ[part][u][0] = make_float4(Q[0], Q[1], Q[2], Q[3]);
+  mapQ[part][u][1] = make_float4(Q[4], Q[5], Q[6], Q[7]);
+  __syncthreads();
+  {
+    // warp w composes the 32 ranges' maps of unit w, lane = range: an
+    // inclusive scan of S -> P S + Q (the later map applied after the
+    // earlier); the state entering range r is the composed Q of ranges 0 .. r-1
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float cp[8], cq[8];
+    {
+      const float4 p0 = mapP[lane][w][0], p1 = mapP[lane][w][1], q0 = mapQ[lane][w][0], q1 = mapQ[lane][w][1];
+      cp[0] = p0.x; cp[1] = p0.y; cp[2] = p0.z; cp[3] = p0.w; cp[4] = p1.x; cp[5] = p1.y; cp[6] = p1.z; cp[7] = p1.w;
+      cq[0] = q0.x; cq[1] = q0.y; cq[2] = q0.z; cq[3] = q0.w; cq[4] = q1.x; cq[5] = q1.y; cq[6] = q1.z; cq[7] = q1.w;
+    }
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float pp = __shfl_up_sync(0xffffffffu, cp[e], off);
+        const float qq = __shfl_up_sync(0xffffffffu, cq[e], off);
+        if (lane >= off) { cq[e] = fmaf(cp[e], qq, cq[e]); cp[e] *= pp; }
+      }
+    }
+    float sin[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      sin[e] = __shfl_up_sync(0xffffffffu, cq[e], 1);
+      if (lane == 0) sin[e] = 0.f;
+    }
+    __syncthreads();                      // every map read before the entering states overwrite them
+    mapQ[lane][w][0] = make_float4(sin[0], sin[1], sin[2], sin[3]);
+    mapQ[lane][w][1] = make_float4(sin[4], sin[5], sin[6], sin[7]);
+  }
   __syncthreads();
   float S[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) S[e] = 0.f;
-  for (int r = 0; r < part; ++r) {
-    const float4 p0 = mapP[r][u][0], p1 = mapP[r][u][1], r0 = mapR[r][u][0], r1 = mapR[r][u][1];
-    const float pp[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-    const float rr[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-#pragma unroll
-    for (int e = 0; e < 8; ++e) S[e] = fmaf(pp[e], S[e], rr[e]);
+  {
+    const float4 s0 = mapQ[part][u][0], s1 = mapQ[part][u][1];
+    S[0] = s0.x; S[1] = s0.y; S[2] = s0.z; S[3] = s0.w; S[4] = s1.x; S[5] = s1.y; S[6] = s1.z; S[7] = s1.w;
   }
   for (int c0 = ca; c0 < cb; c0 += kScanWin) {
-    float4 d[kScanWin][2], a[kScanWin][2];
+    float d[kScanWin][8], a[kScanWin][8];
 #pragma unroll
     for (int w = 0; w < kScanWin; ++w) {
       if (c0 + w < cb) {
-        const uint8_t* t = base + (size_t)(c0 + w) * kStateTile;
-        d[w][0] = *reinterpret_cast<const float4*>(t + o);
-        d[w][1] = *reinterpret_cast<const float4*>(t + kTile + o);
-        a[w][0] = *reinterpret_cast<const float4*>(abase + (size_t)(c0 + w) * kD);
-        a[w][1] = *reinterpret_cast<const float4*>(abase + (size_t)(c0 + w) * kD + 4);
+        tile_load8(base + (size_t)(c0 + w) * kStateTile, j, u, d[w]);
+        const float4 a0 = *reinterpret_cast<const float4*>(abase + (size_t)(c0 + w) * kD);
+        const float4 a1 = *reinterpret_cast<const float4*>(abase + (size_t)(c0 + w) * kD + 4);
+        a[w][0] = a0.x; a[w][1] = a0.y; a[w][2] = a0.z; a[w][3] = a0.w;
+        a[w][4] = a1.x; a[w][5] = a1.y; a[w][6] = a1.z; a[w][7] = a1.w;
       }
     }
 #pragma unroll
     for (int w = 0; w < kScanWin; ++w) {
       if (c0 + w < cb) {
         const int c = c0 + w;
-        const float dd[8] = {d[w][0].x, d[w][0].y, d[w][0].z, d[w][0].w, d[w][1].x, d[w][1].y, d[w][1].z, d[w][1].w};
-        const float aa[8] = {a[w][0].x, a[w][0].y, a[w][0].z, a[w][0].w, a[w][1].x, a[w][1].y, a[w][1].z, a[w][1].w};
-        if (p.states) {
+        if (p.inclusive) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) S[e] = fmaf(aa[e], S[e], dd[e]);
-          float* dst = p.states + ((size_t)bhl * p.nc + c) * (kD * kD) + (size_t)(8 * u) * kD + j;
+          for (int e = 0; e < 8; ++e) S[e] = fmaf(a[w][e], S[e], d[w][e]);
+          float* dst = p.states + ((size_t)bhl * p.n + c) * (kD * kD) + (size_t)(8 * u) * kD + j;
 #pragma unroll
           for (int e = 0; e < 8; ++e) dst[e * kD] = S[e];
         } else {
-          // the state the chunk starts from, as the bf16 terms hi + lo
-          uint32_t hi[4], lo[4];
+          tile_store8(base + (size_t)c * kStateTile, j, u, S);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) split2(S[2 * e], S[2 * e + 1], hi[e], lo[e]);
-          uint8_t* t = base + (size_t)c * kStateTile;
-          *reinterpret_cast<uint4*>(t + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-          *reinterpret_cast<uint4*>(t + kTile + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) S[e] = fmaf(aa[e], S[e], dd[e]);
+          for (int e = 0; e < 8; ++e) S[e] = fmaf(a[w][e], S[e], d[w][e]);
         }
       }
     }
@@ -478,62 +567,56 @@ gla_chunk_scan(const __grid_constant__ PipeParams p) {
 
 // =========================================================== output (K4)
 struct OutPipeLayout {
-  // per slot, operand tiles (1024-aligned): S^T hi, k~ hi, S^T lo, k~ lo, q~
-  // hi, lo, V hi, lo; [S^T; k~] hi and lo are each one 128-row K-major B
+  static constexpr int kSlots = 3;
+  // per slot (1024-aligned tiles): S^T hi, k (operand layout; k~ hi in
+  // place), S^T lo, k~ lo, q (q~ hi in place), q~ lo, v (the B operand of
+  // P V), gate (fp32 rows).  [S^T; k~] hi and lo are each one 128-row K-major B.
   static constexpr int kSH = 0, kKH = kTile, kSL = 2 * kTile, kKL = 3 * kTile, kQH = 4 * kTile,
-                       kQL = 5 * kTile, kVH = 6 * kTile, kVL = 7 * kTile;
-  static constexpr int kOp = 8 * kTile;
-  // per slot, staging: q, k (row-major), v (operand layout), gate (fp32 rows)
-  static constexpr int kRq = 0, kRk = kTile, kRv = 2 * kTile, kRg = 3 * kTile;
-  static constexpr int kRaw = 3 * kTile + kGTile;
-  static constexpr int kOffRaw = 2 * kOp;
-  static constexpr int kMisc = 2 * kOp + 2 * kRaw;
-  // tensor memory per slot (256 columns): o [0, 64), scores [64, 128), P hi [128, 160), P lo [160, 192)
+                       kQL = 5 * kTile, kV = 6 * kTile, kG = 7 * kTile;
+  static constexpr int kSlot = 7 * kTile + kGTile;
+  static constexpr int kMisc = kSlots * kSlot;
+  // tensor memory per slot (128 columns): o [0, 64), the scores [64, 128),
+  // overwritten in place by P (hi [64, 96), lo [96, 128))
   static constexpr int kTmemCols = 512;
 };
 struct OutPipeMisc {
-  uint64_t full[2];     // staging landed
-  uint64_t sfull[2];    // state tiles (and a direct v) landed
-  uint64_t rawfree[2];  // builders done with the staging
-  uint64_t built[2];    // q~, k~, V tiles written
-  uint64_t mma1[2];     // q~ [S^T; k~]^T complete
-  uint64_t pready[2];   // P written (tensor memory, or the q~ tiles for an exact chunk)
-  uint64_t mma2[2];     // P V complete (the slot's operand tiles are free)
-  uint64_t tfree[2];    // o read out (the slot's tensor memory is free)
+  uint64_t full[OutPipeLayout::kSlots];     // q, k, v, g landed
+  uint64_t built[OutPipeLayout::kSlots];    // q~, k~, S^T tiles written
+  uint64_t mma1[OutPipeLayout::kSlots];     // q~ [S^T; k~]^T complete
+  uint64_t pready[OutPipeLayout::kSlots];   // P in tensor memory
+  uint64_t mma2[OutPipeLayout::kSlots];     // P V complete
+  uint64_t tfree[OutPipeLayout::kSlots];    // o read out (the slot is free)
   uint32_t tmem;
   int abort;
-  int exact[2];
+  int exact[OutPipeLayout::kSlots];
   alignas(16) float part[kWarps][kD];
   alignas(16) float wv[kD];
+  alignas(16) float ac[OutPipeLayout::kSlots][kD];   // the chunk's e^{Gam}
 };
 constexpr int kOutPipeSmem = OutPipeLayout::kMisc + (int)sizeof(OutPipeMisc) + 1024;
 static_assert(kOutPipeSmem <= 227 * 1024, "output pipeline must fit one SM");
 
-// A bf16 v read in scan order by a box load lands in the V operand tile itself.
-__device__ __forceinline__ bool v_direct(bool two_term_v, bool tma, const Item& it) {
-  return !two_term_v && tma && it.rmask == 0;
-}
+// |q|, |k| below this keep every unmasked score below 2^15 in magnitude
+// (64 x 22 x 22 < 2^15; the decay factors of an unmasked pair are at most
+// one), so P fits the fp16 terms of P V for fp16 inputs.
+constexpr float kQKMaxF16 = 22.0f;
 
 template <typename T>
 __global__ void __launch_bounds__(kPipeThreads, 1)
 gla_out_pipe(const __grid_constant__ PipeParams p, const __grid_constant__ Maps mp) {
   using L = OutPipeLayout;
-  constexpr bool kV2 = std::is_same<T, __half>::value;   // fp16 V: two bf16 terms
+  constexpr int NS = L::kSlots;
+  constexpr bool kH = std::is_same<T, __half>::value;   // P V in fp16 terms (else bf16)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   OutPipeMisc& m = *reinterpret_cast<OutPipeMisc*>(sm + L::kMisc);
-  auto op = [&](int s) -> uint8_t* { return sm + s * L::kOp; };
-  auto raw = [&](int s) -> uint8_t* { return sm + L::kOffRaw + s * L::kRaw; };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int total = p.nbh * p.nc;
-  const int nit = pipe_count(total);
+  const int nit = cta_items(p);
   const bool tma = p.tma != 0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(&m.full[s], tma ? 1 : 32);
-      mbar_init(&m.sfull[s], 1);
-      mbar_init(&m.rawfree[s], 1);
       mbar_init(&m.built[s], 1);
       mbar_init(&m.mma1[s], 1);
       mbar_init(&m.pready[s], 1);
@@ -555,110 +638,66 @@ gla_out_pipe(const __grid_constant__ PipeParams p, const __grid_constant__ Maps 
   bool failed = false;
 
   if (warp == kWarpLoad) {
-    // ---- loader.  q, k, v, g are complete before the scan kernel lets this
-    // one start, so staging loads need no wait; the state tiles do.
-    int nr = 0, ns = 0;
-    bool waited = false;
-    unsigned long long t_idle = 0;
-    while (ns < nit) {
-      bool progressed = false;
-      if (nr < nit) {
-        const int s = nr & 1, use = nr >> 1;
-        bool ok = use == 0 || (lane == 0 && mbar_test(&m.rawfree[s], (uint32_t)(use - 1) & 1u));
+    // ---- loader: q, k, v, g of chunk n into slot n % 3, once the slot's
+    // previous chunk has been read out.  They are inputs, complete before the
+    // scan kernel let this one start.
+    int issued = 0;
+    for (int n = 0; n < nit; ++n) {
+      const int s = n % NS, use = n / NS;
+      uint8_t* sl = sm + s * L::kSlot;
+      if (n >= NS) {
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait(&m.tfree[s], (uint32_t)(use - 1) & 1u);
         ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (ok) {
-          const Item it = pipe_item(p, pipe_index(nr));
-          uint8_t* r = raw(s);
-          const bool vd = v_direct(kV2, tma, it);
-          if (tma) {
-            if (lane == 0) {
-              mbar_arrive_tx(&m.full[s], 2 * kTile + kGTile + (vd ? 0 : kTile));
-              box_load(p, mp, kMapQ, r + L::kRq, &m.full[s], it);
-              box_load(p, mp, kMapK, r + L::kRk, &m.full[s], it);
-              if (!vd) box_load(p, mp, kMapV, r + L::kRv, &m.full[s], it);
-              box_load(p, mp, kMapG, r + L::kRg, &m.full[s], it);
-            }
-          } else {
-            gather_chunk(p, it, lane, 7u, r + L::kRq, r + L::kRk, r + L::kRv, r + L::kRg, &m.full[s]);
-          }
-          ++nr;
-          progressed = true;
-        }
+        if (!ok || __shfl_sync(0xffffffffu, aborted(&m.abort), 0)) { failed = true; break; }
       }
-      if (ns < nr) {
-        const int s = ns & 1, use = ns >> 1;
-        bool ok = use == 0 || (lane == 0 && mbar_test(&m.mma2[s], (uint32_t)(use - 1) & 1u));
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (ok) {
-          if (!waited) {
-            pdl_wait();                   // the state tiles come from the scan kernel
-            pdl_trigger();
-            waited = true;
-          }
-          const Item it = pipe_item(p, pipe_index(ns));
-          if (lane == 0) {
-            const bool vd = v_direct(kV2, tma, it);
-            const uint8_t* src = p.st + ((size_t)it.bhl * p.nc + it.c) * kStateTile;
-            mbar_arrive_tx(&m.sfull[s], kStateTile + (vd ? kTile : 0));
-            bulk_g2s(op(s) + L::kSH, src, kTile, &m.sfull[s]);
-            bulk_g2s(op(s) + L::kSL, src + kTile, kTile, &m.sfull[s]);
-            if (vd) box_load(p, mp, kMapV, op(s) + L::kVH, &m.sfull[s], it);
-          }
-          ++ns;
-          progressed = true;
+      const Item it = item_at(p, n);
+      if (tma) {
+        if (lane == 0) {
+          mbar_arrive_tx(&m.full[s], 3 * kTile + kGTile);
+          box_load(p, mp, kMapQ, sl + L::kQH, &m.full[s], it);
+          box_load(p, mp, kMapK, sl + L::kKH, &m.full[s], it);
+          box_load(p, mp, kMapV, sl + L::kV, &m.full[s], it);
+          box_load(p, mp, kMapG, sl + L::kG, &m.full[s], it);
         }
-      }
-      if (progressed) {
-        t_idle = 0;
       } else {
-        if (__shfl_sync(0xffffffffu, aborted(&m.abort), 0)) { failed = true; break; }
-        const unsigned long long now = globaltimer();
-        if (t_idle == 0) t_idle = now;
-        else if (now - t_idle > kWaitNs) { failed = true; break; }
+        gather_chunk(p, it, lane, 7u, sl + L::kQH, sl + L::kKH, sl + L::kV, sl + L::kG, &m.full[s]);
       }
+      issued = n + 1;
     }
-    if (!waited) { pdl_wait(); pdl_trigger(); }
-    // every copy issued lands before the CTA leaves
-    if (lane == 0) {
-      for (int n = max(0, nr - 2); n < nr; ++n)
-        if (!mbar_wait(&m.full[n & 1], (uint32_t)(n >> 1) & 1u)) failed = true;
-      for (int n = max(0, ns - 2); n < ns; ++n)
-        if (!mbar_wait(&m.sfull[n & 1], (uint32_t)(n >> 1) & 1u)) failed = true;
-    }
+    if (lane == 0)
+      for (int n = max(0, issued - NS); n < issued; ++n)
+        if (!mbar_wait(&m.full[n % NS], (uint32_t)(n / NS) & 1u)) failed = true;
     if (!tma) cp_async_wait<0>();
     if (failed && lane == 0) m.abort = 1;
   } else if (warp == kWarpMma) {
     if (lane == 0) {
       constexpr uint32_t kIdQSK = idesc_bf16(0, 0, 128);   // both K-major, N = 128: q~ [S^T; k~]^T
-      constexpr uint32_t kIdPV = idesc_bf16(0, 1);          // A K-major, B MN-major: P V
+      constexpr uint32_t kIdQS = idesc_bf16(0, 0);          // q~ S alone (an exact chunk)
+      constexpr uint32_t kIdPV = kH ? idesc_f16(0, 1) : idesc_bf16(0, 1);   // A in tensor memory, B MN-major
       int n1 = 0, n2 = 0;
       unsigned long long t_idle = 0;
       while (n2 < nit) {
         bool progressed = false;
         if (n1 < nit) {
-          const int s = n1 & 1, use = n1 >> 1;
-          if (mbar_test(&m.built[s], (uint32_t)use & 1u) && mbar_test(&m.sfull[s], (uint32_t)use & 1u) &&
-              (use == 0 || mbar_test(&m.tfree[s], (uint32_t)(use - 1) & 1u))) {
+          const int s = n1 % NS, use = n1 / NS;
+          if (mbar_test(&m.built[s], (uint32_t)use & 1u)) {
             tc_after_sync();
-            uint8_t* o = op(s);
-            mma_terms<kStepK, kStepK>(tm + 256u * s, desc_k(o + L::kQH), desc_k(o + L::kQL),
-                                      desc_k(o + L::kSH), desc_k(o + L::kSL), true, kIdQSK, false);
+            uint8_t* o = sm + s * L::kSlot;
+            mma_terms<kStepK, kStepK>(tm + 128u * s, desc_k(o + L::kQH), desc_k(o + L::kQL), desc_k(o + L::kSH),
+                                      desc_k(o + L::kSL), true, m.exact[s] ? kIdQS : kIdQSK, false);
             mma_commit(&m.mma1[s]);
             ++n1;
             progressed = true;
           }
         }
         if (n2 < n1) {
-          const int s = n2 & 1, use = n2 >> 1;
+          const int s = n2 % NS, use = n2 / NS;
           if (mbar_test(&m.pready[s], (uint32_t)use & 1u)) {
             tc_after_sync();
-            uint8_t* o = op(s);
-            const uint32_t d = tm + 256u * s;
-            const uint64_t vh = desc_mn(o + L::kVH), vl = desc_mn(o + L::kVL);
-            if (!m.exact[s])
-              mma_terms_ts<kStepMN>(d, d + 128, d + 160, vh, vl, kV2, kIdPV);
-            else   // an exact chunk's P is in the q~ tiles
-              mma_terms<kStepK, kStepMN>(d, desc_k(o + L::kQH), desc_k(o + L::kQL), vh, vl, kV2, kIdPV, true);
+            const uint32_t d = tm + 128u * s;
+            // o += P V: P hi, lo in tensor memory, V one exact term
+            mma_terms_ts<kStepMN>(d, d + 64, d + 96, desc_mn(sm + s * L::kSlot + L::kV), 0, false, kIdPV);
             mma_commit(&m.mma2[s]);
             ++n2;
             progressed = true;
@@ -671,184 +710,187 @@ gla_out_pipe(const __grid_constant__ PipeParams p, const __grid_constant__ Maps 
           const unsigned long long now = globaltimer();
           if (t_idle == 0) t_idle = now;
           else if (now - t_idle > kWaitNs) { failed = true; break; }
+          __nanosleep(32);
         }
       }
       // the last products complete before tensor memory is released
-      if (n1 > n2 && !mbar_wait(&m.mma1[(n1 - 1) & 1], (uint32_t)((n1 - 1) >> 1) & 1u)) failed = true;
-      if (n2 > 0 && !mbar_wait(&m.mma2[(n2 - 1) & 1], (uint32_t)((n2 - 1) >> 1) & 1u)) failed = true;
+      if (n1 > n2 && !mbar_wait(&m.mma1[(n1 - 1) % NS], (uint32_t)((n1 - 1) / NS) & 1u)) failed = true;
+      if (n2 > 0 && !mbar_wait(&m.mma2[(n2 - 1) % NS], (uint32_t)((n2 - 1) / NS) & 1u)) failed = true;
       if (failed) m.abort = 1;
     }
   } else if (warp < kWarpEpi0) {
-    // ---- builders: cumsum, exact-chunk test, q~ = q e^{G}, k~ = k e^{-G}
-    // and V as two-term bf16 operand tiles in scan order
+    // ---- builders.  Per chunk: the state entering it as two-term bf16 S^T
+    // tiles, the in-chunk cumsum and exact-chunk test, q~ = q e^{G}, k~ = k
+    // e^{-G} as two-term bf16 (hi in place), and the state carried on:
+    // S^T <- S^T diag(a_c) + dS_c^T.  State thread: row sj = bt / 4 (value
+    // dim), units su, su + 1 (key dims 8 su .. 8 su + 15).
+    pdl_wait();                           // the segments' entering states come from the scan
+    pdl_trigger();
     const int bt = threadIdx.x - 32 * kWarpBuild0, bw = bt >> 5;
     const int dc = 2 * lane, tb = 8 * bw;
-    bool prev_exact[2] = {false, false};
+    const int sj = bt >> 2, su = 2 * (bt & 3);
+    float S[16];
     for (int n = 0; n < nit; ++n) {
-      const int s = n & 1, use = n >> 1;
-      const Item it = pipe_item(p, pipe_index(n));
-      const bool vd = v_direct(kV2, tma, it);
-      uint8_t* r = raw(s);
-      uint8_t* o = op(s);
-      failed |= !mbar_wait(&m.full[s], (uint32_t)use & 1u);
-      if (use > 0) {
-        failed |= !mbar_wait(&m.mma2[s], (uint32_t)(use - 1) & 1u);   // the slot's tiles are free
-        // after an exact chunk the epilogue warps read its flag before it is rewritten
-        if (prev_exact[s]) failed |= !mbar_wait(&m.tfree[s], (uint32_t)(use - 1) & 1u);
+      const int s = n % NS, use = n / NS;
+      uint8_t* o = sm + s * L::kSlot;
+      const Item it = item_at(p, n);
+      // this chunk's increment (for the state after it), and at a segment
+      // start the entering state, requested before the waits
+      float dsn[16];
+      {
+        const uint8_t* t = p.dS + ((size_t)it.bhl * p.nc + it.c) * kStateTile;
+        tile_load8(t, sj, su, dsn);
+        tile_load8(t, sj, su + 1, dsn + 8);
+        if (it.first) {
+          const uint8_t* ts = p.segS + (size_t)it.sg * kStateTile;
+          tile_load8(ts, sj, su, S);
+          tile_load8(ts, sj, su + 1, S + 8);
+        }
       }
+      failed |= !mbar_wait(&m.full[s], (uint32_t)use & 1u);
       if (named_barrier_or(kBarBuild, kThreads, failed || aborted(&m.abort))) { failed = true; break; }
-      float* G = reinterpret_cast<float*>(r + L::kRg);
+      // the state entering the chunk: S^T hi, lo
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) split2(S[8 * h + 2 * e], S[8 * h + 2 * e + 1], hi[e], lo[e]);
+        const uint32_t off = sw_unit(sj, su + h);
+        *reinterpret_cast<uint4*>(o + L::kSH + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(o + L::kSL + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+      float* G = reinterpret_cast<float*>(o + L::kG);
       float2 gc[8];
-      chunk_cumsum(G, gc, m.part, bw, tb, dc, it.rmask);
+      const float2 tot = chunk_cumsum(G, gc, m.part, bw, tb, dc, it.rmask);
+      // the chunk's decay factors, computed as the summary kernel computes them
+      if (bw == 0) *reinterpret_cast<float2*>(&m.ac[s][dc]) = make_float2(expf(tot.x), expf(tot.y));
+      uint32_t qr[8], kr[8];
       int bad = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t off = sw16((tb + i) ^ it.rmask, dc);
+        qr[i] = *reinterpret_cast<const uint32_t*>(o + L::kQH + off);
+        kr[i] = *reinterpret_cast<const uint32_t*>(o + L::kKH + off);
         bad |= !(gc[i].x <= 0.f && gc[i].x >= -kSpanMax && gc[i].y <= 0.f && gc[i].y >= -kSpanMax);
-      const T* qst = reinterpret_cast<const T*>(r + L::kRq);
-      const T* kst = reinterpret_cast<const T*>(r + L::kRk);
-      {
-        uint32_t qr[8], kr[8], vr[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int rs = (tb + i) ^ it.rmask;
-          qr[i] = *reinterpret_cast<const uint32_t*>(qst + rs * kD + dc);
-          kr[i] = *reinterpret_cast<const uint32_t*>(kst + rs * kD + dc);
-          vr[i] = vd ? 0u : *reinterpret_cast<const uint32_t*>(r + L::kRv + sw16(rs, dc));
+        if (kH) {
+          const float2 qq = ld2(reinterpret_cast<const T*>(&qr[i])), kk = ld2(reinterpret_cast<const T*>(&kr[i]));
+          bad |= !(fabsf(qq.x) < kQKMaxF16 && fabsf(qq.y) < kQKMaxF16 && fabsf(kk.x) < kQKMaxF16 &&
+                   fabsf(kk.y) < kQKMaxF16);
         }
+      }
+      // with G in [-kSpanMax, 0] everywhere no factor leaves [e^{-kSpanMax}, e^{kSpanMax}]
+      const bool exact = named_barrier_or(kBarBuild, kThreads, bad != 0);
+      if (!exact) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const uint32_t off = sw16(tb + i, dc);
+          const uint32_t off = sw16((tb + i) ^ it.rmask, dc);
           const float2 qq = ld2(reinterpret_cast<const T*>(&qr[i])), kk = ld2(reinterpret_cast<const T*>(&kr[i]));
           const float x0 = gc[i].x * kLog2e, x1 = gc[i].y * kLog2e;
           put2x(o + L::kQH, o + L::kQL, off, qq.x * ex2(x0), qq.y * ex2(x1));
           put2x(o + L::kKH, o + L::kKL, off, kk.x * ex2(-x0), kk.y * ex2(-x1));
-          if (!vd) {
-            if (kV2) {
-              const float2 vv = ld2(reinterpret_cast<const T*>(&vr[i]));
-              put2x(o + L::kVH, o + L::kVL, off, vv.x, vv.y);
-            } else {
-              *reinterpret_cast<uint32_t*>(o + L::kVH + off) = vr[i];
-            }
-          }
         }
-      }
-      fence_async_smem();
-      // with G in [-kSpanMax, 0] everywhere no factor leaves [e^{-kSpanMax}, e^{kSpanMax}]
-      const bool exact = named_barrier_or(kBarBuild, kThreads, bad != 0);
-      prev_exact[s] = exact;
-      if (bt == 0) {
-        m.exact[s] = exact ? 1 : 0;
-        mbar_arrive_one(&m.built[s]);
-        if (!exact) mbar_arrive_one(&m.rawfree[s]);
-      }
-      if (exact) {
-        // scores on CUDA cores, P_ji = sum_d q_jd k_id e^{G_jd - G_id}, into
-        // the q~ tiles once the first product has read them; G in scan order
+      } else {
+        // scores on CUDA cores, P_rc = sum_x q_rx k_cx e^{G_rx - G_cx} for key c
+        // at or before query r (staging rows; scan offset = row ^ rmask), with
+        // G in place of the gate rows; then q~ for o = q~ S
 #pragma unroll
-        for (int i = 0; i < 8; ++i) *reinterpret_cast<float2*>(G + (tb + i) * kD + dc) = gc[i];
+        for (int i = 0; i < 8; ++i) *reinterpret_cast<float2*>(G + ((tb + i) ^ it.rmask) * kD + dc) = gc[i];
         named_barrier(kBarBuild, kThreads);
-        failed |= !mbar_wait(&m.mma1[s], (uint32_t)use & 1u);
-        const int j = bt >> 2, ib = (bt & 3) * 16;
+        const int qd = warp & 3, half = bw >> 2;
+        const int r = qd * 16 + (lane & 15), cb = half * 32 + (lane >> 4) * 16;
+        const int sr = r ^ it.rmask;
         float acc[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) acc[e] = 0.f;
-        if (j < it.ntok && !failed) {
-          const T* qj_row = qst + (j ^ it.rmask) * kD;
+        if (sr < it.ntok) {
           for (int x = 0; x < kD; ++x) {
-            const float qj = Elem<T>::to_f(qj_row[x]);
-            const float gj = G[j * kD + x];
+            const float qx = Elem<T>::to_f(*reinterpret_cast<const T*>(o + L::kQH + sw16(r, x)));
+            const float gx = G[r * kD + x];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-              const int i = ib + e;
-              if (i <= j)
-                acc[e] = fmaf(qj * Elem<T>::to_f(kst[(i ^ it.rmask) * kD + x]), expf(gj - G[i * kD + x]), acc[e]);
+              const int c = cb + e;
+              if ((c ^ it.rmask) <= sr)
+                acc[e] = fmaf(qx * Elem<T>::to_f(*reinterpret_cast<const T*>(o + L::kKH + sw16(c, x))),
+                              expf(gx - G[c * kD + x]), acc[e]);
             }
           }
         }
+        named_barrier(kBarBuild, kThreads);   // q, k read before q~ overwrites q
 #pragma unroll
-        for (int e = 0; e < 16; e += 4)
-          put4(o + L::kQH, o + L::kQL, sw16(j, ib + e), acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
-        fence_async_smem();
-        named_barrier(kBarBuild, kThreads);
-        if (bt == 0) {
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t off = sw16((tb + i) ^ it.rmask, dc);
+          const float2 qq = ld2(reinterpret_cast<const T*>(&qr[i]));
+          put2x(o + L::kQH, o + L::kQL, off, qq.x * expf(gc[i].x), qq.y * expf(gc[i].y));
+        }
+        uint32_t ph[8], pl[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (kH) split2h(acc[2 * e], acc[2 * e + 1], ph[e], pl[e]);
+          else split2(acc[2 * e], acc[2 * e + 1], ph[e], pl[e]);
+        }
+        const uint32_t tms = tm + 128u * s + ((uint32_t)(qd * 32) << 16);
+        tmem_st8x2(tms + 64 + 16 * half, ph);
+        tmem_st8x2(tms + 96 + 16 * half, pl);
+        tmem_st_wait();
+        tc_before_sync();
+      }
+      // the state after the chunk (the decay factors were written before the
+      // exact-chunk barrier)
+#pragma unroll
+      for (int e = 0; e < 16; e += 4) {
+        const float4 an = *reinterpret_cast<const float4*>(&m.ac[s][8 * su + e]);
+        S[e] = fmaf(an.x, S[e], dsn[e]);
+        S[e + 1] = fmaf(an.y, S[e + 1], dsn[e + 1]);
+        S[e + 2] = fmaf(an.z, S[e + 2], dsn[e + 2]);
+        S[e + 3] = fmaf(an.w, S[e + 3], dsn[e + 3]);
+      }
+      fence_async_smem();
+      named_barrier(kBarBuild, kThreads);
+      if (bt == 0) {
+        m.exact[s] = exact ? 1 : 0;
+        mbar_arrive_one(&m.built[s]);
+        if (exact) {
           atomicAdd(&g_gtr_exact_chunks, 1ull);
           mbar_arrive_one(&m.pready[s]);
-          mbar_arrive_one(&m.rawfree[s]);
         }
       }
     }
     if (failed && bt == 0) m.abort = 1;
   } else {
-    // ---- epilogue warps: P (masked two-term scores back into tensor memory),
-    // then RMSNorm x w x SiLU(z) and the stores at the tokens' grid rows.
+    // ---- epilogue warps, one chunk behind: P of chunk n (masked two-term
+    // scores back into tensor memory, in place), then the epilogue of chunk
+    // n - 1: RMSNorm x w x SiLU(z), stored at the tokens' grid rows.
     // Thread: accumulator row `row` (TMEM lane quadrant warp % 4), columns
-    // ch*16 .. +15 and 32 + ch*16 .. +15.
+    // c0 .. c0+15 and c1 .. c1+15.
     const int qd = warp & 3;
     const int row = qd * 16 + (lane & 15), ch = lane >> 4;
     const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
     const bool out32 = ((uintptr_t)p.out & 31) == 0;
     const int c0 = ch * 16, c1 = 32 + ch * 16;
-    for (int n = 0; n < nit; ++n) {
-      const int s = n & 1, use = n >> 1;
-      const Item it = pipe_item(p, pipe_index(n));
-      const uint32_t tms = tm + 256u * s + lane_base;
-      const bool live = row < it.ntok;
-      const long long grow = live ? item_row(p, it, row) : 0;
-      // this row's z, requested before the products complete
-      uint4 z0a = make_uint4(0u, 0u, 0u, 0u), z0b = z0a, z1a = z0a, z1b = z0a;
-      if (live) {
-        const uint4* zp = reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.z) + grow * kD);
-        z0a = __ldg(zp + c0 / 8);
-        z0b = __ldg(zp + c0 / 8 + 1);
-        z1a = __ldg(zp + c1 / 8);
-        z1b = __ldg(zp + c1 / 8 + 1);
+    // z of a chunk's rows for its epilogue (zeros past the chunk's end)
+    auto load_z = [&](int n, uint4 (&zq)[4]) {
+      const Item it = item_at(p, n);
+      const int sr = row ^ it.rmask;
+      zq[0] = zq[1] = zq[2] = zq[3] = make_uint4(0u, 0u, 0u, 0u);
+      if (sr < it.ntok) {
+        const uint4* zr = reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.z) + item_row(p, it, sr) * kD);
+        zq[0] = __ldg(zr + c0 / 8);
+        zq[1] = __ldg(zr + c0 / 8 + 1);
+        zq[2] = __ldg(zr + c1 / 8);
+        zq[3] = __ldg(zr + c1 / 8 + 1);
       }
-      failed |= !mbar_wait(&m.mma1[s], (uint32_t)use & 1u);
-      failed |= !mbar_wait(&m.built[s], (uint32_t)use & 1u);
-      if (named_barrier_or(kBarEpi, 128, failed || aborted(&m.abort))) { failed = true; break; }
-      tc_after_sync();
-      if (!m.exact[s]) {
-        float sa[16], sb[16];
-        tmem_ld16x2(tms + 64, sa);
-        tmem_ld16x2(tms + 96, sb);
-        tmem_ld_wait(sa);
-        tmem_ld_wait(sb);
-        uint32_t ha[8], la[8], hb[8], lb[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float a0 = c0 + 2 * e <= row ? sa[2 * e] : 0.f, a1 = c0 + 2 * e + 1 <= row ? sa[2 * e + 1] : 0.f;
-          const float b0 = c1 + 2 * e <= row ? sb[2 * e] : 0.f, b1 = c1 + 2 * e + 1 <= row ? sb[2 * e + 1] : 0.f;
-          split2(a0, a1, ha[e], la[e]);
-          split2(b0, b1, hb[e], lb[e]);
-        }
-        tmem_st8x2(tms + 128, ha);
-        tmem_st8x2(tms + 144, hb);
-        tmem_st8x2(tms + 160, la);
-        tmem_st8x2(tms + 176, lb);
-        tmem_st_wait();
-        tc_before_sync();
-        named_barrier(kBarEpi, 128);
-        if (warp == kWarpEpi0 && lane == 0) mbar_arrive_one(&m.pready[s]);
-      }
-      // the output gate w * SiLU(z) while P V runs
-      float wz[32];
-      {
-        const uint4 zs[4] = {z0a, z0b, z1a, z1b};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int cb = (q < 2 ? c0 : c1) + 8 * (q & 1);
-          const float4 za = Vec4<T>::from_bits(make_uint2(zs[q].x, zs[q].y));
-          const float4 zb = Vec4<T>::from_bits(make_uint2(zs[q].z, zs[q].w));
-          const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
-#pragma unroll
-          for (int e = 0; e < 8; ++e) wz[8 * q + e] = m.wv[cb + e] * silu_fast(zz[e]);
-        }
-      }
+    };
+    uint4 zp[4];
+    auto epilogue = [&](int n, const uint4 (&zq)[4]) {
+      const int s = n % NS, use = n / NS;
+      const Item it = item_at(p, n);
+      const int sr = row ^ it.rmask;
+      const bool live = sr < it.ntok;
       failed |= !mbar_wait(&m.mma2[s], (uint32_t)use & 1u);
       tc_after_sync();
       float oa[16], ob[16];
-      tmem_ld16x2(tms, oa);
-      tmem_ld16x2(tms + 32, ob);
+      tmem_ld16x2(tm + 128u * s + lane_base, oa);
+      tmem_ld16x2(tm + 128u * s + lane_base + 32, ob);
       tmem_ld_wait(oa);
       tmem_ld_wait(ob);
       tc_before_sync();
@@ -860,14 +902,21 @@ gla_out_pipe(const __grid_constant__ PipeParams p, const __grid_constant__ Maps 
       ss += __shfl_xor_sync(0xffffffffu, ss, 16);
       if (live && !failed) {
         const float inv = rsqrtf(ss * (1.0f / kD) + kRmsEps);
-        T* dst = reinterpret_cast<T*>(p.out) + grow * kD;
+        T* dst = reinterpret_cast<T*>(p.out) + item_row(p, it, sr) * kD;
         uint4 y[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
+          const int cb = (q < 2 ? c0 : c1) + 8 * (q & 1);
           const float* x = q < 2 ? oa + 8 * (q & 1) : ob + 8 * (q & 1);
-          const float* wq = wz + 8 * q;
-          const uint2 lo = pack4<T>(x[0] * inv * wq[0], x[1] * inv * wq[1], x[2] * inv * wq[2], x[3] * inv * wq[3]);
-          const uint2 hi = pack4<T>(x[4] * inv * wq[4], x[5] * inv * wq[5], x[6] * inv * wq[6], x[7] * inv * wq[7]);
+          const uint4 zz = zq[q];
+          const float4 za = Vec4<T>::from_bits(make_uint2(zz.x, zz.y));
+          const float4 zb = Vec4<T>::from_bits(make_uint2(zz.z, zz.w));
+          const float zv[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
+          float yv[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) yv[e] = x[e] * inv * (m.wv[cb + e] * silu_fast(zv[e]));
+          const uint2 lo = pack4<T>(yv[0], yv[1], yv[2], yv[3]);
+          const uint2 hi = pack4<T>(yv[4], yv[5], yv[6], yv[7]);
           y[q] = make_uint4(lo.x, lo.y, hi.x, hi.y);
         }
         if (out32) {
@@ -880,6 +929,61 @@ gla_out_pipe(const __grid_constant__ PipeParams p, const __grid_constant__ Maps 
           reinterpret_cast<uint4*>(dst + c1)[1] = y[3];
         }
       }
+    };
+    for (int n = 0; n < nit; ++n) {
+      const int s = n % NS, use = n / NS;
+      const Item it = item_at(p, n);
+      const uint32_t tms = tm + 128u * s + lane_base;
+      // z of the previous chunk, whose epilogue follows this chunk's P
+      if (n >= 1) load_z(n - 1, zp);
+      failed |= !mbar_wait(&m.mma1[s], (uint32_t)use & 1u);
+      failed |= !mbar_wait(&m.built[s], (uint32_t)use & 1u);
+      if (named_barrier_or(kBarEpi, 128, failed || aborted(&m.abort))) { failed = true; break; }
+      tc_after_sync();
+      if (!m.exact[s]) {
+        // P = scores masked to keys at or before the query (scan positions),
+        // two terms, written over the scores: this warp owns these rows, and
+        // every load completes before a store
+        float sa[16], sb[16];
+        tmem_ld16x2(tms + 64, sa);
+        tmem_ld16x2(tms + 96, sb);
+        tmem_ld_wait(sa);
+        tmem_ld_wait(sb);
+        const int sr = row ^ it.rmask;
+        uint32_t ha[8], la[8], hb[8], lb[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float a0 = ((c0 + 2 * e) ^ it.rmask) <= sr ? sa[2 * e] : 0.f;
+          const float a1 = ((c0 + 2 * e + 1) ^ it.rmask) <= sr ? sa[2 * e + 1] : 0.f;
+          const float b0 = ((c1 + 2 * e) ^ it.rmask) <= sr ? sb[2 * e] : 0.f;
+          const float b1 = ((c1 + 2 * e + 1) ^ it.rmask) <= sr ? sb[2 * e + 1] : 0.f;
+          if (kH) {
+            split2h(a0, a1, ha[e], la[e]);
+            split2h(b0, b1, hb[e], lb[e]);
+          } else {
+            split2(a0, a1, ha[e], la[e]);
+            split2(b0, b1, hb[e], lb[e]);
+          }
+        }
+        tmem_st8x2(tms + 64, ha);
+        tmem_st8x2(tms + 80, hb);
+        tmem_st8x2(tms + 96, la);
+        tmem_st8x2(tms + 112, lb);
+        tmem_st_wait();
+        tc_before_sync();
+        named_barrier(kBarEpi, 128);
+        if (warp == kWarpEpi0 && lane == 0) mbar_arrive_one(&m.pready[s]);
+      }
+      if (n >= 1) epilogue(n - 1, zp);
+    }
+    // (uniform across the epilogue warps: the last epilogue has a barrier)
+    if (!named_barrier_or(kBarEpi, 128, failed)) {
+      if (nit > 0) {
+        load_z(nit - 1, zp);
+        epilogue(nit - 1, zp);
+      }
+    } else {
+      failed = true;
     }
     if (failed && threadIdx.x == 32 * kWarpEpi0) m.abort = 1;
   }
