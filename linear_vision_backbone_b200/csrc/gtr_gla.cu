@@ -15,7 +15,6 @@
 #include "simt_kernels.cuh"
 #include "scan_kernel.cuh"
 #include "tc_kernels.cuh"
-#include "pipe_kernels.cuh"
 #include "gate_tc.cuh"
 #include "mixer_proj.cuh"
 
@@ -58,7 +57,6 @@ struct Plan {
   int B, H, gh, gw, T, dk, dv, dir, chunk, dtype;
   int dev;
   int path;        // GTR_PATH_SIMT or GTR_PATH_TC
-  int pipe;        // 1: the chunk-parallel tensor-core pipeline (a state per chunk)
   int nc;          // chunks per sequence
   int nseg;        // segments per sequence
   int seg_chunks;  // chunks in the longest segment
@@ -140,55 +138,15 @@ int choose_path(int dk, int dv, int chunk, int dtype) {
   return tc_supported(dk, dv, chunk, dtype) ? (int)GTR_PATH_TC : (int)GTR_PATH_SIMT;
 }
 
-// Workspace of the tensor-core pipeline for nbh sequences of nc chunks in
-// nseg segments: chunk increments (a 16 KB state tile per chunk), chunk
-// decay factors (64 fp32), segment states (a tile per segment), segment
-// decay factors; each region 256-byte aligned.
-struct PipeWs {
-  uint8_t* dS; float* a; uint8_t* segS; float* segA;
-};
-inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
-size_t pipe_ws_bytes(long long nbh, int nc, int nseg) {
-  return align256((size_t)nbh * nc * tc::kStateTile) + align256((size_t)nbh * nc * 64 * sizeof(float)) +
-         align256((size_t)nbh * nseg * tc::kStateTile) + (size_t)nbh * nseg * 64 * sizeof(float);
-}
-PipeWs pipe_ws(void* base, long long nbh, int nc, int nseg) {
-  PipeWs w;
-  char* b = (char*)base;
-  w.dS = (uint8_t*)b;
-  b += align256((size_t)nbh * nc * tc::kStateTile);
-  w.a = (float*)b;
-  b += align256((size_t)nbh * nc * 64 * sizeof(float));
-  w.segS = (uint8_t*)b;
-  b += align256((size_t)nbh * nseg * tc::kStateTile);
-  w.segA = (float*)b;
-  return w;
-}
-
-// `legacy`: the segment-walking tensor-core kernels (the gate-fused call);
-// otherwise tensor-core shapes run the chunk-parallel pipeline, whose
-// workspace holds one state tile (16 KB) and one decay vector per chunk.
 int make_plan(Plan* p, int dev, int B, int H, int gh, int gw, int dk, int dv, int dir, int chunk,
-              int dtype, int force_nseg, bool legacy = false, int force_path = 0) {
+              int dtype, int force_nseg) {
   p->B = B; p->H = H; p->gh = gh; p->gw = gw; p->T = gh * gw; p->dev = dev;
   p->dk = dk; p->dv = dv; p->dir = dir; p->chunk = chunk; p->dtype = dtype;
-  const int path = force_path ? force_path : choose_path(dk, dv, chunk, dtype);
+  const int path = choose_path(dk, dv, chunk, dtype);
   if (path < 0) return path;
   p->path = path;
   p->nc = (p->T + chunk - 1) / chunk;
   const long long bh = (long long)B * H;
-  p->pipe = path == GTR_PATH_TC && !legacy;
-  if (p->pipe) {
-    if (bh * p->nc >= (1LL << 31)) return GTR_ERR_UNSUPPORTED;   // chunks are counted in an int
-    // one segment per CTA when the sequences leave SMs over; a CTA walks
-    // several segments otherwise
-    const long long per = sm_count(dev) / (bh > 0 ? bh : 1);
-    p->nseg = (int)(per < 1 ? 1 : (per > p->nc ? p->nc : per));
-    p->seg_chunks = (p->nc + p->nseg - 1) / p->nseg;
-    p->offA = 0;
-    p->ws_bytes = pipe_ws_bytes(bh, p->nc, p->nseg);
-    return GTR_OK;
-  }
   const int per_sm = path == GTR_PATH_TC ? tc_blocks_per_sm(dk, dv) : 4;
   const long long slots = (long long)sm_count(dev) * per_sm;
   if (force_nseg > 0) {
@@ -328,7 +286,7 @@ int tmap_chunk(CUtensorMap* map, CUtensorMapDataType dt, int es, const void* bas
 // g may be null; `g_store` adds the store map of the g the summary kernel
 // writes (32-column boxes, SWIZZLE_128B).
 bool chunk_maps(const Plan& p, const void* q, const void* k, const void* v, const float* g, tc::Maps* maps,
-                const float* low = nullptr, const float* g_store = nullptr, bool swizzle_qk = false) {
+                const float* low = nullptr, const float* g_store = nullptr) {
   for (const void* a : {q, k, v, (const void*)g, (const void*)low, (const void*)g_store})
     if (((uintptr_t)a & 15) != 0) return false;
   bool orient[2] = {false, false};
@@ -342,8 +300,8 @@ bool chunk_maps(const Plan& p, const void* q, const void* k, const void* v, cons
   *maps = tc::Maps{};
   for (int o = 0; o < 2; ++o) {
     if (!orient[o]) continue;
-    if ((q && tmap_chunk(&maps->t[o][tc::kMapQ], dt, 2, q, p, o, swizzle_qk)) ||
-        tmap_chunk(&maps->t[o][tc::kMapK], dt, 2, k, p, o, swizzle_qk) ||
+    if ((q && tmap_chunk(&maps->t[o][tc::kMapQ], dt, 2, q, p, o, false)) ||
+        tmap_chunk(&maps->t[o][tc::kMapK], dt, 2, k, p, o, false) ||
         tmap_chunk(&maps->t[o][tc::kMapV], dt, 2, v, p, o, true) ||
         (g && tmap_chunk(&maps->t[o][tc::kMapG], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, g, p, o, false)) ||
         (low && tmap_chunk(&maps->t[o][tc::kMapL], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, low, p, o, false,
@@ -511,55 +469,6 @@ int launch_scan(const Plan& p, float* wsS, const float* wsA, int inclusive, cuda
              : GTR_ERR_CUDA;
 }
 
-// ---- the tensor-core pipeline (pipe_kernels.cuh)
-template <typename T>
-int launch_pipe_typed(int stage, const tc::PipeParams& pp, const tc::Maps& mp, cudaStream_t st, int dev) {
-  static bool done_sum[kMaxDevices], done_out[kMaxDevices];
-  const long long segs = (long long)pp.nbh * pp.nseg;
-  const unsigned grid = (unsigned)(segs < sm_count(dev) ? segs : sm_count(dev));
-  if (stage == 0) {
-    if (int rc = ensure_smem(tc::gla_sum_pipe<T>, tc::kSumPipeSmem, done_sum, dev)) return rc;
-    return launch_pdl(tc::gla_sum_pipe<T>, dim3(grid), dim3(tc::kPipeThreads), tc::kSumPipeSmem, st, pp, mp)
-               ? GTR_ERR_CUDA
-               : GTR_OK;
-  }
-  if (int rc = ensure_smem(tc::gla_out_pipe<T>, tc::kOutPipeSmem, done_out, dev)) return rc;
-  return launch_pdl(tc::gla_out_pipe<T>, dim3(grid), dim3(tc::kPipeThreads), tc::kOutPipeSmem, st, pp, mp)
-             ? GTR_ERR_CUDA
-             : GTR_OK;
-}
-
-// The affine scan over `n` state tiles per sequence for nbh sequences (see
-// gla_tile_scan): in place (entering states) or, with `states`, inclusive fp32.
-int launch_tile_scan(uint8_t* tiles, const float* a, float* states, int n, int nbh, cudaStream_t st) {
-  const tc::ScanParams sp{tiles, a, states, n, states ? 1 : 0};
-  return launch_pdl(tc::gla_tile_scan, dim3((unsigned)nbh * 64u), dim3(tc::kTileScanThreads), 0, st, sp)
-             ? GTR_ERR_CUDA
-             : GTR_OK;
-}
-
-// One stage of the pipeline for sequences bh0 .. bh0 + nbh - 1 with their
-// workspace `w`: 0 = chunk summaries (and segment maps), 1 = scan over the
-// segments, 2 = chunk outputs.
-int launch_pipe(const Plan& p, int stage, const void* q, const void* k, const void* v, const float* g,
-                const void* z, const float* w, void* out, const PipeWs& ws, int bh0, int nbh, cudaStream_t st) {
-  if (stage == 1) return launch_tile_scan(ws.segS, ws.segA, nullptr, p.nseg, nbh, st);
-  tc::PipeParams pp{q, k, v, g, z, w, ws.dS, ws.a, ws.segS, ws.segA, out,
-                    p.H, p.T, p.gh, p.gw, p.dir, p.nc, p.nseg, bh0, nbh, 0};
-  tc::Maps maps;
-  pp.tma = chunk_maps(p, stage == 2 ? q : nullptr, k, v, g, &maps, nullptr, nullptr, true) ? 1 : 0;
-  static const tc::Maps kNoMaps{};
-  const tc::Maps& mp = pp.tma ? maps : kNoMaps;
-  const int s = stage == 0 ? 0 : 1;
-  return p.dtype == GTR_F16 ? launch_pipe_typed<__half>(s, pp, mp, st, p.dev)
-                            : launch_pipe_typed<__nv_bfloat16>(s, pp, mp, st, p.dev);
-}
-
-// The three stages for sequences bh0 .. bh0 + nbh - 1 with their workspace at
-// `ws` (events as gtr_gla_fwd_timed; null when not wanted).
-int run_pipe(const Plan& p, const void* q, const void* k, const void* v, const float* g, const void* z,
-             const float* w, void* out, void* ws, int bh0, int nbh, cudaStream_t st, void* const* ev);
-
 // Record a caller event; inside stream capture it becomes an external event
 // node, so a replayed graph records real timestamps.
 int record(void* const* ev, int i, cudaStream_t st) {
@@ -570,19 +479,6 @@ int record(void* const* ev, int i, cudaStream_t st) {
                             ? cudaEventRecordWithFlags((cudaEvent_t)ev[i], st, cudaEventRecordExternal)
                             : cudaEventRecord((cudaEvent_t)ev[i], st);
   return e == cudaSuccess ? GTR_OK : GTR_ERR_CUDA;
-}
-
-int run_pipe(const Plan& p, const void* q, const void* k, const void* v, const float* g, const void* z,
-             const float* w, void* out, void* ws, int bh0, int nbh, cudaStream_t st, void* const* ev) {
-  const PipeWs pw = pipe_ws(ws, nbh, p.nc, p.nseg);
-  int rc;
-  if ((rc = record(ev, 0, st))) return rc;
-  if ((rc = launch_pipe(p, 0, q, k, v, g, z, w, out, pw, bh0, nbh, st))) return rc;
-  if ((rc = record(ev, 1, st))) return rc;
-  if ((rc = launch_pipe(p, 1, q, k, v, g, z, w, out, pw, bh0, nbh, st))) return rc;
-  if ((rc = record(ev, 2, st))) return rc;
-  if ((rc = launch_pipe(p, 2, q, k, v, g, z, w, out, pw, bh0, nbh, st))) return rc;
-  return record(ev, 3, st);
 }
 
 int gla_fwd_impl(const void* q, const void* k, const void* v, const float* g, const void* z,
@@ -601,10 +497,9 @@ int gla_fwd_impl(const void* q, const void* k, const void* v, const float* g, co
   if ((rc = make_plan(&p, dev, B, H, gh, gw, dk, dv, dir, chunk, dtype, 0))) return rc;
   void* ws = nullptr;
   if ((rc = get_workspace(dev, stream, p.ws_bytes, &ws))) return rc;
-  cudaStream_t st = (cudaStream_t)stream;
-  if (p.pipe) return run_pipe(p, q, k, v, g, z, w, out, ws, 0, B * H, st, ev);
   float* wsS = (float*)ws;
   float* wsA = (float*)((char*)ws + p.offA);
+  cudaStream_t st = (cudaStream_t)stream;
   if ((rc = record(ev, 0, st))) return rc;
   if ((rc = launch_stage(p, q, k, v, g, z, w, out, wsS, wsA, st, 0))) return rc;
   if ((rc = record(ev, 1, st))) return rc;
@@ -642,7 +537,7 @@ int gla_fwd_gated_impl(const void* x, int x_dtype, const void* packed, const flo
   int dev;
   if ((rc = current_device(&dev))) return rc;
   Plan p;
-  if ((rc = make_plan(&p, dev, B, H, gh, gw, dk, dv, dir, chunk, dtype, 0, true))) return rc;
+  if ((rc = make_plan(&p, dev, B, H, gh, gw, dk, dv, dir, chunk, dtype, 0))) return rc;
   cudaStream_t st = (cudaStream_t)stream;
   if ((rc = record(ev, 0, st))) return rc;
   if (p.path != GTR_PATH_TC) {
@@ -714,38 +609,20 @@ int gla_fwd_noalloc_impl(const void* q, const void* k, const void* v, const floa
   if ((rc = current_device(&dev))) return rc;
   Plan p;
   if ((rc = make_plan(&p, dev, B, H, gh, gw, dk, dv, dir, chunk, dtype, 0))) return rc;
-  cudaStream_t st = (cudaStream_t)stream;
-  if (p.pipe) {
-    // the tensor-core pipeline keeps a state tile per chunk and per segment:
-    // as many sequences per round of its three kernels as the static scratch holds
-    const size_t per_seq = ((size_t)p.nc + p.nseg) * (tc::kStateTile + dk * sizeof(float));
-    const size_t group = (kStaticScratchBytes - 4 * 256) / per_seq;
-    if (group >= 1) {
-      void* ws = nullptr;
-      if ((rc = static_scratch(dev, &ws))) return rc;
-      const int nbh = B * H;
-      for (int bh0 = 0; bh0 < nbh; bh0 += (int)group) {
-        const int n = nbh - bh0 < (int)group ? nbh - bh0 : (int)group;
-        if ((rc = run_pipe(p, q, k, v, g, z, w, out, ws, bh0, n, st, nullptr))) return rc;
-      }
-      return GTR_OK;
-    }
-    // a sequence longer than that runs the segment-walking SIMT kernels
-    if ((rc = make_plan(&p, dev, B, H, gh, gw, dk, dv, dir, chunk, dtype, 0, false, GTR_PATH_SIMT))) return rc;
-  }
   if (p.ws_bytes > kStaticScratchBytes) {
     // fewer, longer segments until the boundary states fit the static scratch
     const size_t per_seg = (size_t)B * H * ((size_t)dk * dv + dk) * sizeof(float);
     const size_t max_nseg = (kStaticScratchBytes - 256) / per_seg;
     if (max_nseg < 1) return GTR_ERR_NO_MEMORY;
     const int nseg = (int)(max_nseg < (size_t)p.nc ? max_nseg : (size_t)p.nc);
-    if ((rc = make_plan(&p, dev, B, H, gh, gw, dk, dv, dir, chunk, dtype, nseg, false, p.path))) return rc;
+    if ((rc = make_plan(&p, dev, B, H, gh, gw, dk, dv, dir, chunk, dtype, nseg))) return rc;
     if (p.ws_bytes > kStaticScratchBytes) return GTR_ERR_NO_MEMORY;
   }
   void* ws = nullptr;
   if ((rc = static_scratch(dev, &ws))) return rc;
   float* wsS = (float*)ws;
   float* wsA = (float*)((char*)ws + p.offA);
+  cudaStream_t st = (cudaStream_t)stream;
   if ((rc = launch_stage(p, q, k, v, g, z, w, out, wsS, wsA, st, 0))) return rc;
   if ((rc = launch_scan(p, wsS, wsA, 0, st))) return rc;
   return launch_stage(p, q, k, v, g, z, w, out, wsS, wsA, st, 1);
@@ -998,20 +875,10 @@ gtr_status_t gtr_gla_chunk_states(const void* k, const void* v, const float* g, 
   // one chunk per segment: the scan then gives the state after every chunk
   if ((rc = make_plan(&p, dev, B, H, grid_h, grid_w, dk, dv, dir, chunk, dtype, 0x7fffffff)))
     return (gtr_status_t)rc;
-  cudaStream_t st = (cudaStream_t)stream;
-  if (p.pipe) {
-    // the pipeline's summary kernel, then the scan over its chunk increments
-    // in inclusive fp32 mode
-    void* ws = nullptr;
-    if ((rc = get_workspace(dev, stream, p.ws_bytes, &ws))) return (gtr_status_t)rc;
-    const PipeWs pw = pipe_ws(ws, (long long)B * H, p.nc, p.nseg);
-    if ((rc = launch_pipe(p, 0, nullptr, k, v, g, nullptr, nullptr, nullptr, pw, 0, B * H, st)))
-      return (gtr_status_t)rc;
-    return (gtr_status_t)launch_tile_scan(pw.dS, pw.a, states, p.nc, B * H, st);
-  }
   void* ws = nullptr;
   const size_t lbytes = (size_t)B * H * p.nseg * dk * sizeof(float);
   if ((rc = get_workspace(dev, stream, lbytes, &ws))) return (gtr_status_t)rc;
+  cudaStream_t st = (cudaStream_t)stream;
   if ((rc = launch_stage(p, nullptr, k, v, g, nullptr, nullptr, nullptr, states, (float*)ws, st, 0)))
     return (gtr_status_t)rc;
   return (gtr_status_t)launch_scan(p, states, (const float*)ws, 1, st);
