@@ -167,15 +167,20 @@ GTR_API gtr_status_t gtr_gla_fwd(const void *q, const void *k, const void *v, co
  * on demand.  Same arguments and result as gtr_gla_fwd; this call allocates
  * nothing and calls no allocating routine.
  *   Scratch: a static device array of GTR_NOALLOC_SCRATCH_BYTES (8 MiB) that
- *   every GPU loading the library reserves until the process exits.  The
+ *   a GPU holds from the library's first call on it until the process exits
+ *   (the CUDA runtime loads the library's device code onto a GPU lazily, at
+ *   its first kernel launch or symbol lookup there, and the array comes with
+ *   it).  A caller that must not allocate later should therefore make one
+ *   call on each device at start-up, before memory fills up and before any
+ *   stream capture; if the array cannot be placed the call returns
+ *   GTR_ERR_NO_MEMORY.  The
  *   boundary states need B*H*nseg*(dk*dv + dk)*4 bytes; when the usual segment
  *   plan needs more, longer segments are used (same result up to rounding).
  *   If even one segment per sequence does not fit, i.e.
  *   B*H*(dk*dv + dk)*4 + 256 > 8 MiB, the call returns GTR_ERR_NO_MEMORY and
  *   launches nothing.
- *   The first call on a device looks up the array's device address (once per
- *   device, with that device current); make that first call before any stream
- *   capture.
+ *   The first call on a device also looks up the array's device address
+ *   (once per device, with that device current).
  *   All calls share the one array and it keeps the last call's contents;
  *   nothing in it needs to start at zero (every element is written before it
  *   is read within a call).  Calls whose work overlaps on the GPU (other

@@ -585,9 +585,12 @@ int static_scratch(int dev, void** out) {
   std::lock_guard<std::mutex> lk(g_mu);
   if (!g_static_scratch_ptr[dev]) {
     void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_gtr_static_scratch) != cudaSuccess || !ptr) {
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_gtr_static_scratch);
+    if (e != cudaSuccess || !ptr) {
       (void)cudaGetLastError();
-      return GTR_ERR_CUDA;
+      // the array is placed on the device when the library's module first
+      // loads there; on a full device that placement is what fails
+      return e == cudaErrorMemoryAllocation ? GTR_ERR_NO_MEMORY : GTR_ERR_CUDA;
     }
     g_static_scratch_ptr[dev] = ptr;
   }

@@ -27,25 +27,7 @@ namespace {
 
 constexpr int kMixThreads = 128;
 
-// Eight consecutive channels, 16 bytes of storage, widened to fp32.
-__device__ __forceinline__ void widen8(const uint4& r, const __half*, float (&f)[8]) {
-  const __half2* p = reinterpret_cast<const __half2*>(&r);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 t = __half22float2(p[i]);
-    f[2 * i] = t.x;
-    f[2 * i + 1] = t.y;
-  }
-}
-__device__ __forceinline__ void widen8(const uint4& r, const __nv_bfloat16*, float (&f)[8]) {
-  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&r);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 t = __bfloat1622float2(p[i]);
-    f[2 * i] = t.x;
-    f[2 * i + 1] = t.y;
-  }
-}
+// Eight consecutive channels (16 bytes of storage) rounded from fp32.
 __device__ __forceinline__ uint4 narrow8(const float (&f)[8], const __half*) {
   uint4 r;
   __half2* p = reinterpret_cast<__half2*>(&r);
@@ -59,6 +41,48 @@ __device__ __forceinline__ uint4 narrow8(const float (&f)[8], const __nv_bfloat1
 #pragma unroll
   for (int i = 0; i < 4; ++i) p[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
   return r;
+}
+
+// Two fp32 lanes per instruction (sm_100 fma.rn.f32x2): a pair of
+// floats in one 64-bit register, the first in the low half.
+typedef unsigned long long f2_t;
+__device__ __forceinline__ f2_t pk2(float a, float b) {
+  f2_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float2 up2(f2_t r) {
+  float a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+  return make_float2(a, b);
+}
+__device__ __forceinline__ f2_t fma2(f2_t a, f2_t b, f2_t c) {
+  f2_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+// Eight consecutive channels as four fp32 pairs.
+__device__ __forceinline__ void widen8x2(const uint4& r, const __half*, f2_t (&f)[4]) {
+  const __half2* p = reinterpret_cast<const __half2*>(&r);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __half22float2(p[i]);
+    f[i] = pk2(t.x, t.y);
+  }
+}
+__device__ __forceinline__ void widen8x2(const uint4& r, const __nv_bfloat16*, f2_t (&f)[4]) {
+  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&r);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __bfloat1622float2(p[i]);
+    f[i] = pk2(t.x, t.y);
+  }
+}
+// SiLU(g) x a for a pair: g / (1 + 2^{-g log2 e}) x a, the exponential and
+// the reciprocal by the hardware approximations (relative error near 1e-7).
+__device__ __forceinline__ float2 silu_times2(float2 g, float2 a) {
+  const float ea = __expf(-g.x), eb = __expf(-g.y);
+  return make_float2(__fdividef(g.x, 1.f + ea) * a.x, __fdividef(g.y, 1.f + eb) * a.y);
 }
 
 // A block owns a tile of kTileCols grid columns x 64 channels over a strip of
@@ -135,7 +159,8 @@ __global__ void __launch_bounds__(kMixThreads, 4) sswiglu_mix_kernel(const E* __
     cp16(slot + kValBytes + threadIdx.x * 16, gv ? ub + ((size_t)yg * gw + x) * ldu + c : ub, gv);
   };
 
-  float w[3][3][8], bias[8];
+  // taps and bias of the thread's eight channels, as four channel pairs
+  f2_t w[3][3][4], bias[4];
   const int cl = cok ? c : 0;
 #pragma unroll
   for (int i = 0; i < 3; ++i)
@@ -143,17 +168,16 @@ __global__ void __launch_bounds__(kMixThreads, 4) sswiglu_mix_kernel(const E* __
     for (int j = 0; j < 3; ++j) {
       const float4* p = reinterpret_cast<const float4*>(cw + (size_t)(i * 3 + j) * C + cl);
       const float4 a = __ldg(p), q = __ldg(p + 1);
-      w[i][j][0] = a.x; w[i][j][1] = a.y; w[i][j][2] = a.z; w[i][j][3] = a.w;
-      w[i][j][4] = q.x; w[i][j][5] = q.y; w[i][j][6] = q.z; w[i][j][7] = q.w;
+      w[i][j][0] = pk2(a.x, a.y); w[i][j][1] = pk2(a.z, a.w);
+      w[i][j][2] = pk2(q.x, q.y); w[i][j][3] = pk2(q.z, q.w);
     }
   if (cb) {
     const float4* p = reinterpret_cast<const float4*>(cb + cl);
     const float4 a = __ldg(p), q = __ldg(p + 1);
-    bias[0] = a.x; bias[1] = a.y; bias[2] = a.z; bias[3] = a.w;
-    bias[4] = q.x; bias[5] = q.y; bias[6] = q.z; bias[7] = q.w;
+    bias[0] = pk2(a.x, a.y); bias[1] = pk2(a.z, a.w); bias[2] = pk2(q.x, q.y); bias[3] = pk2(q.z, q.w);
   } else {
 #pragma unroll
-    for (int k = 0; k < 8; ++k) bias[k] = 0.f;
+    for (int k = 0; k < 4; ++k) bias[k] = pk2(0.f, 0.f);
   }
 
 #pragma unroll
@@ -161,34 +185,39 @@ __global__ void __launch_bounds__(kMixThreads, 4) sswiglu_mix_kernel(const E* __
     if (y0 - 1 + i <= y1) issue(y0 - 1 + i);
     cp_commit();
   }
-  float acc_prev[8], acc_cur[8];   // partial sums of output rows r-1 and r
+  f2_t acc_prev[4], acc_cur[4];    // partial sums of output rows r-1 and r (channel pairs)
 #pragma unroll
-  for (int k = 0; k < 8; ++k) acc_prev[k] = acc_cur[k] = bias[k];
+  for (int k = 0; k < 4; ++k) acc_prev[k] = acc_cur[k] = bias[k];
   for (int r = y0 - 1; r <= y1; ++r) {
     cp_wait<kStages - 2>();
     __syncthreads();
     const unsigned char* slot = ring + ((r - y0 + 1) % kStages) * kSlotBytes;
-    float vl[8], vm[8], vr[8];
-    widen8(*reinterpret_cast<const uint4*>(slot + (col * kOcts + oct) * 16), (const E*)nullptr, vl);
-    widen8(*reinterpret_cast<const uint4*>(slot + ((col + 1) * kOcts + oct) * 16), (const E*)nullptr, vm);
-    widen8(*reinterpret_cast<const uint4*>(slot + ((col + 2) * kOcts + oct) * 16), (const E*)nullptr, vr);
-    float acc_next[8];
+    f2_t vl[4], vm[4], vr[4];
+    widen8x2(*reinterpret_cast<const uint4*>(slot + (col * kOcts + oct) * 16), (const E*)nullptr, vl);
+    widen8x2(*reinterpret_cast<const uint4*>(slot + ((col + 1) * kOcts + oct) * 16), (const E*)nullptr, vm);
+    widen8x2(*reinterpret_cast<const uint4*>(slot + ((col + 2) * kOcts + oct) * 16), (const E*)nullptr, vr);
+    f2_t acc_next[4];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      acc_next[k] = bias[k] + w[0][0][k] * vl[k] + w[0][1][k] * vm[k] + w[0][2][k] * vr[k];
-      acc_cur[k] += w[1][0][k] * vl[k] + w[1][1][k] * vm[k] + w[1][2][k] * vr[k];
-      acc_prev[k] += w[2][0][k] * vl[k] + w[2][1][k] * vm[k] + w[2][2][k] * vr[k];
+    for (int k = 0; k < 4; ++k) {
+      acc_next[k] = fma2(w[0][2][k], vr[k], fma2(w[0][1][k], vm[k], fma2(w[0][0][k], vl[k], bias[k])));
+      acc_cur[k] = fma2(w[1][2][k], vr[k], fma2(w[1][1][k], vm[k], fma2(w[1][0][k], vl[k], acc_cur[k])));
+      acc_prev[k] = fma2(w[2][2][k], vr[k], fma2(w[2][1][k], vm[k], fma2(w[2][0][k], vl[k], acc_prev[k])));
     }
     const int y = r - 1;   // output row completed by input row r
     if (ok && y >= y0) {
-      float gt[8], o[8];
-      widen8(*reinterpret_cast<const uint4*>(slot + kValBytes + threadIdx.x * 16), (const E*)nullptr, gt);
+      f2_t gt[4];
+      widen8x2(*reinterpret_cast<const uint4*>(slot + kValBytes + threadIdx.x * 16), (const E*)nullptr, gt);
+      float o[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) o[k] = gt[k] / (1.f + __expf(-gt[k])) * acc_prev[k];
+      for (int k = 0; k < 4; ++k) {
+        const float2 v = silu_times2(up2(gt[k]), up2(acc_prev[k]));
+        o[2 * k] = v.x;
+        o[2 * k + 1] = v.y;
+      }
       *reinterpret_cast<uint4*>(hb + ((size_t)y * gw + x) * C + c) = narrow8(o, (const E*)nullptr);
     }
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < 4; ++k) {
       acc_prev[k] = acc_cur[k];
       acc_cur[k] = acc_next[k];
     }
