@@ -16,6 +16,7 @@
 #include "scan_kernel.cuh"
 #include "tc_kernels.cuh"
 #include "gate_tc.cuh"
+#include "gemm_kernel.cuh"
 #include "mixer_proj.cuh"
 
 namespace {
@@ -633,6 +634,53 @@ int gla_fwd_noalloc_impl(const void* q, const void* k, const void* v, const floa
 
 }  // namespace
 
+namespace gtr {
+
+// The projections' GEMM (gemm_tc.cuh, gemm_kernel.cuh).
+int gemm_tc(int dtype, const void* A, int lda, const void* B, int ldb, void* const* C, int nout, int ncols,
+            int ldc, int M, int N, int K, cudaStream_t st) {
+  if (dtype != GTR_F16 && dtype != GTR_BF16) return GTR_ERR_UNSUPPORTED;
+  if (M <= 0 || N <= 0 || K <= 0) return GTR_OK;
+  if (nout < 1 || nout > gemm::kMaxOut) return GTR_ERR_UNSUPPORTED;
+  if (nout == 1) ncols = N;
+  if (nout > 1 && (ncols % gemm::kBN != 0 || (long long)nout * ncols != N)) return GTR_ERR_UNSUPPORTED;
+  // tensor maps: 16-byte aligned bases and row pitches
+  if (lda % 8 || ldb % 8 || ldc % 8 || ncols % 8 || !aligned16(A) || !aligned16(B)) return GTR_ERR_UNSUPPORTED;
+  for (int o = 0; o < nout; ++o)
+    if (!C[o] || !aligned16(C[o])) return GTR_ERR_UNSUPPORTED;
+  int dev;
+  if (int rc = current_device(&dev)) return rc;
+  const CUtensorMapDataType dt = dtype == GTR_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  gemm::Maps mp{};
+  if (int rc = tmap_2d(&mp.a, dt, A, (unsigned long long)M, (unsigned long long)K, (unsigned long long)lda * 2,
+                       gemm::kBK, gemm::kBM))
+    return rc;
+  if (int rc = tmap_2d(&mp.b, dt, B, (unsigned long long)K, (unsigned long long)N, (unsigned long long)ldb * 2, 64,
+                       gemm::kBK))
+    return rc;
+  for (int o = 0; o < nout; ++o)
+    if (int rc = tmap_2d(&mp.c[o], dt, C[o], (unsigned long long)M, (unsigned long long)ncols,
+                         (unsigned long long)ldc * 2, 64, gemm::kBM))
+      return rc;
+  gemm::Params p{M, N, K, nout, ncols, (M + gemm::kBM - 1) / gemm::kBM, (N + gemm::kBN - 1) / gemm::kBN,
+                 (K + gemm::kBK - 1) / gemm::kBK};
+  const long long tiles = (long long)p.mt * p.nt;
+  const unsigned grid = (unsigned)(tiles < sm_count(dev) ? tiles : sm_count(dev));
+  static bool done_h[kMaxDevices], done_b[kMaxDevices];
+  if (dtype == GTR_BF16) {
+    if (int rc = ensure_smem(gemm::gemm_tc_kernel<true>, gemm::kSmem, done_b, dev)) return rc;
+    return launch_pdl(gemm::gemm_tc_kernel<true>, dim3(grid), dim3(gemm::kThreads), gemm::kSmem, st, p, mp)
+               ? GTR_ERR_CUDA
+               : GTR_OK;
+  }
+  if (int rc = ensure_smem(gemm::gemm_tc_kernel<false>, gemm::kSmem, done_h, dev)) return rc;
+  return launch_pdl(gemm::gemm_tc_kernel<false>, dim3(grid), dim3(gemm::kThreads), gemm::kSmem, st, p, mp)
+             ? GTR_ERR_CUDA
+             : GTR_OK;
+}
+
+}  // namespace gtr
+
 extern "C" {
 
 int gtr_abi_version(void) { return GTR_ABI_VERSION; }
@@ -825,10 +873,29 @@ gtr_status_t gtr_mixer_in_proj(const void* x, const void* w_in, void* q, void* k
     return GTR_ERR_ALIGNMENT;
   int dev;
   if (int rc = current_device(&dev)) return (gtr_status_t)rc;
-  const cudaDataType dt = dtype == GTR_F16 ? CUDA_R_16F : CUDA_R_16BF;
   const int ldw = (int)(2 * (n_q + n_v));
   const char* W = (const char*)w_in;
   cudaStream_t st = (cudaStream_t)stream;
+  {
+    // our tensor-core GEMM: the four column blocks as one launch with four
+    // outputs when they are equally wide whole tiles, else one launch each
+    void* outs4[4] = {q, k, v, z};
+    int rc = gtr::gemm_tc(dtype, x, d_model, W, ldw, outs4, 4, (int)n_q, (int)n_q, (int)N, ldw, d_model, st);
+    if (n_q != n_v || rc == GTR_ERR_UNSUPPORTED) {
+      const long long off[4] = {0, n_q, 2 * n_q, 2 * n_q + n_v};
+      const long long width[4] = {n_q, n_q, n_v, n_v};
+      rc = GTR_OK;
+      for (int i = 0; i < 4 && rc == GTR_OK; ++i) {
+        if (width[i] == 0) continue;
+        void* o1[1] = {outs4[i]};
+        rc = gtr::gemm_tc(dtype, x, d_model, W + off[i] * 2, ldw, o1, 1, (int)width[i], (int)width[i], (int)N,
+                          (int)width[i], d_model, st);
+      }
+    }
+    if (rc != GTR_ERR_UNSUPPORTED) return (gtr_status_t)rc;
+  }
+  // shapes the tensor maps cannot address: cuBLAS
+  const cudaDataType dt = dtype == GTR_F16 ? CUDA_R_16F : CUDA_R_16BF;
   // column blocks of W: q | k | v | z.  Four equal blocks whose outputs lie
   // equally spaced in memory go out as one strided-batched product.
   const long long gap = (const char*)k - (const char*)q;
@@ -859,6 +926,11 @@ gtr_status_t gtr_mixer_out_proj(const void* y, const void* w_out, void* out, lon
   if (!aligned16(y) || !aligned16(w_out) || !aligned16(out)) return GTR_ERR_ALIGNMENT;
   int dev;
   if (int rc = current_device(&dev)) return (gtr_status_t)rc;
+  void* o1[1] = {out};
+  const int rc = gtr::gemm_tc(dtype, y, d_in, w_out, d_out, o1, 1, d_out, d_out, (int)N, d_out, d_in,
+                              (cudaStream_t)stream);
+  if (rc != GTR_ERR_UNSUPPORTED) return (gtr_status_t)rc;
+  // shapes the tensor maps cannot address: cuBLAS
   const cudaDataType dt = dtype == GTR_F16 ? CUDA_R_16F : CUDA_R_16BF;
   return (gtr_status_t)blas_gemm_rowmajor(dev, (cudaStream_t)stream, dt, y, d_in, w_out, d_out, out, d_out, (int)N,
                                           d_in, d_out);

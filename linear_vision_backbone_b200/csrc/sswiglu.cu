@@ -10,7 +10,8 @@
 //
 // The mixing step is one HBM-bound kernel (it reads u once and writes h once;
 // the halo columns and rows are re-read from L2);
-// the two projections are dense GEMMs run by cuBLAS (mixer_proj.cuh).
+// the two projections are dense GEMMs on the library's tensor-core GEMM
+// (gemm_tc.cuh), cuBLAS only for shapes outside its tensor maps.
 //
 // Layout: u [B, gh*gw, 2C] (gate channels [0, C), value channels [C, 2C)),
 // h [B, gh*gw, C], token t = row * gw + column, all rows of one 16-bit type;
@@ -21,6 +22,7 @@
 #include <stdint.h>
 
 #include "gtr_gla.h"
+#include "gemm_tc.cuh"
 #include "mixer_proj.cuh"
 
 namespace {
@@ -98,7 +100,7 @@ __device__ __forceinline__ float2 silu_times2(float2 g, float2 a) {
 // (a copy of source size 0 reads nothing).
 constexpr int kTileCols = 16;
 constexpr int kOcts = 8;                                      // 8 x 8 = 64 channels per tile
-constexpr int kStages = 6;
+constexpr int kStages = 16;
 constexpr int kValBytes = (kTileCols + 2) * kOcts * 16;       // 2304
 constexpr int kGateBytes = kTileCols * kOcts * 16;            // 2048
 constexpr int kSlotBytes = kValBytes + kGateBytes;            // 4352
@@ -116,11 +118,11 @@ __device__ __forceinline__ void cp_wait() {
 }
 
 template <typename E>
-__global__ void __launch_bounds__(kMixThreads, 4) sswiglu_mix_kernel(const E* __restrict__ u, E* __restrict__ h,
+__global__ void __launch_bounds__(kMixThreads, 3) sswiglu_mix_kernel(const E* __restrict__ u, E* __restrict__ h,
                                                                      const float* __restrict__ cw,
                                                                      const float* __restrict__ cb, int gh, int gw,
                                                                      int C, int rows, int nstrip, int ncx, int ncg) {
-  __shared__ __align__(128) unsigned char ring[kStages * kSlotBytes];
+  extern __shared__ __align__(128) unsigned char ring[];   // kStages * kSlotBytes
   long long bid = blockIdx.x;
   const int cgi = (int)(bid % ncg);
   bid /= ncg;
@@ -250,7 +252,15 @@ int mix_launch(const void* u, const float* cw, const float* cb, void* h, int B, 
   int dev = 0, sms = 0, per_sm = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return GTR_ERR_CUDA;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) sms = 148;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sswiglu_mix_kernel<E>, kMixThreads, 0) !=
+  constexpr int smem = kStages * kSlotBytes;
+  static bool attr_done[64];
+  if (dev < 64 && !attr_done[dev]) {
+    if (cudaFuncSetAttribute(sswiglu_mix_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return GTR_ERR_CUDA;
+    attr_done[dev] = true;
+  }
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sswiglu_mix_kernel<E>, kMixThreads, smem) !=
           cudaSuccess ||
       per_sm <= 0)
     per_sm = 1;
@@ -264,7 +274,7 @@ int mix_launch(const void* u, const float* cw, const float* cb, void* h, int B, 
   const int ns = (gh + rows - 1) / rows;
   const long long blocks = tiles * ns;
   if (blocks > 0x7fffffffLL) return GTR_ERR_INVALID_ARG;
-  sswiglu_mix_kernel<E><<<(unsigned)blocks, kMixThreads, 0, st>>>((const E*)u, (E*)h, cw, cb, gh, gw, C, rows,
+  sswiglu_mix_kernel<E><<<(unsigned)blocks, kMixThreads, smem, st>>>((const E*)u, (E*)h, cw, cb, gh, gw, C, rows,
                                                                  ns, ncx, ncg);
   return cudaGetLastError() == cudaSuccess ? GTR_OK : GTR_ERR_CUDA;
 }
@@ -311,11 +321,20 @@ GTR_API gtr_status_t gtr_sswiglu_fwd(const void* x, const void* w_in, const floa
   const cudaDataType dt = dtype == GTR_F16 ? CUDA_R_16F : CUDA_R_16BF;
   const int N = B * grid_h * grid_w;
   if (C == 0) return cudaMemsetAsync(y, 0, (size_t)N * d_model * 2, st) == cudaSuccess ? GTR_OK : GTR_ERR_CUDA;
-  if ((rc = gtr::blas_gemm_rowmajor(dev, st, dt, x, d_model, w_in, 2 * C, u, 2 * C, N, d_model, 2 * C)))
-    return (gtr_status_t)rc;
+  // the expansion and the projection on our tensor-core GEMM; cuBLAS for the
+  // shapes its tensor maps cannot address
+  void* ou[1] = {u};
+  rc = gtr::gemm_tc(dtype, x, d_model, w_in, 2 * C, ou, 1, 2 * C, 2 * C, N, 2 * C, d_model, st);
+  if (rc == GTR_ERR_UNSUPPORTED)
+    rc = gtr::blas_gemm_rowmajor(dev, st, dt, x, d_model, w_in, 2 * C, u, 2 * C, N, d_model, 2 * C);
+  if (rc) return (gtr_status_t)rc;
   if ((rc = gtr_sswiglu_mix(u, conv_w, conv_b, h, B, grid_h, grid_w, C, ksize, dtype, stream)))
     return (gtr_status_t)rc;
-  return (gtr_status_t)gtr::blas_gemm_rowmajor(dev, st, dt, h, C, w_out, d_model, y, d_model, N, C, d_model);
+  void* oy[1] = {y};
+  rc = gtr::gemm_tc(dtype, h, C, w_out, d_model, oy, 1, d_model, d_model, N, d_model, C, st);
+  if (rc == GTR_ERR_UNSUPPORTED)
+    rc = gtr::blas_gemm_rowmajor(dev, st, dt, h, C, w_out, d_model, y, d_model, N, C, d_model);
+  return (gtr_status_t)rc;
 }
 
 }  // extern "C"
