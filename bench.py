@@ -605,9 +605,9 @@ def make_step(binding, wl, params, x_dtype, chunk, stream, fused=False):
 
 def mixer_line(binding, dev, wl, host, steps=200):
     """The token mixer around the timed step (the next row of the hot path):
-    the input projection x -> q, k, v, z and the output projection y W_o as
-    cuBLAS GEMMs (16-bit, fp32 accumulation, random weights of the workload's
-    shapes), each timed alone on graphs, and the whole mixer step (input
+    the input projection x -> q, k, v, z and the output projection y W_o on the
+    library's tcgen05 GEMM (16-bit operands, fp32 accumulation in TMEM, random
+    weights of the workload's shapes), each timed alone on graphs, and the whole mixer step (input
     projection, gate, GLA, output projection).  Tensor-bound: FLOP/s against
     the measured bf16 GEMM peak."""
     dt = host["q"].dtype
@@ -668,7 +668,7 @@ def mixer_line(binding, dev, wl, host, steps=200):
         kind = "measured"
     except (OSError, KeyError, ValueError):
         peak, kind = 1590.0, "fallback"
-    return {"workload": workload_text(wl), "gemm": "cuBLAS (cublasGemmEx, fp32 accumulation)",
+    return {"workload": workload_text(wl), "gemm": "gemm_tc_kernel (tcgen05, 128x128 tiles, fp32 accumulation)",
             "in_proj": {"ms": ms_in, "tflops": fl_in / (ms_in * 1e-3) / 1e12,
                         "frac": fl_in / (ms_in * 1e-3) / 1e12 / peak},
             "out_proj": {"ms": ms_out, "tflops": fl_out / (ms_out * 1e-3) / 1e12,
@@ -691,8 +691,8 @@ def sswiglu_line(binding, dev, wl, steps=200):
     """The Spatial SwiGLU block on the workload's token grid (hidden width 1024,
     random weights): the mixing kernel alone (HBM-bound; two input sets
     alternate, 200 MB together, more than L2) with its achieved GB/s against
-    the measured copy bandwidth, and the whole block (two cuBLAS projections and
-    the mixing kernel) on warm buffers."""
+    the measured copy bandwidth, and the whole block (the two projections on the
+    library's tcgen05 GEMM and the mixing kernel) on warm buffers."""
     B, gh, gw, dm, C = wl.B, wl.gh, wl.gw, wl.d_model, SSWIGLU_HIDDEN
     T = gh * gw
     gen = torch.Generator().manual_seed(23)

@@ -247,16 +247,19 @@ GTR_API gtr_status_t gtr_gla_fwd_gated_timed(const void *x, int x_dtype, const v
  * The token mixer's projections on either side of the GLA (GTR article
  * 方法详解 §1: q, k, v and the output gate z are linear maps of the block input
  * x, and the mixer output is mapped back to the model width).  Plain dense
- * GEMMs with fp32 accumulation, run by cuBLAS, which the library loads with
- * dlopen at the first call (GTR_ERR_UNSUPPORTED if it cannot be loaded); make
- * the first call on a device outside stream capture.  16-bit dtype only
+ * GEMMs with fp32 accumulation on the library's tcgen05 GEMM kernel (128 x 128
+ * output tiles, operands staged by TMA, accumulators in tensor memory).  Row
+ * pitches or column blocks that are not multiples of 8 elements go to cuBLAS,
+ * which the library then loads with dlopen (GTR_ERR_UNSUPPORTED if it cannot
+ * be loaded; make such a first call on a device outside stream capture).
+ * 16-bit dtype only
  * (GTR_F16 or GTR_BF16; GTR_F32 is GTR_ERR_UNSUPPORTED); every pointer a
  * device pointer, 16-byte aligned, row-major.
  *   gtr_mixer_in_proj: x [B*T, d_model], w_in [d_model, 2 H dk + 2 H dv] whose
  *     column blocks are W_q | W_k | W_v | W_z -> q = x W_q, k = x W_k ([B, T, H,
  *     dk]), v = x W_v, z = x W_z ([B, T, H, dv]), rounded to dtype.  When dk ==
- *     dv and q, k, v, z lie at equal, non-overlapping distances in memory (one
- *     [4, B, T, H, dk] buffer) the four products are one batched call.
+ *     dv and H dk is a multiple of 128 the four products are one launch with
+ *     four outputs, else one launch each.
  *   gtr_mixer_out_proj: out [N, d_out] = y [N, d_in] w_out [d_in, d_out].
  *   Sizes of zero are an empty problem (GTR_OK, nothing launched).
  */
@@ -290,9 +293,8 @@ GTR_API gtr_status_t gtr_mixer_out_proj(const void *y, const void *w_out, void *
  *   gtr_sswiglu_fwd: x [B*T, d_model], w_in [d_model, 2C], w_out [C, d_model]
  *     -> y [B*T, d_model]; u [B*T, 2C] and h [B*T, C] are caller-provided
  *     scratch that receive the expansion and the hidden activation.  The two
- *     projections are cuBLAS GEMMs with fp32 accumulation (loaded as for
- *     gtr_mixer_in_proj; make the first call on a device outside stream
- *     capture).  C = 0 writes y = 0.
+ *     projections run on the GEMM of gtr_mixer_in_proj (fp32 accumulation,
+ *     the same cuBLAS fallback).  C = 0 writes y = 0.
  */
 GTR_API gtr_status_t gtr_sswiglu_mix(const void *u, const float *conv_w, const float *conv_b, void *h,
                                      int B, int grid_h, int grid_w, int C, int ksize, int dtype,

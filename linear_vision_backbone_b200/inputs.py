@@ -166,3 +166,51 @@ def make_custom(B: int, H: int, gh: int, gw: int, dk: int, dv: int, dtype: str, 
         "g": (torch.nn.functional.logsigmoid(u) * g_scale).contiguous(),
         "w": w.float().contiguous(),
     }
+
+
+def make_stack(nblocks: int, B: int, gh: int, gw: int, *, d_model: int = 384, H: int = 6, dk: int = 64,
+               dv: int = 64, hidden: int = 1024, rank: int = 16, dtype: str = "f16", seed: int = 0,
+               random_norms: bool = False, bias_std: float = 0.0):
+    """Random-init input and weights of a stack of GTR blocks (the block's
+    shapes: the token mixer's projections, the rank-``rank`` gate, the
+    S-SwiGLU expansion to 2 * ``hidden`` channels, its 3x3 depthwise taps and
+    its projection back to ``d_model``).
+
+    Draw order: x [B, gh*gw, d_model] ~ N(0, 1) (fp32, the residual stream),
+    then per block norm_mixer, w_in, w_down, w_up, gate_bias, gla_norm, w_o,
+    norm_ffn, w_e, conv_w, conv_b, w_p.  Projection weights ~ N(0, 1/fan_in),
+    rounded to ``dtype`` (w_down and w_up stay fp32, as the gate takes them);
+    taps ~ N(0, 1)/3 and conv_b ~ N(0, 1)*0.1 (fp32); normalisation weights are
+    ones, or N(1, 0.1^2) with ``random_norms``; gate_bias ~ N(0, 1)*bias_std
+    (None when bias_std is 0).  Returns (x, [block dict, ...]).
+    """
+    dt = DTYPES[dtype]
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(seed)
+    T = gh * gw
+    x = _randn(gen, B, T, d_model).contiguous()
+
+    def norm(n):
+        w = 1.0 + 0.1 * _randn(gen, n)
+        return (w if random_norms else torch.ones(n)).float().contiguous()
+
+    def proj(fan_in, n):
+        return (_randn(gen, fan_in, n) / math.sqrt(fan_in)).to(dt).contiguous()
+
+    blocks = []
+    for _ in range(nblocks):
+        p = {"norm_mixer": norm(d_model),
+             "w_in": proj(d_model, 2 * H * dk + 2 * H * dv),
+             "w_down": (_randn(gen, d_model, rank) / math.sqrt(d_model)).float().contiguous(),
+             "w_up": (_randn(gen, rank, H * dk) / math.sqrt(rank)).float().contiguous()}
+        b = _randn(gen, H * dk) * bias_std
+        p["gate_bias"] = b.float().contiguous() if bias_std else None
+        p["gla_norm"] = norm(dv)
+        p["w_o"] = proj(H * dv, d_model)
+        p["norm_ffn"] = norm(d_model)
+        p["w_e"] = proj(d_model, 2 * hidden)
+        p["conv_w"] = (_randn(gen, 3, 3, hidden) / 3.0).float().contiguous()
+        p["conv_b"] = (_randn(gen, hidden) * 0.1).float().contiguous()
+        p["w_p"] = proj(hidden, d_model)
+        blocks.append(p)
+    return x, blocks

@@ -22,12 +22,21 @@ Functions (each cites the page passage it follows in ``gla_oracle.c``):
   feed-forward block: SiLU(gate) times the depthwise-convolved value branch on
   the token grid, between two projections (GTR article, 方法详解 §2), in
   numpy fp64.
+* :func:`rmsnorm`, :func:`gtr_block`, :func:`gtr_stack` -- blocks of the
+  12-block backbone (GTR article, 方法详解 §1: the GLA at each block's core,
+  scan directions cycling LR, RL, TB, BT with depth) with the S-SwiGLU half,
+  pre-normalised and residual (the pages leave the wiring blank), in numpy
+  fp64, optionally rounding what each stage hands on to a 16-bit storage type.
 
 Pins: every function here is checked in ``tests/test_oracle_pins.py`` against
 results fixed independently of it (the quadratic masked form, plain causal
 linear attention at g = 0, the memoryless limit, T = 1, explicit grid flips and
 transposes, closed forms of the gate, scipy's 2-D correlation and brute-force
-loops for the depthwise convolution).
+loops for the depthwise convolution); the block stack in
+``tests/test_oracle_stack.py`` against a second fp64 implementation (the GLA's
+quadratic masked form, torch's rms_norm and grouped conv2d) and against
+properties of the stack (residual identity, direction by block index, grid
+transposition).
 """
 from __future__ import annotations
 
@@ -222,3 +231,89 @@ def sswiglu(x, w_in, weight, bias, w_out, *, gh: int, gw: int) -> np.ndarray:
     expansion x W_in -> [gate | value], the grid-mixed gated product h, and the
     projection back h W_out.  x [B, T, Cm], w_in [Cm, 2C], w_out [C, Cm]."""
     return linear(sswiglu_mix(linear(x, w_in), weight, bias, gh=gh, gw=gw), w_out)
+
+
+# ---------------------------------------------------------------------------
+# The stack of GTR blocks (GTR article, 方法详解 §1: a single-scale topology of
+# 12 blocks, each built around the Key-only GLA, whose scan direction cycles
+# LR, RL, TB, BT from Block 1 to Block 12; 方法详解 §2: the Spatial SwiGLU
+# feed-forward half).  The pages do not print a block's wiring.  Reading used
+# here: pre-normalisation with a residual around each half,
+#     x <- x + W_o-projection of GLA(mixer inputs of RMSNorm(x) * gamma_mixer)
+#     x <- x + S-SwiGLU(RMSNorm(x) * gamma_ffn),
+# with RMSNorm's epsilon 1e-5 as for the GLA output, the gate computed from the
+# same normalised input as q, k, v and z, and no final normalisation.
+
+STACK_DIRS = ("LR", "RL", "TB", "BT")
+
+
+def rmsnorm(x, weight=None, eps: float = 1e-5) -> np.ndarray:
+    """x / sqrt(mean(x^2) + eps) * weight over the last axis, fp64."""
+    x = _f64(x)
+    r = x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    return r if weight is None else r * _f64(weight)
+
+
+def store(a, dtype):
+    """``a`` rounded (round-to-nearest-even) to the storage type ``dtype``
+    (a torch dtype, or None for no rounding) and widened back to fp64: the
+    value a stage hands to the next when the pipeline keeps it in that type."""
+    a = _f64(a)
+    if dtype is None:
+        return a
+    import torch
+    return torch.from_numpy(a).to(dtype).double().numpy()
+
+
+def gtr_block(x, p, *, gh: int, gw: int, H: int, direction: str, tau: float = 16.0,
+              act_dtype=None):
+    """One GTR block on the fp64 residual stream x [B, T, d_model].
+
+    ``p`` holds the block's weights: norm_mixer [d_model], w_in [d_model,
+    2 H dk + 2 H dv] (column blocks W_q | W_k | W_v | W_z), w_down [d_model, r],
+    w_up [r, H dk], gate_bias [H dk] or None, gla_norm [dv] or None, w_o [H dv,
+    d_model], norm_ffn [d_model], w_e [d_model, 2C] (gate | value), conv_w
+    [3, 3, C], conv_b [C] or None, w_p [C, d_model].
+
+    ``act_dtype`` (None, torch.float16 or torch.bfloat16): when given, every
+    tensor that one stage hands to the next is rounded to it as a pipeline that
+    stores activations in that type does (the normalised inputs, q, k, v, z,
+    the GLA output, the S-SwiGLU expansion and hidden activation, and both
+    projections' outputs), the gate's g and the residual stream to fp32; each
+    stage computes in fp64 from the rounded values it receives.
+    """
+    f32 = None if act_dtype is None else __import__("torch").float32
+    s = lambda a: store(a, act_dtype)
+    x = _f64(x)
+    B, T, dm = x.shape
+    w_in = _f64(p["w_in"])
+    n_q = _f64(p["w_up"]).shape[1]
+    dk = n_q // H
+    dv = (w_in.shape[1] - 2 * n_q) // (2 * H)
+    a = s(rmsnorm(x, p["norm_mixer"]))
+    qkvz = s(linear(a, w_in))
+    q = qkvz[..., :n_q].reshape(B, T, H, dk)
+    k = qkvz[..., n_q:2 * n_q].reshape(B, T, H, dk)
+    v = qkvz[..., 2 * n_q:2 * n_q + H * dv].reshape(B, T, H, dv)
+    z = qkvz[..., 2 * n_q + H * dv:].reshape(B, T, H, dv)
+    g = store(gate(a, p["w_down"], p["w_up"], p.get("gate_bias"), tau), f32).reshape(B, T, H, dk)
+    y = s(gla_fwd(q, k, v, g, z, p.get("gla_norm"), gh=gh, gw=gw, direction=direction))
+    x = store(x + s(linear(y.reshape(B, T, H * dv), p["w_o"])), f32)
+    c = s(rmsnorm(x, p["norm_ffn"]))
+    u = s(linear(c, p["w_e"]))
+    h = s(sswiglu_mix(u, p["conv_w"], p.get("conv_b"), gh=gh, gw=gw))
+    return store(x + s(linear(h, p["w_p"])), f32)
+
+
+def gtr_stack(x, blocks, *, gh: int, gw: int, H: int, tau: float = 16.0, directions=None,
+              act_dtype=None) -> np.ndarray:
+    """The blocks applied in order to x [B, T, d_model]; block i scans in
+    direction ``directions[i]``, by default STACK_DIRS[i % 4] (LR, RL, TB, BT,
+    LR, ...).  Returns the residual stream after the last block, fp64."""
+    x = _f64(x)
+    if act_dtype is not None:
+        x = store(x, __import__("torch").float32)
+    for i, p in enumerate(blocks):
+        d = STACK_DIRS[i % 4] if directions is None else directions[i]
+        x = gtr_block(x, p, gh=gh, gw=gw, H=H, direction=d, tau=tau, act_dtype=act_dtype)
+    return x
