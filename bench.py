@@ -502,11 +502,13 @@ def run_ours(args, world, rank, local):
     others = None
     mixer = None
     ffn = None
+    stack = None
     if not args.no_secondary and args.workload == "16k":
         secondary = secondary_line(binding, dev)
         others = configs_lines(binding, dev)
         mixer = mixer_line(binding, dev, wl, host)
         ffn = sswiglu_line(binding, dev, wl)
+        stack = stack_line(binding, dev, wl)
 
     if rank == 0:
         cpu = oracle_rate(wl, seconds=10.0)
@@ -546,6 +548,8 @@ def run_ours(args, world, rank, local):
             line["mixer"] = mixer
         if ffn is not None:
             line["sswiglu"] = ffn
+        if stack is not None:
+            line["stack"] = stack
         print(json.dumps(line), flush=True)
 
     graphs.clear()
@@ -742,6 +746,57 @@ def sswiglu_line(binding, dev, wl, steps=200):
             "mix_gbs": gbs, "peak_gbs": peak, "peak_kind": kind, "mix_frac": gbs / peak,
             "block_ms": ms_block, "block_tokens_per_s": B * T / (ms_block * 1e-3),
             "l2": "mix: two alternating input sets (200 MB); block: warm"}
+
+
+STACK_BLOCKS = 12
+
+
+def stack_line(binding, dev, wl, reps=50):
+    """The 12-block stack on the workload's token grid (random weights:
+    d_model 384, six heads of 64, S-SwiGLU hidden width 1024, fp16
+    activations, fp32 residual stream), block i scanning LR, RL, TB, BT for
+    i mod 4, captured once into one CUDA graph (after an uncaptured call on
+    the same stream) and replayed; each replay runs all 12 blocks on the
+    residual stream the previous one left.  Reports ms per forward, tokens/s
+    and the GEMM FLOP rate over the whole forward."""
+    from linear_vision_backbone_b200 import inputs as gin2
+    B, gh, gw, H, d, dm, C = wl.B, wl.gh, wl.gw, 6, 64, 384, SSWIGLU_HIDDEN
+    x, blocks = gin2.make_stack(STACK_BLOCKS, B, gh, gw, d_model=dm, H=H, dk=d, dv=d, hidden=C,
+                                dtype="f16", seed=11)
+    stream = torch.cuda.Stream(device=dev)
+    w = binding.stack_weights(blocks, torch.float16, H, d, dev, stream=stream)
+    ws = torch.empty(binding.stack_workspace_bytes(B, gh, gw, dm, H, d, d, C), device=dev,
+                     dtype=torch.uint8)
+    xd = x.to(dev)
+    kw = dict(grid_h=gh, grid_w=gw, H=H, dk=d, dv=d, dtype=torch.float16, workspace=ws, stream=stream)
+    with torch.cuda.stream(stream):
+        binding.stack_fwd(xd, w, **kw)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        binding.stack_fwd(xd, w, **kw)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+        a.record(stream)
+        for _ in range(reps):
+            g.replay()
+        b.record(stream)
+    stream.synchronize()
+    ms = a.elapsed_time(b) / reps
+    del g
+    N = B * gh * gw
+    flops = STACK_BLOCKS * 2.0 * N * (dm * 4 * H * d + H * d * dm + dm * 2 * C + C * dm)
+    # per block: in-projection, gate, the GLA's three kernels, out-projection,
+    # add + norm, expansion, mixing, projection, add + norm; one norm first
+    per_block = 11
+    return {"workload": f"{STACK_BLOCKS} GTR blocks, {B}x{gh}x{gw} tokens, d_model {dm}, H {H}, d {d}, "
+                        f"S-SwiGLU hidden {C}, fp16 activations, fp32 residual",
+            "ms": ms, "tokens_per_s": N / (ms * 1e-3), "gemm_tflops": flops / (ms * 1e-3) / 1e12,
+            "kernels_per_forward": 1 + STACK_BLOCKS * per_block,
+            "graph": "one CUDA graph per forward, replayed",
+            "l2": "warm (16-bit weights 46 MB, activations of one block about 200 MB)"}
 
 
 def step_alg_bytes(wl):

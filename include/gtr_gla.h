@@ -305,6 +305,60 @@ GTR_API gtr_status_t gtr_sswiglu_fwd(const void *x, const void *w_in, const floa
                                      int dtype, void *stream);
 
 /*
+ * A stack of GTR blocks (GTR article, 方法详解 §1: the single-scale backbone of
+ * 12 blocks, each built around the Key-only GLA, block i scanning in direction
+ * LR, RL, TB, BT for i mod 4 = 0, 1, 2, 3; 方法详解 §2: the Spatial SwiGLU
+ * feed-forward half).  The pages leave the wiring blank; each block here is
+ *     a = RMSNorm(x) * norm_mixer
+ *     x += GLA(a W_q, a W_k, a W_v, gate(a), a W_z) W_o     (gla_norm on the GLA output)
+ *     c = RMSNorm(x) * norm_ffn
+ *     x += S-SwiGLU(c)                                      (as gtr_sswiglu_fwd, 3x3 taps)
+ * with RMSNorm's epsilon 1e-5, gate(a) = logsigmoid(a W_down W_up + bias)/tau
+ * at rank 16, and no normalisation after the last block.
+ *
+ * x [B, grid_h*grid_w, d_model] fp32 (grid order) is the residual stream,
+ * updated in place.  Every other activation is kept in `dtype` (GTR_F16 or
+ * GTR_BF16; GTR_F32 is GTR_ERR_UNSUPPORTED) in the caller's workspace of
+ * gtr_stack_workspace_bytes bytes (GTR_ERR_NO_MEMORY if smaller), 16-byte
+ * aligned.  blocks is a HOST array of nblocks entries whose members are
+ * device pointers owned by the caller; 16-bit members are in `dtype`, the
+ * others fp32; gate_packed is gtr_gate_pack's output for that block's W_down
+ * [d_model, 16] and W_up [16, H dk] with x_dtype = dtype.  dirs is a host array
+ * of nblocks directions (GTR_LR .. GTR_BT) or NULL for the rotation above.
+ * The GLA stage takes gtr_gla_fwd's workspace for `stream` (grown at its first
+ * use on that stream), so capture a stack into a CUDA graph only after one
+ * uncaptured call on the capturing stream.  Shapes: d_model a multiple of 64
+ * up to 384 and H dk a multiple of 64 up to 448 (the packed gate), dk, dv in
+ * {16, 32, 64, 128}, hidden a multiple of 8, chunk in {16, 32, 64, 128}; every
+ * stage's shape check runs before the first launch (GTR_ERR_UNSUPPORTED or
+ * GTR_ERR_INVALID_ARG, nothing launched), as do the pointer and alignment
+ * checks.  A CUDA error in a later stage returns GTR_ERR_CUDA with x partly
+ * updated.  nblocks = 0 or an empty grid is GTR_OK with nothing launched.
+ * Launches on `stream` and returns without synchronising.
+ */
+typedef struct gtr_block_weights {
+  const float *norm_mixer; /* [d_model] RMSNorm weight before the token mixer */
+  const void *w_in;        /* [d_model, 2 H dk + 2 H dv]: W_q | W_k | W_v | W_z */
+  const void *gate_packed; /* gtr_gate_pack output (W_down, W_up of this block) */
+  const float *gate_bias;  /* [H dk] or NULL */
+  const float *gla_norm;   /* [dv] RMSNorm weight of the GLA output, or NULL (ones) */
+  const void *w_o;         /* [H dv, d_model] */
+  const float *norm_ffn;   /* [d_model] RMSNorm weight before the S-SwiGLU half */
+  const void *w_e;         /* [d_model, 2 hidden]: gate channels, then value channels */
+  const float *conv_w;     /* [3, 3, hidden] depthwise taps */
+  const float *conv_b;     /* [hidden] or NULL */
+  const void *w_p;         /* [hidden, d_model] */
+} gtr_block_weights;
+
+/* Workspace bytes of gtr_stack_fwd (0 for negative sizes). */
+GTR_API size_t gtr_stack_workspace_bytes(int B, int grid_h, int grid_w, int d_model, int H, int dk, int dv,
+                                         int hidden);
+GTR_API gtr_status_t gtr_stack_fwd(float *x, const gtr_block_weights *blocks, int nblocks, const int *dirs,
+                                   int B, int grid_h, int grid_w, int d_model, int H, int dk, int dv,
+                                   int hidden, float tau, int chunk, int dtype, void *workspace,
+                                   size_t workspace_bytes, void *stream);
+
+/*
  * Chunk-boundary states, for testing the first two stages on their own: the
  * state each chunk of `chunk` scan positions ends with,
  *   states [B, H, ceil(T/chunk), dk, dv] fp32, entry c = S after scan position

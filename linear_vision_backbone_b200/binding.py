@@ -28,8 +28,17 @@ EXPORTS = (
     "gtr_gla_set_path", "gtr_gla_path_for", "gtr_last_device_status", "gtr_gla_segment_chunks",
     "gtr_gla_fwd_noalloc", "gtr_gate_packed_bytes", "gtr_gate_pack", "gtr_gate_fwd_packed",
     "gtr_gla_segment_count", "gtr_gla_fwd_gated", "gtr_gla_fwd_gated_timed", "gtr_mixer_in_proj",
-    "gtr_mixer_out_proj", "gtr_sswiglu_mix", "gtr_sswiglu_fwd",
+    "gtr_mixer_out_proj", "gtr_sswiglu_mix", "gtr_sswiglu_fwd", "gtr_stack_workspace_bytes",
+    "gtr_stack_fwd",
 )
+
+BLOCK_FIELDS = ("norm_mixer", "w_in", "gate_packed", "gate_bias", "gla_norm", "w_o", "norm_ffn", "w_e",
+                "conv_w", "conv_b", "w_p")
+
+
+class BlockWeights(ctypes.Structure):
+    """``gtr_block_weights``: one block's device pointers, in the header's order."""
+    _fields_ = [(n, ctypes.c_void_p) for n in BLOCK_FIELDS]
 
 _lock = threading.Lock()
 _lib = None
@@ -79,6 +88,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
             "gtr_mixer_out_proj": ([P, P, P, ctypes.c_longlong, I, I, I, P], I),
             "gtr_sswiglu_mix": ([P, P, P, P, I, I, I, I, I, I, P], I),
             "gtr_sswiglu_fwd": ([P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P], I),
+            "gtr_stack_workspace_bytes": ([I, I, I, I, I, I, I, I], Z),
+            "gtr_stack_fwd": ([P, P, I, P, I, I, I, I, I, I, I, I, F, I, I, P, Z, P], I),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -345,6 +356,62 @@ def sswiglu_fwd(x, w_in, conv_w, conv_b, w_out, *, grid_h: int, grid_w: int, scr
                                 _stream(stream))
     _check("gtr_sswiglu_fwd", rc)
     return y
+
+
+def stack_workspace_bytes(B: int, grid_h: int, grid_w: int, d_model: int, H: int, dk: int, dv: int,
+                          hidden: int) -> int:
+    return int(load().gtr_stack_workspace_bytes(B, grid_h, grid_w, d_model, H, dk, dv, hidden))
+
+
+def stack_weights(blocks, dtype: torch.dtype, H: int, dk: int, device, stream=None):
+    """Device copies of host block weights (dicts with the keys of
+    ``BLOCK_FIELDS`` except gate_packed, plus w_down and w_up), with each
+    block's gate weights packed by ``gtr_gate_pack`` for x of ``dtype``."""
+    out = []
+    for p in blocks:
+        d = {n: (None if p.get(n) is None else p[n].to(device).contiguous())
+             for n in BLOCK_FIELDS if n != "gate_packed"}
+        d["gate_packed"] = gate_pack(p["w_down"].to(device).contiguous(), p["w_up"].to(device).contiguous(),
+                                     dtype, H, dk, stream=stream)
+        out.append(d)
+    return out
+
+
+def stack_fwd(x, blocks, *, grid_h: int, grid_w: int, H: int, dk: int, dv: int, dtype: torch.dtype,
+              tau: float = 16.0, chunk: int = 64, directions: Optional[Sequence[str]] = None,
+              workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """``gtr_stack_fwd``: the blocks applied in order to the fp32 residual
+    stream x [B, grid_h*grid_w, d_model] in place (returns x).  ``blocks`` are
+    dicts of device tensors (``stack_weights``); every other activation is in
+    ``dtype``; ``workspace`` is a uint8 device tensor of at least
+    ``stack_workspace_bytes`` bytes, allocated when not given."""
+    _need(x, "x", torch.float32)
+    if x.dim() != 3 or x.shape[1] != grid_h * grid_w:
+        raise ValueError("x must be [B, grid_h * grid_w, d_model]")
+    B, T, dm = x.shape
+    if not blocks:
+        return x
+    hidden = blocks[0]["w_p"].shape[0]
+    arr = (BlockWeights * len(blocks))()
+    for i, p in enumerate(blocks):
+        for n in BLOCK_FIELDS:
+            t = p.get(n)
+            if t is not None:
+                _need(t, n)
+                setattr(arr[i], n, t.data_ptr())
+    dirs = None
+    if directions is not None:
+        if len(directions) != len(blocks):
+            raise ValueError("one direction per block")
+        dirs = (ctypes.c_int * len(blocks))(*[DIR_IDS[d] for d in directions])
+    need = stack_workspace_bytes(B, grid_h, grid_w, dm, H, dk, dv, hidden)
+    if workspace is None:
+        workspace = torch.empty(need, device=x.device, dtype=torch.uint8)
+    rc = load().gtr_stack_fwd(_ptr(x), arr, len(blocks), dirs, B, grid_h, grid_w, dm, H, dk, dv, hidden,
+                              float(tau), int(chunk), DTYPE_IDS[dtype], _ptr(workspace), workspace.numel(),
+                              _stream(stream))
+    _check("gtr_stack_fwd", rc)
+    return x
 
 
 def gla_fwd_noalloc(q, k, v, g, z, w=None, *, grid_h: int, grid_w: int, direction: str = "LR",

@@ -255,9 +255,11 @@ def rmsnorm(x, weight=None, eps: float = 1e-5) -> np.ndarray:
 
 
 def store(a, dtype):
-    """``a`` rounded (round-to-nearest-even) to the storage type ``dtype``
-    (a torch dtype, or None for no rounding) and widened back to fp64: the
-    value a stage hands to the next when the pipeline keeps it in that type."""
+    """``a`` rounded to the storage type ``dtype`` (a torch dtype, or None for
+    no rounding) and widened back to fp64: the value a stage hands to the next
+    when the pipeline keeps it in that type.  torch's CPU cast rounds fp64 to
+    fp32 and then to a 16-bit type, each step to nearest-even: the rounding of
+    a pipeline that computes in fp32 and stores 16 bits."""
     a = _f64(a)
     if dtype is None:
         return a

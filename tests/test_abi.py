@@ -171,3 +171,48 @@ def test_sswiglu_rejects_invalid_arguments(lib):
     assert fwd(None, None, None, None, None, None, None, None, 1, 4, 4, 0, 1024, 3, 1, S) == 0
     assert fwd(P, P, P, P, P, P, None, P, 1, 4, 4, 384, 1024, 3, 1, S) == -1
     assert fwd(P, P, P, P, P, P, P, ctypes.c_void_p(8), 1, 4, 4, 384, 1024, 3, 1, S) == -3
+
+
+def test_stack_rejects_invalid_arguments(lib):
+    P = ctypes.c_void_p(16)
+    S = None
+    fwd = lib.gtr_stack_fwd
+    blk = (binding.BlockWeights * 2)()
+    for b in blk:
+        for n in binding.BLOCK_FIELDS:
+            setattr(b, n, 4096)
+    need = lib.gtr_stack_workspace_bytes(1, 8, 8, 384, 6, 64, 64, 1024)
+    assert need > 0 and lib.gtr_stack_workspace_bytes(-1, 8, 8, 384, 6, 64, 64, 1024) == 0
+    W = ctypes.c_void_p(1 << 20)
+    # x, blocks, nblocks, dirs, B, gh, gw, d_model, H, dk, dv, hidden, tau, chunk, dtype, ws, ws_bytes, stream
+    args = [P, blk, 2, None, 1, 8, 8, 384, 6, 64, 64, 1024, 16.0, 64, 1, W, need, S]
+
+    def call(**kw):
+        a = list(args)
+        names = ["x", "blocks", "n", "dirs", "B", "gh", "gw", "dm", "H", "dk", "dv", "hidden", "tau", "chunk",
+                 "dtype", "ws", "ws_bytes", "stream"]
+        for k, v in kw.items():
+            a[names.index(k)] = v
+        return fwd(*a)
+
+    assert call(B=-1) == -1
+    assert call(n=-1) == -1
+    assert call(tau=0.0) == -1
+    assert call(dtype=0) == -2                     # fp32 activations
+    assert call(dtype=7) == -1
+    assert call(dk=48, dv=48, H=8) == -2           # no GLA kernel for dk = 48
+    assert call(dm=320 + 8) == -2                  # the packed gate takes multiples of 64
+    assert call(hidden=1020) == -2                 # S-SwiGLU width not a multiple of 8
+    assert call(chunk=48) == -2
+    assert call(n=0) == 0 and call(B=0) == 0       # empty: nothing launched
+    assert call(x=None) == -1 and call(blocks=None) == -1 and call(ws=None) == -1
+    assert call(ws_bytes=need - 1) == -4
+    assert call(x=ctypes.c_void_p(20)) == -3
+    blk[1].w_o = None
+    assert call() == -1
+    blk[1].w_o = 4096
+    blk[0].conv_w = 4100
+    assert call() == -3
+    blk[0].conv_w = 4096
+    bad_dirs = (ctypes.c_int * 2)(0, 4)            # per-batch rotation is not a block direction
+    assert call(dirs=bad_dirs) == -1
