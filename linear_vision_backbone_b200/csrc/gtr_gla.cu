@@ -16,7 +16,6 @@
 #include "scan_kernel.cuh"
 #include "tc_kernels.cuh"
 #include "gate_tc.cuh"
-#include "gemm_kernel.cuh"
 #include "mixer_proj.cuh"
 
 namespace {
@@ -634,52 +633,9 @@ int gla_fwd_noalloc_impl(const void* q, const void* k, const void* v, const floa
 
 }  // namespace
 
-namespace gtr {
-
-// The projections' GEMM (gemm_tc.cuh, gemm_kernel.cuh).
-int gemm_tc(int dtype, const void* A, int lda, const void* B, int ldb, void* const* C, int nout, int ncols,
-            int ldc, int M, int N, int K, cudaStream_t st) {
-  if (dtype != GTR_F16 && dtype != GTR_BF16) return GTR_ERR_UNSUPPORTED;
-  if (M <= 0 || N <= 0 || K <= 0) return GTR_OK;
-  if (nout < 1 || nout > gemm::kMaxOut) return GTR_ERR_UNSUPPORTED;
-  if (nout == 1) ncols = N;
-  if (nout > 1 && (ncols % gemm::kBN != 0 || (long long)nout * ncols != N)) return GTR_ERR_UNSUPPORTED;
-  // tensor maps: 16-byte aligned bases and row pitches
-  if (lda % 8 || ldb % 8 || ldc % 8 || ncols % 8 || !aligned16(A) || !aligned16(B)) return GTR_ERR_UNSUPPORTED;
-  for (int o = 0; o < nout; ++o)
-    if (!C[o] || !aligned16(C[o])) return GTR_ERR_UNSUPPORTED;
-  int dev;
-  if (int rc = current_device(&dev)) return rc;
-  const CUtensorMapDataType dt = dtype == GTR_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  gemm::Maps mp{};
-  if (int rc = tmap_2d(&mp.a, dt, A, (unsigned long long)M, (unsigned long long)K, (unsigned long long)lda * 2,
-                       gemm::kBK, gemm::kBM))
-    return rc;
-  if (int rc = tmap_2d(&mp.b, dt, B, (unsigned long long)K, (unsigned long long)N, (unsigned long long)ldb * 2, 64,
-                       gemm::kBK))
-    return rc;
-  for (int o = 0; o < nout; ++o)
-    if (int rc = tmap_2d(&mp.c[o], dt, C[o], (unsigned long long)M, (unsigned long long)ncols,
-                         (unsigned long long)ldc * 2, 64, gemm::kBM))
-      return rc;
-  gemm::Params p{M, N, K, nout, ncols, (M + gemm::kBM - 1) / gemm::kBM, (N + gemm::kBN - 1) / gemm::kBN,
-                 (K + gemm::kBK - 1) / gemm::kBK};
-  const long long tiles = (long long)p.mt * p.nt;
-  const unsigned grid = (unsigned)(tiles < sm_count(dev) ? tiles : sm_count(dev));
-  static bool done_h[kMaxDevices], done_b[kMaxDevices];
-  if (dtype == GTR_BF16) {
-    if (int rc = ensure_smem(gemm::gemm_tc_kernel<true>, gemm::kSmem, done_b, dev)) return rc;
-    return launch_pdl(gemm::gemm_tc_kernel<true>, dim3(grid), dim3(gemm::kThreads), gemm::kSmem, st, p, mp)
-               ? GTR_ERR_CUDA
-               : GTR_OK;
-  }
-  if (int rc = ensure_smem(gemm::gemm_tc_kernel<false>, gemm::kSmem, done_h, dev)) return rc;
-  return launch_pdl(gemm::gemm_tc_kernel<false>, dim3(grid), dim3(gemm::kThreads), gemm::kSmem, st, p, mp)
-             ? GTR_ERR_CUDA
-             : GTR_OK;
-}
-
-}  // namespace gtr
+// The projections' GEMM: its host side (tensor maps, tile width, launch),
+// after the helpers above that it uses.
+#include "gemm_host.cuh"
 
 extern "C" {
 
