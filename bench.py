@@ -272,6 +272,33 @@ def aggregate_value(units_per_rank: int, steps: int, ms_max: float, world: int) 
 
 
 # ---------------------------------------------------------------- CPU oracle
+def oracle_rate_config(wl, seconds=2.0):
+    """Token-heads/s of the fp64 oracle on a bounded sample of any workload:
+    the gate + GLA of the first grid rows for the projected workloads (as
+    oracle_rate), the GLA on its drawn gates for the others (every head of
+    batch entry 0 over the first rows holding about 4096 tokens)."""
+    if wl.recipe == "proj":
+        return oracle_rate(wl, seconds=seconds, rows=8)
+    import oracle
+    cores = os.cpu_count() or 1
+    used = min(oracle.set_threads(cores), wl.H)
+    d = gin.make_inputs(wl)
+    rows = max(1, min(wl.gh, 4096 // wl.gw))
+    T = rows * wl.gw
+    q, k, v, g, z = (d[n][:1, :T] for n in ("q", "k", "v", "g", "z"))
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        oracle.gla_fwd(q, k, v, g, z, d["w"], gh=rows, gw=wl.gw, direction=wl.dirs[0])
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return {"value": n * T * wl.H / el, "unit": "token-heads/s", "cores": used, "kind": "oracle",
+            "sample": f"GLA of all {wl.H} heads over the first {rows}x{wl.gw}={T} tokens of the "
+                      f"{wl.name} workload (batch entry 0), {n} repetitions in {el:.2f} s, fp64"}
+
+
 def oracle_rate(wl, seconds=10.0, rows=32):
     """Token-heads/s of the fp64 oracle (gate + GLA) on a bounded sample: every
     head of the first `rows` grid rows of batch entry 0, repeated for about
@@ -515,6 +542,11 @@ def run_ours(args, world, rank, local):
 
     if rank == 0:
         cpu = oracle_rate(wl, seconds=10.0)
+        if others is not None:
+            for name, c in others.items():
+                c["cpu_oracle"] = oracle_rate_config(config_workload(name), seconds=2.0)
+        if secondary is not None:
+            secondary["cpu_oracle"] = oracle_rate_config(gin.WORKLOADS["640"], seconds=2.0)
         line = {
             "metric": "GLA fwd token-heads/s (gate projection + Key-only GLA)",
             "value": value, "unit": "token-heads/s", "n_gpus": world, "steps": args.steps,
@@ -887,13 +919,20 @@ def secondary_line(binding, dev, steps=2000):
     return config_line(binding, dev, gin.WORKLOADS["640"], steps=steps)
 
 
+def config_workload(name):
+    """The workload of a name in the configs entry: a workload's own name, or
+    sweep-<grid> for the sweep at that square grid."""
+    if name.startswith("sweep-"):
+        return gin.WORKLOADS["sweep"].with_grid(int(name.split("-")[1]))
+    return gin.WORKLOADS[name]
+
+
 def configs_lines(binding, dev):
     """Every other workload: the batched 640x640 case and the d = 128 sweep."""
-    out = {"640b8": config_line(binding, dev, gin.WORKLOADS["640b8"], steps=500),
-           "tiny": config_line(binding, dev, gin.WORKLOADS["tiny"], steps=500)}
+    out = {n: config_line(binding, dev, config_workload(n), steps=500) for n in ("640b8", "tiny")}
     for gsz in gin.SWEEP_GRIDS:
-        wl = gin.WORKLOADS["sweep"].with_grid(gsz)
-        out[f"sweep-{gsz}"] = config_line(binding, dev, wl, steps=100 if gsz >= 128 else 300)
+        name = f"sweep-{gsz}"
+        out[name] = config_line(binding, dev, config_workload(name), steps=100 if gsz >= 128 else 300)
     return out
 
 
