@@ -83,7 +83,7 @@ int gemm_tc(int dtype, const void* A, int lda, const void* B, int ldb, void* con
     return rc;
   for (int o = 0; o < nout; ++o)
     if (int rc = tmap_2d(&mp.c[o], dt, C[o], (unsigned long long)M, (unsigned long long)ncols,
-                         (unsigned long long)ldc * 2, 64, gemm::kBM))
+                         (unsigned long long)ldc * 2, 64, 32))
       return rc;
   // Tile choice, as measured on the projections' shapes (16384 rows): CTA
   // pairs on 256 x 256 tiles only for deep products (K >= 1024, N whole tiles
