@@ -141,29 +141,35 @@ __global__ void __launch_bounds__(kMixThreads, 3) sswiglu_mix_kernel(const E* __
   const E* ub = u + (size_t)b * gh * gw * ldu;
   E* hb = h + (size_t)b * gh * gw * C;
   const bool cok = c < C;
+  const int cl = cok ? c : 0;
 
-  // stage input row r (value) and output row r - 1 (gate) into r's slot
-  auto issue = [&](int r) {
-    unsigned char* slot = ring + ((r - y0 + 1) % kStages) * kSlotBytes;
+  // Row-0 addresses of the pieces this thread copies and stores (clamped to a
+  // valid piece where the copy reads nothing); a row adds rs (input) or hrs
+  // (output) elements.
+  const size_t rs = (size_t)gw * ldu, hrs = (size_t)gw * C;
+  const int xc = ok ? x : 0;
+  const E* vcol = ub + C + cl + (size_t)xc * ldu;
+  const E* vleft = ub + C + cl + (size_t)(x0 > 0 ? x0 - 1 : 0) * ldu;
+  const E* vright = ub + C + cl + (size_t)(x0 + kTileCols < gw ? x0 + kTileCols : 0) * ldu;
+  const E* gcol = ub + cl + (size_t)xc * ldu;
+  E* hcol = hb + (size_t)xc * C + cl;
+
+  // stage input row r (value) and output row r - 1 (gate) into slot `si`
+  auto issue = [&](int r, int si) {
+    unsigned char* slot = ring + si * kSlotBytes;
     const bool rok = r >= 0 && r < gh;
-    const E* vrow = ub + (size_t)(rok ? r : 0) * gw * ldu + C + (cok ? c : 0);
-    cp16(slot + ((col + 1) * kOcts + oct) * 16, ok && rok ? vrow + (size_t)x * ldu : ub, ok && rok);
-    if (col == 0) {
-      const bool v = cok && rok && x0 > 0;
-      cp16(slot + oct * 16, v ? vrow + (size_t)(x0 - 1) * ldu : ub, v);
-    }
-    if (col == kTileCols - 1) {
-      const bool v = cok && rok && x0 + kTileCols < gw;
-      cp16(slot + ((kTileCols + 1) * kOcts + oct) * 16, v ? vrow + (size_t)(x0 + kTileCols) * ldu : ub, v);
-    }
+    const size_t ro = (size_t)(rok ? r : 0) * rs;
+    cp16(slot + ((col + 1) * kOcts + oct) * 16, vcol + ro, ok && rok);
+    if (col == 0) cp16(slot + oct * 16, vleft + ro, cok && rok && x0 > 0);
+    if (col == kTileCols - 1)
+      cp16(slot + ((kTileCols + 1) * kOcts + oct) * 16, vright + ro, cok && rok && x0 + kTileCols < gw);
     const int yg = r - 1;
     const bool gv = ok && yg >= y0 && yg < y1;
-    cp16(slot + kValBytes + threadIdx.x * 16, gv ? ub + ((size_t)yg * gw + x) * ldu + c : ub, gv);
+    cp16(slot + kValBytes + threadIdx.x * 16, gcol + (size_t)(gv ? yg : 0) * rs, gv);
   };
 
   // taps and bias of the thread's eight channels, as four channel pairs
   f2_t w[3][3][4], bias[4];
-  const int cl = cok ? c : 0;
 #pragma unroll
   for (int i = 0; i < 3; ++i)
 #pragma unroll
@@ -184,16 +190,17 @@ __global__ void __launch_bounds__(kMixThreads, 3) sswiglu_mix_kernel(const E* __
 
 #pragma unroll
   for (int i = 0; i < kStages - 1; ++i) {
-    if (y0 - 1 + i <= y1) issue(y0 - 1 + i);
+    if (y0 - 1 + i <= y1) issue(y0 - 1 + i, i);
     cp_commit();
   }
   f2_t acc_prev[4], acc_cur[4];    // partial sums of output rows r-1 and r (channel pairs)
 #pragma unroll
   for (int k = 0; k < 4; ++k) acc_prev[k] = acc_cur[k] = bias[k];
-  for (int r = y0 - 1; r <= y1; ++r) {
+  static_assert((kStages & (kStages - 1)) == 0, "ring index by mask");
+  for (int r = y0 - 1, si = 0; r <= y1; ++r, si = (si + 1) & (kStages - 1)) {
     cp_wait<kStages - 2>();
     __syncthreads();
-    const unsigned char* slot = ring + ((r - y0 + 1) % kStages) * kSlotBytes;
+    const unsigned char* slot = ring + si * kSlotBytes;
     f2_t vl[4], vm[4], vr[4];
     widen8x2(*reinterpret_cast<const uint4*>(slot + (col * kOcts + oct) * 16), (const E*)nullptr, vl);
     widen8x2(*reinterpret_cast<const uint4*>(slot + ((col + 1) * kOcts + oct) * 16), (const E*)nullptr, vm);
@@ -216,7 +223,7 @@ __global__ void __launch_bounds__(kMixThreads, 3) sswiglu_mix_kernel(const E* __
         o[2 * k] = v.x;
         o[2 * k + 1] = v.y;
       }
-      *reinterpret_cast<uint4*>(hb + ((size_t)y * gw + x) * C + c) = narrow8(o, (const E*)nullptr);
+      *reinterpret_cast<uint4*>(hcol + (size_t)y * hrs) = narrow8(o, (const E*)nullptr);
     }
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -224,7 +231,7 @@ __global__ void __launch_bounds__(kMixThreads, 3) sswiglu_mix_kernel(const E* __
       acc_cur[k] = acc_next[k];
     }
     // the slot of row r - 1, read by every thread before this iteration's barrier
-    if (r + kStages - 1 <= y1) issue(r + kStages - 1);
+    if (r + kStages - 1 <= y1) issue(r + kStages - 1, (si + kStages - 1) & (kStages - 1));
     cp_commit();
   }
   cp_wait<0>();
