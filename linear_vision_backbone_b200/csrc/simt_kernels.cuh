@@ -10,9 +10,10 @@
 //                o_s = q_s S_s, then RMSNorm x SiLU(z) in the epilogue.
 // Inside a segment this path applies the recurrence of 方法详解 §1 token by
 // token, S = diag(exp g_s) S + k_s^T v_s, with the dk x dv state spread over
-// the 256 threads of the block (thread -> column j = tid % dv and rows
-// i = tid / dv + r * (256 / dv)).  Every product is an fp32 FMA: no
-// factorisation of the decay, so no overflow whatever the gate values.
+// the 256 threads of the block (thread -> column j = tid % dv and the ROWS
+// consecutive rows i = (tid / dv) * ROWS + r, so that a warp reads the staged
+// per-row values of a token as 16-byte broadcasts).  Every product is an fp32
+// FMA: no factorisation of the decay, so no overflow whatever the gate values.
 #pragma once
 #include "common.cuh"
 
@@ -34,6 +35,19 @@ __device__ __forceinline__ size_t token_row(int b, int t, int T_, int H, int h) 
   return ((size_t)b * T_ + t) * H + h;
 }
 
+// Four consecutive staged floats (16-byte aligned) when ROWS is a multiple of
+// four, else one at a time.
+template <int ROWS>
+__device__ __forceinline__ void rows4(const float* p, int r, float (&x)[4]) {
+  if constexpr (ROWS % 4 == 0) {
+    const float4 f = *reinterpret_cast<const float4*>(p + r);
+    x[0] = f.x; x[1] = f.y; x[2] = f.z; x[3] = f.w;
+  } else {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) x[e] = (r + e < ROWS) ? p[r + e] : 0.f;
+  }
+}
+
 template <typename T, int ROWS>
 __global__ void __launch_bounds__(kSimtThreads)
 gla_summary_simt(const T* __restrict__ k, const T* __restrict__ v, const float* __restrict__ g,
@@ -49,7 +63,7 @@ gla_summary_simt(const T* __restrict__ k, const T* __restrict__ v, const float* 
   const int d = dir_of_batch(dir, b);
   if (d < 0 || d > 3) { if (threadIdx.x == 0) gtr_flag(kStatusBadDir); return; }
   const int tid = threadIdx.x;
-  const int nrg = kSimtThreads / dv, j = tid % dv, rg = tid / dv;
+  const int j = tid % dv, rg = tid / dv;
   const int nc = (T_ + chunk - 1) / chunk;
   const int s0 = seg_first_chunk(seg, nc, nseg) * chunk;
   const int s1 = min(T_, seg_first_chunk(seg + 1, nc, nseg) * chunk);
@@ -76,10 +90,16 @@ gla_summary_simt(const T* __restrict__ k, const T* __restrict__ v, const float* 
     __syncthreads();
     for (int u = 0; u < nb; ++u) {
       const float vj = vs[u * dv + j];
+      const float* ar = as + u * dk + rg * ROWS;
+      const float* kr = ks + u * dk + rg * ROWS;
 #pragma unroll
-      for (int r = 0; r < ROWS; ++r) {
-        const int i = rg + r * nrg;
-        S[r] = fmaf(as[u * dk + i], S[r], ks[u * dk + i] * vj);
+      for (int r = 0; r < ROWS; r += 4) {
+        float a4[4], k4[4];
+        rows4<ROWS>(ar, r, a4);
+        rows4<ROWS>(kr, r, k4);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (r + e < ROWS) S[r + e] = fmaf(a4[e], S[r + e], k4[e] * vj);
       }
     }
     if (tid < dk)
@@ -87,7 +107,7 @@ gla_summary_simt(const T* __restrict__ k, const T* __restrict__ v, const float* 
   }
   float* outS = wsS + ((size_t)bh * nseg + seg) * dk * dv;
 #pragma unroll
-  for (int r = 0; r < ROWS; ++r) outS[(size_t)(rg + r * nrg) * dv + j] = S[r];
+  for (int r = 0; r < ROWS; ++r) outS[(size_t)(rg * ROWS + r) * dv + j] = S[r];
   if (tid < dk) wsA[((size_t)bh * nseg + seg) * dk + tid] = expf(lsum);   // segment decay factor
 }
 
@@ -117,7 +137,7 @@ gla_output_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __res
   const float* inS = wsS + ((size_t)bh * nseg + seg) * dk * dv;
   float S[ROWS];
 #pragma unroll
-  for (int r = 0; r < ROWS; ++r) S[r] = inS[(size_t)(rg + r * nrg) * dv + j];
+  for (int r = 0; r < ROWS; ++r) S[r] = inS[(size_t)(rg * ROWS + r) * dv + j];
   for (int sb = s0; sb < s1; sb += kSimtBatch) {
     const int nb = min(kSimtBatch, s1 - sb);
     __syncthreads();
@@ -137,12 +157,22 @@ gla_output_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __res
     __syncthreads();
     for (int u = 0; u < nb; ++u) {
       const float vj = vs[u * dv + j];
+      const float* ar = as + u * dk + rg * ROWS;
+      const float* kr = ks + u * dk + rg * ROWS;
+      const float* qr = qs + u * dk + rg * ROWS;
       float part = 0.f;
 #pragma unroll
-      for (int r = 0; r < ROWS; ++r) {
-        const int i = rg + r * nrg;
-        S[r] = fmaf(as[u * dk + i], S[r], ks[u * dk + i] * vj);
-        part = fmaf(qs[u * dk + i], S[r], part);
+      for (int r = 0; r < ROWS; r += 4) {
+        float a4[4], k4[4], q4[4];
+        rows4<ROWS>(ar, r, a4);
+        rows4<ROWS>(kr, r, k4);
+        rows4<ROWS>(qr, r, q4);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (r + e < ROWS) {
+            S[r + e] = fmaf(a4[e], S[r + e], k4[e] * vj);
+            part = fmaf(q4[e], S[r + e], part);
+          }
       }
       po[(u * nrg + rg) * dv + j] = part;
     }
