@@ -15,6 +15,7 @@
 #include "simt_kernels.cuh"
 #include "scan_kernel.cuh"
 #include "tc_kernels.cuh"
+#include "tc128_kernels.cuh"
 #include "gate_tc.cuh"
 #include "mixer_proj.cuh"
 
@@ -128,7 +129,7 @@ int check_gla_args(int B, int H, int gh, int gw, int dk, int dv, int dir, int ch
 }
 
 bool tc_supported(int dk, int dv, int chunk, int dtype) {
-  return tc_shape_supported(dk, dv, chunk, dtype);
+  return tc_shape_supported(dk, dv, chunk, dtype) || tc128_shape_supported(dk, dv, chunk, dtype);
 }
 
 int choose_path(int dk, int dv, int chunk, int dtype) {
@@ -149,6 +150,16 @@ int make_plan(Plan* p, int dev, int B, int H, int gh, int gw, int dk, int dv, in
   const long long bh = (long long)B * H;
   const int per_sm = path == GTR_PATH_TC ? tc_blocks_per_sm(dk, dv) : 4;
   const long long slots = (long long)sm_count(dev) * per_sm;
+  if (path == GTR_PATH_TC && dk == tc128::kD) {
+    // the d = 128 tensor-core kernels take every chunk as its own segment; a
+    // plan with longer segments runs on the SIMT kernels
+    if (force_nseg > 0 && force_nseg < p->nc) {
+      if (g_path_setting.load() == GTR_PATH_TC) return GTR_ERR_UNSUPPORTED;
+      p->path = GTR_PATH_SIMT;
+    } else {
+      force_nseg = p->nc;
+    }
+  }
   if (force_nseg > 0) {
     p->nseg = force_nseg < p->nc ? force_nseg : p->nc;
   } else {
@@ -446,6 +457,10 @@ int launch_simt(const Plan& p, const void* q, const void* k, const void* v, cons
 int launch_stage(const Plan& p, const void* q, const void* k, const void* v, const float* g,
                  const void* z, const float* w, void* out, float* wsS, float* wsA, cudaStream_t st,
                  int stage) {
+  if (p.path == GTR_PATH_TC && p.dk == tc128::kD) {
+    const tc128::Params pp{q, k, v, g, z, w, wsS, wsA, out, p.H, p.T, p.gh, p.gw, p.dir, p.nc};
+    return launch_tc128(p.dtype, stage, pp, p.B * p.H, st, p.dev) ? GTR_ERR_CUDA : GTR_OK;
+  }
   if (p.path == GTR_PATH_TC) {
     tc::Maps maps;
     const bool boxes = chunk_maps(p, stage == 1 ? q : nullptr, k, v, g, &maps);
@@ -540,7 +555,7 @@ int gla_fwd_gated_impl(const void* x, int x_dtype, const void* packed, const flo
   if ((rc = make_plan(&p, dev, B, H, gh, gw, dk, dv, dir, chunk, dtype, 0))) return rc;
   cudaStream_t st = (cudaStream_t)stream;
   if ((rc = record(ev, 0, st))) return rc;
-  if (p.path != GTR_PATH_TC) {
+  if (p.path != GTR_PATH_TC || dk != tc::kD) {
     if ((rc = gate_fwd_packed_launch(x_dtype, x, packed, bias, g_out, N, d_model, (int)HD, tau, st, dev)))
       return rc;
     if ((rc = record(ev, 1, st))) return rc;

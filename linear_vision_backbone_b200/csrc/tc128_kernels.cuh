@@ -1,0 +1,562 @@
+// tc128_kernels.cuh -- the tensor-core path of the Key-only GLA for head
+// dimensions dk = dv = 128 (16-bit q/k/v/z, fp32 gates, 64-token chunks).
+//
+// The chunkwise operator of the GTR article (方法详解 §4: chunk summaries on
+// tensor cores, a light pass over the chunk-boundary states, chunk outputs
+// with the scores kept on chip and the output gate fused into the epilogue),
+// with every chunk an independent block:
+//
+//   gla_sum_tc128  per (sequence, chunk): the state the chunk produces from
+//                  zero, dS = sum_t diag(e^{Gam - G_t}) k_t^T v_t (G_t the
+//                  in-chunk cumulative log-gate through token t, Gam its
+//                  total, so every weight is at most one), as one
+//                  tcgen05.mma product dS^T = V^T k^ (M = 128 value dims,
+//                  N = 128 key dims, K = 64 tokens) with k^ in two 16-bit
+//                  terms, and the chunk's decay factor e^{Gam}.
+//   (the boundary scan over chunks, scan_kernel.cuh, turns dS into the state
+//   each chunk starts from)
+//   gla_out_tc128  per (sequence, chunk): o = q~ S + mask(q~ k~^T) V with
+//                  q~ = q e^{G} and k~ = k e^{-G} referenced to the chunk
+//                  start, each operand in two bf16 terms (hi + lo) and the
+//                  products hi hi + hi lo + lo hi accumulated in fp32 in
+//                  tensor memory (M = 64 tokens); then RMSNorm over the 128
+//                  value dims x w x SiLU(z), stored at the tokens' grid rows.
+//                  Chunks whose log-gate span exceeds kSpan nats (where k~
+//                  would leave the terms' precision) take their scores from
+//                  an exact CUDA-core sum instead.
+//
+// Tiles in shared memory use the 128-byte swizzle of the tensor cores'
+// operand layout: a tile of R rows x 128 columns (16-bit) is two column
+// halves of 64, each R rows of 128 bytes; element (r, c) of half c / 64 sits
+// at r * 128 + ((c % 64 / 8) ^ (r % 8)) * 16 + (c % 8) * 2.  The same bytes
+// are a K-major operand when the rows are M or N and a MN-major operand when
+// the rows are K.
+#pragma once
+#include "tc_kernels.cuh"
+
+namespace gtr {
+namespace tc128 {
+
+using tc::saddr;
+
+constexpr int kC = 64;             // tokens per chunk
+constexpr int kD = 128;            // dk = dv
+constexpr int kThreads = 256;
+constexpr float kSpan = 20.0f;     // the chunk's log-gate span (nats) beyond which its scores are exact
+constexpr int kHalf64 = kC * 128;  // one 64-column half of a 64-row tile: 8 KB
+constexpr int kTile64 = 2 * kHalf64;           // 64 rows x 128 columns, 16-bit: 16 KB
+constexpr int kHalf128 = kD * 128;             // one half of a 128-row tile: 16 KB
+constexpr int kTile128 = 2 * kHalf128;         // 128 rows x 128 columns, 16-bit: 32 KB
+constexpr int kGBytes = kC * kD * 4;           // fp32 gate / cumulative log-gate: 32 KB
+
+struct Params {
+  const void* q; const void* k; const void* v; const float* g; const void* z; const float* w;
+  float* wsS; float* wsA; void* out;
+  int H, T, gh, gw, dir, nc;
+};
+
+// byte offset of element (r, c) in a swizzled tile of `rows` rows x 128 columns
+__device__ __forceinline__ uint32_t sw_off(int rows, int r, int c) {
+  return (uint32_t)((c >> 6) * rows * 128 + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) + (c & 7) * 2);
+}
+// the same for the 16-byte unit holding columns [8u, 8u + 8) of row r
+__device__ __forceinline__ uint32_t sw_unit_off(int rows, int r, int u) {
+  return (uint32_t)((u >> 3) * rows * 128 + r * 128 + (((u & 7) ^ (r & 7)) << 4));
+}
+
+// Instruction descriptor, kind::f16 with fp32 accumulation: bf16 or fp16 A and
+// B, A / B K-major (0) or MN-major (1), M x N.
+__host__ __device__ constexpr uint32_t idesc(bool bf16, int a_mn, int b_mn, int m, int n) {
+  return (1u << 4) | (bf16 ? (1u << 7) | (1u << 10) : 0u) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+         ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
+template <typename T> struct Half2;
+template <> struct Half2<__half> {
+  using t2 = __half2;
+  static __device__ __forceinline__ t2 from(float a, float b) { return __floats2half2_rn(a, b); }
+  static __device__ __forceinline__ float2 to(t2 x) { return __half22float2(x); }
+};
+template <> struct Half2<__nv_bfloat16> {
+  using t2 = __nv_bfloat162;
+  static __device__ __forceinline__ t2 from(float a, float b) { return __floats2bfloat162_rn(a, b); }
+  static __device__ __forceinline__ float2 to(t2 x) { return __bfloat1622float2(x); }
+};
+
+// Eight values as a 16-byte unit of type T, and the remainders x - T(x) as a
+// second unit (the two-term split of an fp32 value).
+template <typename T>
+__device__ __forceinline__ void split8(const float (&x)[8], uint4& hi, uint4& lo) {
+  using H = Half2<T>;
+  typename H::t2 h[4], l[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    h[e] = H::from(x[2 * e], x[2 * e + 1]);
+    const float2 f = H::to(h[e]);
+    l[e] = H::from(x[2 * e] - f.x, x[2 * e + 1] - f.y);
+  }
+  memcpy(&hi, h, 16);
+  memcpy(&lo, l, 16);
+}
+template <typename T>
+__device__ __forceinline__ void widen8(const uint4& u, float (&x)[8]) {
+  using H = Half2<T>;
+  typename H::t2 h[4];
+  memcpy(h, &u, 16);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = H::to(h[e]);
+    x[2 * e] = f.x;
+    x[2 * e + 1] = f.y;
+  }
+}
+
+// 32 lanes x 32 bit, 32 consecutive columns (thread t of warp w <- lane 32 (w % 4) + t).
+__device__ __forceinline__ void tmem_ld32x32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Token row (b T + grid index) H + h of scan offset t of the chunk, or -1 past the sequence.
+__device__ __forceinline__ long long chunk_row(const Params& p, int b, int h, int d, int c, int t) {
+  const int s = c * kC + t;
+  if (s >= p.T) return -1;
+  return ((long long)b * p.T + scan_to_grid(d, s, p.T, p.gh, p.gw)) * p.H + h;
+}
+
+// 16-byte copy global -> shared that reads `bytes` (16 or 0) and zero-fills the rest.
+__device__ __forceinline__ void cp16(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr(dst)), "l"(src), "r"(bytes)
+               : "memory");
+}
+
+// Copies one chunk: thread tid takes token t = tid / 4 and a quarter qq = tid % 4
+// of its record -- four 16-byte units of each 16-bit tensor (into the
+// swizzled 64-row tiles) and eight of the fp32 gate row (plain row-major).
+template <typename T>
+__device__ __forceinline__ void gather(const Params& p, long long row, int t, int qq, uint8_t* Q, uint8_t* K,
+                                       uint8_t* V, float* G) {
+  const uint32_t ok = row >= 0 ? 16u : 0u;
+  const long long rr = row >= 0 ? row : 0;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int u = qq * 4 + e;
+    const uint32_t off = sw_unit_off(kC, t, u);
+    if (Q) cp16(Q + off, (const T*)p.q + rr * kD + u * 8, ok);
+    cp16(K + off, (const T*)p.k + rr * kD + u * 8, ok);
+    cp16(V + off, (const T*)p.v + rr * kD + u * 8, ok);
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const int u = qq * 8 + e;
+    cp16(G + t * kD + u * 4, p.g + rr * kD + u * 4, ok);
+  }
+}
+
+// In-place inclusive cumulative sum of the gate over the chunk's 64 tokens,
+// one key dim per thread (threads 0..127).
+__device__ __forceinline__ void cumsum(float* G, int tid) {
+  if (tid < kD) {
+    float s = 0.f;
+#pragma unroll 8
+    for (int t = 0; t < kC; ++t) {
+      s += G[t * kD + tid];
+      G[t * kD + tid] = s;
+    }
+  }
+}
+
+// Waits for an mbarrier phase, bounded; false on timeout.
+__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity) { return tc::mbar_wait(bar, parity); }
+
+// ---------------------------------------------------------------------------
+// Summary: dS^T = V^T k^ for one chunk, written as dS [dk][dv] fp32, and e^{Gam}.
+struct SumLayout {
+  static constexpr int kK = 0;                     // k tile, then k^ hi in place
+  static constexpr int kKlo = kK + kTile64;        // k^ lo
+  static constexpr int kV = kKlo + kTile64;        // v tile (the MN-major A operand V^T)
+  static constexpr int kG = kV + kTile64;          // gates, then cumulative
+  static constexpr int kMisc = kG + kGBytes;
+  static constexpr int kSmem = kMisc + 256 + 1024;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads, 2) gla_sum_tc128(const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* K = sm + SumLayout::kK;
+  uint8_t* Klo = sm + SumLayout::kKlo;
+  uint8_t* V = sm + SumLayout::kV;
+  float* G = reinterpret_cast<float*>(sm + SumLayout::kG);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + SumLayout::kMisc);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SumLayout::kMisc + 8);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / p.H, h = bh - b * p.H;
+  const int d = dir_of_batch(p.dir, b);
+  if (d < 0 || d > 3) {
+    if (tid == 0) gtr_flag(kStatusBadDir);
+    return;
+  }
+  if (tid == 0) {
+    tc::mbar_init(bar, 1);
+    tc::mbar_fence_init();
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(tmem_slot, 128);
+    tc::tmem_relinquish();
+  }
+  pdl_wait();                                      // the gates may come from the kernel before
+  pdl_trigger();
+  const int t = tid >> 2, qq = tid & 3;
+  gather<T>(p, chunk_row(p, b, h, d, c, t), t, qq, nullptr, K, V, G);
+  tc::cp_async_commit();
+  tc::cp_async_wait<0>();
+  __syncthreads();
+  cumsum(G, tid);
+  __syncthreads();
+  // k^ = k e^{Gam - G_t} in two terms of k's type: unit (t, u) per thread step
+  for (int it = tid; it < kC * 16; it += kThreads) {
+    const int r = it >> 4, u = it & 15;
+    const uint32_t off = sw_unit_off(kC, r, u);
+    float x[8];
+    widen8<T>(*reinterpret_cast<const uint4*>(K + off), x);
+    const float* gr = G + r * kD + u * 8;
+    const float* gl = G + (kC - 1) * kD + u * 8;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[e] *= __expf(gl[e] - gr[e]);
+    uint4 hi, lo;
+    split8<T>(x, hi, lo);
+    *reinterpret_cast<uint4*>(K + off) = hi;
+    *reinterpret_cast<uint4*>(Klo + off) = lo;
+  }
+  tc::fence_async_smem();
+  tc::tc_before_sync();
+  __syncthreads();
+  tc::tc_after_sync();
+  const uint32_t tm = *tmem_slot;
+  bool ok = true;
+  if (tid == 0) {
+    // D [dv][dk] = V^T (MN-major A, M = 128) x k^ (MN-major B, N = 128), K = 64 tokens
+    constexpr uint32_t id = idesc(std::is_same<T, __nv_bfloat16>::value, 1, 1, 128, 128);
+    const uint64_t a = tc::desc_mn(V), bh_ = tc::desc_mn(K), bl = tc::desc_mn(Klo);
+#pragma unroll
+    for (int ks = 0; ks < kC / 16; ++ks) tc::mma_f16(tm, a + ks * tc::kStepMN, bh_ + ks * tc::kStepMN, id, ks > 0);
+#pragma unroll
+    for (int ks = 0; ks < kC / 16; ++ks) tc::mma_f16(tm, a + ks * tc::kStepMN, bl + ks * tc::kStepMN, id, 1u);
+    tc::mma_commit(bar);
+  }
+  ok = wait_phase(bar, 0);
+  tc::tc_after_sync();
+  float* dS = p.wsS + ((size_t)bh * p.nc + c) * kD * kD;
+  if (warp < 4 && ok) {
+    // lane j of quadrant `warp` holds row j of dS^T, i.e. column j of dS
+    const int j = warp * 32 + lane;
+#pragma unroll 1
+    for (int c0 = 0; c0 < kD; c0 += 32) {
+      float v[32];
+      tmem_ld32x32(tm + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) dS[(size_t)(c0 + i) * kD + j] = v[i];
+    }
+  }
+  if (tid < kD) p.wsA[((size_t)bh * p.nc + c) * kD + tid] = __expf(G[(kC - 1) * kD + tid]);
+  if (!ok && lane == 0) gtr_flag(kStatusMbarTimeout);
+  tc::tc_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tm, 128);
+}
+
+// ---------------------------------------------------------------------------
+// Output of one chunk from the state it starts from.
+struct OutLayout {
+  static constexpr int kQ = 0;                     // q tile, then q~ hi in place
+  static constexpr int kQlo = kQ + kTile64;
+  static constexpr int kK = kQlo + kTile64;        // k tile, then k~ hi in place
+  static constexpr int kKlo = kK + kTile64;
+  static constexpr int kV = kKlo + kTile64;        // v (bf16: the one term; fp16: bf16 hi in place)
+  static constexpr int kVlo = kV + kTile64;        // fp16 v: bf16 lo
+  static constexpr int kG = kVlo + kTile64;        // gates, then cumulative
+  static constexpr int kS = kG + kGBytes;          // S [dk][dv] hi, lo: MN-major B, 128 rows
+  static constexpr int kP = kS + 2 * kTile128;     // P hi, lo: K-major A, 64 x 64
+  static constexpr int kMisc = kP + 2 * kHalf64;
+  static constexpr int kSmem = kMisc + 1024 + 1024;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads, 1) gla_out_tc128(const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* Q = sm + OutLayout::kQ;
+  uint8_t* Qlo = sm + OutLayout::kQlo;
+  uint8_t* K = sm + OutLayout::kK;
+  uint8_t* Klo = sm + OutLayout::kKlo;
+  uint8_t* V = sm + OutLayout::kV;
+  uint8_t* Vlo = sm + OutLayout::kVlo;
+  float* G = reinterpret_cast<float*>(sm + OutLayout::kG);
+  uint8_t* S = sm + OutLayout::kS;
+  uint8_t* P = sm + OutLayout::kP;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OutLayout::kMisc);            // two phases
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OutLayout::kMisc + 16);
+  float* rowss = reinterpret_cast<float*>(sm + OutLayout::kMisc + 64);           // [2][64] partial sums
+  constexpr bool kBF = std::is_same<T, __nv_bfloat16>::value;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / p.H, h = bh - b * p.H;
+  const int d = dir_of_batch(p.dir, b);
+  if (d < 0 || d > 3) {
+    if (tid == 0) gtr_flag(kStatusBadDir);
+    return;
+  }
+  if (tid == 0) {
+    tc::mbar_init(bar, 1);
+    tc::mbar_fence_init();
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(tmem_slot, 256);
+    tc::tmem_relinquish();
+  }
+  // q, k, v, g and z were complete before the summary stage ran; the
+  // boundary states need the scan, so wait before anything else reads
+  pdl_wait();
+  pdl_trigger();
+  const int t = tid >> 2, qq = tid & 3;
+  const long long my_row = chunk_row(p, b, h, d, c, t);
+  gather<T>(p, my_row, t, qq, Q, K, V, G);
+  tc::cp_async_commit();
+  // S [dk][dv] -> two bf16 terms in the MN-major B layout (rows = dk = K)
+  const float* Sg = p.wsS + ((size_t)bh * p.nc + c) * kD * kD;
+  for (int it = tid; it < kD * 16; it += kThreads) {
+    const int i = it >> 4, u = it & 15;
+    const float4 a = *reinterpret_cast<const float4*>(Sg + (size_t)i * kD + u * 8);
+    const float4 e = *reinterpret_cast<const float4*>(Sg + (size_t)i * kD + u * 8 + 4);
+    const float x[8] = {a.x, a.y, a.z, a.w, e.x, e.y, e.z, e.w};
+    uint4 hi, lo;
+    split8<__nv_bfloat16>(x, hi, lo);
+    const uint32_t off = sw_unit_off(kD, i, u);
+    *reinterpret_cast<uint4*>(S + off) = hi;
+    *reinterpret_cast<uint4*>(S + kTile128 + off) = lo;
+  }
+  tc::cp_async_wait<0>();
+  __syncthreads();
+  cumsum(G, tid);
+  __syncthreads();
+  // a chunk whose log-gate span leaves [-kSpan, 0] takes exact scores
+  const bool exact = __syncthreads_or(tid < kD && G[(kC - 1) * kD + tid] < -kSpan) != 0;
+  // q~ = q e^{G}, k~ = k e^{-G} (not for an exact chunk), v split for fp16, all in place
+  for (int it = tid; it < kC * 16; it += kThreads) {
+    const int r = it >> 4, u = it & 15;
+    const uint32_t off = sw_unit_off(kC, r, u);
+    const float* gr = G + r * kD + u * 8;
+    float x[8];
+    uint4 hi, lo;
+    widen8<T>(*reinterpret_cast<const uint4*>(Q + off), x);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[e] *= __expf(gr[e]);
+    split8<__nv_bfloat16>(x, hi, lo);
+    *reinterpret_cast<uint4*>(Q + off) = hi;
+    *reinterpret_cast<uint4*>(Qlo + off) = lo;
+    if (!exact) {
+      widen8<T>(*reinterpret_cast<const uint4*>(K + off), x);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[e] *= __expf(-gr[e]);
+      split8<__nv_bfloat16>(x, hi, lo);
+      *reinterpret_cast<uint4*>(K + off) = hi;
+      *reinterpret_cast<uint4*>(Klo + off) = lo;
+    }
+    if (!kBF) {
+      widen8<T>(*reinterpret_cast<const uint4*>(V + off), x);
+      split8<__nv_bfloat16>(x, hi, lo);        // exact: an fp16 value is bf16 hi + bf16 lo
+      *reinterpret_cast<uint4*>(V + off) = hi;
+      *reinterpret_cast<uint4*>(Vlo + off) = lo;
+    }
+  }
+  tc::fence_async_smem();
+  tc::tc_before_sync();
+  __syncthreads();
+  tc::tc_after_sync();
+  const uint32_t tm = *tmem_slot;
+  const uint32_t tmO = tm, tmP = tm + 128;         // o: columns [0, 128); scores: [128, 192)
+  constexpr uint32_t kIdScores = idesc(true, 0, 0, 64, 64);    // q~ (K-major) x k~ (K-major)
+  constexpr uint32_t kIdQS = idesc(true, 0, 1, 64, 128);       // q~ (K-major) x S (MN-major)
+  constexpr uint32_t kIdPV = idesc(true, 0, 1, 64, 128);       // P (K-major) x V (MN-major)
+  if (tid == 0) {
+    const uint64_t qh = tc::desc_k(Q), ql = tc::desc_k(Qlo);
+    const uint64_t sh = tc::sdesc(saddr(S), kHalf128, 1024), sl = tc::sdesc(saddr(S + kTile128), kHalf128, 1024);
+    // o = q~ S: K = 128 key dims, two 64-column halves of the q~ tiles
+#pragma unroll
+    for (int ks = 0; ks < kD / 16; ++ks) {
+      const uint64_t ao = (uint64_t)((ks >> 2) * (kHalf64 >> 4) + (ks & 3) * tc::kStepK);
+      const uint64_t bo = (uint64_t)(ks * tc::kStepMN);
+      tc::mma_f16(tmO, qh + ao, sh + bo, kIdQS, ks > 0);
+      tc::mma_f16(tmO, qh + ao, sl + bo, kIdQS, 1u);
+      tc::mma_f16(tmO, ql + ao, sh + bo, kIdQS, 1u);
+    }
+    if (!exact) {
+      const uint64_t kh = tc::desc_k(K), kl = tc::desc_k(Klo);
+#pragma unroll
+      for (int ks = 0; ks < kD / 16; ++ks) {
+        const uint64_t o = (uint64_t)((ks >> 2) * (kHalf64 >> 4) + (ks & 3) * tc::kStepK);
+        tc::mma_f16(tmP, qh + o, kh + o, kIdScores, ks > 0);
+        tc::mma_f16(tmP, qh + o, kl + o, kIdScores, 1u);
+        tc::mma_f16(tmP, ql + o, kh + o, kIdScores, 1u);
+      }
+    }
+    tc::mma_commit(bar);
+  }
+  bool ok = wait_phase(bar, 0);
+  tc::tc_after_sync();
+  // P: thread (quadrant qd = warp % 4, half hf = warp / 4) holds row r = 16 qd + lane % 16,
+  // columns s0 .. s0 + 15 with s0 = 32 hf + 16 (lane / 16)
+  const int qd = warp & 3, hf = warp >> 2;
+  const int r = qd * 16 + (lane & 15);
+  const int s0 = hf * 32 + (lane >> 4) * 16;
+  const int ntok = min(kC, p.T - c * kC);
+  {
+    float sc[16];
+    if (!exact) {
+      float tv[16];
+      tc::tmem_ld16x2(tmP + ((uint32_t)(qd * 32) << 16) + (uint32_t)(hf * 32), tv);
+      tc::tmem_ld_wait(tv);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) sc[e] = tv[e];
+    } else {
+      // exact scores from the 16-bit q, k rows: sum_i q_r[i] k_s[i] e^{G_r[i] - G_s[i]}
+      const long long rq = chunk_row(p, b, h, d, c, r);
+#pragma unroll 1
+      for (int e = 0; e < 16; ++e) {
+        const int s = s0 + e;
+        float acc = 0.f;
+        if (s <= r && r < ntok) {
+          const long long rk = chunk_row(p, b, h, d, c, s);
+          const T* qr = (const T*)p.q + rq * kD;
+          const T* kr = (const T*)p.k + rk * kD;
+          for (int i = 0; i < kD; ++i)
+            acc = fmaf(ld_f(qr + i) * ld_f(kr + i), __expf(G[r * kD + i] - G[s * kD + i]), acc);
+        }
+        sc[e] = acc;
+      }
+      if (tid == 0) atomicAdd(&g_gtr_exact_chunks, 1ull);
+    }
+    // causal mask (s <= r), two bf16 terms into the K-major P tiles
+#pragma unroll
+    for (int hb = 0; hb < 2; ++hb) {
+      float x[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[e] = (s0 + hb * 8 + e <= r) ? sc[hb * 8 + e] : 0.f;
+      uint4 hi, lo;
+      split8<__nv_bfloat16>(x, hi, lo);
+      const uint32_t off = (uint32_t)(r * 128 + ((((s0 >> 3) + hb) ^ (r & 7)) << 4));
+      *reinterpret_cast<uint4*>(P + off) = hi;
+      *reinterpret_cast<uint4*>(P + kHalf64 + off) = lo;
+    }
+  }
+  tc::fence_async_smem();
+  tc::tc_before_sync();
+  __syncthreads();
+  tc::tc_after_sync();
+  if (tid == 0) {
+    // o += P V: K = 64 tokens
+    const uint64_t ph = tc::desc_k(P), pl = tc::desc_k(P + kHalf64);
+    const uint64_t vh = tc::desc_mn(V), vl = tc::desc_mn(Vlo);
+#pragma unroll
+    for (int ks = 0; ks < kC / 16; ++ks) {
+      const uint64_t ao = (uint64_t)(ks * tc::kStepK), bo = (uint64_t)(ks * tc::kStepMN);
+      tc::mma_f16(tmO, ph + ao, vh + bo, kIdPV, 1u);
+      tc::mma_f16(tmO, pl + ao, vh + bo, kIdPV, 1u);
+      if (!kBF) tc::mma_f16(tmO, ph + ao, vl + bo, kIdPV, 1u);
+    }
+    tc::mma_commit(bar);
+  }
+  ok = wait_phase(bar, 1) && ok;
+  tc::tc_after_sync();
+  // epilogue: row r, columns 64 hf + [16 (lane / 16), + 16) and 64 hf + 32 + [16 (lane / 16), + 16)
+  float o[32];
+  {
+    float a[16], e2[16];
+    const uint32_t base = tmO + ((uint32_t)(qd * 32) << 16) + (uint32_t)(hf * 64);
+    tc::tmem_ld16x2(base, a);
+    tc::tmem_ld_wait(a);
+    tc::tmem_ld16x2(base + 32, e2);
+    tc::tmem_ld_wait(e2);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      o[e] = a[e];
+      o[16 + e] = e2[e];
+    }
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int e = 0; e < 32; ++e) ss = fmaf(o[e], o[e], ss);
+  ss += __shfl_xor_sync(0xffffffffu, ss, 16);
+  if ((lane >> 4) == 0) rowss[hf * kC + r] = ss;
+  __syncthreads();
+  const float tot = rowss[r] + rowss[kC + r];
+  const float inv = rsqrtf(tot / (float)kD + kRmsEps);
+  if (r < ntok && ok) {
+    const long long orow = chunk_row(p, b, h, d, c, r);
+    const T* zr = (const T*)p.z + orow * kD;
+    T* outr = (T*)p.out + orow * kD;
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {
+      const int j0 = hf * 64 + part * 32 + (lane >> 4) * 16;
+      float zf[16];
+      widen8<T>(*reinterpret_cast<const uint4*>(zr + j0), *reinterpret_cast<float(*)[8]>(zf));
+      widen8<T>(*reinterpret_cast<const uint4*>(zr + j0 + 8), *reinterpret_cast<float(*)[8]>(zf + 8));
+      float y[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float wj = p.w ? __ldg(p.w + j0 + e) : 1.0f;
+        y[e] = o[part * 16 + e] * inv * wj * tc::silu_fast(zf[e]);
+      }
+      uint4 u0, u1, l0, l1;
+      // the output is one rounding of y to T (the lo terms are discarded)
+      split8<T>(*reinterpret_cast<float(*)[8]>(y), u0, l0);
+      split8<T>(*reinterpret_cast<float(*)[8]>(y + 8), u1, l1);
+      *reinterpret_cast<uint4*>(outr + j0) = u0;
+      *reinterpret_cast<uint4*>(outr + j0 + 8) = u1;
+    }
+  }
+  if (!ok && lane == 0) gtr_flag(kStatusMbarTimeout);
+  tc::tc_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tm, 256);
+}
+
+}  // namespace tc128
+
+inline bool tc128_shape_supported(int dk, int dv, int chunk, int dtype) {
+  return dk == tc128::kD && dv == tc128::kD && chunk == tc128::kC && (dtype == kF16 || dtype == kBF16);
+}
+
+// stage 0: summaries of every chunk; stage 1: outputs of every chunk.
+inline int launch_tc128(int dtype, int stage, const tc128::Params& p, int BH, cudaStream_t st, int dev) {
+  static bool done[4][64];
+  const dim3 grid((unsigned)p.nc, (unsigned)BH);
+  auto go = [&](auto kern, int smem, bool* flag) -> int {
+    if (!flag[dev]) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return -5;
+      flag[dev] = true;
+    }
+    return launch_pdl(kern, grid, dim3(tc128::kThreads), (size_t)smem, st, p);
+  };
+  if (stage == 0)
+    return dtype == kF16 ? go(tc128::gla_sum_tc128<__half>, tc128::SumLayout::kSmem, done[0])
+                         : go(tc128::gla_sum_tc128<__nv_bfloat16>, tc128::SumLayout::kSmem, done[1]);
+  return dtype == kF16 ? go(tc128::gla_out_tc128<__half>, tc128::OutLayout::kSmem, done[2])
+                       : go(tc128::gla_out_tc128<__nv_bfloat16>, tc128::OutLayout::kSmem, done[3]);
+}
+
+}  // namespace gtr
