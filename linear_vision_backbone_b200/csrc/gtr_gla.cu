@@ -478,7 +478,15 @@ int launch_stage(const Plan& p, const void* q, const void* k, const void* v, con
 int launch_scan(const Plan& p, float* wsS, const float* wsA, int inclusive, cudaStream_t st) {
   const long long total = (long long)p.B * p.H * p.dk * p.dv;
   const long long blocks = (total + 31) / 32;   // 32 elements per block
-  return launch_pdl(gla_state_scan, dim3((unsigned)blocks), dim3(kScanThreads), 0, st, wsS,
+  // sixteen ranges per block only for very long scans: the wider blocks keep
+  // fewer elements in flight (measured slower at 64 and 256 segments, faster
+  // at 1024)
+  if (p.nseg >= 512)
+    return launch_pdl(gla_state_scan<kScanPartsWide>, dim3((unsigned)blocks), dim3(32 * kScanPartsWide), 0, st,
+                      wsS, (const float*)wsA, total, p.nseg, p.dk, p.dv, inclusive) == 0
+               ? GTR_OK
+               : GTR_ERR_CUDA;
+  return launch_pdl(gla_state_scan<kScanParts>, dim3((unsigned)blocks), dim3(kScanThreads), 0, st, wsS,
                     (const float*)wsA, total, p.nseg, p.dk, p.dv, inclusive) == 0
              ? GTR_OK
              : GTR_ERR_CUDA;

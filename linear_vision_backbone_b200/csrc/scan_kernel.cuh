@@ -23,7 +23,8 @@
 
 namespace gtr {
 
-constexpr int kScanParts = 4;
+constexpr int kScanParts = 4;             // ranges per block
+constexpr int kScanPartsWide = 16;        // ranges per block for very long scans
 constexpr int kScanThreads = 32 * kScanParts;
 constexpr int kScanReg = 12;
 
@@ -41,11 +42,15 @@ __device__ __forceinline__ void scan_window(const float* pd, const float* pa, in
   }
 }
 
-// at most 64 registers: eight blocks per SM, so a 16k-token, 6-head problem
-// (768 blocks) is resident in one wave
-__global__ void __launch_bounds__(kScanThreads, 8)
+// at most 64 registers: eight blocks of four ranges per SM, so a 16k-token,
+// 6-head problem (768 blocks) is resident in one wave; sixteen ranges per
+// block (two blocks per SM) when the segments are many, so that each range
+// stays short
+template <int kParts>
+__global__ void __launch_bounds__(32 * kParts, 32 / kParts)
 gla_state_scan(float* __restrict__ wsS, const float* __restrict__ wsA, long long total, int nseg,
                int dk, int dv, int inclusive) {
+  constexpr int kScanParts = kParts;
   __shared__ float mapP[kScanParts][32], mapR[kScanParts][32];
   pdl_wait();                             // the summaries are complete
   pdl_trigger();

@@ -165,17 +165,24 @@ __device__ __forceinline__ void gather(const Params& p, long long row, int t, in
   }
 }
 
-// In-place inclusive cumulative sum of the gate over the chunk's 64 tokens,
-// one key dim per thread (threads 0..127).
+// In-place inclusive cumulative sum of the gate over the chunk's 64 tokens:
+// thread tid sums key dim tid % 128 over tokens [32 (tid / 128), + 32); the
+// second half then adds the first half's total.  Ends with a block barrier.
 __device__ __forceinline__ void cumsum(float* G, int tid) {
-  if (tid < kD) {
-    float s = 0.f;
+  const int i = tid & (kD - 1), t0 = (tid >> 7) * (kC / 2);
+  float s = 0.f;
 #pragma unroll 8
-    for (int t = 0; t < kC; ++t) {
-      s += G[t * kD + tid];
-      G[t * kD + tid] = s;
-    }
+  for (int t = t0; t < t0 + kC / 2; ++t) {
+    s += G[t * kD + i];
+    G[t * kD + i] = s;
   }
+  __syncthreads();
+  if (t0 > 0) {
+    const float base = G[(t0 - 1) * kD + i];
+#pragma unroll 8
+    for (int t = t0; t < t0 + kC / 2; ++t) G[t * kD + i] += base;
+  }
+  __syncthreads();
 }
 
 // Waits for an mbarrier phase, bounded; false on timeout.
@@ -226,7 +233,6 @@ __global__ void __launch_bounds__(kThreads, 2) gla_sum_tc128(const Params p) {
   tc::cp_async_wait<0>();
   __syncthreads();
   cumsum(G, tid);
-  __syncthreads();
   // k^ = k e^{Gam - G_t} in two terms of k's type: unit (t, u) per thread step
   for (int it = tid; it < kC * 16; it += kThreads) {
     const int r = it >> 4, u = it & 15;
@@ -336,23 +342,32 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc128(const Params p) {
   const long long my_row = chunk_row(p, b, h, d, c, t);
   gather<T>(p, my_row, t, qq, Q, K, V, G);
   tc::cp_async_commit();
-  // S [dk][dv] -> two bf16 terms in the MN-major B layout (rows = dk = K)
-  const float* Sg = p.wsS + ((size_t)bh * p.nc + c) * kD * kD;
-  for (int it = tid; it < kD * 16; it += kThreads) {
-    const int i = it >> 4, u = it & 15;
-    const float4 a = *reinterpret_cast<const float4*>(Sg + (size_t)i * kD + u * 8);
-    const float4 e = *reinterpret_cast<const float4*>(Sg + (size_t)i * kD + u * 8 + 4);
-    const float x[8] = {a.x, a.y, a.z, a.w, e.x, e.y, e.z, e.w};
-    uint4 hi, lo;
-    split8<__nv_bfloat16>(x, hi, lo);
-    const uint32_t off = sw_unit_off(kD, i, u);
-    *reinterpret_cast<uint4*>(S + off) = hi;
-    *reinterpret_cast<uint4*>(S + kTile128 + off) = lo;
+  // S [dk][dv] -> two bf16 terms in the MN-major B layout (rows = dk = K);
+  // all eight units' loads are issued before the first is converted
+  {
+    const float* Sg = p.wsS + ((size_t)bh * p.nc + c) * kD * kD;
+    constexpr int kUnits = kD * 16 / kThreads;
+    float4 sa[kUnits], sb[kUnits];
+#pragma unroll
+    for (int n = 0; n < kUnits; ++n) {
+      const int it = tid + n * kThreads, i = it >> 4, u = it & 15;
+      sa[n] = *reinterpret_cast<const float4*>(Sg + (size_t)i * kD + u * 8);
+      sb[n] = *reinterpret_cast<const float4*>(Sg + (size_t)i * kD + u * 8 + 4);
+    }
+#pragma unroll
+    for (int n = 0; n < kUnits; ++n) {
+      const int it = tid + n * kThreads, i = it >> 4, u = it & 15;
+      const float x[8] = {sa[n].x, sa[n].y, sa[n].z, sa[n].w, sb[n].x, sb[n].y, sb[n].z, sb[n].w};
+      uint4 hi, lo;
+      split8<__nv_bfloat16>(x, hi, lo);
+      const uint32_t off = sw_unit_off(kD, i, u);
+      *reinterpret_cast<uint4*>(S + off) = hi;
+      *reinterpret_cast<uint4*>(S + kTile128 + off) = lo;
+    }
   }
   tc::cp_async_wait<0>();
   __syncthreads();
   cumsum(G, tid);
-  __syncthreads();
   // a chunk whose log-gate span leaves [-kSpan, 0] takes exact scores
   const bool exact = __syncthreads_or(tid < kD && G[(kC - 1) * kD + tid] < -kSpan) != 0;
   // q~ = q e^{G}, k~ = k e^{-G} (not for an exact chunk), v split for fp16, all in place
