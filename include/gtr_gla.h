@@ -80,7 +80,7 @@ typedef enum { GTR_LR = 0, GTR_RL = 1, GTR_TB = 2, GTR_BT = 3, GTR_ROTATE_BATCH 
 typedef enum {
     GTR_PATH_AUTO = 0,  /* tensor-core path where supported, else SIMT */
     GTR_PATH_SIMT = 1,  /* exact fp32 CUDA-core path, every dtype and head dim */
-    GTR_PATH_TC = 2     /* tcgen05/TMEM path: 16-bit dtypes, dk = dv = 64 */
+    GTR_PATH_TC = 2     /* tcgen05/TMEM path: 16-bit dtypes, chunk 64, dk = dv = 64 or 128 */
 } gtr_path_t;
 
 #define GTR_ABI_VERSION 1
@@ -146,6 +146,10 @@ GTR_API gtr_status_t gtr_gate_fwd_packed(const void *x, int x_dtype, const void 
  *   dk, dv in {16, 32, 64, 128}; chunk (the chunk length C) in {16, 32, 64,
  *   128}; the result does not depend on C beyond rounding.  T = grid_h*grid_w
  *   must fit in an int.  `out` must not alias any input.
+ *   Kernels: tcgen05 tensor-core kernels for 16-bit dtypes with chunk 64 and
+ *   dk = dv = 64 (segments of chunks walked with the state on chip) or
+ *   dk = dv = 128 (every chunk its own block, 64 KB of fp32 state per chunk
+ *   in the workspace); the exact fp32 CUDA-core kernels otherwise.
  *   Workspace: fp32 segment states taken from a library-owned buffer cached
  *   per (device, stream) and grown on demand with cudaMalloc (so the first call
  *   for a shape must not happen during stream capture), or from the buffer
@@ -213,8 +217,8 @@ GTR_API gtr_status_t gtr_gla_fwd_timed(const void *q, const void *k, const void 
  *   bias [H*dk] fp32 or NULL; tau > 0.  q, k, v, outgate, rms_w, out, the sizes,
  *   dir, chunk and dtype as in gtr_gla_fwd; g_out [B, T, H, dk] fp32 receives g
  *   (the output stage reads it back; it must not alias another argument).
- *   Where gtr_gla_fwd takes its tensor-core path (dk = dv = 64, chunk 64, 16-bit
- *   dtype) the gate is split at its rank-16 bottleneck: one kernel writes
+ *   Where gtr_gla_fwd takes its tensor-core path with dk = dv = 64 (chunk 64,
+ *   16-bit dtype) the gate is split at its rank-16 bottleneck: one kernel writes
  *   x W_down ([B*T, 16] fp32, 64 bytes per token, in the workspace, which
  *   therefore grows by B*T*64 bytes), and the summary kernel forms g chunk by
  *   chunk from it, so the gate costs no pass of its own over g.  g_out and
