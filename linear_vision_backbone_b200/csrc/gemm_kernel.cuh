@@ -32,7 +32,6 @@ constexpr int kATile = kBM * kBK * 2;            // 16 KB
 constexpr int kBox = 32 * 64 * 2;                // one warp's 32 rows x 64 columns output box: 4 KB
 constexpr int kEpiBoxes = 2;                     // per epilogue warp (a ring of two)
 constexpr int kThreads = 6 * 32;
-constexpr int kWarpEpi0 = 2;
 constexpr int kMaxOut = 4;
 
 template <int kBN>

@@ -477,19 +477,21 @@ int launch_stage(const Plan& p, const void* q, const void* k, const void* v, con
 
 int launch_scan(const Plan& p, float* wsS, const float* wsA, int inclusive, cudaStream_t st) {
   const long long total = (long long)p.B * p.H * p.dk * p.dv;
-  const long long blocks = (total + 31) / 32;   // 32 elements per block
-  // sixteen ranges per block only for very long scans: the wider blocks keep
-  // fewer elements in flight (measured slower at 64 and 256 segments, faster
-  // at 1024)
-  if (p.nseg >= 512)
-    return launch_pdl(gla_state_scan<kScanPartsWide>, dim3((unsigned)blocks), dim3(32 * kScanPartsWide), 0, st,
-                      wsS, (const float*)wsA, total, p.nseg, p.dk, p.dv, inclusive) == 0
+  const long long groups = (total + 31) / 32;   // 32 elements per group
+  auto go = [&](auto kern, int parts, int gpb) {
+    const long long blocks = (groups + gpb - 1) / gpb;
+    return launch_pdl(kern, dim3((unsigned)blocks), dim3(32 * parts * gpb), 0, st, wsS, wsA, total, p.nseg,
+                      p.dk, p.dv, inclusive) == 0
                ? GTR_OK
                : GTR_ERR_CUDA;
-  return launch_pdl(gla_state_scan<kScanParts>, dim3((unsigned)blocks), dim3(kScanThreads), 0, st, wsS,
-                    (const float*)wsA, total, p.nseg, p.dk, p.dv, inclusive) == 0
-             ? GTR_OK
-             : GTR_ERR_CUDA;
+  };
+  // segments that fit one register window: one warp per group, four groups
+  // per block; sixteen ranges per group only for very long scans (the wider
+  // blocks keep fewer elements in flight: measured slower at 64 and 256
+  // segments, faster at 1024)
+  if (p.nseg <= kScanReg) return go(gla_state_scan<1, 4>, 1, 4);
+  if (p.nseg >= 512) return go(gla_state_scan<kScanPartsWide, 1>, kScanPartsWide, 1);
+  return go(gla_state_scan<kScanParts, 1>, kScanParts, 1);
 }
 
 // Record a caller event; inside stream capture it becomes an external event

@@ -10,10 +10,9 @@
 // dS in place (exclusive form: the state each segment starts from) or, with
 // `inclusive`, the state each segment ends with.
 //
-// A block takes 32 consecutive elements (one coalesced 128-byte line per
-// segment) and splits their segments into kScanParts consecutive ranges, one
-// per warp.  Each warp first reduces its range to one affine map
-// S -> P S + R (P the product of the range's A, R its scan from zero), the
+// A group of 32 consecutive elements (one coalesced 128-byte line per
+// segment) has its segments split into consecutive ranges, one per warp.
+// Each warp first reduces its range to one affine map S -> P S + R (P the product of the range's A, R its scan from zero), the
 // warps exchange the maps through shared memory, and each range then replays
 // its recurrence from the state composed of the maps before it.  A range of
 // up to kScanReg segments stays in registers between the two passes, so the
@@ -23,9 +22,8 @@
 
 namespace gtr {
 
-constexpr int kScanParts = 4;             // ranges per block
-constexpr int kScanPartsWide = 16;        // ranges per block for very long scans
-constexpr int kScanThreads = 32 * kScanParts;
+constexpr int kScanParts = 4;             // ranges per group
+constexpr int kScanPartsWide = 16;        // ranges per group for very long scans
 constexpr int kScanReg = 12;
 
 // Pass 1 / pass 2 over `n` segments held in registers (n <= kScanReg); the
@@ -42,25 +40,30 @@ __device__ __forceinline__ void scan_window(const float* pd, const float* pa, in
   }
 }
 
-// at most 64 registers: eight blocks of four ranges per SM, so a 16k-token,
-// 6-head problem (768 blocks) is resident in one wave; sixteen ranges per
-// block (two blocks per SM) when the segments are many, so that each range
-// stays short
-template <int kParts>
-__global__ void __launch_bounds__(32 * kParts, 32 / kParts)
+// at most 64 registers, 1024 threads per SM.  A block holds kGroups groups of
+// 32 elements, each group's segments split into kParts ranges (one warp
+// each): four ranges of one group per block, so a 16k-token, 6-head problem
+// (768 blocks) is resident in one wave; sixteen ranges per group when the
+// segments are many, so that each range stays short; one range for each of
+// four groups when the segments fit one register window, so that problems of
+// many short sequences need a quarter of the blocks
+template <int kParts, int kGroups>
+__global__ void __launch_bounds__(32 * kParts * kGroups, 32 / (kParts * kGroups))
 gla_state_scan(float* __restrict__ wsS, const float* __restrict__ wsA, long long total, int nseg,
                int dk, int dv, int inclusive) {
   constexpr int kScanParts = kParts;
-  __shared__ float mapP[kScanParts][32], mapR[kScanParts][32];
+  __shared__ float mapP[kGroups][kScanParts][32], mapR[kGroups][kScanParts][32];
   pdl_wait();                             // the summaries are complete
   pdl_trigger();
-  const int lane = threadIdx.x & 31, part = threadIdx.x >> 5;
-  // 32 elements per block; dk * dv is a multiple of 32, so a block stays in one (b, h)
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int grp = warp / kScanParts, part = warp - grp * kScanParts;
+  // 32 elements per group; dk * dv is a multiple of 32, so a group stays in one (b, h)
   const int dkdv = dk * dv;
   const int per_bh = dkdv >> 5;
-  const long long bh = blockIdx.x / per_bh;
-  const int rem = (int)(blockIdx.x - bh * per_bh) * 32 + lane;
-  const bool live = (long long)blockIdx.x * 32 + lane < total;
+  const long long gi = (long long)blockIdx.x * kGroups + grp;
+  const long long bh = gi / per_bh;
+  const int rem = (int)(gi - bh * per_bh) * 32 + lane;
+  const bool live = gi * 32 + lane < total;
   const int i = rem / dv;
   const int len = (nseg + kScanParts - 1) / kScanParts;
   const int sa = min(nseg, part * len), sb = min(nseg, sa + len);
@@ -86,13 +89,13 @@ gla_state_scan(float* __restrict__ wsS, const float* __restrict__ wsA, long long
       }
     }
   }
-  mapP[part][lane] = P;
-  mapR[part][lane] = R;
+  mapP[grp][part][lane] = P;
+  mapR[grp][part][lane] = R;
   __syncthreads();
   if (!live) return;
   // the state entering this range
   float S = 0.f;
-  for (int r = 0; r < part; ++r) S = fmaf(mapP[r][lane], S, mapR[r][lane]);
+  for (int r = 0; r < part; ++r) S = fmaf(mapP[grp][r][lane], S, mapR[grp][r][lane]);
 
   // pass 2: the states, from registers when the range is one window
   for (int s0 = 0; s0 < n; s0 += kScanReg) {
