@@ -286,42 +286,63 @@ __global__ void __launch_bounds__(kThreads, 2) gla_sum_tc128(const Params p) {
 }
 
 // ---------------------------------------------------------------------------
-// Output of one chunk from the state it starts from.
+// Output of one chunk from the state it starts from, computed transposed so
+// that the state is an operand in tensor memory rather than shared memory:
+//   o^T = S^T q~^T + V^T P^T      (M = 128 value dims, N = 64 tokens)
+// with S^T [dv][dk] written to tensor memory as two bf16 terms (the A
+// operand), q~ and P read from shared memory as K-major B operands and V as
+// the MN-major A operand.  The scores q~ k~^T (M = 64) are as before.  With
+// bf16 inputs a block takes 112 KB of shared memory, so two blocks share an
+// SM; P is written over the key tiles once the scores are read.
+template <typename T>
 struct OutLayout {
-  static constexpr int kQ = 0;                     // q tile, then q~ hi in place
+  static constexpr bool kTwoV = !std::is_same<T, __nv_bfloat16>::value;   // fp16 v: bf16 hi + lo
+  static constexpr int kQ = 0;                     // q tile, then q~ hi; later the row sums
   static constexpr int kQlo = kQ + kTile64;
-  static constexpr int kK = kQlo + kTile64;        // k tile, then k~ hi in place
+  static constexpr int kK = kQlo + kTile64;        // k tile, then k~ hi; then P hi, P lo
   static constexpr int kKlo = kK + kTile64;
-  static constexpr int kV = kKlo + kTile64;        // v (bf16: the one term; fp16: bf16 hi in place)
-  static constexpr int kVlo = kV + kTile64;        // fp16 v: bf16 lo
-  static constexpr int kG = kVlo + kTile64;        // gates, then cumulative
-  static constexpr int kS = kG + kGBytes;          // S [dk][dv] hi, lo: MN-major B, 128 rows
-  static constexpr int kP = kS + 2 * kTile128;     // P hi, lo: K-major A, 64 x 64
-  static constexpr int kMisc = kP + 2 * kHalf64;
-  static constexpr int kSmem = kMisc + 1024 + 1024;
+  static constexpr int kV = kKlo + kTile64;
+  static constexpr int kVlo = kV + kTile64;        // fp16 v only
+  static constexpr int kG = kVlo + (kTwoV ? kTile64 : 0);
+  static constexpr int kMisc = kG + kGBytes;
+  static constexpr int kSmem = kMisc + 128;
+  static constexpr int kBlocksPerSM = kTwoV ? 1 : 2;
 };
 
+// 32 lanes x 32 bit, `N` consecutive columns from registers (thread t of warp w -> lane 32 (w % 4) + t).
+__device__ __forceinline__ void tmem_st32x16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
 template <typename T>
-__global__ void __launch_bounds__(kThreads, 1) gla_out_tc128(const Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* Q = sm + OutLayout::kQ;
-  uint8_t* Qlo = sm + OutLayout::kQlo;
-  uint8_t* K = sm + OutLayout::kK;
-  uint8_t* Klo = sm + OutLayout::kKlo;
-  uint8_t* V = sm + OutLayout::kV;
-  uint8_t* Vlo = sm + OutLayout::kVlo;
-  float* G = reinterpret_cast<float*>(sm + OutLayout::kG);
-  uint8_t* S = sm + OutLayout::kS;
-  uint8_t* P = sm + OutLayout::kP;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OutLayout::kMisc);            // two phases
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OutLayout::kMisc + 16);
-  float* rowss = reinterpret_cast<float*>(sm + OutLayout::kMisc + 64);           // [2][64] partial sums
-  constexpr bool kBF = std::is_same<T, __nv_bfloat16>::value;
+__global__ void __launch_bounds__(kThreads, OutLayout<T>::kBlocksPerSM) gla_out_tc128(const Params p) {
+  using L = OutLayout<T>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = smem_raw;
+  uint8_t* Q = sm + L::kQ;
+  uint8_t* Qlo = sm + L::kQlo;
+  uint8_t* K = sm + L::kK;
+  uint8_t* Klo = sm + L::kKlo;
+  uint8_t* V = sm + L::kV;
+  uint8_t* Vlo = sm + L::kVlo;
+  float* G = reinterpret_cast<float*>(sm + L::kG);
+  uint8_t* P = K;                                  // after the scores: P hi, then P lo 8 KB on
+  float* rowss = reinterpret_cast<float*>(Q);      // after the first products: [4][64] partial sums
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::kMisc);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kMisc + 16);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x, bh = blockIdx.y;
   const int b = bh / p.H, h = bh - b * p.H;
   const int d = dir_of_batch(p.dir, b);
+  if ((saddr(smem_raw) & 1023u) != 0u) {           // the swizzled tiles need 1024-byte alignment
+    if (tid == 0) gtr_flag(kStatusBadShape);
+    return;
+  }
   if (d < 0 || d > 3) {
     if (tid == 0) gtr_flag(kStatusBadDir);
     return;
@@ -334,36 +355,42 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc128(const Params p) {
     tc::tmem_alloc(tmem_slot, 256);
     tc::tmem_relinquish();
   }
-  // q, k, v, g and z were complete before the summary stage ran; the
-  // boundary states need the scan, so wait before anything else reads
-  pdl_wait();
+  pdl_wait();                                      // the boundary states come from the scan
   pdl_trigger();
   const int t = tid >> 2, qq = tid & 3;
-  const long long my_row = chunk_row(p, b, h, d, c, t);
-  gather<T>(p, my_row, t, qq, Q, K, V, G);
+  gather<T>(p, chunk_row(p, b, h, d, c, t), t, qq, Q, K, V, G);
   tc::cp_async_commit();
-  // S [dk][dv] -> two bf16 terms in the MN-major B layout (rows = dk = K);
-  // all eight units' loads are issued before the first is converted
+  tc::tc_before_sync();
+  __syncthreads();                                 // the barrier and the TMEM address
+  tc::tc_after_sync();
+  const uint32_t tm = *tmem_slot;
+  // tensor memory: S^T hi [0, 64), S^T lo [64, 128), o^T [128, 192), scores [192, 256)
+  const uint32_t tmSh = tm, tmSl = tm + 64, tmO = tm + 128, tmP = tm + 192;
+  const int qd = warp & 3, hf = warp >> 2;
+  const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
   {
-    const float* Sg = p.wsS + ((size_t)bh * p.nc + c) * kD * kD;
-    constexpr int kUnits = kD * 16 / kThreads;
-    float4 sa[kUnits], sb[kUnits];
+    // S^T row j = 32 qd + lane (a value dim), key dims 64 hf .. 64 hf + 63, from S [dk][dv]
+    const float* Sg = p.wsS + ((size_t)bh * p.nc + c) * kD * kD + 32 * qd + lane;
 #pragma unroll
-    for (int n = 0; n < kUnits; ++n) {
-      const int it = tid + n * kThreads, i = it >> 4, u = it & 15;
-      sa[n] = *reinterpret_cast<const float4*>(Sg + (size_t)i * kD + u * 8);
-      sb[n] = *reinterpret_cast<const float4*>(Sg + (size_t)i * kD + u * 8 + 4);
-    }
+    for (int part = 0; part < 2; ++part) {
+      const int i0 = 64 * hf + 32 * part;
+      float sv[32];
 #pragma unroll
-    for (int n = 0; n < kUnits; ++n) {
-      const int it = tid + n * kThreads, i = it >> 4, u = it & 15;
-      const float x[8] = {sa[n].x, sa[n].y, sa[n].z, sa[n].w, sb[n].x, sb[n].y, sb[n].z, sb[n].w};
-      uint4 hi, lo;
-      split8<__nv_bfloat16>(x, hi, lo);
-      const uint32_t off = sw_unit_off(kD, i, u);
-      *reinterpret_cast<uint4*>(S + off) = hi;
-      *reinterpret_cast<uint4*>(S + kTile128 + off) = lo;
+      for (int e = 0; e < 32; ++e) sv[e] = Sg[(size_t)(i0 + e) * kD];
+      uint32_t hw[16], lw[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(sv[2 * e], sv[2 * e + 1]);
+        const float2 f = __bfloat1622float2(hi);
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(sv[2 * e] - f.x, sv[2 * e + 1] - f.y);
+        memcpy(&hw[e], &hi, 4);
+        memcpy(&lw[e], &lo, 4);
+      }
+      // two key dims per 32-bit column, the even one in the low half
+      tmem_st32x16(tmSh + lane_base + (uint32_t)(i0 >> 1), hw);
+      tmem_st32x16(tmSl + lane_base + (uint32_t)(i0 >> 1), lw);
     }
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
   }
   tc::cp_async_wait<0>();
   __syncthreads();
@@ -391,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc128(const Params p) {
       *reinterpret_cast<uint4*>(K + off) = hi;
       *reinterpret_cast<uint4*>(Klo + off) = lo;
     }
-    if (!kBF) {
+    if (L::kTwoV) {
       widen8<T>(*reinterpret_cast<const uint4*>(V + off), x);
       split8<__nv_bfloat16>(x, hi, lo);        // exact: an fp16 value is bf16 hi + bf16 lo
       *reinterpret_cast<uint4*>(V + off) = hi;
@@ -402,22 +429,19 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc128(const Params p) {
   tc::tc_before_sync();
   __syncthreads();
   tc::tc_after_sync();
-  const uint32_t tm = *tmem_slot;
-  const uint32_t tmO = tm, tmP = tm + 128;         // o: columns [0, 128); scores: [128, 192)
+  constexpr uint32_t kIdOT = idesc(true, 0, 0, 128, 64);       // S^T (tensor memory) x q~^T (K-major)
   constexpr uint32_t kIdScores = idesc(true, 0, 0, 64, 64);    // q~ (K-major) x k~ (K-major)
-  constexpr uint32_t kIdQS = idesc(true, 0, 1, 64, 128);       // q~ (K-major) x S (MN-major)
-  constexpr uint32_t kIdPV = idesc(true, 0, 1, 64, 128);       // P (K-major) x V (MN-major)
+  constexpr uint32_t kIdVP = idesc(true, 1, 0, 128, 64);       // V^T (MN-major) x P^T (K-major)
   if (tid == 0) {
     const uint64_t qh = tc::desc_k(Q), ql = tc::desc_k(Qlo);
-    const uint64_t sh = tc::sdesc(saddr(S), kHalf128, 1024), sl = tc::sdesc(saddr(S + kTile128), kHalf128, 1024);
-    // o = q~ S: K = 128 key dims, two 64-column halves of the q~ tiles
+    // o^T = S^T q~^T: K = 128 key dims, 8 tensor-memory columns per step of 16
 #pragma unroll
     for (int ks = 0; ks < kD / 16; ++ks) {
-      const uint64_t ao = (uint64_t)((ks >> 2) * (kHalf64 >> 4) + (ks & 3) * tc::kStepK);
-      const uint64_t bo = (uint64_t)(ks * tc::kStepMN);
-      tc::mma_f16(tmO, qh + ao, sh + bo, kIdQS, ks > 0);
-      tc::mma_f16(tmO, qh + ao, sl + bo, kIdQS, 1u);
-      tc::mma_f16(tmO, ql + ao, sh + bo, kIdQS, 1u);
+      const uint64_t bo = (uint64_t)((ks >> 2) * (kHalf64 >> 4) + (ks & 3) * tc::kStepK);
+      const uint32_t ao = (uint32_t)(ks * 8);
+      tc::mma_f16_ts(tmO, tmSh + ao, qh + bo, kIdOT, ks > 0);
+      tc::mma_f16_ts(tmO, tmSh + ao, ql + bo, kIdOT, 1u);
+      tc::mma_f16_ts(tmO, tmSl + ao, qh + bo, kIdOT, 1u);
     }
     if (!exact) {
       const uint64_t kh = tc::desc_k(K), kl = tc::desc_k(Klo);
@@ -433,9 +457,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc128(const Params p) {
   }
   bool ok = wait_phase(bar, 0);
   tc::tc_after_sync();
-  // P: thread (quadrant qd = warp % 4, half hf = warp / 4) holds row r = 16 qd + lane % 16,
+  // P: thread (quadrant qd, half hf) holds score row r = 16 qd + lane % 16,
   // columns s0 .. s0 + 15 with s0 = 32 hf + 16 (lane / 16)
-  const int qd = warp & 3, hf = warp >> 2;
   const int r = qd * 16 + (lane & 15);
   const int s0 = hf * 32 + (lane >> 4) * 16;
   const int ntok = min(kC, p.T - c * kC);
@@ -443,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc128(const Params p) {
     float sc[16];
     if (!exact) {
       float tv[16];
-      tc::tmem_ld16x2(tmP + ((uint32_t)(qd * 32) << 16) + (uint32_t)(hf * 32), tv);
+      tc::tmem_ld16x2(tmP + lane_base + (uint32_t)(hf * 32), tv);
       tc::tmem_ld_wait(tv);
 #pragma unroll
       for (int e = 0; e < 16; ++e) sc[e] = tv[e];
@@ -465,7 +488,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc128(const Params p) {
       }
       if (tid == 0) atomicAdd(&g_gtr_exact_chunks, 1ull);
     }
-    // causal mask (s <= r), two bf16 terms into the K-major P tiles
+    // the key tiles have been read by the scores product (or were never used):
+    // causal mask (s <= r), two bf16 terms into the K-major P tiles there
 #pragma unroll
     for (int hb = 0; hb < 2; ++hb) {
       float x[8];
@@ -483,65 +507,45 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc128(const Params p) {
   __syncthreads();
   tc::tc_after_sync();
   if (tid == 0) {
-    // o += P V: K = 64 tokens
-    const uint64_t ph = tc::desc_k(P), pl = tc::desc_k(P + kHalf64);
+    // o^T += V^T P^T: K = 64 tokens
     const uint64_t vh = tc::desc_mn(V), vl = tc::desc_mn(Vlo);
+    const uint64_t ph = tc::desc_k(P), pl = tc::desc_k(P + kHalf64);
 #pragma unroll
     for (int ks = 0; ks < kC / 16; ++ks) {
-      const uint64_t ao = (uint64_t)(ks * tc::kStepK), bo = (uint64_t)(ks * tc::kStepMN);
-      tc::mma_f16(tmO, ph + ao, vh + bo, kIdPV, 1u);
-      tc::mma_f16(tmO, pl + ao, vh + bo, kIdPV, 1u);
-      if (!kBF) tc::mma_f16(tmO, ph + ao, vl + bo, kIdPV, 1u);
+      const uint64_t ao = (uint64_t)(ks * tc::kStepMN), bo = (uint64_t)(ks * tc::kStepK);
+      tc::mma_f16(tmO, vh + ao, ph + bo, kIdVP, 1u);
+      tc::mma_f16(tmO, vh + ao, pl + bo, kIdVP, 1u);
+      if (L::kTwoV) tc::mma_f16(tmO, vl + ao, ph + bo, kIdVP, 1u);
     }
     tc::mma_commit(bar);
   }
   ok = wait_phase(bar, 1) && ok;
   tc::tc_after_sync();
-  // epilogue: row r, columns 64 hf + [16 (lane / 16), + 16) and 64 hf + 32 + [16 (lane / 16), + 16)
+  // epilogue: lane j = 32 qd + lane holds o[t][j] for tokens t0 .. t0 + 31, t0 = 32 hf
+  const int j = qd * 32 + lane, t0 = hf * 32;
   float o[32];
-  {
-    float a[16], e2[16];
-    const uint32_t base = tmO + ((uint32_t)(qd * 32) << 16) + (uint32_t)(hf * 64);
-    tc::tmem_ld16x2(base, a);
-    tc::tmem_ld_wait(a);
-    tc::tmem_ld16x2(base + 32, e2);
-    tc::tmem_ld_wait(e2);
+  tmem_ld32x32(tmO + lane_base + (uint32_t)t0, o);
+  // sum over the value dims of o[t][.]^2: this warp's 32, then the four quadrants
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      o[e] = a[e];
-      o[16 + e] = e2[e];
-    }
+  for (int e = 0; e < 32; ++e) {
+    float sq = o[e] * o[e];
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, m);
+    if (lane == e) rowss[qd * kC + t0 + e] = sq;
   }
-  float ss = 0.f;
-#pragma unroll
-  for (int e = 0; e < 32; ++e) ss = fmaf(o[e], o[e], ss);
-  ss += __shfl_xor_sync(0xffffffffu, ss, 16);
-  if ((lane >> 4) == 0) rowss[hf * kC + r] = ss;
   __syncthreads();
-  const float tot = rowss[r] + rowss[kC + r];
-  const float inv = rsqrtf(tot / (float)kD + kRmsEps);
-  if (r < ntok && ok) {
-    const long long orow = chunk_row(p, b, h, d, c, r);
-    const T* zr = (const T*)p.z + orow * kD;
-    T* outr = (T*)p.out + orow * kD;
+  const float wj = p.w ? __ldg(p.w + j) : 1.0f;
+  if (ok) {
 #pragma unroll
-    for (int part = 0; part < 2; ++part) {
-      const int j0 = hf * 64 + part * 32 + (lane >> 4) * 16;
-      float zf[16];
-      widen8<T>(*reinterpret_cast<const uint4*>(zr + j0), *reinterpret_cast<float(*)[8]>(zf));
-      widen8<T>(*reinterpret_cast<const uint4*>(zr + j0 + 8), *reinterpret_cast<float(*)[8]>(zf + 8));
-      float y[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const float wj = p.w ? __ldg(p.w + j0 + e) : 1.0f;
-        y[e] = o[part * 16 + e] * inv * wj * tc::silu_fast(zf[e]);
+    for (int e = 0; e < 32; ++e) {
+      const int tk = t0 + e;
+      if (tk < ntok) {
+        const float tot = rowss[tk] + rowss[kC + tk] + rowss[2 * kC + tk] + rowss[3 * kC + tk];
+        const float inv = rsqrtf(tot / (float)kD + kRmsEps);
+        const long long orow = chunk_row(p, b, h, d, c, tk);
+        const float zj = ld_f((const T*)p.z + orow * kD + j);
+        ((T*)p.out)[orow * kD + j] = Elem<T>::from_f(o[e] * inv * wj * tc::silu_fast(zj));
       }
-      uint4 u0, u1, l0, l1;
-      // the output is one rounding of y to T (the lo terms are discarded)
-      split8<T>(*reinterpret_cast<float(*)[8]>(y), u0, l0);
-      split8<T>(*reinterpret_cast<float(*)[8]>(y + 8), u1, l1);
-      *reinterpret_cast<uint4*>(outr + j0) = u0;
-      *reinterpret_cast<uint4*>(outr + j0 + 8) = u1;
     }
   }
   if (!ok && lane == 0) gtr_flag(kStatusMbarTimeout);
@@ -562,7 +566,12 @@ inline int launch_tc128(int dtype, int stage, const tc128::Params& p, int BH, cu
   const dim3 grid((unsigned)p.nc, (unsigned)BH);
   auto go = [&](auto kern, int smem, bool* flag) -> int {
     if (!flag[dev]) {
-      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return -5;
+      // all of the SM's unified L1 / shared memory as shared memory, so that
+      // two blocks of 112 KB (or of the summary's 81 KB) fit side by side
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+          cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+        return -5;
       flag[dev] = true;
     }
     return launch_pdl(kern, grid, dim3(tc128::kThreads), (size_t)smem, st, p);
@@ -570,8 +579,8 @@ inline int launch_tc128(int dtype, int stage, const tc128::Params& p, int BH, cu
   if (stage == 0)
     return dtype == kF16 ? go(tc128::gla_sum_tc128<__half>, tc128::SumLayout::kSmem, done[0])
                          : go(tc128::gla_sum_tc128<__nv_bfloat16>, tc128::SumLayout::kSmem, done[1]);
-  return dtype == kF16 ? go(tc128::gla_out_tc128<__half>, tc128::OutLayout::kSmem, done[2])
-                       : go(tc128::gla_out_tc128<__nv_bfloat16>, tc128::OutLayout::kSmem, done[3]);
+  return dtype == kF16 ? go(tc128::gla_out_tc128<__half>, tc128::OutLayout<__half>::kSmem, done[2])
+                       : go(tc128::gla_out_tc128<__nv_bfloat16>, tc128::OutLayout<__nv_bfloat16>::kSmem, done[3]);
 }
 
 }  // namespace gtr
