@@ -101,6 +101,13 @@ def test_given_directions_and_graph_replay():
     del g
 
 
+def test_twelve_blocks_bf16_ragged_grid_norms_and_bias():
+    # 13 x 17 = 221 tokens (three chunks and a half), random norm weights and gate bias
+    x, blocks = inputs.make_stack(12, 2, 13, 17, dtype="bf16", seed=12, random_norms=True, bias_std=0.5)
+    got, _ = _run(x, blocks, "bf16", 13, 17)
+    _check(got, x, blocks, "bf16", 13, 17, what="12 blocks bf16 13x17")
+
+
 def test_full_size_16k_four_blocks():
     # the 128x128 grid (16384 tokens) through LR, RL, TB, BT
     x, blocks = inputs.make_stack(4, 1, 128, 128, dtype="f16", seed=8)

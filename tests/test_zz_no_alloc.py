@@ -79,6 +79,15 @@ def test_noalloc_longer_segments_on_the_tensor_core_path():
     _two_calls(B, H, gh, gw, 64, 64, "f16", "TB", 64, seeds=(9, 10))
 
 
+def test_noalloc_d128_tensor_core_path():
+    # 64 chunks of one head: 64 x 64 KB of chunk states fit the scratch, so the
+    # d = 128 tensor-core kernels run (one chunk per segment)
+    B, H, gh, gw = 1, 1, 64, 64
+    assert binding.path_for(B, H, gh, gw, 128, 128, 64, torch.bfloat16) == "tc"
+    assert binding.workspace_bytes(B, H, gh, gw, 128, 128, 64, torch.bfloat16) <= SCRATCH
+    _two_calls(B, H, gh, gw, 128, 128, "bf16", "TB", 64, seeds=(12, 13))
+
+
 def test_noalloc_rejects_problems_beyond_the_scratch():
     # B*H*(dk*dv + dk)*4 = 128*66048 bytes > 8 MiB: not even one segment per sequence fits
     B, H, dk = 32, 4, 128
