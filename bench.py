@@ -211,8 +211,8 @@ def read_traffic(kernel_name: str, src_hash: str):
 def kernel_source_hash():
     """Hash of the CUDA sources the gate + GLA step is compiled from (the
     translation unit gtr_gla.cu and the headers beside it, less the projection
-    GEMM's own headers gemm_*.cuh and mixer_proj.cuh, which define no code the
-    step runs; another .cu file is its own translation unit and cannot change
+    GEMM's own headers gemm_*.cuh and mixer_proj.cuh and the 128-dim head
+    kernels tc128_kernels.cuh, which define no code the step runs; another .cu file is its own translation unit and cannot change
     these kernels), with comments and blank space removed, so that a figure
     measured on a kernel stays attached to it through comment edits."""
     import hashlib
@@ -222,7 +222,7 @@ def kernel_source_hash():
     for name in sorted(os.listdir(csrc)):
         if name.endswith(".cu") and name != "gtr_gla.cu":
             continue
-        if name.startswith("gemm_") or name == "mixer_proj.cuh":
+        if name.startswith("gemm_") or name in ("mixer_proj.cuh", "tc128_kernels.cuh"):
             continue
         with open(os.path.join(csrc, name), encoding="utf-8") as f:
             text = f.read()
