@@ -304,8 +304,9 @@ struct OutLayout {
   static constexpr int kV = kKlo + kTile64;
   static constexpr int kVlo = kV + kTile64;        // fp16 v only
   static constexpr int kG = kVlo + (kTwoV ? kTile64 : 0);
-  static constexpr int kMisc = kG + kGBytes;
-  static constexpr int kSmem = kMisc + 128;
+  static constexpr int kMisc = kG + kGBytes;      // barrier, TMEM address
+  static constexpr int kRows = kMisc + 128;        // the chunk's 64 token rows
+  static constexpr int kSmem = kRows + kC * 8;
   static constexpr int kBlocksPerSM = kTwoV ? 1 : 2;
 };
 
@@ -335,6 +336,7 @@ __global__ void __launch_bounds__(kThreads, OutLayout<T>::kBlocksPerSM) gla_out_
   float* rowss = reinterpret_cast<float*>(Q);      // after the first products: [4][64] partial sums
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::kMisc);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kMisc + 16);
+  long long* rows = reinterpret_cast<long long*>(sm + L::kRows);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x, bh = blockIdx.y;
   const int b = bh / p.H, h = bh - b * p.H;
@@ -358,10 +360,12 @@ __global__ void __launch_bounds__(kThreads, OutLayout<T>::kBlocksPerSM) gla_out_
   pdl_wait();                                      // the boundary states come from the scan
   pdl_trigger();
   const int t = tid >> 2, qq = tid & 3;
-  gather<T>(p, chunk_row(p, b, h, d, c, t), t, qq, Q, K, V, G);
+  const long long my_row = chunk_row(p, b, h, d, c, t);
+  gather<T>(p, my_row, t, qq, Q, K, V, G);
   tc::cp_async_commit();
+  if (qq == 0) rows[t] = my_row;
   tc::tc_before_sync();
-  __syncthreads();                                 // the barrier and the TMEM address
+  __syncthreads();                                 // the barrier, the TMEM address, the rows
   tc::tc_after_sync();
   const uint32_t tm = *tmem_slot;
   // tensor memory: S^T hi [0, 64), S^T lo [64, 128), o^T [128, 192), scores [192, 256)
@@ -525,6 +529,12 @@ __global__ void __launch_bounds__(kThreads, OutLayout<T>::kBlocksPerSM) gla_out_
   const int j = qd * 32 + lane, t0 = hf * 32;
   float o[32];
   tmem_ld32x32(tmO + lane_base + (uint32_t)t0, o);
+  // z of the 32 tokens, all requested before any output is stored (out and z
+  // are different buffers, but the compiler cannot know that)
+  float zv[32];
+#pragma unroll
+  for (int e = 0; e < 32; ++e)
+    zv[e] = (t0 + e < ntok) ? ld_f((const T*)p.z + rows[t0 + e] * kD + j) : 0.f;
   // sum over the value dims of o[t][.]^2: this warp's 32, then the four quadrants
 #pragma unroll
   for (int e = 0; e < 32; ++e) {
@@ -542,9 +552,7 @@ __global__ void __launch_bounds__(kThreads, OutLayout<T>::kBlocksPerSM) gla_out_
       if (tk < ntok) {
         const float tot = rowss[tk] + rowss[kC + tk] + rowss[2 * kC + tk] + rowss[3 * kC + tk];
         const float inv = rsqrtf(tot / (float)kD + kRmsEps);
-        const long long orow = chunk_row(p, b, h, d, c, tk);
-        const float zj = ld_f((const T*)p.z + orow * kD + j);
-        ((T*)p.out)[orow * kD + j] = Elem<T>::from_f(o[e] * inv * wj * tc::silu_fast(zj));
+        ((T*)p.out)[rows[tk] * kD + j] = Elem<T>::from_f(o[e] * inv * wj * tc::silu_fast(zv[e]));
       }
     }
   }
