@@ -535,26 +535,34 @@ __global__ void __launch_bounds__(kThreads, OutLayout<T>::kBlocksPerSM) gla_out_
 #pragma unroll
   for (int e = 0; e < 32; ++e)
     zv[e] = (t0 + e < ntok) ? ld_f((const T*)p.z + rows[t0 + e] * kD + j) : 0.f;
-  // sum over the value dims of o[t][.]^2: this warp's 32, then the four quadrants
+  // sum over the value dims of o[t][.]^2 for the 32 tokens at once: a
+  // transposing butterfly (each step a lane keeps half of its sums and adds
+  // its partner's copy of that half; 31 shuffles) leaves lane l with this
+  // warp's sum for token t0 + l; then the four quadrants through shared memory
+  float sq[32];
+#pragma unroll
+  for (int e = 0; e < 32; ++e) sq[e] = o[e] * o[e];
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) {
+    const bool up = (lane & m) != 0;
+#pragma unroll
+    for (int e = 0; e < m; ++e) {
+      const float send = up ? sq[e] : sq[m + e];
+      const float keep = up ? sq[m + e] : sq[e];
+      sq[e] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+    }
+  }
+  rowss[qd * kC + t0 + lane] = sq[0];
+  __syncthreads();
+  // lane l: 1 / RMS of token t0 + l, handed to the other lanes by shuffles
+  const float tot = rowss[t0 + lane] + rowss[kC + t0 + lane] + rowss[2 * kC + t0 + lane] + rowss[3 * kC + t0 + lane];
+  const float inv_l = rsqrtf(tot / (float)kD + kRmsEps);
+  const float wj = p.w ? __ldg(p.w + j) : 1.0f;
 #pragma unroll
   for (int e = 0; e < 32; ++e) {
-    float sq = o[e] * o[e];
-#pragma unroll
-    for (int m = 16; m > 0; m >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, m);
-    if (lane == e) rowss[qd * kC + t0 + e] = sq;
-  }
-  __syncthreads();
-  const float wj = p.w ? __ldg(p.w + j) : 1.0f;
-  if (ok) {
-#pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const int tk = t0 + e;
-      if (tk < ntok) {
-        const float tot = rowss[tk] + rowss[kC + tk] + rowss[2 * kC + tk] + rowss[3 * kC + tk];
-        const float inv = rsqrtf(tot / (float)kD + kRmsEps);
-        ((T*)p.out)[rows[tk] * kD + j] = Elem<T>::from_f(o[e] * inv * wj * tc::silu_fast(zv[e]));
-      }
-    }
+    const float inv = __shfl_sync(0xffffffffu, inv_l, e);
+    if (ok && t0 + e < ntok)
+      ((T*)p.out)[rows[t0 + e] * kD + j] = Elem<T>::from_f(o[e] * inv * wj * tc::silu_fast(zv[e]));
   }
   if (!ok && lane == 0) gtr_flag(kStatusMbarTimeout);
   tc::tc_before_sync();
