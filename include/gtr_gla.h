@@ -147,9 +147,9 @@ GTR_API gtr_status_t gtr_gate_fwd_packed(const void *x, int x_dtype, const void 
  *   128}; the result does not depend on C beyond rounding.  T = grid_h*grid_w
  *   must fit in an int.  `out` must not alias any input.
  *   Kernels: tcgen05 tensor-core kernels for 16-bit dtypes with chunk 64 and
- *   dk = dv = 64 (segments of chunks walked with the state on chip) or
- *   dk = dv = 128 (every chunk its own block, 64 KB of fp32 state per chunk
- *   in the workspace); the exact fp32 CUDA-core kernels otherwise.
+ *   dk = dv = 64 or 128 (segments of chunks walked with the state on chip,
+ *   one fp32 state per segment in the workspace); the exact fp32 CUDA-core
+ *   kernels otherwise.
  *   Workspace: fp32 segment states taken from a library-owned buffer cached
  *   per (device, stream) and grown on demand with cudaMalloc (so the first call
  *   for a shape must not happen during stream capture), or from the buffer

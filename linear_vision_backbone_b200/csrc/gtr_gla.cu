@@ -148,18 +148,10 @@ int make_plan(Plan* p, int dev, int B, int H, int gh, int gw, int dk, int dv, in
   p->path = path;
   p->nc = (p->T + chunk - 1) / chunk;
   const long long bh = (long long)B * H;
-  const int per_sm = path == GTR_PATH_TC ? tc_blocks_per_sm(dk, dv) : 4;
+  const int per_sm = path != GTR_PATH_TC ? 4
+                     : dk == tc128::kD ? tc128_blocks_per_sm(dtype)
+                                       : tc_blocks_per_sm(dk, dv);
   const long long slots = (long long)sm_count(dev) * per_sm;
-  if (path == GTR_PATH_TC && dk == tc128::kD) {
-    // the d = 128 tensor-core kernels take every chunk as its own segment; a
-    // plan with longer segments runs on the SIMT kernels
-    if (force_nseg > 0 && force_nseg < p->nc) {
-      if (g_path_setting.load() == GTR_PATH_TC) return GTR_ERR_UNSUPPORTED;
-      p->path = GTR_PATH_SIMT;
-    } else {
-      force_nseg = p->nc;
-    }
-  }
   if (force_nseg > 0) {
     p->nseg = force_nseg < p->nc ? force_nseg : p->nc;
   } else {
@@ -458,7 +450,7 @@ int launch_stage(const Plan& p, const void* q, const void* k, const void* v, con
                  const void* z, const float* w, void* out, float* wsS, float* wsA, cudaStream_t st,
                  int stage) {
   if (p.path == GTR_PATH_TC && p.dk == tc128::kD) {
-    const tc128::Params pp{q, k, v, g, z, w, wsS, wsA, out, p.H, p.T, p.gh, p.gw, p.dir, p.nc};
+    const tc128::Params pp{q, k, v, g, z, w, wsS, wsA, out, p.H, p.T, p.gh, p.gw, p.dir, p.nc, p.nseg};
     return launch_tc128(p.dtype, stage, pp, p.B * p.H, st, p.dev) ? GTR_ERR_CUDA : GTR_OK;
   }
   if (p.path == GTR_PATH_TC) {

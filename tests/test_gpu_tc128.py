@@ -93,6 +93,37 @@ def test_chunk_states(direction):
     assert worst <= 1.0, worst
 
 
+@pytest.mark.parametrize("dtype", ("f16", "bf16"))
+@pytest.mark.parametrize("direction", ("LR", "BT", "ROTATE"))
+def test_segments_of_several_chunks(dtype, direction):
+    # 8 sequences of 99 chunks (the last one 28 tokens): more chunks than the
+    # SMs hold blocks, so every block walks a run of chunks with the state
+    # carried on chip from one chunk to the next
+    B, H, gh, gw = 2, 4, 90, 70
+    dt = inputs.DTYPES[dtype]
+    assert binding.segment_chunks(B, H, gh, gw, D, D, 64, dt) > 1
+    d = inputs.make_custom(B, H, gh, gw, D, D, dtype, seed=351, qk_std=D ** -0.5, w_random=True)
+    y, ref = _run(d, gh, gw, direction)
+    assert_close(y, ref, dt, f"d128 segments {dtype} {direction}")
+    rc, bits, _ = binding.device_status()
+    assert rc == 0 and bits == 0, (rc, bits)
+
+
+def test_segments_with_exact_chunks_inside():
+    # a log-gate span near 20 nats per chunk: some chunks of a segment take the
+    # exact scores and carry the state with k^ = k e^{Gam - G}, the others
+    # with k~ = k e^{-G}
+    B, H, gh, gw = 2, 4, 90, 70
+    assert binding.segment_chunks(B, H, gh, gw, D, D, 64, torch.bfloat16) > 1
+    d = inputs.make_custom(B, H, gh, gw, D, D, "bf16", seed=361, qk_std=D ** -0.5, g_scale=0.32)
+    binding.device_status()
+    y, ref = _run(d, gh, gw, "TB")
+    assert_close(y, ref, torch.bfloat16, "d128 mixed exact chunks")
+    rc, bits, exact = binding.device_status()
+    assert rc == 0 and bits == 0
+    assert 0 < exact < B * H * 99, exact
+
+
 def test_strong_decay_takes_the_exact_path():
     # about -12 nats per token: every chunk's span leaves the factorised range
     gh, gw = 16, 16

@@ -63,7 +63,8 @@ def test_noalloc_simt_path_two_calls():
 
 
 def test_noalloc_longer_segments_when_states_exceed_scratch():
-    # the usual plan for this shape needs more than 8 MiB of boundary states (SIMT path)
+    # the usual plan for this shape needs more than 8 MiB of boundary states
+    # (74 segments per sequence); the scratch takes 31, each walking 8-9 chunks
     B, H, gh, gw, dk = 1, 4, 128, 128, 128
     assert binding.workspace_bytes(B, H, gh, gw, dk, dk, 64, torch.bfloat16) > SCRATCH
     _two_calls(B, H, gh, gw, dk, dk, "bf16", "LR", 64, seeds=(7, 8))
