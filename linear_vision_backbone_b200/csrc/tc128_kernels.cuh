@@ -129,12 +129,7 @@ __device__ __forceinline__ void tmem_ld32x32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Token row (b T + grid index) H + h of scan offset t of the chunk, or -1 past the sequence.
-__device__ __forceinline__ long long chunk_row(const Params& p, int b, int h, int d, int c, int t) {
-  const int s = c * kC + t;
-  if (s >= p.T) return -1;
-  return ((long long)b * p.T + scan_to_grid(d, s, p.T, p.gh, p.gw)) * p.H + h;
-}
+
 
 // 16-byte copy global -> shared that reads `bytes` (16 or 0) and zero-fills the rest.
 __device__ __forceinline__ void cp16(void* dst, const void* src, uint32_t bytes) {
@@ -142,30 +137,53 @@ __device__ __forceinline__ void cp16(void* dst, const void* src, uint32_t bytes)
                : "memory");
 }
 
-// Copies one chunk: thread tid takes token t = tid / 4 and a quarter qq = tid % 4
-// of its record -- four 16-byte units of each 16-bit tensor (into the
-// swizzled 64-row tiles) and eight of the fp32 gate row (plain row-major).
-// A null tile is not copied.
+// Token of the chunk whose copies thread tid makes, e = 0..3: half a warp per
+// token, so that one copy instruction of a warp moves two whole 256-byte rows
+// of a 16-bit tensor (or two halves of 512-byte gate rows).
+__device__ __forceinline__ int gtok(int tid, int e) { return 2 * (tid >> 5) + ((tid >> 4) & 1) + 16 * e; }
+
+// Grid index of token t of chunk c in scan order, or -1 past the sequence.
+__device__ __forceinline__ int chunk_gidx(const Params& p, int d, int c, int t) {
+  const int s = c * kC + t;
+  return s < p.T ? scan_to_grid(d, s, p.T, p.gh, p.gw) : -1;
+}
+__device__ __forceinline__ long long row_of(const Params& p, int b, int h, int gi) {
+  return gi < 0 ? -1 : ((long long)b * p.T + gi) * p.H + h;
+}
+
+// Copies one chunk whose token rows (or -1, zero-filled) are rows[e] for
+// tokens gtok(tid, e): unit tid % 16 of each 16-bit tensor (into the swizzled
+// 64-row tiles) and units tid % 16 and tid % 16 + 16 of the fp32 gate row
+// (plain row-major).  A null tile is not copied.
 template <typename T>
-__device__ __forceinline__ void gather(const Params& p, long long row, int t, int qq, uint8_t* Q, uint8_t* K,
+__device__ __forceinline__ void gather(const Params& p, const long long (&rows)[4], int tid, uint8_t* Q, uint8_t* K,
                                        uint8_t* V, float* G) {
-  const uint32_t ok = row >= 0 ? 16u : 0u;
-  const long long rr = row >= 0 ? row : 0;
+  const int u = tid & 15;
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
-    const int u = qq * 4 + e;
-    const uint32_t off = sw_unit_off(kC, t, u);
+    const int tt = gtok(tid, e);
+    const uint32_t ok = rows[e] >= 0 ? 16u : 0u;
+    const long long rr = rows[e] >= 0 ? rows[e] : 0;
+    const uint32_t off = sw_unit_off(kC, tt, u);
     if (Q) cp16(Q + off, (const T*)p.q + rr * kD + u * 8, ok);
     if (K) cp16(K + off, (const T*)p.k + rr * kD + u * 8, ok);
     if (V) cp16(V + off, (const T*)p.v + rr * kD + u * 8, ok);
-  }
-  if (G) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int u = qq * 8 + e;
-      cp16(G + t * kD + u * 4, p.g + rr * kD + u * 4, ok);
+    if (G) {
+      cp16(G + tt * kD + u * 4, p.g + rr * kD + u * 4, ok);
+      cp16(G + tt * kD + (u + 16) * 4, p.g + rr * kD + (u + 16) * 4, ok);
     }
   }
+}
+
+// The token rows of chunk c for the copies of thread tid.
+__device__ __forceinline__ void chunk_rows4(const Params& p, int b, int h, int d, int c, int tid, long long (&rows)[4]) {
+#pragma unroll
+  for (int e = 0; e < 4; ++e) rows[e] = row_of(p, b, h, chunk_gidx(p, d, c, gtok(tid, e)));
+}
+
+// Token row (b T + grid index) H + h of scan offset t of chunk c, or -1 past the sequence.
+__device__ __forceinline__ long long chunk_row(const Params& p, int b, int h, int d, int c, int t) {
+  return row_of(p, b, h, chunk_gidx(p, d, c, t));
 }
 
 // In-place inclusive cumulative sum of the gate over the chunk's 64 tokens:
@@ -201,22 +219,22 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity) { ret
 // G_t} (Gam_c, G_t now within the chunk), every weight at most one.  Written
 // as dS [dk][dv] fp32 and e^{Lam} at the end.
 struct SumLayout {
-  static constexpr int kK = 0;                     // k tile, then k^ hi in place
-  static constexpr int kKlo = kK + kTile64;        // k^ lo
-  static constexpr int kV = kKlo + kTile64;        // v tile (the MN-major A operand V^T)
-  static constexpr int kG = kV + kTile64;          // gates, then cumulative
+  static constexpr int kK = 0;                     // k tiles (two buffers), then k^ hi in place
+  static constexpr int kV = kK + 2 * kTile64;      // v tiles (two buffers; the MN-major A operand V^T)
+  static constexpr int kKlo = kV + 2 * kTile64;    // k^ lo
+  static constexpr int kG = kKlo + kTile64;        // gates, then cumulative
   static constexpr int kLam = kG + kGBytes;        // log-decay of the chunks after the current one
   static constexpr int kMisc = kLam + kD * 4;
-  static constexpr int kSmem = kMisc + 256 + 1024;
+  static constexpr int kSmem = kMisc + 256;
 };
+static_assert(2 * (SumLayout::kSmem + 1024) <= 228 * 1024,
+              "two summary blocks (and the 1 KB each reserves) must fit one SM");
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads, 2) gla_sum_tc128(const Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* K = sm + SumLayout::kK;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = smem_raw;
   uint8_t* Klo = sm + SumLayout::kKlo;
-  uint8_t* V = sm + SumLayout::kV;
   float* G = reinterpret_cast<float*>(sm + SumLayout::kG);
   float* Lam = reinterpret_cast<float*>(sm + SumLayout::kLam);
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + SumLayout::kMisc);
@@ -226,6 +244,10 @@ __global__ void __launch_bounds__(kThreads, 2) gla_sum_tc128(const Params p) {
   const int b = bh / p.H, h = bh - b * p.H;
   const int d = dir_of_batch(p.dir, b);
   const int c_lo = seg_first_chunk(seg, p.nc, p.nseg), c_hi = seg_first_chunk(seg + 1, p.nc, p.nseg);
+  if ((saddr(smem_raw) & 1023u) != 0u) {           // the swizzled tiles need 1024-byte alignment
+    if (tid == 0) gtr_flag(kStatusBadShape);
+    return;
+  }
   if (d < 0 || d > 3) {
     if (tid == 0) gtr_flag(kStatusBadDir);
     return;
@@ -241,17 +263,27 @@ __global__ void __launch_bounds__(kThreads, 2) gla_sum_tc128(const Params p) {
   }
   pdl_wait();                                      // the gates may come from the kernel before
   pdl_trigger();
-  const int t = tid >> 2, qq = tid & 3;
   constexpr uint32_t id = idesc(std::is_same<T, __nv_bfloat16>::value, 1, 1, 128, 128);
   uint32_t tm = 0, phase = 0;
   bool ok = true;
-  gather<T>(p, chunk_row(p, b, h, d, c_hi - 1, t), t, qq, nullptr, K, V, G);
+  long long rows4[4];
+  chunk_rows4(p, b, h, d, c_hi - 1, tid, rows4);
+  gather<T>(p, rows4, tid, nullptr, sm + SumLayout::kK, sm + SumLayout::kV, G);
   tc::cp_async_commit();
-  for (int c = c_hi - 1; c >= c_lo; --c) {
+  int bi = 0;                                      // this chunk's k, v buffer
+  for (int c = c_hi - 1; c >= c_lo; --c, bi ^= 1) {
     const bool more = c > c_lo;
-    const long long next_row = more ? chunk_row(p, b, h, d, c - 1, t) : -1;
+    uint8_t* K = sm + SumLayout::kK + bi * kTile64;
+    uint8_t* V = sm + SumLayout::kV + bi * kTile64;
     tc::cp_async_wait<0>();                        // this chunk's copies made by this thread
     __syncthreads();
+    if (more) {
+      // the other buffer was read by the previous chunk's product: the next k, v into it
+      chunk_rows4(p, b, h, d, c - 1, tid, rows4);
+      gather<T>(p, rows4, tid, nullptr, sm + SumLayout::kK + (bi ^ 1) * kTile64,
+                sm + SumLayout::kV + (bi ^ 1) * kTile64, nullptr);
+      tc::cp_async_commit();
+    }
     cumsum(G, tid);
     const float gam = tid < kD ? G[(kC - 1) * kD + tid] : 0.f;
     // k^ = k e^{Lam + Gam_c - G_t} in two terms of k's type: unit (t, u) per thread step
@@ -277,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 2) gla_sum_tc128(const Params p) {
     __syncthreads();
     tc::tc_after_sync();
     if (more) {
-      gather<T>(p, next_row, t, qq, nullptr, nullptr, nullptr, G);   // the gates are read: the next ones
+      gather<T>(p, rows4, tid, nullptr, nullptr, nullptr, G);   // the gates are read: the next ones
       tc::cp_async_commit();
     }
     tm = *tmem_slot;
@@ -296,12 +328,8 @@ __global__ void __launch_bounds__(kThreads, 2) gla_sum_tc128(const Params p) {
     phase ^= 1u;
     tc::tc_after_sync();
     if (tid < kD) Lam[tid] += gam;
-    // k^ and V are read; a timed-out wait ends the walk in every thread
+    // k^ lo and this buffer are read; a timed-out wait ends the walk in every thread
     if (!__syncthreads_and(ok)) break;
-    if (more) {
-      gather<T>(p, next_row, t, qq, nullptr, K, V, nullptr);
-      tc::cp_async_commit();
-    }
   }
   tc::cp_async_wait<0>();                          // no copy may land after the block exits
   float* dS = p.wsS + ((size_t)bh * p.nseg + seg) * kD * kD;
@@ -354,7 +382,8 @@ struct OutLayout {
   static constexpr int kVlo = kV + kTile64;        // fp16 v only
   static constexpr int kG = kVlo + (kTwoV ? kTile64 : 0);   // gates; then the row sums and e^{Gam}
   static constexpr int kMisc = kG + kGBytes;      // barrier, TMEM address
-  static constexpr int kSmem = kMisc + 128;
+  static constexpr int kIdx = kMisc + 128;         // grid indices of the tokens of two chunks (by parity)
+  static constexpr int kSmem = kIdx + 2 * kC * 4;
   static constexpr int kBlocksPerSM = kTwoV ? 1 : 2;
 };
 static_assert(2 * (OutLayout<__nv_bfloat16>::kSmem + 1024) <= 228 * 1024,
@@ -423,6 +452,7 @@ __global__ void __launch_bounds__(kThreads, OutLayout<T>::kBlocksPerSM) gla_out_
   T* Ze = reinterpret_cast<T*>(Zt);
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::kMisc);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kMisc + 16);
+  int* gidx = reinterpret_cast<int*>(sm + L::kIdx);   // [2][64]: chunk c at c % 2
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int seg = blockIdx.x, bh = blockIdx.y;
   const int b = bh / p.H, h = bh - b * p.H;
@@ -446,15 +476,20 @@ __global__ void __launch_bounds__(kThreads, OutLayout<T>::kBlocksPerSM) gla_out_
   }
   pdl_wait();                                      // the boundary states come from the scan
   pdl_trigger();
-  // the first chunk's copies go out first; each thread copies (and at the end
-  // stores) token t of the chunk, a quarter qq of its record
-  const int t = tid >> 2, qq = tid & 3;
-  long long my_row = chunk_row(p, b, h, d, c_lo, t);
-  gather<T>(p, my_row, t, qq, Q, K, V, G);
+  // the first chunk's copies go out first
+  if (tid < kC) gidx[(c_lo & 1) * kC + tid] = chunk_gidx(p, d, c_lo, tid);
+  long long rows4[4];
+  chunk_rows4(p, b, h, d, c_lo, tid, rows4);
+  gather<T>(p, rows4, tid, Q, K, V, G);
   tc::cp_async_commit();
   tc::tc_before_sync();
-  __syncthreads();                                 // the barrier, the TMEM address
+  __syncthreads();                                 // the barrier, the TMEM address, the grid indices
   tc::tc_after_sync();
+  // the rows of this thread's tokens of chunk cc, from the grid indices
+  auto rows_of = [&](int cc, long long (&rows)[4]) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) rows[e] = row_of(p, b, h, gidx[(cc & 1) * kC + gtok(tid, e)]);
+  };
   const uint32_t tm = *tmem_slot;
   // tensor memory: S^T hi [0, 64), S^T lo [64, 128), o^T [128, 192), scores
   // [192, 256); the state increment over [128, 256) after both are read
@@ -493,9 +528,10 @@ __global__ void __launch_bounds__(kThreads, OutLayout<T>::kBlocksPerSM) gla_out_
   bool ok = true;
   for (int c = c_lo; c < c_hi; ++c) {
     const bool carry = c + 1 < c_hi;               // the next chunk needs this one's end state
-    const long long next_row = carry ? chunk_row(p, b, h, d, c + 1, t) : -1;
     tc::cp_async_wait<0>();                        // this chunk's copies made by this thread
     __syncthreads();
+    // the next chunk's grid indices (that half was last read before the barrier)
+    if (carry && tid < kC) gidx[((c + 1) & 1) * kC + tid] = chunk_gidx(p, d, c + 1, tid);
     cumsum(G, tid);
     // a chunk whose log-gate span leaves [-kSpan, 0] takes exact scores
     const bool exact = __syncthreads_or(tid < kD && G[(kC - 1) * kD + tid] < -kSpan) != 0;
@@ -561,11 +597,14 @@ __global__ void __launch_bounds__(kThreads, OutLayout<T>::kBlocksPerSM) gla_out_
     phase ^= 1u;
     tc::tc_after_sync();
     {
-      // the q tiles are read: this chunk's z into the lo tile, row-major, 16-byte units of token t
-      const uint32_t zok = my_row >= 0 ? 16u : 0u;
-      const T* zr = (const T*)p.z + (my_row >= 0 ? my_row : 0) * kD;
+      // the q tiles are read: this chunk's z into the lo tile, row-major 256-byte rows
+      long long zr[4];
+      rows_of(c, zr);
+      const int u = tid & 15;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) cp16(Zt + t * 256 + (qq * 4 + e) * 16, zr + (qq * 4 + e) * 8, zok);
+      for (int e = 0; e < 4; ++e)
+        cp16(Zt + gtok(tid, e) * 256 + u * 16, (const T*)p.z + (zr[e] >= 0 ? zr[e] : 0) * kD + u * 8,
+             zr[e] >= 0 ? 16u : 0u);
       tc::cp_async_commit();
     }
     const int ntok = min(kC, p.T - c * kC);
@@ -630,7 +669,8 @@ __global__ void __launch_bounds__(kThreads, OutLayout<T>::kBlocksPerSM) gla_out_
     tc::tc_after_sync();
     if (carry) {
       // P is read: the next chunk's q over it
-      gather<T>(p, next_row, t, qq, Q, nullptr, nullptr, nullptr);
+      rows_of(c + 1, rows4);
+      gather<T>(p, rows4, tid, Q, nullptr, nullptr, nullptr);
       tc::cp_async_commit();
     }
     float o[32];
@@ -728,17 +768,21 @@ __global__ void __launch_bounds__(kThreads, OutLayout<T>::kBlocksPerSM) gla_out_
     if (!__syncthreads_and(ok)) break;
     tc::tc_after_sync();
     if (carry) {
-      gather<T>(p, next_row, t, qq, nullptr, K, V, G);   // the next chunk's k, v and gates
+      rows_of(c + 1, rows4);
+      gather<T>(p, rows4, tid, nullptr, K, V, G);   // the next chunk's k, v and gates
       tc::cp_async_commit();
     }
-    // token t's output row: four 16-byte units
-    if (t < ntok) {
-      T* dst = (T*)p.out + my_row * kD;
+    {
+      // the output rows: half a warp per 256-byte row
+      long long orow[4];
+      rows_of(c, orow);
+      const int u = tid & 15;
 #pragma unroll
       for (int e = 0; e < 4; ++e)
-        *reinterpret_cast<uint4*>(dst + (qq * 4 + e) * 8) = *reinterpret_cast<const uint4*>(Zt + t * 256 + (qq * 4 + e) * 16);
+        if (orow[e] >= 0)
+          *reinterpret_cast<uint4*>((T*)p.out + orow[e] * kD + u * 8) =
+              *reinterpret_cast<const uint4*>(Zt + gtok(tid, e) * 256 + u * 16);
     }
-    my_row = next_row;
   }
   tc::cp_async_wait<0>();                          // no copy may land after the block exits
   if (!ok && lane == 0) gtr_flag(kStatusMbarTimeout);
