@@ -483,6 +483,9 @@ int launch_scan(const Plan& p, float* wsS, const float* wsA, int inclusive, cuda
   // segments, faster at 1024)
   if (p.nseg <= kScanReg) return go(gla_state_scan<1, 4>, 1, 4);
   if (p.nseg >= 512) return go(gla_state_scan<kScanPartsWide, 1>, kScanPartsWide, 1);
+  // ranges of up to 24 segments in one window (one load latency instead of four)
+  if (p.nseg > kScanParts * kScanReg && p.nseg <= kScanParts * kScanRegLong)
+    return go(gla_state_scan<kScanParts, 1, kScanRegLong>, kScanParts, 1);
   return go(gla_state_scan<kScanParts, 1>, kScanParts, 1);
 }
 

@@ -15,8 +15,8 @@
 // Each warp first reduces its range to one affine map S -> P S + R (P the product of the range's A, R its scan from zero), the
 // warps exchange the maps through shared memory, and each range then replays
 // its recurrence from the state composed of the maps before it.  A range of
-// up to kScanReg segments stays in registers between the two passes, so the
-// whole pass costs one load latency, not one per segment.
+// up to one register window of segments stays in registers between the two
+// passes, so the whole pass costs one load latency, not one per segment.
 #pragma once
 #include "common.cuh"
 
@@ -24,15 +24,16 @@ namespace gtr {
 
 constexpr int kScanParts = 4;             // ranges per group
 constexpr int kScanPartsWide = 16;        // ranges per group for very long scans
-constexpr int kScanReg = 12;
+constexpr int kScanReg = 12;              // segments per register window
+constexpr int kScanRegLong = 24;          // the window of four ranges of up to 96 segments
 
-// Pass 1 / pass 2 over `n` segments held in registers (n <= kScanReg); the
+// Pass 1 / pass 2 over `n` segments held in registers (n <= kReg); the
 // full-window case is unrolled without predicates.
-template <bool kFull>
-__device__ __forceinline__ void scan_window(const float* pd, const float* pa, int n, int dkdv, int dk, float (&dS)[kScanReg],
-                                            float (&a)[kScanReg]) {
+template <bool kFull, int kReg>
+__device__ __forceinline__ void scan_window(const float* pd, const float* pa, int n, int dkdv, int dk, float (&dS)[kReg],
+                                            float (&a)[kReg]) {
 #pragma unroll
-  for (int u = 0; u < kScanReg; ++u) {
+  for (int u = 0; u < kReg; ++u) {
     if (kFull || u < n) {
       dS[u] = pd[u * dkdv];
       a[u] = pa[u * dk];
@@ -40,15 +41,16 @@ __device__ __forceinline__ void scan_window(const float* pd, const float* pa, in
   }
 }
 
-// at most 64 registers, 1024 threads per SM.  A block holds kGroups groups of
+// at most 64 registers, 1024 threads per SM (128 registers and 512 threads
+// with the long window).  A block holds kGroups groups of
 // 32 elements, each group's segments split into kParts ranges (one warp
 // each): four ranges of one group per block, so a 16k-token, 6-head problem
 // (768 blocks) is resident in one wave; sixteen ranges per group when the
 // segments are many, so that each range stays short; one range for each of
 // four groups when the segments fit one register window, so that problems of
 // many short sequences need a quarter of the blocks
-template <int kParts, int kGroups>
-__global__ void __launch_bounds__(32 * kParts * kGroups, 32 / (kParts * kGroups))
+template <int kParts, int kGroups, int kReg = kScanReg>
+__global__ void __launch_bounds__(32 * kParts * kGroups, 32 / (kParts * kGroups) * kScanReg / kReg)
 gla_state_scan(float* __restrict__ wsS, const float* __restrict__ wsA, long long total, int nseg,
                int dk, int dv, int inclusive) {
   constexpr int kScanParts = kParts;
@@ -73,15 +75,15 @@ gla_state_scan(float* __restrict__ wsS, const float* __restrict__ wsA, long long
   const float* A = wsA + (size_t)bh * nseg * dk + (size_t)sa * dk + i;
 
   // pass 1: this range as one map S -> P S + R
-  float dS[kScanReg], a[kScanReg];
+  float dS[kReg], a[kReg];
   float P = 1.f, R = 0.f;
   if (live) {
-    for (int s0 = 0; s0 < n; s0 += kScanReg) {
-      const int m = min(kScanReg, n - s0);
-      if (m == kScanReg) scan_window<true>(p + s0 * dkdv, A + s0 * dk, m, dkdv, dk, dS, a);
-      else scan_window<false>(p + s0 * dkdv, A + s0 * dk, m, dkdv, dk, dS, a);
+    for (int s0 = 0; s0 < n; s0 += kReg) {
+      const int m = min(kReg, n - s0);
+      if (m == kReg) scan_window<true, kReg>(p + s0 * dkdv, A + s0 * dk, m, dkdv, dk, dS, a);
+      else scan_window<false, kReg>(p + s0 * dkdv, A + s0 * dk, m, dkdv, dk, dS, a);
 #pragma unroll
-      for (int u = 0; u < kScanReg; ++u) {
+      for (int u = 0; u < kReg; ++u) {
         if (u < m) {
           R = fmaf(a[u], R, dS[u]);
           P *= a[u];
@@ -98,20 +100,20 @@ gla_state_scan(float* __restrict__ wsS, const float* __restrict__ wsA, long long
   for (int r = 0; r < part; ++r) S = fmaf(mapP[grp][r][lane], S, mapR[grp][r][lane]);
 
   // pass 2: the states, from registers when the range is one window
-  for (int s0 = 0; s0 < n; s0 += kScanReg) {
-    const int m = min(kScanReg, n - s0);
-    if (n > kScanReg) scan_window<false>(p + s0 * dkdv, A + s0 * dk, m, dkdv, dk, dS, a);
+  for (int s0 = 0; s0 < n; s0 += kReg) {
+    const int m = min(kReg, n - s0);
+    if (n > kReg) scan_window<false, kReg>(p + s0 * dkdv, A + s0 * dk, m, dkdv, dk, dS, a);
     float* q = p + s0 * dkdv;
     if (inclusive) {
 #pragma unroll
-      for (int u = 0; u < kScanReg; ++u)
+      for (int u = 0; u < kReg; ++u)
         if (u < m) {
           S = fmaf(a[u], S, dS[u]);
           q[u * dkdv] = S;
         }
     } else {
 #pragma unroll
-      for (int u = 0; u < kScanReg; ++u)
+      for (int u = 0; u < kReg; ++u)
         if (u < m) {
           q[u * dkdv] = S;
           S = fmaf(a[u], S, dS[u]);

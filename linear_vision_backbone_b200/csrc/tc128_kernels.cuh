@@ -2,28 +2,30 @@
 // dimensions dk = dv = 128 (16-bit q/k/v/z, fp32 gates, 64-token chunks).
 //
 // The chunkwise operator of the GTR article (方法详解 §4: chunk summaries on
-// tensor cores, a light pass over the chunk-boundary states, chunk outputs
+// tensor cores, a light pass over the segment-boundary states, chunk outputs
 // with the scores kept on chip and the output gate fused into the epilogue),
-// with every chunk an independent block:
+// one block per segment (a run of consecutive chunks of one sequence):
 //
-//   gla_sum_tc128  per (sequence, chunk): the state the chunk produces from
-//                  zero, dS = sum_t diag(e^{Gam - G_t}) k_t^T v_t (G_t the
-//                  in-chunk cumulative log-gate through token t, Gam its
-//                  total, so every weight is at most one), as one
-//                  tcgen05.mma product dS^T = V^T k^ (M = 128 value dims,
-//                  N = 128 key dims, K = 64 tokens) with k^ in two 16-bit
-//                  terms, and the chunk's decay factor e^{Gam}.
-//   (the boundary scan over chunks, scan_kernel.cuh, turns dS into the state
-//   each chunk starts from)
-//   gla_out_tc128  per (sequence, chunk): o = q~ S + mask(q~ k~^T) V with
-//                  q~ = q e^{G} and k~ = k e^{-G} referenced to the chunk
-//                  start, each operand in two bf16 terms (hi + lo) and the
-//                  products hi hi + hi lo + lo hi accumulated in fp32 in
-//                  tensor memory (M = 64 tokens); then RMSNorm over the 128
-//                  value dims x w x SiLU(z), stored at the tokens' grid rows.
-//                  Chunks whose log-gate span exceeds kSpan nats (where k~
-//                  would leave the terms' precision) take their scores from
-//                  an exact CUDA-core sum instead.
+//   gla_sum_tc128  per (sequence, segment): the state the segment produces
+//                  from zero, dS = sum_t diag(e^{Gam - G_t}) k_t^T v_t (G_t
+//                  the cumulative log-gate through token t, Gam the
+//                  segment's total, so every weight is at most one), one
+//                  tcgen05.mma product dS^T += V^T k^ per chunk (M = 128
+//                  value dims, N = 128 key dims, K = 64 tokens) with k^ in
+//                  two 16-bit terms, chunks taken last first; and the
+//                  segment's decay factor e^{Gam}.
+//   (the boundary scan over segments, scan_kernel.cuh, turns dS into the
+//   state each segment starts from)
+//   gla_out_tc128  per (sequence, segment), chunk by chunk:
+//                  o = q~ S + mask(q~ k~^T) V with q~ = q e^{G} and
+//                  k~ = k e^{-G} referenced to the chunk start, each operand
+//                  in two bf16 terms (hi + lo) and the products hi hi +
+//                  hi lo + lo hi accumulated in fp32 in tensor memory; then
+//                  RMSNorm over the 128 value dims x w x SiLU(z), stored at
+//                  the tokens' grid rows; then the state carried to the next
+//                  chunk on chip.  Chunks whose log-gate span exceeds kSpan
+//                  nats (where k~ would leave the terms' precision) take
+//                  their scores from an exact CUDA-core sum instead.
 //
 // Tiles in shared memory use the 128-byte swizzle of the tensor cores'
 // operand layout: a tile of R rows x 128 columns (16-bit) is two column

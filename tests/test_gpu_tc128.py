@@ -78,9 +78,10 @@ def test_matches_the_simt_kernels():
     assert_close(y_simt, ref, torch.float16, "simt")
 
 
-@pytest.mark.parametrize("direction", ("LR", "BT"))
-def test_chunk_states(direction):
-    gh, gw = 20, 13
+@pytest.mark.parametrize("direction,gh,gw", [("LR", 20, 13), ("BT", 20, 13), ("TB", 80, 56)])
+def test_chunk_states(direction, gh, gw):
+    # 80 x 56: 70 chunks, so the boundary scan holds each range of segments in
+    # one long register window
     d = inputs.make_custom(2, 2, gh, gw, D, D, "bf16", seed=331)
     st = binding.chunk_states(d["k"].cuda(), d["v"].cuda(), d["g"].cuda(), grid_h=gh, grid_w=gw,
                               direction=direction, chunk=64)
