@@ -47,8 +47,6 @@ constexpr int kThreads = 256;
 constexpr float kSpan = 20.0f;     // the chunk's log-gate span (nats) beyond which its scores are exact
 constexpr int kHalf64 = kC * 128;  // one 64-column half of a 64-row tile: 8 KB
 constexpr int kTile64 = 2 * kHalf64;           // 64 rows x 128 columns, 16-bit: 16 KB
-constexpr int kHalf128 = kD * 128;             // one half of a 128-row tile: 16 KB
-constexpr int kTile128 = 2 * kHalf128;         // 128 rows x 128 columns, 16-bit: 32 KB
 constexpr int kGBytes = kC * kD * 4;           // fp32 gate / cumulative log-gate: 32 KB
 
 struct Params {
@@ -57,11 +55,8 @@ struct Params {
   int H, T, gh, gw, dir, nc, nseg;   // segment s walks chunks [s nc / nseg, (s + 1) nc / nseg)
 };
 
-// byte offset of element (r, c) in a swizzled tile of `rows` rows x 128 columns
-__device__ __forceinline__ uint32_t sw_off(int rows, int r, int c) {
-  return (uint32_t)((c >> 6) * rows * 128 + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) + (c & 7) * 2);
-}
-// the same for the 16-byte unit holding columns [8u, 8u + 8) of row r
+// byte offset of the 16-byte unit holding columns [8u, 8u + 8) of row r in a
+// swizzled tile of `rows` rows x 128 columns
 __device__ __forceinline__ uint32_t sw_unit_off(int rows, int r, int u) {
   return (uint32_t)((u >> 3) * rows * 128 + r * 128 + (((u & 7) ^ (r & 7)) << 4));
 }
